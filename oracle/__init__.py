@@ -1,0 +1,130 @@
+"""fp64 CPU oracle for the GTR key-decay gated-linear-attention forward pass.
+
+TEST INFRASTRUCTURE, NOT PRODUCT CODE.  Only ``tests/``,
+``__graft_entry__.smoke()`` and ``bench.py``'s ``cpu_baseline`` / reference
+leg may import this package.  It shares no code with the CUDA path under
+``recurrent_vision_backbone_b200/`` and imports nothing from it.
+
+The arithmetic lives in ``gla_oracle.c`` (token-by-token recurrence in fp64,
+OpenMP over the independent (batch, head) sequences); this module only builds
+that file with gcc and marshals numpy arrays into it.
+
+What it follows: the GTR news article (tokendh.com), section
+"线性注意力到底在省什么" (gated linear attention, forget gate on the key side
+only, value-side decay fixed to 1) and section "单向扫描的致命缺陷，以及GTR怎么补"
+(four scan directions).  Pinned by ``tests/test_oracle_pins.py``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gla_oracle.c")
+_LIB = os.path.join(_HERE, "libgla_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+L2R, R2L, T2B, B2T = 0, 1, 2, 3
+DIRECTIONS = {"L2R": L2R, "R2L": R2L, "T2B": T2B, "B2T": B2T}
+
+
+def compile_oracle(src: str = _SRC, out: str = _LIB, extra_flags=()) -> str:
+    """Compile the C oracle into a shared library (plain gcc, no fast-math)."""
+    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", *extra_flags,
+           src, "-o", out, "-lm"]
+    subprocess.run(cmd, check=True)
+    return out
+
+
+def build(force: bool = False) -> str:
+    """Build ``libgla_oracle.so`` next to its source if missing or stale."""
+    with _lock:
+        stale = (not os.path.exists(_LIB)
+                 or os.path.getmtime(_LIB) < os.path.getmtime(_SRC))
+        if force or stale:
+            compile_oracle()
+    return _LIB
+
+
+def load_library(path: str) -> ctypes.CDLL:
+    lib = ctypes.CDLL(path)
+    dp = ctypes.POINTER(ctypes.c_double)
+    lib.gla_oracle_fwd_range.restype = ctypes.c_int
+    lib.gla_oracle_fwd_range.argtypes = [dp, dp, dp, dp] + [ctypes.c_int] * 7 + [
+        ctypes.c_long, ctypes.c_long, dp, dp, dp]
+    lib.gla_oracle_scan_to_token.restype = ctypes.c_long
+    lib.gla_oracle_scan_to_token.argtypes = [ctypes.c_long, ctypes.c_int, ctypes.c_int,
+                                             ctypes.c_int]
+    lib.gla_oracle_max_threads.restype = ctypes.c_int
+    lib.gla_oracle_set_threads.argtypes = [ctypes.c_int]
+    return lib
+
+
+def _get():
+    global _lib
+    if _lib is None:
+        _lib = load_library(build())
+    return _lib
+
+
+def _f64(x) -> np.ndarray:
+    if hasattr(x, "detach"):  # torch tensor -> numpy without importing torch here
+        x = x.detach().cpu().numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def scan_to_token(p: int, H: int, W: int, direction: int) -> int:
+    return int(_get().gla_oracle_scan_to_token(p, H, W, direction))
+
+
+def max_threads() -> int:
+    return int(_get().gla_oracle_max_threads())
+
+
+def set_threads(n: int) -> None:
+    _get().gla_oracle_set_threads(int(n))
+
+
+def gla_forward(q, k, v, g, H: int, W: int, direction: int, s0=None,
+                p_begin: int = 0, p_end: int | None = None, out=None, lib=None):
+    """Run the oracle.
+
+    q, k, g: [B, N, heads, dk]; v: [B, N, heads, dv]; s0: [B, heads, dk, dv] or None.
+    Processes scan positions [p_begin, p_end) (default: the whole grid).
+    Returns (out [B, N, heads, dv] fp64, s_final [B, heads, dk, dv] fp64).
+    Rows of ``out`` for tokens outside the range are zero (or keep the values of
+    a caller-supplied ``out``).
+    """
+    lib = lib or _get()
+    q, k, v, g = _f64(q), _f64(k), _f64(v), _f64(g)
+    B, N, heads, dk = q.shape
+    dv = v.shape[-1]
+    if N != H * W:
+        raise ValueError(f"N={N} != H*W={H * W}")
+    if k.shape != q.shape or g.shape != q.shape or v.shape[:3] != q.shape[:3]:
+        raise ValueError("shape mismatch between q, k, v, g")
+    s0a = None if s0 is None else _f64(s0)
+    if s0a is not None and s0a.shape != (B, heads, dk, dv):
+        raise ValueError("s0 must be [B, heads, dk, dv]")
+    o = np.zeros((B, N, heads, dv)) if out is None else out
+    if o.dtype != np.float64 or not o.flags["C_CONTIGUOUS"]:
+        raise ValueError("out must be contiguous fp64")
+    sf = np.zeros((B, heads, dk, dv))
+    pe = N if p_end is None else int(p_end)
+    rc = lib.gla_oracle_fwd_range(_ptr(q), _ptr(k), _ptr(v), _ptr(g), B, heads, H, W,
+                                  dk, dv, int(direction), int(p_begin), pe, _ptr(s0a),
+                                  _ptr(o), _ptr(sf))
+    if rc != 0:
+        raise RuntimeError(f"gla_oracle_fwd_range failed with code {rc}")
+    return o, sf

@@ -1,0 +1,158 @@
+"""Independent fp64 restatements used to pin the oracle (test-side only).
+
+Nothing here is imported by the oracle or by the CUDA path, and nothing here
+imports either of them.  Each function computes a quantity the oracle must
+reproduce, by a different route:
+
+* ``scan_permutation``: the four scan orders as numpy flips/transposes of the
+  index grid (GTR news article, section "单向扫描的致命缺陷，以及GTR怎么补").
+* ``brute_force``: the O(N^2) closed form of the key-decay recurrence,
+      o_t = sum_{s<=t} sum_i q_ti (prod_{r=s+1..t} a_ri) k_si v_s
+            + sum_i q_ti (prod_{r=0..t} a_ri) S0[i,:],
+  with a_t = exp(g_t) decaying key channels only (same article, section
+  "线性注意力到底在省什么").
+* ``linear_attention_prefix``: the a == 1 special case, causal linear attention
+  by prefix sums.
+* ``chunkwise``: the chunked form of the same recurrence (same article,
+  section "速度到底快在哪，TensorRT部署做了什么": parallel work inside a chunk,
+  only the boundary state carried from chunk to chunk), written with 16-token
+  sub-blocks and decay factors that never exceed 1 off the diagonal sub-blocks.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+def scan_permutation(H: int, W: int, direction: int) -> np.ndarray:
+    """perm[p] = memory token index visited at scan position p."""
+    idx = np.arange(H * W).reshape(H, W)
+    if direction == 0:      # L->R, row-major
+        grid = idx
+    elif direction == 1:    # R->L: rows top to bottom, each row right to left
+        grid = idx[:, ::-1]
+    elif direction == 2:    # T->B: columns left to right, each column top to bottom
+        grid = idx.T
+    elif direction == 3:    # B->T: columns left to right, each column bottom to top
+        grid = idx[::-1, :].T
+    else:
+        raise ValueError(direction)
+    return np.ascontiguousarray(grid).reshape(-1)
+
+
+def _sequences(x, perm):
+    """[B, N, heads, d] -> list over (b, h) of scan-ordered [N, d] arrays."""
+    B, N, heads, d = x.shape
+    return [x[b, perm, h, :] for b in range(B) for h in range(heads)]
+
+
+def brute_force(q, k, v, g, H, W, direction, s0=None):
+    """O(N^2 dk) closed form; returns (out [B,N,heads,dv], s_final [B,heads,dk,dv])."""
+    q, k, v, g = (np.asarray(t, dtype=np.float64) for t in (q, k, v, g))
+    B, N, heads, dk = q.shape
+    dv = v.shape[-1]
+    perm = scan_permutation(H, W, direction)
+    out = np.zeros((B, N, heads, dv))
+    sf = np.zeros((B, heads, dk, dv))
+    for b in range(B):
+        for h in range(heads):
+            Q, K, V, A = q[b, perm, h], k[b, perm, h], v[b, perm, h], np.exp(g[b, perm, h])
+            S0 = np.zeros((dk, dv)) if s0 is None else np.asarray(s0[b, h], np.float64)
+            for t in range(N):
+                w = np.ones(dk)          # prod_{r=s+1..t} a_r, built from s = t down
+                acc = np.zeros(dv)
+                for s in range(t, -1, -1):
+                    acc += np.dot(Q[t] * w, K[s]) * V[s]
+                    w = w * A[s]
+                acc += (Q[t] * w) @ S0   # w = prod_{r=0..t} a_r
+                out[b, perm[t], h] = acc
+            w = np.ones(dk)
+            S = np.zeros((dk, dv))
+            for s in range(N - 1, -1, -1):
+                S += np.outer(w * K[s], V[s])
+                w = w * A[s]
+            sf[b, h] = S + w[:, None] * S0
+    return out, sf
+
+
+def linear_attention_prefix(q, k, v, H, W, direction, s0=None):
+    """a == 1: o_t = q_t (S0 + sum_{s<=t} k_s^T v_s), by a cumulative sum."""
+    q, k, v = (np.asarray(t, dtype=np.float64) for t in (q, k, v))
+    B, N, heads, dk = q.shape
+    dv = v.shape[-1]
+    perm = scan_permutation(H, W, direction)
+    out = np.zeros((B, N, heads, dv))
+    sf = np.zeros((B, heads, dk, dv))
+    for b in range(B):
+        for h in range(heads):
+            Q, K, V = q[b, perm, h], k[b, perm, h], v[b, perm, h]
+            S0 = np.zeros((dk, dv)) if s0 is None else np.asarray(s0[b, h], np.float64)
+            states = np.cumsum(K[:, :, None] * V[:, None, :], axis=0) + S0[None]
+            out[b, perm, h] = np.einsum("ti,tij->tj", Q, states)
+            sf[b, h] = states[-1]
+    return out, sf
+
+
+def chunkwise(q, k, v, g, H, W, direction, s0=None, chunk=64, sub=16):
+    """Chunked fp64 restatement; must equal the token-by-token recurrence.
+
+    Per chunk of ``chunk`` scan positions (the tail is padded with q=k=v=0,
+    g=0), split into sub-blocks of ``sub`` tokens, with a = exp(g):
+      pi[t]  = prod of a over the sub-block from its first token to t (inclusive)
+      sig[s] = prod of a over the sub-block strictly after s
+      T[L]   = prod of a over sub-block L
+    inter-chunk : O += (Q * pi * prod_{L<I} T[L]) @ S_prev
+    intra-chunk : score(t in I, s in J<=I) = sum_i Q_ti K_si sig_si * c_ti,
+                  c = pi * prod_{J<L<I} T[L]  (I > J, all factors <= 1)
+                  c = pi / T[J]               (I == J, the diagonal sub-block)
+                  masked to s <= t, then O += scores @ V
+    state       : S = prod_L T[L] * S_prev + (K * sig * prod_{L>J} T[L])^T V
+    """
+    q, k, v, g = (np.asarray(t, dtype=np.float64) for t in (q, k, v, g))
+    B, N, heads, dk = q.shape
+    dv = v.shape[-1]
+    sub = min(sub, chunk)
+    assert chunk % sub == 0
+    nb = chunk // sub
+    perm = scan_permutation(H, W, direction)
+    out = np.zeros((B, N, heads, dv))
+    sf = np.zeros((B, heads, dk, dv))
+    nchunks = -(-N // chunk)
+    for b in range(B):
+        for h in range(heads):
+            S = np.zeros((dk, dv)) if s0 is None else np.array(s0[b, h], np.float64)
+            for c in range(nchunks):
+                p0, p1 = c * chunk, min((c + 1) * chunk, N)
+                n = p1 - p0
+                Q = np.zeros((chunk, dk)); K = np.zeros((chunk, dk))
+                V = np.zeros((chunk, dv)); G = np.zeros((chunk, dk))
+                rows = perm[p0:p1]
+                Q[:n], K[:n], V[:n], G[:n] = (q[b, rows, h], k[b, rows, h],
+                                              v[b, rows, h], g[b, rows, h])
+                A = np.exp(G)
+                blk = A.reshape(nb, sub, dk)
+                pi = np.cumprod(blk, axis=1).reshape(chunk, dk)
+                rev = np.cumprod(blk[:, ::-1, :], axis=1)[:, ::-1, :]   # inclusive suffix
+                sig = np.concatenate([rev[:, 1:, :], np.ones((nb, 1, dk))], axis=1)
+                sig = sig.reshape(chunk, dk)
+                T = np.prod(blk, axis=1)                                # [nb, dk]
+                blk_of = np.arange(chunk) // sub
+                before = np.array([np.prod(T[:I], axis=0) for I in range(nb)])
+                after = np.array([np.prod(T[I + 1:], axis=0) for I in range(nb)])
+                O = (Q * pi * before[blk_of]) @ S
+                Ksig = K * sig
+                scores = np.zeros((chunk, chunk))
+                for J in range(nb):
+                    cols = slice(J * sub, (J + 1) * sub)
+                    for I in range(J, nb):
+                        rws = slice(I * sub, (I + 1) * sub)
+                        if I == J:
+                            cq = pi[rws] / T[J]
+                        else:
+                            cq = pi[rws] * np.prod(T[J + 1:I], axis=0)
+                        scores[rws, cols] = (Q[rws] * cq) @ Ksig[cols].T
+                scores = np.tril(scores)
+                O += scores @ V
+                out[b, rows, h] = O[:n]
+                S = np.prod(T, axis=0)[:, None] * S + (Ksig * after[blk_of]).T @ V
+            sf[b, h] = S
+    return out, sf
