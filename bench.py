@@ -1,0 +1,461 @@
+"""Throughput benchmark of the GTR token-mixer forward pass on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
+
+One step = one layer call per scan direction (L->R, R->L, T->B, B->T) of the
+1.6K-token workload (B=1, 16 heads, 40x40 patch grid, dk=dv=64, fp16, chunk 64),
+each call on its own freshly drawn inputs.  The metric is spatial tokens per
+second (B*N per call, all heads included) over the whole job.  The same line
+also reports the 16.4K-token workload (B=1, 16 heads, 128x128) measured the
+same way.
+
+Inputs live in HBM before timing starts and rotate over enough distinct sets
+that their footprint is several times the 126 MB L2, so no call reads inputs
+the previous ones left in L2.  The timed steps are replayed from a CUDA graph
+(the launches would otherwise be host-bound), bracketed by a barrier and a
+device synchronise, timed with CUDA events, max over ranks.  Under torchrun each
+rank runs its own independent batch (weak scaling, no collective in the data
+path).  ``--impl reference`` times the fp64 CPU oracle on this host's cores on a
+bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+import torch.distributed as dist  # noqa: E402
+
+from recurrent_vision_backbone_b200.inputs import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "GLA fwd tokens/s at 1.6K & 16.4K tokens (FP16, C=64); % of roofline"
+PRIMARY = "gtr640_b1h16_40x40"
+SECONDARY = "hires_b1h16_128x128"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+DIRS = (0, 1, 2, 3)
+
+
+# ------------------------------------------------------------------ accounting
+def bytes_alg(w) -> int:
+    """Algorithmic HBM bytes of one call: read q, k, g, v and write o once (fp16),
+    plus the fp32 initial and final states where the workload has them."""
+    th = w.B * w.N * w.heads
+    b = th * 2 * (3 * w.dk + 2 * w.dv)
+    per_state = w.B * w.heads * w.dk * w.dv * 4
+    if w.init_std:
+        b += per_state
+    if w.final_state:
+        b += per_state
+    return b
+
+
+def flops_alg(w, chunk=64) -> int:
+    """Algorithmic FLOPs of one call: causal intra-chunk term, inter-chunk term and
+    state update (per token-head (C+1)(dk+dv) + 4 dk dv)."""
+    th = w.B * w.N * w.heads
+    return th * ((chunk + 1) * (w.dk + w.dv) + 4 * w.dk * w.dv)
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            d = json.load(fh)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha1()
+    csrc = os.path.join(ROOT, "recurrent_vision_backbone_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as fh:
+                h.update(fh.read())
+    return h.hexdigest()[:12]
+
+
+def recorded_traffic(workload_name: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
+    current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", f"gla_fwd_kernel_{workload_name}.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m_sha = re.search(r"kernel_source_sha1:\s*([0-9a-f]+)", text)
+    m_tr = re.search(r"traffic_bytes_per_launch:\s*([0-9]+)", text)
+    if not m_sha or not m_tr or m_sha.group(1) != kernel_source_hash():
+        return None
+    return int(m_tr.group(1))
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, flag in zip(names, parts[5:9]):
+                if flag.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ GPU arm
+class Workload:
+    """Rotating device-resident input sets for one workload and the graph that
+    replays `group` steps of 4 direction calls over them."""
+
+    def __init__(self, w, rank, device, n_sets=None):
+        from recurrent_vision_backbone_b200 import gla
+        self.gla = gla
+        self.w = w
+        per_call = bytes_alg(w)
+        if n_sets is None:
+            n_sets = max(4, -(-4 * L2_BYTES // (per_call * len(DIRS))))
+        self.n_sets = int(n_sets)
+        self.sets = []
+        for s in range(self.n_sets):
+            calls = []
+            for d in DIRS:
+                inp = make_inputs(w.B, w.heads, w.H, w.W, w.dk, w.dv,
+                                  seed=w.seed(d, 100 + s) + 7919 * rank,
+                                  init_std=w.init_std, z_mean_per_head=w.z_mean_per_head,
+                                  device=device)
+                out = torch.empty((w.B, w.N, w.heads, w.dv), dtype=torch.float16, device=device)
+                sf = (torch.empty((w.B, w.heads, w.dk, w.dv), dtype=torch.float32, device=device)
+                      if w.final_state else None)
+                calls.append((d, inp, out, sf))
+            self.sets.append(calls)
+        self.graph = None
+
+    def launch_step(self, s, stream):
+        for d, inp, out, sf in self.sets[s % self.n_sets]:
+            self.gla.gtr_gla_fwd(inp["q"], inp["k"], inp["v"], inp["g"], self.w.H, self.w.W, d,
+                                 init_state=inp["s0"], out=out, final_state=sf, stream=stream)
+
+    def capture(self, stream):
+        # warm the launch path once outside capture
+        with torch.cuda.stream(stream):
+            self.launch_step(0, stream)
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for s in range(self.n_sets):
+                self.launch_step(s, torch.cuda.current_stream())
+        self.graph = g
+        return self.n_sets  # steps per replay
+
+    def tokens_per_step(self):
+        return len(DIRS) * self.w.B * self.w.N
+
+
+def timed_replays(wl, replays, stream, world):
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(replays):
+        wl.graph.replay()
+    end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = start.elapsed_time(end)
+    if world > 1:
+        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return ms
+
+
+def measure(wl, steps, warmup, stream, world):
+    per_replay = wl.capture(stream)
+    replays = max(1, -(-steps // per_replay))
+    warm = max(1, -(-warmup // per_replay))
+    for _ in range(warm):
+        wl.graph.replay()
+    torch.cuda.synchronize()
+    assert wl.gla.device_status() == wl.gla.GTR_OK
+    ms = timed_replays(wl, replays, stream, world)
+    assert wl.gla.device_status() == wl.gla.GTR_OK
+    n_steps = replays * per_replay
+    return ms, n_steps
+
+
+def roofline(w, ms_per_launch, workload_name):
+    peak, which = measured_peaks()
+    b = bytes_alg(w)
+    achieved = b / (ms_per_launch * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "traffic": recorded_traffic(workload_name),
+            "peak_source": which, "bytes_alg_per_launch": b, "flops_alg_per_launch": flops_alg(w)}
+
+
+def e2e_measure(w, steps, device, rank):
+    """Tokens/s through the public call with host buffers: every step copies that
+    step's inputs from pinned host memory and reads the outputs back."""
+    from recurrent_vision_backbone_b200 import gla
+    host = []
+    for d in DIRS:
+        inp = make_inputs(w.B, w.heads, w.H, w.W, w.dk, w.dv, seed=w.seed(d, 500) + 7919 * rank,
+                          init_std=w.init_std, z_mean_per_head=w.z_mean_per_head)
+        hp = {n: (t.pin_memory() if t is not None else None) for n, t in inp.items()}
+        host.append((d, hp))
+    dev = {d: {n: (torch.empty_like(t, device=device) if t is not None else None)
+               for n, t in hp.items()} for d, hp in host}
+    outs = {d: torch.empty((w.B, w.N, w.heads, w.dv), dtype=torch.float16, device=device)
+            for d in DIRS}
+    sfs = {d: (torch.empty((w.B, w.heads, w.dk, w.dv), dtype=torch.float32, device=device)
+               if w.final_state else None) for d in DIRS}
+    h_out = {d: torch.empty_like(outs[d], device="cpu").pin_memory() for d in DIRS}
+    h_sf = {d: (torch.empty_like(sfs[d], device="cpu").pin_memory() if w.final_state else None)
+            for d in DIRS}
+    stream = torch.cuda.current_stream()
+    h2d = sum(t.numel() * t.element_size() for _, hp in host for t in hp.values() if t is not None)
+    d2h = sum(o.numel() * o.element_size() for o in h_out.values()) + sum(
+        s.numel() * s.element_size() for s in h_sf.values() if s is not None)
+
+    def one_step():
+        for d, hp in host:
+            for n, t in hp.items():
+                if t is not None:
+                    dev[d][n].copy_(t, non_blocking=True)
+            gla.gtr_gla_fwd(dev[d]["q"], dev[d]["k"], dev[d]["v"], dev[d]["g"], w.H, w.W, d,
+                            init_state=dev[d]["s0"], out=outs[d], final_state=sfs[d],
+                            stream=stream)
+            h_out[d].copy_(outs[d], non_blocking=True)
+            if sfs[d] is not None:
+                h_sf[d].copy_(sfs[d], non_blocking=True)
+
+    for _ in range(3):
+        one_step()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(steps):
+        one_step()
+    end.record(stream)
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(end)
+    return ms, steps, h2d, d2h
+
+
+def gpu_arm(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", init_method="env://", timeout=timedelta(seconds=120),
+                                device_id=device)
+    from recurrent_vision_backbone_b200 import gla
+    gla.load()
+    stream = torch.cuda.Stream(device=device)
+    w1 = WORKLOADS[PRIMARY]
+    wl = Workload(w1, rank, device)
+    clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
+                          else local)
+    clocks.start()
+    ms, n_steps = measure(wl, args.steps, args.warmup, stream, world)
+    clk = clocks.stop()
+    launches = n_steps * len(DIRS)
+    ms_step = ms / n_steps
+    value = world * wl.tokens_per_step() * n_steps / (ms * 1e-3)
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": n_steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 6),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+        "data": "synthetic",
+        "config": {"workload": PRIMARY, "B": w1.B, "heads": w1.heads, "grid": [w1.H, w1.W],
+                   "tokens_per_call": w1.B * w1.N, "dk": w1.dk, "dv": w1.dv, "chunk": 64,
+                   "calls_per_step": len(DIRS), "directions": "L2R,R2L,T2B,B2T",
+                   "l2": f"inputs rotate over {wl.n_sets} sets of 4 calls "
+                         f"({wl.n_sets * 4 * bytes_alg(w1) / 2**20:.0f} MiB > 3x L2)",
+                   "timing": "CUDA graph replay, CUDA events, max over ranks",
+                   "parallelism": f"dp{world} (independent batches)"},
+        "roofline": roofline(w1, ms / launches, PRIMARY),
+        "gpu_launches": launches,
+        "clocks": clk,
+    }
+    del wl
+    torch.cuda.empty_cache()
+    if not args.no_secondary:
+        w2 = WORKLOADS[SECONDARY]
+        wl2 = Workload(w2, rank, device)
+        ms2, n2 = measure(wl2, max(8, args.steps // 16), max(3, args.warmup // 16), stream, world)
+        line["secondary"] = {
+            "workload": SECONDARY, "tokens_per_call": w2.B * w2.N,
+            "value": round(world * wl2.tokens_per_step() * n2 / (ms2 * 1e-3), 1),
+            "unit": "tokens/s", "steps": n2, "ms_per_step": round(ms2 / n2, 6),
+            "roofline": roofline(w2, ms2 / (n2 * len(DIRS)), SECONDARY),
+            "gpu_launches": n2 * len(DIRS)}
+        del wl2
+        torch.cuda.empty_cache()
+    # end to end through the public call with host buffers
+    e_steps = max(3, min(args.steps, args.e2e_steps))
+    ems, en, h2d, d2h = e2e_measure(w1, e_steps, device, rank)
+    if world > 1:
+        t = torch.tensor([ems], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ems = float(t.item())
+    line["e2e"] = {"value": round(world * len(DIRS) * w1.B * w1.N * en / (ems * 1e-3), 1),
+                   "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                   "steps": en}
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w1, budget_s=args.cpu_seconds)
+    else:
+        line["cpu_baseline"] = None
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------ CPU arm
+def cpu_baseline(w, budget_s=15.0):
+    import oracle
+    oracle.build()
+    threads = oracle.max_threads()
+    # time only the oracle calls, on the full head set, for as many steps as fit the budget
+    tok = 0
+    spent = 0.0
+    steps = 0
+    while spent < budget_s and steps < 1000:
+        for d in DIRS:
+            inp = make_inputs(w.B, w.heads, w.H, w.W, w.dk, w.dv, seed=w.seed(d, 900 + steps),
+                              init_std=w.init_std, z_mean_per_head=w.z_mean_per_head)
+            f = {n: t.float().numpy() for n, t in inp.items() if t is not None}
+            t1 = time.perf_counter()
+            oracle.gla_forward(f["q"], f["k"], f["v"], f["g"], w.H, w.W, d, f.get("s0"))
+            spent += time.perf_counter() - t1
+            tok += w.B * w.N
+        steps += 1
+    return {"value": round(tok / spent, 1), "unit": "tokens/s", "cores": threads,
+            "kind": "oracle",
+            "sample": f"{steps} full steps ({steps * len(DIRS)} calls) of {w.name}, "
+                      f"fp64 token-by-token, OpenMP over the {w.B * w.heads} sequences; "
+                      f"oracle time only ({spent:.1f} s)"}
+
+
+def reference_arm(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    threads = oracle.max_threads()
+    w = WORKLOADS[PRIMARY]
+    # size the per-step sample so that warmup + steps stay within ~2 minutes
+    probe = time.perf_counter()
+    f = {n: t.float().numpy() for n, t in make_inputs(w.B, 1, w.H, w.W, w.dk, w.dv, seed=1).items()
+         if t is not None}
+    oracle.gla_forward(f["q"], f["k"], f["v"], f["g"], w.H, w.W, 0)
+    per_head_call = max(time.perf_counter() - probe, 1e-4)
+    total_calls = (args.steps + args.warmup) * len(DIRS)
+    heads = int(max(1, min(w.heads, 120.0 / (total_calls * per_head_call))))
+    spent = 0.0
+    for it in range(args.warmup + args.steps):
+        for d in DIRS:
+            inp = make_inputs(w.B, heads, w.H, w.W, w.dk, w.dv, seed=w.seed(d, 900 + it))
+            f = {n: t.float().numpy() for n, t in inp.items() if t is not None}
+            t1 = time.perf_counter()
+            oracle.gla_forward(f["q"], f["k"], f["v"], f["g"], w.H, w.W, d)
+            if it >= args.warmup:
+                spent += time.perf_counter() - t1
+    frac = heads / w.heads
+    tokens = args.steps * len(DIRS) * w.B * w.N * frac
+    value = tokens / spent
+    sample = (f"{heads} of {w.heads} heads of {w.name} per call (tokens scaled by "
+              f"{frac:.4f}), {args.steps} timed steps x 4 directions, fp64 token-by-token oracle")
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 1), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(spent / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": PRIMARY, "B": w.B, "heads": w.heads, "grid": [w.H, w.W],
+                       "dk": w.dk, "dv": w.dv, "chunk": 64, "calls_per_step": len(DIRS)},
+            "cpu_baseline": {"value": round(value, 1), "unit": "tokens/s", "cores": threads,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 1), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=400)
+    ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        reference_arm(args)
+    else:
+        gpu_arm(args)
+
+
+if __name__ == "__main__":
+    main()

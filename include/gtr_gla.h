@@ -1,0 +1,113 @@
+/*
+ * gtr_gla.h -- C ABI of the GTR token-mixer forward pass on B200 (sm_100a).
+ *
+ * The operation (GTR news article, tokendh.com, section "线性注意力到底在省什么";
+ * GTR: Gated Token Recurrence for Efficient Dense Prediction, abstract):
+ * a gated linear attention whose learnable forget gate decays the recurrent
+ * state on the key side only, the value-side decay being fixed to 1.  For one
+ * (batch b, head h) sequence, over scan positions t = 0 .. N-1:
+ *
+ *     a_t = exp(g_t)                         g_t <= 0, one value per key channel
+ *     S_t = diag(a_t) S_{t-1} + k_t^T v_t    S is dk x dv, S_{-1} = init_state or 0
+ *     o_t = q_t S_t
+ *
+ * The patch grid (Hgrid x Wgrid, token n = y*Wgrid + x) is scanned in one of
+ * four orders (same article, section "单向扫描的致命缺陷，以及GTR怎么补"):
+ *     GTR_L2R  row-major, each row left to right
+ *     GTR_R2L  rows top to bottom, each row right to left (the mirrored grid)
+ *     GTR_T2B  column-major, each column top to bottom
+ *     GTR_B2T  columns left to right, each column bottom to top
+ * The state is carried across rows/columns; the direction only changes which
+ * token is visited at scan position t.  Tensors stay in grid order in memory.
+ *
+ * The forward pass is computed chunkwise, 64 scan positions per chunk, in FP16
+ * with FP32 accumulation (same article, section "速度到底快在哪，TensorRT部署做了什么":
+ * parallel work inside a chunk, only the chunk-boundary state carried in order).
+ *
+ * Memory layouts (all device pointers, C-contiguous, 16-byte aligned):
+ *     q, k, g : IEEE binary16 [B, N, heads, dk]     N = Hgrid * Wgrid
+ *     v, out  : IEEE binary16 [B, N, heads, dv]
+ *     init_state, final_state : float32 [B, heads, dk, dv]
+ * g is the log-decay itself (already divided by the gate temperature); q is
+ * used as given (no scaling, no feature map, no normaliser).
+ *
+ * Ownership: every buffer belongs to the caller; the library never frees or
+ * keeps a pointer after a call returns.  All work is enqueued on `stream`
+ * (a cudaStream_t, NULL = legacy default stream); no call synchronises the host
+ * except gtr_gla_device_status.
+ *
+ * Errors: argument checks run on the host before anything is enqueued and
+ * return GTR_ERR_INVALID_ARG / GTR_ERR_UNSUPPORTED with nothing launched.
+ * A failed launch returns GTR_ERR_CUDA.  Device-side waits are bounded; if one
+ * runs out the kernel records GTR_ERR_TIMEOUT in a device error word that
+ * gtr_gla_device_status reports.
+ */
+#ifndef GTR_GLA_H
+#define GTR_GLA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t gtr_half_t;   /* IEEE 754 binary16 bit pattern */
+
+typedef enum { GTR_L2R = 0, GTR_R2L = 1, GTR_T2B = 2, GTR_B2T = 3 } gtr_dir_t;
+
+typedef enum {
+    GTR_OK = 0,
+    GTR_ERR_INVALID_ARG = 1,  /* null/negative/misaligned/overflowing/aliased arguments */
+    GTR_ERR_UNSUPPORTED = 2,  /* valid but not built: chunk != 64, dk not in {64,128}, dv != 64 */
+    GTR_ERR_CUDA = 3,         /* a CUDA runtime call or kernel launch failed */
+    GTR_ERR_TIMEOUT = 4       /* a bounded device-side wait ran out (see gtr_gla_device_status) */
+} gtr_status_t;
+
+/*
+ * Forward pass of one token-mixer layer call.
+ *   q, k, v, g      inputs (device), layouts above; may not alias `out`.
+ *   B, heads        batch size and number of heads (>= 1).
+ *   Hgrid, Wgrid    patch grid; N = Hgrid*Wgrid >= 0 (N == 0 is a no-op that
+ *                   still copies init_state to final_state).
+ *   dk, dv          key and value head dims: dk in {64, 128}, dv == 64.
+ *   direction       gtr_dir_t scan order.
+ *   chunk           chunk length; 64 (the only value built).
+ *   init_state      float32 [B, heads, dk, dv] or NULL for a zero state.
+ *   out             float16 [B, N, heads, dv], fully written.
+ *   final_state     float32 [B, heads, dk, dv] or NULL; the state after the last
+ *                   scan position.  May equal init_state (in-place carry).
+ *   stream          cudaStream_t to enqueue on.
+ */
+gtr_status_t gtr_gla_fwd(const gtr_half_t *q, const gtr_half_t *k, const gtr_half_t *v,
+                         const gtr_half_t *g, int B, int heads, int Hgrid, int Wgrid,
+                         int dk, int dv, int direction, int chunk,
+                         const float *init_state, gtr_half_t *out, float *final_state,
+                         void *stream);
+
+/*
+ * Syncs `stream`, then reads and clears the device error word (and any sticky
+ * CUDA error).  Returns GTR_OK, GTR_ERR_TIMEOUT or GTR_ERR_CUDA.
+ */
+gtr_status_t gtr_gla_device_status(void *stream);
+
+/* Static text for a status code (never NULL). */
+const char *gtr_status_str(gtr_status_t status);
+
+/*
+ * Launch plan the library would use for a shape on the current device:
+ * writes the cluster size (CTAs cooperating on one sequence), the number of
+ * clusters and the dynamic shared memory per CTA.  Host-only query; returns
+ * GTR_ERR_* like gtr_gla_fwd's argument checks.
+ */
+gtr_status_t gtr_gla_plan(int B, int heads, int Hgrid, int Wgrid, int dk, int dv,
+                          int *cluster_size, int *num_clusters, int *smem_bytes);
+
+/* Library version, "major.minor.patch". */
+const char *gtr_gla_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GTR_GLA_H */

@@ -1,0 +1,143 @@
+"""Python binding of the C ABI in include/gtr_gla.h (argument marshalling only).
+
+Every step of the token mixer runs in the CUDA library ``libgtr_gla.so``; this
+module only checks tensor metadata, passes raw device pointers and the CUDA
+stream through ``ctypes``, and turns status codes into exceptions.  There is no
+CPU or PyTorch fallback: if the library is missing or no GPU is present the
+calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgtr_gla.so")
+
+GTR_OK, GTR_ERR_INVALID_ARG, GTR_ERR_UNSUPPORTED, GTR_ERR_CUDA, GTR_ERR_TIMEOUT = range(5)
+L2R, R2L, T2B, B2T = 0, 1, 2, 3
+
+EXPORTED_SYMBOLS = ("gtr_gla_fwd", "gtr_gla_device_status", "gtr_status_str", "gtr_gla_plan",
+                    "gtr_gla_version")
+
+_lock = threading.Lock()
+_lib = None
+
+
+class GTRError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {status_str(status)} (status {status})")
+        self.status = status
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the CUDA library (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(path):
+            raise RuntimeError(
+                f"{path} is missing: build it with `python -m recurrent_vision_backbone_b200.build`")
+        lib = ctypes.CDLL(path)
+        vp, i = ctypes.c_void_p, ctypes.c_int
+        lib.gtr_gla_fwd.restype = i
+        lib.gtr_gla_fwd.argtypes = [vp, vp, vp, vp] + [i] * 8 + [vp, vp, vp, vp]
+        lib.gtr_gla_device_status.restype = i
+        lib.gtr_gla_device_status.argtypes = [vp]
+        lib.gtr_status_str.restype = ctypes.c_char_p
+        lib.gtr_status_str.argtypes = [i]
+        lib.gtr_gla_plan.restype = i
+        ip = ctypes.POINTER(ctypes.c_int)
+        lib.gtr_gla_plan.argtypes = [i] * 6 + [ip, ip, ip]
+        lib.gtr_gla_version.restype = ctypes.c_char_p
+        _lib = lib
+        return lib
+
+
+def status_str(status: int) -> str:
+    try:
+        return load().gtr_status_str(int(status)).decode()
+    except Exception:  # library not loadable: plain text
+        return {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "CUDA error",
+                4: "device-side wait timed out"}.get(int(status), "unknown status")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def gtr_gla_fwd(q, k, v, g, Hgrid: int, Wgrid: int, direction: int, init_state=None,
+                out=None, final_state=None, chunk: int = 64, stream=None):
+    """One token-mixer call on device tensors.
+
+    q, k, g: fp16 [B, N, heads, dk]; v: fp16 [B, N, heads, dv] (CUDA, contiguous).
+    init_state: fp32 [B, heads, dk, dv] or None.  final_state: an fp32 tensor to
+    fill, True to allocate one, or None to skip it.  Returns (out, final_state).
+    """
+    lib = load()
+    B, N, heads, dk = q.shape
+    dv = v.shape[-1]
+    for name, t in (("q", q), ("k", k), ("g", g), ("v", v)):
+        if t.dtype != torch.float16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA float16 tensor")
+    if k.shape != q.shape or g.shape != q.shape or tuple(v.shape[:3]) != (B, N, heads):
+        raise ValueError("q, k, g must be [B,N,heads,dk] and v [B,N,heads,dv]")
+    if N != Hgrid * Wgrid:
+        raise ValueError(f"N={N} does not match the grid {Hgrid}x{Wgrid}")
+    if out is None:
+        out = torch.empty((B, N, heads, dv), dtype=torch.float16, device=q.device)
+    if final_state is True:
+        final_state = torch.empty((B, heads, dk, dv), dtype=torch.float32, device=q.device)
+    for name, t in (("init_state", init_state), ("final_state", final_state)):
+        if t is not None and (t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous()
+                              or tuple(t.shape) != (B, heads, dk, dv)):
+            raise ValueError(f"{name} must be a contiguous CUDA float32 [B,heads,dk,dv] tensor")
+    st = lib.gtr_gla_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), B, heads, Hgrid, Wgrid, dk, dv,
+                         int(direction), int(chunk), _ptr(init_state), _ptr(out),
+                         _ptr(final_state), _stream_handle(stream))
+    if st != GTR_OK:
+        raise GTRError(st, "gtr_gla_fwd")
+    return out, final_state
+
+
+def gtr_gla_fwd_raw(q_ptr: int, k_ptr: int, v_ptr: int, g_ptr: int, B: int, heads: int,
+                    Hgrid: int, Wgrid: int, dk: int, dv: int, direction: int, chunk: int,
+                    init_ptr: int, out_ptr: int, final_ptr: int, stream_handle: int) -> int:
+    """Direct pass-through of raw pointers; returns the status code."""
+    return load().gtr_gla_fwd(ctypes.c_void_p(q_ptr), ctypes.c_void_p(k_ptr),
+                              ctypes.c_void_p(v_ptr), ctypes.c_void_p(g_ptr), B, heads, Hgrid,
+                              Wgrid, dk, dv, direction, chunk,
+                              ctypes.c_void_p(init_ptr) if init_ptr else None,
+                              ctypes.c_void_p(out_ptr),
+                              ctypes.c_void_p(final_ptr) if final_ptr else None,
+                              ctypes.c_void_p(stream_handle))
+
+
+def device_status(stream=None) -> int:
+    """Sync the stream; return (and clear) the device error status."""
+    return int(load().gtr_gla_device_status(_stream_handle(stream)))
+
+
+def plan(B: int, heads: int, Hgrid: int, Wgrid: int, dk: int, dv: int):
+    """(cluster_size, num_clusters, smem_bytes) the library would launch with."""
+    lib = load()
+    a, b, c = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    st = lib.gtr_gla_plan(B, heads, Hgrid, Wgrid, dk, dv, ctypes.byref(a), ctypes.byref(b),
+                          ctypes.byref(c))
+    if st != GTR_OK:
+        raise GTRError(st, "gtr_gla_plan")
+    return a.value, b.value, c.value
+
+
+def version() -> str:
+    return load().gtr_gla_version().decode()

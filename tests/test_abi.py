@@ -1,0 +1,61 @@
+"""The C-ABI library loads and exports every symbol include/gtr_gla.h declares (CPU only).
+
+No compute call is made here; host-only queries that need no GPU are exercised.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from recurrent_vision_backbone_b200 import build, gla
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gtr_gla.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"\b(gtr_[a-z_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib_path():
+    return build.build()
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    assert "gtr_gla_fwd" in names and "gtr_gla_device_status" in names
+    assert set(names) == set(gla.EXPORTED_SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol(lib_path):
+    out = subprocess.run(["nm", "-D", "--defined-only", lib_path], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r"\bT (gtr_\w+)", out))
+    missing = set(declared_functions()) - exported
+    assert not missing, f"not exported: {missing}"
+
+
+def test_library_loads_and_answers_host_queries(lib_path):
+    lib = gla.load(lib_path)
+    assert gla.version().count(".") == 2
+    assert gla.status_str(gla.GTR_ERR_TIMEOUT) == "device-side wait timed out"
+    assert lib.gtr_status_str(99) == b"unknown status"
+
+
+def test_library_is_built_for_sm100a(lib_path):
+    # the fat binary must carry sm_100a code (cuobjdump-free check: nvcc's -gencode is in
+    # the build command and the ELF has an .nv_fatbin section)
+    assert "arch=compute_100a,code=sm_100a" in " ".join(build.nvcc_cmd())
+    out = subprocess.run(["readelf", "-S", lib_path], capture_output=True, text=True).stdout
+    assert ".nv_fatbin" in out
+
+
+def test_header_compiles_as_c(tmp_path):
+    src = tmp_path / "t.c"
+    src.write_text('#include "gtr_gla.h"\nint main(void){ return (int)GTR_OK; }\n')
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-o", str(tmp_path / "t")], check=True)
