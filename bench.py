@@ -36,7 +36,7 @@ sys.path.insert(0, ROOT)
 import torch  # noqa: E402
 import torch.distributed as dist  # noqa: E402
 
-from recurrent_vision_backbone_b200.inputs import WORKLOADS, make_inputs  # noqa: E402
+from recurrent_vision_backbone_b200.inputs import DIR_NAMES, WORKLOADS, make_inputs  # noqa: E402
 
 METRIC = "GLA fwd tokens/s at 1.6K & 16.4K tokens (FP16, C=64); % of roofline"
 PRIMARY = "gtr640_b1h16_40x40"
@@ -153,6 +153,29 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+# ------------------------------------------------------------------ ranks
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Seed of a rank's inputs: every rank draws its own independent batch (weak scaling)."""
+    return int(base_seed) + 7919 * int(rank)
+
+
+def shard_sequences(n_seq: int, world: int, rank: int) -> range:
+    """Contiguous slice of the (batch, head) sequences a rank owns when one batch is split
+    across ranks; sequences are independent, so no collective is needed on the data path."""
+    lo = n_seq * rank // world
+    hi = n_seq * (rank + 1) // world
+    return range(lo, hi)
+
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    """Max of a per-rank measurement over all ranks (timings are reported as the max)."""
+    if world <= 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ------------------------------------------------------------------ GPU arm
 class Workload:
     """Rotating device-resident input sets for one workload and the graph that
@@ -164,14 +187,14 @@ class Workload:
         self.w = w
         per_call = bytes_alg(w)
         if n_sets is None:
-            n_sets = max(4, -(-4 * L2_BYTES // (per_call * len(DIRS))))
+            n_sets = max(4, -(-4 * L2_BYTES // (per_call * len(w.call_directions()))))
         self.n_sets = int(n_sets)
         self.sets = []
         for s in range(self.n_sets):
             calls = []
-            for d in DIRS:
+            for c, d in enumerate(w.call_directions()):
                 inp = make_inputs(w.B, w.heads, w.H, w.W, w.dk, w.dv,
-                                  seed=w.seed(d, 100 + s) + 7919 * rank,
+                                  seed=rank_seed(w.seed(d, 100 + 16 * s + c), rank),
                                   init_std=w.init_std, z_mean_per_head=w.z_mean_per_head,
                                   device=device)
                 out = torch.empty((w.B, w.N, w.heads, w.dv), dtype=torch.float16, device=device)
@@ -198,8 +221,11 @@ class Workload:
         self.graph = g
         return self.n_sets  # steps per replay
 
+    def calls_per_step(self):
+        return len(self.w.call_directions())
+
     def tokens_per_step(self):
-        return len(DIRS) * self.w.B * self.w.N
+        return self.calls_per_step() * self.w.B * self.w.N
 
 
 def timed_replays(wl, replays, stream, world):
@@ -207,27 +233,24 @@ def timed_replays(wl, replays, stream, world):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    start.record(stream)
-    for _ in range(replays):
-        wl.graph.replay()
-    end.record(stream)
+    with torch.cuda.stream(stream):   # replay on the stream the events are recorded on
+        start.record(stream)
+        for _ in range(replays):
+            wl.graph.replay()
+        end.record(stream)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    ms = start.elapsed_time(end)
-    if world > 1:
-        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    return ms
+    return max_over_ranks(start.elapsed_time(end), world, "cuda")
 
 
 def measure(wl, steps, warmup, stream, world):
     per_replay = wl.capture(stream)
     replays = max(1, -(-steps // per_replay))
     warm = max(1, -(-warmup // per_replay))
-    for _ in range(warm):
-        wl.graph.replay()
+    with torch.cuda.stream(stream):
+        for _ in range(warm):
+            wl.graph.replay()
     torch.cuda.synchronize()
     assert wl.gla.device_status() == wl.gla.GTR_OK
     ms = timed_replays(wl, replays, stream, world)
@@ -245,41 +268,44 @@ def roofline(w, ms_per_launch, workload_name):
             "peak_source": which, "bytes_alg_per_launch": b, "flops_alg_per_launch": flops_alg(w)}
 
 
+def call_inputs(w, d, seed, heads=None, device="cpu"):
+    """Inputs of one call of workload w (optionally only its first `heads` heads)."""
+    h = w.heads if heads is None else heads
+    zm = None if w.z_mean_per_head is None else tuple(w.z_mean_per_head[:h])
+    return make_inputs(w.B, h, w.H, w.W, w.dk, w.dv, seed=seed, init_std=w.init_std,
+                       z_mean_per_head=zm, device=device)
+
+
 def e2e_measure(w, steps, device, rank):
     """Tokens/s through the public call with host buffers: every step copies that
     step's inputs from pinned host memory and reads the outputs back."""
     from recurrent_vision_backbone_b200 import gla
-    host = []
-    for d in DIRS:
-        inp = make_inputs(w.B, w.heads, w.H, w.W, w.dk, w.dv, seed=w.seed(d, 500) + 7919 * rank,
-                          init_std=w.init_std, z_mean_per_head=w.z_mean_per_head)
-        hp = {n: (t.pin_memory() if t is not None else None) for n, t in inp.items()}
-        host.append((d, hp))
-    dev = {d: {n: (torch.empty_like(t, device=device) if t is not None else None)
-               for n, t in hp.items()} for d, hp in host}
-    outs = {d: torch.empty((w.B, w.N, w.heads, w.dv), dtype=torch.float16, device=device)
-            for d in DIRS}
-    sfs = {d: (torch.empty((w.B, w.heads, w.dk, w.dv), dtype=torch.float32, device=device)
-               if w.final_state else None) for d in DIRS}
-    h_out = {d: torch.empty_like(outs[d], device="cpu").pin_memory() for d in DIRS}
-    h_sf = {d: (torch.empty_like(sfs[d], device="cpu").pin_memory() if w.final_state else None)
-            for d in DIRS}
+    calls = []
+    for c, d in enumerate(w.call_directions()):
+        inp = call_inputs(w, d, rank_seed(w.seed(d, 500 + c), rank))
+        hp = {n: t.pin_memory() for n, t in inp.items() if t is not None}
+        dv = {n: torch.empty_like(t, device=device) for n, t in hp.items()}
+        out = torch.empty((w.B, w.N, w.heads, w.dv), dtype=torch.float16, device=device)
+        sf = (torch.empty((w.B, w.heads, w.dk, w.dv), dtype=torch.float32, device=device)
+              if w.final_state else None)
+        h_out = torch.empty_like(out, device="cpu").pin_memory()
+        h_sf = None if sf is None else torch.empty_like(sf, device="cpu").pin_memory()
+        calls.append((d, hp, dv, out, sf, h_out, h_sf))
     stream = torch.cuda.current_stream()
-    h2d = sum(t.numel() * t.element_size() for _, hp in host for t in hp.values() if t is not None)
-    d2h = sum(o.numel() * o.element_size() for o in h_out.values()) + sum(
-        s.numel() * s.element_size() for s in h_sf.values() if s is not None)
+    h2d = sum(t.numel() * t.element_size() for c in calls for t in c[1].values())
+    d2h = sum(c[5].numel() * c[5].element_size() + (0 if c[6] is None else
+                                                   c[6].numel() * c[6].element_size())
+              for c in calls)
 
     def one_step():
-        for d, hp in host:
+        for d, hp, dv, out, sf, h_out, h_sf in calls:
             for n, t in hp.items():
-                if t is not None:
-                    dev[d][n].copy_(t, non_blocking=True)
-            gla.gtr_gla_fwd(dev[d]["q"], dev[d]["k"], dev[d]["v"], dev[d]["g"], w.H, w.W, d,
-                            init_state=dev[d]["s0"], out=outs[d], final_state=sfs[d],
-                            stream=stream)
-            h_out[d].copy_(outs[d], non_blocking=True)
-            if sfs[d] is not None:
-                h_sf[d].copy_(sfs[d], non_blocking=True)
+                dv[n].copy_(t, non_blocking=True)
+            gla.gtr_gla_fwd(dv["q"], dv["k"], dv["v"], dv["g"], w.H, w.W, d,
+                            init_state=dv.get("s0"), out=out, final_state=sf, stream=stream)
+            h_out.copy_(out, non_blocking=True)
+            if sf is not None:
+                h_sf.copy_(sf, non_blocking=True)
 
     for _ in range(3):
         one_step()
@@ -307,14 +333,16 @@ def gpu_arm(args):
     from recurrent_vision_backbone_b200 import gla
     gla.load()
     stream = torch.cuda.Stream(device=device)
-    w1 = WORKLOADS[PRIMARY]
+    primary = args.workload
+    w1 = WORKLOADS[primary]
     wl = Workload(w1, rank, device)
     clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
                           else local)
     clocks.start()
     ms, n_steps = measure(wl, args.steps, args.warmup, stream, world)
     clk = clocks.stop()
-    launches = n_steps * len(DIRS)
+    launches = n_steps * wl.calls_per_step()
+    wl_calls = wl.calls_per_step()
     ms_step = ms / n_steps
     value = world * wl.tokens_per_step() * n_steps / (ms * 1e-3)
     line = {
@@ -322,20 +350,22 @@ def gpu_arm(args):
         "steps": n_steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 6),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
         "data": "synthetic",
-        "config": {"workload": PRIMARY, "B": w1.B, "heads": w1.heads, "grid": [w1.H, w1.W],
+        "config": {"workload": primary, "B": w1.B, "heads": w1.heads, "grid": [w1.H, w1.W],
                    "tokens_per_call": w1.B * w1.N, "dk": w1.dk, "dv": w1.dv, "chunk": 64,
-                   "calls_per_step": len(DIRS), "directions": "L2R,R2L,T2B,B2T",
-                   "l2": f"inputs rotate over {wl.n_sets} sets of 4 calls "
-                         f"({wl.n_sets * 4 * bytes_alg(w1) / 2**20:.0f} MiB > 3x L2)",
+                   "calls_per_step": wl.calls_per_step(),
+                   "directions": ",".join(DIR_NAMES[d] for d in w1.call_directions()),
+                   "l2": f"inputs rotate over {wl.n_sets} sets of {wl.calls_per_step()} calls "
+                         f"({wl.n_sets * wl.calls_per_step() * bytes_alg(w1) / 2**20:.0f} MiB"
+                         f" > 3x L2)",
                    "timing": "CUDA graph replay, CUDA events, max over ranks",
                    "parallelism": f"dp{world} (independent batches)"},
-        "roofline": roofline(w1, ms / launches, PRIMARY),
+        "roofline": roofline(w1, ms / launches, primary),
         "gpu_launches": launches,
         "clocks": clk,
     }
     del wl
     torch.cuda.empty_cache()
-    if not args.no_secondary:
+    if not args.no_secondary and primary != SECONDARY:
         w2 = WORKLOADS[SECONDARY]
         wl2 = Workload(w2, rank, device)
         ms2, n2 = measure(wl2, max(8, args.steps // 16), max(3, args.warmup // 16), stream, world)
@@ -343,18 +373,15 @@ def gpu_arm(args):
             "workload": SECONDARY, "tokens_per_call": w2.B * w2.N,
             "value": round(world * wl2.tokens_per_step() * n2 / (ms2 * 1e-3), 1),
             "unit": "tokens/s", "steps": n2, "ms_per_step": round(ms2 / n2, 6),
-            "roofline": roofline(w2, ms2 / (n2 * len(DIRS)), SECONDARY),
-            "gpu_launches": n2 * len(DIRS)}
+            "roofline": roofline(w2, ms2 / (n2 * wl2.calls_per_step()), SECONDARY),
+            "gpu_launches": n2 * wl2.calls_per_step()}
         del wl2
         torch.cuda.empty_cache()
     # end to end through the public call with host buffers
     e_steps = max(3, min(args.steps, args.e2e_steps))
     ems, en, h2d, d2h = e2e_measure(w1, e_steps, device, rank)
-    if world > 1:
-        t = torch.tensor([ems], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ems = float(t.item())
-    line["e2e"] = {"value": round(world * len(DIRS) * w1.B * w1.N * en / (ems * 1e-3), 1),
+    ems = max_over_ranks(ems, world, "cuda")
+    line["e2e"] = {"value": round(world * wl_calls * w1.B * w1.N * en / (ems * 1e-3), 1),
                    "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                    "steps": en}
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
@@ -370,31 +397,32 @@ def gpu_arm(args):
 
 # ------------------------------------------------------------------ CPU arm
 def cpu_baseline(w, budget_s=15.0):
+    """The oracle as it stands, on this host's cores, on whole steps of the workload
+    until the oracle time reaches the budget."""
     import oracle
     oracle.build()
     threads = oracle.max_threads()
-    # time only the oracle calls, on the full head set, for as many steps as fit the budget
-    tok = 0
-    spent = 0.0
-    steps = 0
+    tok, spent, steps = 0, 0.0, 0
     while spent < budget_s and steps < 1000:
-        for d in DIRS:
-            inp = make_inputs(w.B, w.heads, w.H, w.W, w.dk, w.dv, seed=w.seed(d, 900 + steps),
-                              init_std=w.init_std, z_mean_per_head=w.z_mean_per_head)
-            f = {n: t.float().numpy() for n, t in inp.items() if t is not None}
+        for c, d in enumerate(w.call_directions()):
+            f = {n: t.float().numpy() for n, t in call_inputs(w, d, w.seed(d, 900 + c)).items()
+                 if t is not None}
             t1 = time.perf_counter()
             oracle.gla_forward(f["q"], f["k"], f["v"], f["g"], w.H, w.W, d, f.get("s0"))
             spent += time.perf_counter() - t1
             tok += w.B * w.N
         steps += 1
+    ncalls = steps * len(w.call_directions())
     return {"value": round(tok / spent, 1), "unit": "tokens/s", "cores": threads,
             "kind": "oracle",
-            "sample": f"{steps} full steps ({steps * len(DIRS)} calls) of {w.name}, "
-                      f"fp64 token-by-token, OpenMP over the {w.B * w.heads} sequences; "
-                      f"oracle time only ({spent:.1f} s)"}
+            "sample": f"{steps} full steps ({ncalls} calls) of {w.name}, fp64 token-by-token, "
+                      f"OpenMP over the {w.B * w.heads} sequences; oracle time only "
+                      f"({spent:.1f} s)"}
 
 
 def reference_arm(args):
+    """The reference arm: the fp64 oracle on this host's cores, on a per-step sample of
+    the workload's heads sized so that warmup + steps end within about two minutes."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -402,35 +430,37 @@ def reference_arm(args):
     import oracle
     oracle.build()
     threads = oracle.max_threads()
-    w = WORKLOADS[PRIMARY]
-    # size the per-step sample so that warmup + steps stay within ~2 minutes
-    probe = time.perf_counter()
-    f = {n: t.float().numpy() for n, t in make_inputs(w.B, 1, w.H, w.W, w.dk, w.dv, seed=1).items()
+    w = WORKLOADS[args.workload]
+    dirs = w.call_directions()
+    f = {n: t.float().numpy() for n, t in call_inputs(w, dirs[0], 1, heads=1).items()
          if t is not None}
-    oracle.gla_forward(f["q"], f["k"], f["v"], f["g"], w.H, w.W, 0)
-    per_head_call = max(time.perf_counter() - probe, 1e-4)
-    total_calls = (args.steps + args.warmup) * len(DIRS)
+    t0 = time.perf_counter()
+    oracle.gla_forward(f["q"], f["k"], f["v"], f["g"], w.H, w.W, dirs[0], f.get("s0"))
+    per_head_call = max(time.perf_counter() - t0, 1e-4)
+    total_calls = (args.steps + args.warmup) * len(dirs)
     heads = int(max(1, min(w.heads, 120.0 / (total_calls * per_head_call))))
     spent = 0.0
     for it in range(args.warmup + args.steps):
-        for d in DIRS:
-            inp = make_inputs(w.B, heads, w.H, w.W, w.dk, w.dv, seed=w.seed(d, 900 + it))
-            f = {n: t.float().numpy() for n, t in inp.items() if t is not None}
+        for c, d in enumerate(dirs):
+            f = {n: t.float().numpy() for n, t in
+                 call_inputs(w, d, w.seed(d, 900 + 16 * it + c), heads=heads).items()
+                 if t is not None}
             t1 = time.perf_counter()
-            oracle.gla_forward(f["q"], f["k"], f["v"], f["g"], w.H, w.W, d)
+            oracle.gla_forward(f["q"], f["k"], f["v"], f["g"], w.H, w.W, d, f.get("s0"))
             if it >= args.warmup:
                 spent += time.perf_counter() - t1
     frac = heads / w.heads
-    tokens = args.steps * len(DIRS) * w.B * w.N * frac
+    tokens = args.steps * len(dirs) * w.B * w.N * frac
     value = tokens / spent
     sample = (f"{heads} of {w.heads} heads of {w.name} per call (tokens scaled by "
-              f"{frac:.4f}), {args.steps} timed steps x 4 directions, fp64 token-by-token oracle")
+              f"{frac:.4f}), {args.steps} timed steps x {len(dirs)} calls, fp64 "
+              f"token-by-token oracle, {threads} OpenMP threads")
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 1), "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(spent / args.steps * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": PRIMARY, "B": w.B, "heads": w.heads, "grid": [w.H, w.W],
-                       "dk": w.dk, "dv": w.dv, "chunk": 64, "calls_per_step": len(DIRS)},
+            "config": {"workload": w.name, "B": w.B, "heads": w.heads, "grid": [w.H, w.W],
+                       "dk": w.dk, "dv": w.dv, "chunk": 64, "calls_per_step": len(dirs)},
             "cpu_baseline": {"value": round(value, 1), "unit": "tokens/s", "cores": threads,
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": round(value, 1), "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -444,6 +474,8 @@ def main():
     ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=400)
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=PRIMARY,
+                    help="workload timed as the headline (default: the 1.6K-token one)")
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-secondary", action="store_true")

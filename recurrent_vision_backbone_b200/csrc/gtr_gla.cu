@@ -34,6 +34,7 @@
 
 #include <cstdint>
 #include <cstdio>
+#include <cstdlib>
 #include <mutex>
 
 #include "../../include/gtr_gla.h"
@@ -51,6 +52,9 @@ constexpr int kTile = 64 * 128;       // one [64 rows][64 fp16] 128B-swizzled ti
 constexpr int kTmemCols = 256;
 constexpr int kMaxCluster = 16;
 constexpr float kDiagMinTotal = 3.3546262e-4f;  // exp(-8): smallest safe sub-block total
+constexpr float kFastMinDecay = 2.4787522e-3f;  // exp(-6): smallest chunk decay for the fast path
+constexpr float kFastMaxK = 100.f;              // |k| / P stays inside fp16 on the fast path
+constexpr float kDiagMaxQ = 20.f;               // |q| / T stays inside fp16 on a diagonal block
 constexpr uint64_t kWaitLimitNs = 200ull * 1000ull * 1000ull;  // 200 ms per bounded wait
 
 enum : unsigned { kErrTimeout = 1u };
@@ -58,38 +62,37 @@ enum : unsigned { kErrTimeout = 1u };
 __device__ unsigned int g_error_word;
 
 // ------------------------------------------------------------------ smem map
+// The q and k tiles are overwritten in place by the gated operands (Qint, and
+// K/P or K*sigma*after): ~104 KB per CTA at dk=64, ~182 KB at dk=128.
 template <int DK>
 struct Smem {
     static constexpr int NSUB = DK / 64;
-    static constexpr int q = 0;
-    static constexpr int k = q + NSUB * kTile;
-    static constexpr int g = k + NSUB * kTile;
-    static constexpr int v0 = g + NSUB * kTile;
+    static constexpr int q = 0;                           // raw q, then Q*pi*before   [64][DK]
+    static constexpr int k = q + NSUB * kTile;            // raw k, then K/P or K*sig*after
+    static constexpr int g = k + NSUB * kTile;            // raw g                     [64][DK]
+    static constexpr int v0 = g + NSUB * kTile;           // v, double buffered        [64][64]
     static constexpr int v1 = v0 + kTile;
     static constexpr int qj = v1 + kTile;                 // packed Q^(J), rows 16J..63
     static constexpr int qj_bytes = NSUB * (64 + 48 + 32 + 16) * 128;
-    static constexpr int kbar = qj + qj_bytes;            // K * sigma          [64][DK]
-    static constexpr int qint = kbar + NSUB * kTile;      // Q * pi * before    [64][DK]
-    static constexpr int kst = qint + NSUB * kTile;       // K * sigma * after  [64][DK]
-    static constexpr int p = kst + NSUB * kTile;          // masked scores      [64][64]
-    static constexpr int sop = p + kTile;                 // S_prev fp16        [DK][64]
-    static constexpr int agg = sop + NSUB * kTile;        // dS fp32            [DK][64]
-    static constexpr int dvec = agg + DK * 256;           // d = prod of a      [DK]
-    static constexpr int tsh = dvec + DK * 4;             // sub-block totals   [4][DK]
-    static constexpr int diag = tsh + 4 * DK * 4;         // exact diag blocks  [4][16][16]
-    static constexpr int rowoff = diag + 4 * 16 * 16 * 4; // token rows         [2][64]
-    static constexpr int misc = rowoff + 2 * 64 * 4;      // flags, mbarrier, tmem addr
+    static constexpr int kbar = qj + qj_bytes;            // K * sigma                 [64][DK]
+    static constexpr int p = kbar + NSUB * kTile;         // masked scores / out staging [64][64]
+    static constexpr int sop = p + kTile;                 // S_prev fp16               [DK][64]
+    static constexpr int diag = sop;                      // exact diag blocks, aliases sop
+    static constexpr int agg = sop + NSUB * kTile;        // dS fp32                   [DK][64]
+    static constexpr int dvec = agg + DK * 256;           // d = prod of a             [DK]
+    static constexpr int htot = dvec + DK * 4;            // half-block totals         [8][DK]
+    static constexpr int rowoff = htot + 8 * DK * 4;      // token rows                [2][64]
+    static constexpr int misc = rowoff + 2 * 64 * 4;      // flags, maxima, mbarrier, tmem addr
     static constexpr int bytes = misc + 64;
     static constexpr int alloc = bytes + 1024;            // + alignment slack
-    // scan staging aliases the Q^(J) region (free between MMA completion and the
-    // next round's gating): float4 [P][slice] then float [P][DK]
-    static constexpr int stage = qj;
-    static constexpr int stage_bytes = qj_bytes;
+    static constexpr int min_blocks = 1;   // thread-block clusters never co-reside two per SM here
 
     static __host__ __device__ constexpr int qj_region(int J) {
         return NSUB * 128 * (J == 0 ? 0 : J == 1 ? 64 : J == 2 ? 112 : 144);
     }
 };
+static_assert(Smem<128>::alloc <= 227 * 1024, "dk=128 fits one CTA per SM");
+static_assert(4 * 16 * 16 * 4 <= 64 * 128, "diag blocks fit in the aliased S_prev tile");
 
 // 128B-swizzled [rows][64 fp16] tile: byte offset of (row, col) inside a sub-tile
 __device__ __forceinline__ uint32_t sw_off(int row, int col) {
@@ -126,41 +129,35 @@ struct Params {
 __device__ __forceinline__ void set_error(unsigned e) { atomicOr(&g_error_word, e); }
 
 // ------------------------------------------------------------------ loads
-// Issues the cp.async copies of one chunk's q/k/g (into the shared raw tiles)
-// and v (into vbuf); rows with rowoff < 0 are zero-filled.
+// 16-byte cp.async copies of one chunk's rows into 128B-swizzled tiles; two rows
+// per thread (tensor pair x 64 rows = 128 threads each half of the block).  Rows
+// whose token index is negative (past the end of the grid) are zero-filled.
+// which == 0: g and v (v into vbuf); which == 1: q and k.
 template <int DK>
-__device__ __forceinline__ void issue_chunk_loads(const Params &P, uint8_t *sm, const int *rowoff,
-                                                  uint32_t vbuf_addr) {
+__device__ __forceinline__ void issue_loads(const Params &P, uint32_t sbase, const int *rowoff,
+                                            uint32_t vbuf_addr, int which) {
     using L = Smem<DK>;
-    constexpr int CPR = DK / 8;              // 16-byte pieces per q/k/g row
-    constexpr int QKG = 3 * 64 * CPR;
-    constexpr int TOTAL = QKG + 64 * 8;
-    const uint32_t base = smem_u32(sm);
     const int tid = threadIdx.x;
-#pragma unroll 4
-    for (int pid = tid; pid < TOTAL; pid += kThreads) {
-        const __half *src;
-        uint32_t dst;
-        int row;
-        if (pid < QKG) {
-            const int tsel = pid / (64 * CPR);
-            const int rem = pid - tsel * (64 * CPR);
-            row = rem / CPR;
-            const int cc = rem - row * CPR;
-            const __half *tb = tsel == 0 ? P.q : (tsel == 1 ? P.k : P.g);
-            const int ro = rowoff[row];
-            src = tb + (size_t)(ro < 0 ? 0 : ro) * DK + cc * 8;
-            const uint32_t tile = base + (tsel == 0 ? L::q : (tsel == 1 ? L::k : L::g));
-            dst = tile + (cc >> 3) * kTile + sw_off(row, (cc & 7) * 8);
-            cp_async16(dst, src, ro < 0 ? 0u : 16u);
-        } else {
-            const int rem = pid - QKG;
-            row = rem >> 3;
-            const int cc = rem & 7;
-            const int ro = rowoff[row];
-            src = P.v + (size_t)(ro < 0 ? 0 : ro) * kDV + cc * 8;
-            dst = vbuf_addr + sw_off(row, cc * 8);
-            cp_async16(dst, src, ro < 0 ? 0u : 16u);
+    const int sel = tid >> 7, row = (tid >> 1) & 63, part = tid & 1;
+    const int ro = rowoff[row];
+    const uint32_t nbytes = ro < 0 ? 0u : 16u;
+    const size_t r0 = (size_t)(ro < 0 ? 0 : ro);
+    if (which == 1 || sel == 0) {
+        // q/k/g row: DK/8 pieces, split between the two threads of the pair
+        const __half *base = which == 1 ? (sel == 0 ? P.q : P.k) : P.g;
+        const uint32_t tile = sbase + (which == 1 ? (sel == 0 ? L::q : L::k) : L::g);
+        const __half *src = base + r0 * DK;
+#pragma unroll
+        for (int i = 0; i < DK / 16; ++i) {
+            const int pc = part * (DK / 16) + i;
+            cp_async16(tile + (pc >> 3) * kTile + sw_off(row, (pc & 7) * 8), src + pc * 8, nbytes);
+        }
+    } else {
+        const __half *src = P.v + r0 * kDV;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int pc = part * 4 + i;
+            cp_async16(vbuf_addr + sw_off(row, pc * 8), src + pc * 8, nbytes);
         }
     }
     cp_async_commit();
@@ -183,11 +180,32 @@ __device__ __forceinline__ void fill_rowoff(const Params &P, int seq, int c, int
     }
 }
 
+__device__ __forceinline__ float2 ld_h2(const uint8_t *p) {
+    return __half22float2(*reinterpret_cast<const __half2 *>(p));
+}
+__device__ __forceinline__ void st_h2(uint8_t *p, float x, float y) {
+    *reinterpret_cast<__half2 *>(p) = __floats2half2_rn(x, y);
+}
+__device__ __forceinline__ float exp_f(float x) { return __expf(x); }
+
+// 16 TMEM lanes x 256 bit, 4 repeats (32 columns): thread t gets, for repeat c,
+// rows (lane base + t/4, + 8) and columns (col + 8c + 2(t%4), +1).
+__device__ __forceinline__ void tmem_ld_16x256b_x4(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+}
+
 // ------------------------------------------------------------------ kernel
 template <int DK>
-__global__ void __launch_bounds__(kThreads, 1) gla_fwd_kernel(const Params P) {
+__global__ void __launch_bounds__(kThreads, Smem<DK>::min_blocks) gla_fwd_kernel(const Params P) {
     using L = Smem<DK>;
-    constexpr int ITEMS = DK / 64;        // (channel, sub-block) items per thread in gating
+    constexpr int NP = DK / 64;           // channel pairs per thread in gating
     constexpr int NF4 = DK * kDV / 4;     // float4 elements of the state
     constexpr int MAXM = (NF4 + kThreads - 1) / kThreads;
 
@@ -198,18 +216,19 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_kernel(const Params P) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     const uint32_t rank = cluster_ctarank();
-    // cluster size = gridDim.x / number of clusters
     const uint32_t ncl = nclusters_x();
     const int CP = (int)(gridDim.x / ncl);
     const int cl = (int)cluster_id_x();
 
-    float *tsh = reinterpret_cast<float *>(sm + L::tsh);
+    float *htot = reinterpret_cast<float *>(sm + L::htot);
     float *dvec = reinterpret_cast<float *>(sm + L::dvec);
     float *diagx = reinterpret_cast<float *>(sm + L::diag);
     int *rowoff0 = reinterpret_cast<int *>(sm + L::rowoff);
-    int *flags = reinterpret_cast<int *>(sm + L::misc);          // [4] diag fallback flags
-    uint64_t *mbar = reinterpret_cast<uint64_t *>(sm + L::misc + 16);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::misc + 32);
+    int *flags = reinterpret_cast<int *>(sm + L::misc);                // [4] diag fallback flags
+    unsigned *qmax = reinterpret_cast<unsigned *>(sm + L::misc + 16);  // [4] max |q| per block (bits)
+    unsigned *kmax = reinterpret_cast<unsigned *>(sm + L::misc + 32);  // max |k| in the chunk (bits)
+    uint64_t *mbar = reinterpret_cast<uint64_t *>(sm + L::misc + 40);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::misc + 48);
 
     if (warp == 0) {
         tmem_alloc(tmem_slot, kTmemCols);
@@ -219,7 +238,8 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_kernel(const Params P) {
         mbar_init(mbar, 1);
         fence_mbar_init();
     }
-    if (tid < 4) flags[tid] = 0;
+    if (tid < 4) { flags[tid] = 0; qmax[tid] = 0u; }
+    if (tid == 0) *kmax = 0u;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -227,25 +247,31 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_kernel(const Params P) {
     uint32_t mma_phase = 0;
     bool timed_out = false;
 
+    // gating thread map: warp -> (sub-block I, half hf), lane -> channel pair(s)
+    const int gI = warp >> 1, ghf = warp & 1, gt0 = 16 * gI + 8 * ghf, gh = 2 * gI + ghf;
+    // readout thread map for M=64 accumulators: subpartition, column half
+    const int sp = warp & 3, chalf = warp >> 2;
+    const int rrow0 = 16 * sp + (lane >> 2);          // and rrow0 + 8
+    const int rcol0 = 32 * chalf + 2 * (lane & 3);    // + 8c, +1
+
     // element slice of the state owned by this CTA in the scan
     const int slo = (int)((long)rank * NF4 / CP);
     const int shi = (int)((long)(rank + 1) * NF4 / CP);
     const int nloc = shi - slo;
 
-    int cur = 0;  // rowoff buffer of the current chunk
-    int vb = 0;   // v buffer of the current chunk
-    // prime the first chunk
+    int cur = 0, vb = 0;
     {
         const int seq0 = cl < P.n_seq ? cl : -1;
         const int c0 = (seq0 >= 0 && (int)rank < P.n_chunks) ? (int)rank : -1;
         fill_rowoff(P, seq0, c0, rowoff0);
         __syncthreads();
-        if (c0 >= 0) issue_chunk_loads<DK>(P, sm, rowoff0, sbase + L::v0);
+        if (c0 >= 0) {
+            issue_loads<DK>(P, sbase, rowoff0, sbase + L::v0, 0);
+            issue_loads<DK>(P, sbase, rowoff0, sbase + L::v0, 1);
+        }
     }
 
     for (int seq = cl; seq < P.n_seq; seq += (int)ncl) {
-        const int b = seq / P.heads, h = seq - b * P.heads;
-        // running state for this CTA's slice, fp32 registers
         float4 S[MAXM];
 #pragma unroll
         for (int m = 0; m < MAXM; ++m) {
@@ -263,105 +289,6 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_kernel(const Params P) {
             int *rowoff_nxt = rowoff0 + (cur ^ 1) * 64;
             const uint32_t vaddr = sbase + (vb ? L::v1 : L::v0);
             const uint32_t vnext = sbase + (vb ? L::v0 : L::v1);
-
-            cp_async_wait_all();
-            __syncthreads();
-
-            // ---------------- gating pass 1: a = exp(g), pi, sigma, sub-block totals
-            float pa[ITEMS][16];   // pi (inclusive prefix product inside the sub-block)
-            float sa[ITEMS][16];   // sigma (exclusive suffix product inside the sub-block)
-            if (valid) {
-#pragma unroll
-                for (int it = 0; it < ITEMS; ++it) {
-                    const int item = tid + it * kThreads;
-                    const int i = item % DK, I = item / DK;
-                    const uint8_t *gt = sm + L::g + (i >> 6) * kTile;
-                    float a[16];
-#pragma unroll
-                    for (int u = 0; u < 16; ++u) {
-                        const int t = I * kSub + u;
-                        const float gv = __half2float(
-                            *reinterpret_cast<const __half *>(gt + sw_off(t, i & 63)));
-                        a[u] = __expf(gv);
-                    }
-                    float run = 1.f;
-#pragma unroll
-                    for (int u = 0; u < 16; ++u) { run *= a[u]; pa[it][u] = run; }
-                    run = 1.f;
-#pragma unroll
-                    for (int u = 15; u >= 0; --u) { sa[it][u] = run; run *= a[u]; }
-                    const float T = pa[it][15];
-                    tsh[I * DK + i] = T;
-                    if (!(T >= kDiagMinTotal)) atomicOr(&flags[I], 1);
-                }
-            }
-            __syncthreads();
-
-            // ---------------- gating pass 2: UMMA operands (fp16, swizzled)
-            if (valid) {
-#pragma unroll
-                for (int it = 0; it < ITEMS; ++it) {
-                    const int item = tid + it * kThreads;
-                    const int i = item % DK, I = item / DK;
-                    const int ci = i & 63, si = i >> 6;
-                    float T[4];
-#pragma unroll
-                    for (int L2 = 0; L2 < 4; ++L2) T[L2] = tsh[L2 * DK + i];
-                    float before = 1.f, after = 1.f;
-#pragma unroll
-                    for (int L2 = 0; L2 < 4; ++L2) {
-                        if (L2 < I) before *= T[L2];
-                        if (L2 > I) after *= T[L2];
-                    }
-                    if (I == 0) dvec[i] = T[0] * T[1] * T[2] * T[3];
-                    // coefficient of Q^(J) rows in sub-block I
-                    const bool diag_bad = flags[I] != 0;
-                    float tI = T[0];
-#pragma unroll
-                    for (int L2 = 1; L2 < 4; ++L2)
-                        if (L2 == I) tI = T[L2];
-                    float coef[4];
-#pragma unroll
-                    for (int J = 0; J < 4; ++J) {
-                        float cj = 1.f;
-#pragma unroll
-                        for (int L2 = 0; L2 < 4; ++L2)
-                            if (L2 > J && L2 < I) cj *= T[L2];
-                        coef[J] = (J == I) ? (diag_bad ? 0.f : 1.f / tI) : cj;
-                    }
-                    const uint8_t *qt = sm + L::q + si * kTile;
-                    const uint8_t *kt = sm + L::k + si * kTile;
-#pragma unroll
-                    for (int u = 0; u < 16; ++u) {
-                        const int t = I * kSub + u;
-                        const uint32_t o = sw_off(t, ci);
-                        const float qv = __half2float(*reinterpret_cast<const __half *>(qt + o));
-                        const float kv = __half2float(*reinterpret_cast<const __half *>(kt + o));
-                        const float qp = qv * pa[it][u];
-                        const float ks = kv * sa[it][u];
-                        *reinterpret_cast<__half *>(sm + L::qint + si * kTile + o) =
-                            __float2half_rn(qp * before);
-                        *reinterpret_cast<__half *>(sm + L::kbar + si * kTile + o) =
-                            __float2half_rn(ks);
-                        *reinterpret_cast<__half *>(sm + L::kst + si * kTile + o) =
-                            __float2half_rn(ks * after);
-#pragma unroll
-                        for (int J = 0; J < 4; ++J) {
-                            if (J <= I) {
-                                float val = qp * coef[J];
-                                if (J == I && !(fabsf(val) <= 60000.f)) {
-                                    val = 0.f;
-                                    atomicOr(&flags[I], 2);
-                                }
-                                const int rows_j = 64 - 16 * J;
-                                uint8_t *dst = sm + L::qj + L::qj_region(J) + si * rows_j * 128 +
-                                               sw_off(t - 16 * J, ci);
-                                *reinterpret_cast<__half *>(dst) = __float2half_rn(val);
-                            }
-                        }
-                    }
-                }
-            }
             // rows of the next chunk (this sequence, or the first round of the next)
             int nseq = seq, nc = c + CP;
             if (nc >= P.n_chunks) {
@@ -370,53 +297,235 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_kernel(const Params P) {
                 if (nseq >= P.n_seq) nseq = -1;
             }
             fill_rowoff(P, nseq, nc, rowoff_nxt);
-            fence_proxy_async_cta();
+
+            cp_async_wait_all();
             __syncthreads();
 
-            // ---------------- exact diagonal sub-blocks where the factorisation is unsafe
-            const int anyflag = valid ? (flags[0] | flags[1] | flags[2] | flags[3]) : 0;
-            if (anyflag) {
-                const uint8_t *qt = sm + L::q, *kt = sm + L::k, *gt = sm + L::g;
-                for (int pr = tid; pr < 4 * 256; pr += kThreads) {
-                    const int I = pr >> 8, u = (pr >> 4) & 15, w = pr & 15;
-                    if (!flags[I] || w > u) continue;
-                    const int tu = I * kSub + u, tw = I * kSub + w;
-                    float acc = 0.f;
-                    for (int i = 0; i < DK; ++i) {
-                        const int si = i >> 6, ci = i & 63;
-                        float lg = 0.f;
-                        for (int rr = tw + 1; rr <= tu; ++rr)
-                            lg += __half2float(*reinterpret_cast<const __half *>(
-                                gt + si * kTile + sw_off(rr, ci)));
-                        const float qv = __half2float(
-                            *reinterpret_cast<const __half *>(qt + si * kTile + sw_off(tu, ci)));
-                        const float kv = __half2float(
-                            *reinterpret_cast<const __half *>(kt + si * kTile + sw_off(tw, ci)));
-                        acc += qv * kv * __expf(lg);
+            bool slow = false;   // CTA-uniform: sub-block factorisation for this chunk
+            if (valid) {
+                // ------------- gating pass 1: a = exp(g); half-block prefix/suffix products
+                float pl[8][2 * NP], sl[8][2 * NP];
+                __half2 qh[8][NP], kh[8][NP];
+                float qm = 0.f, km = 0.f;
+#pragma unroll
+                for (int p2 = 0; p2 < NP; ++p2) {
+                    float a0[8], a1[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const uint32_t o = p2 * kTile + sw_off(gt0 + u, 2 * lane);
+                        const float2 gv = ld_h2(sm + L::g + o);
+                        qh[u][p2] = *reinterpret_cast<const __half2 *>(sm + L::q + o);
+                        kh[u][p2] = *reinterpret_cast<const __half2 *>(sm + L::k + o);
+                        a0[u] = exp_f(gv.x);
+                        a1[u] = exp_f(gv.y);
+                        const float2 qf = __half22float2(qh[u][p2]), kf = __half22float2(kh[u][p2]);
+                        qm = fmaxf(qm, fmaxf(fabsf(qf.x), fabsf(qf.y)));
+                        km = fmaxf(km, fmaxf(fabsf(kf.x), fabsf(kf.y)));
                     }
-                    diagx[(I * 16 + u) * 16 + w] = acc;
+                    float r0 = 1.f, r1 = 1.f;
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        r0 *= a0[u]; r1 *= a1[u];
+                        pl[u][2 * p2] = r0; pl[u][2 * p2 + 1] = r1;
+                    }
+                    r0 = 1.f; r1 = 1.f;
+#pragma unroll
+                    for (int u = 7; u >= 0; --u) {
+                        sl[u][2 * p2] = r0; sl[u][2 * p2 + 1] = r1;
+                        r0 *= a0[u]; r1 *= a1[u];
+                    }
+                    *reinterpret_cast<float2 *>(htot + gh * DK + 64 * p2 + 2 * lane) =
+                        make_float2(pl[7][2 * p2], pl[7][2 * p2 + 1]);
+                }
+                // block maxima of |q| and chunk maximum of |k| (non-negative floats order as uints)
+                {
+                    const unsigned wq = __reduce_max_sync(0xffffffffu, __float_as_uint(qm));
+                    const unsigned wk = __reduce_max_sync(0xffffffffu, __float_as_uint(km));
+                    if (lane == 0) {
+                        atomicMax(&qmax[gI], wq);
+                        atomicMax(kmax, wk);
+                    }
                 }
                 __syncthreads();
+                // ------------- chunk-level factors for my channels
+                float dch[2 * NP], bef[2 * NP], aft[2 * NP];
+                bool bad = __uint_as_float(*kmax) > kFastMaxK;
+#pragma unroll
+                for (int p2 = 0; p2 < NP; ++p2) {
+                    float2 ht[8];
+#pragma unroll
+                    for (int h8 = 0; h8 < 8; ++h8)
+                        ht[h8] = *reinterpret_cast<const float2 *>(htot + h8 * DK + 64 * p2 + 2 * lane);
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        float d = 1.f, bf = 1.f, af = 1.f;
+#pragma unroll
+                        for (int h8 = 0; h8 < 8; ++h8) {
+                            const float x = e ? ht[h8].y : ht[h8].x;
+                            d *= x;
+                            if (h8 < gh) bf *= x;
+                            if (h8 > gh) af *= x;
+                        }
+                        dch[2 * p2 + e] = d; bef[2 * p2 + e] = bf; aft[2 * p2 + e] = af;
+                        bad |= !(d >= kFastMinDecay);
+                    }
+                }
+                slow = __syncthreads_or(bad) != 0;
+                if (gh == 0) {
+#pragma unroll
+                    for (int p2 = 0; p2 < NP; ++p2)
+                        *reinterpret_cast<float2 *>(dvec + 64 * p2 + 2 * lane) =
+                            make_float2(dch[2 * p2], dch[2 * p2 + 1]);
+                }
+                if (!slow) {
+                    // ------------- fast path (in place): Qint = q * P, Kt = k / P  (P >= e^-6)
+#pragma unroll
+                    for (int p2 = 0; p2 < NP; ++p2) {
+                        const float i0 = aft[2 * p2] / dch[2 * p2];
+                        const float i1 = aft[2 * p2 + 1] / dch[2 * p2 + 1];
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            const uint32_t o = p2 * kTile + sw_off(gt0 + u, 2 * lane);
+                            const float2 qv = __half22float2(qh[u][p2]);
+                            const float2 kv = __half22float2(kh[u][p2]);
+                            st_h2(sm + L::q + o, qv.x * (pl[u][2 * p2] * bef[2 * p2]),
+                                  qv.y * (pl[u][2 * p2 + 1] * bef[2 * p2 + 1]));
+                            st_h2(sm + L::k + o, kv.x * (sl[u][2 * p2] * i0),
+                                  kv.y * (sl[u][2 * p2 + 1] * i1));
+                        }
+                    }
+                } else {
+                    // ------------- sub-block path: every off-diagonal factor <= 1
+                    float T[4][2 * NP];
+#pragma unroll
+                    for (int p2 = 0; p2 < NP; ++p2)
+#pragma unroll
+                        for (int L4 = 0; L4 < 4; ++L4) {
+                            const float2 h0 = *reinterpret_cast<const float2 *>(
+                                htot + (2 * L4) * DK + 64 * p2 + 2 * lane);
+                            const float2 h1 = *reinterpret_cast<const float2 *>(
+                                htot + (2 * L4 + 1) * DK + 64 * p2 + 2 * lane);
+                            T[L4][2 * p2] = h0.x * h1.x;
+                            T[L4][2 * p2 + 1] = h0.y * h1.y;
+                        }
+                    // diagonal sub-block I needs the exact path if some channel decays by more
+                    // than e^8 inside it, or if q * e^8 could leave the fp16 range
+                    bool dbad = false;
+#pragma unroll
+                    for (int j = 0; j < 2 * NP; ++j)
+#pragma unroll
+                        for (int L4 = 0; L4 < 4; ++L4)
+                            if (L4 == gI) dbad |= !(T[L4][j] >= kDiagMinTotal);
+                    dbad |= __uint_as_float(qmax[gI]) > kDiagMaxQ;
+                    if (__any_sync(0xffffffffu, dbad) && lane == 0) atomicOr(&flags[gI], 1);
+                    __syncthreads();
+                    const int anyflag = flags[0] | flags[1] | flags[2] | flags[3];
+                    if (anyflag) {
+                        // exact fp32 diagonal sub-blocks, from the raw tiles (still intact)
+                        const uint8_t *qt = sm + L::q, *kt = sm + L::k, *gt = sm + L::g;
+                        for (int pr = tid; pr < 4 * 256; pr += kThreads) {
+                            const int I = pr >> 8, u = (pr >> 4) & 15, w = pr & 15;
+                            if (!flags[I] || w > u) continue;
+                            const int tu = I * kSub + u, tw = I * kSub + w;
+                            float acc = 0.f;
+                            for (int i = 0; i < DK; ++i) {
+                                const int si = i >> 6, ci = i & 63;
+                                float lg = 0.f;
+                                for (int rr = tw + 1; rr <= tu; ++rr)
+                                    lg += __half2float(*reinterpret_cast<const __half *>(
+                                        gt + si * kTile + sw_off(rr, ci)));
+                                const float qv = __half2float(*reinterpret_cast<const __half *>(
+                                    qt + si * kTile + sw_off(tu, ci)));
+                                const float kv = __half2float(*reinterpret_cast<const __half *>(
+                                    kt + si * kTile + sw_off(tw, ci)));
+                                acc += qv * kv * exp_f(lg);
+                            }
+                            diagx[(I * 16 + u) * 16 + w] = acc;
+                        }
+                        __syncthreads();
+                    }
+                    const bool diag_bad = flags[gI] != 0;
+#pragma unroll
+                    for (int p2 = 0; p2 < NP; ++p2) {
+                        float cf[2][4], bI[2], aI[2], hin[2], hout[2];
+                        const float2 h0 = *reinterpret_cast<const float2 *>(
+                            htot + (2 * gI) * DK + 64 * p2 + 2 * lane);
+                        const float2 h1 = *reinterpret_cast<const float2 *>(
+                            htot + (2 * gI + 1) * DK + 64 * p2 + 2 * lane);
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int j = 2 * p2 + e;
+                            float b0 = 1.f, a0 = 1.f, tI = 1.f;
+#pragma unroll
+                            for (int L4 = 0; L4 < 4; ++L4) {
+                                if (L4 < gI) b0 *= T[L4][j];
+                                if (L4 > gI) a0 *= T[L4][j];
+                                if (L4 == gI) tI = T[L4][j];
+                            }
+                            bI[e] = b0; aI[e] = a0;
+#pragma unroll
+                            for (int J = 0; J < 4; ++J) {
+                                float cj = 1.f;
+#pragma unroll
+                                for (int L4 = 0; L4 < 4; ++L4)
+                                    if (L4 > J && L4 < gI) cj *= T[L4][j];
+                                cf[e][J] = (J == gI) ? (diag_bad ? 0.f : 1.f / tI) : cj;
+                            }
+                            // pi / sigma inside the 16-block from the half-local products
+                            hin[e] = ghf ? (e ? h0.y : h0.x) : 1.f;
+                            hout[e] = ghf ? 1.f : (e ? h1.y : h1.x);
+                        }
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            const int t = gt0 + u;
+                            const uint32_t o = p2 * kTile + sw_off(t, 2 * lane);
+                            const float2 qv = __half22float2(qh[u][p2]);
+                            const float2 kv = __half22float2(kh[u][p2]);
+                            const float qp0 = qv.x * (pl[u][2 * p2] * hin[0]);
+                            const float qp1 = qv.y * (pl[u][2 * p2 + 1] * hin[1]);
+                            const float ks0 = kv.x * (sl[u][2 * p2] * hout[0]);
+                            const float ks1 = kv.y * (sl[u][2 * p2 + 1] * hout[1]);
+                            st_h2(sm + L::q + o, qp0 * bI[0], qp1 * bI[1]);
+                            st_h2(sm + L::kbar + o, ks0, ks1);
+                            st_h2(sm + L::k + o, ks0 * aI[0], ks1 * aI[1]);
+#pragma unroll
+                            for (int J = 0; J < 4; ++J) {
+                                if (J <= gI) {
+                                    const int rows_j = 64 - 16 * J;
+                                    st_h2(sm + L::qj + L::qj_region(J) + p2 * rows_j * 128 +
+                                              sw_off(t - 16 * J, 2 * lane),
+                                          qp0 * cf[0][J], qp1 * cf[1][J]);
+                                }
+                            }
+                        }
+                    }
+                }
             }
+            fence_proxy_async_cta();
+            __syncthreads();
+            // g tile and the other v buffer are free: prefetch the next chunk's g and v
+            if (nc >= 0) issue_loads<DK>(P, sbase, rowoff_nxt, vnext, 0);
 
-            // prefetch the next chunk (raw q/k/g tiles are no longer needed)
-            if (nc >= 0) issue_chunk_loads<DK>(P, sm, rowoff_nxt, vnext);
-
-            // ---------------- MMA 1: dS and the four score column blocks
+            // ------------- MMA 1: dS (dS / d on the fast path) and the scores
             if (valid && tid == 0) {
                 tc_fence_after();
                 {
                     constexpr uint32_t id = idesc_f16_f32(DK, kDV, true, true);
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        const uint64_t a = desc_sw128(sbase + L::kst + kk * 2048, kTile, 1024);
-                        const uint64_t bd = desc_sw128(vaddr + kk * 2048, kTile, 1024);
-                        umma_f16(tmem + 0, a, bd, id, kk > 0 ? 1u : 0u);
-                    }
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_f16(tmem + 0, desc_sw128(sbase + L::k + kk * 2048, kTile, 1024),
+                                 desc_sw128(vaddr + kk * 2048, kTile, 1024), id, kk > 0 ? 1u : 0u);
                 }
-                {
-                    constexpr uint32_t id = idesc_f16_f32(64, 16, false, false);
+                if (!slow) {
+                    constexpr uint32_t id = idesc_f16_f32(64, 64, false, false);
 #pragma unroll
+                    for (int kk = 0; kk < DK / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * kTile + (kk & 3) * 32;
+                        umma_f16(tmem + 64, desc_sw128(sbase + L::q + off, 16, 1024),
+                                 desc_sw128(sbase + L::k + off, 16, 1024), id, kk > 0 ? 1u : 0u);
+                    }
+                } else {
+                    constexpr uint32_t id = idesc_f16_f32(64, 16, false, false);
                     for (int J = 0; J < 4; ++J) {
                         const int rows_j = 64 - 16 * J;
 #pragma unroll
@@ -439,111 +548,118 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_kernel(const Params P) {
                 }
                 mma_phase ^= 1u;
                 tc_fence_after();
-                if (warp < 4) {
-                    // scores -> masked fp16 P (row t = 16*warp + lane)
-                    uint32_t rr[64];
-                    const uint32_t ta = tmem + ((uint32_t)(32 * warp) << 16) + 64;
-                    tmem_ld16(ta + 0, *reinterpret_cast<uint32_t(*)[16]>(&rr[0]));
-                    tmem_ld16(ta + 16, *reinterpret_cast<uint32_t(*)[16]>(&rr[16]));
-                    tmem_ld16(ta + 32, *reinterpret_cast<uint32_t(*)[16]>(&rr[32]));
-                    tmem_ld16(ta + 48, *reinterpret_cast<uint32_t(*)[16]>(&rr[48]));
-                    tmem_ld_wait();
-                    if (lane < 16) {
-                        const int t = 16 * warp + lane;
-                        const int It = t >> 4;
-                        const bool fb = flags[It] != 0;
+                // scores -> masked fp16 P: this warp's 16 rows x 32 columns; dS -> fp32
+                // aggregate tile for the cluster scan (fast path: rows scaled by d)
+                uint32_t rs[16], rd[(DK == 64) ? 16 : 32];
+                tmem_ld_16x256b_x4(tmem + ((uint32_t)(32 * sp) << 16) + 64 + 32 * chalf, rs);
+                if (DK == 64) {
+                    tmem_ld_16x256b_x4(tmem + ((uint32_t)(32 * sp) << 16) + 32 * chalf,
+                                       *reinterpret_cast<uint32_t(*)[16]>(&rd[0]));
+                } else {
+                    const uint32_t ta = tmem + ((uint32_t)(32 * sp) << 16) + 32 * chalf;
+                    tmem_ld16(ta, *reinterpret_cast<uint32_t(*)[16]>(&rd[0]));
+                    tmem_ld16(ta + 16, *reinterpret_cast<uint32_t(*)[16]>(&rd[(DK == 64) ? 0 : 16]));
+                }
+                tmem_ld_wait();
+                {
+                    uint32_t *rr = rs;
+                    const bool fb = slow && (flags[sp] != 0);
 #pragma unroll
-                        for (int c8 = 0; c8 < 8; ++c8) {
-                            uint32_t pk[4];
+                    for (int cc = 0; cc < 4; ++cc) {
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                float x[2];
-#pragma unroll
-                                for (int z = 0; z < 2; ++z) {
-                                    const int s = c8 * 8 + e * 2 + z;
-                                    float val = __uint_as_float(rr[s]);
-                                    if (fb && (s >> 4) == It) val = diagx[(It * 16 + (t & 15)) * 16 + (s & 15)];
-                                    x[z] = s <= t ? val : 0.f;
-                                }
-                                pk[e] = pack_half2(x[0], x[1]);
+                        for (int hh = 0; hh < 2; ++hh) {
+                            const int row = rrow0 + 8 * hh;
+                            const int col = rcol0 + 8 * cc;
+                            float x0 = __uint_as_float(rr[4 * cc + 2 * hh]);
+                            float x1 = __uint_as_float(rr[4 * cc + 2 * hh + 1]);
+                            if (fb && (col >> 4) == sp) {
+                                x0 = diagx[(sp * 16 + (row & 15)) * 16 + (col & 15)];
+                                x1 = diagx[(sp * 16 + (row & 15)) * 16 + ((col + 1) & 15)];
                             }
-                            *reinterpret_cast<uint4 *>(sm + L::p + t * 128 + (((c8 ^ (t & 7)) & 7) << 4)) =
-                                make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                            x0 = col <= row ? x0 : 0.f;
+                            x1 = col + 1 <= row ? x1 : 0.f;
+                            st_h2(sm + L::p + sw_off(row, col), x0, x1);
+                        }
+                    }
+                }
+                if (DK == 64) {
+                    const uint32_t *rr = rd;
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int i = rrow0 + 8 * hh;
+                        const float sc = slow ? 1.f : dvec[i];
+#pragma unroll
+                        for (int cc = 0; cc < 4; ++cc) {
+                            const int col = rcol0 + 8 * cc;
+                            *reinterpret_cast<float2 *>(sm + L::agg + agg_off(i, col >> 2) +
+                                                        (col & 3) * 4) =
+                                make_float2(sc * __uint_as_float(rr[4 * cc + 2 * hh]),
+                                            sc * __uint_as_float(rr[4 * cc + 2 * hh + 1]));
                         }
                     }
                 } else {
-                    // dS -> fp32 aggregate tile for the cluster scan
-                    const int sub = warp - 4;
-                    uint32_t rr[64];
-                    const uint32_t ta = tmem + ((uint32_t)(32 * sub) << 16);
-                    tmem_ld16(ta + 0, *reinterpret_cast<uint32_t(*)[16]>(&rr[0]));
-                    tmem_ld16(ta + 16, *reinterpret_cast<uint32_t(*)[16]>(&rr[16]));
-                    tmem_ld16(ta + 32, *reinterpret_cast<uint32_t(*)[16]>(&rr[32]));
-                    tmem_ld16(ta + 48, *reinterpret_cast<uint32_t(*)[16]>(&rr[48]));
-                    tmem_ld_wait();
-                    const bool has_row = DK == 128 || lane < 16;
-                    if (has_row) {
-                        const int i = DK == 128 ? 32 * sub + lane : 16 * sub + lane;
+                    // M = 128: row i in lane i; this warp: rows 32*sp + lane, 32 columns
+                    const uint32_t *rr = rd;
+                    const int i = 32 * sp + lane;
+                    const float sc = slow ? 1.f : dvec[i];
 #pragma unroll
-                        for (int c4 = 0; c4 < 16; ++c4)
-                            *reinterpret_cast<float4 *>(sm + L::agg + agg_off(i, c4)) =
-                                make_float4(__uint_as_float(rr[4 * c4]), __uint_as_float(rr[4 * c4 + 1]),
-                                            __uint_as_float(rr[4 * c4 + 2]), __uint_as_float(rr[4 * c4 + 3]));
-                    }
+                    for (int c4 = 0; c4 < 8; ++c4)
+                        *reinterpret_cast<float4 *>(sm + L::agg + agg_off(i, 8 * chalf + c4)) =
+                            make_float4(sc * __uint_as_float(rr[4 * c4]), sc * __uint_as_float(rr[4 * c4 + 1]),
+                                        sc * __uint_as_float(rr[4 * c4 + 2]), sc * __uint_as_float(rr[4 * c4 + 3]));
                 }
             }
             fence_proxy_async_cta();
             tc_fence_before();
             cluster_sync();   // every chunk's (d, dS) of this round is visible cluster-wide
-            if (tid < 4) flags[tid] = 0;  // every reader of this round's flags has passed the barrier
+            if (tid < 4) { flags[tid] = 0; qmax[tid] = 0u; }
+            if (tid == 0) *kmax = 0u;
 
-            // ---------------- state pass, step A: stage peers' (d, dS) slices locally
-            float4 *stg = reinterpret_cast<float4 *>(sm + L::stage);
-            float *stgd = reinterpret_cast<float *>(sm + L::stage + (size_t)CP * nloc * 16);
-            for (int x = tid; x < nvalid * nloc; x += kThreads) {
-                const int j = x / nloc, el = x - j * nloc;
-                const int e = slo + el, i = e >> 4, c4 = e & 15;
-                stg[x] = ld_dsmem_f4(mapa(sbase + L::agg + agg_off(i, c4), (uint32_t)j));
-            }
-            {
-                const int ilo = slo >> 4, ihi = (shi + 15) >> 4;   // rows touched by the slice
-                const int nr = ihi - ilo;
-                for (int x = tid; x < nvalid * nr; x += kThreads) {
-                    const int j = x / nr, ii = x - j * nr;
-                    stgd[j * DK + ilo + ii] =
-                        ld_dsmem_f32(mapa(sbase + L::dvec + (ilo + ii) * 4, (uint32_t)j));
-                }
-            }
-            __syncthreads();
-            // ---------------- step B: chain the slice through the round's chunks
+            // ------------- state pass: chain this CTA's slice of the state through the
+            // round's chunks.  Peers' (d, dS) are fetched over DSMEM four chunks at a time
+            // so the round trips overlap; S_prev goes straight into each chunk's operand tile.
 #pragma unroll
             for (int m = 0; m < MAXM; ++m) {
                 const int el = tid + m * kThreads;
                 if (el < nloc) {
                     const int e = slo + el, i = e >> 4, c4 = e & 15;
+                    const uint32_t aoff = sbase + L::agg + agg_off(i, c4);
+                    const uint32_t doff = sbase + L::dvec + i * 4;
                     const uint32_t soff = sbase + L::sop + sw_off(i, 4 * c4);
-                    for (int j = 0; j < nvalid; ++j) {
-                        st_dsmem_v2(mapa(soff, (uint32_t)j), pack_half2(S[m].x, S[m].y),
-                                    pack_half2(S[m].z, S[m].w));
-                        const float4 a4 = stg[j * nloc + el];
-                        const float d = stgd[j * DK + i];
-                        S[m].x = fmaf(d, S[m].x, a4.x);
-                        S[m].y = fmaf(d, S[m].y, a4.y);
-                        S[m].z = fmaf(d, S[m].z, a4.z);
-                        S[m].w = fmaf(d, S[m].w, a4.w);
+                    for (int j0 = 0; j0 < nvalid; j0 += 4) {
+                        float4 a4[4];
+                        float dd[4];
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            if (j0 + q4 < nvalid) {
+                                a4[q4] = ld_dsmem_f4(mapa(aoff, (uint32_t)(j0 + q4)));
+                                dd[q4] = ld_dsmem_f32(mapa(doff, (uint32_t)(j0 + q4)));
+                            }
+                        }
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            if (j0 + q4 < nvalid) {
+                                st_dsmem_v2(mapa(soff, (uint32_t)(j0 + q4)), pack_half2(S[m].x, S[m].y),
+                                            pack_half2(S[m].z, S[m].w));
+                                S[m].x = fmaf(dd[q4], S[m].x, a4[q4].x);
+                                S[m].y = fmaf(dd[q4], S[m].y, a4[q4].y);
+                                S[m].z = fmaf(dd[q4], S[m].z, a4[q4].z);
+                                S[m].w = fmaf(dd[q4], S[m].w, a4[q4].w);
+                            }
+                        }
                     }
                 }
             }
             fence_proxy_async_cluster();
             cluster_sync();   // every S_prev tile of this round is written
 
-            // ---------------- MMA 2: O = Qint S_prev + tril(scores) V
+            // ------------- MMA 2: O = Qint S_prev + tril(scores) V
             if (valid && tid == 0) {
                 tc_fence_after();
                 constexpr uint32_t id = idesc_f16_f32(64, kDV, false, true);
 #pragma unroll
                 for (int kk = 0; kk < DK / 16; ++kk) {
-                    const uint32_t aa = sbase + L::qint + (kk >> 2) * kTile + (kk & 3) * 32;
+                    const uint32_t aa = sbase + L::q + (kk >> 2) * kTile + (kk & 3) * 32;
                     const uint32_t bb = sbase + L::sop + kk * 2048;
                     umma_f16(tmem + 128, desc_sw128(aa, 16, 1024), desc_sw128(bb, kTile, 1024), id,
                              kk > 0 ? 1u : 0u);
@@ -563,35 +679,37 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_kernel(const Params P) {
                 }
                 mma_phase ^= 1u;
                 tc_fence_after();
-                if (warp < 4) {
-                    uint32_t rr[64];
-                    const uint32_t ta = tmem + ((uint32_t)(32 * warp) << 16) + 128;
-                    tmem_ld16(ta + 0, *reinterpret_cast<uint32_t(*)[16]>(&rr[0]));
-                    tmem_ld16(ta + 16, *reinterpret_cast<uint32_t(*)[16]>(&rr[16]));
-                    tmem_ld16(ta + 32, *reinterpret_cast<uint32_t(*)[16]>(&rr[32]));
-                    tmem_ld16(ta + 48, *reinterpret_cast<uint32_t(*)[16]>(&rr[48]));
+                {
+                    // O -> fp16, staged (swizzled) in the P tile, then coalesced rows to global
+                    uint32_t rr[16];
+                    tmem_ld_16x256b_x4(tmem + ((uint32_t)(32 * sp) << 16) + 128 + 32 * chalf, rr);
                     tmem_ld_wait();
-                    if (lane < 16) {
-                        const int t = 16 * warp + lane;
-                        const int ro = rowoff_cur[t];
-                        if (ro >= 0) {
-                            uint4 *dst = reinterpret_cast<uint4 *>(P.out + (size_t)ro * kDV);
 #pragma unroll
-                            for (int c8 = 0; c8 < 8; ++c8)
-                                dst[c8] = make_uint4(
-                                    pack_half2(__uint_as_float(rr[8 * c8 + 0]), __uint_as_float(rr[8 * c8 + 1])),
-                                    pack_half2(__uint_as_float(rr[8 * c8 + 2]), __uint_as_float(rr[8 * c8 + 3])),
-                                    pack_half2(__uint_as_float(rr[8 * c8 + 4]), __uint_as_float(rr[8 * c8 + 5])),
-                                    pack_half2(__uint_as_float(rr[8 * c8 + 6]), __uint_as_float(rr[8 * c8 + 7])));
-                        }
-                    }
+                    for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh)
+                            st_h2(sm + L::p + sw_off(rrow0 + 8 * hh, rcol0 + 8 * cc),
+                                  __uint_as_float(rr[4 * cc + 2 * hh]),
+                                  __uint_as_float(rr[4 * cc + 2 * hh + 1]));
+                }
+            }
+            // q/k tiles (Qint, K operands) and the staging are consumed: prefetch next q, k
+            __syncthreads();
+            if (nc >= 0) issue_loads<DK>(P, sbase, rowoff_nxt, vnext, 1);
+            if (valid) {
+#pragma unroll
+                for (int x = tid; x < 64 * 8; x += kThreads) {
+                    const int row = x >> 3, c8 = x & 7;
+                    const int ro = rowoff_cur[row];
+                    if (ro >= 0)
+                        *reinterpret_cast<uint4 *>(P.out + (size_t)ro * kDV + 8 * c8) =
+                            *reinterpret_cast<const uint4 *>(sm + L::p + sw_off(row, 8 * c8));
                 }
             }
             tc_fence_before();
             cur ^= 1;
             vb ^= 1;
         }
-        // final state of this sequence
         if (P.sf != nullptr) {
 #pragma unroll
             for (int m = 0; m < MAXM; ++m) {
@@ -600,16 +718,11 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_kernel(const Params P) {
                     reinterpret_cast<float4 *>(P.sf + (size_t)seq * DK * kDV)[slo + el] = S[m];
             }
         }
-        (void)b;
-        (void)h;
     }
 
     cp_async_wait_all();
     __syncthreads();
-    if (timed_out) {
-        // let any MMA still in flight finish before giving TMEM back
-        mbar_wait_bounded(mbar, mma_phase ^ 1u, kWaitLimitNs);
-    }
+    if (timed_out) mbar_wait_bounded(mbar, mma_phase ^ 1u, kWaitLimitNs);
     cluster_sync();   // no CTA leaves while a peer may still touch its shared memory
     if (warp == 0) tmem_dealloc(tmem, kTmemCols);
 }
@@ -619,53 +732,133 @@ struct Plan {
     int cluster, clusters, smem;
 };
 
-static int g_num_sms = 0;
 static std::mutex g_mu;
+static int g_num_sms[64];
+// max co-resident clusters per (device, dk index, cluster size); 0 = not queried
+static int g_max_active[64][2][kMaxCluster + 1];
 
-static int num_sms() {
-    std::lock_guard<std::mutex> lk(g_mu);
-    if (g_num_sms == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        int n = 0;
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-            n = 148;
-        g_num_sms = n;
-    }
-    return g_num_sms;
+static int current_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+    return dev;
 }
 
-static Plan make_plan(long n_seq, long n_chunks, int dk, int sms) {
-    Plan p{};
-    p.smem = dk == 64 ? Smem<64>::alloc : Smem<128>::alloc;
-    long cp = n_seq > 0 ? sms / n_seq : 1;
-    if (n_chunks == 0 || cp < 1) cp = 1;
-    if (cp > kMaxCluster) cp = kMaxCluster;
-    if (n_chunks > 0 && cp > n_chunks) cp = n_chunks;
-    if (cp < 1) cp = 1;
-    // the scan staging (P slices of dS plus P rows of d) must fit its region
-    const int nf4 = dk * kDV / 4;
-    const int stage_bytes = dk == 64 ? Smem<64>::stage_bytes : Smem<128>::stage_bytes;
-    while (cp > 1 && (long)(nf4 + cp) * 16 + (long)cp * dk * 4 > stage_bytes) --cp;
-    p.cluster = (int)cp;
-    long ncl = sms / cp;
-    if (ncl > n_seq) ncl = n_seq;
-    if (ncl < 1) ncl = 1;
-    p.clusters = (int)ncl;
-    return p;
+static int num_sms(int dev) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_num_sms[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+            cudaGetLastError();
+            n = 148;
+        }
+        g_num_sms[dev] = n;
+    }
+    return g_num_sms[dev];
+}
+
+template <int DK>
+static cudaError_t prepare_kernel(int cluster) {
+    auto kern = gla_fwd_kernel<DK>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Smem<DK>::alloc);
+    if (e == cudaSuccess && cluster > 8)
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    return e;
+}
+
+template <int DK>
+static int max_active_clusters(int dev, int cluster, int sms) {
+    int &slot = g_max_active[dev][DK == 64 ? 0 : 1][cluster];
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (slot != 0) return slot;
+    }
+    int n = 0;
+    if (prepare_kernel<DK>(cluster) == cudaSuccess) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(cluster * (sms / cluster)), 1, 1);
+        cfg.blockDim = dim3(kThreads, 1, 1);
+        cfg.dynamicSmemBytes = (size_t)Smem<DK>::alloc;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)cluster;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaOccupancyMaxActiveClusters(&n, gla_fwd_kernel<DK>, &cfg) != cudaSuccess) n = 0;
+    }
+    cudaGetLastError();
+    if (n <= 0) n = -1;   // cluster size not schedulable
+    std::lock_guard<std::mutex> lk(g_mu);
+    slot = n;
+    return n;
+}
+
+// Picks the cluster size that minimises (waves of clusters) x (rounds per sequence),
+// preferring the smaller cluster on ties; the scan staging bounds it at 15.
+template <int DK>
+static Plan make_plan_dk(long n_seq, long n_chunks, int dev, bool query) {
+    Plan best{1, 1, Smem<DK>::alloc};
+    const int sms = num_sms(dev);
+    const int nf4 = DK * kDV / 4;
+    long best_cost = -1;
+    for (int cp = 1; cp <= kMaxCluster; ++cp) {
+        if (n_chunks > 0 && cp > n_chunks) break;
+        if (n_chunks == 0 && cp > 1) break;
+        int act = query ? max_active_clusters<DK>(dev, cp, sms) : sms / cp;
+        if (act <= 0) continue;
+        const long ncl = n_seq < act ? n_seq : act;
+        const long waves = (n_seq + ncl - 1) / ncl;
+        const long rounds = n_chunks > 0 ? (n_chunks + cp - 1) / cp : 0;
+        const long cost = waves * (rounds + 1);
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best.cluster = cp;
+            best.clusters = (int)(ncl < 1 ? 1 : ncl);
+        }
+    }
+    return best;
+}
+
+// GTR_CLUSTER_SIZE=<n> (tuning knob) forces the cluster size when n is feasible
+// for the shape; the number of clusters then follows the occupancy query.
+static int forced_cluster() {
+    const char *e = getenv("GTR_CLUSTER_SIZE");
+    if (!e || !*e) return 0;
+    const int n = atoi(e);
+    return (n >= 1 && n <= kMaxCluster) ? n : 0;
+}
+
+template <int DK>
+static Plan plan_forced(long n_seq, long n_chunks, int dev, int cp, bool query) {
+    Plan pl{1, 1, Smem<DK>::alloc};
+    const int nf4 = DK * kDV / 4;
+    if (n_chunks > 0 && cp > n_chunks) return make_plan_dk<DK>(n_seq, n_chunks, dev, query);
+    const int sms = num_sms(dev);
+    const int act = query ? max_active_clusters<DK>(dev, cp, sms) : sms / cp;
+    if (act <= 0) return make_plan_dk<DK>(n_seq, n_chunks, dev, query);
+    pl.cluster = cp;
+    pl.clusters = (int)(n_seq < act ? n_seq : act);
+    return pl;
+}
+
+static Plan make_plan(long n_seq, long n_chunks, int dk, bool query) {
+    const int dev = current_device();
+    const int fc = forced_cluster();
+    if (fc > 0)
+        return dk == 64 ? plan_forced<64>(n_seq, n_chunks, dev, fc, query)
+                        : plan_forced<128>(n_seq, n_chunks, dev, fc, query);
+    return dk == 64 ? make_plan_dk<64>(n_seq, n_chunks, dev, query)
+                    : make_plan_dk<128>(n_seq, n_chunks, dev, query);
 }
 
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 template <int DK>
 static cudaError_t launch(const Params &prm, const Plan &pl, cudaStream_t stream) {
-    auto kern = gla_fwd_kernel<DK>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem);
+    cudaError_t e = prepare_kernel<DK>(pl.cluster);
     if (e != cudaSuccess) return e;
-    if (pl.cluster > 8) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-        if (e != cudaSuccess) return e;
-    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(pl.cluster * pl.clusters), 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
@@ -678,7 +871,7 @@ static cudaError_t launch(const Params &prm, const Plan &pl, cudaStream_t stream
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, prm);
+    return cudaLaunchKernelEx(&cfg, gla_fwd_kernel<DK>, prm);
 }
 
 }  // namespace gtr
@@ -739,7 +932,7 @@ extern "C" gtr_status_t gtr_gla_fwd(const gtr_half_t *q, const gtr_half_t *k,
     prm.dir = direction;
     prm.n_seq = B * heads;
     prm.n_chunks = (prm.N + kChunk - 1) / kChunk;
-    const Plan pl = make_plan(prm.n_seq, prm.n_chunks, dk, num_sms());
+    const Plan pl = make_plan(prm.n_seq, prm.n_chunks, dk, true);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const cudaError_t e = dk == 64 ? launch<64>(prm, pl, s) : launch<128>(prm, pl, s);
     return e == cudaSuccess ? GTR_OK : GTR_ERR_CUDA;
@@ -777,7 +970,10 @@ extern "C" gtr_status_t gtr_gla_plan(int B, int heads, int Hgrid, int Wgrid, int
     if (B <= 0 || heads <= 0 || Hgrid < 0 || Wgrid < 0) return GTR_ERR_INVALID_ARG;
     if ((dk != 64 && dk != 128) || dv != kDV) return GTR_ERR_UNSUPPORTED;
     const long long N = (long long)Hgrid * Wgrid;
-    const Plan pl = make_plan((long)B * heads, (long)((N + kChunk - 1) / kChunk), dk, num_sms());
+    int ndev = 0;
+    const bool gpu = cudaGetDeviceCount(&ndev) == cudaSuccess && ndev > 0;
+    cudaGetLastError();
+    const Plan pl = make_plan((long)B * heads, (long)((N + kChunk - 1) / kChunk), dk, gpu);
     if (cluster_size) *cluster_size = pl.cluster;
     if (num_clusters) *num_clusters = pl.clusters;
     if (smem_bytes) *smem_bytes = pl.smem;
