@@ -103,6 +103,12 @@ const char *gtr_status_str(gtr_status_t status);
 gtr_status_t gtr_gla_plan(int B, int heads, int Hgrid, int Wgrid, int dk, int dv,
                           int *cluster_size, int *num_clusters, int *smem_bytes);
 
+/*
+ * Text of the last CUDA error a gtr_gla_fwd call on this host thread returned
+ * GTR_ERR_CUDA for ("no error" if none); static storage, never NULL.
+ */
+const char *gtr_gla_last_error(void);
+
 /* Library version, "major.minor.patch". */
 const char *gtr_gla_version(void);
 

@@ -35,6 +35,7 @@
 #include <cstdint>
 #include <cstdio>
 #include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include "../../include/gtr_gla.h"
@@ -727,15 +728,43 @@ __global__ void __launch_bounds__(kThreads, Smem<DK>::min_blocks) gla_fwd_kernel
     if (warp == 0) tmem_dealloc(tmem, kTmemCols);
 }
 
+}  // namespace gtr
+
+#include "gla_fwd_ws.cuh"
+
+namespace gtr {
+
 // ------------------------------------------------------------------ host
 struct Plan {
-    int cluster, clusters, smem;
+    int cluster, clusters, smem, threads;
+    const void *fn;
 };
+
+// A kernel variant: entry point, block size, dynamic shared memory, cache slot.
+struct KSpec {
+    const void *fn;
+    int threads;
+    int smem;
+    int slot;
+};
+
+// dk = 64 with at least two chunks per sequence runs the warp-specialised kernel
+// (clusters of >= 2 CTAs); everything else the basic one.  GTR_KERNEL=basic (tuning
+// knob) forces the basic kernel.
+static KSpec spec_for(int dk, long n_chunks) {
+    const char *e = getenv("GTR_KERNEL");
+    const bool basic = (e && !strcmp(e, "basic")) || n_chunks < ws::kMinCluster;
+    if (dk == 64 && !basic)
+        return KSpec{reinterpret_cast<const void *>(&ws::gla_fwd_ws_kernel), ws::kThreads, ws::L::alloc, 2};
+    if (dk == 64)
+        return KSpec{reinterpret_cast<const void *>(&gla_fwd_kernel<64>), kThreads, Smem<64>::alloc, 0};
+    return KSpec{reinterpret_cast<const void *>(&gla_fwd_kernel<128>), kThreads, Smem<128>::alloc, 1};
+}
 
 static std::mutex g_mu;
 static int g_num_sms[64];
-// max co-resident clusters per (device, dk index, cluster size); 0 = not queried
-static int g_max_active[64][2][kMaxCluster + 1];
+// max co-resident clusters per (device, kernel variant, cluster size); 0 = not queried
+static int g_max_active[64][3][kMaxCluster + 1];
 
 static int current_device() {
     int dev = 0;
@@ -756,37 +785,40 @@ static int num_sms(int dev) {
     return g_num_sms[dev];
 }
 
-template <int DK>
-static cudaError_t prepare_kernel(int cluster) {
-    auto kern = gla_fwd_kernel<DK>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         Smem<DK>::alloc);
+static cudaError_t prepare_kernel(const KSpec &k, int cluster) {
+    cudaError_t e = cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, k.smem);
     if (e == cudaSuccess && cluster > 8)
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        e = cudaFuncSetAttribute(k.fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     return e;
 }
 
-template <int DK>
-static int max_active_clusters(int dev, int cluster, int sms) {
-    int &slot = g_max_active[dev][DK == 64 ? 0 : 1][cluster];
+static void fill_config(cudaLaunchConfig_t &cfg, cudaLaunchAttribute *attr, const KSpec &k,
+                        int cluster, int clusters, cudaStream_t stream) {
+    cfg = cudaLaunchConfig_t{};
+    cfg.gridDim = dim3((unsigned)(cluster * clusters), 1, 1);
+    cfg.blockDim = dim3((unsigned)k.threads, 1, 1);
+    cfg.dynamicSmemBytes = (size_t)k.smem;
+    cfg.stream = stream;
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)cluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+}
+
+static int max_active_clusters(const KSpec &k, int dev, int cluster, int sms) {
+    int &slot = g_max_active[dev][k.slot][cluster];
     {
         std::lock_guard<std::mutex> lk(g_mu);
         if (slot != 0) return slot;
     }
     int n = 0;
-    if (prepare_kernel<DK>(cluster) == cudaSuccess) {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((unsigned)(cluster * (sms / cluster)), 1, 1);
-        cfg.blockDim = dim3(kThreads, 1, 1);
-        cfg.dynamicSmemBytes = (size_t)Smem<DK>::alloc;
+    if (prepare_kernel(k, cluster) == cudaSuccess) {
+        cudaLaunchConfig_t cfg;
         cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = (unsigned)cluster;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        if (cudaOccupancyMaxActiveClusters(&n, gla_fwd_kernel<DK>, &cfg) != cudaSuccess) n = 0;
+        fill_config(cfg, attr, k, cluster, sms / cluster, 0);
+        if (cudaOccupancyMaxActiveClusters(&n, k.fn, &cfg) != cudaSuccess) n = 0;
     }
     cudaGetLastError();
     if (n <= 0) n = -1;   // cluster size not schedulable
@@ -795,18 +827,29 @@ static int max_active_clusters(int dev, int cluster, int sms) {
     return n;
 }
 
-// Picks the cluster size that minimises (waves of clusters) x (rounds per sequence),
-// preferring the smaller cluster on ties; the scan staging bounds it at 15.
-template <int DK>
-static Plan make_plan_dk(long n_seq, long n_chunks, int dev, bool query) {
-    Plan best{1, 1, Smem<DK>::alloc};
+// GTR_CLUSTER_SIZE=<n> (tuning knob) forces the cluster size when it is feasible.
+static int forced_cluster() {
+    const char *e = getenv("GTR_CLUSTER_SIZE");
+    if (!e || !*e) return 0;
+    const int n = atoi(e);
+    return (n >= 1 && n <= kMaxCluster) ? n : 0;
+}
+
+// Picks the cluster size that minimises (waves of clusters) x (rounds per sequence + 1),
+// preferring the smaller cluster on ties.
+static Plan make_plan(long n_seq, long n_chunks, int dk, bool query) {
+    const KSpec k = spec_for(dk, n_chunks);
+    const int cp_min = k.slot == 2 ? ws::kMinCluster : 1;
+    const int dev = current_device();
     const int sms = num_sms(dev);
-    const int nf4 = DK * kDV / 4;
+    Plan best{cp_min, 1, k.smem, k.threads, k.fn};
+    const int fc = forced_cluster();
     long best_cost = -1;
-    for (int cp = 1; cp <= kMaxCluster; ++cp) {
+    for (int cp = cp_min; cp <= kMaxCluster; ++cp) {
         if (n_chunks > 0 && cp > n_chunks) break;
         if (n_chunks == 0 && cp > 1) break;
-        int act = query ? max_active_clusters<DK>(dev, cp, sms) : sms / cp;
+        if (fc > 0 && cp != fc) continue;
+        const int act = query ? max_active_clusters(k, dev, cp, sms) : sms / cp;
         if (act <= 0) continue;
         const long ncl = n_seq < act ? n_seq : act;
         const long waves = (n_seq + ncl - 1) / ncl;
@@ -818,60 +861,23 @@ static Plan make_plan_dk(long n_seq, long n_chunks, int dev, bool query) {
             best.clusters = (int)(ncl < 1 ? 1 : ncl);
         }
     }
+    if (best_cost < 0 && fc > 0) return make_plan(n_seq, n_chunks, dk, query);
     return best;
 }
 
-// GTR_CLUSTER_SIZE=<n> (tuning knob) forces the cluster size when n is feasible
-// for the shape; the number of clusters then follows the occupancy query.
-static int forced_cluster() {
-    const char *e = getenv("GTR_CLUSTER_SIZE");
-    if (!e || !*e) return 0;
-    const int n = atoi(e);
-    return (n >= 1 && n <= kMaxCluster) ? n : 0;
-}
-
-template <int DK>
-static Plan plan_forced(long n_seq, long n_chunks, int dev, int cp, bool query) {
-    Plan pl{1, 1, Smem<DK>::alloc};
-    const int nf4 = DK * kDV / 4;
-    if (n_chunks > 0 && cp > n_chunks) return make_plan_dk<DK>(n_seq, n_chunks, dev, query);
-    const int sms = num_sms(dev);
-    const int act = query ? max_active_clusters<DK>(dev, cp, sms) : sms / cp;
-    if (act <= 0) return make_plan_dk<DK>(n_seq, n_chunks, dev, query);
-    pl.cluster = cp;
-    pl.clusters = (int)(n_seq < act ? n_seq : act);
-    return pl;
-}
-
-static Plan make_plan(long n_seq, long n_chunks, int dk, bool query) {
-    const int dev = current_device();
-    const int fc = forced_cluster();
-    if (fc > 0)
-        return dk == 64 ? plan_forced<64>(n_seq, n_chunks, dev, fc, query)
-                        : plan_forced<128>(n_seq, n_chunks, dev, fc, query);
-    return dk == 64 ? make_plan_dk<64>(n_seq, n_chunks, dev, query)
-                    : make_plan_dk<128>(n_seq, n_chunks, dev, query);
-}
+static thread_local cudaError_t g_last_cuda_error = cudaSuccess;
 
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-template <int DK>
-static cudaError_t launch(const Params &prm, const Plan &pl, cudaStream_t stream) {
-    cudaError_t e = prepare_kernel<DK>(pl.cluster);
+static cudaError_t launch(const Params &prm, const Plan &pl, int dk, cudaStream_t stream) {
+    const KSpec k = spec_for(dk, prm.n_chunks);
+    cudaError_t e = prepare_kernel(k, pl.cluster);
     if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(pl.cluster * pl.clusters), 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = (size_t)pl.smem;
-    cfg.stream = stream;
+    cudaLaunchConfig_t cfg;
     cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)pl.cluster;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, gla_fwd_kernel<DK>, prm);
+    fill_config(cfg, attr, k, pl.cluster, pl.clusters, stream);
+    void *args[] = {const_cast<Params *>(&prm)};
+    return cudaLaunchKernelExC(&cfg, k.fn, args);
 }
 
 }  // namespace gtr
@@ -934,8 +940,13 @@ extern "C" gtr_status_t gtr_gla_fwd(const gtr_half_t *q, const gtr_half_t *k,
     prm.n_chunks = (prm.N + kChunk - 1) / kChunk;
     const Plan pl = make_plan(prm.n_seq, prm.n_chunks, dk, true);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const cudaError_t e = dk == 64 ? launch<64>(prm, pl, s) : launch<128>(prm, pl, s);
-    return e == cudaSuccess ? GTR_OK : GTR_ERR_CUDA;
+    const cudaError_t e = launch(prm, pl, dk, s);
+    if (e != cudaSuccess) {
+        g_last_cuda_error = e;
+        cudaGetLastError();   // clear the non-sticky launch error
+        return GTR_ERR_CUDA;
+    }
+    return GTR_OK;
 }
 
 extern "C" gtr_status_t gtr_gla_device_status(void *stream) {
@@ -980,4 +991,8 @@ extern "C" gtr_status_t gtr_gla_plan(int B, int heads, int Hgrid, int Wgrid, int
     return GTR_OK;
 }
 
-extern "C" const char *gtr_gla_version(void) { return "0.1.0"; }
+extern "C" const char *gtr_gla_version(void) { return "0.2.0"; }
+
+extern "C" const char *gtr_gla_last_error(void) {
+    return g_last_cuda_error == cudaSuccess ? "no error" : cudaGetErrorString(g_last_cuda_error);
+}

@@ -21,7 +21,7 @@ GTR_OK, GTR_ERR_INVALID_ARG, GTR_ERR_UNSUPPORTED, GTR_ERR_CUDA, GTR_ERR_TIMEOUT 
 L2R, R2L, T2B, B2T = 0, 1, 2, 3
 
 EXPORTED_SYMBOLS = ("gtr_gla_fwd", "gtr_gla_device_status", "gtr_status_str", "gtr_gla_plan",
-                    "gtr_gla_version")
+                    "gtr_gla_version", "gtr_gla_last_error")
 
 _lock = threading.Lock()
 _lib = None
@@ -29,7 +29,10 @@ _lib = None
 
 class GTRError(RuntimeError):
     def __init__(self, status: int, where: str):
-        super().__init__(f"{where}: {status_str(status)} (status {status})")
+        detail = ""
+        if status == GTR_ERR_CUDA and _lib is not None:
+            detail = f" [{_lib.gtr_gla_last_error().decode()}]"
+        super().__init__(f"{where}: {status_str(status)} (status {status}){detail}")
         self.status = status
 
 
@@ -54,6 +57,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         ip = ctypes.POINTER(ctypes.c_int)
         lib.gtr_gla_plan.argtypes = [i] * 6 + [ip, ip, ip]
         lib.gtr_gla_version.restype = ctypes.c_char_p
+        lib.gtr_gla_last_error.restype = ctypes.c_char_p
         _lib = lib
         return lib
 
