@@ -33,8 +33,16 @@
  *
  * Ownership: every buffer belongs to the caller; the library never frees or
  * keeps a pointer after a call returns.  All work is enqueued on `stream`
- * (a cudaStream_t, NULL = legacy default stream); no call synchronises the host
- * except gtr_gla_device_status.
+ * (a cudaStream_t, NULL = legacy default stream).  No call synchronises the host
+ * except gtr_gla_device_status and the first gtr_gla_fwd call on a device that
+ * needs a workspace (it allocates and zero-fills the library's cached one).
+ *
+ * Workspace: for some shapes (dk = 64 with few sequences) one sequence is split
+ * into spans that run on different SMs; they exchange one 16.6 KB aggregate per
+ * span through a device workspace.  gtr_gla_fwd uses a workspace cached by the
+ * library, one per device (about 5 MB), so gtr_gla_fwd calls on one device must
+ * not run concurrently on different streams: such callers use gtr_gla_fwd_ws
+ * with one workspace each.
  *
  * Errors: argument checks run on the host before anything is enqueued and
  * return GTR_ERR_INVALID_ARG / GTR_ERR_UNSUPPORTED with nothing launched.
@@ -86,8 +94,34 @@ gtr_status_t gtr_gla_fwd(const gtr_half_t *q, const gtr_half_t *k, const gtr_hal
                          void *stream);
 
 /*
+ * Bytes of workspace gtr_gla_fwd_ws needs for a shape on the current device
+ * (0: none needed, or arguments gtr_gla_fwd would reject).  Host-only query.
+ */
+size_t gtr_gla_workspace_bytes(int B, int heads, int Hgrid, int Wgrid, int dk, int dv, int chunk);
+
+/*
+ * gtr_gla_fwd with a caller-owned workspace: same arguments and results, plus
+ *   workspace        device memory, 256-byte aligned, at least
+ *                    gtr_gla_workspace_bytes(...) bytes (may be NULL when that is 0).
+ *                    It must be zero-filled before its first use; every call that
+ *                    completes without a device error leaves it zero-filled again.
+ *                    After GTR_ERR_TIMEOUT the caller zero-fills it again.
+ *   workspace_bytes  its size.
+ * Calls that share a workspace must not overlap in time (same stream is fine).
+ * A missing, short or misaligned workspace returns GTR_ERR_INVALID_ARG.
+ * (No counterpart on the pages: this is the library's memory contract.)
+ */
+gtr_status_t gtr_gla_fwd_ws(const gtr_half_t *q, const gtr_half_t *k, const gtr_half_t *v,
+                            const gtr_half_t *g, int B, int heads, int Hgrid, int Wgrid,
+                            int dk, int dv, int direction, int chunk,
+                            const float *init_state, gtr_half_t *out, float *final_state,
+                            void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Syncs `stream`, then reads and clears the device error word (and any sticky
- * CUDA error).  Returns GTR_OK, GTR_ERR_TIMEOUT or GTR_ERR_CUDA.
+ * CUDA error).  Returns GTR_OK, GTR_ERR_TIMEOUT or GTR_ERR_CUDA.  On
+ * GTR_ERR_TIMEOUT it also zero-fills the library's cached workspace of the
+ * current device.
  */
 gtr_status_t gtr_gla_device_status(void *stream);
 
@@ -96,8 +130,9 @@ const char *gtr_status_str(gtr_status_t status);
 
 /*
  * Launch plan the library would use for a shape on the current device:
- * writes the cluster size (CTAs cooperating on one sequence), the number of
- * clusters and the dynamic shared memory per CTA.  Host-only query; returns
+ * writes the number of CTAs cooperating on one sequence (spans, or the size of
+ * a thread-block cluster), the number of such CTA groups in the grid and the
+ * dynamic shared memory per CTA.  Host-only query; returns
  * GTR_ERR_* like gtr_gla_fwd's argument checks.
  */
 gtr_status_t gtr_gla_plan(int B, int heads, int Hgrid, int Wgrid, int dk, int dv,

@@ -1,0 +1,901 @@
+// gla_fwd_span.cuh -- span-parallel GTR token-mixer forward kernel for dk = dv = 64
+// (included by gtr_gla.cu, which holds the shared helpers and the C ABI).
+//
+// Decomposition.  Each (batch, head) sequence is cut into P contiguous spans of
+// chunks; one CTA owns one span (persistent CTAs loop over sequences).  Inside a
+// span the chunk-to-chunk state pass (GTR news article, section
+// "速度到底快在哪，TensorRT部署做了什么": only the chunk-boundary state is passed in order)
+// is purely local, so no per-chunk traffic crosses CTAs:
+//
+//   phase 1  stream the span's chunks from a zero state (span 0: from S0):
+//            loader warp 12 stages raw rows with cp.async; group A (warps 0-7) builds
+//            the gated operands, issues MMA 1 (scores, state delta) and, in its TMEM
+//            readout, writes S_prev (fp16 MMA operand) and updates the fp32 state
+//            S <- d * S + dS in shared memory; group B (warps 8-11) issues MMA 2
+//            (O = Qint S_prev + tril(scores) V) and stores the outputs.
+//   phase 2  publish the span's aggregate (state reached from zero, product of the
+//            decays) to the workspace; span 0 publishes its inclusive state.
+//   phase 3  look back: fold the aggregates of the earlier spans into S_in, the true
+//            state entering this span.
+//   phase 4  correct the outputs for the missing S_in term.  For a chunk c starting
+//            D_c (per key channel, product of the decays since the span start) into the
+//            span, the term is (Q * P) diag(D_c) S_in.  The first kHold chunks keep
+//            their fp32 outputs in TMEM and get the exact term added by one MMA each;
+//            later chunks get it by re-reading q, g and o, unless a bound shows the term
+//            is below 2^-22 of the chunk's largest output (the decays make it vanish
+//            after a few chunks for the gates on the pages' workloads).
+//   phase 5  the last span writes the final state  D_span * S_in + S_local.
+//
+// All spans of a sequence are co-resident (cooperative launch), so the look-back
+// waits always end; every wait is bounded anyway.
+#pragma once
+
+namespace gtr {
+namespace sp {
+
+constexpr int kThreadsA = 256;              // warps 0-7
+constexpr int kThreadsB = 128;              // warps 8-11
+constexpr int kThreads = kThreadsA + kThreadsB + 32;   // + loader warp 12
+constexpr int kDK = 64;
+constexpr int kHold = 5;                    // chunks per span whose outputs wait in TMEM
+constexpr int kMaxSpan = 64;                // chunks of a later span with recorded decays
+constexpr uint32_t kBarA = 1, kBarB = 2;
+constexpr int kAggFloats = kDK * kDV + kDK; // state + decay product
+constexpr uint32_t kColMma1 = 0, kColWork = 128, kColHold = 192;
+constexpr int kSpanTmemCols = 512;
+
+// ------------------------------------------------------------------ smem map
+struct L {
+    static constexpr int stg = 0;                   // raw rows q,k,g,v (or q,-,g,o) [64][128 B] x 4
+    static constexpr int qint = stg + 4 * kTile;    // working Qint, x2
+    static constexpr int kt = qint + 2 * kTile;     // K / P (or K * sigma * after)
+    static constexpr int vop = kt + kTile;          // V swizzled, x2
+    static constexpr int p = vop + 2 * kTile;       // masked scores, x2
+    static constexpr int qj = p + 2 * kTile;        // packed Q^(J) (sub-block path)
+    static constexpr int qj_bytes = (64 + 48 + 32 + 16) * 128;
+    static constexpr int kbar = qj + qj_bytes;      // K * sigma (sub-block path)
+    static constexpr int sop = kbar + kTile;        // S_prev fp16, x2
+    static constexpr int sst = sop + 2 * kTile;     // running state fp32 [64][64] swizzled
+    static constexpr int ost = sst + 64 * 256;      // output staging
+    static constexpr int ring = ost + kTile;        // Qint of the held chunks
+    static constexpr int dcum = ring + kHold * kTile;   // D_c per chunk of the span [kMaxSpan][64]
+    static constexpr int dloc = dcum + kMaxSpan * 256;  // d of the current chunk [64]
+    static constexpr int dacc = dloc + 256;         // running product of decays [64]
+    static constexpr int htot = dacc + 256;         // half-block totals [8][64]
+    static constexpr int diag = htot + 8 * 64 * 4;  // exact diagonal blocks [4][16][16]
+    static constexpr int rowb = diag + 4 * 16 * 16 * 4; // token rows [3 teams][64]
+    static constexpr int cmeta = rowb + 3 * 64 * 4; // per chunk: max|q|, max|o| [kMaxSpan][2]
+    static constexpr int skipf = cmeta + kMaxSpan * 8;  // per chunk: correction negligible
+    static constexpr int rmax = skipf + kMaxSpan * 4;   // row maxima of |S_in| [64]
+    static constexpr int misc = rmax + 256;         // per parity: flags[4] qmax[4] kmax
+    static constexpr int bars = misc + 128;
+    static constexpr int bytes = bars + 24 * 8;
+    static constexpr int alloc = bytes + 1024;
+    // after phase 1 the score tiles hold S_in (fp32 [64][64], swizzled)
+    static constexpr int sin = p;
+
+    static __host__ __device__ constexpr int qj_region(int J) {
+        return 128 * (J == 0 ? 0 : J == 1 ? 64 : J == 2 ? 112 : 144);
+    }
+};
+static_assert(L::alloc <= 227 * 1024, "shared memory budget");
+
+enum {
+    B_STGF = 0,   // raw rows landed (32 loader arrivals)
+    B_STGE = 1,   // group A done with the staging buffer
+    B_MMA1 = 2,
+    B_MMA2 = 3,
+    B_OPSF = 4,   // [2] operands of a chunk ready for MMA 2
+    B_OPSE = 6,   // [2] MMA 2 done with them
+    B_FIX = 8,    // correction MMAs complete
+    B_TMEM = 10   // (uint32_t) TMEM base
+};
+
+// Workspace protocol.  hdr[0] counts completed launches (the generation), hdr[1]
+// counts CTAs that finished the current launch.  A span publishes its aggregate
+// by storing tag = generation + 1 into its flag; readers wait for exactly that
+// tag, so flags never need clearing and stale tags of earlier launches are
+// never mistaken for fresh ones.  The last CTA of a launch advances the
+// generation.  The header and flags sit at fixed offsets whatever the shape.
+struct Work {
+    int P;        // spans per sequence
+    int Lc;       // chunks per span (the last span may be shorter)
+    float *ws;    // [n_seq][P][kAggFloats] aggregates
+    unsigned long long *flags;   // [n_seq][P] publish tags
+    unsigned long long *hdr;     // [2]: generation, finished CTAs
+};
+
+__device__ __forceinline__ uint64_t *bar(uint8_t *sm, int i) {
+    return reinterpret_cast<uint64_t *>(sm + L::bars) + i;
+}
+// Bounded wait; after the first timeout a thread stops waiting (its results are
+// garbage then, but the kernel still ends and the error word reports it).
+__device__ __forceinline__ void wait_l(uint64_t *b, uint32_t parity, bool &to) {
+    if (to) return;
+    if (!mbar_wait_bounded(b, parity, kWaitLimitNs)) {
+        to = true;
+        set_error(kErrTimeout);
+    }
+}
+
+// Loader: 16-byte cp.async of chunk c's rows of up to four tensors into staging.
+// Null tensors are skipped; rows past the grid are zero-filled.
+__device__ __forceinline__ void load_rows4(const Params &P, uint8_t *sm, int seq, int c, int lane,
+                                           const __half *t0, const __half *t1, const __half *t2,
+                                           const __half *t3) {
+    const uint32_t st = smem_u32(sm + L::stg);
+    const int b = seq / P.heads, h = seq - b * P.heads;
+    const int p0 = c * kChunk;
+    const __half *tens[4] = {t0, t1, t2, t3};
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        const int t = lane + 32 * half;
+        const bool ok = p0 + t < P.N;
+        size_t ro = 0;
+        if (ok) ro = (size_t)((b * P.N + scan_to_token(p0 + t, P.H, P.W, P.dir)) * P.heads + h);
+        const uint32_t nb = ok ? 16u : 0u;
+#pragma unroll
+        for (int ten = 0; ten < 4; ++ten) {
+            if (tens[ten] == nullptr) continue;
+            const __half *src = tens[ten] + ro * 64;
+#pragma unroll
+            for (int pc = 0; pc < 8; ++pc)
+                cp_async16(st + ten * kTile + t * 128 + 16 * pc, src + 8 * pc, nb);
+        }
+    }
+}
+
+__device__ __forceinline__ unsigned long long ld_acquire_gpu(const unsigned long long *p) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_gpu(unsigned long long *p, unsigned long long v) {
+    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+// Epilogue of one 64x64 fp32 accumulator at TMEM column `col` by a team of four
+// consecutive warps (warp w reads TMEM lanes 32 (w % 4) ..; tb = thread in the team,
+// named barrier `bar_id`): adds `addend` rows from an unswizzled fp16 staging tile if
+// non-null, converts to fp16 through the staging tile `os`, stores at the token rows
+// in `rowb`; returns this thread's max |value|.
+__device__ __forceinline__ float store_chunk_out(const Params &P, uint32_t tmem, uint32_t col,
+                                                 int bw, int lane, int tb, const uint8_t *addend,
+                                                 uint32_t bar_id, uint8_t *os, const int *rowb) {
+    uint32_t r0[16], r1[16];
+    const uint32_t ta = tmem + ((uint32_t)(32 * bw) << 16) + col;
+    tmem_ld_16x256b_x4(ta, r0);
+    tmem_ld_16x256b_x4(ta + 32, r1);
+    tmem_ld_wait();
+    const int row0 = 16 * bw + (lane >> 2);
+    const int col0 = 2 * (lane & 3);
+    float mx = 0.f;
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const int row = row0 + 8 * hh;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const int col = col0 + 8 * cc + 32 * half;
+                const uint32_t *rr = half ? r1 : r0;
+                float x0 = __uint_as_float(rr[4 * cc + 2 * hh]);
+                float x1 = __uint_as_float(rr[4 * cc + 2 * hh + 1]);
+                if (addend) {
+                    const float2 a = ld_h2(addend + row * 128 + 2 * col);
+                    x0 += a.x;
+                    x1 += a.y;
+                }
+                mx = fmaxf(mx, fmaxf(fabsf(x0), fabsf(x1)));
+                st_h2(os + sw_off(row, col), x0, x1);
+            }
+        }
+    tc_fence_before();
+    named_sync(bar_id, 128);
+#pragma unroll
+    for (int x = tb; x < 64 * 8; x += 128) {
+        const int row = x >> 3, c8 = x & 7;
+        const int ro = rowb[row];
+        if (ro >= 0)
+            *reinterpret_cast<uint4 *>(P.out + (size_t)ro * kDV + 8 * c8) =
+                *reinterpret_cast<const uint4 *>(os + sw_off(row, 8 * c8));
+    }
+    named_sync(bar_id, 128);
+    return mx;
+}
+
+__device__ __forceinline__ void fill_rows(const Params &P, int seq, int c, int *rowb, int tb) {
+    if (tb < 64) {
+        const int p = c * kChunk + tb;
+        int ro = -1;
+        if (p < P.N) {
+            const int bb = seq / P.heads, hh = seq - bb * P.heads;
+            ro = (bb * P.N + scan_to_token(p, P.H, P.W, P.dir)) * P.heads + hh;
+        }
+        rowb[tb] = ro;
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 1) gla_fwd_span_kernel(const Params P, const Work Wk) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(sm);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int PS = Wk.P;
+    const int kspan = (int)blockIdx.x % PS;
+    const int grp = (int)blockIdx.x / PS, ngrp = (int)gridDim.x / PS;
+
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar(sm, B_TMEM));
+    float *dcum = reinterpret_cast<float *>(sm + L::dcum);
+    float *dloc = reinterpret_cast<float *>(sm + L::dloc);
+    float *dacc = reinterpret_cast<float *>(sm + L::dacc);
+    float *cmeta = reinterpret_cast<float *>(sm + L::cmeta);
+    int *rowb = reinterpret_cast<int *>(sm + L::rowb);
+
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, kSpanTmemCols);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        mbar_init(bar(sm, B_STGF), 32);
+        mbar_init(bar(sm, B_STGE), 1);
+        mbar_init(bar(sm, B_MMA1), 1);
+        mbar_init(bar(sm, B_MMA2), 1);
+        mbar_init(bar(sm, B_OPSF), 1);
+        mbar_init(bar(sm, B_OPSF + 1), 1);
+        mbar_init(bar(sm, B_OPSE), 1);
+        mbar_init(bar(sm, B_OPSE + 1), 1);
+        mbar_init(bar(sm, B_FIX), 1);
+        fence_mbar_init();
+    }
+    if (tid < 24) reinterpret_cast<unsigned *>(sm + L::misc)[tid] = 0u;
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    bool to = false;
+    // publish tag of this launch (the generation only changes after every CTA of
+    // the previous launch has finished)
+    const unsigned long long tag = PS > 1 ? __ldcg(Wk.hdr) + 1ull : 0ull;
+    // running barrier phase counters (kept identical in every role that waits on them)
+    uint32_t n_stg = 0, n_mma1 = 0, n_mma2 = 0;
+    uint32_t n_ops[2] = {0u, 0u}, n_fix = 0u;
+
+    for (int seq = grp; seq < P.n_seq; seq += ngrp) {
+        const int c0 = kspan * Wk.Lc;
+        const int nch = min(Wk.Lc, P.n_chunks - c0);   // >= 1 (host guarantees)
+        const int hold = kspan > 0 ? min(kHold, nch) : 0;
+        const bool later = kspan > 0;
+
+        // ---------------- phase 1 prologue: running state and decay product
+        {
+            float *sst = reinterpret_cast<float *>(sm + L::sst);
+            for (int e = tid; e < kDK * kDV / 4; e += kThreads) {
+                const int i = e >> 4, c4 = e & 15;
+                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (!later && P.s0 != nullptr)
+                    v = reinterpret_cast<const float4 *>(P.s0 + (size_t)seq * kDK * kDV)[e];
+                *reinterpret_cast<float4 *>(reinterpret_cast<uint8_t *>(sst) + agg_off(i, c4)) = v;
+            }
+            if (tid < 64) dacc[tid] = 1.f;
+            if (tid < kMaxSpan * 2) cmeta[tid] = 0.f;
+        }
+        __syncthreads();
+
+        if (warp < 8) {
+            // ================================================= group A
+            const int gI = warp >> 1, ghf = warp & 1, gt0 = 16 * gI + 8 * ghf, gh = 2 * gI + ghf;
+            const int sp = warp & 3, chalf = warp >> 2;
+            const int rrow0 = 16 * sp + (lane >> 2);
+            const int rcol0 = 32 * chalf + 2 * (lane & 3);
+            float *htot = reinterpret_cast<float *>(sm + L::htot);
+            float *diagx = reinterpret_cast<float *>(sm + L::diag);
+            const uint8_t *st = sm + L::stg;
+            for (int ci = 0; ci < nch; ++ci) {
+                const int b = ci & 1;
+                int *flags = reinterpret_cast<int *>(sm + L::misc + 48 * b);
+                unsigned *qmax = reinterpret_cast<unsigned *>(sm + L::misc + 48 * b + 16);
+                unsigned *kmax = reinterpret_cast<unsigned *>(sm + L::misc + 48 * b + 32);
+                const int nrows = min(kChunk, P.N - (c0 + ci) * kChunk);
+                const bool held = ci < hold;
+                uint8_t *qo = sm + L::qint + b * kTile;
+                // a held chunk also keeps Qint * D_c (D_c = decay since the span start)
+                uint8_t *qr = sm + L::ring + (held ? ci : 0) * kTile;
+                const float2 dc = *reinterpret_cast<const float2 *>(dacc + 2 * lane);
+                const bool pub = PS > 1 && kspan < PS - 1 && ci == nch - 1;
+                wait_l(bar(sm, B_STGF), n_stg & 1u, to);
+                ++n_stg;
+                wait_l(bar(sm, B_OPSE + b), (n_ops[b] & 1u) ^ 1u, to);
+                // ---------- pass 1
+                float pl[8][2], sl[8][2];
+                __half2 qh[8], kh[8];
+                __half2 qm2 = __float2half2_rn(0.f), km2 = __float2half2_rn(0.f);
+                {
+                    float a0[8], a1[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const uint32_t o = (gt0 + u) * 128 + 4 * lane;
+                        const float2 gv = ld_h2(st + 2 * kTile + o);
+                        qh[u] = *reinterpret_cast<const __half2 *>(st + o);
+                        kh[u] = *reinterpret_cast<const __half2 *>(st + kTile + o);
+                        a0[u] = exp_f(gv.x);
+                        a1[u] = exp_f(gv.y);
+                        qm2 = __hmax2(qm2, __habs2(qh[u]));
+                        km2 = __hmax2(km2, __habs2(kh[u]));
+                    }
+                    float r0 = 1.f, r1 = 1.f;
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        r0 *= a0[u]; r1 *= a1[u];
+                        pl[u][0] = r0; pl[u][1] = r1;
+                    }
+                    r0 = 1.f; r1 = 1.f;
+#pragma unroll
+                    for (int u = 7; u >= 0; --u) {
+                        sl[u][0] = r0; sl[u][1] = r1;
+                        r0 *= a0[u]; r1 *= a1[u];
+                    }
+                    *reinterpret_cast<float2 *>(htot + gh * 64 + 2 * lane) = make_float2(pl[7][0], pl[7][1]);
+                }
+                {
+                    const float qm = fmaxf(__low2float(qm2), __high2float(qm2));
+                    const float km = fmaxf(__low2float(km2), __high2float(km2));
+                    const unsigned wq = __reduce_max_sync(0xffffffffu, __float_as_uint(qm));
+                    const unsigned wk = __reduce_max_sync(0xffffffffu, __float_as_uint(km));
+                    if (lane == 0) {
+                        atomicMax(&qmax[gI], wq);
+                        atomicMax(kmax, wk);
+                    }
+                }
+                {
+                    uint8_t *vo = sm + L::vop + b * kTile;
+#pragma unroll
+                    for (int x = tid; x < 64 * 8; x += kThreadsA) {
+                        const int t = x >> 3, c8 = x & 7;
+                        *reinterpret_cast<uint4 *>(vo + sw_off(t, 8 * c8)) =
+                            *reinterpret_cast<const uint4 *>(st + 3 * kTile + t * 128 + 16 * c8);
+                    }
+                }
+                named_sync(kBarA, kThreadsA);
+                // ---------- chunk factors
+                float dch[2], bef[2], aft[2];
+                bool bad = __uint_as_float(*kmax) > kFastMaxK;
+                {
+                    float2 ht[8];
+#pragma unroll
+                    for (int h8 = 0; h8 < 8; ++h8)
+                        ht[h8] = *reinterpret_cast<const float2 *>(htot + h8 * 64 + 2 * lane);
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        float d = 1.f, bf = 1.f, af = 1.f;
+#pragma unroll
+                        for (int h8 = 0; h8 < 8; ++h8) {
+                            const float x = e ? ht[h8].y : ht[h8].x;
+                            d *= x;
+                            if (h8 < gh) bf *= x;
+                            if (h8 > gh) af *= x;
+                        }
+                        dch[e] = d; bef[e] = bf; aft[e] = af;
+                        bad |= !(d >= kFastMinDecay);
+                    }
+                }
+                const bool slow = named_sync_or(kBarA, kThreadsA, bad);
+                if (gh == 0) *reinterpret_cast<float2 *>(dloc + 2 * lane) = make_float2(dch[0], dch[1]);
+                if (!slow) {
+                    const float i0 = aft[0] / dch[0], i1 = aft[1] / dch[1];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const uint32_t o = sw_off(gt0 + u, 2 * lane);
+                        const float2 qv = __half22float2(qh[u]);
+                        const float2 kv = __half22float2(kh[u]);
+                        const float a0 = qv.x * (pl[u][0] * bef[0]), a1 = qv.y * (pl[u][1] * bef[1]);
+                        st_h2(qo + o, a0, a1);
+                        if (held) st_h2(qr + o, a0 * dc.x, a1 * dc.y);
+                        st_h2(sm + L::kt + o, kv.x * (sl[u][0] * i0), kv.y * (sl[u][1] * i1));
+                    }
+                } else {
+                    float T[4][2];
+#pragma unroll
+                    for (int L4 = 0; L4 < 4; ++L4) {
+                        const float2 h0 = *reinterpret_cast<const float2 *>(htot + (2 * L4) * 64 + 2 * lane);
+                        const float2 h1 = *reinterpret_cast<const float2 *>(htot + (2 * L4 + 1) * 64 + 2 * lane);
+                        T[L4][0] = h0.x * h1.x;
+                        T[L4][1] = h0.y * h1.y;
+                    }
+                    bool dbad = false;
+#pragma unroll
+                    for (int L4 = 0; L4 < 4; ++L4)
+                        if (L4 == gI) dbad |= !(T[L4][0] >= kDiagMinTotal) || !(T[L4][1] >= kDiagMinTotal);
+                    dbad |= __uint_as_float(qmax[gI]) > kDiagMaxQ;
+                    if (__any_sync(0xffffffffu, dbad) && lane == 0) atomicOr(&flags[gI], 1);
+                    named_sync(kBarA, kThreadsA);
+                    const int anyflag = flags[0] | flags[1] | flags[2] | flags[3];
+                    if (anyflag) {
+                        for (int pr = tid; pr < 4 * 256; pr += kThreadsA) {
+                            const int I = pr >> 8, u = (pr >> 4) & 15, w = pr & 15;
+                            if (!flags[I] || w > u) continue;
+                            const int tu = I * kSub + u, tw = I * kSub + w;
+                            float acc = 0.f;
+                            if (tu < nrows) {
+                                for (int i = 0; i < kDK; ++i) {
+                                    float lg = 0.f;
+                                    for (int r2 = tw + 1; r2 <= tu; ++r2)
+                                        lg += __half2float(*reinterpret_cast<const __half *>(st + 2 * kTile + r2 * 128 + 2 * i));
+                                    const float qv = __half2float(*reinterpret_cast<const __half *>(st + tu * 128 + 2 * i));
+                                    const float kv = __half2float(*reinterpret_cast<const __half *>(st + kTile + tw * 128 + 2 * i));
+                                    acc += qv * kv * exp_f(lg);
+                                }
+                            }
+                            diagx[(I * 16 + u) * 16 + w] = acc;
+                        }
+                        named_sync(kBarA, kThreadsA);
+                    }
+                    const bool diag_bad = flags[gI] != 0;
+                    float cf[2][4], bI[2], aI[2], hin[2], hout[2];
+                    const float2 h0 = *reinterpret_cast<const float2 *>(htot + (2 * gI) * 64 + 2 * lane);
+                    const float2 h1 = *reinterpret_cast<const float2 *>(htot + (2 * gI + 1) * 64 + 2 * lane);
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        float b0 = 1.f, a0 = 1.f, tI = 1.f;
+#pragma unroll
+                        for (int L4 = 0; L4 < 4; ++L4) {
+                            if (L4 < gI) b0 *= T[L4][e];
+                            if (L4 > gI) a0 *= T[L4][e];
+                            if (L4 == gI) tI = T[L4][e];
+                        }
+                        bI[e] = b0; aI[e] = a0;
+#pragma unroll
+                        for (int J = 0; J < 4; ++J) {
+                            float cj = 1.f;
+#pragma unroll
+                            for (int L4 = 0; L4 < 4; ++L4)
+                                if (L4 > J && L4 < gI) cj *= T[L4][e];
+                            cf[e][J] = (J == gI) ? (diag_bad ? 0.f : 1.f / tI) : cj;
+                        }
+                        hin[e] = ghf ? (e ? h0.y : h0.x) : 1.f;
+                        hout[e] = ghf ? 1.f : (e ? h1.y : h1.x);
+                    }
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const int t = gt0 + u;
+                        const uint32_t o = sw_off(t, 2 * lane);
+                        const float2 qv = __half22float2(qh[u]);
+                        const float2 kv = __half22float2(kh[u]);
+                        const float qp0 = qv.x * (pl[u][0] * hin[0]);
+                        const float qp1 = qv.y * (pl[u][1] * hin[1]);
+                        const float ks0 = kv.x * (sl[u][0] * hout[0]);
+                        const float ks1 = kv.y * (sl[u][1] * hout[1]);
+                        st_h2(qo + o, qp0 * bI[0], qp1 * bI[1]);
+                        if (held) st_h2(qr + o, qp0 * bI[0] * dc.x, qp1 * bI[1] * dc.y);
+                        st_h2(sm + L::kbar + o, ks0, ks1);
+                        st_h2(sm + L::kt + o, ks0 * aI[0], ks1 * aI[1]);
+#pragma unroll
+                        for (int J = 0; J < 4; ++J)
+                            if (J <= gI)
+                                st_h2(sm + L::qj + L::qj_region(J) + sw_off(t - 16 * J, 2 * lane),
+                                      qp0 * cf[0][J], qp1 * cf[1][J]);
+                    }
+                }
+                fence_proxy_async_cta();
+                named_sync(kBarA, kThreadsA);
+                if (tid == 0) mbar_arrive(bar(sm, B_STGE));   // the loader may refill staging
+                // ---------- MMA 1
+                if (tid == 0) {
+                    tc_fence_after();
+                    const uint32_t kta = sbase + L::kt;
+                    const uint32_t va = sbase + L::vop + b * kTile;
+                    constexpr uint32_t id_ds = idesc_f16_f32(64, kDV, true, true);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_f16(tmem + kColMma1, desc_sw128(kta + kk * 2048, kTile, 1024),
+                                 desc_sw128(va + kk * 2048, kTile, 1024), id_ds, kk > 0 ? 1u : 0u);
+                    if (!slow) {
+                        constexpr uint32_t id = idesc_f16_f32(64, 64, false, false);
+                        const uint32_t qa = smem_u32(qo);
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            umma_f16(tmem + kColMma1 + 64, desc_sw128(qa + kk * 32, 16, 1024),
+                                     desc_sw128(kta + kk * 32, 16, 1024), id, kk > 0 ? 1u : 0u);
+                    } else {
+                        constexpr uint32_t id = idesc_f16_f32(64, 16, false, false);
+                        for (int J = 0; J < 4; ++J) {
+#pragma unroll
+                            for (int kk = 0; kk < 4; ++kk) {
+                                const uint32_t aa = sbase + L::qj + L::qj_region(J) - 16 * J * 128 + kk * 32;
+                                const uint32_t bb = sbase + L::kbar + 16 * J * 128 + kk * 32;
+                                umma_f16(tmem + kColMma1 + 64 + 16 * J, desc_sw128(aa, 16, 1024),
+                                         desc_sw128(bb, 16, 1024), id, kk > 0 ? 1u : 0u);
+                            }
+                        }
+                    }
+                    umma_commit(bar(sm, B_MMA1));
+                }
+                wait_l(bar(sm, B_MMA1), n_mma1 & 1u, to);
+                ++n_mma1;
+                tc_fence_after();
+                uint32_t rs[16], rd[16];
+                tmem_ld_16x256b_x4(tmem + ((uint32_t)(32 * sp) << 16) + kColMma1 + 64 + 32 * chalf, rs);
+                tmem_ld_16x256b_x4(tmem + ((uint32_t)(32 * sp) << 16) + kColMma1 + 32 * chalf, rd);
+                tmem_ld_wait();
+                {
+                    // masked scores -> P
+                    uint8_t *pt = sm + L::p + b * kTile;
+                    const bool fb = slow && (flags[sp] != 0);
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc) {
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            const int row = rrow0 + 8 * hh;
+                            const int col = rcol0 + 8 * cc;
+                            float x0 = __uint_as_float(rs[4 * cc + 2 * hh]);
+                            float x1 = __uint_as_float(rs[4 * cc + 2 * hh + 1]);
+                            if (fb && (col >> 4) == sp) {
+                                x0 = diagx[(sp * 16 + (row & 15)) * 16 + (col & 15)];
+                                x1 = diagx[(sp * 16 + (row & 15)) * 16 + ((col + 1) & 15)];
+                            }
+                            x0 = col <= row ? x0 : 0.f;
+                            x1 = col + 1 <= row ? x1 : 0.f;
+                            st_h2(pt + sw_off(row, col), x0, x1);
+                        }
+                    }
+                }
+                {
+                    // state: S_prev (fp16 operand) <- S; S <- d * S + dS
+                    uint8_t *sst = sm + L::sst;
+                    uint8_t *so = sm + L::sop + b * kTile;
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int i = rrow0 + 8 * hh;
+                        const float di = dloc[i];
+                        const float scl = slow ? 1.f : di;
+#pragma unroll
+                        for (int cc = 0; cc < 4; ++cc) {
+                            const int col = rcol0 + 8 * cc;
+                            float2 *sp2 = reinterpret_cast<float2 *>(sst + agg_off(i, col >> 2) + (col & 3) * 4);
+                            const float2 s = *sp2;
+                            st_h2(so + sw_off(i, col), s.x, s.y);
+                            const float2 sn = make_float2(fmaf(di, s.x, scl * __uint_as_float(rd[4 * cc + 2 * hh])),
+                                                          fmaf(di, s.y, scl * __uint_as_float(rd[4 * cc + 2 * hh + 1])));
+                            *sp2 = sn;
+                            // the span's last chunk publishes its state straight from here
+                            if (pub)
+                                *reinterpret_cast<float2 *>(Wk.ws + ((size_t)seq * PS + kspan) * kAggFloats +
+                                                            i * kDV + col) = sn;
+                        }
+                    }
+                }
+                tc_fence_before();
+                fence_proxy_async_cta();
+                named_sync(kBarA, kThreadsA);
+                if (tid < 64) {
+                    if (ci < kMaxSpan) dcum[ci * 64 + tid] = dacc[tid];
+                    dacc[tid] *= dloc[tid];
+                }
+                if (tid == 64) {
+                    const unsigned m = max(max(qmax[0], qmax[1]), max(qmax[2], qmax[3]));
+                    if (ci < kMaxSpan) cmeta[2 * ci] = __uint_as_float(m);
+                }
+                if (pub) {
+                    // aggregate = (state reached from zero, product of the span's decays)
+                    if (tid < 64) Wk.ws[((size_t)seq * PS + kspan) * kAggFloats + kDK * kDV + tid] = dacc[tid];
+                    __threadfence();
+                    named_sync(kBarA, kThreadsA);
+                    if (tid == 0) st_release_gpu(Wk.flags + (size_t)seq * PS + kspan, tag);
+                }
+                if (tid == 0) mbar_arrive(bar(sm, B_OPSF + b));
+                named_sync(kBarA, kThreadsA);
+                if (tid < 4) { flags[tid] = 0; qmax[tid] = 0u; }
+                if (tid == 0) *kmax = 0u;
+                ++n_ops[b];
+            }
+        } else if (warp < 12) {
+            // ================================================= group B
+            const int tb = tid - kThreadsA, bw = warp - 8;
+            int *rows2 = rowb + 2 * 64;
+            for (int ci = 0; ci < nch; ++ci) {
+                const int b = ci & 1;
+                const bool held = ci < hold;
+                fill_rows(P, seq, c0 + ci, rows2, tb);
+                wait_l(bar(sm, B_OPSF + b), n_ops[b] & 1u, to);
+                const uint32_t dcol = held ? kColHold + 64 * ci : kColWork;
+                if (tb == 0) {
+                    tc_fence_after();
+                    constexpr uint32_t id = idesc_f16_f32(64, kDV, false, true);
+                    const uint32_t qa = sbase + L::qint + b * kTile;
+                    const uint32_t sa = sbase + L::sop + b * kTile;
+                    const uint32_t pa = sbase + L::p + b * kTile;
+                    const uint32_t va = sbase + L::vop + b * kTile;
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_f16(tmem + dcol, desc_sw128(qa + kk * 32, 16, 1024),
+                                 desc_sw128(sa + kk * 2048, kTile, 1024), id, kk > 0 ? 1u : 0u);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_f16(tmem + dcol, desc_sw128(pa + kk * 32, 16, 1024),
+                                 desc_sw128(va + kk * 2048, kTile, 1024), id, 1u);
+                    umma_commit(bar(sm, B_MMA2));
+                }
+                wait_l(bar(sm, B_MMA2), n_mma2 & 1u, to);
+                ++n_mma2;
+                tc_fence_after();
+                if (tb == 0) mbar_arrive(bar(sm, B_OPSE + b));
+                ++n_ops[b];
+                named_sync(kBarB, kThreadsB);   // row table visible to every group-B thread
+                if (!held) {
+                    const float mx = store_chunk_out(P, tmem, kColWork, bw, lane, tb, nullptr, kBarB,
+                                                     sm + L::ost, rows2);
+                    if (later && ci < kMaxSpan) {
+                        const unsigned w = __reduce_max_sync(0xffffffffu, __float_as_uint(mx));
+                        if (lane == 0) atomicMax(reinterpret_cast<unsigned *>(cmeta + 2 * ci + 1), w);
+                    }
+                }
+            }
+        } else {
+            // ================================================= loader (warp 12)
+            for (int ci = 0; ci < nch; ++ci) {
+                wait_l(bar(sm, B_STGE), (n_stg & 1u) ^ 1u, to);
+                load_rows4(P, sm, seq, c0 + ci, lane, P.q, P.k, P.g, P.v);
+                cp_async_mbar_arrive_noinc(bar(sm, B_STGF));
+                ++n_stg;
+            }
+            cp_async_wait_all();
+        }
+        __syncthreads();
+        // Each role advanced only the barrier counters it waits on (A: staging, MMA 1,
+        // operands; B: operands, MMA 2; loader: staging); bring the others level.
+        if (warp >= 8) n_mma1 += (uint32_t)nch;
+        if (warp < 8 || warp >= 12) n_mma2 += (uint32_t)nch;
+        if (warp >= 8 && warp < 12) n_stg += (uint32_t)nch;
+        if (warp >= 12) {
+            n_ops[0] += (uint32_t)((nch + 1) / 2);
+            n_ops[1] += (uint32_t)(nch / 2);
+        }
+
+        // ---------------- phase 3: look back over the earlier spans
+        if (later) {
+            if (tid < kspan) {
+                const unsigned long long *f = Wk.flags + (size_t)seq * PS + tid;
+                if (ld_acquire_gpu(f) != tag) {
+                    const uint64_t t0 = globaltimer_ns();
+                    while (ld_acquire_gpu(f) != tag) {
+                        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                            to = true;
+                            set_error(kErrTimeout);
+                            break;
+                        }
+                    }
+                }
+            }
+            __syncthreads();
+            // S_in = S_out(span 0), then S_in = D_j * S_in + S_j for j = 1 .. kspan-1
+            float *sin = reinterpret_cast<float *>(sm + L::sin);
+            unsigned *rmax = reinterpret_cast<unsigned *>(sm + L::rmax);
+            if (tid < 64) rmax[tid] = 0u;
+            __syncthreads();
+            const float *wseq = Wk.ws + (size_t)seq * PS * kAggFloats;
+            for (int e = tid; e < kDK * kDV / 4; e += kThreads) {
+                const int i = e >> 4, c4 = e & 15;
+                float4 s = __ldcg(reinterpret_cast<const float4 *>(wseq) + e);
+                // the later aggregates, four loads in flight at a time
+                for (int j0 = 1; j0 < kspan; j0 += 4) {
+                    float4 a[4];
+                    float dj[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        if (j0 + u < kspan) {
+                            const float *wj = wseq + (size_t)(j0 + u) * kAggFloats;
+                            a[u] = __ldcg(reinterpret_cast<const float4 *>(wj) + e);
+                            dj[u] = __ldcg(wj + kDK * kDV + i);
+                        }
+                    }
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        if (j0 + u < kspan) {
+                            s.x = fmaf(dj[u], s.x, a[u].x);
+                            s.y = fmaf(dj[u], s.y, a[u].y);
+                            s.z = fmaf(dj[u], s.z, a[u].z);
+                            s.w = fmaf(dj[u], s.w, a[u].w);
+                        }
+                    }
+                }
+                *reinterpret_cast<float4 *>(reinterpret_cast<uint8_t *>(sin) + agg_off(i, c4)) = s;
+                const float m = fmaxf(fmaxf(fabsf(s.x), fabsf(s.y)), fmaxf(fabsf(s.z), fabsf(s.w)));
+                atomicMax(rmax + i, __float_as_uint(m));   // non-negative: integer order = float order
+            }
+            __syncthreads();   // S_in and its row maxima complete
+            // Chunks past the held ones: is the term negligible?  One warp per chunk:
+            //   |term[t][j]| <= max|q| * sum_i D_c[i] * max_j |S_in[i][j]|   (P_t <= 1),
+            // negligible when below 2^-16 of the chunk's largest output, i.e. under a
+            // 32nd of the fp16 rounding step of that output.  (Later spans have at most
+            // kMaxSpan chunks.)
+            {
+                const float *rmf = reinterpret_cast<const float *>(rmax);
+                int *skipf = reinterpret_cast<int *>(sm + L::skipf);
+                for (int ci = hold + warp; ci < nch; ci += kThreads / 32) {
+                    float part = fmaf(dcum[ci * 64 + 2 * lane], rmf[2 * lane],
+                                      dcum[ci * 64 + 2 * lane + 1] * rmf[2 * lane + 1]);
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+                    if (lane == 0) skipf[ci] = cmeta[2 * ci] * part <= 1.52587890625e-5f * cmeta[2 * ci + 1];
+                }
+            }
+            __syncthreads();
+        }
+
+        // ---------------- phase 4: add the S_in term to this span's outputs
+        if (later) {
+            const float *sin = reinterpret_cast<const float *>(sm + L::sin);
+            // held chunks: their ring tiles hold Qint * D_c, so one B tile (S_in, fp16)
+            // serves them all; the MMAs accumulate onto the chunks' outputs in TMEM
+            if (hold > 0) {
+                uint8_t *bt = sm + L::sop;
+                for (int e = tid; e < kDK * kDV / 4; e += kThreads) {
+                    const int i = e >> 4, c4 = e & 15;
+                    const float4 s = *reinterpret_cast<const float4 *>(reinterpret_cast<const uint8_t *>(sin) + agg_off(i, c4));
+                    *reinterpret_cast<uint2 *>(bt + sw_off(i, 4 * c4)) =
+                        make_uint2(pack_half2(s.x, s.y), pack_half2(s.z, s.w));
+                }
+                fence_proxy_async_cta();
+                __syncthreads();
+                if (tid == 0) {
+                    tc_fence_after();
+                    constexpr uint32_t id = idesc_f16_f32(64, kDV, false, true);
+                    const uint32_t ba = smem_u32(bt);
+                    for (int ci = 0; ci < hold; ++ci) {
+                        const uint32_t qa = sbase + L::ring + ci * kTile;
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            umma_f16(tmem + kColHold + 64 * ci, desc_sw128(qa + kk * 32, 16, 1024),
+                                     desc_sw128(ba + kk * 2048, kTile, 1024), id, 1u);
+                    }
+                    umma_commit(bar(sm, B_FIX));
+                }
+                wait_l(bar(sm, B_FIX), n_fix & 1u, to);
+                ++n_fix;
+                tc_fence_after();
+                // epilogues: three teams of four warps, held chunk ci on team ci % 3
+                if (warp < 12) {
+                    const int team = warp >> 2, tb = tid - 128 * team, bw = warp & 3;
+                    int *rows = rowb + 64 * team;
+                    uint8_t *os = team < 2 ? sm + L::stg + team * kTile : sm + L::ost;
+                    for (int ci = team; ci < hold; ci += 3) {
+                        fill_rows(P, seq, c0 + ci, rows, tb);
+                        named_sync(3 + team, 128);
+                        store_chunk_out(P, tmem, kColHold + 64 * ci, bw, lane, tb, nullptr, 3 + team, os,
+                                        rows);
+                    }
+                }
+                __syncthreads();
+            }
+            // later chunks: exact re-read correction unless the term is provably negligible
+            // (spans after the first have at most kMaxSpan chunks)
+            const int *skipf = reinterpret_cast<const int *>(sm + L::skipf);
+            for (int ci = hold; ci < nch; ++ci) {
+                if (skipf[ci]) continue;
+                // load q, g, o rows of this chunk (all threads), rebuild Q * P * D_c
+                {
+                    const uint32_t stq = smem_u32(sm + L::stg);
+                    const int bq = seq / P.heads, hq = seq - bq * P.heads;
+                    const int p0 = (c0 + ci) * kChunk;
+                    for (int x = tid; x < 3 * 64 * 8; x += kThreads) {
+                        const int ten = x / 512, rem = x - ten * 512, t = rem >> 3, pc = rem & 7;
+                        const bool ok = p0 + t < P.N;
+                        size_t ro = 0;
+                        if (ok) ro = (size_t)((bq * P.N + scan_to_token(p0 + t, P.H, P.W, P.dir)) * P.heads + hq);
+                        const __half *src = ten == 0 ? P.q + ro * 64 : (ten == 1 ? P.g + ro * 64 : P.out + ro * 64);
+                        const int slot = ten == 0 ? 0 : (ten == 1 ? 2 : 3);
+                        cp_async16(stq + slot * kTile + t * 128 + 16 * pc, src + 8 * pc, ok ? 16u : 0u);
+                    }
+                    cp_async_commit();
+                    cp_async_wait_all();
+                }
+                __syncthreads();
+                {
+                    // 256 threads: (half-block, channel pair) as in gating; products from the
+                    // chunk start
+                    float *htot = reinterpret_cast<float *>(sm + L::htot);
+                    const int gI = warp >> 1, ghf = warp & 1, gt0 = 16 * gI + 8 * ghf, gh = 2 * gI + ghf;
+                    float pl[8][2];
+                    if (warp < 8) {
+                        float r0 = 1.f, r1 = 1.f;
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            const float2 gv = ld_h2(sm + L::stg + 2 * kTile + (gt0 + u) * 128 + 4 * lane);
+                            r0 *= exp_f(gv.x);
+                            r1 *= exp_f(gv.y);
+                            pl[u][0] = r0; pl[u][1] = r1;
+                        }
+                        *reinterpret_cast<float2 *>(htot + gh * 64 + 2 * lane) = make_float2(r0, r1);
+                    }
+                    __syncthreads();
+                    if (warp < 8) {
+                        float bf0 = 1.f, bf1 = 1.f;
+                        for (int h8 = 0; h8 < gh; ++h8) {
+                            const float2 x = *reinterpret_cast<const float2 *>(htot + h8 * 64 + 2 * lane);
+                            bf0 *= x.x;
+                            bf1 *= x.y;
+                        }
+                        const float D0 = dcum[ci * 64 + 2 * lane] * bf0, D1 = dcum[ci * 64 + 2 * lane + 1] * bf1;
+                        uint8_t *qo = sm + L::qint;
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            const float2 qv = ld_h2(sm + L::stg + (gt0 + u) * 128 + 4 * lane);
+                            st_h2(qo + sw_off(gt0 + u, 2 * lane), qv.x * pl[u][0] * D0, qv.y * pl[u][1] * D1);
+                        }
+                    }
+                    // S_in as the fp16 operand
+                    uint8_t *bt = sm + L::sop;
+                    for (int e = tid; e < kDK * kDV / 4; e += kThreads) {
+                        const int i = e >> 4, c4 = e & 15;
+                        const float4 s = *reinterpret_cast<const float4 *>(reinterpret_cast<const uint8_t *>(sin) + agg_off(i, c4));
+                        *reinterpret_cast<uint2 *>(bt + sw_off(i, 4 * c4)) =
+                            make_uint2(pack_half2(s.x, s.y), pack_half2(s.z, s.w));
+                    }
+                }
+                fence_proxy_async_cta();
+                __syncthreads();
+                if (tid == 0) {
+                    tc_fence_after();
+                    constexpr uint32_t id = idesc_f16_f32(64, kDV, false, true);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_f16(tmem + kColWork, desc_sw128(sbase + L::qint + kk * 32, 16, 1024),
+                                 desc_sw128(sbase + L::sop + kk * 2048, kTile, 1024), id, kk > 0 ? 1u : 0u);
+                    umma_commit(bar(sm, B_FIX));
+                }
+                wait_l(bar(sm, B_FIX), n_fix & 1u, to);
+                ++n_fix;
+                tc_fence_after();
+                if (warp >= 8 && warp < 12) {
+                    const int tb = tid - kThreadsA, bw = warp - 8;
+                    fill_rows(P, seq, c0 + ci, rowb + 128, tb);
+                    named_sync(kBarB, kThreadsB);
+                    store_chunk_out(P, tmem, kColWork, bw, lane, tb, sm + L::stg + 3 * kTile, kBarB,
+                                    sm + L::ost, rowb + 128);
+                }
+                __syncthreads();
+            }
+        }
+
+        // ---------------- phase 5: final state of the sequence
+        if (kspan == PS - 1 && P.sf != nullptr) {
+            const float *sst = reinterpret_cast<const float *>(sm + L::sst);
+            const float *sin = reinterpret_cast<const float *>(sm + L::sin);
+            for (int e = tid; e < kDK * kDV / 4; e += kThreads) {
+                const int i = e >> 4, c4 = e & 15;
+                float4 s = *reinterpret_cast<const float4 *>(reinterpret_cast<const uint8_t *>(sst) + agg_off(i, c4));
+                if (later) {
+                    const float di = dacc[i];
+                    const float4 a = *reinterpret_cast<const float4 *>(reinterpret_cast<const uint8_t *>(sin) + agg_off(i, c4));
+                    s.x = fmaf(di, a.x, s.x);
+                    s.y = fmaf(di, a.y, s.y);
+                    s.z = fmaf(di, a.z, s.z);
+                    s.w = fmaf(di, a.w, s.w);
+                }
+                reinterpret_cast<float4 *>(P.sf + (size_t)seq * kDK * kDV)[e] = s;
+            }
+        }
+        __syncthreads();   // staging / state tiles are reused by the next sequence
+    }
+
+    // the last CTA to finish advances the workspace generation
+    if (PS > 1 && tid == 0) {
+        __threadfence();
+        if (atomicAdd(Wk.hdr + 1, 1ull) == (unsigned long long)(gridDim.x - 1)) {
+            Wk.hdr[1] = 0ull;
+            Wk.hdr[0] = tag;
+            __threadfence();
+        }
+    }
+    // after a timeout some MMA may still be in flight: give it time before freeing TMEM
+    if (__syncthreads_or(to)) {
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 1000000ull) {
+        }
+    }
+    if (warp == 0) tmem_dealloc(tmem, kSpanTmemCols);
+}
+
+}  // namespace sp
+}  // namespace gtr

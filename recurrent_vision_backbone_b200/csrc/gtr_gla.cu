@@ -731,14 +731,12 @@ __global__ void __launch_bounds__(kThreads, Smem<DK>::min_blocks) gla_fwd_kernel
 }  // namespace gtr
 
 #include "gla_fwd_ws.cuh"
+#include "gla_fwd_span.cuh"
 
 namespace gtr {
 
 // ------------------------------------------------------------------ host
-struct Plan {
-    int cluster, clusters, smem, threads;
-    const void *fn;
-};
+enum KernelKind { kBasic64 = 0, kBasic128 = 1, kCluster = 2, kSpan = 3, kKinds = 4 };
 
 // A kernel variant: entry point, block size, dynamic shared memory, cache slot.
 struct KSpec {
@@ -748,23 +746,45 @@ struct KSpec {
     int slot;
 };
 
-// dk = 64 with at least two chunks per sequence runs the warp-specialised kernel
-// (clusters of >= 2 CTAs); everything else the basic one.  GTR_KERNEL=basic (tuning
-// knob) forces the basic kernel.
-static KSpec spec_for(int dk, long n_chunks) {
+struct Plan {
+    int kind;
+    int cluster;       // CTAs working on one sequence (cluster size or spans)
+    int clusters;      // groups of such CTAs in the grid
+    int span_len;      // chunks per span (span kernel)
+    int smem, threads;
+    size_t ws_bytes;   // workspace the launch needs (span kernel with >= 2 spans)
+};
+
+// dk = 64 runs the span kernel; dk = 128 the basic one.  GTR_KERNEL=basic|cluster
+// (tuning knob) selects one of the other dk = 64 kernels instead.
+static KSpec spec_of(int kind) {
+    switch (kind) {
+    case kBasic64:
+        return KSpec{reinterpret_cast<const void *>(&gla_fwd_kernel<64>), kThreads, Smem<64>::alloc, kBasic64};
+    case kBasic128:
+        return KSpec{reinterpret_cast<const void *>(&gla_fwd_kernel<128>), kThreads, Smem<128>::alloc, kBasic128};
+    case kCluster:
+        return KSpec{reinterpret_cast<const void *>(&ws::gla_fwd_ws_kernel), ws::kThreads, ws::L::alloc, kCluster};
+    default:
+        return KSpec{reinterpret_cast<const void *>(&sp::gla_fwd_span_kernel), sp::kThreads, sp::L::alloc, kSpan};
+    }
+}
+
+static int kind_for(int dk, long n_chunks) {
+    if (dk != 64) return kBasic128;
+    if (n_chunks == 0) return kBasic64;   // only copies init_state to final_state
     const char *e = getenv("GTR_KERNEL");
-    const bool basic = (e && !strcmp(e, "basic")) || n_chunks < ws::kMinCluster;
-    if (dk == 64 && !basic)
-        return KSpec{reinterpret_cast<const void *>(&ws::gla_fwd_ws_kernel), ws::kThreads, ws::L::alloc, 2};
-    if (dk == 64)
-        return KSpec{reinterpret_cast<const void *>(&gla_fwd_kernel<64>), kThreads, Smem<64>::alloc, 0};
-    return KSpec{reinterpret_cast<const void *>(&gla_fwd_kernel<128>), kThreads, Smem<128>::alloc, 1};
+    if (e && !strcmp(e, "basic")) return kBasic64;
+    if (e && !strcmp(e, "cluster") && n_chunks >= ws::kMinCluster) return kCluster;
+    return kSpan;
 }
 
 static std::mutex g_mu;
 static int g_num_sms[64];
 // max co-resident clusters per (device, kernel variant, cluster size); 0 = not queried
-static int g_max_active[64][3][kMaxCluster + 1];
+static int g_max_active[64][kKinds][kMaxCluster + 1];
+// co-resident CTAs of the span kernel per device; 0 = not queried
+static int g_span_capacity[64];
 
 static int current_device() {
     int dev = 0;
@@ -799,11 +819,17 @@ static void fill_config(cudaLaunchConfig_t &cfg, cudaLaunchAttribute *attr, cons
     cfg.blockDim = dim3((unsigned)k.threads, 1, 1);
     cfg.dynamicSmemBytes = (size_t)k.smem;
     cfg.stream = stream;
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)cluster;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
+    if (k.slot == kSpan) {
+        // all spans of a sequence must be resident together: cooperative launch
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+    } else {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)cluster;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+    }
     cfg.numAttrs = 1;
 }
 
@@ -827,7 +853,25 @@ static int max_active_clusters(const KSpec &k, int dev, int cluster, int sms) {
     return n;
 }
 
-// GTR_CLUSTER_SIZE=<n> (tuning knob) forces the cluster size when it is feasible.
+static int span_capacity(int dev, int sms, bool query) {
+    if (!query) return sms;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (g_span_capacity[dev] != 0) return g_span_capacity[dev];
+    }
+    const KSpec k = spec_of(kSpan);
+    int per_sm = 0;
+    if (prepare_kernel(k, 1) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k.fn, k.threads, (size_t)k.smem) != cudaSuccess)
+        per_sm = 0;
+    cudaGetLastError();
+    const int cap = per_sm > 0 ? per_sm * sms : -1;
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_span_capacity[dev] = cap;
+    return cap;
+}
+
+// GTR_CLUSTER_SIZE=<n> (tuning knob) forces the cluster size / span count when feasible.
 static int forced_cluster() {
     const char *e = getenv("GTR_CLUSTER_SIZE");
     if (!e || !*e) return 0;
@@ -835,47 +879,161 @@ static int forced_cluster() {
     return (n >= 1 && n <= kMaxCluster) ? n : 0;
 }
 
-// Picks the cluster size that minimises (waves of clusters) x (rounds per sequence + 1),
-// preferring the smaller cluster on ties.
-static Plan make_plan(long n_seq, long n_chunks, int dk, bool query) {
-    const KSpec k = spec_for(dk, n_chunks);
-    const int cp_min = k.slot == 2 ? ws::kMinCluster : 1;
-    const int dev = current_device();
-    const int sms = num_sms(dev);
-    Plan best{cp_min, 1, k.smem, k.threads, k.fn};
-    const int fc = forced_cluster();
+static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Workspace of the span kernel: a 256-byte header (launch generation, finished
+// CTAs), the publish flags of up to 2 * capacity (sequence, span) pairs, then the
+// aggregates.  Header and flags sit at the same offsets for every shape on a device.
+static size_t span_flags_bytes(int cap) { return align256((size_t)2 * cap * sizeof(unsigned long long)); }
+static size_t span_ws_bytes(long n_seq, int spans, int cap) {
+    if (spans < 2) return 0;
+    return 256 + span_flags_bytes(cap) + align256((size_t)n_seq * spans * sp::kAggFloats * sizeof(float));
+}
+
+// Span plan: P spans of Lc chunks per sequence (Lc <= 64 when P > 1), grid of whole
+// span groups within the co-resident capacity.  Minimises (sequence passes) x
+// (chunks per span + 2), the 2 standing for the look-back and the corrections;
+// several spans per sequence only while the sequences alone leave SMs idle.
+static Plan span_plan(long n_seq, long n_chunks, int cap) {
+    const KSpec k = spec_of(kSpan);
+    Plan best{kSpan, 1, 1, (int)n_chunks, k.smem, k.threads, 0};
     long best_cost = -1;
-    for (int cp = cp_min; cp <= kMaxCluster; ++cp) {
-        if (n_chunks > 0 && cp > n_chunks) break;
-        if (n_chunks == 0 && cp > 1) break;
-        if (fc > 0 && cp != fc) continue;
-        const int act = query ? max_active_clusters(k, dev, cp, sms) : sms / cp;
-        if (act <= 0) continue;
-        const long ncl = n_seq < act ? n_seq : act;
-        const long waves = (n_seq + ncl - 1) / ncl;
-        const long rounds = n_chunks > 0 ? (n_chunks + cp - 1) / cp : 0;
-        const long cost = waves * (rounds + 1);
+    const int fc = forced_cluster();
+    for (int P = 1; P <= kMaxCluster && P <= n_chunks && P <= cap; ++P) {
+        const long Lc = (n_chunks + P - 1) / P;
+        if ((n_chunks + Lc - 1) / Lc != P) continue;   // same split as a smaller P
+        if (P > 1 && (Lc > sp::kMaxSpan || n_seq * P > 2L * cap)) continue;
+        if (fc > 0 && P != fc) continue;
+        const long groups = n_seq < cap / P ? n_seq : cap / P;
+        const long passes = (n_seq + groups - 1) / groups;
+        const long cost = passes * (Lc + (P > 1 ? 2 : 0));
         if (best_cost < 0 || cost < best_cost) {
             best_cost = cost;
-            best.cluster = cp;
-            best.clusters = (int)(ncl < 1 ? 1 : ncl);
+            best.cluster = P;
+            best.clusters = (int)groups;
+            best.span_len = (int)Lc;
         }
     }
-    if (best_cost < 0 && fc > 0) return make_plan(n_seq, n_chunks, dk, query);
+    if (best_cost < 0 && fc > 0) {   // forced span count not feasible: plan freely
+        Plan p1{kSpan, 1, (int)(n_seq < cap ? n_seq : cap), (int)n_chunks, k.smem, k.threads, 0};
+        return p1;
+    }
+    best.ws_bytes = span_ws_bytes(n_seq, best.cluster, cap);
     return best;
+}
+
+// Cluster plan: the cluster size that minimises (waves of clusters) x (rounds per
+// sequence + 1), preferring the smaller cluster on ties.
+static Plan cluster_plan(int kind, long n_seq, long n_chunks, int dev, int sms, bool query) {
+    const KSpec k = spec_of(kind);
+    const int cp_min = kind == kCluster ? ws::kMinCluster : 1;
+    Plan best{kind, cp_min, 1, 0, k.smem, k.threads, 0};
+    const int fc = forced_cluster();
+    long best_cost = -1;
+    for (int pass = 0; pass < 2 && best_cost < 0; ++pass) {
+        for (int cp = cp_min; cp <= kMaxCluster; ++cp) {
+            if (n_chunks > 0 && cp > n_chunks) break;
+            if (n_chunks == 0 && cp > 1) break;
+            if (pass == 0 && fc > 0 && cp != fc) continue;
+            const int act = query ? max_active_clusters(k, dev, cp, sms) : sms / cp;
+            if (act <= 0) continue;
+            const long ncl = n_seq < act ? n_seq : act;
+            const long waves = (n_seq + ncl - 1) / ncl;
+            const long rounds = n_chunks > 0 ? (n_chunks + cp - 1) / cp : 0;
+            const long cost = waves * (rounds + 1);
+            if (best_cost < 0 || cost < best_cost) {
+                best_cost = cost;
+                best.cluster = cp;
+                best.clusters = (int)(ncl < 1 ? 1 : ncl);
+            }
+        }
+    }
+    return best;
+}
+
+static Plan make_plan(long n_seq, long n_chunks, int dk, bool query) {
+    const int kind = kind_for(dk, n_chunks);
+    const int dev = current_device();
+    const int sms = num_sms(dev);
+    if (kind == kSpan) {
+        const int cap = span_capacity(dev, sms, query);
+        if (cap > 0) return span_plan(n_seq, n_chunks, cap);
+        return cluster_plan(kBasic64, n_seq, n_chunks, dev, sms, query);
+    }
+    return cluster_plan(kind, n_seq, n_chunks, dev, sms, query);
+}
+
+// Library-cached workspace of gtr_gla_fwd, one per device: sized for the largest
+// span plan (n_seq * spans <= 2 * capacity), allocated and zero-filled by the first
+// call that needs it.
+struct DefaultWs {
+    void *ptr;
+    size_t bytes;
+};
+static DefaultWs g_default_ws[64];
+
+static size_t default_ws_bytes(int cap) {
+    if (cap <= 0) return 0;
+    return 256 + span_flags_bytes(cap) + align256((size_t)2 * cap * sp::kAggFloats * sizeof(float));
+}
+
+static cudaError_t default_workspace(int dev, size_t need, cudaStream_t stream, void **ptr) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    DefaultWs &w = g_default_ws[dev];
+    if (w.ptr != nullptr && w.bytes >= need) {
+        *ptr = w.ptr;
+        return cudaSuccess;
+    }
+    if (w.ptr != nullptr) return cudaErrorInvalidValue;   // the plan bound guarantees this never happens
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    cudaError_t e = cudaStreamIsCapturing(stream, &cs);
+    if (e != cudaSuccess) return e;
+    if (cs != cudaStreamCaptureStatusNone) return cudaErrorStreamCaptureUnsupported;
+    const int sms = g_num_sms[dev] > 0 ? g_num_sms[dev] : 148;
+    const int cap = g_span_capacity[dev] > 0 ? g_span_capacity[dev] : sms;
+    size_t bytes = default_ws_bytes(cap);
+    if (bytes < need) bytes = need;
+    void *p = nullptr;
+    e = cudaMalloc(&p, bytes);
+    if (e != cudaSuccess) return e;
+    e = cudaMemset(p, 0, bytes);
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) {
+        cudaFree(p);
+        return e;
+    }
+    w.ptr = p;
+    w.bytes = bytes;
+    *ptr = p;
+    return cudaSuccess;
 }
 
 static thread_local cudaError_t g_last_cuda_error = cudaSuccess;
 
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-static cudaError_t launch(const Params &prm, const Plan &pl, int dk, cudaStream_t stream) {
-    const KSpec k = spec_for(dk, prm.n_chunks);
-    cudaError_t e = prepare_kernel(k, pl.cluster);
+static cudaError_t launch(const Params &prm, const Plan &pl, void *workspace, cudaStream_t stream) {
+    const int dev = current_device();
+    const KSpec k = spec_of(pl.kind);
+    cudaError_t e = prepare_kernel(k, pl.kind == kSpan ? 1 : pl.cluster);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg;
     cudaLaunchAttribute attr[1];
     fill_config(cfg, attr, k, pl.cluster, pl.clusters, stream);
+    if (pl.kind == kSpan) {
+        sp::Work wk{};
+        wk.P = pl.cluster;
+        wk.Lc = pl.span_len;
+        if (pl.ws_bytes > 0) {
+            uint8_t *base = static_cast<uint8_t *>(workspace);
+            const int cap = span_capacity(dev, num_sms(dev), true);
+            wk.hdr = reinterpret_cast<unsigned long long *>(base);
+            wk.flags = reinterpret_cast<unsigned long long *>(base + 256);
+            wk.ws = reinterpret_cast<float *>(base + 256 + span_flags_bytes(cap));
+        }
+        void *args[] = {const_cast<Params *>(&prm), &wk};
+        return cudaLaunchKernelExC(&cfg, k.fn, args);
+    }
     void *args[] = {const_cast<Params *>(&prm)};
     return cudaLaunchKernelExC(&cfg, k.fn, args);
 }
@@ -914,14 +1072,9 @@ static gtr_status_t check_args(const void *q, const void *k, const void *v, cons
     return GTR_OK;
 }
 
-extern "C" gtr_status_t gtr_gla_fwd(const gtr_half_t *q, const gtr_half_t *k,
-                                    const gtr_half_t *v, const gtr_half_t *g, int B, int heads,
-                                    int Hgrid, int Wgrid, int dk, int dv, int direction, int chunk,
-                                    const float *init_state, gtr_half_t *out, float *final_state,
-                                    void *stream) {
-    const gtr_status_t st = check_args(q, k, v, g, B, heads, Hgrid, Wgrid, dk, dv, direction,
-                                       chunk, init_state, out, final_state);
-    if (st != GTR_OK) return st;
+static Params make_params(const gtr_half_t *q, const gtr_half_t *k, const gtr_half_t *v,
+                          const gtr_half_t *g, int B, int heads, int Hgrid, int Wgrid, int direction,
+                          const float *init_state, gtr_half_t *out, float *final_state) {
     Params prm{};
     prm.q = reinterpret_cast<const __half *>(q);
     prm.k = reinterpret_cast<const __half *>(k);
@@ -938,15 +1091,65 @@ extern "C" gtr_status_t gtr_gla_fwd(const gtr_half_t *q, const gtr_half_t *k,
     prm.dir = direction;
     prm.n_seq = B * heads;
     prm.n_chunks = (prm.N + kChunk - 1) / kChunk;
+    return prm;
+}
+
+static gtr_status_t cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return GTR_OK;
+    g_last_cuda_error = e;
+    cudaGetLastError();   // clear a non-sticky error
+    return GTR_ERR_CUDA;
+}
+
+extern "C" gtr_status_t gtr_gla_fwd(const gtr_half_t *q, const gtr_half_t *k,
+                                    const gtr_half_t *v, const gtr_half_t *g, int B, int heads,
+                                    int Hgrid, int Wgrid, int dk, int dv, int direction, int chunk,
+                                    const float *init_state, gtr_half_t *out, float *final_state,
+                                    void *stream) {
+    const gtr_status_t st = check_args(q, k, v, g, B, heads, Hgrid, Wgrid, dk, dv, direction,
+                                       chunk, init_state, out, final_state);
+    if (st != GTR_OK) return st;
+    const Params prm = make_params(q, k, v, g, B, heads, Hgrid, Wgrid, direction, init_state, out,
+                                   final_state);
     const Plan pl = make_plan(prm.n_seq, prm.n_chunks, dk, true);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const cudaError_t e = launch(prm, pl, dk, s);
-    if (e != cudaSuccess) {
-        g_last_cuda_error = e;
-        cudaGetLastError();   // clear the non-sticky launch error
-        return GTR_ERR_CUDA;
+    void *ws = nullptr;
+    if (pl.ws_bytes > 0) {
+        const gtr_status_t wst = cuda_status(default_workspace(current_device(), pl.ws_bytes, s, &ws));
+        if (wst != GTR_OK) return wst;
     }
-    return GTR_OK;
+    return cuda_status(launch(prm, pl, ws, s));
+}
+
+extern "C" size_t gtr_gla_workspace_bytes(int B, int heads, int Hgrid, int Wgrid, int dk, int dv,
+                                          int chunk) {
+    if (B <= 0 || heads <= 0 || Hgrid < 0 || Wgrid < 0 || chunk != kChunk) return 0;
+    if ((dk != 64 && dk != 128) || dv != kDV) return 0;
+    const long long N = (long long)Hgrid * Wgrid;
+    if (N > 0x7fffffffLL || (long long)B * heads > 0x7fffffffLL) return 0;
+    int ndev = 0;
+    const bool gpu = cudaGetDeviceCount(&ndev) == cudaSuccess && ndev > 0;
+    cudaGetLastError();
+    return make_plan((long)B * heads, (long)((N + kChunk - 1) / kChunk), dk, gpu).ws_bytes;
+}
+
+extern "C" gtr_status_t gtr_gla_fwd_ws(const gtr_half_t *q, const gtr_half_t *k,
+                                       const gtr_half_t *v, const gtr_half_t *g, int B, int heads,
+                                       int Hgrid, int Wgrid, int dk, int dv, int direction,
+                                       int chunk, const float *init_state, gtr_half_t *out,
+                                       float *final_state, void *workspace, size_t workspace_bytes,
+                                       void *stream) {
+    const gtr_status_t st = check_args(q, k, v, g, B, heads, Hgrid, Wgrid, dk, dv, direction,
+                                       chunk, init_state, out, final_state);
+    if (st != GTR_OK) return st;
+    const Params prm = make_params(q, k, v, g, B, heads, Hgrid, Wgrid, direction, init_state, out,
+                                   final_state);
+    const Plan pl = make_plan(prm.n_seq, prm.n_chunks, dk, true);
+    if (pl.ws_bytes > 0 &&
+        (workspace == nullptr || workspace_bytes < pl.ws_bytes ||
+         (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0))
+        return GTR_ERR_INVALID_ARG;
+    return cuda_status(launch(prm, pl, workspace, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 extern "C" gtr_status_t gtr_gla_device_status(void *stream) {
@@ -960,6 +1163,14 @@ extern "C" gtr_status_t gtr_gla_device_status(void *stream) {
     if (word != 0) {
         const unsigned zero = 0;
         cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero));
+        // a span launch that timed out can leave publish flags set: clear the cached
+        // workspace of this device so the next call starts from zero
+        const int dev = current_device();
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (g_default_ws[dev].ptr != nullptr) {
+            cudaMemset(g_default_ws[dev].ptr, 0, g_default_ws[dev].bytes);
+            cudaDeviceSynchronize();
+        }
         return GTR_ERR_TIMEOUT;
     }
     return GTR_OK;
@@ -991,7 +1202,7 @@ extern "C" gtr_status_t gtr_gla_plan(int B, int heads, int Hgrid, int Wgrid, int
     return GTR_OK;
 }
 
-extern "C" const char *gtr_gla_version(void) { return "0.2.0"; }
+extern "C" const char *gtr_gla_version(void) { return "0.3.0"; }
 
 extern "C" const char *gtr_gla_last_error(void) {
     return g_last_cuda_error == cudaSuccess ? "no error" : cudaGetErrorString(g_last_cuda_error);

@@ -20,8 +20,9 @@ LIB_PATH = os.path.join(_HERE, "libgtr_gla.so")
 GTR_OK, GTR_ERR_INVALID_ARG, GTR_ERR_UNSUPPORTED, GTR_ERR_CUDA, GTR_ERR_TIMEOUT = range(5)
 L2R, R2L, T2B, B2T = 0, 1, 2, 3
 
-EXPORTED_SYMBOLS = ("gtr_gla_fwd", "gtr_gla_device_status", "gtr_status_str", "gtr_gla_plan",
-                    "gtr_gla_version", "gtr_gla_last_error")
+EXPORTED_SYMBOLS = ("gtr_gla_fwd", "gtr_gla_workspace_bytes", "gtr_gla_fwd_ws",
+                    "gtr_gla_device_status", "gtr_status_str", "gtr_gla_plan", "gtr_gla_version",
+                    "gtr_gla_last_error")
 
 _lock = threading.Lock()
 _lib = None
@@ -49,6 +50,11 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         vp, i = ctypes.c_void_p, ctypes.c_int
         lib.gtr_gla_fwd.restype = i
         lib.gtr_gla_fwd.argtypes = [vp, vp, vp, vp] + [i] * 8 + [vp, vp, vp, vp]
+        lib.gtr_gla_workspace_bytes.restype = ctypes.c_size_t
+        lib.gtr_gla_workspace_bytes.argtypes = [i] * 7
+        lib.gtr_gla_fwd_ws.restype = i
+        lib.gtr_gla_fwd_ws.argtypes = ([vp, vp, vp, vp] + [i] * 8 + [vp, vp, vp]
+                                       + [vp, ctypes.c_size_t, vp])
         lib.gtr_gla_device_status.restype = i
         lib.gtr_gla_device_status.argtypes = [vp]
         lib.gtr_status_str.restype = ctypes.c_char_p
@@ -80,15 +86,7 @@ def _stream_handle(stream) -> ctypes.c_void_p:
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def gtr_gla_fwd(q, k, v, g, Hgrid: int, Wgrid: int, direction: int, init_state=None,
-                out=None, final_state=None, chunk: int = 64, stream=None):
-    """One token-mixer call on device tensors.
-
-    q, k, g: fp16 [B, N, heads, dk]; v: fp16 [B, N, heads, dv] (CUDA, contiguous).
-    init_state: fp32 [B, heads, dk, dv] or None.  final_state: an fp32 tensor to
-    fill, True to allocate one, or None to skip it.  Returns (out, final_state).
-    """
-    lib = load()
+def _prepare(q, k, v, g, Hgrid, Wgrid, init_state, out, final_state):
     B, N, heads, dk = q.shape
     dv = v.shape[-1]
     for name, t in (("q", q), ("k", k), ("g", g), ("v", v)):
@@ -106,11 +104,53 @@ def gtr_gla_fwd(q, k, v, g, Hgrid: int, Wgrid: int, direction: int, init_state=N
         if t is not None and (t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous()
                               or tuple(t.shape) != (B, heads, dk, dv)):
             raise ValueError(f"{name} must be a contiguous CUDA float32 [B,heads,dk,dv] tensor")
+    return (B, heads, dk, dv), out, final_state
+
+
+def gtr_gla_fwd(q, k, v, g, Hgrid: int, Wgrid: int, direction: int, init_state=None,
+                out=None, final_state=None, chunk: int = 64, stream=None):
+    """One token-mixer call on device tensors.
+
+    q, k, g: fp16 [B, N, heads, dk]; v: fp16 [B, N, heads, dv] (CUDA, contiguous).
+    init_state: fp32 [B, heads, dk, dv] or None.  final_state: an fp32 tensor to
+    fill, True to allocate one, or None to skip it.  Returns (out, final_state).
+    """
+    lib = load()
+    (B, heads, dk, dv), out, final_state = _prepare(q, k, v, g, Hgrid, Wgrid, init_state, out,
+                                                    final_state)
     st = lib.gtr_gla_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), B, heads, Hgrid, Wgrid, dk, dv,
                          int(direction), int(chunk), _ptr(init_state), _ptr(out),
                          _ptr(final_state), _stream_handle(stream))
     if st != GTR_OK:
         raise GTRError(st, "gtr_gla_fwd")
+    return out, final_state
+
+
+def workspace_bytes(B: int, heads: int, Hgrid: int, Wgrid: int, dk: int, dv: int,
+                    chunk: int = 64) -> int:
+    """Workspace gtr_gla_fwd_ws needs for a shape on the current device (0: none)."""
+    return int(load().gtr_gla_workspace_bytes(B, heads, Hgrid, Wgrid, dk, dv, chunk))
+
+
+def new_workspace(nbytes: int, device) -> torch.Tensor:
+    """A zero-filled device buffer usable as a workspace (at least one byte)."""
+    return torch.zeros(max(int(nbytes), 1), dtype=torch.uint8, device=device)
+
+
+def gtr_gla_fwd_ws(q, k, v, g, Hgrid: int, Wgrid: int, direction: int, workspace,
+                   init_state=None, out=None, final_state=None, chunk: int = 64, stream=None):
+    """gtr_gla_fwd with a caller-owned workspace (a CUDA uint8 tensor or None)."""
+    lib = load()
+    (B, heads, dk, dv), out, final_state = _prepare(q, k, v, g, Hgrid, Wgrid, init_state, out,
+                                                    final_state)
+    if workspace is not None and (not workspace.is_cuda or not workspace.is_contiguous()):
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.gtr_gla_fwd_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(g), B, heads, Hgrid, Wgrid, dk, dv,
+                            int(direction), int(chunk), _ptr(init_state), _ptr(out),
+                            _ptr(final_state), _ptr(workspace), nbytes, _stream_handle(stream))
+    if st != GTR_OK:
+        raise GTRError(st, "gtr_gla_fwd_ws")
     return out, final_state
 
 
@@ -133,7 +173,7 @@ def device_status(stream=None) -> int:
 
 
 def plan(B: int, heads: int, Hgrid: int, Wgrid: int, dk: int, dv: int):
-    """(cluster_size, num_clusters, smem_bytes) the library would launch with."""
+    """(CTAs per sequence, CTA groups, smem_bytes) the library would launch with."""
     lib = load()
     a, b, c = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
     st = lib.gtr_gla_plan(B, heads, Hgrid, Wgrid, dk, dv, ctypes.byref(a), ctypes.byref(b),
