@@ -117,6 +117,34 @@ gtr_status_t gtr_gla_fwd_ws(const gtr_half_t *q, const gtr_half_t *k, const gtr_
                             const float *init_state, gtr_half_t *out, float *final_state,
                             void *workspace, size_t workspace_bytes, void *stream);
 
+/* Size of the library's static device scratch used by gtr_gla_fwd_static: 4 MiB. */
+#define GTR_STATIC_WS_BYTES (4u << 20)
+
+/*
+ * gtr_gla_fwd that allocates nothing.  The paper has no counterpart: this is a
+ * memory-management variant of the library's own call.  Same arguments, results
+ * and argument errors as gtr_gla_fwd.  Where the shape's plan needs a workspace
+ * (gtr_gla_workspace_bytes > 0), the span kernel's workspace lives in one
+ * file-scope device array of GTR_STATIC_WS_BYTES bytes inside the library instead
+ * of memory from an allocator; no call makes cudaMalloc, cudaFree or any other
+ * allocating call.
+ *   - Set-up: the first call on a device that needs the scratch looks up its
+ *     device address (cudaGetSymbolAddress) with that device current and
+ *     zero-fills its header and publish flags (the part that must start at zero;
+ *     the kernel keeps it consistent from then on), synchronising the host once.
+ *     Make that first call before any stream capture begins.
+ *   - Limit: a shape whose plan needs more than GTR_STATIC_WS_BYTES returns
+ *     GTR_ERR_UNSUPPORTED with nothing launched.
+ *   - The scratch is shared by every gtr_gla_fwd_static call on the device:
+ *     calls that overlap in time (different streams or host threads) race on it
+ *     and give wrong results.  Calls in order on one stream are fine.
+ */
+gtr_status_t gtr_gla_fwd_static(const gtr_half_t *q, const gtr_half_t *k, const gtr_half_t *v,
+                                const gtr_half_t *g, int B, int heads, int Hgrid, int Wgrid,
+                                int dk, int dv, int direction, int chunk,
+                                const float *init_state, gtr_half_t *out, float *final_state,
+                                void *stream);
+
 /*
  * Syncs `stream`, then reads and clears the device error word (and any sticky
  * CUDA error).  Returns GTR_OK, GTR_ERR_TIMEOUT or GTR_ERR_CUDA.  On

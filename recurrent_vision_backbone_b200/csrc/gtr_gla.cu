@@ -1152,6 +1152,53 @@ extern "C" gtr_status_t gtr_gla_fwd_ws(const gtr_half_t *q, const gtr_half_t *k,
     return cuda_status(launch(prm, pl, workspace, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+// ------------------------------------------------------------------ static scratch
+namespace gtr {
+
+constexpr size_t kStaticWsBytes = GTR_STATIC_WS_BYTES;
+static __device__ __align__(256) unsigned char g_static_ws[kStaticWsBytes];
+static void *g_static_ws_ptr[64];
+
+// Device address of the static scratch on the current device `dev`, looked up once
+// (with `dev` current); the first lookup also zero-fills the header and flags.
+static cudaError_t static_scratch(int dev, void **ptr) {
+    const int cap = span_capacity(dev, num_sms(dev), true);
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_static_ws_ptr[dev] == nullptr) {
+        void *p = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&p, g_static_ws);
+        if (e != cudaSuccess) return e;
+        e = cudaMemset(p, 0, 256 + span_flags_bytes(cap > 0 ? cap : num_sms(dev)));
+        if (e == cudaSuccess) e = cudaDeviceSynchronize();
+        if (e != cudaSuccess) return e;
+        g_static_ws_ptr[dev] = p;
+    }
+    *ptr = g_static_ws_ptr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace gtr
+
+extern "C" gtr_status_t gtr_gla_fwd_static(const gtr_half_t *q, const gtr_half_t *k,
+                                           const gtr_half_t *v, const gtr_half_t *g, int B,
+                                           int heads, int Hgrid, int Wgrid, int dk, int dv,
+                                           int direction, int chunk, const float *init_state,
+                                           gtr_half_t *out, float *final_state, void *stream) {
+    const gtr_status_t st = check_args(q, k, v, g, B, heads, Hgrid, Wgrid, dk, dv, direction,
+                                       chunk, init_state, out, final_state);
+    if (st != GTR_OK) return st;
+    const Params prm = make_params(q, k, v, g, B, heads, Hgrid, Wgrid, direction, init_state, out,
+                                   final_state);
+    const Plan pl = make_plan(prm.n_seq, prm.n_chunks, dk, true);
+    if (pl.ws_bytes > kStaticWsBytes) return GTR_ERR_UNSUPPORTED;
+    void *ws = nullptr;
+    if (pl.ws_bytes > 0) {
+        const gtr_status_t wst = cuda_status(static_scratch(current_device(), &ws));
+        if (wst != GTR_OK) return wst;
+    }
+    return cuda_status(launch(prm, pl, ws, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 extern "C" gtr_status_t gtr_gla_device_status(void *stream) {
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (cudaStreamSynchronize(s) != cudaSuccess) {

@@ -19,9 +19,10 @@ LIB_PATH = os.path.join(_HERE, "libgtr_gla.so")
 
 GTR_OK, GTR_ERR_INVALID_ARG, GTR_ERR_UNSUPPORTED, GTR_ERR_CUDA, GTR_ERR_TIMEOUT = range(5)
 L2R, R2L, T2B, B2T = 0, 1, 2, 3
+STATIC_WS_BYTES = 4 << 20   # GTR_STATIC_WS_BYTES
 
 EXPORTED_SYMBOLS = ("gtr_gla_fwd", "gtr_gla_workspace_bytes", "gtr_gla_fwd_ws",
-                    "gtr_gla_device_status", "gtr_status_str", "gtr_gla_plan", "gtr_gla_version",
+                    "gtr_gla_fwd_static", "gtr_gla_device_status", "gtr_status_str", "gtr_gla_plan", "gtr_gla_version",
                     "gtr_gla_last_error")
 
 _lock = threading.Lock()
@@ -50,6 +51,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         vp, i = ctypes.c_void_p, ctypes.c_int
         lib.gtr_gla_fwd.restype = i
         lib.gtr_gla_fwd.argtypes = [vp, vp, vp, vp] + [i] * 8 + [vp, vp, vp, vp]
+        lib.gtr_gla_fwd_static.restype = i
+        lib.gtr_gla_fwd_static.argtypes = [vp, vp, vp, vp] + [i] * 8 + [vp, vp, vp, vp]
         lib.gtr_gla_workspace_bytes.restype = ctypes.c_size_t
         lib.gtr_gla_workspace_bytes.argtypes = [i] * 7
         lib.gtr_gla_fwd_ws.restype = i
@@ -123,6 +126,24 @@ def gtr_gla_fwd(q, k, v, g, Hgrid: int, Wgrid: int, direction: int, init_state=N
                          _ptr(final_state), _stream_handle(stream))
     if st != GTR_OK:
         raise GTRError(st, "gtr_gla_fwd")
+    return out, final_state
+
+
+def gtr_gla_fwd_static(q, k, v, g, Hgrid: int, Wgrid: int, direction: int, init_state=None,
+                       out=None, final_state=None, chunk: int = 64, stream=None):
+    """gtr_gla_fwd whose workspace is the library's static device scratch (no allocation
+    by the library; calls must not overlap in time).  Shapes whose plan needs more than
+    STATIC_WS_BYTES raise GTRError(GTR_ERR_UNSUPPORTED)."""
+    lib = load()
+    (B, heads, dk, dv), out, final_state = _prepare(q, k, v, g, Hgrid, Wgrid, init_state, out,
+                                                    final_state)
+    st = lib.gtr_gla_fwd_static(_ptr(q), _ptr(k), _ptr(v), _ptr(g), B, heads, Hgrid, Wgrid, dk,
+                                dv, int(direction), int(chunk), _ptr(init_state), _ptr(out),
+                                _ptr(final_state), _stream_handle(stream))
+    if st != GTR_OK:
+        raise GTRError(st, "gtr_gla_fwd_static" + (
+            f" (plan needs more than the {STATIC_WS_BYTES}-byte static scratch)"
+            if st == GTR_ERR_UNSUPPORTED and dk == 64 and dv == 64 and chunk == 64 else ""))
     return out, final_state
 
 
