@@ -87,10 +87,14 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:12]
 
 
+# the kernel every dk = 64 call of the bench workloads launches
+KERNEL = "gla_fwd_span_kernel"
+
+
 def recorded_traffic(workload_name: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on the
     current kernel source; else None."""
-    path = os.path.join(ROOT, "profiles", f"gla_fwd_kernel_{workload_name}.md")
+    path = os.path.join(ROOT, "profiles", f"{KERNEL}_{workload_name}.md")
     try:
         text = open(path).read()
     except OSError:
@@ -263,7 +267,8 @@ def roofline(w, ms_per_launch, workload_name):
     peak, which = measured_peaks()
     b = bytes_alg(w)
     achieved = b / (ms_per_launch * 1e-3) / 1e9
-    return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+    return {"kernel": KERNEL, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+            "unit": "GB/s",
             "frac": round(achieved / peak, 4), "traffic": recorded_traffic(workload_name),
             "peak_source": which, "bytes_alg_per_launch": b, "flops_alg_per_launch": flops_alg(w)}
 
@@ -335,7 +340,7 @@ def gpu_arm(args):
     stream = torch.cuda.Stream(device=device)
     primary = args.workload
     w1 = WORKLOADS[primary]
-    wl = Workload(w1, rank, device)
+    wl = Workload(w1, rank, device, n_sets=args.sets)
     clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
                           else local)
     clocks.start()
@@ -367,7 +372,7 @@ def gpu_arm(args):
     torch.cuda.empty_cache()
     if not args.no_secondary and primary != SECONDARY:
         w2 = WORKLOADS[SECONDARY]
-        wl2 = Workload(w2, rank, device)
+        wl2 = Workload(w2, rank, device, n_sets=args.sets)
         ms2, n2 = measure(wl2, max(8, args.steps // 16), max(3, args.warmup // 16), stream, world)
         line["secondary"] = {
             "workload": SECONDARY, "tokens_per_call": w2.B * w2.N,
@@ -479,6 +484,9 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--sets", type=int, default=None,
+                    help="rotating input sets (default: enough to exceed 4x L2); small "
+                         "profiler captures use fewer")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -67,7 +67,8 @@ struct L {
     static constexpr int cmeta = rowb + 3 * 64 * 4; // per chunk: max|q|, max|o| [kMaxSpan][2]
     static constexpr int skipf = cmeta + kMaxSpan * 8;  // per chunk: correction negligible
     static constexpr int rmax = skipf + kMaxSpan * 4;   // row maxima of |S_in| [64]
-    static constexpr int misc = rmax + 256;         // per parity: flags[4] qmax[4] kmax
+    static constexpr int ltab = rmax + 256;         // loader's token rows [64]
+    static constexpr int misc = ltab + 256;         // per parity: flags[4] qmax[4] kmax
     static constexpr int bars = misc + 128;
     static constexpr int bytes = bars + 24 * 8;
     static constexpr int alloc = bytes + 1024;
@@ -118,30 +119,32 @@ __device__ __forceinline__ void wait_l(uint64_t *b, uint32_t parity, bool &to) {
     }
 }
 
-// Loader: 16-byte cp.async of chunk c's rows of up to four tensors into staging.
-// Null tensors are skipped; rows past the grid are zero-filled.
-__device__ __forceinline__ void load_rows4(const Params &P, uint8_t *sm, int seq, int c, int lane,
-                                           const __half *t0, const __half *t1, const __half *t2,
-                                           const __half *t3) {
+// Loader warp: the 64 rows of chunk c of q, k, g, v into the staging tiles (row t at
+// byte t * 128) with 16-byte cp.async, eight lanes per 128-byte row so that one warp
+// instruction moves four whole rows.  Rows past the grid are zero-filled.
+__device__ __forceinline__ void load_chunk(const Params &P, uint8_t *sm, int seq, int c, int lane) {
     const uint32_t st = smem_u32(sm + L::stg);
+    int *rowtab = reinterpret_cast<int *>(sm + L::ltab);
     const int b = seq / P.heads, h = seq - b * P.heads;
-    const int p0 = c * kChunk;
-    const __half *tens[4] = {t0, t1, t2, t3};
+    __syncwarp();   // every lane is done with the previous chunk's table
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
-        const int t = lane + 32 * half;
-        const bool ok = p0 + t < P.N;
-        size_t ro = 0;
-        if (ok) ro = (size_t)((b * P.N + scan_to_token(p0 + t, P.H, P.W, P.dir)) * P.heads + h);
-        const uint32_t nb = ok ? 16u : 0u;
-#pragma unroll
-        for (int ten = 0; ten < 4; ++ten) {
-            if (tens[ten] == nullptr) continue;
-            const __half *src = tens[ten] + ro * 64;
-#pragma unroll
-            for (int pc = 0; pc < 8; ++pc)
-                cp_async16(st + ten * kTile + t * 128 + 16 * pc, src + 8 * pc, nb);
-        }
+        const int t = lane + 32 * half, p = c * kChunk + t;
+        rowtab[t] = p < P.N ? (b * P.N + scan_to_token(p, P.H, P.W, P.dir)) * P.heads + h : -1;
+    }
+    __syncwarp();
+    const int sub = lane >> 3, pc = lane & 7;
+#pragma unroll 4
+    for (int i = 0; i < 16; ++i) {
+        const int t = 4 * i + sub;
+        const int ro = rowtab[t];
+        const uint32_t nb = ro >= 0 ? 16u : 0u;
+        const size_t off = (size_t)(ro >= 0 ? ro : 0) * 64 + 8 * pc;
+        const uint32_t d = st + t * 128 + 16 * pc;
+        cp_async16(d, P.q + off, nb);
+        cp_async16(d + kTile, P.k + off, nb);
+        cp_async16(d + 2 * kTile, P.g + off, nb);
+        cp_async16(d + 3 * kTile, P.v + off, nb);
     }
 }
 
@@ -635,7 +638,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_span_kernel(const Params 
             // ================================================= loader (warp 12)
             for (int ci = 0; ci < nch; ++ci) {
                 wait_l(bar(sm, B_STGE), (n_stg & 1u) ^ 1u, to);
-                load_rows4(P, sm, seq, c0 + ci, lane, P.q, P.k, P.g, P.v);
+                load_chunk(P, sm, seq, c0 + ci, lane);
                 cp_async_mbar_arrive_noinc(bar(sm, B_STGF));
                 ++n_stg;
             }

@@ -8,26 +8,26 @@
 // FP32 accumulation (section "速度到底快在哪，TensorRT部署做了什么": the heavy work of a
 // chunk is parallel, only the chunk-boundary state is passed in order).
 //
-// Kernel structure (one launch per call):
-//   * A thread-block cluster of P CTAs owns one sequence at a time (clusters loop
-//     over sequences).  In round r, CTA `rank` processes chunk r*P + rank.
-//   * Per chunk, inside one CTA:
-//       - q/k/g/v rows are fetched with 16-byte cp.async straight into 128B-swizzled
-//         UMMA tiles; the scan direction is applied only in the row addresses.
-//       - a = exp(g); inside each 16-token sub-block the inclusive prefix product pi
-//         and exclusive suffix product sigma of a, and the sub-block totals T.
-//         Every decay factor fed to the tensor cores is a product of a's <= 1,
-//         except the diagonal sub-blocks, whose factor pi/T is bounded by exp(8)
-//         and falls back to an exact fp32 evaluation beyond that.
-//       - tcgen05.mma (fp16 x fp16 -> fp32 in TMEM):
-//           dS     = (K * sigma * after)^T V                    (64..128 x 64)
-//           scores = (Q * pi * c_J) (K * sigma)^T  per key sub-block J
-//           O      = (Q * pi * before) S_prev + tril(scores) V
-//   * The chunk-to-chunk state pass S_c = d_c * S_{c-1} + dS_c is the only
-//     sequential step.  It runs as an element-sliced scan over the cluster:
-//     CTA j reads slice j of every chunk's (d_c, dS_c) from its peers' shared
-//     memory (DSMEM), chains it in fp32, and writes S_{c-1} (fp16) straight into
-//     the owning CTA's UMMA operand tile.
+// Kernels (one launch per call):
+//   * gla_fwd_span.cuh (dk = 64): each sequence is cut into spans of chunks that run
+//     on separate SMs with purely local state chains; one aggregate per span through
+//     a workspace, a look-back fold, and a deferred correction of the later spans'
+//     outputs.  The default for dk = 64.
+//   * gla_fwd_kernel<DK> below (dk = 64 or 128): a thread-block cluster of P CTAs
+//     owns one sequence at a time; in round r CTA `rank` processes chunk r*P + rank
+//     and the chunk-to-chunk state pass S_c = d_c * S_{c-1} + dS_c runs as an
+//     element-sliced scan over the cluster through distributed shared memory.
+//   * gla_fwd_ws.cuh (dk = 64): the cluster decomposition with warp-specialised
+//     roles and mbarrier hand-offs.
+//   Per chunk, in every kernel: q/k/g/v rows are staged with 16-byte cp.async (the
+//   scan direction is applied only in the row addresses); a = exp(g) with
+//   sub-block prefix/suffix products and totals, so that every decay factor fed to
+//   the tensor cores is a product of a's <= 1 except the diagonal sub-blocks,
+//   whose factor pi/T is bounded by exp(8) and falls back to an exact fp32
+//   evaluation beyond that; then tcgen05.mma (fp16 x fp16 -> fp32 in TMEM):
+//       dS     = (K * sigma * after)^T V
+//       scores = (Q * pi * c_J) (K * sigma)^T  per key sub-block J
+//       O      = (Q * pi * before) S_prev + tril(scores) V
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
