@@ -7,14 +7,20 @@
 // "速度到底快在哪，TensorRT部署做了什么": only the chunk-boundary state is passed in order)
 // is purely local, so no per-chunk traffic crosses CTAs:
 //
-//   phase 1  stream the span's chunks from a zero state (span 0: from S0):
-//            loader warp 12 stages raw rows with cp.async; group A (warps 0-7) builds
-//            the gated operands, issues MMA 1 (scores, state delta) and, in its TMEM
-//            readout, writes S_prev (fp16 MMA operand) and updates the fp32 state
-//            S <- d * S + dS in shared memory; group B (warps 8-11) issues MMA 2
-//            (O = Qint S_prev + tril(scores) V) and stores the outputs.
-//   phase 2  publish the span's aggregate (state reached from zero, product of the
-//            decays) to the workspace; span 0 publishes its inclusive state.
+//   phase 1  stream the span's chunks from a zero state (span 0: from S0), as a
+//            three-role pipeline over two buffers:
+//              loader (warp 12)   cp.async of q, k, g rows into staging and of v
+//                                 straight into its swizzled operand tile;
+//              group A (warps 0-7) gating of chunk c (Qint = q P, K~ = k / P, ...)
+//                                 while MMA 1 of chunk c-1 runs, then MMA 1(c) =
+//                                 (dS, scores) once group B has read chunk c-1;
+//              group B (warps 8-11) TMEM readout of chunk c: scores into the causal
+//                                 P tile, MMA 2(c) = Qint S_prev + P V, and while it
+//                                 runs S <- d * S + dS in shared memory (its fp16
+//                                 copy is S_prev of chunk c+1); output stores.
+//   phase 2  the span's last readout publishes its aggregate (state reached from
+//            zero, product of the decays) to the workspace; span 0 publishes its
+//            inclusive state.
 //   phase 3  look back: fold the aggregates of the earlier spans into S_in, the true
 //            state entering this span.
 //   phase 4  correct the outputs for the missing S_in term.  For a chunk c starting
@@ -22,7 +28,7 @@
 //            span, the term is (Q * P) diag(D_c) S_in.  The first kHold chunks keep
 //            their fp32 outputs in TMEM and get the exact term added by one MMA each;
 //            later chunks get it by re-reading q, g and o, unless a bound shows the term
-//            is below 2^-22 of the chunk's largest output (the decays make it vanish
+//            is below 2^-16 of the chunk's largest output (the decays make it vanish
 //            after a few chunks for the gates on the pages' workloads).
 //   phase 5  the last span writes the final state  D_span * S_in + S_local.
 //
@@ -37,43 +43,44 @@ constexpr int kThreadsA = 256;              // warps 0-7
 constexpr int kThreadsB = 128;              // warps 8-11
 constexpr int kThreads = kThreadsA + kThreadsB + 32;   // + loader warp 12
 constexpr int kDK = 64;
-constexpr int kHold = 5;                    // chunks per span whose outputs wait in TMEM
-constexpr int kMaxSpan = 64;                // chunks of a later span with recorded decays
-constexpr uint32_t kBarA = 1, kBarB = 2;
+constexpr int kHold = 4;                    // chunks per span whose outputs wait in TMEM
+constexpr int kMaxSpan = 32;                // chunks of a span with recorded decays
+constexpr uint32_t kBarA = 1, kBarB = 2;    // named barriers; 3..5: phase-4 epilogue teams
 constexpr int kAggFloats = kDK * kDV + kDK; // state + decay product
-constexpr uint32_t kColMma1 = 0, kColWork = 128, kColHold = 192;
+// TMEM columns: dS of MMA 1 (two buffers), scores of MMA 1, MMA 2 work block, the
+// held chunks' output blocks
+constexpr uint32_t kColDS = 0, kColScores = 128, kColWork = 192, kColHold = 256;
 constexpr int kSpanTmemCols = 512;
 
 // ------------------------------------------------------------------ smem map
 struct L {
-    static constexpr int stg = 0;                   // raw rows q,k,g,v (or q,-,g,o) [64][128 B] x 4
-    static constexpr int qint = stg + 4 * kTile;    // working Qint, x2
-    static constexpr int kt = qint + 2 * kTile;     // K / P (or K * sigma * after)
-    static constexpr int vop = kt + kTile;          // V swizzled, x2
-    static constexpr int p = vop + 2 * kTile;       // masked scores, x2
-    static constexpr int qj = p + 2 * kTile;        // packed Q^(J) (sub-block path)
+    static constexpr int stg_bytes = 3 * kTile;         // raw rows q, k, g [64][128 B]
+    static constexpr int stg = 0;                       // x2 buffers
+    static constexpr int vop = stg + 2 * stg_bytes;     // V swizzled (loaded directly), x3
+    static constexpr int qint = vop + 3 * kTile;        // Q * P, x2
+    static constexpr int kt = qint + 2 * kTile;         // K / P or K * sigma * after, x2
+    static constexpr int p = kt + 2 * kTile;            // masked scores, then output staging
+    static constexpr int qj = p + kTile;                // packed Q^(J) (sub-block path)
     static constexpr int qj_bytes = (64 + 48 + 32 + 16) * 128;
-    static constexpr int kbar = qj + qj_bytes;      // K * sigma (sub-block path)
-    static constexpr int sop = kbar + kTile;        // S_prev fp16, x2
-    static constexpr int sst = sop + 2 * kTile;     // running state fp32 [64][64] swizzled
-    static constexpr int ost = sst + 64 * 256;      // output staging
-    static constexpr int ring = ost + kTile;        // Qint of the held chunks
-    static constexpr int dcum = ring + kHold * kTile;   // D_c per chunk of the span [kMaxSpan][64]
-    static constexpr int dloc = dcum + kMaxSpan * 256;  // d of the current chunk [64]
-    static constexpr int dacc = dloc + 256;         // running product of decays [64]
-    static constexpr int htot = dacc + 256;         // half-block totals [8][64]
-    static constexpr int diag = htot + 8 * 64 * 4;  // exact diagonal blocks [4][16][16]
-    static constexpr int rowb = diag + 4 * 16 * 16 * 4; // token rows [3 teams][64]
-    static constexpr int cmeta = rowb + 3 * 64 * 4; // per chunk: max|q|, max|o| [kMaxSpan][2]
+    static constexpr int kbar = qj + qj_bytes;          // K * sigma (sub-block path)
+    static constexpr int sop = kbar + kTile;            // S_prev fp16, x2
+    static constexpr int sst = sop + 2 * kTile;         // running state fp32 [64][64] swizzled
+    static constexpr int ring = sst + 64 * 256;         // Qint * D_c of the held chunks
+    static constexpr int dcum = ring + kHold * kTile;   // D_c, c = 0 .. kMaxSpan [kMaxSpan+1][64]
+    static constexpr int dloc = dcum + (kMaxSpan + 1) * 256;   // chunk decay d [2][64]
+    static constexpr int htot = dloc + 2 * 256;         // half-block totals [8][64]
+    static constexpr int diag = htot + 8 * 64 * 4;      // exact diagonal blocks [2][4][16][16]
+    static constexpr int rowb = diag + 2 * 4 * 16 * 16 * 4; // token rows [3 teams][64]
+    static constexpr int cmeta = rowb + 3 * 64 * 4;     // per chunk: max|q|, max|o| [kMaxSpan][2]
     static constexpr int skipf = cmeta + kMaxSpan * 8;  // per chunk: correction negligible
     static constexpr int rmax = skipf + kMaxSpan * 4;   // row maxima of |S_in| [64]
-    static constexpr int ltab = rmax + 256;         // loader's token rows [64]
-    static constexpr int misc = ltab + 256;         // per parity: flags[4] qmax[4] kmax
+    static constexpr int ltab = rmax + 256;             // loader's token rows [64]
+    static constexpr int misc = ltab + 256;             // per parity (64 B): flags[4] qmax[4] kmax
     static constexpr int bars = misc + 128;
     static constexpr int bytes = bars + 24 * 8;
     static constexpr int alloc = bytes + 1024;
-    // after phase 1 the score tiles hold S_in (fp32 [64][64], swizzled)
-    static constexpr int sin = p;
+    // after phase 1 the K~ tiles hold S_in (fp32 [64][64], swizzled)
+    static constexpr int sin = kt;
 
     static __host__ __device__ constexpr int qj_region(int J) {
         return 128 * (J == 0 ? 0 : J == 1 ? 64 : J == 2 ? 112 : 144);
@@ -82,14 +89,17 @@ struct L {
 static_assert(L::alloc <= 227 * 1024, "shared memory budget");
 
 enum {
-    B_STGF = 0,   // raw rows landed (32 loader arrivals)
-    B_STGE = 1,   // group A done with the staging buffer
-    B_MMA1 = 2,
-    B_MMA2 = 3,
-    B_OPSF = 4,   // [2] operands of a chunk ready for MMA 2
-    B_OPSE = 6,   // [2] MMA 2 done with them
-    B_FIX = 8,    // correction MMAs complete
-    B_TMEM = 10   // (uint32_t) TMEM base
+    B_STGF = 0,   // [2] staging (+ V tile) landed: 32 loader arrivals
+    B_STGE = 2,   // [2] group A done with the staging buffer
+    B_MMA1 = 19,  // [2] MMA 1 of a chunk of this parity complete (waited by groups A and B)
+    B_SCON = 5,   // group B has read the scores out of TMEM
+    B_OPSF = 6,   // [2] S_prev of a chunk ready for its MMA 2
+    B_OPSE = 8,   // [2] MMA 2 done with Qint, S_prev of a buffer (tcgen05.commit)
+    B_MMA2 = 10,
+    B_FIX = 11,   // correction MMAs complete
+    B_TMEM = 13,  // (uint32_t) TMEM base
+    B_VE = 14,    // [3] MMA 2 done with a V tile (tcgen05.commit)
+    B_GATE = 17   // [2] group A's gating of a chunk done (operands, flags, diagonal blocks)
 };
 
 // Workspace protocol.  hdr[0] counts completed launches (the generation), hdr[1]
@@ -118,19 +128,31 @@ __device__ __forceinline__ void wait_l(uint64_t *b, uint32_t parity, bool &to) {
         set_error(kErrTimeout);
     }
 }
+// Waits for phase `k` of a barrier whose phases complete in order, given the count
+// `seen` of phases this thread has already observed (never more than one phase can
+// be ahead of the waiter for the barriers this is used on).
+__device__ __forceinline__ void wait_phase(uint64_t *b, uint32_t &seen, uint32_t k, bool &to) {
+    while (seen <= k) {
+        wait_l(b, seen & 1u, to);
+        ++seen;
+    }
+}
 
-// Loader warp: the 64 rows of chunk c of q, k, g, v into the staging tiles (row t at
-// byte t * 128) with 16-byte cp.async, eight lanes per 128-byte row so that one warp
-// instruction moves four whole rows.  Rows past the grid are zero-filled.
-__device__ __forceinline__ void load_chunk(const Params &P, uint8_t *sm, int seq, int c, int lane) {
-    const uint32_t st = smem_u32(sm + L::stg);
+// Loader warp: chunk c's 64 rows of q, k, g into staging buffer `b` (row t at byte
+// t * 128, unswizzled) and of v into the swizzled operand tile vop[vb], with 16-byte
+// cp.async, eight lanes per 128-byte row so that one warp instruction moves four
+// whole rows.  Rows past the grid are zero-filled.
+__device__ __forceinline__ void load_chunk(const Params &P, uint8_t *sm, int seq, int c, int b,
+                                           int vb, int lane) {
+    const uint32_t st = smem_u32(sm + L::stg + b * L::stg_bytes);
+    const uint32_t vo = smem_u32(sm + L::vop + vb * kTile);
     int *rowtab = reinterpret_cast<int *>(sm + L::ltab);
-    const int b = seq / P.heads, h = seq - b * P.heads;
+    const int bb = seq / P.heads, h = seq - bb * P.heads;
     __syncwarp();   // every lane is done with the previous chunk's table
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
         const int t = lane + 32 * half, p = c * kChunk + t;
-        rowtab[t] = p < P.N ? (b * P.N + scan_to_token(p, P.H, P.W, P.dir)) * P.heads + h : -1;
+        rowtab[t] = p < P.N ? (bb * P.N + scan_to_token(p, P.H, P.W, P.dir)) * P.heads + h : -1;
     }
     __syncwarp();
     const int sub = lane >> 3, pc = lane & 7;
@@ -144,7 +166,7 @@ __device__ __forceinline__ void load_chunk(const Params &P, uint8_t *sm, int seq
         cp_async16(d, P.q + off, nb);
         cp_async16(d + kTile, P.k + off, nb);
         cp_async16(d + 2 * kTile, P.g + off, nb);
-        cp_async16(d + 3 * kTile, P.v + off, nb);
+        cp_async16(vo + sw_off(t, 8 * pc), P.v + off, nb);
     }
 }
 
@@ -219,6 +241,361 @@ __device__ __forceinline__ void fill_rows(const Params &P, int seq, int c, int *
     }
 }
 
+// Per-parity scratch of group A (64 bytes): flags[4] (sub-block uses the exact
+// diagonal), qmax[4] (max |q| per sub-block), kmax (max |k|), slow.
+__device__ __forceinline__ int *misc_flags(uint8_t *sm, int b) {
+    return reinterpret_cast<int *>(sm + L::misc + 64 * b);
+}
+__device__ __forceinline__ unsigned *misc_qmax(uint8_t *sm, int b) {
+    return reinterpret_cast<unsigned *>(sm + L::misc + 64 * b + 16);
+}
+__device__ __forceinline__ unsigned *misc_kmax(uint8_t *sm, int b) {
+    return reinterpret_cast<unsigned *>(sm + L::misc + 64 * b + 32);
+}
+__device__ __forceinline__ int *misc_slow(uint8_t *sm, int b) {   // chunk took the sub-block path
+    return reinterpret_cast<int *>(sm + L::misc + 64 * b + 36);
+}
+
+// Group A (threads 0..255): gating of chunk ci of the span from staging buffer b.
+// Writes Qint -> qint[b], K~ -> kt[b] (sub-block path: also Q^(J) -> qj, K sigma ->
+// kbar, exact diagonal blocks -> diag[b]), Qint * D_ci -> ring[ci] for a held chunk,
+// the chunk decay d -> dloc[b] and D_{ci+1} -> dcum, then signals GATE[b].  The
+// sub-block path first waits for MMA 1 of chunk ci-1 (phase index `m1_prev`; it may
+// still read qj / kbar).  Returns true on the sub-block path.
+__device__ __forceinline__ bool gate_chunk(const Params &P, uint8_t *sm, int ci, int b, int nrows,
+                                           bool held, uint32_t &m1_seen, uint32_t m1_prev, bool &to) {
+    // (m1_seen / m1_prev: phase count and index of MMA 1 of chunk ci-1 on MMA1[b ^ 1])
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int gI = warp >> 1, ghf = warp & 1, gt0 = 16 * gI + 8 * ghf, gh = 2 * gI + ghf;
+    float *htot = reinterpret_cast<float *>(sm + L::htot);
+    float *diagx = reinterpret_cast<float *>(sm + L::diag) + b * 1024;
+    float *dcum = reinterpret_cast<float *>(sm + L::dcum);
+    const uint8_t *st = sm + L::stg + b * L::stg_bytes;
+    uint8_t *qo = sm + L::qint + b * kTile;
+    uint8_t *ko = sm + L::kt + b * kTile;
+    uint8_t *qr = sm + L::ring + (held ? ci : 0) * kTile;
+    int *flags = misc_flags(sm, b);
+    unsigned *qmax = misc_qmax(sm, b);
+    unsigned *kmax = misc_kmax(sm, b);
+    // group B read this parity's flags and diagonal blocks (chunk ci-2) before its MMA 2,
+    // whose completion released this buffer
+    if (tid < 4) flags[tid] = 0;
+    // ---------- pass 1: a = exp(g), half-block prefix / suffix products and totals
+    float pl[8][2], sl[8][2];
+    __half2 qh[8], kh[8];
+    {
+        __half2 qm2 = __float2half2_rn(0.f), km2 = __float2half2_rn(0.f);
+        float a0[8], a1[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const uint32_t o = (gt0 + u) * 128 + 4 * lane;
+            const float2 gv = ld_h2(st + 2 * kTile + o);
+            qh[u] = *reinterpret_cast<const __half2 *>(st + o);
+            kh[u] = *reinterpret_cast<const __half2 *>(st + kTile + o);
+            a0[u] = exp_f(gv.x);
+            a1[u] = exp_f(gv.y);
+            qm2 = __hmax2(qm2, __habs2(qh[u]));
+            km2 = __hmax2(km2, __habs2(kh[u]));
+        }
+        float r0 = 1.f, r1 = 1.f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            r0 *= a0[u];
+            r1 *= a1[u];
+            pl[u][0] = r0;
+            pl[u][1] = r1;
+        }
+        r0 = 1.f;
+        r1 = 1.f;
+#pragma unroll
+        for (int u = 7; u >= 0; --u) {
+            sl[u][0] = r0;
+            sl[u][1] = r1;
+            r0 *= a0[u];
+            r1 *= a1[u];
+        }
+        *reinterpret_cast<float2 *>(htot + gh * 64 + 2 * lane) = make_float2(pl[7][0], pl[7][1]);
+        const float qm = fmaxf(__low2float(qm2), __high2float(qm2));
+        const float km = fmaxf(__low2float(km2), __high2float(km2));
+        const unsigned wq = __reduce_max_sync(0xffffffffu, __float_as_uint(qm));
+        const unsigned wk = __reduce_max_sync(0xffffffffu, __float_as_uint(km));
+        if (lane == 0) {
+            atomicMax(&qmax[gI], wq);
+            atomicMax(kmax, wk);
+        }
+    }
+    named_sync(kBarA, kThreadsA);
+    // ---------- chunk factors for my two channels
+    float dch[2], bef[2], aft[2];
+    bool bad = __uint_as_float(*kmax) > kFastMaxK;
+    {
+        float2 ht[8];
+#pragma unroll
+        for (int h8 = 0; h8 < 8; ++h8) ht[h8] = *reinterpret_cast<const float2 *>(htot + h8 * 64 + 2 * lane);
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            float d = 1.f, bf = 1.f, af = 1.f;
+#pragma unroll
+            for (int h8 = 0; h8 < 8; ++h8) {
+                const float x = e ? ht[h8].y : ht[h8].x;
+                d *= x;
+                if (h8 < gh) bf *= x;
+                if (h8 > gh) af *= x;
+            }
+            dch[e] = d;
+            bef[e] = bf;
+            aft[e] = af;
+            bad |= !(d >= kFastMinDecay);
+        }
+    }
+    const bool slow = named_sync_or(kBarA, kThreadsA, bad);
+    const float2 dc = *reinterpret_cast<const float2 *>(dcum + (held ? ci : 0) * 64 + 2 * lane);
+    if (gh == 0) {
+        *reinterpret_cast<float2 *>(sm + L::dloc + b * 256 + 8 * lane) = make_float2(dch[0], dch[1]);
+        if (ci + 1 <= kMaxSpan) {
+            const float2 d0 = *reinterpret_cast<const float2 *>(dcum + ci * 64 + 2 * lane);
+            *reinterpret_cast<float2 *>(dcum + (ci + 1) * 64 + 2 * lane) =
+                make_float2(d0.x * dch[0], d0.y * dch[1]);
+        }
+    }
+    if (!slow) {
+        // ---------- fast path: Qint = q P, K~ = k / P (= k * suffix / d)
+        const float i0 = aft[0] / dch[0], i1 = aft[1] / dch[1];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const uint32_t o = sw_off(gt0 + u, 2 * lane);
+            const float2 qv = __half22float2(qh[u]);
+            const float2 kv = __half22float2(kh[u]);
+            const float a0 = qv.x * (pl[u][0] * bef[0]), a1 = qv.y * (pl[u][1] * bef[1]);
+            st_h2(qo + o, a0, a1);
+            if (held) st_h2(qr + o, a0 * dc.x, a1 * dc.y);
+            st_h2(ko + o, kv.x * (sl[u][0] * i0), kv.y * (sl[u][1] * i1));
+        }
+    } else {
+        // ---------- sub-block path: 16-token sub-blocks, factors <= 1 off the diagonal
+        float T[4][2];
+#pragma unroll
+        for (int L4 = 0; L4 < 4; ++L4) {
+            const float2 h0 = *reinterpret_cast<const float2 *>(htot + (2 * L4) * 64 + 2 * lane);
+            const float2 h1 = *reinterpret_cast<const float2 *>(htot + (2 * L4 + 1) * 64 + 2 * lane);
+            T[L4][0] = h0.x * h1.x;
+            T[L4][1] = h0.y * h1.y;
+        }
+        bool dbad = false;
+#pragma unroll
+        for (int L4 = 0; L4 < 4; ++L4)
+            if (L4 == gI) dbad |= !(T[L4][0] >= kDiagMinTotal) || !(T[L4][1] >= kDiagMinTotal);
+        dbad |= __uint_as_float(qmax[gI]) > kDiagMaxQ;
+        if (__any_sync(0xffffffffu, dbad) && lane == 0) atomicOr(&flags[gI], 1);
+        named_sync(kBarA, kThreadsA);
+        const int anyflag = flags[0] | flags[1] | flags[2] | flags[3];
+        if (anyflag) {
+            for (int pr = tid; pr < 4 * 256; pr += kThreadsA) {
+                const int I = pr >> 8, u = (pr >> 4) & 15, w = pr & 15;
+                if (!flags[I] || w > u) continue;
+                const int tu = I * kSub + u, tw = I * kSub + w;
+                float acc = 0.f;
+                if (tu < nrows) {
+                    for (int i = 0; i < kDK; ++i) {
+                        float lg = 0.f;
+                        for (int r2 = tw + 1; r2 <= tu; ++r2)
+                            lg += __half2float(*reinterpret_cast<const __half *>(st + 2 * kTile + r2 * 128 + 2 * i));
+                        const float qv = __half2float(*reinterpret_cast<const __half *>(st + tu * 128 + 2 * i));
+                        const float kv = __half2float(*reinterpret_cast<const __half *>(st + kTile + tw * 128 + 2 * i));
+                        acc += qv * kv * exp_f(lg);
+                    }
+                }
+                diagx[(I * 16 + u) * 16 + w] = acc;
+            }
+        }
+        // MMA 1 of the previous chunk may still read qj / kbar
+        if (ci > 0) {
+            wait_phase(bar(sm, B_MMA1 + (b ^ 1)), m1_seen, m1_prev, to);
+            tc_fence_after();
+        }
+        named_sync(kBarA, kThreadsA);
+        const bool diag_bad = flags[gI] != 0;
+        float cf[2][4], bI[2], aI[2], hin[2], hout[2];
+        const float2 h0 = *reinterpret_cast<const float2 *>(htot + (2 * gI) * 64 + 2 * lane);
+        const float2 h1 = *reinterpret_cast<const float2 *>(htot + (2 * gI + 1) * 64 + 2 * lane);
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            float b0 = 1.f, a0 = 1.f, tI = 1.f;
+#pragma unroll
+            for (int L4 = 0; L4 < 4; ++L4) {
+                if (L4 < gI) b0 *= T[L4][e];
+                if (L4 > gI) a0 *= T[L4][e];
+                if (L4 == gI) tI = T[L4][e];
+            }
+            bI[e] = b0;
+            aI[e] = a0;
+#pragma unroll
+            for (int J = 0; J < 4; ++J) {
+                float cj = 1.f;
+#pragma unroll
+                for (int L4 = 0; L4 < 4; ++L4)
+                    if (L4 > J && L4 < gI) cj *= T[L4][e];
+                cf[e][J] = (J == gI) ? (diag_bad ? 0.f : 1.f / tI) : cj;
+            }
+            hin[e] = ghf ? (e ? h0.y : h0.x) : 1.f;
+            hout[e] = ghf ? 1.f : (e ? h1.y : h1.x);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int t = gt0 + u;
+            const uint32_t o = sw_off(t, 2 * lane);
+            const float2 qv = __half22float2(qh[u]);
+            const float2 kv = __half22float2(kh[u]);
+            const float qp0 = qv.x * (pl[u][0] * hin[0]);
+            const float qp1 = qv.y * (pl[u][1] * hin[1]);
+            const float ks0 = kv.x * (sl[u][0] * hout[0]);
+            const float ks1 = kv.y * (sl[u][1] * hout[1]);
+            st_h2(qo + o, qp0 * bI[0], qp1 * bI[1]);
+            if (held) st_h2(qr + o, qp0 * bI[0] * dc.x, qp1 * bI[1] * dc.y);
+            st_h2(sm + L::kbar + o, ks0, ks1);
+            st_h2(ko + o, ks0 * aI[0], ks1 * aI[1]);
+#pragma unroll
+            for (int J = 0; J < 4; ++J)
+                if (J <= gI)
+                    st_h2(sm + L::qj + L::qj_region(J) + sw_off(t - 16 * J, 2 * lane), qp0 * cf[0][J],
+                          qp1 * cf[1][J]);
+        }
+    }
+    fence_proxy_async_cta();
+    named_sync(kBarA, kThreadsA);
+    if (tid == 0) {
+        mbar_arrive(bar(sm, B_STGE + b));   // the loader may refill this staging buffer
+        *misc_slow(sm, b) = slow ? 1 : 0;
+        mbar_arrive(bar(sm, B_GATE + b));   // operands ready: MMA 1 may be issued
+    }
+    if (tid == 64) {   // max |q| of the chunk (for the phase-4 bound); clear the maxima
+        const unsigned m = max(max(qmax[0], qmax[1]), max(qmax[2], qmax[3]));
+        if (ci < kMaxSpan) reinterpret_cast<float *>(sm + L::cmeta)[2 * ci] = __uint_as_float(m);
+        qmax[0] = qmax[1] = qmax[2] = qmax[3] = 0u;
+        *kmax = 0u;
+    }
+    return slow;
+}
+
+// MMA 1 of the chunk in buffer b (one thread): dS = K~^T V into TMEM dS buffer b,
+// scores = Qint K~^T (or the four sub-block products) into the scores columns.
+__device__ __forceinline__ void issue_mma1(uint32_t sbase, uint32_t tmem, int b, int vb, bool slow,
+                                           uint64_t *done) {
+    tc_fence_after();
+    const uint32_t kta = sbase + L::kt + b * kTile;
+    const uint32_t va = sbase + L::vop + vb * kTile;
+    constexpr uint32_t id_ds = idesc_f16_f32(64, kDV, true, true);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+        umma_f16(tmem + kColDS + 64 * b, desc_sw128(kta + kk * 2048, kTile, 1024),
+                 desc_sw128(va + kk * 2048, kTile, 1024), id_ds, kk > 0 ? 1u : 0u);
+    if (!slow) {
+        constexpr uint32_t id = idesc_f16_f32(64, 64, false, false);
+        const uint32_t qa = sbase + L::qint + b * kTile;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+            umma_f16(tmem + kColScores, desc_sw128(qa + kk * 32, 16, 1024),
+                     desc_sw128(kta + kk * 32, 16, 1024), id, kk > 0 ? 1u : 0u);
+    } else {
+        constexpr uint32_t id = idesc_f16_f32(64, 16, false, false);
+        for (int J = 0; J < 4; ++J) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                const uint32_t aa = sbase + L::qj + L::qj_region(J) - 16 * J * 128 + kk * 32;
+                const uint32_t bb = sbase + L::kbar + 16 * J * 128 + kk * 32;
+                umma_f16(tmem + kColScores + 16 * J, desc_sw128(aa, 16, 1024),
+                         desc_sw128(bb, 16, 1024), id, kk > 0 ? 1u : 0u);
+            }
+        }
+    }
+    umma_commit(done);
+}
+
+// Group B (warps 8-11), MMA 1 of a chunk complete: TMEM -> registers of the scores
+// (columns 64..127).  Warp q holds TMEM lanes 32q.. =
+// rows 16q .. 16q+15; thread rows 16q + lane/4 (+8), columns 2 (lane % 4) + 8 j (+1),
+// the second register set for columns 32 and up.
+struct BRegs {
+    uint32_t s0[16], s1[16];
+};
+
+__device__ __forceinline__ void load_tmem_b(uint32_t tmem, BRegs &r) {
+    const uint32_t ta = tmem + ((uint32_t)(32 * ((threadIdx.x >> 5) & 3)) << 16);
+    tc_fence_after();
+    tmem_ld_16x256b_x4(ta + kColScores, r.s0);
+    tmem_ld_16x256b_x4(ta + kColScores + 32, r.s1);
+    tmem_ld_wait();
+}
+
+// Scores -> causal fp16 P tile; with `fb` (this warp's sub-block uses the exact
+// diagonal) the diagonal block comes from diag[b].
+__device__ __forceinline__ void store_scores(uint8_t *sm, const BRegs &r, int b, bool fb) {
+    const int lane = threadIdx.x & 31, q = (threadIdx.x >> 5) & 3;
+    const float *diagx = reinterpret_cast<const float *>(sm + L::diag) + b * 1024;
+    uint8_t *pt = sm + L::p;
+    const int row0 = 16 * q + (lane >> 2), col0 = 2 * (lane & 3);
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const int row = row0 + 8 * hh;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const int col = col0 + 8 * cc + 32 * half;
+                const uint32_t *rr = half ? r.s1 : r.s0;
+                float x0 = __uint_as_float(rr[4 * cc + 2 * hh]);
+                float x1 = __uint_as_float(rr[4 * cc + 2 * hh + 1]);
+                if (fb && (col >> 4) == q) {
+                    x0 = diagx[(q * 16 + (row & 15)) * 16 + (col & 15)];
+                    x1 = diagx[(q * 16 + (row & 15)) * 16 + ((col + 1) & 15)];
+                }
+                x0 = col <= row ? x0 : 0.f;
+                x1 = col + 1 <= row ? x1 : 0.f;
+                st_h2(pt + sw_off(row, col), x0, x1);
+            }
+        }
+}
+
+// Group A (warps 0-7), MMA 1 of chunk cr complete: TMEM readout of dS(cr) and the
+// state update S <- d * S + dS (dS comes scaled by 1/d on the fast path) in the fp32
+// tile, d from dloc[b]; the new state also goes to `so_next` (fp16 S_prev operand of
+// chunk cr+1's MMA 2) and to `agg` (the span's published aggregate) when non-null.
+// Warp w reads TMEM lanes of quarter w % 4 (rows 16 (w % 4) ..) and columns
+// 32 (w / 4) ..: 16 elements per thread.  Ends with group A past its writes.
+__device__ __forceinline__ void update_state_a(uint8_t *sm, uint32_t tmem, int b, bool slow,
+                                               uint8_t *so_next, float *agg) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int sp = warp & 3, chalf = warp >> 2;
+    const int rrow0 = 16 * sp + (lane >> 2);
+    const int rcol0 = 32 * chalf + 2 * (lane & 3);
+    tc_fence_after();
+    uint32_t rd[16];
+    tmem_ld_16x256b_x4(tmem + ((uint32_t)(32 * sp) << 16) + kColDS + 64 * b + 32 * chalf, rd);
+    tmem_ld_wait();
+    const float *dloc = reinterpret_cast<const float *>(sm + L::dloc + b * 256);
+    uint8_t *sst = sm + L::sst;
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+        const int i = rrow0 + 8 * hh;
+        const float di = dloc[i];
+        const float scl = slow ? 1.f : di;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+            const int col = rcol0 + 8 * cc;
+            float2 *sp2 = reinterpret_cast<float2 *>(sst + agg_off(i, col >> 2) + (col & 3) * 4);
+            const float2 s = *sp2;
+            const float2 sn = make_float2(fmaf(di, s.x, scl * __uint_as_float(rd[4 * cc + 2 * hh])),
+                                          fmaf(di, s.y, scl * __uint_as_float(rd[4 * cc + 2 * hh + 1])));
+            *sp2 = sn;
+            if (so_next != nullptr) st_h2(so_next + sw_off(i, col), sn.x, sn.y);
+            if (agg != nullptr) *reinterpret_cast<float2 *>(agg + i * kDV + col) = sn;
+        }
+    }
+    tc_fence_before();
+    fence_proxy_async_cta();
+    named_sync(kBarA, kThreadsA);
+}
+
 __global__ void __launch_bounds__(kThreads, 1) gla_fwd_span_kernel(const Params P, const Work Wk) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>(
@@ -231,8 +608,6 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_span_kernel(const Params 
 
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar(sm, B_TMEM));
     float *dcum = reinterpret_cast<float *>(sm + L::dcum);
-    float *dloc = reinterpret_cast<float *>(sm + L::dloc);
-    float *dacc = reinterpret_cast<float *>(sm + L::dacc);
     float *cmeta = reinterpret_cast<float *>(sm + L::cmeta);
     int *rowb = reinterpret_cast<int *>(sm + L::rowb);
 
@@ -241,18 +616,21 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_span_kernel(const Params 
         tmem_relinquish();
     }
     if (tid == 0) {
-        mbar_init(bar(sm, B_STGF), 32);
-        mbar_init(bar(sm, B_STGE), 1);
-        mbar_init(bar(sm, B_MMA1), 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar(sm, B_STGF + i), 32);
+            mbar_init(bar(sm, B_STGE + i), 1);
+            mbar_init(bar(sm, B_OPSE + i), 1);
+        }
+        for (int i = 0; i < 2; ++i) mbar_init(bar(sm, B_MMA1 + i), 1);
+        mbar_init(bar(sm, B_SCON), 1);
         mbar_init(bar(sm, B_MMA2), 1);
-        mbar_init(bar(sm, B_OPSF), 1);
-        mbar_init(bar(sm, B_OPSF + 1), 1);
-        mbar_init(bar(sm, B_OPSE), 1);
-        mbar_init(bar(sm, B_OPSE + 1), 1);
         mbar_init(bar(sm, B_FIX), 1);
+        for (int i = 0; i < 2; ++i) mbar_init(bar(sm, B_GATE + i), 1);
+        for (int i = 0; i < 2; ++i) mbar_init(bar(sm, B_OPSF + i), 1);
+        for (int i = 0; i < 3; ++i) mbar_init(bar(sm, B_VE + i), 1);
         fence_mbar_init();
     }
-    if (tid < 24) reinterpret_cast<unsigned *>(sm + L::misc)[tid] = 0u;
+    if (tid < 32) reinterpret_cast<unsigned *>(sm + L::misc)[tid] = 0u;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -261,354 +639,108 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_span_kernel(const Params 
     // publish tag of this launch (the generation only changes after every CTA of
     // the previous launch has finished)
     const unsigned long long tag = PS > 1 ? __ldcg(Wk.hdr) + 1ull : 0ull;
-    // running barrier phase counters (kept identical in every role that waits on them)
-    uint32_t n_stg = 0, n_mma1 = 0, n_mma2 = 0;
-    uint32_t n_ops[2] = {0u, 0u}, n_fix = 0u;
+    // Barrier phase counters.  Each role counts only the barriers it waits on, and
+    // every role walks every chunk, so the counts stay consistent across sequences.
+    uint32_t nuse[2] = {0u, 0u};        // uses of buffer 0 / 1 (per role)
+    uint32_t nvuse[3] = {0u, 0u, 0u};   // loader: uses of V tile 0 / 1 / 2
+    uint32_t m1s[2] = {0u, 0u};         // MMA 1 phases observed, per parity
+    uint32_t sc_seen = 0;               // score-readout phases observed (loader lane 0)
+    uint32_t m2_seen = 0, g_seen = 0, n_fix = 0;
 
     for (int seq = grp; seq < P.n_seq; seq += ngrp) {
         const int c0 = kspan * Wk.Lc;
         const int nch = min(Wk.Lc, P.n_chunks - c0);   // >= 1 (host guarantees)
         const int hold = kspan > 0 ? min(kHold, nch) : 0;
         const bool later = kspan > 0;
-
-        // ---------------- phase 1 prologue: running state and decay product
+        float *agg = (PS > 1 && kspan < PS - 1) ? Wk.ws + ((size_t)seq * PS + kspan) * kAggFloats
+                                                : nullptr;
+        // ---------------- phase 1 prologue: running state and decay products
         {
-            float *sst = reinterpret_cast<float *>(sm + L::sst);
+            uint8_t *sst = sm + L::sst;
             for (int e = tid; e < kDK * kDV / 4; e += kThreads) {
                 const int i = e >> 4, c4 = e & 15;
                 float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (!later && P.s0 != nullptr)
                     v = reinterpret_cast<const float4 *>(P.s0 + (size_t)seq * kDK * kDV)[e];
-                *reinterpret_cast<float4 *>(reinterpret_cast<uint8_t *>(sst) + agg_off(i, c4)) = v;
+                *reinterpret_cast<float4 *>(sst + agg_off(i, c4)) = v;
+                // S_prev of chunk 0, the fp16 operand of its MMA 2
+                *reinterpret_cast<uint2 *>(sm + L::sop + sw_off(i, 4 * c4)) =
+                    make_uint2(pack_half2(v.x, v.y), pack_half2(v.z, v.w));
             }
-            if (tid < 64) dacc[tid] = 1.f;
+            if (tid < 64) dcum[tid] = 1.f;
             if (tid < kMaxSpan * 2) cmeta[tid] = 0.f;
         }
+        fence_proxy_async_cta();
         __syncthreads();
+        if (tid == 0) mbar_arrive(bar(sm, B_OPSF));   // S_prev of chunk 0 is ready
+        // phase indices at the start of the sequence: chunk c is use c/2 of parity c%2
+        const uint32_t m1b0 = m1s[0], m1b1 = m1s[1], sc_base = sc_seen;
 
         if (warp < 8) {
             // ================================================= group A
-            const int gI = warp >> 1, ghf = warp & 1, gt0 = 16 * gI + 8 * ghf, gh = 2 * gI + ghf;
-            const int sp = warp & 3, chalf = warp >> 2;
-            const int rrow0 = 16 * sp + (lane >> 2);
-            const int rcol0 = 32 * chalf + 2 * (lane & 3);
-            float *htot = reinterpret_cast<float *>(sm + L::htot);
-            float *diagx = reinterpret_cast<float *>(sm + L::diag);
-            const uint8_t *st = sm + L::stg;
-            for (int ci = 0; ci < nch; ++ci) {
-                const int b = ci & 1;
-                int *flags = reinterpret_cast<int *>(sm + L::misc + 48 * b);
-                unsigned *qmax = reinterpret_cast<unsigned *>(sm + L::misc + 48 * b + 16);
-                unsigned *kmax = reinterpret_cast<unsigned *>(sm + L::misc + 48 * b + 32);
-                const int nrows = min(kChunk, P.N - (c0 + ci) * kChunk);
-                const bool held = ci < hold;
-                uint8_t *qo = sm + L::qint + b * kTile;
-                // a held chunk also keeps Qint * D_c (D_c = decay since the span start)
-                uint8_t *qr = sm + L::ring + (held ? ci : 0) * kTile;
-                const float2 dc = *reinterpret_cast<const float2 *>(dacc + 2 * lane);
-                const bool pub = PS > 1 && kspan < PS - 1 && ci == nch - 1;
-                wait_l(bar(sm, B_STGF), n_stg & 1u, to);
-                ++n_stg;
-                wait_l(bar(sm, B_OPSE + b), (n_ops[b] & 1u) ^ 1u, to);
-                // ---------- pass 1
-                float pl[8][2], sl[8][2];
-                __half2 qh[8], kh[8];
-                __half2 qm2 = __float2half2_rn(0.f), km2 = __float2half2_rn(0.f);
-                {
-                    float a0[8], a1[8];
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const uint32_t o = (gt0 + u) * 128 + 4 * lane;
-                        const float2 gv = ld_h2(st + 2 * kTile + o);
-                        qh[u] = *reinterpret_cast<const __half2 *>(st + o);
-                        kh[u] = *reinterpret_cast<const __half2 *>(st + kTile + o);
-                        a0[u] = exp_f(gv.x);
-                        a1[u] = exp_f(gv.y);
-                        qm2 = __hmax2(qm2, __habs2(qh[u]));
-                        km2 = __hmax2(km2, __habs2(kh[u]));
-                    }
-                    float r0 = 1.f, r1 = 1.f;
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        r0 *= a0[u]; r1 *= a1[u];
-                        pl[u][0] = r0; pl[u][1] = r1;
-                    }
-                    r0 = 1.f; r1 = 1.f;
-#pragma unroll
-                    for (int u = 7; u >= 0; --u) {
-                        sl[u][0] = r0; sl[u][1] = r1;
-                        r0 *= a0[u]; r1 *= a1[u];
-                    }
-                    *reinterpret_cast<float2 *>(htot + gh * 64 + 2 * lane) = make_float2(pl[7][0], pl[7][1]);
+            // Iteration it: gating of chunk it (while MMA 1 of chunk it-1 runs; the
+            // loader warp issues MMA 1(it) once it is signalled), then the state update
+            // from dS(it-1), i.e. S_prev of chunk it.
+            bool slow_prev = false;
+            for (int it = 0; it <= nch; ++it) {
+                const int b = it & 1;
+                bool slow = false;
+                if (it < nch) {
+                    wait_l(bar(sm, B_STGF + b), nuse[b] & 1u, to);
+                    wait_l(bar(sm, B_OPSE + b), (nuse[b] & 1u) ^ 1u, to);
+                    ++nuse[b];
+                    const int nrows = min(kChunk, P.N - (c0 + it) * kChunk);
+                    slow = gate_chunk(P, sm, it, b, nrows, it < hold, m1s[b ^ 1],
+                                      (b ? m1b0 : m1b1) + ((it - 1) >> 1), to);
                 }
-                {
-                    const float qm = fmaxf(__low2float(qm2), __high2float(qm2));
-                    const float km = fmaxf(__low2float(km2), __high2float(km2));
-                    const unsigned wq = __reduce_max_sync(0xffffffffu, __float_as_uint(qm));
-                    const unsigned wk = __reduce_max_sync(0xffffffffu, __float_as_uint(km));
-                    if (lane == 0) {
-                        atomicMax(&qmax[gI], wq);
-                        atomicMax(kmax, wk);
-                    }
-                }
-                {
-                    uint8_t *vo = sm + L::vop + b * kTile;
-#pragma unroll
-                    for (int x = tid; x < 64 * 8; x += kThreadsA) {
-                        const int t = x >> 3, c8 = x & 7;
-                        *reinterpret_cast<uint4 *>(vo + sw_off(t, 8 * c8)) =
-                            *reinterpret_cast<const uint4 *>(st + 3 * kTile + t * 128 + 16 * c8);
-                    }
-                }
-                named_sync(kBarA, kThreadsA);
-                // ---------- chunk factors
-                float dch[2], bef[2], aft[2];
-                bool bad = __uint_as_float(*kmax) > kFastMaxK;
-                {
-                    float2 ht[8];
-#pragma unroll
-                    for (int h8 = 0; h8 < 8; ++h8)
-                        ht[h8] = *reinterpret_cast<const float2 *>(htot + h8 * 64 + 2 * lane);
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        float d = 1.f, bf = 1.f, af = 1.f;
-#pragma unroll
-                        for (int h8 = 0; h8 < 8; ++h8) {
-                            const float x = e ? ht[h8].y : ht[h8].x;
-                            d *= x;
-                            if (h8 < gh) bf *= x;
-                            if (h8 > gh) af *= x;
-                        }
-                        dch[e] = d; bef[e] = bf; aft[e] = af;
-                        bad |= !(d >= kFastMinDecay);
-                    }
-                }
-                const bool slow = named_sync_or(kBarA, kThreadsA, bad);
-                if (gh == 0) *reinterpret_cast<float2 *>(dloc + 2 * lane) = make_float2(dch[0], dch[1]);
-                if (!slow) {
-                    const float i0 = aft[0] / dch[0], i1 = aft[1] / dch[1];
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const uint32_t o = sw_off(gt0 + u, 2 * lane);
-                        const float2 qv = __half22float2(qh[u]);
-                        const float2 kv = __half22float2(kh[u]);
-                        const float a0 = qv.x * (pl[u][0] * bef[0]), a1 = qv.y * (pl[u][1] * bef[1]);
-                        st_h2(qo + o, a0, a1);
-                        if (held) st_h2(qr + o, a0 * dc.x, a1 * dc.y);
-                        st_h2(sm + L::kt + o, kv.x * (sl[u][0] * i0), kv.y * (sl[u][1] * i1));
-                    }
-                } else {
-                    float T[4][2];
-#pragma unroll
-                    for (int L4 = 0; L4 < 4; ++L4) {
-                        const float2 h0 = *reinterpret_cast<const float2 *>(htot + (2 * L4) * 64 + 2 * lane);
-                        const float2 h1 = *reinterpret_cast<const float2 *>(htot + (2 * L4 + 1) * 64 + 2 * lane);
-                        T[L4][0] = h0.x * h1.x;
-                        T[L4][1] = h0.y * h1.y;
-                    }
-                    bool dbad = false;
-#pragma unroll
-                    for (int L4 = 0; L4 < 4; ++L4)
-                        if (L4 == gI) dbad |= !(T[L4][0] >= kDiagMinTotal) || !(T[L4][1] >= kDiagMinTotal);
-                    dbad |= __uint_as_float(qmax[gI]) > kDiagMaxQ;
-                    if (__any_sync(0xffffffffu, dbad) && lane == 0) atomicOr(&flags[gI], 1);
-                    named_sync(kBarA, kThreadsA);
-                    const int anyflag = flags[0] | flags[1] | flags[2] | flags[3];
-                    if (anyflag) {
-                        for (int pr = tid; pr < 4 * 256; pr += kThreadsA) {
-                            const int I = pr >> 8, u = (pr >> 4) & 15, w = pr & 15;
-                            if (!flags[I] || w > u) continue;
-                            const int tu = I * kSub + u, tw = I * kSub + w;
-                            float acc = 0.f;
-                            if (tu < nrows) {
-                                for (int i = 0; i < kDK; ++i) {
-                                    float lg = 0.f;
-                                    for (int r2 = tw + 1; r2 <= tu; ++r2)
-                                        lg += __half2float(*reinterpret_cast<const __half *>(st + 2 * kTile + r2 * 128 + 2 * i));
-                                    const float qv = __half2float(*reinterpret_cast<const __half *>(st + tu * 128 + 2 * i));
-                                    const float kv = __half2float(*reinterpret_cast<const __half *>(st + kTile + tw * 128 + 2 * i));
-                                    acc += qv * kv * exp_f(lg);
-                                }
-                            }
-                            diagx[(I * 16 + u) * 16 + w] = acc;
-                        }
+                if (it > 0) {
+                    wait_phase(bar(sm, B_MMA1 + (b ^ 1)), m1s[b ^ 1], (b ? m1b0 : m1b1) + ((it - 1) >> 1), to);
+                    const bool pub = agg != nullptr && it == nch;
+                    update_state_a(sm, tmem, b ^ 1, slow_prev, it < nch ? sm + L::sop + b * kTile : nullptr,
+                                   pub ? agg : nullptr);
+                    if (pub) {
+                        // aggregate = (state reached from zero, product of the span's decays)
+                        if (tid < 64) agg[kDK * kDV + tid] = dcum[nch * 64 + tid];
+                        __threadfence();
                         named_sync(kBarA, kThreadsA);
+                        if (tid == 0) st_release_gpu(Wk.flags + (size_t)seq * PS + kspan, tag);
                     }
-                    const bool diag_bad = flags[gI] != 0;
-                    float cf[2][4], bI[2], aI[2], hin[2], hout[2];
-                    const float2 h0 = *reinterpret_cast<const float2 *>(htot + (2 * gI) * 64 + 2 * lane);
-                    const float2 h1 = *reinterpret_cast<const float2 *>(htot + (2 * gI + 1) * 64 + 2 * lane);
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        float b0 = 1.f, a0 = 1.f, tI = 1.f;
-#pragma unroll
-                        for (int L4 = 0; L4 < 4; ++L4) {
-                            if (L4 < gI) b0 *= T[L4][e];
-                            if (L4 > gI) a0 *= T[L4][e];
-                            if (L4 == gI) tI = T[L4][e];
-                        }
-                        bI[e] = b0; aI[e] = a0;
-#pragma unroll
-                        for (int J = 0; J < 4; ++J) {
-                            float cj = 1.f;
-#pragma unroll
-                            for (int L4 = 0; L4 < 4; ++L4)
-                                if (L4 > J && L4 < gI) cj *= T[L4][e];
-                            cf[e][J] = (J == gI) ? (diag_bad ? 0.f : 1.f / tI) : cj;
-                        }
-                        hin[e] = ghf ? (e ? h0.y : h0.x) : 1.f;
-                        hout[e] = ghf ? 1.f : (e ? h1.y : h1.x);
-                    }
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const int t = gt0 + u;
-                        const uint32_t o = sw_off(t, 2 * lane);
-                        const float2 qv = __half22float2(qh[u]);
-                        const float2 kv = __half22float2(kh[u]);
-                        const float qp0 = qv.x * (pl[u][0] * hin[0]);
-                        const float qp1 = qv.y * (pl[u][1] * hin[1]);
-                        const float ks0 = kv.x * (sl[u][0] * hout[0]);
-                        const float ks1 = kv.y * (sl[u][1] * hout[1]);
-                        st_h2(qo + o, qp0 * bI[0], qp1 * bI[1]);
-                        if (held) st_h2(qr + o, qp0 * bI[0] * dc.x, qp1 * bI[1] * dc.y);
-                        st_h2(sm + L::kbar + o, ks0, ks1);
-                        st_h2(sm + L::kt + o, ks0 * aI[0], ks1 * aI[1]);
-#pragma unroll
-                        for (int J = 0; J < 4; ++J)
-                            if (J <= gI)
-                                st_h2(sm + L::qj + L::qj_region(J) + sw_off(t - 16 * J, 2 * lane),
-                                      qp0 * cf[0][J], qp1 * cf[1][J]);
-                    }
+                    if (tid == 0 && it < nch) mbar_arrive(bar(sm, B_OPSF + b));   // S_prev of chunk it
                 }
-                fence_proxy_async_cta();
-                named_sync(kBarA, kThreadsA);
-                if (tid == 0) mbar_arrive(bar(sm, B_STGE));   // the loader may refill staging
-                // ---------- MMA 1
-                if (tid == 0) {
-                    tc_fence_after();
-                    const uint32_t kta = sbase + L::kt;
-                    const uint32_t va = sbase + L::vop + b * kTile;
-                    constexpr uint32_t id_ds = idesc_f16_f32(64, kDV, true, true);
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        umma_f16(tmem + kColMma1, desc_sw128(kta + kk * 2048, kTile, 1024),
-                                 desc_sw128(va + kk * 2048, kTile, 1024), id_ds, kk > 0 ? 1u : 0u);
-                    if (!slow) {
-                        constexpr uint32_t id = idesc_f16_f32(64, 64, false, false);
-                        const uint32_t qa = smem_u32(qo);
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            umma_f16(tmem + kColMma1 + 64, desc_sw128(qa + kk * 32, 16, 1024),
-                                     desc_sw128(kta + kk * 32, 16, 1024), id, kk > 0 ? 1u : 0u);
-                    } else {
-                        constexpr uint32_t id = idesc_f16_f32(64, 16, false, false);
-                        for (int J = 0; J < 4; ++J) {
-#pragma unroll
-                            for (int kk = 0; kk < 4; ++kk) {
-                                const uint32_t aa = sbase + L::qj + L::qj_region(J) - 16 * J * 128 + kk * 32;
-                                const uint32_t bb = sbase + L::kbar + 16 * J * 128 + kk * 32;
-                                umma_f16(tmem + kColMma1 + 64 + 16 * J, desc_sw128(aa, 16, 1024),
-                                         desc_sw128(bb, 16, 1024), id, kk > 0 ? 1u : 0u);
-                            }
-                        }
-                    }
-                    umma_commit(bar(sm, B_MMA1));
-                }
-                wait_l(bar(sm, B_MMA1), n_mma1 & 1u, to);
-                ++n_mma1;
-                tc_fence_after();
-                uint32_t rs[16], rd[16];
-                tmem_ld_16x256b_x4(tmem + ((uint32_t)(32 * sp) << 16) + kColMma1 + 64 + 32 * chalf, rs);
-                tmem_ld_16x256b_x4(tmem + ((uint32_t)(32 * sp) << 16) + kColMma1 + 32 * chalf, rd);
-                tmem_ld_wait();
-                {
-                    // masked scores -> P
-                    uint8_t *pt = sm + L::p + b * kTile;
-                    const bool fb = slow && (flags[sp] != 0);
-#pragma unroll
-                    for (int cc = 0; cc < 4; ++cc) {
-#pragma unroll
-                        for (int hh = 0; hh < 2; ++hh) {
-                            const int row = rrow0 + 8 * hh;
-                            const int col = rcol0 + 8 * cc;
-                            float x0 = __uint_as_float(rs[4 * cc + 2 * hh]);
-                            float x1 = __uint_as_float(rs[4 * cc + 2 * hh + 1]);
-                            if (fb && (col >> 4) == sp) {
-                                x0 = diagx[(sp * 16 + (row & 15)) * 16 + (col & 15)];
-                                x1 = diagx[(sp * 16 + (row & 15)) * 16 + ((col + 1) & 15)];
-                            }
-                            x0 = col <= row ? x0 : 0.f;
-                            x1 = col + 1 <= row ? x1 : 0.f;
-                            st_h2(pt + sw_off(row, col), x0, x1);
-                        }
-                    }
-                }
-                {
-                    // state: S_prev (fp16 operand) <- S; S <- d * S + dS
-                    uint8_t *sst = sm + L::sst;
-                    uint8_t *so = sm + L::sop + b * kTile;
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        const int i = rrow0 + 8 * hh;
-                        const float di = dloc[i];
-                        const float scl = slow ? 1.f : di;
-#pragma unroll
-                        for (int cc = 0; cc < 4; ++cc) {
-                            const int col = rcol0 + 8 * cc;
-                            float2 *sp2 = reinterpret_cast<float2 *>(sst + agg_off(i, col >> 2) + (col & 3) * 4);
-                            const float2 s = *sp2;
-                            st_h2(so + sw_off(i, col), s.x, s.y);
-                            const float2 sn = make_float2(fmaf(di, s.x, scl * __uint_as_float(rd[4 * cc + 2 * hh])),
-                                                          fmaf(di, s.y, scl * __uint_as_float(rd[4 * cc + 2 * hh + 1])));
-                            *sp2 = sn;
-                            // the span's last chunk publishes its state straight from here
-                            if (pub)
-                                *reinterpret_cast<float2 *>(Wk.ws + ((size_t)seq * PS + kspan) * kAggFloats +
-                                                            i * kDV + col) = sn;
-                        }
-                    }
-                }
-                tc_fence_before();
-                fence_proxy_async_cta();
-                named_sync(kBarA, kThreadsA);
-                if (tid < 64) {
-                    if (ci < kMaxSpan) dcum[ci * 64 + tid] = dacc[tid];
-                    dacc[tid] *= dloc[tid];
-                }
-                if (tid == 64) {
-                    const unsigned m = max(max(qmax[0], qmax[1]), max(qmax[2], qmax[3]));
-                    if (ci < kMaxSpan) cmeta[2 * ci] = __uint_as_float(m);
-                }
-                if (pub) {
-                    // aggregate = (state reached from zero, product of the span's decays)
-                    if (tid < 64) Wk.ws[((size_t)seq * PS + kspan) * kAggFloats + kDK * kDV + tid] = dacc[tid];
-                    __threadfence();
-                    named_sync(kBarA, kThreadsA);
-                    if (tid == 0) st_release_gpu(Wk.flags + (size_t)seq * PS + kspan, tag);
-                }
-                if (tid == 0) mbar_arrive(bar(sm, B_OPSF + b));
-                named_sync(kBarA, kThreadsA);
-                if (tid < 4) { flags[tid] = 0; qmax[tid] = 0u; }
-                if (tid == 0) *kmax = 0u;
-                ++n_ops[b];
+                slow_prev = slow;
             }
         } else if (warp < 12) {
             // ================================================= group B
             const int tb = tid - kThreadsA, bw = warp - 8;
             int *rows2 = rowb + 2 * 64;
-            for (int ci = 0; ci < nch; ++ci) {
-                const int b = ci & 1;
-                const bool held = ci < hold;
-                fill_rows(P, seq, c0 + ci, rows2, tb);
-                wait_l(bar(sm, B_OPSF + b), n_ops[b] & 1u, to);
-                const uint32_t dcol = held ? kColHold + 64 * ci : kColWork;
+            for (int c = 0; c < nch; ++c) {
+                const int b = c & 1;
+                const bool held = c < hold;
+                fill_rows(P, seq, c0 + c, rows2, tb);
+                wait_l(bar(sm, B_GATE + b), (g_seen >> b) & 1u, to);   // bit b: parity of GATE[b]
+                g_seen ^= 1u << b;
+                wait_phase(bar(sm, B_MMA1 + b), m1s[b], (b ? m1b1 : m1b0) + (c >> 1), to);
+                BRegs r;
+                load_tmem_b(tmem, r);
+                const bool fb = misc_flags(sm, b)[warp & 3] != 0;
+                tc_fence_before();
+                named_sync(kBarB, kThreadsB);
+                if (tb == 0) mbar_arrive(bar(sm, B_SCON));   // TMEM columns 0..127 free for MMA 1
+                store_scores(sm, r, b, fb);
+                fence_proxy_async_cta();
+                named_sync(kBarB, kThreadsB);
                 if (tb == 0) {
+                    // only the issuing thread waits for S_prev of chunk c (a lagging
+                    // waiter could miss a phase: the next one follows MMA 2 of chunk c)
+                    wait_l(bar(sm, B_OPSF + b), nuse[b] & 1u, to);
+                    ++nuse[b];
                     tc_fence_after();
+                    const uint32_t dcol = held ? kColHold + 64 * c : kColWork;
                     constexpr uint32_t id = idesc_f16_f32(64, kDV, false, true);
                     const uint32_t qa = sbase + L::qint + b * kTile;
                     const uint32_t sa = sbase + L::sop + b * kTile;
-                    const uint32_t pa = sbase + L::p + b * kTile;
-                    const uint32_t va = sbase + L::vop + b * kTile;
+                    const uint32_t pa = sbase + L::p;
+                    const uint32_t va = sbase + L::vop + (c % 3) * kTile;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         umma_f16(tmem + dcol, desc_sw128(qa + kk * 32, 16, 1024),
@@ -618,43 +750,55 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_span_kernel(const Params 
                         umma_f16(tmem + dcol, desc_sw128(pa + kk * 32, 16, 1024),
                                  desc_sw128(va + kk * 2048, kTile, 1024), id, 1u);
                     umma_commit(bar(sm, B_MMA2));
+                    umma_commit(bar(sm, B_OPSE + b));    // Qint, S_prev tiles free
+                    umma_commit(bar(sm, B_VE + c % 3));  // V tile free
                 }
-                wait_l(bar(sm, B_MMA2), n_mma2 & 1u, to);
-                ++n_mma2;
+                wait_l(bar(sm, B_MMA2), m2_seen & 1u, to);
+                ++m2_seen;
                 tc_fence_after();
-                if (tb == 0) mbar_arrive(bar(sm, B_OPSE + b));
-                ++n_ops[b];
-                named_sync(kBarB, kThreadsB);   // row table visible to every group-B thread
                 if (!held) {
+                    // the P tile is free again: it stages the outputs
                     const float mx = store_chunk_out(P, tmem, kColWork, bw, lane, tb, nullptr, kBarB,
-                                                     sm + L::ost, rows2);
-                    if (later && ci < kMaxSpan) {
+                                                     sm + L::p, rows2);
+                    if (later && c < kMaxSpan) {
                         const unsigned w = __reduce_max_sync(0xffffffffu, __float_as_uint(mx));
-                        if (lane == 0) atomicMax(reinterpret_cast<unsigned *>(cmeta + 2 * ci + 1), w);
+                        if (lane == 0) atomicMax(reinterpret_cast<unsigned *>(cmeta + 2 * c + 1), w);
                     }
                 }
             }
         } else {
             // ================================================= loader (warp 12)
-            for (int ci = 0; ci < nch; ++ci) {
-                wait_l(bar(sm, B_STGE), (n_stg & 1u) ^ 1u, to);
-                load_chunk(P, sm, seq, c0 + ci, lane);
-                cp_async_mbar_arrive_noinc(bar(sm, B_STGF));
-                ++n_stg;
+            // Loads run two chunks ahead; lane 0 also issues MMA 1 of each chunk once
+            // group A has gated it and group B has read the previous chunk's scores.
+            auto load = [&](int c) {
+                const int b = c & 1, vb = c % 3;
+                wait_l(bar(sm, B_STGE + b), (nuse[b] & 1u) ^ 1u, to);
+                wait_l(bar(sm, B_VE + vb), (nvuse[vb] & 1u) ^ 1u, to);
+                ++nuse[b];
+                ++nvuse[vb];
+                load_chunk(P, sm, seq, c0 + c, b, vb, lane);
+                cp_async_mbar_arrive_noinc(bar(sm, B_STGF + b));
+            };
+            load(0);
+            if (nch > 1) load(1);
+            for (int c = 0; c < nch; ++c) {
+                const int b = c & 1;
+                if (lane == 0) {
+                    // GATE[b] next completes for chunk c+2, whose staging is only loaded
+                    // after this wait, so no phase can be missed
+                    wait_l(bar(sm, B_GATE + b), (g_seen >> b) & 1u, to);
+                    g_seen ^= 1u << b;
+                    if (c > 0) wait_phase(bar(sm, B_SCON), sc_seen, sc_base + c - 1, to);
+                    fence_proxy_async_cta();
+                    issue_mma1(sbase, tmem, b, c % 3, *misc_slow(sm, b) != 0, bar(sm, B_MMA1 + b));
+                }
+                __syncwarp();
+                if (c + 2 < nch) load(c + 2);
             }
-            cp_async_wait_all();
+            if (lane == 0) wait_phase(bar(sm, B_SCON), sc_seen, sc_base + nch - 1, to);
+            __syncwarp();
         }
         __syncthreads();
-        // Each role advanced only the barrier counters it waits on (A: staging, MMA 1,
-        // operands; B: operands, MMA 2; loader: staging); bring the others level.
-        if (warp >= 8) n_mma1 += (uint32_t)nch;
-        if (warp < 8 || warp >= 12) n_mma2 += (uint32_t)nch;
-        if (warp >= 8 && warp < 12) n_stg += (uint32_t)nch;
-        if (warp >= 12) {
-            n_ops[0] += (uint32_t)((nch + 1) / 2);
-            n_ops[1] += (uint32_t)(nch / 2);
-        }
-
         // ---------------- phase 3: look back over the earlier spans
         if (later) {
             if (tid < kspan) {
@@ -761,7 +905,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_span_kernel(const Params 
                 if (warp < 12) {
                     const int team = warp >> 2, tb = tid - 128 * team, bw = warp & 3;
                     int *rows = rowb + 64 * team;
-                    uint8_t *os = team < 2 ? sm + L::stg + team * kTile : sm + L::ost;
+                    uint8_t *os = sm + L::stg + team * kTile;
                     for (int ci = team; ci < hold; ci += 3) {
                         fill_rows(P, seq, c0 + ci, rows, tb);
                         named_sync(3 + team, 128);
@@ -855,7 +999,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_span_kernel(const Params 
                     fill_rows(P, seq, c0 + ci, rowb + 128, tb);
                     named_sync(kBarB, kThreadsB);
                     store_chunk_out(P, tmem, kColWork, bw, lane, tb, sm + L::stg + 3 * kTile, kBarB,
-                                    sm + L::ost, rowb + 128);
+                                    sm + L::stg + 4 * kTile, rowb + 128);
                 }
                 __syncthreads();
             }
@@ -869,7 +1013,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_span_kernel(const Params 
                 const int i = e >> 4, c4 = e & 15;
                 float4 s = *reinterpret_cast<const float4 *>(reinterpret_cast<const uint8_t *>(sst) + agg_off(i, c4));
                 if (later) {
-                    const float di = dacc[i];
+                    const float di = dcum[nch * 64 + i];
                     const float4 a = *reinterpret_cast<const float4 *>(reinterpret_cast<const uint8_t *>(sin) + agg_off(i, c4));
                     s.x = fmaf(di, a.x, s.x);
                     s.y = fmaf(di, a.y, s.y);
