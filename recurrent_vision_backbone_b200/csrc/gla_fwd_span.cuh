@@ -92,7 +92,7 @@ enum {
     B_STGF = 0,   // [2] staging (+ V tile) landed: 32 loader arrivals
     B_STGE = 2,   // [2] group A done with the staging buffer
     B_MMA1 = 19,  // [2] MMA 1 of a chunk of this parity complete (waited by groups A and B)
-    B_SCON = 5,   // group B has read the scores out of TMEM
+    B_SCON = 5,   // MMA 2 has consumed P, held in the scores' TMEM columns (tcgen05.commit)
     B_OPSF = 6,   // [2] S_prev of a chunk ready for its MMA 2
     B_OPSE = 8,   // [2] MMA 2 done with Qint, S_prev of a buffer (tcgen05.commit)
     B_MMA2 = 10,
@@ -360,16 +360,17 @@ __device__ __forceinline__ bool gate_chunk(const Params &P, uint8_t *sm, int ci,
     }
     if (!slow) {
         // ---------- fast path: Qint = q P, K~ = k / P (= k * suffix / d)
+        // The factors (P in [e^-6, 1], suffix / d in [1, e^6]) are rounded to fp16 and
+        // applied with packed fp16 multiplies.
         const float i0 = aft[0] / dch[0], i1 = aft[1] / dch[1];
+        const __half2 dch2 = __floats2half2_rn(dc.x, dc.y);
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
             const uint32_t o = sw_off(gt0 + u, 2 * lane);
-            const float2 qv = __half22float2(qh[u]);
-            const float2 kv = __half22float2(kh[u]);
-            const float a0 = qv.x * (pl[u][0] * bef[0]), a1 = qv.y * (pl[u][1] * bef[1]);
-            st_h2(qo + o, a0, a1);
-            if (held) st_h2(qr + o, a0 * dc.x, a1 * dc.y);
-            st_h2(ko + o, kv.x * (sl[u][0] * i0), kv.y * (sl[u][1] * i1));
+            const __half2 qi = __hmul2(qh[u], __floats2half2_rn(pl[u][0] * bef[0], pl[u][1] * bef[1]));
+            *reinterpret_cast<__half2 *>(qo + o) = qi;
+            if (held) *reinterpret_cast<__half2 *>(qr + o) = __hmul2(qi, dch2);
+            *reinterpret_cast<__half2 *>(ko + o) = __hmul2(kh[u], __floats2half2_rn(sl[u][0] * i0, sl[u][1] * i1));
         }
     } else {
         // ---------- sub-block path: 16-token sub-blocks, factors <= 1 off the diagonal
@@ -527,20 +528,23 @@ __device__ __forceinline__ void load_tmem_b(uint32_t tmem, BRegs &r) {
     tmem_ld_wait();
 }
 
-// Scores -> causal fp16 P tile; with `fb` (this warp's sub-block uses the exact
-// diagonal) the diagonal block comes from diag[b].
-__device__ __forceinline__ void store_scores(uint8_t *sm, const BRegs &r, int b, bool fb) {
+// Scores -> causal fp16 P, written back over the scores' own TMEM columns as the A
+// operand of MMA 2 (M=64 lane layout, fp16 pairs packed per 32-bit column: the
+// thread's pair (row, columns 2k, 2k+1) is packed column k).  With `fb` (this warp's
+// sub-block uses the exact diagonal) the diagonal block comes from diag[b].
+__device__ __forceinline__ void store_p_tmem(uint8_t *sm, uint32_t tmem, const BRegs &r, int b,
+                                             bool fb) {
     const int lane = threadIdx.x & 31, q = (threadIdx.x >> 5) & 3;
     const float *diagx = reinterpret_cast<const float *>(sm + L::diag) + b * 1024;
-    uint8_t *pt = sm + L::p;
     const int row0 = 16 * q + (lane >> 2), col0 = 2 * (lane & 3);
+    uint32_t v[16];
 #pragma unroll
-    for (int cc = 0; cc < 4; ++cc)
+    for (int half = 0; half < 2; ++half)
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            const int row = row0 + 8 * hh;
+        for (int cc = 0; cc < 4; ++cc)
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
+            for (int hh = 0; hh < 2; ++hh) {
+                const int row = row0 + 8 * hh;
                 const int col = col0 + 8 * cc + 32 * half;
                 const uint32_t *rr = half ? r.s1 : r.s0;
                 float x0 = __uint_as_float(rr[4 * cc + 2 * hh]);
@@ -551,9 +555,15 @@ __device__ __forceinline__ void store_scores(uint8_t *sm, const BRegs &r, int b,
                 }
                 x0 = col <= row ? x0 : 0.f;
                 x1 = col + 1 <= row ? x1 : 0.f;
-                st_h2(pt + sw_off(row, col), x0, x1);
+                v[2 * (cc + 4 * half) + hh] = pack_half2(x0, x1);   // packed column 4 j + lane % 4
             }
-        }
+    asm volatile(
+        "tcgen05.st.sync.aligned.16x128b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            tmem + ((uint32_t)(32 * q) << 16) + kColScores),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+        "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+        : "memory");
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 // Group A (warps 0-7), MMA 1 of chunk cr complete: TMEM readout of dS(cr) and the
@@ -594,6 +604,21 @@ __device__ __forceinline__ void update_state_a(uint8_t *sm, uint32_t tmem, int b
     tc_fence_before();
     fence_proxy_async_cta();
     named_sync(kBarA, kThreadsA);
+}
+
+// Loader warp: chunk c of the span into staging buffer c % 2 and V tile c % 3 once
+// group A is done with the staging buffer (chunk c-2) and MMA 2 with the V tile
+// (chunk c-3).
+__device__ __forceinline__ void loader_load(const Params &P, uint8_t *sm, int seq, int c0, int c,
+                                            int lane, uint32_t (&nuse)[2], uint32_t (&nvuse)[3],
+                                            bool &to) {
+    const int b = c & 1, vb = c % 3;
+    wait_l(bar(sm, B_STGE + b), (nuse[b] & 1u) ^ 1u, to);
+    wait_l(bar(sm, B_VE + vb), (nvuse[vb] & 1u) ^ 1u, to);
+    ++nuse[b];
+    ++nvuse[vb];
+    load_chunk(P, sm, seq, c0 + c, b, vb, lane);
+    cp_async_mbar_arrive_noinc(bar(sm, B_STGF + b));
 }
 
 __global__ void __launch_bounds__(kThreads, 1) gla_fwd_span_kernel(const Params P, const Work Wk) {
@@ -722,12 +747,8 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_span_kernel(const Params 
                 wait_phase(bar(sm, B_MMA1 + b), m1s[b], (b ? m1b1 : m1b0) + (c >> 1), to);
                 BRegs r;
                 load_tmem_b(tmem, r);
-                const bool fb = misc_flags(sm, b)[warp & 3] != 0;
+                store_p_tmem(sm, tmem, r, b, misc_flags(sm, b)[warp & 3] != 0);
                 tc_fence_before();
-                named_sync(kBarB, kThreadsB);
-                if (tb == 0) mbar_arrive(bar(sm, B_SCON));   // TMEM columns 0..127 free for MMA 1
-                store_scores(sm, r, b, fb);
-                fence_proxy_async_cta();
                 named_sync(kBarB, kThreadsB);
                 if (tb == 0) {
                     // only the issuing thread waits for S_prev of chunk c (a lagging
@@ -739,19 +760,19 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_span_kernel(const Params 
                     constexpr uint32_t id = idesc_f16_f32(64, kDV, false, true);
                     const uint32_t qa = sbase + L::qint + b * kTile;
                     const uint32_t sa = sbase + L::sop + b * kTile;
-                    const uint32_t pa = sbase + L::p;
                     const uint32_t va = sbase + L::vop + (c % 3) * kTile;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         umma_f16(tmem + dcol, desc_sw128(qa + kk * 32, 16, 1024),
                                  desc_sw128(sa + kk * 2048, kTile, 1024), id, kk > 0 ? 1u : 0u);
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        umma_f16(tmem + dcol, desc_sw128(pa + kk * 32, 16, 1024),
-                                 desc_sw128(va + kk * 2048, kTile, 1024), id, 1u);
+                    for (int kk = 0; kk < 4; ++kk)   // P from TMEM: K step 16 = 8 packed columns
+                        umma_f16_ta(tmem + dcol, tmem + kColScores + 8 * kk,
+                                    desc_sw128(va + kk * 2048, kTile, 1024), id, 1u);
                     umma_commit(bar(sm, B_MMA2));
                     umma_commit(bar(sm, B_OPSE + b));    // Qint, S_prev tiles free
                     umma_commit(bar(sm, B_VE + c % 3));  // V tile free
+                    umma_commit(bar(sm, B_SCON));        // scores / P columns free for MMA 1
                 }
                 wait_l(bar(sm, B_MMA2), m2_seen & 1u, to);
                 ++m2_seen;
@@ -770,17 +791,8 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_span_kernel(const Params 
             // ================================================= loader (warp 12)
             // Loads run two chunks ahead; lane 0 also issues MMA 1 of each chunk once
             // group A has gated it and group B has read the previous chunk's scores.
-            auto load = [&](int c) {
-                const int b = c & 1, vb = c % 3;
-                wait_l(bar(sm, B_STGE + b), (nuse[b] & 1u) ^ 1u, to);
-                wait_l(bar(sm, B_VE + vb), (nvuse[vb] & 1u) ^ 1u, to);
-                ++nuse[b];
-                ++nvuse[vb];
-                load_chunk(P, sm, seq, c0 + c, b, vb, lane);
-                cp_async_mbar_arrive_noinc(bar(sm, B_STGF + b));
-            };
-            load(0);
-            if (nch > 1) load(1);
+            loader_load(P, sm, seq, c0, 0, lane, nuse, nvuse, to);
+            if (nch > 1) loader_load(P, sm, seq, c0, 1, lane, nuse, nvuse, to);
             for (int c = 0; c < nch; ++c) {
                 const int b = c & 1;
                 if (lane == 0) {
@@ -793,7 +805,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_span_kernel(const Params 
                     issue_mma1(sbase, tmem, b, c % 3, *misc_slow(sm, b) != 0, bar(sm, B_MMA1 + b));
                 }
                 __syncwarp();
-                if (c + 2 < nch) load(c + 2);
+                if (c + 2 < nch) loader_load(P, sm, seq, c0, c + 2, lane, nuse, nvuse, to);
             }
             if (lane == 0) wait_phase(bar(sm, B_SCON), sc_seen, sc_base + nch - 1, to);
             __syncwarp();
