@@ -103,9 +103,13 @@ size_t gtr_gla_workspace_bytes(int B, int heads, int Hgrid, int Wgrid, int dk, i
  * gtr_gla_fwd with a caller-owned workspace: same arguments and results, plus
  *   workspace        device memory, 256-byte aligned, at least
  *                    gtr_gla_workspace_bytes(...) bytes (may be NULL when that is 0).
- *                    It must be zero-filled before its first use; every call that
- *                    completes without a device error leaves it zero-filled again.
- *                    After GTR_ERR_TIMEOUT the caller zero-fills it again.
+ *                    It must be zero-filled before its first use.  Its first
+ *                    part (the spans' publish flags, 2 x 4 bytes per SM of the
+ *                    device, rounded up to 256) must be zero when a call starts:
+ *                    every call that completes without a device error leaves it
+ *                    zero again; the rest holds the spans' aggregates, which any
+ *                    call overwrites before reading.  After GTR_ERR_TIMEOUT the
+ *                    caller zero-fills the workspace again.
  *   workspace_bytes  its size.
  * Calls that share a workspace must not overlap in time (same stream is fine).
  * A missing, short or misaligned workspace returns GTR_ERR_INVALID_ARG.
@@ -130,8 +134,9 @@ gtr_status_t gtr_gla_fwd_ws(const gtr_half_t *q, const gtr_half_t *k, const gtr_
  * allocating call.
  *   - Set-up: the first call on a device that needs the scratch looks up its
  *     device address (cudaGetSymbolAddress) with that device current and
- *     zero-fills its header and publish flags (the part that must start at zero;
- *     the kernel keeps it consistent from then on), synchronising the host once.
+ *     zero-fills its publish flags (the part that must be zero when a call
+ *     starts; every call that completes without a device error leaves them
+ *     zero again), synchronising the host once.
  *     Make that first call before any stream capture begins.
  *   - Limit: a shape whose plan needs more than GTR_STATIC_WS_BYTES returns
  *     GTR_ERR_UNSUPPORTED with nothing launched.
@@ -148,8 +153,8 @@ gtr_status_t gtr_gla_fwd_static(const gtr_half_t *q, const gtr_half_t *k, const 
 /*
  * Syncs `stream`, then reads and clears the device error word (and any sticky
  * CUDA error).  Returns GTR_OK, GTR_ERR_TIMEOUT or GTR_ERR_CUDA.  On
- * GTR_ERR_TIMEOUT it also zero-fills the library's cached workspace of the
- * current device.
+ * GTR_ERR_TIMEOUT it also zero-fills the library's workspaces of the current
+ * device (the cached one and the static scratch).
  */
 gtr_status_t gtr_gla_device_status(void *stream);
 

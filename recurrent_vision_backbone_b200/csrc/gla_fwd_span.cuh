@@ -8,19 +8,20 @@
 // is purely local, so no per-chunk traffic crosses CTAs:
 //
 //   phase 1  stream the span's chunks from a zero state (span 0: from S0), as a
-//            three-role pipeline over two buffers:
+//            pipeline over two operand buffers:
 //              loader (warp 12)   cp.async of q, k, g rows into staging and of v
-//                                 straight into its swizzled operand tile;
-//              group A (warps 0-7) gating of chunk c (Qint = q P, K~ = k / P, ...)
-//                                 while MMA 1 of chunk c-1 runs, then MMA 1(c) =
-//                                 (dS, scores) once group B has read chunk c-1;
-//              group B (warps 8-11) TMEM readout of chunk c: scores into the causal
-//                                 P tile, MMA 2(c) = Qint S_prev + P V, and while it
-//                                 runs S <- d * S + dS in shared memory (its fp16
-//                                 copy is S_prev of chunk c+1); output stores.
-//   phase 2  the span's last readout publishes its aggregate (state reached from
-//            zero, product of the decays) to the workspace; span 0 publishes its
-//            inclusive state.
+//                                 straight into its swizzled operand tile, two
+//                                 chunks ahead; lane 0 issues MMA 1(c) = (dS,
+//                                 scores) once chunk c is gated and MMA 2(c-1) has
+//                                 consumed the scores' TMEM columns;
+//              group A (warps 0-7) gating of chunk c (Qint = q P, K~ = k / P, ...),
+//                                 then S <- d * S + dS of chunk c-1 from TMEM (its
+//                                 fp16 copy is S_prev of chunk c);
+//              group B (warps 8-11) scores of chunk c from TMEM into the causal fp16
+//                                 P tile, written back to TMEM, MMA 2(c) = Qint S_prev
+//                                 + P V (P as the TMEM A operand), output stores;
+//   phase 2  the span's last state update publishes its aggregate (state reached
+//            from zero, product of the decays) to the workspace.
 //   phase 3  look back: fold the aggregates of the earlier spans into S_in, the true
 //            state entering this span.
 //   phase 4  correct the outputs for the missing S_in term.  For a chunk c starting
@@ -46,6 +47,7 @@ constexpr int kDK = 64;
 constexpr int kHold = 4;                    // chunks per span whose outputs wait in TMEM
 constexpr int kMaxSpan = 32;                // chunks of a span with recorded decays
 constexpr uint32_t kBarA = 1, kBarB = 2;    // named barriers; 3..5: phase-4 epilogue teams
+constexpr uint32_t kBarPro = 6;             // groups A and B: sequence prologue
 constexpr int kAggFloats = kDK * kDV + kDK; // state + decay product
 // TMEM columns: dS of MMA 1 (two buffers), scores of MMA 1, MMA 2 work block, the
 // held chunks' output blocks
@@ -102,18 +104,17 @@ enum {
     B_GATE = 17   // [2] group A's gating of a chunk done (operands, flags, diagonal blocks)
 };
 
-// Workspace protocol.  hdr[0] counts completed launches (the generation), hdr[1]
-// counts CTAs that finished the current launch.  A span publishes its aggregate
-// by storing tag = generation + 1 into its flag; readers wait for exactly that
-// tag, so flags never need clearing and stale tags of earlier launches are
-// never mistaken for fresh ones.  The last CTA of a launch advances the
-// generation.  The header and flags sit at fixed offsets whatever the shape.
+// Workspace protocol.  Every flag is zero when a launch starts.  Span k of a
+// sequence publishes its aggregate by storing (release) the number of its readers,
+// P - 1 - k, into its flag; each later span waits (acquire) for a non-zero flag and
+// then takes one off it (a reduction, nothing waits on it).  The last reader
+// leaves the flag at zero, so the workspace is clean again when the launch ends and
+// any shape may use it next.  The flags sit at a fixed offset whatever the shape.
 struct Work {
     int P;        // spans per sequence
     int Lc;       // chunks per span (the last span may be shorter)
     float *ws;    // [n_seq][P][kAggFloats] aggregates
-    unsigned long long *flags;   // [n_seq][P] publish tags
-    unsigned long long *hdr;     // [2]: generation, finished CTAs
+    unsigned *flags;   // [n_seq][P] publish flags: readers still to come
 };
 
 __device__ __forceinline__ uint64_t *bar(uint8_t *sm, int i) {
@@ -170,13 +171,16 @@ __device__ __forceinline__ void load_chunk(const Params &P, uint8_t *sm, int seq
     }
 }
 
-__device__ __forceinline__ unsigned long long ld_acquire_gpu(const unsigned long long *p) {
-    unsigned long long v;
-    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
-__device__ __forceinline__ void st_release_gpu(unsigned long long *p, unsigned long long v) {
-    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+__device__ __forceinline__ void st_release_gpu(unsigned *p, unsigned v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ void red_dec_gpu(unsigned *p) {   // *p -= 1, relaxed, no result
+    asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(0xffffffffu) : "memory");
 }
 
 // Epilogue of one 64x64 fp32 accumulator at TMEM column `col` by a team of four
@@ -661,9 +665,6 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_span_kernel(const Params 
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     bool to = false;
-    // publish tag of this launch (the generation only changes after every CTA of
-    // the previous launch has finished)
-    const unsigned long long tag = PS > 1 ? __ldcg(Wk.hdr) + 1ull : 0ull;
     // Barrier phase counters.  Each role counts only the barriers it waits on, and
     // every role walks every chunk, so the counts stay consistent across sequences.
     uint32_t nuse[2] = {0u, 0u};        // uses of buffer 0 / 1 (per role)
@@ -680,9 +681,10 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_span_kernel(const Params 
         float *agg = (PS > 1 && kspan < PS - 1) ? Wk.ws + ((size_t)seq * PS + kspan) * kAggFloats
                                                 : nullptr;
         // ---------------- phase 1 prologue: running state and decay products
-        {
+        // (groups A and B; the loader warp starts loading the sequence meanwhile)
+        if (warp < 12) {
             uint8_t *sst = sm + L::sst;
-            for (int e = tid; e < kDK * kDV / 4; e += kThreads) {
+            for (int e = tid; e < kDK * kDV / 4; e += kThreadsA + kThreadsB) {
                 const int i = e >> 4, c4 = e & 15;
                 float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (!later && P.s0 != nullptr)
@@ -694,10 +696,10 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_span_kernel(const Params 
             }
             if (tid < 64) dcum[tid] = 1.f;
             if (tid < kMaxSpan * 2) cmeta[tid] = 0.f;
+            fence_proxy_async_cta();
+            named_sync(kBarPro, kThreadsA + kThreadsB);
+            if (tid == 0) mbar_arrive(bar(sm, B_OPSF));   // S_prev of chunk 0 is ready
         }
-        fence_proxy_async_cta();
-        __syncthreads();
-        if (tid == 0) mbar_arrive(bar(sm, B_OPSF));   // S_prev of chunk 0 is ready
         // phase indices at the start of the sequence: chunk c is use c/2 of parity c%2
         const uint32_t m1b0 = m1s[0], m1b1 = m1s[1], sc_base = sc_seen;
 
@@ -725,10 +727,12 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_span_kernel(const Params 
                                    pub ? agg : nullptr);
                     if (pub) {
                         // aggregate = (state reached from zero, product of the span's decays)
+                        // (the CTA barrier orders every thread's stores before thread 0's
+                        // release at gpu scope)
                         if (tid < 64) agg[kDK * kDV + tid] = dcum[nch * 64 + tid];
-                        __threadfence();
                         named_sync(kBarA, kThreadsA);
-                        if (tid == 0) st_release_gpu(Wk.flags + (size_t)seq * PS + kspan, tag);
+                        if (tid == 0)   // readers to come: spans kspan+1 .. PS-1
+                            st_release_gpu(Wk.flags + (size_t)seq * PS + kspan, (unsigned)(PS - 1 - kspan));
                     }
                     if (tid == 0 && it < nch) mbar_arrive(bar(sm, B_OPSF + b));   // S_prev of chunk it
                 }
@@ -814,10 +818,11 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_span_kernel(const Params 
         // ---------------- phase 3: look back over the earlier spans
         if (later) {
             if (tid < kspan) {
-                const unsigned long long *f = Wk.flags + (size_t)seq * PS + tid;
-                if (ld_acquire_gpu(f) != tag) {
+                unsigned *f = Wk.flags + (size_t)seq * PS + tid;
+                bool seen = ld_acquire_gpu(f) != 0u;
+                if (!seen) {
                     const uint64_t t0 = globaltimer_ns();
-                    while (ld_acquire_gpu(f) != tag) {
+                    while (!(seen = ld_acquire_gpu(f) != 0u)) {
                         if (globaltimer_ns() - t0 > kWaitLimitNs) {
                             to = true;
                             set_error(kErrTimeout);
@@ -825,6 +830,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_span_kernel(const Params 
                         }
                     }
                 }
+                if (seen) red_dec_gpu(f);   // one reader fewer to come
             }
             __syncthreads();
             // S_in = S_out(span 0), then S_in = D_j * S_in + S_j for j = 1 .. kspan-1
@@ -1038,15 +1044,6 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_span_kernel(const Params 
         __syncthreads();   // staging / state tiles are reused by the next sequence
     }
 
-    // the last CTA to finish advances the workspace generation
-    if (PS > 1 && tid == 0) {
-        __threadfence();
-        if (atomicAdd(Wk.hdr + 1, 1ull) == (unsigned long long)(gridDim.x - 1)) {
-            Wk.hdr[1] = 0ull;
-            Wk.hdr[0] = tag;
-            __threadfence();
-        }
-    }
     // after a timeout some MMA may still be in flight: give it time before freeing TMEM
     if (__syncthreads_or(to)) {
         const uint64_t t0 = globaltimer_ns();

@@ -881,13 +881,13 @@ static int forced_cluster() {
 
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Workspace of the span kernel: a 256-byte header (launch generation, finished
-// CTAs), the publish flags of up to 2 * capacity (sequence, span) pairs, then the
-// aggregates.  Header and flags sit at the same offsets for every shape on a device.
-static size_t span_flags_bytes(int cap) { return align256((size_t)2 * cap * sizeof(unsigned long long)); }
+// Workspace of the span kernel: the publish flags of up to 2 * capacity (sequence,
+// span) pairs, zero between launches, then the aggregates.  The flags sit at the same
+// offset for every shape on a device.
+static size_t span_flags_bytes(int cap) { return align256((size_t)2 * cap * sizeof(unsigned)); }
 static size_t span_ws_bytes(long n_seq, int spans, int cap) {
     if (spans < 2) return 0;
-    return 256 + span_flags_bytes(cap) + align256((size_t)n_seq * spans * sp::kAggFloats * sizeof(float));
+    return span_flags_bytes(cap) + align256((size_t)n_seq * spans * sp::kAggFloats * sizeof(float));
 }
 
 // Span plan: P spans of Lc chunks per sequence (Lc <= 64 when P > 1), grid of whole
@@ -974,7 +974,7 @@ static DefaultWs g_default_ws[64];
 
 static size_t default_ws_bytes(int cap) {
     if (cap <= 0) return 0;
-    return 256 + span_flags_bytes(cap) + align256((size_t)2 * cap * sp::kAggFloats * sizeof(float));
+    return span_flags_bytes(cap) + align256((size_t)2 * cap * sp::kAggFloats * sizeof(float));
 }
 
 static cudaError_t default_workspace(int dev, size_t need, cudaStream_t stream, void **ptr) {
@@ -1027,9 +1027,8 @@ static cudaError_t launch(const Params &prm, const Plan &pl, void *workspace, cu
         if (pl.ws_bytes > 0) {
             uint8_t *base = static_cast<uint8_t *>(workspace);
             const int cap = span_capacity(dev, num_sms(dev), true);
-            wk.hdr = reinterpret_cast<unsigned long long *>(base);
-            wk.flags = reinterpret_cast<unsigned long long *>(base + 256);
-            wk.ws = reinterpret_cast<float *>(base + 256 + span_flags_bytes(cap));
+            wk.flags = reinterpret_cast<unsigned *>(base);
+            wk.ws = reinterpret_cast<float *>(base + span_flags_bytes(cap));
         }
         void *args[] = {const_cast<Params *>(&prm), &wk};
         return cudaLaunchKernelExC(&cfg, k.fn, args);
@@ -1160,7 +1159,7 @@ static __device__ __align__(256) unsigned char g_static_ws[kStaticWsBytes];
 static void *g_static_ws_ptr[64];
 
 // Device address of the static scratch on the current device `dev`, looked up once
-// (with `dev` current); the first lookup also zero-fills the header and flags.
+// (with `dev` current); the first lookup also zero-fills the publish flags.
 static cudaError_t static_scratch(int dev, void **ptr) {
     const int cap = span_capacity(dev, num_sms(dev), true);
     std::lock_guard<std::mutex> lk(g_mu);
@@ -1168,7 +1167,7 @@ static cudaError_t static_scratch(int dev, void **ptr) {
         void *p = nullptr;
         cudaError_t e = cudaGetSymbolAddress(&p, g_static_ws);
         if (e != cudaSuccess) return e;
-        e = cudaMemset(p, 0, 256 + span_flags_bytes(cap > 0 ? cap : num_sms(dev)));
+        e = cudaMemset(p, 0, span_flags_bytes(cap > 0 ? cap : num_sms(dev)));
         if (e == cudaSuccess) e = cudaDeviceSynchronize();
         if (e != cudaSuccess) return e;
         g_static_ws_ptr[dev] = p;
@@ -1210,14 +1209,13 @@ extern "C" gtr_status_t gtr_gla_device_status(void *stream) {
     if (word != 0) {
         const unsigned zero = 0;
         cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero));
-        // a span launch that timed out can leave publish flags set: clear the cached
-        // workspace of this device so the next call starts from zero
+        // a span launch that timed out can leave publish flags set: clear the library's
+        // workspaces of this device (cached and static) so the next call starts from zero
         const int dev = current_device();
         std::lock_guard<std::mutex> lk(g_mu);
-        if (g_default_ws[dev].ptr != nullptr) {
-            cudaMemset(g_default_ws[dev].ptr, 0, g_default_ws[dev].bytes);
-            cudaDeviceSynchronize();
-        }
+        if (g_default_ws[dev].ptr != nullptr) cudaMemset(g_default_ws[dev].ptr, 0, g_default_ws[dev].bytes);
+        if (g_static_ws_ptr[dev] != nullptr) cudaMemset(g_static_ws_ptr[dev], 0, kStaticWsBytes);
+        cudaDeviceSynchronize();
         return GTR_ERR_TIMEOUT;
     }
     return GTR_OK;

@@ -108,10 +108,12 @@ def test_in_place_carry_with_spans(monkeypatch):
     assert_parity(st.cpu().numpy(), rs, "carried state")
 
 
-def _header(ws):
-    """(launch generation, CTAs finished in the current launch) of a workspace."""
-    h = ws[:16].view(torch.int64).cpu().tolist()
-    return h[0], h[1]
+def _flags_clear(ws):
+    """The workspace's publish flags (2 x 4 bytes per SM, rounded up to 256) are zero:
+    every reader of a span's aggregate took itself off that span's flag."""
+    sms = torch.cuda.get_device_properties(ws.device).multi_processor_count
+    n = (2 * 4 * sms + 255) // 256 * 256
+    return int(torch.count_nonzero(ws[:n]).item()) == 0
 
 
 def test_caller_workspace_matches_default():
@@ -132,7 +134,7 @@ def test_caller_workspace_matches_default():
         torch.cuda.synchronize()
         assert gla.device_status() == gla.GTR_OK
         assert torch.equal(o1, o2) and torch.equal(s1, s2)
-        assert _header(ws) == (call + 1, 0)
+        assert _flags_clear(ws)
         ro, rs = run_oracle(inp, w.H, w.W, d)
         assert_parity(o1.float().cpu().numpy(), ro, f"call {call} out")
         assert_parity(s1.cpu().numpy(), rs, f"call {call} state")
@@ -163,6 +165,7 @@ def test_workspace_shared_across_shapes(monkeypatch):
                                      final_state=True)
             torch.cuda.synchronize()
             assert gla.device_status() == gla.GTR_OK
+            assert _flags_clear(ws)
             ro, rs = run_oracle(inp, H, W, d)
             for what, o, st in (("caller ws", o1, s1), ("library ws", o2, s2)):
                 assert_parity(o.float().cpu().numpy(), ro, f"{what} shape {i} rep {rep} out")
