@@ -484,24 +484,42 @@ __device__ __forceinline__ bool gate_chunk(const Params &P, uint8_t *sm, int ci,
 
 // MMA 1 of the chunk in buffer b (one thread): dS = K~^T V into TMEM dS buffer b,
 // scores = Qint K~^T (or the four sub-block products) into the scores columns.
+// (Called by a whole converged warp; one elected lane issues.)
 __device__ __forceinline__ void issue_mma1(uint32_t sbase, uint32_t tmem, int b, int vb, bool slow,
                                            uint64_t *done) {
     tc_fence_after();
     const uint32_t kta = sbase + L::kt + b * kTile;
     const uint32_t va = sbase + L::vop + vb * kTile;
-    constexpr uint32_t id_ds = idesc_f16_f32(64, kDV, true, true);
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk)
-        umma_f16(tmem + kColDS + 64 * b, desc_sw128(kta + kk * 2048, kTile, 1024),
-                 desc_sw128(va + kk * 2048, kTile, 1024), id_ds, kk > 0 ? 1u : 0u);
+    const uint32_t qa = sbase + L::qint + b * kTile;
     if (!slow) {
-        constexpr uint32_t id = idesc_f16_f32(64, 64, false, false);
-        const uint32_t qa = sbase + L::qint + b * kTile;
+        uint64_t d_k[4], d_v[4], d_q[4], d_kr[4];
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            d_k[kk] = desc_sw128(kta + kk * 2048, kTile, 1024);
+            d_v[kk] = desc_sw128(va + kk * 2048, kTile, 1024);
+            d_q[kk] = desc_sw128(qa + kk * 32, 16, 1024);
+            d_kr[kk] = desc_sw128(kta + kk * 32, 16, 1024);
+        }
+        if (elect_one_sync()) {
+            constexpr uint32_t id_ds = idesc_f16_f32(64, kDV, true, true);
+            constexpr uint32_t id = idesc_f16_f32(64, 64, false, false);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                umma_f16(tmem + kColDS + 64 * b, d_k[kk], d_v[kk], id_ds, kk > 0 ? 1u : 0u);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                umma_f16(tmem + kColScores, d_q[kk], d_kr[kk], id, kk > 0 ? 1u : 0u);
+            umma_commit(done);
+        }
+        __syncwarp();
+        return;
+    }
+    if (elect_one_sync()) {
+        constexpr uint32_t id_ds = idesc_f16_f32(64, kDV, true, true);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-            umma_f16(tmem + kColScores, desc_sw128(qa + kk * 32, 16, 1024),
-                     desc_sw128(kta + kk * 32, 16, 1024), id, kk > 0 ? 1u : 0u);
-    } else {
+            umma_f16(tmem + kColDS + 64 * b, desc_sw128(kta + kk * 2048, kTile, 1024),
+                     desc_sw128(va + kk * 2048, kTile, 1024), id_ds, kk > 0 ? 1u : 0u);
         constexpr uint32_t id = idesc_f16_f32(64, 16, false, false);
         for (int J = 0; J < 4; ++J) {
 #pragma unroll
@@ -512,8 +530,9 @@ __device__ __forceinline__ void issue_mma1(uint32_t sbase, uint32_t tmem, int b,
                          desc_sw128(bb, 16, 1024), id, kk > 0 ? 1u : 0u);
             }
         }
+        umma_commit(done);
     }
-    umma_commit(done);
+    __syncwarp();
 }
 
 // Group B (warps 8-11), MMA 1 of a chunk complete: TMEM -> registers of the scores
@@ -754,29 +773,39 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_span_kernel(const Params 
                 store_p_tmem(sm, tmem, r, b, misc_flags(sm, b)[warp & 3] != 0);
                 tc_fence_before();
                 named_sync(kBarB, kThreadsB);
-                if (tb == 0) {
-                    // only the issuing thread waits for S_prev of chunk c (a lagging
-                    // waiter could miss a phase: the next one follows MMA 2 of chunk c)
+                if (bw == 0) {
+                    // only the issuing warp (converged) waits for S_prev of chunk c (a
+                    // lagging waiter could miss a phase: the next one follows MMA 2 of
+                    // chunk c); one elected lane issues
                     wait_l(bar(sm, B_OPSF + b), nuse[b] & 1u, to);
                     ++nuse[b];
+                    __syncwarp();
                     tc_fence_after();
                     const uint32_t dcol = held ? kColHold + 64 * c : kColWork;
-                    constexpr uint32_t id = idesc_f16_f32(64, kDV, false, true);
                     const uint32_t qa = sbase + L::qint + b * kTile;
                     const uint32_t sa = sbase + L::sop + b * kTile;
                     const uint32_t va = sbase + L::vop + (c % 3) * kTile;
+                    uint64_t d_q[4], d_s[4], d_v[4];
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        umma_f16(tmem + dcol, desc_sw128(qa + kk * 32, 16, 1024),
-                                 desc_sw128(sa + kk * 2048, kTile, 1024), id, kk > 0 ? 1u : 0u);
+                    for (int kk = 0; kk < 4; ++kk) {
+                        d_q[kk] = desc_sw128(qa + kk * 32, 16, 1024);
+                        d_s[kk] = desc_sw128(sa + kk * 2048, kTile, 1024);
+                        d_v[kk] = desc_sw128(va + kk * 2048, kTile, 1024);
+                    }
+                    if (elect_one_sync()) {
+                        constexpr uint32_t id = idesc_f16_f32(64, kDV, false, true);
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)   // P from TMEM: K step 16 = 8 packed columns
-                        umma_f16_ta(tmem + dcol, tmem + kColScores + 8 * kk,
-                                    desc_sw128(va + kk * 2048, kTile, 1024), id, 1u);
-                    umma_commit(bar(sm, B_MMA2));
-                    umma_commit(bar(sm, B_OPSE + b));    // Qint, S_prev tiles free
-                    umma_commit(bar(sm, B_VE + c % 3));  // V tile free
-                    umma_commit(bar(sm, B_SCON));        // scores / P columns free for MMA 1
+                        for (int kk = 0; kk < 4; ++kk)
+                            umma_f16(tmem + dcol, d_q[kk], d_s[kk], id, kk > 0 ? 1u : 0u);
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)   // P from TMEM: K step 16 = 8 packed columns
+                            umma_f16_ta(tmem + dcol, tmem + kColScores + 8 * kk, d_v[kk], id, 1u);
+                        umma_commit(bar(sm, B_MMA2));
+                        umma_commit(bar(sm, B_OPSE + b));    // Qint, S_prev tiles free
+                        umma_commit(bar(sm, B_VE + c % 3));  // V tile free
+                        umma_commit(bar(sm, B_SCON));        // scores / P columns free for MMA 1
+                    }
+                    __syncwarp();
                 }
                 wait_l(bar(sm, B_MMA2), m2_seen & 1u, to);
                 ++m2_seen;
@@ -799,19 +828,18 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_span_kernel(const Params 
             if (nch > 1) loader_load(P, sm, seq, c0, 1, lane, nuse, nvuse, to);
             for (int c = 0; c < nch; ++c) {
                 const int b = c & 1;
-                if (lane == 0) {
-                    // GATE[b] next completes for chunk c+2, whose staging is only loaded
-                    // after this wait, so no phase can be missed
-                    wait_l(bar(sm, B_GATE + b), (g_seen >> b) & 1u, to);
-                    g_seen ^= 1u << b;
-                    if (c > 0) wait_phase(bar(sm, B_SCON), sc_seen, sc_base + c - 1, to);
-                    fence_proxy_async_cta();
-                    issue_mma1(sbase, tmem, b, c % 3, *misc_slow(sm, b) != 0, bar(sm, B_MMA1 + b));
-                }
+                // (the whole warp waits; its lanes run converged.)  GATE[b] next
+                // completes for chunk c+2, whose staging is only loaded after this
+                // wait, so no phase can be missed
+                wait_l(bar(sm, B_GATE + b), (g_seen >> b) & 1u, to);
+                g_seen ^= 1u << b;
+                if (c > 0) wait_phase(bar(sm, B_SCON), sc_seen, sc_base + c - 1, to);
                 __syncwarp();
+                fence_proxy_async_cta();
+                issue_mma1(sbase, tmem, b, c % 3, *misc_slow(sm, b) != 0, bar(sm, B_MMA1 + b));
                 if (c + 2 < nch) loader_load(P, sm, seq, c0, c + 2, lane, nuse, nvuse, to);
             }
-            if (lane == 0) wait_phase(bar(sm, B_SCON), sc_seen, sc_base + nch - 1, to);
+            wait_phase(bar(sm, B_SCON), sc_seen, sc_base + nch - 1, to);
             __syncwarp();
         }
         __syncthreads();
@@ -903,18 +931,21 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_span_kernel(const Params 
                 }
                 fence_proxy_async_cta();
                 __syncthreads();
-                if (tid == 0) {
+                if (warp == 0) {
                     tc_fence_after();
-                    constexpr uint32_t id = idesc_f16_f32(64, kDV, false, true);
-                    const uint32_t ba = smem_u32(bt);
-                    for (int ci = 0; ci < hold; ++ci) {
-                        const uint32_t qa = sbase + L::ring + ci * kTile;
+                    if (elect_one_sync()) {
+                        constexpr uint32_t id = idesc_f16_f32(64, kDV, false, true);
+                        const uint32_t ba = smem_u32(bt);
+                        for (int ci = 0; ci < hold; ++ci) {
+                            const uint32_t qa = sbase + L::ring + ci * kTile;
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            umma_f16(tmem + kColHold + 64 * ci, desc_sw128(qa + kk * 32, 16, 1024),
-                                     desc_sw128(ba + kk * 2048, kTile, 1024), id, 1u);
+                            for (int kk = 0; kk < 4; ++kk)
+                                umma_f16(tmem + kColHold + 64 * ci, desc_sw128(qa + kk * 32, 16, 1024),
+                                         desc_sw128(ba + kk * 2048, kTile, 1024), id, 1u);
+                        }
+                        umma_commit(bar(sm, B_FIX));
                     }
-                    umma_commit(bar(sm, B_FIX));
+                    __syncwarp();
                 }
                 wait_l(bar(sm, B_FIX), n_fix & 1u, to);
                 ++n_fix;
@@ -1000,14 +1031,17 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_span_kernel(const Params 
                 }
                 fence_proxy_async_cta();
                 __syncthreads();
-                if (tid == 0) {
+                if (warp == 0) {
                     tc_fence_after();
-                    constexpr uint32_t id = idesc_f16_f32(64, kDV, false, true);
+                    if (elect_one_sync()) {
+                        constexpr uint32_t id = idesc_f16_f32(64, kDV, false, true);
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        umma_f16(tmem + kColWork, desc_sw128(sbase + L::qint + kk * 32, 16, 1024),
-                                 desc_sw128(sbase + L::sop + kk * 2048, kTile, 1024), id, kk > 0 ? 1u : 0u);
-                    umma_commit(bar(sm, B_FIX));
+                        for (int kk = 0; kk < 4; ++kk)
+                            umma_f16(tmem + kColWork, desc_sw128(sbase + L::qint + kk * 32, 16, 1024),
+                                     desc_sw128(sbase + L::sop + kk * 2048, kTile, 1024), id, kk > 0 ? 1u : 0u);
+                        umma_commit(bar(sm, B_FIX));
+                    }
+                    __syncwarp();
                 }
                 wait_l(bar(sm, B_FIX), n_fix & 1u, to);
                 ++n_fix;

@@ -102,6 +102,16 @@ __device__ __forceinline__ void umma_commit(uint64_t *bar) {
         : "memory");
 }
 
+// One lane of a converged warp (the lowest active) gets true.  Issuing tcgen05.mma
+// from inside this predicate lets the operands stay warp-uniform; a plain
+// single-thread branch measured about twice the issue time.
+__device__ __forceinline__ bool elect_one_sync() {
+    uint32_t is_leader;
+    asm volatile("{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}\n"
+                 : "=r"(is_leader));
+    return is_leader != 0;
+}
+
 __device__ __forceinline__ void tc_fence_before() {
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
