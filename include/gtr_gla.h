@@ -158,6 +158,19 @@ gtr_status_t gtr_gla_fwd_static(const gtr_half_t *q, const gtr_half_t *k, const 
  */
 gtr_status_t gtr_gla_device_status(void *stream);
 
+/*
+ * Self-test of the device-side failure path (no counterpart on the pages: this
+ * checks the library's own error reporting).  Enqueues on `stream` a one-CTA
+ * kernel whose waits (an mbarrier nothing arrives on, a flag nothing sets) run
+ * through the same bounded-wait code as the forward kernels, with a limit of
+ * limit_us microseconds (1 .. 1000000) instead of their 200 ms.  Both waits run
+ * out; the kernel sets the device error word and ends normally, so the next
+ * gtr_gla_device_status returns GTR_ERR_TIMEOUT (and clears it), and the context
+ * stays usable.  Returns GTR_ERR_INVALID_ARG for a limit out of range, else the
+ * launch status.
+ */
+gtr_status_t gtr_gla_selftest_timeout(unsigned limit_us, void *stream);
+
 /* Static text for a status code (never NULL). */
 const char *gtr_status_str(gtr_status_t status);
 

@@ -182,6 +182,14 @@ __device__ __forceinline__ void st_release_gpu(unsigned *p, unsigned v) {
 __device__ __forceinline__ void red_dec_gpu(unsigned *p) {   // *p -= 1, relaxed, no result
     asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(0xffffffffu) : "memory");
 }
+// Waits (acquire) until *f is non-zero, for at most limit_ns; false if the limit ran out.
+__device__ __forceinline__ bool flag_wait_bounded(const unsigned *f, uint64_t limit_ns) {
+    if (ld_acquire_gpu(f) != 0u) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (ld_acquire_gpu(f) == 0u)
+        if (globaltimer_ns() - t0 > limit_ns) return false;
+    return true;
+}
 
 // Epilogue of one 64x64 fp32 accumulator at TMEM column `col` by a team of four
 // consecutive warps (warp w reads TMEM lanes 32 (w % 4) ..; tb = thread in the team,
@@ -847,18 +855,12 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_span_kernel(const Params 
         if (later) {
             if (tid < kspan) {
                 unsigned *f = Wk.flags + (size_t)seq * PS + tid;
-                bool seen = ld_acquire_gpu(f) != 0u;
-                if (!seen) {
-                    const uint64_t t0 = globaltimer_ns();
-                    while (!(seen = ld_acquire_gpu(f) != 0u)) {
-                        if (globaltimer_ns() - t0 > kWaitLimitNs) {
-                            to = true;
-                            set_error(kErrTimeout);
-                            break;
-                        }
-                    }
+                if (flag_wait_bounded(f, kWaitLimitNs)) {
+                    red_dec_gpu(f);   // one reader fewer to come
+                } else {
+                    to = true;
+                    set_error(kErrTimeout);
                 }
-                if (seen) red_dec_gpu(f);   // one reader fewer to come
             }
             __syncthreads();
             // S_in = S_out(span 0), then S_in = D_j * S_in + S_j for j = 1 .. kspan-1

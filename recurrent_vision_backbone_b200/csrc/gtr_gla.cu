@@ -1198,6 +1198,34 @@ extern "C" gtr_status_t gtr_gla_fwd_static(const gtr_half_t *q, const gtr_half_t
     return cuda_status(launch(prm, pl, ws, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+namespace gtr {
+
+// Self-test of the device-side failure path: thread 0 waits on an mbarrier that
+// nothing arrives on and thread 32 polls a flag that nothing sets, each through the
+// bounded waits the forward kernels use, for limit_ns; both report kErrTimeout
+// through the device error word and the kernel ends normally.
+static __device__ unsigned g_selftest_flag;   // never written
+
+__global__ void selftest_wait_kernel(uint64_t limit_ns) {
+    __shared__ __align__(8) uint64_t never;
+    if (threadIdx.x == 0) {
+        mbar_init(&never, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && !mbar_wait_bounded(&never, 0, limit_ns)) set_error(kErrTimeout);
+    if (threadIdx.x == 32 && !sp::flag_wait_bounded(&g_selftest_flag, limit_ns)) set_error(kErrTimeout);
+}
+
+}  // namespace gtr
+
+extern "C" gtr_status_t gtr_gla_selftest_timeout(unsigned limit_us, void *stream) {
+    if (limit_us == 0 || limit_us > 1000000u) return GTR_ERR_INVALID_ARG;
+    selftest_wait_kernel<<<1, 64, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        (uint64_t)limit_us * 1000ull);
+    return cuda_status(cudaGetLastError());
+}
+
 extern "C" gtr_status_t gtr_gla_device_status(void *stream) {
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (cudaStreamSynchronize(s) != cudaSuccess) {

@@ -23,7 +23,7 @@ STATIC_WS_BYTES = 4 << 20   # GTR_STATIC_WS_BYTES
 
 EXPORTED_SYMBOLS = ("gtr_gla_fwd", "gtr_gla_workspace_bytes", "gtr_gla_fwd_ws",
                     "gtr_gla_fwd_static", "gtr_gla_device_status", "gtr_status_str", "gtr_gla_plan", "gtr_gla_version",
-                    "gtr_gla_last_error")
+                    "gtr_gla_last_error", "gtr_gla_selftest_timeout")
 
 _lock = threading.Lock()
 _lib = None
@@ -60,6 +60,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
                                        + [vp, ctypes.c_size_t, vp])
         lib.gtr_gla_device_status.restype = i
         lib.gtr_gla_device_status.argtypes = [vp]
+        lib.gtr_gla_selftest_timeout.restype = i
+        lib.gtr_gla_selftest_timeout.argtypes = [ctypes.c_uint, vp]
         lib.gtr_status_str.restype = ctypes.c_char_p
         lib.gtr_status_str.argtypes = [i]
         lib.gtr_gla_plan.restype = i
@@ -191,6 +193,13 @@ def gtr_gla_fwd_raw(q_ptr: int, k_ptr: int, v_ptr: int, g_ptr: int, B: int, head
 def device_status(stream=None) -> int:
     """Sync the stream; return (and clear) the device error status."""
     return int(load().gtr_gla_device_status(_stream_handle(stream)))
+
+
+def selftest_timeout(limit_us: int = 2000, stream=None) -> int:
+    """Enqueue the device failure-path self-test (waits that nothing satisfies, bounded
+    by limit_us); the next device_status() reports GTR_ERR_TIMEOUT.  Returns the
+    launch status."""
+    return int(load().gtr_gla_selftest_timeout(int(limit_us), _stream_handle(stream)))
 
 
 def plan(B: int, heads: int, Hgrid: int, Wgrid: int, dk: int, dv: int):
