@@ -11,13 +11,14 @@
 //            pipeline over two operand buffers:
 //              loader (warp 12)   cp.async of q, k, g rows into staging and of v
 //                                 straight into its swizzled operand tile, two
-//                                 chunks ahead; lane 0 issues MMA 1(c) = (dS,
-//                                 scores) once chunk c is gated and MMA 2(c-1) has
-//                                 consumed the scores' TMEM columns;
+//                                 chunks ahead, as the buffers free up;
 //              group A (warps 0-7) gating of chunk c (Qint = q P, K~ = k / P, ...),
 //                                 then S <- d * S + dS of chunk c-1 from TMEM (its
 //                                 fp16 copy is S_prev of chunk c);
-//              group B (warps 8-11) scores of chunk c from TMEM into the causal fp16
+//              group B (warps 8-11) once chunk c is gated, MMA 1(c) = (dS, scores)
+//                                 (one elected lane: MMA 2(c-1), which consumed the
+//                                 scores' TMEM columns, is complete by then), then the
+//                                 scores of chunk c from TMEM into the causal fp16
 //                                 P tile, written back to TMEM, MMA 2(c) = Qint S_prev
 //                                 + P V (P as the TMEM A operand), output stores;
 //   phase 2  the span's last state update publishes its aggregate (state reached
@@ -94,7 +95,6 @@ enum {
     B_STGF = 0,   // [2] staging (+ V tile) landed: 32 loader arrivals
     B_STGE = 2,   // [2] group A done with the staging buffer
     B_MMA1 = 19,  // [2] MMA 1 of a chunk of this parity complete (waited by groups A and B)
-    B_SCON = 5,   // MMA 2 has consumed P, held in the scores' TMEM columns (tcgen05.commit)
     B_OPSF = 6,   // [2] S_prev of a chunk ready for its MMA 2
     B_OPSE = 8,   // [2] MMA 2 done with Qint, S_prev of a buffer (tcgen05.commit)
     B_MMA2 = 10,
@@ -678,7 +678,6 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_span_kernel(const Params 
             mbar_init(bar(sm, B_OPSE + i), 1);
         }
         for (int i = 0; i < 2; ++i) mbar_init(bar(sm, B_MMA1 + i), 1);
-        mbar_init(bar(sm, B_SCON), 1);
         mbar_init(bar(sm, B_MMA2), 1);
         mbar_init(bar(sm, B_FIX), 1);
         for (int i = 0; i < 2; ++i) mbar_init(bar(sm, B_GATE + i), 1);
@@ -697,7 +696,6 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_span_kernel(const Params 
     uint32_t nuse[2] = {0u, 0u};        // uses of buffer 0 / 1 (per role)
     uint32_t nvuse[3] = {0u, 0u, 0u};   // loader: uses of V tile 0 / 1 / 2
     uint32_t m1s[2] = {0u, 0u};         // MMA 1 phases observed, per parity
-    uint32_t sc_seen = 0;               // score-readout phases observed (loader lane 0)
     uint32_t m2_seen = 0, g_seen = 0, n_fix = 0;
 
     for (int seq = grp; seq < P.n_seq; seq += ngrp) {
@@ -728,7 +726,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_span_kernel(const Params 
             if (tid == 0) mbar_arrive(bar(sm, B_OPSF));   // S_prev of chunk 0 is ready
         }
         // phase indices at the start of the sequence: chunk c is use c/2 of parity c%2
-        const uint32_t m1b0 = m1s[0], m1b1 = m1s[1], sc_base = sc_seen;
+        const uint32_t m1b0 = m1s[0], m1b1 = m1s[1];
 
         if (warp < 8) {
             // ================================================= group A
@@ -775,6 +773,14 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_span_kernel(const Params 
                 fill_rows(P, seq, c0 + c, rows2, tb);
                 wait_l(bar(sm, B_GATE + b), (g_seen >> b) & 1u, to);   // bit b: parity of GATE[b]
                 g_seen ^= 1u << b;
+                // MMA 1(c) (one elected lane of warp 8): the scores' TMEM columns are
+                // free (MMA 2(c-1), complete, consumed P) and so is the dS buffer (group A
+                // read dS(c-2) before gating chunk c)
+                if (bw == 0) {
+                    __syncwarp();
+                    fence_proxy_async_cta();
+                    issue_mma1(sbase, tmem, b, c % 3, *misc_slow(sm, b) != 0, bar(sm, B_MMA1 + b));
+                }
                 wait_phase(bar(sm, B_MMA1 + b), m1s[b], (b ? m1b1 : m1b0) + (c >> 1), to);
                 BRegs r;
                 load_tmem_b(tmem, r);
@@ -811,7 +817,6 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_span_kernel(const Params 
                         umma_commit(bar(sm, B_MMA2));
                         umma_commit(bar(sm, B_OPSE + b));    // Qint, S_prev tiles free
                         umma_commit(bar(sm, B_VE + c % 3));  // V tile free
-                        umma_commit(bar(sm, B_SCON));        // scores / P columns free for MMA 1
                     }
                     __syncwarp();
                 }
@@ -830,25 +835,11 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_span_kernel(const Params 
             }
         } else {
             // ================================================= loader (warp 12)
-            // Loads run two chunks ahead; lane 0 also issues MMA 1 of each chunk once
-            // group A has gated it and group B has read the previous chunk's scores.
+            // Loads run ahead as the staging buffers (once gated) and the V tiles (once
+            // MMA 2 has read them) free up.
             loader_load(P, sm, seq, c0, 0, lane, nuse, nvuse, to);
             if (nch > 1) loader_load(P, sm, seq, c0, 1, lane, nuse, nvuse, to);
-            for (int c = 0; c < nch; ++c) {
-                const int b = c & 1;
-                // (the whole warp waits; its lanes run converged.)  GATE[b] next
-                // completes for chunk c+2, whose staging is only loaded after this
-                // wait, so no phase can be missed
-                wait_l(bar(sm, B_GATE + b), (g_seen >> b) & 1u, to);
-                g_seen ^= 1u << b;
-                if (c > 0) wait_phase(bar(sm, B_SCON), sc_seen, sc_base + c - 1, to);
-                __syncwarp();
-                fence_proxy_async_cta();
-                issue_mma1(sbase, tmem, b, c % 3, *misc_slow(sm, b) != 0, bar(sm, B_MMA1 + b));
-                if (c + 2 < nch) loader_load(P, sm, seq, c0, c + 2, lane, nuse, nvuse, to);
-            }
-            wait_phase(bar(sm, B_SCON), sc_seen, sc_base + nch - 1, to);
-            __syncwarp();
+            for (int c = 2; c < nch; ++c) loader_load(P, sm, seq, c0, c, lane, nuse, nvuse, to);
         }
         __syncthreads();
         // ---------------- phase 3: look back over the earlier spans
