@@ -104,8 +104,8 @@ size_t gtr_gla_workspace_bytes(int B, int heads, int Hgrid, int Wgrid, int dk, i
  *   workspace        device memory, 256-byte aligned, at least
  *                    gtr_gla_workspace_bytes(...) bytes (may be NULL when that is 0).
  *                    It must be zero-filled before its first use.  Its first
- *                    part (the spans' publish flags, 2 x 4 bytes per SM of the
- *                    device, rounded up to 256) must be zero when a call starts:
+ *                    part (the spans' publish flags, 2 x 128 bytes per SM of
+ *                    the device, rounded up to 256) must be zero when a call starts:
  *                    every call that completes without a device error leaves it
  *                    zero again; the rest holds the spans' aggregates, which any
  *                    call overwrites before reading.  After GTR_ERR_TIMEOUT the

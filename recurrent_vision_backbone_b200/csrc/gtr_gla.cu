@@ -884,7 +884,9 @@ static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 // Workspace of the span kernel: the publish flags of up to 2 * capacity (sequence,
 // span) pairs, zero between launches, then the aggregates.  The flags sit at the same
 // offset for every shape on a device.
-static size_t span_flags_bytes(int cap) { return align256((size_t)2 * cap * sizeof(unsigned)); }
+static size_t span_flags_bytes(int cap) {
+    return align256((size_t)2 * cap * sp::kFlagStride * sizeof(unsigned));
+}
 static size_t span_ws_bytes(long n_seq, int spans, int cap) {
     if (spans < 2) return 0;
     return span_flags_bytes(cap) + align256((size_t)n_seq * spans * sp::kAggFloats * sizeof(float));

@@ -109,10 +109,10 @@ def test_in_place_carry_with_spans(monkeypatch):
 
 
 def _flags_clear(ws):
-    """The workspace's publish flags (2 x 4 bytes per SM, rounded up to 256) are zero:
+    """The workspace's publish flags (2 x 128 bytes per SM, rounded up to 256) are zero:
     every reader of a span's aggregate took itself off that span's flag."""
     sms = torch.cuda.get_device_properties(ws.device).multi_processor_count
-    n = (2 * 4 * sms + 255) // 256 * 256
+    n = (2 * 128 * sms + 255) // 256 * 256
     return int(torch.count_nonzero(ws[:n]).item()) == 0
 
 
