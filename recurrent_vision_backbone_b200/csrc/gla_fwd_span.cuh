@@ -365,7 +365,9 @@ __device__ __forceinline__ bool gate_chunk(const Params &P, uint8_t *sm, int ci,
             bad |= !(d >= kFastMinDecay);
         }
     }
-    const bool slow = named_sync_or(kBarA, kThreadsA, bad);
+    // every warp's lanes cover all 64 channels and kmax is already reduced, so a warp
+    // vote gives each warp the chunk's decision without a group barrier
+    const bool slow = __any_sync(0xffffffffu, bad);
     const float2 dc = *reinterpret_cast<const float2 *>(dcum + (held ? ci : 0) * 64 + 2 * lane);
     if (gh == 0) {
         *reinterpret_cast<float2 *>(sm + L::dloc + b * 256 + 8 * lane) = make_float2(dch[0], dch[1]);
