@@ -9,7 +9,7 @@
 //
 //   phase 1  stream the span's chunks from a zero state (span 0: from S0), as a
 //            pipeline over two operand buffers:
-//              loaders (warps 12, 13) cp.async of q, k, g rows into staging and of v
+//              loaders (warps 12 ..) cp.async of q, k, g rows into staging and of v
 //                                 straight into its swizzled operand tile, two
 //                                 chunks ahead, as the buffers free up;
 //              group A (warps 0-7) gating of chunk c (Qint = q P, K~ = k / P, ...),
@@ -43,8 +43,12 @@ namespace sp {
 
 constexpr int kThreadsA = 256;              // warps 0-7
 constexpr int kThreadsB = 128;              // warps 8-11
-constexpr int kLoaders = 2;                 // loader warps 12, 13
-constexpr int kThreads = kThreadsA + kThreadsB + 32 * kLoaders;
+// Loader warps (12 ..): two for long spans; four for spans of at most
+// kShortSpan chunks, which are latency-bound and gain from issuing a chunk's loads
+// faster (long spans lose: more warps share the schedulers with the compute groups)
+template <int NL>
+__host__ __device__ constexpr int span_threads() { return kThreadsA + kThreadsB + 32 * NL; }
+constexpr int kShortSpan = 4;
 constexpr int kDK = 64;
 constexpr int kHold = 4;                    // chunks per span whose outputs wait in TMEM
 constexpr int kMaxSpan = 32;                // chunks of a span with recorded decays
@@ -78,7 +82,7 @@ struct L {
     static constexpr int cmeta = rowb + 3 * 64 * 4;     // per chunk: max|q|, max|o| [kMaxSpan][2]
     static constexpr int skipf = cmeta + kMaxSpan * 8;  // per chunk: correction negligible
     static constexpr int rmax = skipf + kMaxSpan * 4;   // row maxima of |S_in| [64]
-    static constexpr int ltab = rmax + 256;             // loaders' token rows [2][32]
+    static constexpr int ltab = rmax + 256;             // loaders' token rows [64]
     static constexpr int misc = ltab + 256;             // per parity (64 B): flags[4] qmax[4] kmax
     static constexpr int bars = misc + 128;
     static constexpr int bytes = bars + 24 * 8;
@@ -144,27 +148,29 @@ __device__ __forceinline__ void wait_phase(uint64_t *b, uint32_t &seen, uint32_t
     }
 }
 
-// Loader warp `lw` (of kLoaders): its share of chunk c's 64 rows of q, k, g into
+// Loader warp `lw` (of NL): its share of chunk c's 64 rows of q, k, g into
 // staging buffer `b` (row t at byte t * 128, unswizzled) and of v into the swizzled
 // operand tile vop[vb], with 16-byte cp.async, eight lanes per 128-byte row so that
-// one warp instruction moves four whole rows: rows 8 i + 4 lw + (lane / 8), i = 0 .. 7.
+// one warp instruction moves four whole rows: rows 4 (NL i + lw) + lane / 8.
 // Rows past the grid are zero-filled.
+template <int NL>
 __device__ __forceinline__ void load_chunk(const Params &P, uint8_t *sm, int seq, int c, int b,
                                            int vb, int lane, int lw) {
+    constexpr int kRows = 64 / NL;   // rows of this warp
     const uint32_t st = smem_u32(sm + L::stg + b * L::stg_bytes);
     const uint32_t vo = smem_u32(sm + L::vop + vb * kTile);
-    int *rowtab = reinterpret_cast<int *>(sm + L::ltab) + 32 * lw;
+    int *rowtab = reinterpret_cast<int *>(sm + L::ltab) + kRows * lw;
     const int bb = seq / P.heads, h = seq - bb * P.heads;
     __syncwarp();   // every lane is done with the previous chunk's table
-    {
-        const int t = 8 * (lane >> 2) + 4 * lw + (lane & 3), p = c * kChunk + t;
-        rowtab[lane] = p < P.N ? (bb * P.N + scan_to_token(p, P.H, P.W, P.dir)) * P.heads + h : -1;
+    for (int r = lane; r < kRows; r += 32) {
+        const int t = 4 * (NL * (r >> 2) + lw) + (r & 3), p = c * kChunk + t;
+        rowtab[r] = p < P.N ? (bb * P.N + scan_to_token(p, P.H, P.W, P.dir)) * P.heads + h : -1;
     }
     __syncwarp();
     const int sub = lane >> 3, pc = lane & 7;
 #pragma unroll 4
-    for (int i = 0; i < 8; ++i) {
-        const int t = 8 * i + 4 * lw + sub;
+    for (int i = 0; i < kRows / 4; ++i) {
+        const int t = 4 * (NL * i + lw) + sub;
         const int ro = rowtab[4 * i + sub];
         const uint32_t nb = ro >= 0 ? 16u : 0u;
         const size_t off = (size_t)(ro >= 0 ? ro : 0) * 64 + 8 * pc;
@@ -647,6 +653,7 @@ __device__ __forceinline__ void update_state_a(uint8_t *sm, uint32_t tmem, int b
 // Loader warp: chunk c of the span into staging buffer c % 2 and V tile c % 3 once
 // group A is done with the staging buffer (chunk c-2) and MMA 2 with the V tile
 // (chunk c-3).
+template <int NL>
 __device__ __forceinline__ void loader_load(const Params &P, uint8_t *sm, int seq, int c0, int c,
                                             int lane, int lw, uint32_t (&nuse)[2], uint32_t (&nvuse)[3],
                                             bool &to) {
@@ -655,11 +662,13 @@ __device__ __forceinline__ void loader_load(const Params &P, uint8_t *sm, int se
     wait_l(bar(sm, B_VE + vb), (nvuse[vb] & 1u) ^ 1u, to);
     ++nuse[b];
     ++nvuse[vb];
-    load_chunk(P, sm, seq, c0 + c, b, vb, lane, lw);
+    load_chunk<NL>(P, sm, seq, c0 + c, b, vb, lane, lw);
     cp_async_mbar_arrive_noinc(bar(sm, B_STGF + b));
 }
 
-__global__ void __launch_bounds__(kThreads, 1) gla_fwd_span_kernel(const Params P, const Work Wk) {
+template <int NL>
+__global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(const Params P, const Work Wk) {
+    constexpr int kThreads = span_threads<NL>();
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -680,7 +689,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_span_kernel(const Params 
     }
     if (tid == 0) {
         for (int i = 0; i < 2; ++i) {
-            mbar_init(bar(sm, B_STGF + i), 32 * kLoaders);
+            mbar_init(bar(sm, B_STGF + i), 32 * NL);
             mbar_init(bar(sm, B_STGE + i), 1);
             mbar_init(bar(sm, B_OPSE + i), 1);
         }
@@ -841,10 +850,10 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_span_kernel(const Params 
                 }
             }
         } else {
-            // ================================================= loaders (warps 12, 13)
+            // ================================================= loaders (warps 12 ..)
             // Loads run ahead as the staging buffers (once gated) and the V tiles (once
             // MMA 2 has read them) free up.
-            for (int c = 0; c < nch; ++c) loader_load(P, sm, seq, c0, c, lane, warp - 12, nuse, nvuse, to);
+            for (int c = 0; c < nch; ++c) loader_load<NL>(P, sm, seq, c0, c, lane, warp - 12, nuse, nvuse, to);
         }
         __syncthreads();
         // ---------------- phase 3: look back over the earlier spans

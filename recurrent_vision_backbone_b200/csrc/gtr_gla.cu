@@ -736,7 +736,10 @@ __global__ void __launch_bounds__(kThreads, Smem<DK>::min_blocks) gla_fwd_kernel
 namespace gtr {
 
 // ------------------------------------------------------------------ host
-enum KernelKind { kBasic64 = 0, kBasic128 = 1, kCluster = 2, kSpan = 3, kKinds = 4 };
+enum KernelKind { kBasic64 = 0, kBasic128 = 1, kCluster = 2, kSpan = 3, kSpanShort = 4, kKinds = 5 };
+
+// the span kernel with two loader warps (kSpan) or four (kSpanShort: short spans)
+static bool is_span(int kind) { return kind == kSpan || kind == kSpanShort; }
 
 // A kernel variant: entry point, block size, dynamic shared memory, cache slot.
 struct KSpec {
@@ -765,8 +768,12 @@ static KSpec spec_of(int kind) {
         return KSpec{reinterpret_cast<const void *>(&gla_fwd_kernel<128>), kThreads, Smem<128>::alloc, kBasic128};
     case kCluster:
         return KSpec{reinterpret_cast<const void *>(&ws::gla_fwd_ws_kernel), ws::kThreads, ws::L::alloc, kCluster};
+    case kSpanShort:
+        return KSpec{reinterpret_cast<const void *>(&sp::gla_fwd_span_kernel<4>), sp::span_threads<4>(),
+                     sp::L::alloc, kSpanShort};
     default:
-        return KSpec{reinterpret_cast<const void *>(&sp::gla_fwd_span_kernel), sp::kThreads, sp::L::alloc, kSpan};
+        return KSpec{reinterpret_cast<const void *>(&sp::gla_fwd_span_kernel<2>), sp::span_threads<2>(),
+                     sp::L::alloc, kSpan};
     }
 }
 
@@ -820,7 +827,7 @@ static void fill_config(cudaLaunchConfig_t &cfg, cudaLaunchAttribute *attr, cons
     cfg.dynamicSmemBytes = (size_t)k.smem;
     cfg.stream = stream;
     cfg.attrs = attr;
-    if (k.slot == kSpan) {
+    if (is_span(k.slot)) {
         // all spans of a sequence must be resident together: cooperative launch
         attr[0].id = cudaLaunchAttributeCooperative;
         attr[0].val.cooperative = 1;
@@ -921,6 +928,12 @@ static Plan span_plan(long n_seq, long n_chunks, int cap) {
         return p1;
     }
     best.ws_bytes = span_ws_bytes(n_seq, best.cluster, cap);
+    if (best.cluster > 1 && best.span_len <= sp::kShortSpan) {   // latency-bound: four loaders
+        const KSpec ks = spec_of(kSpanShort);
+        best.kind = kSpanShort;
+        best.threads = ks.threads;
+        best.smem = ks.smem;
+    }
     return best;
 }
 
@@ -1017,12 +1030,12 @@ static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 
 static cudaError_t launch(const Params &prm, const Plan &pl, void *workspace, cudaStream_t stream) {
     const int dev = current_device();
     const KSpec k = spec_of(pl.kind);
-    cudaError_t e = prepare_kernel(k, pl.kind == kSpan ? 1 : pl.cluster);
+    cudaError_t e = prepare_kernel(k, is_span(pl.kind) ? 1 : pl.cluster);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg;
     cudaLaunchAttribute attr[1];
     fill_config(cfg, attr, k, pl.cluster, pl.clusters, stream);
-    if (pl.kind == kSpan) {
+    if (is_span(pl.kind)) {
         sp::Work wk{};
         wk.P = pl.cluster;
         wk.Lc = pl.span_len;
