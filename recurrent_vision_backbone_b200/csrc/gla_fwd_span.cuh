@@ -706,6 +706,11 @@ __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(con
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // a launch that follows this one on the stream may be scheduled now (it waits
+    // below for this grid to complete); this grid waits for the one before it
+    // before any global memory access
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     bool to = false;
     // Barrier phase counters.  Each role counts only the barriers it waits on, and
     // every role walks every chunk, so the counts stay consistent across sequences.

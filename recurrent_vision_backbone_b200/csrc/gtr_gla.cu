@@ -828,16 +828,21 @@ static void fill_config(cudaLaunchConfig_t &cfg, cudaLaunchAttribute *attr, cons
     cfg.stream = stream;
     cfg.attrs = attr;
     if (is_span(k.slot)) {
-        // all spans of a sequence must be resident together: cooperative launch
+        // all spans of a sequence must be resident together: cooperative launch; the
+        // next launch on the stream may start its set-up while this one drains (the
+        // kernel waits for its predecessor before touching global memory)
         attr[0].id = cudaLaunchAttributeCooperative;
         attr[0].val.cooperative = 1;
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
+        cfg.numAttrs = 2;
     } else {
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = (unsigned)cluster;
         attr[0].val.clusterDim.y = 1;
         attr[0].val.clusterDim.z = 1;
+        cfg.numAttrs = 1;
     }
-    cfg.numAttrs = 1;
 }
 
 static int max_active_clusters(const KSpec &k, int dev, int cluster, int sms) {
@@ -849,7 +854,7 @@ static int max_active_clusters(const KSpec &k, int dev, int cluster, int sms) {
     int n = 0;
     if (prepare_kernel(k, cluster) == cudaSuccess) {
         cudaLaunchConfig_t cfg;
-        cudaLaunchAttribute attr[1];
+        cudaLaunchAttribute attr[2];
         fill_config(cfg, attr, k, cluster, sms / cluster, 0);
         if (cudaOccupancyMaxActiveClusters(&n, k.fn, &cfg) != cudaSuccess) n = 0;
     }
@@ -1033,7 +1038,7 @@ static cudaError_t launch(const Params &prm, const Plan &pl, void *workspace, cu
     cudaError_t e = prepare_kernel(k, is_span(pl.kind) ? 1 : pl.cluster);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     fill_config(cfg, attr, k, pl.cluster, pl.clusters, stream);
     if (is_span(pl.kind)) {
         sp::Work wk{};
