@@ -283,43 +283,73 @@ def call_inputs(w, d, seed, heads=None, device="cpu"):
 
 def e2e_measure(w, steps, device, rank):
     """Tokens/s through the public call with host buffers: every step copies that
-    step's inputs from pinned host memory and reads the outputs back."""
+    step's inputs from pinned host memory and reads its outputs back.  Uploads,
+    calls and read-backs run on three streams (PCIe carries both directions at
+    once), with two sets of device buffers so that step s+1's uploads overlap step
+    s's read-backs; events order every reuse of a buffer."""
     from recurrent_vision_backbone_b200 import gla
     calls = []
     for c, d in enumerate(w.call_directions()):
         inp = call_inputs(w, d, rank_seed(w.seed(d, 500 + c), rank))
         hp = {n: t.pin_memory() for n, t in inp.items() if t is not None}
-        dv = {n: torch.empty_like(t, device=device) for n, t in hp.items()}
-        out = torch.empty((w.B, w.N, w.heads, w.dv), dtype=torch.float16, device=device)
-        sf = (torch.empty((w.B, w.heads, w.dk, w.dv), dtype=torch.float32, device=device)
-              if w.final_state else None)
-        h_out = torch.empty_like(out, device="cpu").pin_memory()
-        h_sf = None if sf is None else torch.empty_like(sf, device="cpu").pin_memory()
-        calls.append((d, hp, dv, out, sf, h_out, h_sf))
-    stream = torch.cuda.current_stream()
+        sets = []
+        for _ in range(2):
+            dv = {n: torch.empty_like(t, device=device) for n, t in hp.items()}
+            out = torch.empty((w.B, w.N, w.heads, w.dv), dtype=torch.float16, device=device)
+            sf = (torch.empty((w.B, w.heads, w.dk, w.dv), dtype=torch.float32, device=device)
+                  if w.final_state else None)
+            ev = {k: torch.cuda.Event() for k in ("up", "done", "down")}
+            sets.append((dv, out, sf, ev))
+        h_out = torch.empty((w.B, w.N, w.heads, w.dv), dtype=torch.float16).pin_memory()
+        h_sf = (torch.empty((w.B, w.heads, w.dk, w.dv), dtype=torch.float32).pin_memory()
+                if w.final_state else None)
+        calls.append((d, hp, sets, h_out, h_sf))
+    s_up, s_call, s_down = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
     h2d = sum(t.numel() * t.element_size() for c in calls for t in c[1].values())
-    d2h = sum(c[5].numel() * c[5].element_size() + (0 if c[6] is None else
-                                                   c[6].numel() * c[6].element_size())
+    d2h = sum(c[3].numel() * c[3].element_size() + (0 if c[4] is None else
+                                                   c[4].numel() * c[4].element_size())
               for c in calls)
+    used = set()
 
-    def one_step():
-        for d, hp, dv, out, sf, h_out, h_sf in calls:
-            for n, t in hp.items():
-                dv[n].copy_(t, non_blocking=True)
-            gla.gtr_gla_fwd(dv["q"], dv["k"], dv["v"], dv["g"], w.H, w.W, d,
-                            init_state=dv.get("s0"), out=out, final_state=sf, stream=stream)
-            h_out.copy_(out, non_blocking=True)
-            if sf is not None:
-                h_sf.copy_(sf, non_blocking=True)
+    def one_step(step):
+        par = step & 1
+        for ci, (d, hp, sets, h_out, h_sf) in enumerate(calls):
+            dv, out, sf, ev = sets[par]
+            first = (ci, par) not in used
+            used.add((ci, par))
+            with torch.cuda.stream(s_up):
+                if not first:
+                    s_up.wait_event(ev["done"])      # the call two steps back read dv
+                for n, t in hp.items():
+                    dv[n].copy_(t, non_blocking=True)
+                ev["up"].record(s_up)
+            with torch.cuda.stream(s_call):
+                s_call.wait_event(ev["up"])
+                if not first:
+                    s_call.wait_event(ev["down"])    # out / sf of two steps back read back
+                gla.gtr_gla_fwd(dv["q"], dv["k"], dv["v"], dv["g"], w.H, w.W, d,
+                                init_state=dv.get("s0"), out=out, final_state=sf, stream=s_call)
+                ev["done"].record(s_call)
+            with torch.cuda.stream(s_down):
+                s_down.wait_event(ev["done"])
+                h_out.copy_(out, non_blocking=True)
+                if sf is not None:
+                    h_sf.copy_(sf, non_blocking=True)
+                ev["down"].record(s_down)
 
-    for _ in range(3):
-        one_step()
+    for i in range(3):
+        one_step(i)
     torch.cuda.synchronize()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    start.record(stream)
-    for _ in range(steps):
-        one_step()
-    end.record(stream)
+    start.record(s_up)
+    s_call.wait_event(start)
+    s_down.wait_event(start)
+    for i in range(steps):
+        one_step(3 + i)
+    s_down.wait_event(calls[-1][2][(3 + steps - 1) & 1][3]["down"])
+    s_down.wait_stream(s_up)
+    s_down.wait_stream(s_call)
+    end.record(s_down)
     torch.cuda.synchronize()
     ms = start.elapsed_time(end)
     return ms, steps, h2d, d2h
