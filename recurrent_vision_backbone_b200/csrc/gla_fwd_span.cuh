@@ -666,6 +666,65 @@ __device__ __forceinline__ void loader_load(const Params &P, uint8_t *sm, int se
     cp_async_mbar_arrive_noinc(bar(sm, B_STGF + b));
 }
 
+// Phase 4 (all threads): cp.async of chunk c's q, g rows and stored output rows into
+// three unswizzled tiles (row t at byte t * 128) at dst_q, dst_g, dst_o; one group.
+// (Out of line, scalar arguments: it runs once per span and adds nothing to the
+// register pressure of the kernel body.)
+__device__ __noinline__ void load_qgo(const __half *q, const __half *g, const __half *o, int N, int H,
+                                      int W, int dir, int heads, int seq, int c, uint32_t dst_q,
+                                      uint32_t dst_g, uint32_t dst_o, int nthreads) {
+    const int bq = seq / heads, hq = seq - bq * heads;
+    const int p0 = c * kChunk;
+    for (int x = (int)threadIdx.x; x < 3 * 64 * 8; x += nthreads) {
+        const int ten = x / 512, rem = x - ten * 512, t = rem >> 3, pc = rem & 7;
+        const bool ok = p0 + t < N;
+        size_t ro = 0;
+        if (ok) ro = (size_t)((bq * N + scan_to_token(p0 + t, H, W, dir)) * heads + hq);
+        const __half *src = ten == 0 ? q + ro * 64 : (ten == 1 ? g + ro * 64 : o + ro * 64);
+        const uint32_t d = ten == 0 ? dst_q : (ten == 1 ? dst_g : dst_o);
+        cp_async16(d + t * 128 + 16 * pc, src + 8 * pc, ok ? 16u : 0u);
+    }
+    cp_async_commit();
+}
+
+// Phase 4 (all threads; groups A's 256 threads compute): Qint * D_c of a chunk from
+// its raw q, g rows (qs, gs: unswizzled) and the decay product D_c from the span start
+// (dc), into the swizzled K-major tile dst.  Thread layout as in gating.  (Out of
+// line: once per span.)
+__device__ __noinline__ void rebuild_qd(uint8_t *sm, const uint8_t *qs, const uint8_t *gs,
+                                        const float *dc, uint8_t *dst) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    float *htot = reinterpret_cast<float *>(sm + L::htot);
+    const int gI = warp >> 1, ghf = warp & 1, gt0 = 16 * gI + 8 * ghf, gh = 2 * gI + ghf;
+    float pl[8][2];
+    if (warp < 8) {
+        float r0 = 1.f, r1 = 1.f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const float2 gv = ld_h2(gs + (gt0 + u) * 128 + 4 * lane);
+            r0 *= exp_f(gv.x);
+            r1 *= exp_f(gv.y);
+            pl[u][0] = r0; pl[u][1] = r1;
+        }
+        *reinterpret_cast<float2 *>(htot + gh * 64 + 2 * lane) = make_float2(r0, r1);
+    }
+    __syncthreads();
+    if (warp < 8) {
+        float bf0 = 1.f, bf1 = 1.f;
+        for (int h8 = 0; h8 < gh; ++h8) {
+            const float2 x = *reinterpret_cast<const float2 *>(htot + h8 * 64 + 2 * lane);
+            bf0 *= x.x;
+            bf1 *= x.y;
+        }
+        const float D0 = dc[2 * lane] * bf0, D1 = dc[2 * lane + 1] * bf1;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const float2 qv = ld_h2(qs + (gt0 + u) * 128 + 4 * lane);
+            st_h2(dst + sw_off(gt0 + u, 2 * lane), qv.x * pl[u][0] * D0, qv.y * pl[u][1] * D1);
+        }
+    }
+}
+
 template <int NL>
 __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(const Params P, const Work Wk) {
     constexpr int kThreads = span_threads<NL>();
@@ -862,6 +921,17 @@ __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(con
         }
         __syncthreads();
         // ---------------- phase 3: look back over the earlier spans
+        // Chunk kHold, the first past the held ones, is the one whose S_in term is
+        // usually not negligible: its q, g and stored output rows start loading now
+        // into the free V tiles, whether or not it turns out to need them.
+        // (Long spans only: the four-loader instance serves spans of at most
+        // kShortSpan <= kHold chunks.)
+        const bool ext = NL == 2 && later && hold == kHold && nch > kHold;
+        if constexpr (NL == 2) if (ext) {
+            const uint32_t vo = smem_u32(sm + L::vop);
+            load_qgo(P.q, P.g, P.out, P.N, P.H, P.W, P.dir, P.heads, seq, c0 + kHold, vo, vo + kTile,
+                     vo + 2 * kTile, kThreads);
+        }
         if (later) {
             if (tid < kspan) {
                 unsigned *f = Wk.flags + ((size_t)seq * PS + tid) * kFlagStride;
@@ -934,6 +1004,10 @@ __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(con
             // held chunks: their ring tiles hold Qint * D_c, so one B tile (S_in, fp16)
             // serves them all; the MMAs accumulate onto the chunks' outputs in TMEM
             if (hold > 0) {
+                // chunk kHold, if its term is not negligible, joins them: Qint * D_c rebuilt
+                // from the prefetched rows into qint, its correction into the work block,
+                // its stored output added in the epilogue
+                const bool xfix = ext && !(reinterpret_cast<const int *>(sm + L::skipf))[kHold];
                 uint8_t *bt = sm + L::sop;
                 for (int e = tid; e < kDK * kDV / 4; e += kThreads) {
                     const int i = e >> 4, c4 = e & 15;
@@ -941,6 +1015,10 @@ __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(con
                     *reinterpret_cast<uint2 *>(bt + sw_off(i, 4 * c4)) =
                         make_uint2(pack_half2(s.x, s.y), pack_half2(s.z, s.w));
                 }
+                if (ext) cp_async_wait_all();   // the prefetch has landed (needed or not)
+                __syncthreads();
+                if constexpr (NL == 2)
+                    if (xfix) rebuild_qd(sm, sm + L::vop, sm + L::vop + kTile, dcum + kHold * 64, sm + L::qint);
                 fence_proxy_async_cta();
                 __syncthreads();
                 if (warp == 0) {
@@ -955,6 +1033,12 @@ __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(con
                                 umma_f16(tmem + kColHold + 64 * ci, desc_sw128(qa + kk * 32, 16, 1024),
                                          desc_sw128(ba + kk * 2048, kTile, 1024), id, 1u);
                         }
+                        if (xfix) {
+#pragma unroll
+                            for (int kk = 0; kk < 4; ++kk)
+                                umma_f16(tmem + kColWork, desc_sw128(sbase + L::qint + kk * 32, 16, 1024),
+                                         desc_sw128(ba + kk * 2048, kTile, 1024), id, kk > 0 ? 1u : 0u);
+                        }
                         umma_commit(bar(sm, B_FIX));
                     }
                     __syncwarp();
@@ -962,16 +1046,17 @@ __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(con
                 wait_l(bar(sm, B_FIX), n_fix & 1u, to);
                 ++n_fix;
                 tc_fence_after();
-                // epilogues: three teams of four warps, held chunk ci on team ci % 3
+                // epilogues: three teams of four warps, chunk ci on team ci % 3
                 if (warp < 12) {
                     const int team = warp >> 2, tb = tid - 128 * team, bw = warp & 3;
                     int *rows = rowb + 64 * team;
                     uint8_t *os = sm + L::stg + team * kTile;
-                    for (int ci = team; ci < hold; ci += 3) {
+                    for (int ci = team; ci < hold + (xfix ? 1 : 0); ci += 3) {
+                        const bool x = ci == hold;   // chunk kHold: correction + stored output
                         fill_rows(P, seq, c0 + ci, rows, tb);
                         named_sync(3 + team, 128);
-                        store_chunk_out(P, tmem, kColHold + 64 * ci, bw, lane, tb, nullptr, 3 + team, os,
-                                        rows);
+                        store_chunk_out(P, tmem, x ? kColWork : kColHold + 64 * ci, bw, lane, tb,
+                                        x ? sm + L::vop + 2 * kTile : nullptr, 3 + team, os, rows);
                     }
                 }
                 __syncthreads();
@@ -980,58 +1065,72 @@ __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(con
             // (spans after the first have at most kMaxSpan chunks)
             const int *skipf = reinterpret_cast<const int *>(sm + L::skipf);
             for (int ci = hold; ci < nch; ++ci) {
-                if (skipf[ci]) continue;
-                // load q, g, o rows of this chunk (all threads), rebuild Q * P * D_c
-                {
+                if (skipf[ci] || (ext && ci == kHold)) continue;   // (chunk kHold done above)
+                // load q, g, o rows of this chunk (all threads), rebuild Q * P * D_c (long
+                // spans: out of line, which measured faster there; short spans keep the
+                // inline form, which measured faster for them)
+                if constexpr (NL == 2) {
                     const uint32_t stq = smem_u32(sm + L::stg);
-                    const int bq = seq / P.heads, hq = seq - bq * P.heads;
-                    const int p0 = (c0 + ci) * kChunk;
-                    for (int x = tid; x < 3 * 64 * 8; x += kThreads) {
-                        const int ten = x / 512, rem = x - ten * 512, t = rem >> 3, pc = rem & 7;
-                        const bool ok = p0 + t < P.N;
-                        size_t ro = 0;
-                        if (ok) ro = (size_t)((bq * P.N + scan_to_token(p0 + t, P.H, P.W, P.dir)) * P.heads + hq);
-                        const __half *src = ten == 0 ? P.q + ro * 64 : (ten == 1 ? P.g + ro * 64 : P.out + ro * 64);
-                        const int slot = ten == 0 ? 0 : (ten == 1 ? 2 : 3);
-                        cp_async16(stq + slot * kTile + t * 128 + 16 * pc, src + 8 * pc, ok ? 16u : 0u);
-                    }
-                    cp_async_commit();
+                    load_qgo(P.q, P.g, P.out, P.N, P.H, P.W, P.dir, P.heads, seq, c0 + ci, stq,
+                             stq + 2 * kTile, stq + 3 * kTile, kThreads);
                     cp_async_wait_all();
-                }
-                __syncthreads();
-                {
-                    // 256 threads: (half-block, channel pair) as in gating; products from the
-                    // chunk start
-                    float *htot = reinterpret_cast<float *>(sm + L::htot);
-                    const int gI = warp >> 1, ghf = warp & 1, gt0 = 16 * gI + 8 * ghf, gh = 2 * gI + ghf;
-                    float pl[8][2];
-                    if (warp < 8) {
-                        float r0 = 1.f, r1 = 1.f;
-#pragma unroll
-                        for (int u = 0; u < 8; ++u) {
-                            const float2 gv = ld_h2(sm + L::stg + 2 * kTile + (gt0 + u) * 128 + 4 * lane);
-                            r0 *= exp_f(gv.x);
-                            r1 *= exp_f(gv.y);
-                            pl[u][0] = r0; pl[u][1] = r1;
+                    __syncthreads();
+                    rebuild_qd(sm, sm + L::stg, sm + L::stg + 2 * kTile, dcum + ci * 64, sm + L::qint);
+                } else {
+                    // load q, g, o rows of this chunk (all threads), rebuild Q * P * D_c
+                    {
+                        const uint32_t stq = smem_u32(sm + L::stg);
+                        const int bq = seq / P.heads, hq = seq - bq * P.heads;
+                        const int p0 = (c0 + ci) * kChunk;
+                        for (int x = tid; x < 3 * 64 * 8; x += kThreads) {
+                            const int ten = x / 512, rem = x - ten * 512, t = rem >> 3, pc = rem & 7;
+                            const bool ok = p0 + t < P.N;
+                            size_t ro = 0;
+                            if (ok) ro = (size_t)((bq * P.N + scan_to_token(p0 + t, P.H, P.W, P.dir)) * P.heads + hq);
+                            const __half *src = ten == 0 ? P.q + ro * 64 : (ten == 1 ? P.g + ro * 64 : P.out + ro * 64);
+                            const int slot = ten == 0 ? 0 : (ten == 1 ? 2 : 3);
+                            cp_async16(stq + slot * kTile + t * 128 + 16 * pc, src + 8 * pc, ok ? 16u : 0u);
                         }
-                        *reinterpret_cast<float2 *>(htot + gh * 64 + 2 * lane) = make_float2(r0, r1);
+                        cp_async_commit();
+                        cp_async_wait_all();
                     }
                     __syncthreads();
-                    if (warp < 8) {
-                        float bf0 = 1.f, bf1 = 1.f;
-                        for (int h8 = 0; h8 < gh; ++h8) {
-                            const float2 x = *reinterpret_cast<const float2 *>(htot + h8 * 64 + 2 * lane);
-                            bf0 *= x.x;
-                            bf1 *= x.y;
+                    {
+                        // 256 threads: (half-block, channel pair) as in gating; products from the
+                        // chunk start
+                        float *htot = reinterpret_cast<float *>(sm + L::htot);
+                        const int gI = warp >> 1, ghf = warp & 1, gt0 = 16 * gI + 8 * ghf, gh = 2 * gI + ghf;
+                        float pl[8][2];
+                        if (warp < 8) {
+                            float r0 = 1.f, r1 = 1.f;
+    #pragma unroll
+                            for (int u = 0; u < 8; ++u) {
+                                const float2 gv = ld_h2(sm + L::stg + 2 * kTile + (gt0 + u) * 128 + 4 * lane);
+                                r0 *= exp_f(gv.x);
+                                r1 *= exp_f(gv.y);
+                                pl[u][0] = r0; pl[u][1] = r1;
+                            }
+                            *reinterpret_cast<float2 *>(htot + gh * 64 + 2 * lane) = make_float2(r0, r1);
                         }
-                        const float D0 = dcum[ci * 64 + 2 * lane] * bf0, D1 = dcum[ci * 64 + 2 * lane + 1] * bf1;
-                        uint8_t *qo = sm + L::qint;
-#pragma unroll
-                        for (int u = 0; u < 8; ++u) {
-                            const float2 qv = ld_h2(sm + L::stg + (gt0 + u) * 128 + 4 * lane);
-                            st_h2(qo + sw_off(gt0 + u, 2 * lane), qv.x * pl[u][0] * D0, qv.y * pl[u][1] * D1);
+                        __syncthreads();
+                        if (warp < 8) {
+                            float bf0 = 1.f, bf1 = 1.f;
+                            for (int h8 = 0; h8 < gh; ++h8) {
+                                const float2 x = *reinterpret_cast<const float2 *>(htot + h8 * 64 + 2 * lane);
+                                bf0 *= x.x;
+                                bf1 *= x.y;
+                            }
+                            const float D0 = dcum[ci * 64 + 2 * lane] * bf0, D1 = dcum[ci * 64 + 2 * lane + 1] * bf1;
+                            uint8_t *qo = sm + L::qint;
+    #pragma unroll
+                            for (int u = 0; u < 8; ++u) {
+                                const float2 qv = ld_h2(sm + L::stg + (gt0 + u) * 128 + 4 * lane);
+                                st_h2(qo + sw_off(gt0 + u, 2 * lane), qv.x * pl[u][0] * D0, qv.y * pl[u][1] * D1);
+                            }
                         }
                     }
+                }
+                {
                     // S_in as the fp16 operand
                     uint8_t *bt = sm + L::sop;
                     for (int e = tid; e < kDK * kDV / 4; e += kThreads) {
