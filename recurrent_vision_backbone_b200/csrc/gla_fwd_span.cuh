@@ -725,6 +725,41 @@ __device__ __noinline__ void rebuild_qd(uint8_t *sm, const uint8_t *qs, const ui
     }
 }
 
+// Group B (warps 8-11): the state update S <- d * S + dS of a chunk (as group A's,
+// with 32 elements per thread: warp bw reads TMEM lanes of quarter bw, all 64 columns)
+// into the fp32 tile and to `agg`.  Used by the short-span instance for the span's last
+// chunk, which group B reaches first (its held chunks need no epilogue in phase 1).
+__device__ __forceinline__ void update_state_b(uint8_t *sm, uint32_t tmem, int b, bool slow, float *agg,
+                                               int bw, int lane) {
+    const int row0 = 16 * bw + (lane >> 2), col0 = 2 * (lane & 3);
+    uint32_t r0[16], r1[16];
+    const uint32_t ta = tmem + ((uint32_t)(32 * bw) << 16) + kColDS + 64 * b;
+    tmem_ld_16x256b_x4(ta, r0);
+    tmem_ld_16x256b_x4(ta + 32, r1);
+    tmem_ld_wait();
+    const float *dloc = reinterpret_cast<const float *>(sm + L::dloc + b * 256);
+    uint8_t *sst = sm + L::sst;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int i = row0 + 8 * h;
+        const float di = dloc[i];
+        const float scl = slow ? 1.f : di;
+#pragma unroll
+        for (int x = 0; x < 2; ++x)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int col = col0 + 8 * j + 32 * x;
+                const uint32_t *rr = x ? r1 : r0;
+                float2 *sp2 = reinterpret_cast<float2 *>(sst + agg_off(i, col >> 2) + (col & 3) * 4);
+                const float2 sv = *sp2;
+                const float2 sn = make_float2(fmaf(di, sv.x, scl * __uint_as_float(rr[4 * j + 2 * h])),
+                                              fmaf(di, sv.y, scl * __uint_as_float(rr[4 * j + 2 * h + 1])));
+                *sp2 = sn;
+                if (agg != nullptr) *reinterpret_cast<float2 *>(agg + i * kDV + col) = sn;
+            }
+    }
+}
+
 template <int NL>
 __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(const Params P, const Work Wk) {
     constexpr int kThreads = span_threads<NL>();
@@ -827,6 +862,8 @@ __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(con
                 }
                 if (it > 0) {
                     wait_phase(bar(sm, B_MMA1 + (b ^ 1)), m1s[b ^ 1], (b ? m1b0 : m1b1) + ((it - 1) >> 1), to);
+                    if constexpr (NL == 4)
+                        if (it == nch) break;   // the last update is group B's
                     const bool pub = agg != nullptr && it == nch;
                     update_state_a(sm, tmem, b ^ 1, slow_prev, it < nch ? sm + L::sop + b * kTile : nullptr,
                                    pub ? agg : nullptr);
@@ -899,6 +936,23 @@ __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(con
                         umma_commit(bar(sm, B_VE + c % 3));  // V tile free
                     }
                     __syncwarp();
+                }
+                if constexpr (NL == 4) {
+                    if (c == nch - 1) {
+                        // the span's last update (group A's ended with chunk c-1's, which
+                        // warp 8 has seen: S_prev of chunk c), then the publish
+                        named_sync(kBarB, kThreadsB);
+                        tc_fence_after();
+                        const bool slw = *misc_slow(sm, b) != 0;
+                        update_state_b(sm, tmem, b, slw, agg, bw, lane);
+                        if (agg != nullptr) {
+                            if (tb < 64) agg[kDK * kDV + tb] = dcum[nch * 64 + tb];
+                            named_sync(kBarB, kThreadsB);
+                            if (tb == 0)   // readers to come: spans kspan+1 .. PS-1
+                                st_release_gpu(Wk.flags + ((size_t)seq * PS + kspan) * kFlagStride,
+                                               (unsigned)(PS - 1 - kspan));
+                        }
+                    }
                 }
                 wait_l(bar(sm, B_MMA2), m2_seen & 1u, to);
                 ++m2_seen;
