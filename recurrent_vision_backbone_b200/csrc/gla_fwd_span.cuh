@@ -760,6 +760,25 @@ __device__ __forceinline__ void update_state_b(uint8_t *sm, uint32_t tmem, int b
     }
 }
 
+// L2 prefetch of row x (of 128) of the first two chunks of the span that CTA `blk`
+// runs first: its q, k, g and v rows.  It is issued before the wait on the grid
+// ahead on the stream: a prefetch moves nothing into the SM and L2 is where every
+// SM's accesses meet, so a later write by that grid still reaches this grid's loads.
+__device__ __forceinline__ void prefetch_span_rows(const Params &P, const Work &Wk, int blk, int x) {
+    const int PS = Wk.P, kspan = blk % PS, seq = blk / PS;
+    if (seq >= P.n_seq) return;
+    const int c0 = kspan * Wk.Lc;
+    if (x >= min(min(Wk.Lc, P.n_chunks - c0), 2) * kChunk) return;
+    const int p = c0 * kChunk + x;
+    if (p >= P.N) return;
+    const int bb = seq / P.heads, hh = seq - bb * P.heads;
+    const size_t ro = ((size_t)bb * P.N + scan_to_token(p, P.H, P.W, P.dir)) * P.heads + hh;
+    prefetch_l2(P.q + ro * kDK);
+    prefetch_l2(P.k + ro * kDK);
+    prefetch_l2(P.g + ro * kDK);
+    prefetch_l2(P.v + ro * kDV);
+}
+
 template <int NL>
 __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(const Params P, const Work Wk) {
     constexpr int kThreads = span_threads<NL>();
@@ -777,6 +796,10 @@ __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(con
     float *cmeta = reinterpret_cast<float *>(sm + L::cmeta);
     int *rowb = reinterpret_cast<int *>(sm + L::rowb);
 
+    // first data into L2 while the grid ahead finishes: this CTA's span and the span
+    // of the CTA dispatched last (likely the last to find a free SM)
+    if (tid >= 128 && tid < 384)
+        prefetch_span_rows(P, Wk, tid < 256 ? (int)blockIdx.x : (int)(gridDim.x - 1 - blockIdx.x), tid & 127);
     if (warp == 0) {
         tmem_alloc(tmem_slot, kSpanTmemCols);
         tmem_relinquish();
@@ -974,6 +997,122 @@ __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(con
             for (int c = 0; c < nch; ++c) loader_load<NL>(P, sm, seq, c0, c, lane, warp - 12, nuse, nvuse, to);
         }
         __syncthreads();
+        if constexpr (NL == 4) {
+            // ---------------- phases 3-5 of a later span of at most kShortSpan chunks
+            // Every chunk is held (hold == nch): the S_in term needs only the fp16 S_in
+            // tile, and the last span's final state D_span * S_in + S_local is written
+            // as S_in is formed, so S_in never goes through shared memory in fp32.
+            if (later) {
+                // row tables of each epilogue team's first chunk, while the flags come in
+                if (warp < 12 && (warp >> 2) < hold)
+                    fill_rows(P, seq, c0 + (warp >> 2), rowb + 64 * (warp >> 2), tid - 128 * (warp >> 2));
+                if (tid < kspan) {
+                    unsigned *f = Wk.flags + ((size_t)seq * PS + tid) * kFlagStride;
+                    if (flag_wait_bounded(f, kWaitLimitNs)) {
+                        red_dec_gpu(f);   // one reader fewer to come
+                    } else {
+                        to = true;
+                        set_error(kErrTimeout);
+                    }
+                }
+                __syncthreads();
+                // S_in = sum_j (prod_{l>j} D_l) * S_j by Horner over j = 0 .. kspan-1; each
+                // thread forms two float4 of it (rows i and i + 32), two aggregates' loads
+                // in flight for both at a time
+                static_assert(kDK * kDV / 4 == 2 * kThreads, "two float4 of S_in per thread");
+                {
+                    const float *wseq = Wk.ws + (size_t)seq * PS * kAggFloats;
+                    const int e0 = tid, e1 = tid + kThreads;
+                    const int i0 = e0 >> 4, i1 = e1 >> 4, c4 = e0 & 15;
+                    float4 s0 = make_float4(0.f, 0.f, 0.f, 0.f), s1 = s0;
+                    for (int j0 = 0; j0 < kspan; j0 += 2) {
+                        float4 a0[2], a1[2];
+                        float d0[2], d1[2];
+#pragma unroll
+                        for (int u = 0; u < 2; ++u) {
+                            if (j0 + u < kspan) {
+                                const float *wj = wseq + (size_t)(j0 + u) * kAggFloats;
+                                a0[u] = __ldcg(reinterpret_cast<const float4 *>(wj) + e0);
+                                a1[u] = __ldcg(reinterpret_cast<const float4 *>(wj) + e1);
+                                d0[u] = __ldcg(wj + kDK * kDV + i0);
+                                d1[u] = __ldcg(wj + kDK * kDV + i1);
+                            }
+                        }
+#pragma unroll
+                        for (int u = 0; u < 2; ++u) {
+                            if (j0 + u < kspan) {   // (D_j <= 1: the zero start stays zero)
+                                s0.x = fmaf(d0[u], s0.x, a0[u].x);
+                                s0.y = fmaf(d0[u], s0.y, a0[u].y);
+                                s0.z = fmaf(d0[u], s0.z, a0[u].z);
+                                s0.w = fmaf(d0[u], s0.w, a0[u].w);
+                                s1.x = fmaf(d1[u], s1.x, a1[u].x);
+                                s1.y = fmaf(d1[u], s1.y, a1[u].y);
+                                s1.z = fmaf(d1[u], s1.z, a1[u].z);
+                                s1.w = fmaf(d1[u], s1.w, a1[u].w);
+                            }
+                        }
+                    }
+                    uint8_t *bt = sm + L::sop;
+                    *reinterpret_cast<uint2 *>(bt + sw_off(i0, 4 * c4)) =
+                        make_uint2(pack_half2(s0.x, s0.y), pack_half2(s0.z, s0.w));
+                    *reinterpret_cast<uint2 *>(bt + sw_off(i1, 4 * c4)) =
+                        make_uint2(pack_half2(s1.x, s1.y), pack_half2(s1.z, s1.w));
+                    if (kspan == PS - 1 && P.sf != nullptr) {
+                        // final state of the sequence: D_span * S_in + S_local
+                        const uint8_t *sst = sm + L::sst;
+                        float4 f0 = *reinterpret_cast<const float4 *>(sst + agg_off(i0, c4));
+                        float4 f1 = *reinterpret_cast<const float4 *>(sst + agg_off(i1, c4));
+                        const float g0 = dcum[nch * 64 + i0], g1 = dcum[nch * 64 + i1];
+                        f0.x = fmaf(g0, s0.x, f0.x);
+                        f0.y = fmaf(g0, s0.y, f0.y);
+                        f0.z = fmaf(g0, s0.z, f0.z);
+                        f0.w = fmaf(g0, s0.w, f0.w);
+                        f1.x = fmaf(g1, s1.x, f1.x);
+                        f1.y = fmaf(g1, s1.y, f1.y);
+                        f1.z = fmaf(g1, s1.z, f1.z);
+                        f1.w = fmaf(g1, s1.w, f1.w);
+                        float4 *sf = reinterpret_cast<float4 *>(P.sf + (size_t)seq * kDK * kDV);
+                        sf[e0] = f0;
+                        sf[e1] = f1;
+                    }
+                }
+                fence_proxy_async_cta();
+                __syncthreads();
+                // the term for every chunk: one MMA per chunk onto its output in TMEM
+                if (warp == 0) {
+                    tc_fence_after();
+                    if (elect_one_sync()) {
+                        constexpr uint32_t id = idesc_f16_f32(64, kDV, false, true);
+                        const uint32_t ba = sbase + L::sop;
+                        for (int ci = 0; ci < hold; ++ci) {
+                            const uint32_t qa = sbase + L::ring + ci * kTile;
+#pragma unroll
+                            for (int kk = 0; kk < 4; ++kk)
+                                umma_f16(tmem + kColHold + 64 * ci, desc_sw128(qa + kk * 32, 16, 1024),
+                                         desc_sw128(ba + kk * 2048, kTile, 1024), id, 1u);
+                        }
+                        umma_commit(bar(sm, B_FIX));
+                    }
+                    __syncwarp();
+                }
+                wait_l(bar(sm, B_FIX), n_fix & 1u, to);
+                ++n_fix;
+                tc_fence_after();
+                // epilogues: three teams of four warps, chunk ci on team ci % 3
+                if (warp < 12) {
+                    const int team = warp >> 2, tb = tid - 128 * team, bw = warp & 3;
+                    int *rows = rowb + 64 * team;
+                    uint8_t *os = sm + L::stg + team * kTile;
+                    for (int ci = team; ci < hold; ci += 3) {
+                        if (ci != team) {   // (the first chunk's rows are in place)
+                            fill_rows(P, seq, c0 + ci, rows, tb);
+                            named_sync(3 + team, 128);
+                        }
+                        store_chunk_out(P, tmem, kColHold + 64 * ci, bw, lane, tb, nullptr, 3 + team, os, rows);
+                    }
+                }
+            }
+        }
         // ---------------- phase 3: look back over the earlier spans
         // Chunk kHold, the first past the held ones, is the one whose S_in term is
         // usually not negligible: its q, g and stored output rows start loading now
@@ -986,7 +1125,7 @@ __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(con
             load_qgo(P.q, P.g, P.out, P.N, P.H, P.W, P.dir, P.heads, seq, c0 + kHold, vo, vo + kTile,
                      vo + 2 * kTile, kThreads);
         }
-        if (later) {
+        if (NL == 2 && later) {
             if (tid < kspan) {
                 unsigned *f = Wk.flags + ((size_t)seq * PS + tid) * kFlagStride;
                 if (flag_wait_bounded(f, kWaitLimitNs)) {
@@ -1053,7 +1192,7 @@ __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(con
         }
 
         // ---------------- phase 4: add the S_in term to this span's outputs
-        if (later) {
+        if (NL == 2 && later) {
             const float *sin = reinterpret_cast<const float *>(sm + L::sin);
             // held chunks: their ring tiles hold Qint * D_c, so one B tile (S_in, fp16)
             // serves them all; the MMAs accumulate onto the chunks' outputs in TMEM
@@ -1223,7 +1362,7 @@ __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(con
         }
 
         // ---------------- phase 5: final state of the sequence
-        if (kspan == PS - 1 && P.sf != nullptr) {
+        if (kspan == PS - 1 && P.sf != nullptr && (NL == 2 || !later)) {
             const float *sst = reinterpret_cast<const float *>(sm + L::sst);
             const float *sin = reinterpret_cast<const float *>(sm + L::sin);
             for (int e = tid; e < kDK * kDV / 4; e += kThreads) {

@@ -112,6 +112,11 @@ __device__ __forceinline__ bool elect_one_sync() {
     return is_leader != 0;
 }
 
+// Brings the 128-byte line holding `p` (global memory) into L2; nothing reaches the SM.
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(__cvta_generic_to_global(p)));
+}
+
 __device__ __forceinline__ void tc_fence_before() {
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
