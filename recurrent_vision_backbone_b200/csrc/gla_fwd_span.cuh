@@ -616,6 +616,9 @@ __device__ __forceinline__ void store_p_tmem(uint8_t *sm, uint32_t tmem, const B
 // chunk cr+1's MMA 2) and to `agg` (the span's published aggregate) when non-null.
 // Warp w reads TMEM lanes of quarter w % 4 (rows 16 (w % 4) ..) and columns
 // 32 (w / 4) ..: 16 elements per thread.  Ends with group A past its writes.
+// kLoadFirst: every load of the state tile before any store, so that the loads
+// overlap (faster where registers allow: the short-span instance).
+template <bool kLoadFirst>
 __device__ __forceinline__ void update_state_a(uint8_t *sm, uint32_t tmem, int b, bool slow,
                                                uint8_t *so_next, float *agg) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -628,6 +631,16 @@ __device__ __forceinline__ void update_state_a(uint8_t *sm, uint32_t tmem, int b
     tmem_ld_wait();
     const float *dloc = reinterpret_cast<const float *>(sm + L::dloc + b * 256);
     uint8_t *sst = sm + L::sst;
+    float2 sv[2][4];
+    if constexpr (kLoadFirst) {
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                const int i = rrow0 + 8 * hh, col = rcol0 + 8 * cc;
+                sv[hh][cc] = *reinterpret_cast<const float2 *>(sst + agg_off(i, col >> 2) + (col & 3) * 4);
+            }
+    }
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
         const int i = rrow0 + 8 * hh;
@@ -637,7 +650,7 @@ __device__ __forceinline__ void update_state_a(uint8_t *sm, uint32_t tmem, int b
         for (int cc = 0; cc < 4; ++cc) {
             const int col = rcol0 + 8 * cc;
             float2 *sp2 = reinterpret_cast<float2 *>(sst + agg_off(i, col >> 2) + (col & 3) * 4);
-            const float2 s = *sp2;
+            const float2 s = kLoadFirst ? sv[hh][cc] : *sp2;
             const float2 sn = make_float2(fmaf(di, s.x, scl * __uint_as_float(rd[4 * cc + 2 * hh])),
                                           fmaf(di, s.y, scl * __uint_as_float(rd[4 * cc + 2 * hh + 1])));
             *sp2 = sn;
@@ -739,6 +752,17 @@ __device__ __forceinline__ void update_state_b(uint8_t *sm, uint32_t tmem, int b
     tmem_ld_wait();
     const float *dloc = reinterpret_cast<const float *>(sm + L::dloc + b * 256);
     uint8_t *sst = sm + L::sst;
+    // every load of the state before any store, so that the loads overlap
+    float2 sq[2][2][4];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int x = 0; x < 2; ++x)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int i = row0 + 8 * h, col = col0 + 8 * j + 32 * x;
+                sq[h][x][j] = *reinterpret_cast<const float2 *>(sst + agg_off(i, col >> 2) + (col & 3) * 4);
+            }
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
         const int i = row0 + 8 * h;
@@ -751,7 +775,7 @@ __device__ __forceinline__ void update_state_b(uint8_t *sm, uint32_t tmem, int b
                 const int col = col0 + 8 * j + 32 * x;
                 const uint32_t *rr = x ? r1 : r0;
                 float2 *sp2 = reinterpret_cast<float2 *>(sst + agg_off(i, col >> 2) + (col & 3) * 4);
-                const float2 sv = *sp2;
+                const float2 sv = sq[h][x][j];
                 const float2 sn = make_float2(fmaf(di, sv.x, scl * __uint_as_float(rr[4 * j + 2 * h])),
                                               fmaf(di, sv.y, scl * __uint_as_float(rr[4 * j + 2 * h + 1])));
                 *sp2 = sn;
@@ -777,6 +801,17 @@ __device__ __forceinline__ void prefetch_span_rows(const Params &P, const Work &
     prefetch_l2(P.k + ro * kDK);
     prefetch_l2(P.g + ro * kDK);
     prefetch_l2(P.v + ro * kDV);
+}
+
+// The span's aggregate state from the fp32 state tile in shared memory to the
+// workspace (row-major), nthr threads with consecutive indices from 0: whole float4
+// per thread, consecutive threads on consecutive 16 bytes.  (Group A's publish: a
+// second pass over the tile measured faster than its update's scattered 8-byte
+// stores; group B's four warps store straight from the update.)
+__device__ __forceinline__ void store_aggregate(const uint8_t *sm, float *agg, int t, int nthr) {
+    const uint8_t *sst = sm + L::sst;
+    for (int e = t; e < kDK * kDV / 4; e += nthr)
+        reinterpret_cast<float4 *>(agg)[e] = *reinterpret_cast<const float4 *>(sst + agg_off(e >> 4, e & 15));
 }
 
 template <int NL>
@@ -888,9 +923,10 @@ __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(con
                     if constexpr (NL == 4)
                         if (it == nch) break;   // the last update is group B's
                     const bool pub = agg != nullptr && it == nch;
-                    update_state_a(sm, tmem, b ^ 1, slow_prev, it < nch ? sm + L::sop + b * kTile : nullptr,
-                                   pub ? agg : nullptr);
+                    update_state_a<NL == 4>(sm, tmem, b ^ 1, slow_prev, it < nch ? sm + L::sop + b * kTile : nullptr,
+                                   nullptr);
                     if (pub) {
+                        store_aggregate(sm, agg, tid, kThreadsA);
                         // aggregate = (state reached from zero, product of the span's decays)
                         // (the CTA barrier orders every thread's stores before thread 0's
                         // release at gpu scope)
