@@ -945,7 +945,9 @@ __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(con
             int *rows2 = rowb + 2 * 64;
             for (int c = 0; c < nch; ++c) {
                 const int b = c & 1;
-                const bool held = c < hold;
+                // (spans of at most kShortSpan chunks hold every chunk's output in TMEM,
+                // span 0's too: its epilogues wait until it has published)
+                const bool held = NL == 4 || c < hold;
                 fill_rows(P, seq, c0 + c, rows2, tb);
                 wait_l(bar(sm, B_GATE + b), (g_seen >> b) & 1u, to);   // bit b: parity of GATE[b]
                 g_seen ^= 1u << b;
@@ -1144,6 +1146,19 @@ __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(con
                             fill_rows(P, seq, c0 + ci, rows, tb);
                             named_sync(3 + team, 128);
                         }
+                        store_chunk_out(P, tmem, kColHold + 64 * ci, bw, lane, tb, nullptr, 3 + team, os, rows);
+                    }
+                }
+            } else {
+                // span 0: its outputs, complete in TMEM (group B saw every MMA 2 complete)
+                tc_fence_after();
+                if (warp < 12) {
+                    const int team = warp >> 2, tb = tid - 128 * team, bw = warp & 3;
+                    int *rows = rowb + 64 * team;
+                    uint8_t *os = sm + L::stg + team * kTile;
+                    for (int ci = team; ci < nch; ci += 3) {
+                        fill_rows(P, seq, c0 + ci, rows, tb);
+                        named_sync(3 + team, 128);
                         store_chunk_out(P, tmem, kColHold + 64 * ci, bw, lane, tb, nullptr, 3 + team, os, rows);
                     }
                 }
