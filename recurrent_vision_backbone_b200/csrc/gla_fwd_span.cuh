@@ -51,6 +51,7 @@ __host__ __device__ constexpr int span_threads() { return kThreadsA + kThreadsB 
 constexpr int kShortSpan = 4;
 constexpr int kDK = 64;
 constexpr int kHold = 4;                    // chunks per span whose outputs wait in TMEM
+static_assert(kShortSpan <= kHold, "a short span holds every chunk's output in TMEM");
 constexpr int kMaxSpan = 32;                // chunks of a span with recorded decays
 constexpr uint32_t kBarA = 1, kBarB = 2;    // named barriers; 3..5: phase-4 epilogue teams
 constexpr uint32_t kBarPro = 6;             // groups A and B: sequence prologue
