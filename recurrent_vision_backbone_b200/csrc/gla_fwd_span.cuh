@@ -1045,51 +1045,61 @@ __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(con
                 // row tables of each epilogue team's first chunk, while the flags come in
                 if (warp < 12 && (warp >> 2) < hold)
                     fill_rows(P, seq, c0 + (warp >> 2), rowb + 64 * (warp >> 2), tid - 128 * (warp >> 2));
-                if (tid < kspan) {
-                    unsigned *f = Wk.flags + ((size_t)seq * PS + tid) * kFlagStride;
-                    if (flag_wait_bounded(f, kWaitLimitNs)) {
-                        red_dec_gpu(f);   // one reader fewer to come
-                    } else {
-                        to = true;
-                        set_error(kErrTimeout);
-                    }
-                }
-                __syncthreads();
-                // S_in = sum_j (prod_{l>j} D_l) * S_j by Horner over j = 0 .. kspan-1; each
-                // thread forms two float4 of it (rows i and i + 32), two aggregates' loads
-                // in flight for both at a time
+                // S_in = sum_j (prod_{l>j} D_l) * S_j by Horner over j = 0 .. kspan-1, from
+                // the aggregates copied into the phase-1 buffers below the S_in operand
+                // tile (kFoldSlots at a time): warp u waits for span j0 + u's flag and copies
+                // that aggregate at once (cp.async, no registers held), so the copies
+                // overlap the flags' arrival; then each thread forms two float4 of S_in
+                // (rows i and i + 32) from shared memory.
                 static_assert(kDK * kDV / 4 == 2 * kThreads, "two float4 of S_in per thread");
+                constexpr int kAggBytes = kAggFloats * 4;
+                constexpr int kFoldSlots = L::sop / kAggBytes;
+                static_assert(kFoldSlots >= 1 && kAggBytes % 16 == 0, "fold slots");
                 {
                     const float *wseq = Wk.ws + (size_t)seq * PS * kAggFloats;
                     const int e0 = tid, e1 = tid + kThreads;
                     const int i0 = e0 >> 4, i1 = e1 >> 4, c4 = e0 & 15;
                     float4 s0 = make_float4(0.f, 0.f, 0.f, 0.f), s1 = s0;
-                    for (int j0 = 0; j0 < kspan; j0 += 2) {
-                        float4 a0[2], a1[2];
-                        float d0[2], d1[2];
-#pragma unroll
-                        for (int u = 0; u < 2; ++u) {
-                            if (j0 + u < kspan) {
-                                const float *wj = wseq + (size_t)(j0 + u) * kAggFloats;
-                                a0[u] = __ldcg(reinterpret_cast<const float4 *>(wj) + e0);
-                                a1[u] = __ldcg(reinterpret_cast<const float4 *>(wj) + e1);
-                                d0[u] = __ldcg(wj + kDK * kDV + i0);
-                                d1[u] = __ldcg(wj + kDK * kDV + i1);
+                    for (int j0 = 0; j0 < kspan; j0 += kFoldSlots) {
+                        const int nj = min(kFoldSlots, kspan - j0);
+                        for (int u = warp; u < nj; u += kThreads / 32) {
+                            unsigned *f = Wk.flags + ((size_t)seq * PS + j0 + u) * kFlagStride;
+                            int ok = 1;
+                            if (lane == 0) {
+                                ok = flag_wait_bounded(f, kWaitLimitNs) ? 1 : 0;
+                                if (ok) {
+                                    red_dec_gpu(f);   // one reader fewer to come
+                                } else {
+                                    to = true;
+                                    set_error(kErrTimeout);
+                                }
+                            }
+                            // (the warp's copies follow lane 0's acquire)
+                            ok = __shfl_sync(0xffffffffu, ok, 0);
+                            if (ok) {
+                                const float *src = wseq + (size_t)(j0 + u) * kAggFloats;
+                                const uint32_t dst = sbase + u * kAggBytes;
+                                for (int x = lane; x < kAggBytes / 16; x += 32) cp_async16(dst + 16 * x, src + 4 * x, 16);
                             }
                         }
-#pragma unroll
-                        for (int u = 0; u < 2; ++u) {
-                            if (j0 + u < kspan) {   // (D_j <= 1: the zero start stays zero)
-                                s0.x = fmaf(d0[u], s0.x, a0[u].x);
-                                s0.y = fmaf(d0[u], s0.y, a0[u].y);
-                                s0.z = fmaf(d0[u], s0.z, a0[u].z);
-                                s0.w = fmaf(d0[u], s0.w, a0[u].w);
-                                s1.x = fmaf(d1[u], s1.x, a1[u].x);
-                                s1.y = fmaf(d1[u], s1.y, a1[u].y);
-                                s1.z = fmaf(d1[u], s1.z, a1[u].z);
-                                s1.w = fmaf(d1[u], s1.w, a1[u].w);
-                            }
+                        cp_async_commit();
+                        cp_async_wait_all();
+                        __syncthreads();
+                        for (int u = 0; u < nj; ++u) {   // (D_j <= 1: the zero start stays zero)
+                            const float *a = reinterpret_cast<const float *>(sm + u * kAggBytes);
+                            const float4 a0 = reinterpret_cast<const float4 *>(a)[e0];
+                            const float4 a1 = reinterpret_cast<const float4 *>(a)[e1];
+                            const float d0 = a[kDK * kDV + i0], d1 = a[kDK * kDV + i1];
+                            s0.x = fmaf(d0, s0.x, a0.x);
+                            s0.y = fmaf(d0, s0.y, a0.y);
+                            s0.z = fmaf(d0, s0.z, a0.z);
+                            s0.w = fmaf(d0, s0.w, a0.w);
+                            s1.x = fmaf(d1, s1.x, a1.x);
+                            s1.y = fmaf(d1, s1.y, a1.y);
+                            s1.z = fmaf(d1, s1.z, a1.z);
+                            s1.w = fmaf(d1, s1.w, a1.w);
                         }
+                        if (j0 + kFoldSlots < kspan) __syncthreads();   // the slots are reused
                     }
                     uint8_t *bt = sm + L::sop;
                     *reinterpret_cast<uint2 *>(bt + sw_off(i0, 4 * c4)) =
