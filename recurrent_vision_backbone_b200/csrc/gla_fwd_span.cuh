@@ -743,6 +743,10 @@ __device__ __noinline__ void rebuild_qd(uint8_t *sm, const uint8_t *qs, const ui
 // with 32 elements per thread: warp bw reads TMEM lanes of quarter bw, all 64 columns)
 // into the fp32 tile and to `agg`.  Used by the short-span instance for the span's last
 // chunk, which group B reaches first (its held chunks need no epilogue in phase 1).
+// `agg` is written in fragment order, so that every warp store is 512 contiguous
+// bytes: float4 number 256 k + s holds, for slot s = 32 w + l (w < 8: quarter w % 4,
+// column half w / 4; l a lane), row 16 (w % 4) + l / 4 + 8 (k / 2) and columns
+// c, c + 1, c + 8, c + 9 with c = 32 (w / 4) + 2 (l % 4) + 16 (k % 2).
 __device__ __forceinline__ void update_state_b(uint8_t *sm, uint32_t tmem, int b, bool slow, float *agg,
                                                int bw, int lane) {
     const int row0 = 16 * bw + (lane >> 2), col0 = 2 * (lane & 3);
@@ -770,18 +774,23 @@ __device__ __forceinline__ void update_state_b(uint8_t *sm, uint32_t tmem, int b
         const float di = dloc[i];
         const float scl = slow ? 1.f : di;
 #pragma unroll
-        for (int x = 0; x < 2; ++x)
+        for (int x = 0; x < 2; ++x) {
+            const uint32_t *rr = x ? r1 : r0;
+            float2 sn[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int col = col0 + 8 * j + 32 * x;
-                const uint32_t *rr = x ? r1 : r0;
-                float2 *sp2 = reinterpret_cast<float2 *>(sst + agg_off(i, col >> 2) + (col & 3) * 4);
                 const float2 sv = sq[h][x][j];
-                const float2 sn = make_float2(fmaf(di, sv.x, scl * __uint_as_float(rr[4 * j + 2 * h])),
-                                              fmaf(di, sv.y, scl * __uint_as_float(rr[4 * j + 2 * h + 1])));
-                *sp2 = sn;
-                if (agg != nullptr) *reinterpret_cast<float2 *>(agg + i * kDV + col) = sn;
+                sn[j] = make_float2(fmaf(di, sv.x, scl * __uint_as_float(rr[4 * j + 2 * h])),
+                                    fmaf(di, sv.y, scl * __uint_as_float(rr[4 * j + 2 * h + 1])));
+                *reinterpret_cast<float2 *>(sst + agg_off(i, col >> 2) + (col & 3) * 4) = sn[j];
             }
+            if (agg != nullptr) {
+                float4 *a4 = reinterpret_cast<float4 *>(agg) + 32 * (bw + 4 * x) + lane;
+                a4[2 * h * 256] = make_float4(sn[0].x, sn[0].y, sn[1].x, sn[1].y);
+                a4[(2 * h + 1) * 256] = make_float4(sn[2].x, sn[2].y, sn[3].x, sn[3].y);
+            }
+        }
     }
 }
 
@@ -1050,7 +1059,8 @@ __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(con
                 // tile (kFoldSlots at a time): warp u waits for span j0 + u's flag and copies
                 // that aggregate at once (cp.async, no registers held), so the copies
                 // overlap the flags' arrival; then each thread forms two float4 of S_in
-                // (rows i and i + 32) from shared memory.
+                // from shared memory (fragment order, as group B's update stores the
+                // aggregates: rows i and i + 8, columns c, c + 1, c + 8, c + 9).
                 static_assert(kDK * kDV / 4 == 2 * kThreads, "two float4 of S_in per thread");
                 constexpr int kAggBytes = kAggFloats * 4;
                 constexpr int kFoldSlots = L::sop / kAggBytes;
@@ -1058,7 +1068,9 @@ __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(con
                 {
                     const float *wseq = Wk.ws + (size_t)seq * PS * kAggFloats;
                     const int e0 = tid, e1 = tid + kThreads;
-                    const int i0 = e0 >> 4, i1 = e1 >> 4, c4 = e0 & 15;
+                    const int sl = tid & 255, fw = sl >> 5, fl = sl & 31;
+                    const int i0 = 16 * (fw & 3) + (fl >> 2), i1 = i0 + 8;
+                    const int ca = 32 * (fw >> 2) + 2 * (fl & 3) + 16 * (tid >> 8), cb = ca + 8;
                     float4 s0 = make_float4(0.f, 0.f, 0.f, 0.f), s1 = s0;
                     for (int j0 = 0; j0 < kspan; j0 += kFoldSlots) {
                         const int nj = min(kFoldSlots, kspan - j0);
@@ -1102,27 +1114,23 @@ __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(con
                         if (j0 + kFoldSlots < kspan) __syncthreads();   // the slots are reused
                     }
                     uint8_t *bt = sm + L::sop;
-                    *reinterpret_cast<uint2 *>(bt + sw_off(i0, 4 * c4)) =
-                        make_uint2(pack_half2(s0.x, s0.y), pack_half2(s0.z, s0.w));
-                    *reinterpret_cast<uint2 *>(bt + sw_off(i1, 4 * c4)) =
-                        make_uint2(pack_half2(s1.x, s1.y), pack_half2(s1.z, s1.w));
+                    *reinterpret_cast<uint32_t *>(bt + sw_off(i0, ca)) = pack_half2(s0.x, s0.y);
+                    *reinterpret_cast<uint32_t *>(bt + sw_off(i0, cb)) = pack_half2(s0.z, s0.w);
+                    *reinterpret_cast<uint32_t *>(bt + sw_off(i1, ca)) = pack_half2(s1.x, s1.y);
+                    *reinterpret_cast<uint32_t *>(bt + sw_off(i1, cb)) = pack_half2(s1.z, s1.w);
                     if (kspan == PS - 1 && P.sf != nullptr) {
                         // final state of the sequence: D_span * S_in + S_local
                         const uint8_t *sst = sm + L::sst;
-                        float4 f0 = *reinterpret_cast<const float4 *>(sst + agg_off(i0, c4));
-                        float4 f1 = *reinterpret_cast<const float4 *>(sst + agg_off(i1, c4));
+                        const auto st2 = [&](int i, int col) {
+                            return *reinterpret_cast<const float2 *>(sst + agg_off(i, col >> 2) + (col & 3) * 4);
+                        };
                         const float g0 = dcum[nch * 64 + i0], g1 = dcum[nch * 64 + i1];
-                        f0.x = fmaf(g0, s0.x, f0.x);
-                        f0.y = fmaf(g0, s0.y, f0.y);
-                        f0.z = fmaf(g0, s0.z, f0.z);
-                        f0.w = fmaf(g0, s0.w, f0.w);
-                        f1.x = fmaf(g1, s1.x, f1.x);
-                        f1.y = fmaf(g1, s1.y, f1.y);
-                        f1.z = fmaf(g1, s1.z, f1.z);
-                        f1.w = fmaf(g1, s1.w, f1.w);
-                        float4 *sf = reinterpret_cast<float4 *>(P.sf + (size_t)seq * kDK * kDV);
-                        sf[e0] = f0;
-                        sf[e1] = f1;
+                        const float2 f0a = st2(i0, ca), f0b = st2(i0, cb), f1a = st2(i1, ca), f1b = st2(i1, cb);
+                        float *sf = P.sf + (size_t)seq * kDK * kDV;
+                        *reinterpret_cast<float2 *>(sf + i0 * kDV + ca) = make_float2(fmaf(g0, s0.x, f0a.x), fmaf(g0, s0.y, f0a.y));
+                        *reinterpret_cast<float2 *>(sf + i0 * kDV + cb) = make_float2(fmaf(g0, s0.z, f0b.x), fmaf(g0, s0.w, f0b.y));
+                        *reinterpret_cast<float2 *>(sf + i1 * kDV + ca) = make_float2(fmaf(g1, s1.x, f1a.x), fmaf(g1, s1.y, f1a.y));
+                        *reinterpret_cast<float2 *>(sf + i1 * kDV + cb) = make_float2(fmaf(g1, s1.z, f1b.x), fmaf(g1, s1.w, f1b.y));
                     }
                 }
                 fence_proxy_async_cta();
