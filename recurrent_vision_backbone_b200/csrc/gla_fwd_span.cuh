@@ -841,10 +841,11 @@ __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(con
     float *cmeta = reinterpret_cast<float *>(sm + L::cmeta);
     int *rowb = reinterpret_cast<int *>(sm + L::rowb);
 
-    // first data into L2 while the grid ahead finishes: this CTA's span and the span
-    // of the CTA dispatched last (likely the last to find a free SM)
-    if (tid >= 128 && tid < 384)
-        prefetch_span_rows(P, Wk, tid < 256 ? (int)blockIdx.x : (int)(gridDim.x - 1 - blockIdx.x), tid & 127);
+    // first data into L2 while the grid ahead finishes: this CTA's span and, for long
+    // spans, the span of the CTA dispatched last (likely the last to find a free SM;
+    // for short spans the extra traffic measured slower)
+    if (tid >= 128 && (NL == 2 ? tid < 384 : tid < 256))
+        prefetch_span_rows(P, Wk, NL == 2 && tid >= 256 ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x, tid & 127);
     if (warp == 0) {
         tmem_alloc(tmem_slot, kSpanTmemCols);
         tmem_relinquish();
