@@ -77,13 +77,40 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def _code_tokens(src: str) -> str:
+    """C++ source without comments, whitespace runs collapsed (string and character
+    literals kept verbatim): edits to comments or layout leave it unchanged."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            i = src.find("\n", i)
+            i = n if i < 0 else i
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def kernel_source_hash() -> str:
+    """Hash of the kernel sources' code (comments and layout excluded), recorded next
+    to the ncu counters in profiles/ so that a stale capture is not reported."""
     h = hashlib.sha1()
     csrc = os.path.join(ROOT, "recurrent_vision_backbone_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
         if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as fh:
-                h.update(fh.read())
+            with open(os.path.join(csrc, name), encoding="utf-8") as fh:
+                h.update(_code_tokens(fh.read()).encode())
     return h.hexdigest()[:12]
 
 

@@ -20,11 +20,16 @@
 //                                 scores' TMEM columns, is complete by then), then the
 //                                 scores of chunk c from TMEM into the causal fp16
 //                                 P tile, written back to TMEM, MMA 2(c) = Qint S_prev
-//                                 + P V (P as the TMEM A operand), output stores;
+//                                 + P V (P as the TMEM A operand), output stores
+//                                 (spans of at most kShortSpan chunks, span 0 included,
+//                                 keep every output in TMEM until phase 4);
 //   phase 2  the span's last state update publishes its aggregate (state reached
-//            from zero, product of the decays) to the workspace.
+//            from zero, product of the decays) to the workspace (in short spans group
+//            B does that update, right after its last MMA 2).
 //   phase 3  look back: fold the aggregates of the earlier spans into S_in, the true
-//            state entering this span.
+//            state entering this span (short spans: each aggregate is copied into
+//            shared memory as soon as its flag is seen, and the fold writes the fp16
+//            operand of phase 4 directly).
 //   phase 4  correct the outputs for the missing S_in term.  For a chunk c starting
 //            D_c (per key channel, product of the decays since the span start) into the
 //            span, the term is (Q * P) diag(D_c) S_in.  The first kHold chunks keep
