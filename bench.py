@@ -27,6 +27,7 @@ import os
 import re
 import statistics
 import subprocess
+import tempfile
 import sys
 import time
 
@@ -139,14 +140,21 @@ class ClockSampler:
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, path=None):
+        """Samples the GPU's clocks every 100 ms while the timed region runs; the raw
+        samples go to `path` (a CSV) if given, else to a temporary file."""
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+        self.temporary = path is None
+        if path is None:
+            fd, path = tempfile.mkstemp(prefix=f"clocks_gpu{gpu_index}_", suffix=".csv")
+            os.close(fd)
+        self.path = path
 
     def start(self):
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            if os.path.dirname(self.path):
+                os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
@@ -157,6 +165,8 @@ class ClockSampler:
 
     def stop(self):
         if self.proc is None:
+            if self.temporary and os.path.exists(self.path):
+                os.unlink(self.path)
             return None
         self.proc.terminate()
         try:
@@ -178,6 +188,8 @@ class ClockSampler:
             for name, flag in zip(names, parts[5:9]):
                 if flag.lower() == "active":
                     reasons.add(name)
+        if self.temporary:
+            os.unlink(self.path)
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
@@ -399,7 +411,7 @@ def gpu_arm(args):
     w1 = WORKLOADS[primary]
     wl = Workload(w1, rank, device, n_sets=args.sets)
     clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
-                          else local)
+                          else local, args.clocks_csv)
     clocks.start()
     ms, n_steps = measure(wl, args.steps, args.warmup, stream, world)
     clk = clocks.stop()
@@ -545,6 +557,8 @@ def main():
                     help="rotating input sets (default: enough to exceed 4x L2); small "
                          "profiler captures use fewer")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--clocks-csv", default=None,
+                    help="keep the raw nvidia-smi clock samples of the timed region in this CSV")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
