@@ -60,6 +60,8 @@ def load_library(path: str) -> ctypes.CDLL:
     lib.gla_oracle_scan_to_token.restype = ctypes.c_long
     lib.gla_oracle_scan_to_token.argtypes = [ctypes.c_long, ctypes.c_int, ctypes.c_int,
                                              ctypes.c_int]
+    lib.gla_oracle_gate.restype = ctypes.c_int
+    lib.gla_oracle_gate.argtypes = [dp, ctypes.c_long, ctypes.c_double, dp]
     lib.gla_oracle_max_threads.restype = ctypes.c_int
     lib.gla_oracle_set_threads.argtypes = [ctypes.c_int]
     return lib
@@ -128,3 +130,21 @@ def gla_forward(q, k, v, g, H: int, W: int, direction: int, s0=None,
     if rc != 0:
         raise RuntimeError(f"gla_oracle_fwd_range failed with code {rc}")
     return o, sf
+
+
+def gate(z, tau: float, lib=None) -> np.ndarray:
+    """Log-decay of the key-side forget gate from its pre-activation:
+    g = log(sigmoid(z)) / tau, in fp64, elementwise (any shape)."""
+    lib = lib or _get()
+    za = _f64(z)
+    g = np.empty_like(za)
+    rc = lib.gla_oracle_gate(_ptr(za), za.size, float(tau), _ptr(g))
+    if rc != 0:
+        raise RuntimeError(f"gla_oracle_gate failed with code {rc}")
+    return g
+
+
+def gla_forward_z(q, k, v, z, tau: float, H: int, W: int, direction: int, s0=None):
+    """The forward pass with the gate given by its pre-activation z (fp64 gate, then
+    the same recurrence as gla_forward)."""
+    return gla_forward(q, k, v, gate(z, tau), H, W, direction, s0)

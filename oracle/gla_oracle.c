@@ -153,3 +153,26 @@ void gla_oracle_set_threads(int n)
     (void)n;
 #endif
 }
+
+/*
+ * Key-side forget gate from its pre-activation z (GTR news article, section
+ * "线性注意力到底在省什么": a learnable forget gate on the key side; the gate value is
+ * a = sigmoid(z)^(1/tau), so its log-decay is g = log(sigmoid(z)) / tau).
+ *
+ *   log(sigmoid(z)) = -log(1 + exp(-z))
+ *
+ * evaluated as min(z, 0) - log1p(exp(-|z|)): the two forms are equal for either sign
+ * of z (for z < 0, -log(1 + e^-z) = z - log(e^z + 1)), and this one never overflows.
+ * Writes n values of g.  Returns 0, or -1 on a bad argument.
+ */
+int gla_oracle_gate(const double *z, long n, double tau, double *g)
+{
+    if ((!z || !g) && n > 0) return -1;
+    if (n < 0 || !(tau > 0.0)) return -1;
+    for (long i = 0; i < n; ++i) {
+        const double x = z[i];
+        const double ls = (x < 0.0 ? x : 0.0) - log1p(exp(-fabs(x)));
+        g[i] = ls / tau;
+    }
+    return 0;
+}
