@@ -115,14 +115,18 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:12]
 
 
-# the kernel every dk = 64 call of the bench workloads launches
-KERNEL = "gla_fwd_span_kernel"
+def kernel_for(w) -> str:
+    """The kernel a call of workload w launches (one launch per call)."""
+    if w.dk != 64:
+        return "gla_fwd_kernel"
+    return "gla_fwd_pipe_kernel" if os.environ.get("GTR_KERNEL") == "pipe" else "gla_fwd_span_kernel"
 
 
 def recorded_traffic(workload_name: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on the
     current kernel source; else None."""
-    path = os.path.join(ROOT, "profiles", f"{KERNEL}_{workload_name}.md")
+    kernel = kernel_for(WORKLOADS[workload_name])
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload_name}.md")
     try:
         text = open(path).read()
     except OSError:
@@ -252,17 +256,31 @@ class Workload:
             self.gla.gtr_gla_fwd(inp["q"], inp["k"], inp["v"], inp["g"], self.w.H, self.w.W, d,
                                  init_state=inp["s0"], out=out, final_state=sf, stream=stream)
 
-    def capture(self, stream):
-        # warm the launch path once outside capture
-        with torch.cuda.stream(stream):
+    def capture(self, stream, steps):
+        """Graphs replaying the rotating sets: `full` holds one step per set, `part` the
+        first steps % n_sets of them, so that any step count is replayed exactly."""
+        with torch.cuda.stream(stream):   # warm the launch path once outside capture
             self.launch_step(0, stream)
         stream.synchronize()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            for s in range(self.n_sets):
-                self.launch_step(s, torch.cuda.current_stream())
-        self.graph = g
-        return self.n_sets  # steps per replay
+
+        def graph_of(n):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for s in range(n):
+                    self.launch_step(s, torch.cuda.current_stream())
+            return g
+
+        self.graph = graph_of(self.n_sets)
+        r = steps % self.n_sets
+        self.part = graph_of(r) if r else None
+        return self.n_sets
+
+    def replay(self, steps):
+        """Replays exactly `steps` steps (whole rotations, then the remainder)."""
+        for _ in range(steps // self.n_sets):
+            self.graph.replay()
+        if steps % self.n_sets:
+            self.part.replay()
 
     def calls_per_step(self):
         return len(self.w.call_directions())
@@ -271,15 +289,14 @@ class Workload:
         return self.calls_per_step() * self.w.B * self.w.N
 
 
-def timed_replays(wl, replays, stream, world):
+def timed_replays(wl, steps, stream, world):
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     with torch.cuda.stream(stream):   # replay on the stream the events are recorded on
         start.record(stream)
-        for _ in range(replays):
-            wl.graph.replay()
+        wl.replay(steps)
         end.record(stream)
     torch.cuda.synchronize()
     if world > 1:
@@ -287,26 +304,36 @@ def timed_replays(wl, replays, stream, world):
     return max_over_ranks(start.elapsed_time(end), world, "cuda")
 
 
-def measure(wl, steps, warmup, stream, world):
-    per_replay = wl.capture(stream)
-    replays = max(1, -(-steps // per_replay))
-    warm = max(1, -(-warmup // per_replay))
+def measure(wl, steps, warmup, stream, world, clocks=None, clock_window_s=1.0):
+    """W warm-up steps, then exactly `steps` timed steps.  With a clock sampler, the
+    samples cover a window of at least `clock_window_s` of the same replays that ends
+    with the timed region (a timed region of a few ms holds no 100 ms sample)."""
+    per_replay = wl.capture(stream, steps)
     with torch.cuda.stream(stream):
-        for _ in range(warm):
-            wl.graph.replay()
+        wl.replay(max(warmup, 1))
     torch.cuda.synchronize()
     assert wl.gla.device_status() == wl.gla.GTR_OK
-    ms = timed_replays(wl, replays, stream, world)
+    clk = None
+    if clocks is not None:
+        # size the untimed lead-in from one timed rotation
+        t_rot = timed_replays(wl, per_replay, stream, world) * 1e-3
+        lead = max(0, int(clock_window_s / max(t_rot, 1e-6)) + 1)
+        clocks.start()
+        with torch.cuda.stream(stream):
+            for _ in range(lead):
+                wl.graph.replay()
+    ms = timed_replays(wl, steps, stream, world)
+    if clocks is not None:
+        clk = clocks.stop()
     assert wl.gla.device_status() == wl.gla.GTR_OK
-    n_steps = replays * per_replay
-    return ms, n_steps
+    return ms, steps, clk
 
 
 def roofline(w, ms_per_launch, workload_name):
     peak, which = measured_peaks()
     b = bytes_alg(w)
     achieved = b / (ms_per_launch * 1e-3) / 1e9
-    return {"kernel": KERNEL, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+    return {"kernel": kernel_for(w), "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
             "unit": "GB/s",
             "frac": round(achieved / peak, 4), "traffic": recorded_traffic(workload_name),
             "peak_source": which, "bytes_alg_per_launch": b, "flops_alg_per_launch": flops_alg(w)}
@@ -394,6 +421,46 @@ def e2e_measure(w, steps, device, rank):
     return ms, steps, h2d, d2h
 
 
+def config_of(w, world, l2_note, timing):
+    """The line's `config` (the same keys in both arms)."""
+    return {"workload": w.name, "B": w.B, "heads": w.heads, "grid": [w.H, w.W],
+            "tokens_per_call": w.B * w.N, "dk": w.dk, "dv": w.dv, "chunk": 64,
+            "calls_per_step": len(w.call_directions()),
+            "directions": ",".join(DIR_NAMES[d] for d in w.call_directions()),
+            "l2": l2_note, "timing": timing,
+            "parallelism": f"dp{world} (independent batches)"}
+
+
+def run_workload(name, steps, warmup, stream, world, rank, device, sets, sample_clocks, local,
+                 clocks_csv=None):
+    """Times `steps` steps of one workload; returns its numbers and its config."""
+    w = WORKLOADS[name]
+    wl = Workload(w, rank, device, n_sets=sets)
+    clocks = None
+    if sample_clocks:
+        clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
+                              else local, clocks_csv)
+    ms, n_steps, clk = measure(wl, steps, warmup, stream, world, clocks)
+    launches = n_steps * wl.calls_per_step()
+    res = {"workload": name, "tokens_per_call": w.B * w.N,
+           "value": round(world * wl.tokens_per_step() * n_steps / (ms * 1e-3), 1),
+           "unit": "tokens/s", "steps": n_steps, "ms_per_step": round(ms / n_steps, 6),
+           "us_per_call": round(ms * 1e3 / launches, 3),
+           "roofline": roofline(w, ms / launches, name), "gpu_launches": launches,
+           "clocks": clk}
+    l2 = (f"inputs rotate over {wl.n_sets} sets of {wl.calls_per_step()} calls "
+          f"({wl.n_sets * wl.calls_per_step() * bytes_alg(w) / 2**20:.0f} MiB > 3x L2)")
+    cfg = config_of(w, world, l2, "CUDA graph replay (exactly `steps` steps), CUDA events, "
+                                  "max over ranks; clocks sampled over >= 1 s of the same "
+                                  "replays ending with the timed region")
+    del wl
+    torch.cuda.empty_cache()
+    return res, cfg
+
+
+SECONDARIES = ("hires_b1h16_128x128", "b8h16_48x48_stack12", "stress_b4h12_37x53_dk128")
+
+
 def gpu_arm(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -409,52 +476,29 @@ def gpu_arm(args):
     stream = torch.cuda.Stream(device=device)
     primary = args.workload
     w1 = WORKLOADS[primary]
-    wl = Workload(w1, rank, device, n_sets=args.sets)
-    clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
-                          else local, args.clocks_csv)
-    clocks.start()
-    ms, n_steps = measure(wl, args.steps, args.warmup, stream, world)
-    clk = clocks.stop()
-    launches = n_steps * wl.calls_per_step()
-    wl_calls = wl.calls_per_step()
-    ms_step = ms / n_steps
-    value = world * wl.tokens_per_step() * n_steps / (ms * 1e-3)
+    res, cfg = run_workload(primary, args.steps, args.warmup, stream, world, rank, device,
+                            args.sets, True, local, args.clocks_csv)
     line = {
-        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
-        "steps": n_steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 6),
+        "metric": METRIC, "value": res["value"], "unit": "tokens/s", "n_gpus": world,
+        "steps": res["steps"], "warmup": args.warmup, "ms_per_step": res["ms_per_step"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
-        "data": "synthetic",
-        "config": {"workload": primary, "B": w1.B, "heads": w1.heads, "grid": [w1.H, w1.W],
-                   "tokens_per_call": w1.B * w1.N, "dk": w1.dk, "dv": w1.dv, "chunk": 64,
-                   "calls_per_step": wl.calls_per_step(),
-                   "directions": ",".join(DIR_NAMES[d] for d in w1.call_directions()),
-                   "l2": f"inputs rotate over {wl.n_sets} sets of {wl.calls_per_step()} calls "
-                         f"({wl.n_sets * wl.calls_per_step() * bytes_alg(w1) / 2**20:.0f} MiB"
-                         f" > 3x L2)",
-                   "timing": "CUDA graph replay, CUDA events, max over ranks",
-                   "parallelism": f"dp{world} (independent batches)"},
-        "roofline": roofline(w1, ms / launches, primary),
-        "gpu_launches": launches,
-        "clocks": clk,
+        "data": "synthetic", "config": cfg, "roofline": res["roofline"],
+        "gpu_launches": res["gpu_launches"], "clocks": res["clocks"],
+        "us_per_call": res["us_per_call"],
     }
-    del wl
-    torch.cuda.empty_cache()
-    if not args.no_secondary and primary != SECONDARY:
-        w2 = WORKLOADS[SECONDARY]
-        wl2 = Workload(w2, rank, device, n_sets=args.sets)
-        ms2, n2 = measure(wl2, max(8, args.steps // 16), max(3, args.warmup // 16), stream, world)
-        line["secondary"] = {
-            "workload": SECONDARY, "tokens_per_call": w2.B * w2.N,
-            "value": round(world * wl2.tokens_per_step() * n2 / (ms2 * 1e-3), 1),
-            "unit": "tokens/s", "steps": n2, "ms_per_step": round(ms2 / n2, 6),
-            "roofline": roofline(w2, ms2 / (n2 * wl2.calls_per_step()), SECONDARY),
-            "gpu_launches": n2 * wl2.calls_per_step()}
-        del wl2
-        torch.cuda.empty_cache()
+    if not args.no_secondary:
+        line["secondary"] = []
+        for name in SECONDARIES:
+            if name == primary:
+                continue
+            r2, _ = run_workload(name, max(8, args.steps // 16), max(3, args.warmup // 16), stream,
+                                 world, rank, device, args.sets, True, local)
+            line["secondary"].append(r2)
     # end to end through the public call with host buffers
     e_steps = max(3, min(args.steps, args.e2e_steps))
     ems, en, h2d, d2h = e2e_measure(w1, e_steps, device, rank)
     ems = max_over_ranks(ems, world, "cuda")
+    wl_calls = len(w1.call_directions())
     line["e2e"] = {"value": round(world * wl_calls * w1.B * w1.N * en / (ems * 1e-3), 1),
                    "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                    "steps": en}
@@ -533,8 +577,8 @@ def reference_arm(args):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(spent / args.steps * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "B": w.B, "heads": w.heads, "grid": [w.H, w.W],
-                       "dk": w.dk, "dv": w.dv, "chunk": 64, "calls_per_step": len(dirs)},
+            "config": config_of(w, world, "host memory (no GPU L2 involved)",
+                                "wall clock of the oracle calls (time.perf_counter)"),
             "cpu_baseline": {"value": round(value, 1), "unit": "tokens/s", "cores": threads,
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": round(value, 1), "unit": "tokens/s", "h2d_bytes_per_step": 0,

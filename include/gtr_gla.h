@@ -34,15 +34,24 @@
  * Ownership: every buffer belongs to the caller; the library never frees or
  * keeps a pointer after a call returns.  All work is enqueued on `stream`
  * (a cudaStream_t, NULL = legacy default stream).  No call synchronises the host
- * except gtr_gla_device_status and the first gtr_gla_fwd call on a device that
- * needs a workspace (it allocates and zero-fills the library's cached one).
+ * except gtr_gla_device_status and the first gtr_gla_fwd_static call on a device.
  *
  * Workspace: for some shapes (dk = 64 with few sequences) one sequence is split
  * into spans that run on different SMs; they exchange one 16.6 KB aggregate per
  * span through a device workspace.  gtr_gla_fwd uses a workspace cached by the
- * library, one per device (about 5 MB), so gtr_gla_fwd calls on one device must
- * not run concurrently on different streams: such callers use gtr_gla_fwd_ws
- * with one workspace each.
+ * library, one per device (about 5 MB), allocated and zero-filled in stream order
+ * (cudaMallocAsync / cudaMemsetAsync on the caller's stream, no host wait) by the
+ * first call that needs it, or ahead of time by gtr_gla_init.  gtr_gla_fwd calls on
+ * one device must not run concurrently on different streams: such callers use
+ * gtr_gla_fwd_ws with one workspace each.
+ *
+ * Numeric range: the tensor-core operands are fp16, so the running state S (as the
+ * fp16 operand of the next chunk), the masked scores of a chunk and the outputs must
+ * stay below 65504 in magnitude; g must be <= 0 (the log of a forget gate in (0, 1]).
+ * A call whose state, scores or outputs leave that range records GTR_ERR_RANGE in the
+ * device error word (read by gtr_gla_device_status); its outputs are then unusable.
+ * (For inputs like the pages' -- q scaled by dk^-1/2, unit-variance k and v, decaying
+ * gates -- these values stay orders of magnitude below the limit.)
  *
  * Errors: argument checks run on the host before anything is enqueued and
  * return GTR_ERR_INVALID_ARG / GTR_ERR_UNSUPPORTED with nothing launched.
@@ -69,7 +78,8 @@ typedef enum {
     GTR_ERR_INVALID_ARG = 1,  /* null/negative/misaligned/overflowing/aliased arguments */
     GTR_ERR_UNSUPPORTED = 2,  /* valid but not built: chunk != 64, dk not in {64,128}, dv != 64 */
     GTR_ERR_CUDA = 3,         /* a CUDA runtime call or kernel launch failed */
-    GTR_ERR_TIMEOUT = 4       /* a bounded device-side wait ran out (see gtr_gla_device_status) */
+    GTR_ERR_TIMEOUT = 4,      /* a bounded device-side wait ran out (see gtr_gla_device_status) */
+    GTR_ERR_RANGE = 5         /* a value left the fp16 range (see "Numeric range" above) */
 } gtr_status_t;
 
 /*
@@ -92,6 +102,32 @@ gtr_status_t gtr_gla_fwd(const gtr_half_t *q, const gtr_half_t *k, const gtr_hal
                          int dk, int dv, int direction, int chunk,
                          const float *init_state, gtr_half_t *out, float *final_state,
                          void *stream);
+
+/*
+ * gtr_gla_fwd with the forget gate given by its pre-activation: the third input z
+ * (IEEE binary16 [B, N, heads, dk], in place of g) and the temperature tau > 0; the
+ * kernel forms g = log(sigmoid(z)) / tau = (min(z, 0) - log(1 + exp(-|z|))) / tau in
+ * fp32 while it stages each chunk (GTR news article, section "线性注意力到底在省什么":
+ * a learnable forget gate on the key side), so no separate pass over z runs and g is
+ * never rounded to fp16.  Same arguments, layouts, workspace and errors as gtr_gla_fwd,
+ * plus GTR_ERR_INVALID_ARG for tau <= 0 or not finite; dk must be 64 (else
+ * GTR_ERR_UNSUPPORTED).
+ */
+gtr_status_t gtr_gla_fwd_z(const gtr_half_t *q, const gtr_half_t *k, const gtr_half_t *v,
+                           const gtr_half_t *z, float tau, int B, int heads, int Hgrid, int Wgrid,
+                           int dk, int dv, int direction, int chunk,
+                           const float *init_state, gtr_half_t *out, float *final_state,
+                           void *stream);
+
+/*
+ * Allocates and zero-fills, in the order of `stream` (no host wait), the library's
+ * cached workspace of the current device, sized for every shape, so that no later
+ * gtr_gla_fwd call allocates.  Call it before capturing gtr_gla_fwd calls into a
+ * CUDA graph: a first allocation during a capture returns GTR_ERR_CUDA
+ * (cudaErrorStreamCaptureUnsupported) with nothing enqueued.  Calling it again is a
+ * no-op.  (No counterpart on the pages: this is the library's memory contract.)
+ */
+gtr_status_t gtr_gla_init(void *stream);
 
 /*
  * Bytes of workspace gtr_gla_fwd_ws needs for a shape on the current device
@@ -138,8 +174,10 @@ gtr_status_t gtr_gla_fwd_ws(const gtr_half_t *q, const gtr_half_t *k, const gtr_
  *     starts; every call that completes without a device error leaves them
  *     zero again), synchronising the host once.
  *     Make that first call before any stream capture begins.
- *   - Limit: a shape whose plan needs more than GTR_STATIC_WS_BYTES returns
- *     GTR_ERR_UNSUPPORTED with nothing launched.
+ *   - Limit: the call picks the cheapest launch plan whose workspace fits in
+ *     GTR_STATIC_WS_BYTES (one span per sequence needs none, so every shape that
+ *     gtr_gla_fwd accepts runs); only a plan forced past that size by the
+ *     GTR_CLUSTER_SIZE tuning variable falls back to another plan.
  *   - The scratch is shared by every gtr_gla_fwd_static call on the device:
  *     calls that overlap in time (different streams or host threads) race on it
  *     and give wrong results.  Calls in order on one stream are fine.
@@ -152,7 +190,7 @@ gtr_status_t gtr_gla_fwd_static(const gtr_half_t *q, const gtr_half_t *k, const 
 
 /*
  * Syncs `stream`, then reads and clears the device error word (and any sticky
- * CUDA error).  Returns GTR_OK, GTR_ERR_TIMEOUT or GTR_ERR_CUDA.  On
+ * CUDA error).  Returns GTR_OK, GTR_ERR_TIMEOUT, GTR_ERR_RANGE or GTR_ERR_CUDA.  On
  * GTR_ERR_TIMEOUT it also zero-fills the library's workspaces of the current
  * device (the cached one and the static scratch).
  */

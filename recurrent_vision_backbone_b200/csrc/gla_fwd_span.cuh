@@ -202,9 +202,9 @@ __device__ __forceinline__ void red_dec_gpu(unsigned *p) {   // *p -= 1, relaxed
 // Waits (acquire) until *f is non-zero, for at most limit_ns; false if the limit ran out.
 __device__ __forceinline__ bool flag_wait_bounded(const unsigned *f, uint64_t limit_ns) {
     if (ld_acquire_gpu(f) != 0u) return true;
-    const uint64_t t0 = globaltimer_ns();
+    const long long t0 = cycles(), lim = cycles_of_ns(limit_ns);
     while (ld_acquire_gpu(f) == 0u)
-        if (globaltimer_ns() - t0 > limit_ns) return false;
+        if (cycles() - t0 > lim) return false;
     return true;
 }
 

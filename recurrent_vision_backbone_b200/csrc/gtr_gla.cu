@@ -58,7 +58,8 @@ constexpr float kFastMaxK = 100.f;              // |k| / P stays inside fp16 on 
 constexpr float kDiagMaxQ = 20.f;               // |q| / T stays inside fp16 on a diagonal block
 constexpr uint64_t kWaitLimitNs = 200ull * 1000ull * 1000ull;  // 200 ms per bounded wait
 
-enum : unsigned { kErrTimeout = 1u };
+enum : unsigned { kErrTimeout = 1u, kErrRange = 2u };
+constexpr float kHalfMax = 65504.f;   // largest finite fp16
 
 __device__ unsigned int g_error_word;
 
@@ -732,14 +733,19 @@ __global__ void __launch_bounds__(kThreads, Smem<DK>::min_blocks) gla_fwd_kernel
 
 #include "gla_fwd_ws.cuh"
 #include "gla_fwd_span.cuh"
+#include "gla_fwd_pipe.cuh"
 
 namespace gtr {
 
 // ------------------------------------------------------------------ host
-enum KernelKind { kBasic64 = 0, kBasic128 = 1, kCluster = 2, kSpan = 3, kSpanShort = 4, kKinds = 5 };
+enum KernelKind { kBasic64 = 0, kBasic128 = 1, kCluster = 2, kSpan = 3, kSpanShort = 4, kPipe = 5, kPipeZ = 6,
+                  kKinds = 7 };
 
 // the span kernel with two loader warps (kSpan) or four (kSpanShort: short spans)
 static bool is_span(int kind) { return kind == kSpan || kind == kSpanShort; }
+// kernels whose CTAs of one sequence must be co-resident (cooperative launch)
+static bool is_pipe(int kind) { return kind == kPipe || kind == kPipeZ; }
+static bool is_coop(int kind) { return is_span(kind) || is_pipe(kind); }
 
 // A kernel variant: entry point, block size, dynamic shared memory, cache slot.
 struct KSpec {
@@ -771,6 +777,10 @@ static KSpec spec_of(int kind) {
     case kSpanShort:
         return KSpec{reinterpret_cast<const void *>(&sp::gla_fwd_span_kernel<4>), sp::span_threads<4>(),
                      sp::L::alloc, kSpanShort};
+    case kPipe:
+        return KSpec{reinterpret_cast<const void *>(&pp::gla_fwd_pipe_kernel<false>), pp::kThreads, pp::L::alloc, kPipe};
+    case kPipeZ:
+        return KSpec{reinterpret_cast<const void *>(&pp::gla_fwd_pipe_kernel<true>), pp::kThreads, pp::L::alloc, kPipeZ};
     default:
         return KSpec{reinterpret_cast<const void *>(&sp::gla_fwd_span_kernel<2>), sp::span_threads<2>(),
                      sp::L::alloc, kSpan};
@@ -783,6 +793,7 @@ static int kind_for(int dk, long n_chunks) {
     const char *e = getenv("GTR_KERNEL");
     if (e && !strcmp(e, "basic")) return kBasic64;
     if (e && !strcmp(e, "cluster") && n_chunks >= ws::kMinCluster) return kCluster;
+    if (e && !strcmp(e, "pipe")) return kPipe;
     return kSpan;
 }
 
@@ -827,7 +838,7 @@ static void fill_config(cudaLaunchConfig_t &cfg, cudaLaunchAttribute *attr, cons
     cfg.dynamicSmemBytes = (size_t)k.smem;
     cfg.stream = stream;
     cfg.attrs = attr;
-    if (is_span(k.slot)) {
+    if (is_coop(k.slot)) {
         // all spans of a sequence must be resident together: cooperative launch; the
         // next launch on the stream may start its set-up while this one drains (the
         // kernel waits for its predecessor before touching global memory)
@@ -908,15 +919,16 @@ static size_t span_ws_bytes(long n_seq, int spans, int cap) {
 // span groups within the co-resident capacity.  Minimises (sequence passes) x
 // (chunks per span + 2), the 2 standing for the look-back and the corrections;
 // several spans per sequence only while the sequences alone leave SMs idle.
-static Plan span_plan(long n_seq, long n_chunks, int cap) {
-    const KSpec k = spec_of(kSpan);
-    Plan best{kSpan, 1, 1, (int)n_chunks, k.smem, k.threads, 0};
+static Plan span_plan(long n_seq, long n_chunks, int cap, int kind, size_t ws_limit) {
+    const KSpec k = spec_of(kind);
+    Plan best{kind, 1, 1, (int)n_chunks, k.smem, k.threads, 0};
     long best_cost = -1;
     const int fc = forced_cluster();
     for (int P = 1; P <= kMaxCluster && P <= n_chunks && P <= cap; ++P) {
         const long Lc = (n_chunks + P - 1) / P;
         if ((n_chunks + Lc - 1) / Lc != P) continue;   // same split as a smaller P
         if (P > 1 && (Lc > sp::kMaxSpan || n_seq * P > 2L * cap)) continue;
+        if (span_ws_bytes(n_seq, P, cap) > ws_limit) continue;   // (P = 1 needs none)
         if (fc > 0 && P != fc) continue;
         const long groups = n_seq < cap / P ? n_seq : cap / P;
         const long passes = (n_seq + groups - 1) / groups;
@@ -929,11 +941,11 @@ static Plan span_plan(long n_seq, long n_chunks, int cap) {
         }
     }
     if (best_cost < 0 && fc > 0) {   // forced span count not feasible: plan freely
-        Plan p1{kSpan, 1, (int)(n_seq < cap ? n_seq : cap), (int)n_chunks, k.smem, k.threads, 0};
+        Plan p1{kind, 1, (int)(n_seq < cap ? n_seq : cap), (int)n_chunks, k.smem, k.threads, 0};
         return p1;
     }
     best.ws_bytes = span_ws_bytes(n_seq, best.cluster, cap);
-    if (best.cluster > 1 && best.span_len <= sp::kShortSpan) {   // latency-bound: four loaders
+    if (kind == kSpan && best.cluster > 1 && best.span_len <= sp::kShortSpan) {   // latency-bound: four loaders
         const KSpec ks = spec_of(kSpanShort);
         best.kind = kSpanShort;
         best.threads = ks.threads;
@@ -971,21 +983,24 @@ static Plan cluster_plan(int kind, long n_seq, long n_chunks, int dev, int sms, 
     return best;
 }
 
-static Plan make_plan(long n_seq, long n_chunks, int dk, bool query) {
-    const int kind = kind_for(dk, n_chunks);
+// ws_limit: the largest workspace the caller can provide (the static scratch's size
+// for gtr_gla_fwd_static; unlimited otherwise).
+static Plan make_plan(long n_seq, long n_chunks, int dk, bool query, size_t ws_limit = ~size_t(0),
+                      bool gate_z = false) {
+    const int kind = gate_z ? kPipeZ : kind_for(dk, n_chunks);
     const int dev = current_device();
     const int sms = num_sms(dev);
-    if (kind == kSpan) {
+    if (kind == kSpan || is_pipe(kind)) {
         const int cap = span_capacity(dev, sms, query);
-        if (cap > 0) return span_plan(n_seq, n_chunks, cap);
+        if (cap > 0) return span_plan(n_seq, n_chunks, cap, kind, ws_limit);
         return cluster_plan(kBasic64, n_seq, n_chunks, dev, sms, query);
     }
     return cluster_plan(kind, n_seq, n_chunks, dev, sms, query);
 }
 
 // Library-cached workspace of gtr_gla_fwd, one per device: sized for the largest
-// span plan (n_seq * spans <= 2 * capacity), allocated and zero-filled by the first
-// call that needs it.
+// span plan (n_seq * spans <= 2 * capacity), allocated and zero-filled, in the order of
+// the caller's stream, by the first call that needs it (or by gtr_gla_init).
 struct DefaultWs {
     void *ptr;
     size_t bytes;
@@ -1013,13 +1028,14 @@ static cudaError_t default_workspace(int dev, size_t need, cudaStream_t stream, 
     const int cap = g_span_capacity[dev] > 0 ? g_span_capacity[dev] : sms;
     size_t bytes = default_ws_bytes(cap);
     if (bytes < need) bytes = need;
+    // stream-ordered: the allocation and the zero fill run on the caller's stream ahead
+    // of the launch that needs them; the host does not wait
     void *p = nullptr;
-    e = cudaMalloc(&p, bytes);
+    e = cudaMallocAsync(&p, bytes, stream);
     if (e != cudaSuccess) return e;
-    e = cudaMemset(p, 0, bytes);
-    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    e = cudaMemsetAsync(p, 0, bytes, stream);
     if (e != cudaSuccess) {
-        cudaFree(p);
+        cudaFreeAsync(p, stream);
         return e;
     }
     w.ptr = p;
@@ -1032,14 +1048,162 @@ static thread_local cudaError_t g_last_cuda_error = cudaSuccess;
 
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-static cudaError_t launch(const Params &prm, const Plan &pl, void *workspace, cudaStream_t stream) {
+// ------------------------------------------------------------------ TMA maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+static EncodeTiledFn g_encode = nullptr;
+
+static cudaError_t tensor_map_encoder(EncodeTiledFn *fn) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_encode == nullptr) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        const cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+        if (e != cudaSuccess) return e;
+        if (q != cudaDriverEntryPointSuccess || p == nullptr) return cudaErrorNotSupported;
+        g_encode = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    *fn = g_encode;
+    return cudaSuccess;
+}
+
+// Box heights (bit h: 2^h rows) that the memory-contiguous runs of the chunks of a grid
+// scanned in `dir` decompose into: L->R reads whole 64-row boxes; R->L runs end at grid
+// rows, T->B and B->T at grid columns, every run also at chunk boundaries.
+static unsigned used_heights(int H, int W, int dir) {
+    if (dir == GTR_L2R) return 1u << 6;
+    const long N = (long)H * W, run = dir == GTR_R2L ? W : H;
+    unsigned m = 0;
+    for (long p0 = 0; p0 < N; p0 += kChunk) {
+        const long pend = p0 + kChunk < N ? p0 + kChunk : N;
+        for (long p = p0; p < pend;) {
+            const long q = (p / run + 1) * run < pend ? (p / run + 1) * run : pend;
+            m |= (unsigned)(q - p);
+            p = q;
+        }
+    }
+    return m & 0x7fu;
+}
+
+// One tensor ([B, N, heads, d] fp16) as a row view (d, heads, N, B) or a column view
+// (d, heads, W, H, B), box d x 1 x 2^h rows.
+static CUresult encode_map(EncodeTiledFn enc, CUtensorMap *m, const void *ptr, int B, int heads, int H, int W,
+                           int d, bool column, int h) {
+    const cuuint64_t es = 2;
+    cuuint64_t dims[5], strides[4];
+    cuuint32_t box[5], estr[5] = {1, 1, 1, 1, 1};
+    const cuuint64_t N = (cuuint64_t)H * W;
+    dims[0] = (cuuint64_t)d;
+    dims[1] = (cuuint64_t)heads;
+    strides[0] = (cuuint64_t)d * es;
+    strides[1] = (cuuint64_t)heads * d * es;
+    box[0] = (cuuint32_t)d;
+    box[1] = 1;
+    cuuint32_t rank;
+    if (!column) {
+        rank = 4;
+        dims[2] = N;
+        dims[3] = (cuuint64_t)B;
+        strides[2] = N * heads * d * es;
+        box[2] = 1u << h;
+        box[3] = 1;
+    } else {
+        rank = 5;
+        dims[2] = (cuuint64_t)W;
+        dims[3] = (cuuint64_t)H;
+        dims[4] = (cuuint64_t)B;
+        strides[2] = (cuuint64_t)W * heads * d * es;
+        strides[3] = N * heads * d * es;
+        box[2] = 1;
+        box[3] = 1u << h;
+        box[4] = 1;
+    }
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, rank, const_cast<void *>(ptr), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+// Encoded maps of the last few (tensors, shape, direction) combinations.
+struct MapEntry {
+    const void *ptr[4];
+    int B, heads, H, W, dir, dev;
+    unsigned used;
+    bool valid;
+    pp::Maps maps;
+};
+static MapEntry g_maps[32];
+static int g_maps_next;
+
+static cudaError_t pipe_maps(const Params &prm, int dev, pp::Maps *maps, unsigned *used) {
+    const void *ptr[4] = {prm.q, prm.k, prm.g, prm.v};
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        for (const MapEntry &m : g_maps) {
+            if (m.valid && m.dev == dev && m.B == prm.B && m.heads == prm.heads && m.H == prm.H && m.W == prm.W &&
+                m.dir == prm.dir && !memcmp(m.ptr, ptr, sizeof(ptr))) {
+                *maps = m.maps;
+                *used = m.used;
+                return cudaSuccess;
+            }
+        }
+    }
+    EncodeTiledFn enc = nullptr;
+    cudaError_t e = tensor_map_encoder(&enc);
+    if (e != cudaSuccess) return e;
+    MapEntry ent{};
+    memcpy(ent.ptr, ptr, sizeof(ptr));
+    ent.B = prm.B;
+    ent.heads = prm.heads;
+    ent.H = prm.H;
+    ent.W = prm.W;
+    ent.dir = prm.dir;
+    ent.dev = dev;
+    ent.used = used_heights(prm.H, prm.W, prm.dir);
+    const bool column = prm.dir == GTR_T2B || prm.dir == GTR_B2T;
+    for (int ten = 0; ten < 4; ++ten)
+        for (int h = 0; h < 7; ++h) {
+            if (!((ent.used >> h) & 1u)) continue;
+            if (encode_map(enc, &ent.maps.m[ten][h], ptr[ten], prm.B, prm.heads, prm.H, prm.W,
+                           ten == 3 ? kDV : pp::kDK, column, h) != CUDA_SUCCESS)
+                return cudaErrorInvalidValue;
+        }
+    ent.valid = true;
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_maps[g_maps_next] = ent;
+    g_maps_next = (g_maps_next + 1) % (int)(sizeof(g_maps) / sizeof(g_maps[0]));
+    *maps = ent.maps;
+    *used = ent.used;
+    return cudaSuccess;
+}
+
+static cudaError_t launch(const Params &prm, const Plan &pl, void *workspace, cudaStream_t stream,
+                          float inv_tau = 1.f) {
     const int dev = current_device();
     const KSpec k = spec_of(pl.kind);
-    cudaError_t e = prepare_kernel(k, is_span(pl.kind) ? 1 : pl.cluster);
+    cudaError_t e = prepare_kernel(k, is_coop(pl.kind) ? 1 : pl.cluster);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg;
     cudaLaunchAttribute attr[2];
     fill_config(cfg, attr, k, pl.cluster, pl.clusters, stream);
+    if (is_pipe(pl.kind)) {
+        static thread_local pp::Args a;
+        a = pp::Args{};
+        e = pipe_maps(prm, dev, &a.maps, &a.used);
+        if (e != cudaSuccess) return e;
+        a.P = prm;
+        a.PS = pl.cluster;
+        a.Lc = pl.span_len;
+        a.inv_tau = inv_tau;
+        if (pl.ws_bytes > 0) {
+            uint8_t *base = static_cast<uint8_t *>(workspace);
+            const int cap = span_capacity(dev, num_sms(dev), true);
+            a.flags = reinterpret_cast<unsigned *>(base);
+            a.ws = reinterpret_cast<float *>(base + span_flags_bytes(cap));
+        }
+        void *args[] = {&a};
+        return cudaLaunchKernelExC(&cfg, k.fn, args);
+    }
     if (is_span(pl.kind)) {
         sp::Work wk{};
         wk.P = pl.cluster;
@@ -1140,6 +1304,37 @@ extern "C" gtr_status_t gtr_gla_fwd(const gtr_half_t *q, const gtr_half_t *k,
     return cuda_status(launch(prm, pl, ws, s));
 }
 
+extern "C" gtr_status_t gtr_gla_fwd_z(const gtr_half_t *q, const gtr_half_t *k, const gtr_half_t *v,
+                                      const gtr_half_t *z, float tau, int B, int heads, int Hgrid, int Wgrid,
+                                      int dk, int dv, int direction, int chunk, const float *init_state,
+                                      gtr_half_t *out, float *final_state, void *stream) {
+    const gtr_status_t st = check_args(q, k, v, z, B, heads, Hgrid, Wgrid, dk, dv, direction, chunk, init_state,
+                                       out, final_state);
+    if (st != GTR_OK) return st;
+    if (!(tau > 0.f) || !(tau < 3.0e38f)) return GTR_ERR_INVALID_ARG;
+    if (dk != 64) return GTR_ERR_UNSUPPORTED;
+    if ((long long)Hgrid * Wgrid == 0)   // no token: the state copy of the plain call
+        return gtr_gla_fwd(q, k, v, z, B, heads, Hgrid, Wgrid, dk, dv, direction, chunk, init_state, out,
+                           final_state, stream);
+    const Params prm = make_params(q, k, v, z, B, heads, Hgrid, Wgrid, direction, init_state, out, final_state);
+    const Plan pl = make_plan(prm.n_seq, prm.n_chunks, dk, true, ~size_t(0), true);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    void *ws = nullptr;
+    if (pl.ws_bytes > 0) {
+        const gtr_status_t wst = cuda_status(default_workspace(current_device(), pl.ws_bytes, s, &ws));
+        if (wst != GTR_OK) return wst;
+    }
+    return cuda_status(launch(prm, pl, ws, s, 1.f / tau));
+}
+
+extern "C" gtr_status_t gtr_gla_init(void *stream) {
+    const int dev = current_device();
+    const int cap = span_capacity(dev, num_sms(dev), true);
+    if (cap <= 0) return GTR_OK;   // no span plan on this device: no workspace
+    void *ws = nullptr;
+    return cuda_status(default_workspace(dev, default_ws_bytes(cap), reinterpret_cast<cudaStream_t>(stream), &ws));
+}
+
 extern "C" size_t gtr_gla_workspace_bytes(int B, int heads, int Hgrid, int Wgrid, int dk, int dv,
                                           int chunk) {
     if (B <= 0 || heads <= 0 || Hgrid < 0 || Wgrid < 0 || chunk != kChunk) return 0;
@@ -1180,10 +1375,15 @@ static void *g_static_ws_ptr[64];
 
 // Device address of the static scratch on the current device `dev`, looked up once
 // (with `dev` current); the first lookup also zero-fills the publish flags.
-static cudaError_t static_scratch(int dev, void **ptr) {
+static cudaError_t static_scratch(int dev, cudaStream_t stream, void **ptr) {
     const int cap = span_capacity(dev, num_sms(dev), true);
     std::lock_guard<std::mutex> lk(g_mu);
     if (g_static_ws_ptr[dev] == nullptr) {
+        // the set-up synchronises the device: not inside a stream capture
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        cudaError_t ce = cudaStreamIsCapturing(stream, &cs);
+        if (ce != cudaSuccess) return ce;
+        if (cs != cudaStreamCaptureStatusNone) return cudaErrorStreamCaptureUnsupported;
         void *p = nullptr;
         cudaError_t e = cudaGetSymbolAddress(&p, g_static_ws);
         if (e != cudaSuccess) return e;
@@ -1208,11 +1408,13 @@ extern "C" gtr_status_t gtr_gla_fwd_static(const gtr_half_t *q, const gtr_half_t
     if (st != GTR_OK) return st;
     const Params prm = make_params(q, k, v, g, B, heads, Hgrid, Wgrid, direction, init_state, out,
                                    final_state);
-    const Plan pl = make_plan(prm.n_seq, prm.n_chunks, dk, true);
+    // the cheapest plan whose workspace fits the scratch (one span per sequence needs none)
+    const Plan pl = make_plan(prm.n_seq, prm.n_chunks, dk, true, kStaticWsBytes);
     if (pl.ws_bytes > kStaticWsBytes) return GTR_ERR_UNSUPPORTED;
     void *ws = nullptr;
     if (pl.ws_bytes > 0) {
-        const gtr_status_t wst = cuda_status(static_scratch(current_device(), &ws));
+        const gtr_status_t wst =
+            cuda_status(static_scratch(current_device(), reinterpret_cast<cudaStream_t>(stream), &ws));
         if (wst != GTR_OK) return wst;
     }
     return cuda_status(launch(prm, pl, ws, reinterpret_cast<cudaStream_t>(stream)));
@@ -1254,6 +1456,11 @@ extern "C" gtr_status_t gtr_gla_device_status(void *stream) {
     }
     unsigned word = 0;
     if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word)) != cudaSuccess) return GTR_ERR_CUDA;
+    if (word == kErrRange) {
+        const unsigned zero = 0;
+        cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero));
+        return GTR_ERR_RANGE;
+    }
     if (word != 0) {
         const unsigned zero = 0;
         cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero));
@@ -1276,6 +1483,7 @@ extern "C" const char *gtr_status_str(gtr_status_t s) {
     case GTR_ERR_UNSUPPORTED: return "unsupported configuration";
     case GTR_ERR_CUDA: return "CUDA error";
     case GTR_ERR_TIMEOUT: return "device-side wait timed out";
+    case GTR_ERR_RANGE: return "an fp16 operand or output left the fp16 range";
     }
     return "unknown status";
 }

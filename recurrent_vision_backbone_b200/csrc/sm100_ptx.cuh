@@ -45,16 +45,36 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Waits for the phase with the given parity to complete, for at most
-// `limit_ns` nanoseconds.  Returns false if the limit ran out.
+// SM cycle counter: a cheap clock for bounding waits (a %globaltimer read costs about
+// a quarter of a microsecond, which a hand-off on the critical path cannot afford).
+__device__ __forceinline__ long long cycles() { return clock64(); }
+// Cycles standing for `ns` nanoseconds: counted at 2 GHz (at least the SM's top clock),
+// so that the real bound is `ns` or longer at any clock.
+__device__ __forceinline__ long long cycles_of_ns(uint64_t ns) { return (long long)(2 * ns); }
+
+// Waits for the phase with the given parity to complete, for at least `limit_ns`
+// nanoseconds before giving up.  Returns false if the limit ran out.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
                                                   uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
+    const long long t0 = cycles(), lim = cycles_of_ns(limit_ns);
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (globaltimer_ns() - t0 > limit_ns) return false;
+        if (cycles() - t0 > lim) return false;
     }
+}
+
+// Non-blocking test of a phase (for polling several barriers in turn).
+__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
 }
 
 // ---------------------------------------------------------------- tcgen05
@@ -266,10 +286,10 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t pa
 __device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t *bar, uint32_t parity,
                                                           uint64_t limit_ns) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
+    const long long t0 = cycles(), lim = cycles_of_ns(limit_ns);
     while (true) {
         if (mbar_try_wait_cluster(bar, parity)) return true;
-        if (globaltimer_ns() - t0 > limit_ns) return false;
+        if (cycles() - t0 > lim) return false;
     }
 }
 

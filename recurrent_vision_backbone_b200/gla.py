@@ -17,11 +17,11 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libgtr_gla.so")
 
-GTR_OK, GTR_ERR_INVALID_ARG, GTR_ERR_UNSUPPORTED, GTR_ERR_CUDA, GTR_ERR_TIMEOUT = range(5)
+GTR_OK, GTR_ERR_INVALID_ARG, GTR_ERR_UNSUPPORTED, GTR_ERR_CUDA, GTR_ERR_TIMEOUT, GTR_ERR_RANGE = range(6)
 L2R, R2L, T2B, B2T = 0, 1, 2, 3
 STATIC_WS_BYTES = 4 << 20   # GTR_STATIC_WS_BYTES
 
-EXPORTED_SYMBOLS = ("gtr_gla_fwd", "gtr_gla_workspace_bytes", "gtr_gla_fwd_ws",
+EXPORTED_SYMBOLS = ("gtr_gla_fwd", "gtr_gla_fwd_z", "gtr_gla_init", "gtr_gla_workspace_bytes", "gtr_gla_fwd_ws",
                     "gtr_gla_fwd_static", "gtr_gla_device_status", "gtr_status_str", "gtr_gla_plan", "gtr_gla_version",
                     "gtr_gla_last_error", "gtr_gla_selftest_timeout")
 
@@ -51,6 +51,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         vp, i = ctypes.c_void_p, ctypes.c_int
         lib.gtr_gla_fwd.restype = i
         lib.gtr_gla_fwd.argtypes = [vp, vp, vp, vp] + [i] * 8 + [vp, vp, vp, vp]
+        lib.gtr_gla_fwd_z.restype = i
+        lib.gtr_gla_fwd_z.argtypes = [vp, vp, vp, vp, ctypes.c_float] + [i] * 8 + [vp, vp, vp, vp]
         lib.gtr_gla_fwd_static.restype = i
         lib.gtr_gla_fwd_static.argtypes = [vp, vp, vp, vp] + [i] * 8 + [vp, vp, vp, vp]
         lib.gtr_gla_workspace_bytes.restype = ctypes.c_size_t
@@ -60,6 +62,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
                                        + [vp, ctypes.c_size_t, vp])
         lib.gtr_gla_device_status.restype = i
         lib.gtr_gla_device_status.argtypes = [vp]
+        lib.gtr_gla_init.restype = i
+        lib.gtr_gla_init.argtypes = [vp]
         lib.gtr_gla_selftest_timeout.restype = i
         lib.gtr_gla_selftest_timeout.argtypes = [ctypes.c_uint, vp]
         lib.gtr_status_str.restype = ctypes.c_char_p
@@ -78,7 +82,8 @@ def status_str(status: int) -> str:
         return load().gtr_status_str(int(status)).decode()
     except Exception:  # library not loadable: plain text
         return {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "CUDA error",
-                4: "device-side wait timed out"}.get(int(status), "unknown status")
+                4: "device-side wait timed out",
+                5: "an fp16 operand or output left the fp16 range"}.get(int(status), "unknown status")
 
 
 def _ptr(t):
@@ -97,6 +102,12 @@ def _prepare(q, k, v, g, Hgrid, Wgrid, init_state, out, final_state):
     for name, t in (("q", q), ("k", k), ("g", g), ("v", v)):
         if t.dtype != torch.float16 or not t.is_cuda or not t.is_contiguous():
             raise ValueError(f"{name} must be a contiguous CUDA float16 tensor")
+    # the library launches on the current device: every tensor must live there
+    cur = torch.cuda.current_device()
+    for name, t in (("q", q), ("k", k), ("g", g), ("v", v), ("init_state", init_state),
+                    ("out", out), ("final_state", None if final_state is True else final_state)):
+        if t is not None and t.device.index != cur:
+            raise ValueError(f"{name} is on {t.device}, but the current CUDA device is cuda:{cur}")
     if k.shape != q.shape or g.shape != q.shape or tuple(v.shape[:3]) != (B, N, heads):
         raise ValueError("q, k, g must be [B,N,heads,dk] and v [B,N,heads,dv]")
     if N != Hgrid * Wgrid:
@@ -128,6 +139,20 @@ def gtr_gla_fwd(q, k, v, g, Hgrid: int, Wgrid: int, direction: int, init_state=N
                          _ptr(final_state), _stream_handle(stream))
     if st != GTR_OK:
         raise GTRError(st, "gtr_gla_fwd")
+    return out, final_state
+
+
+def gtr_gla_fwd_z(q, k, v, z, tau: float, Hgrid: int, Wgrid: int, direction: int,
+                  init_state=None, out=None, final_state=None, chunk: int = 64, stream=None):
+    """gtr_gla_fwd with the gate's pre-activation z (fp16, the layout of g) and its
+    temperature tau: the kernel forms g = log(sigmoid(z)) / tau while staging."""
+    (B, heads, dk, dv), out, final_state = _prepare(q, k, v, z, Hgrid, Wgrid, init_state, out,
+                                                    final_state)
+    st = load().gtr_gla_fwd_z(_ptr(q), _ptr(k), _ptr(v), _ptr(z), ctypes.c_float(tau), B, heads,
+                              Hgrid, Wgrid, dk, dv, int(direction), int(chunk), _ptr(init_state),
+                              _ptr(out), _ptr(final_state), _stream_handle(stream))
+    if st != GTR_OK:
+        raise GTRError(st, "gtr_gla_fwd_z")
     return out, final_state
 
 
@@ -188,6 +213,14 @@ def gtr_gla_fwd_raw(q_ptr: int, k_ptr: int, v_ptr: int, g_ptr: int, B: int, head
                               ctypes.c_void_p(out_ptr),
                               ctypes.c_void_p(final_ptr) if final_ptr else None,
                               ctypes.c_void_p(stream_handle))
+
+
+def init(stream=None) -> None:
+    """Allocate the library's cached workspace of the current device now (stream-ordered),
+    e.g. before capturing calls into a CUDA graph."""
+    st = load().gtr_gla_init(_stream_handle(stream))
+    if st != GTR_OK:
+        raise GTRError(st, "gtr_gla_init")
 
 
 def device_status(stream=None) -> int:
