@@ -119,6 +119,35 @@ gtr_status_t gtr_gla_fwd_z(const gtr_half_t *q, const gtr_half_t *k, const gtr_h
                            const float *init_state, gtr_half_t *out, float *final_state,
                            void *stream);
 
+/* One layer call of a stack (gtr_gla_fwd_stack): the tensors of gtr_gla_fwd. */
+typedef struct {
+    const gtr_half_t *q, *k, *v, *g;   /* inputs, layouts as above */
+    const float *init_state;           /* float32 [B, heads, dk, dv] or NULL */
+    gtr_half_t *out;                   /* float16 [B, N, heads, dv] */
+    float *final_state;                /* float32 [B, heads, dk, dv] or NULL */
+    int direction;                     /* gtr_dir_t */
+} gtr_gla_layer_t;
+
+/*
+ * A stack of n_layers token-mixer calls of one shape, in order, on `stream`: the GTR
+ * backbone's blocks each scan in one direction, cycling L->R, R->L, T->B, B->T over its
+ * twelve blocks (GTR news article, section "单向扫描的致命缺陷，以及GTR怎么补").  Each layer
+ * has its own tensors and direction; a layer may read an earlier layer's outputs or
+ * final state (stream order).  Consecutive launches overlap (each layer's set-up runs
+ * while the previous one drains).  Outside a stream capture the launches are recorded
+ * once into a CUDA graph per distinct layer list (pointers, directions, shape), on a
+ * private stream of the library's (so `stream` may be the legacy default stream), and
+ * that graph is launched on `stream`, so a repeated stack costs one graph launch of
+ * host time (the eight most recent layer lists are kept); inside a
+ * capture they are simply enqueued into the caller's graph.  Same per-layer arguments,
+ * checks and results as gtr_gla_fwd (a failing layer's index is not reported: every
+ * layer is checked before anything is enqueued).  1 <= n_layers <= 64.
+ * (The pages' model interleaves other operators between these calls; the stack is the
+ * token-mixer part of it.)
+ */
+gtr_status_t gtr_gla_fwd_stack(const gtr_gla_layer_t *layers, int n_layers, int B, int heads,
+                               int Hgrid, int Wgrid, int dk, int dv, int chunk, void *stream);
+
 /*
  * Allocates and zero-fills, in the order of `stream` (no host wait), the library's
  * cached workspace of the current device, sized for every shape, so that no later

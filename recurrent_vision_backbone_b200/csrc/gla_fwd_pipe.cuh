@@ -18,25 +18,27 @@
 // S_in and add the missing term (Qint * D_c) S_in to their outputs, D_c being the decay
 // product from the span start to chunk c.
 //
-// Roles (one CTA = 18 warps):
-//   warp 0       producer: one lane issues the chunk's TMA tensor copies (q, k, g, v)
-//                into a 3-slot staging ring.  The scan direction is applied only in the
-//                copies' coordinates: a chunk is a list of runs of grid tokens that are
-//                contiguous in memory (a row segment, or a column segment at stride W),
-//                each copied in memory order by boxes of 64, 32, .. 1 rows; the lanes
-//                write the table staging row <- scan position (identity for L->R and
-//                T->B, reversed inside each run for R->L and B->T);
-//   warp 1       MMA issuer (one elected lane): MMA 1 = (K~^T V, Qint K~^T) and
-//                MMA 2 = Qint S_prev + P V, tcgen05 kind::f16 with fp32 accumulators
-//                in tensor memory, P read from tensor memory;
-//   warps 2-5    state group U: S (fp32) lives in registers in the accumulator's
+// Roles (one CTA = 16 warps, 128 registers each):
+//   warps 0-3    state group U: S (fp32) lives in registers in the accumulator's
 //                fragment layout; per chunk S <- d * (S + dS), and its fp16 copy is the
-//                next chunk's S_prev operand;
-//   warps 6-9    readout group RE: scores -> causal mask -> fp16 P back into tensor
-//                memory; then the chunk's output tile -> fp16 -> coalesced row stores;
-//   warps 10-17  gating group G: per chunk the cumulative decays, Qint and K~ (or the
+//                next chunk's S_prev operand.  Warp 0 owns the tensor memory and issues
+//                the look-back's bulk copies of the earlier spans' aggregates;
+//   warps 4-7    readout group RE: scores -> causal mask -> fp16 P back into tensor
+//                memory; then the chunk's output tile -> fp16 -> coalesced row stores.
+//                Warp 4 issues the tensor-core work (one elected lane): MMA 1 =
+//                (K~^T V, Qint K~^T) and MMA 2 = Qint S_prev + P V, tcgen05 kind::f16
+//                with fp32 accumulators in tensor memory, P read from tensor memory;
+//   warps 8-15   gating group G, two teams of four warps, team t gating the chunks of
+//                parity t: per chunk the cumulative decays, Qint and K~ (or the
 //                sub-block operands, below) into 128-byte-swizzled operand tiles, and V
-//                into its operand tile in scan order.
+//                into its operand tile in scan order.  A team's first warp then loads
+//                the chunk three ahead into the staging slot it freed: TMA tensor copies
+//                of q, k, g, v into a 3-slot ring.  The scan direction is applied only in
+//                the copies' coordinates: a chunk is a list of runs of grid tokens that
+//                are contiguous in memory (a row segment, or a column segment at stride
+//                W), each copied in memory order by boxes of 64, 32, .. 1 rows; the lanes
+//                write the table staging row <- scan position (identity for L->R and
+//                T->B, reversed inside each run for R->L and B->T).
 // Every hand-off is an mbarrier with a bounded wait; each producer of a double-buffered
 // resource waits for its consumer's release of the previous use, so that no waiter can
 // fall two phases behind.
@@ -56,10 +58,13 @@ constexpr int kDK = 64;
 constexpr int kNStage = 3;                   // staging slots
 constexpr int kRing = 3;                     // chunks of a later span whose Qint * D_c stays in smem
 constexpr int kMaxSpan = 32;                 // chunks of a span with recorded decays (P > 1)
-constexpr int kThreads = 576;                // 18 warps
-constexpr int kWarpProd = 0, kWarpMMA = 1, kWarpU = 2, kWarpRE = 6, kWarpG = 10;
+constexpr int kThreads = 512;                // 16 warps (128 registers each)
+constexpr int kWarpU = 0, kWarpRE = 4, kWarpG = 8;
 constexpr int kUThreads = 128, kREThreads = 128, kGThreads = 256;
-constexpr uint32_t kBarG = 1, kBarU = 2, kBarRE = 3, kBarUP = 4, kBarT0 = 5, kBarT1 = 6;
+constexpr int kTeamThreads = 128;   // a gating team: 4 warps x 16 rows
+// named barriers: gating teams 1 and 7 (team t: 1 + 6 t), all gating warps 8
+constexpr uint32_t kBarU = 2, kBarRE = 3, kBarT0 = 5, kBarT1 = 6, kBarGAll = 8;
+__host__ __device__ constexpr uint32_t bar_team(int team) { return 1u + 6u * (uint32_t)team; }
 constexpr int kAggFloats = kDK * kDV + kDK;  // state + decay product
 constexpr int kAggBytes = kAggFloats * 4;    // 16640
 constexpr int kFoldSlots = 8;                // aggregates copied into smem at a time
@@ -121,14 +126,10 @@ static_assert(L::qint % 1024 == 0 && L::ring % 1024 == 0 && L::ostg % 1024 == 0,
 
 enum {
     B_FULL = 0,     // [3] staging slot landed (TMA transaction count)
-    B_EMPTY = 3,    // [3] staging slot free again (G, or MMA 1 on the sub-block path)
     B_OPFULL = 6,   // [2] G done: Qint, K~, V, d, flags of a chunk
     B_MMA1 = 8,     // [2] MMA 1 complete
-    B_PREADY = 10,  // [2] P written to tensor memory (RE, 128 arrivals)
     B_SPFULL = 12,  // [2] S_prev operand written (U)
     B_MMA2 = 14,    // [2] MMA 2 complete (operands, S_prev, scores free; O ready)
-    B_DSFREE = 16,  // [2] dS read by U (128 arrivals)
-    B_OFREE = 18,   // [2] O read by RE (128 arrivals)
     B_AGG = 20,     // look-back aggregates copied
     B_FIX = 21,     // correction MMAs complete
     B_DRAIN = 22    // every MMA of the sequence's chunks complete (one phase per sequence)
@@ -244,7 +245,7 @@ __device__ __forceinline__ float ld_gate1(const uint8_t *p, float inv_tau) {
     return x;
 }
 
-// ------------------------------------------------------------------ producer
+// ------------------------------------------------------------------ staging loads
 // Staging row table of chunk `cabs` (scan positions p0 .. p0+63): row t of the chunk (in
 // scan order) sits at staging row srow[t].  Lanes write two entries each.
 __device__ __forceinline__ void write_meta(const Params &P, uint8_t *meta, int cabs, int lane) {
@@ -316,20 +317,78 @@ __device__ __forceinline__ uint32_t issue_chunk(const Args &A, uint32_t slot, in
     return (uint32_t)(pend - p0) * kRowBytes;
 }
 
+// Chunk `cabs` of sequence `seq` into staging slot `s` (one warp): the row table, the
+// expected transaction bytes and the copies.
+__device__ __forceinline__ void load_chunk(const Args &A, uint8_t *sm, uint32_t sbase, uint32_t s, int seq,
+                                           int cabs, int lane) {
+    write_meta(A.P, sm + L::meta + s * 128, cabs, lane);
+    __syncwarp();
+    if (lane == 0) {
+        const uint32_t mb = smem_u32(bar(sm, B_FULL + s));
+        const uint32_t slot = sbase + L::stage + s * L::stage_bytes;
+        mbar_arrive_expect_tx(bar(sm, B_FULL + s), issue_chunk(A, slot, seq, cabs, mb, true));
+        issue_chunk(A, slot, seq, cabs, mb, false);
+    }
+    __syncwarp();
+}
+
+// The first kNStage chunks of a sequence (chunk c goes to slot (gc0 + c) % kNStage: the
+// sequence starts where the CTA's running chunk count stands, kept in the caller).
+__device__ __forceinline__ void load_head(const Args &A, uint8_t *sm, uint32_t sbase, uint32_t gc0, int seq,
+                                          int lane) {
+    const int kspan = (int)blockIdx.x % A.PS;
+    const int c0 = kspan * A.Lc;
+    const int nch = min(A.Lc, A.P.n_chunks - c0);
+    for (int c = 0; c < min(kNStage, nch); ++c) load_chunk(A, sm, sbase, (gc0 + c) % kNStage, seq, c0 + c, lane);
+}
+
 // ------------------------------------------------------------------ gating (group G)
-// G warp gw (0..7) owns scan rows 8gw .. 8gw+7 of the chunk, lane l channels 2l, 2l+1.
+// Two gating teams of four warps; team b gates the chunks whose operands go to buffer b
+// (every other chunk), so that two chunks are gated at once.  Warp w of a team owns the
+// chunk's scan rows 16w .. 16w+15 (sub-block w of the sub-block path), lane l channels
+// 2l, 2l+1.
 struct GRegs {
-    __half2 q[8], k[8];
-    float2 g[8], p[8];   // log-decays and their prefix sums within the 8-row group
+    float2 p[16];   // prefix sums of the log-decay over the warp's 16 rows
 };
+
+// Row u of the warp's 16 (staging row from the table words, zero past the grid).
+__device__ __forceinline__ uint32_t row_off(const uint4 &sr, int u, int lane) {
+    const uint32_t w4 = u < 4 ? sr.x : u < 8 ? sr.y : u < 12 ? sr.z : sr.w;
+    return ((w4 >> (8 * (u & 3))) & 0xffu) * 128u + 4u * (uint32_t)lane;
+}
+__device__ __forceinline__ __half2 ld_row_h2(const uint8_t *p, bool ok) {
+    const uint32_t x = ok ? *reinterpret_cast<const uint32_t *>(p) : 0u;
+    return *reinterpret_cast<const __half2 *>(&x);
+}
+
+// Fast-path gating of the warp's sixteen rows (chunk decay >= e^-6, |k| <= 100):
+// Qint = q exp(b), K~ = k exp(-b) with b = off + the row's prefix sum; a held chunk also
+// keeps Qint in its ring tile.  (Two instances: a branch inside the unrolled loop would
+// keep the scheduler from overlapping the rows.)
+template <bool kHeld>
+__device__ __forceinline__ void gate_fast(const GRegs &R, float2 off, const uint8_t *st, const uint4 &sr, int nrows,
+                                          uint8_t *qo, uint8_t *ko, uint8_t *ro, int t0, int lane) {
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+        const uint32_t so = row_off(sr, u, lane);
+        const bool ok = t0 + u < nrows;
+        const __half2 qv = ld_row_h2(st + L::st_q + so, ok), kv = ld_row_h2(st + L::st_k + so, ok);
+        const float x0 = (off.x + R.p[u].x) * kLog2e, x1 = (off.y + R.p[u].y) * kLog2e;
+        const __half2 qi = __hmul2(qv, h2(ex2a(x0), ex2a(x1)));
+        const uint32_t o = sw_off(t0 + u, 2 * lane);
+        sth2(qo + o, qi);
+        sth2(ko + o, __hmul2(kv, h2(ex2a(-x0), ex2a(-x1))));
+        if constexpr (kHeld) sth2(ro + o, qi);
+    }
+}
 
 // Exact fp32 diagonal blocks of the flagged sub-blocks (rare: decay below e^-8 inside 16
 // tokens, or keys too large): value(u, w) = sum_i q[u] k[w] exp(sum_{r=w+1..u} g[r]),
-// stored as fp16 (it becomes an fp16 P entry anyway).
+// stored as fp16 (it becomes an fp16 P entry anyway).  The team's 128 threads.
 template <bool kZ>
 __device__ __noinline__ void exact_diag(const uint8_t *st, const uint8_t *meta, int nrows, const int *flags,
-                                        __half *dst, int tg, float inv_tau) {
-    for (int task = tg; task < 4 * 256; task += kGThreads) {
+                                        __half *dst, int tt, float inv_tau) {
+    for (int task = tt; task < 4 * 256; task += kTeamThreads) {
         const int I = task >> 8, u = (task >> 4) & 15, w = task & 15;
         if (!flags[I] || w > u) continue;
         const int tu = 16 * I + u, tw = 16 * I + w;
@@ -350,63 +409,69 @@ __device__ __noinline__ void exact_diag(const uint8_t *st, const uint8_t *meta, 
 }
 
 // Sub-block path of the gating of one chunk (out of line: the fast path keeps its
-// registers).  Writes Qint and K^ = K * exp(b_C - b) into qo / ko (and Qint * D_c into ro
-// when held), flags the diagonal blocks that need the exact evaluation, evaluates those
-// into diagx[b], then overlays Qd, Kd, A_J and B_J on the chunk's staging slot.
+// registers).  Warp gw's rows are sub-block I = gw, ht[J] the total log-decay of block J.
+// Writes Qint and K^ = K * exp(b_C - b) into qo / ko (and Qint into ro when held), flags
+// the diagonal blocks that need the exact evaluation, evaluates those into diagx[b], then
+// overlays Qd, Kd, A_J and B_J on the chunk's staging slot.
 template <bool kZ>
-__device__ __noinline__ void gate_slow(uint8_t *sm, const GRegs &R, const float2 (&ht)[8], int gw, int lane, int tg,
-                                       uint8_t *st, const uint8_t *meta, int nrows, uint8_t *qo, uint8_t *ko,
-                                       uint8_t *ro, bool held, float2 Dc, int *bfl, int b, float inv_tau) {
-    const int t0 = 8 * gw;
-    const int I = gw >> 1, hb = gw & 1;
-    float2 T[4];
+__device__ __noinline__ void gate_slow(uint8_t *sm, const GRegs &R, const float2 (&ht)[4], int gw, int lane, int tt,
+                                       uint32_t bid, uint8_t *st, const uint8_t *meta, int nrows, uint8_t *qo,
+                                       uint8_t *ko, uint8_t *ro, bool held, int *bfl, int b, float inv_tau) {
+    const int t0 = 16 * gw, I = gw;
+    const uint4 sr = *reinterpret_cast<const uint4 *>(meta + t0);
+    __half2 qh[16], kh[16];
 #pragma unroll
-    for (int J = 0; J < 4; ++J) T[J] = make_float2(ht[2 * J].x + ht[2 * J + 1].x, ht[2 * J].y + ht[2 * J + 1].y);
+    for (int u = 0; u < 16; ++u) {
+        const uint32_t so = row_off(sr, u, lane);
+        qh[u] = ld_row_h2(st + L::st_q + so, t0 + u < nrows);
+        kh[u] = ld_row_h2(st + L::st_k + so, t0 + u < nrows);
+    }
     float2 pre = make_float2(0.f, 0.f), post = make_float2(0.f, 0.f);
 #pragma unroll
     for (int J = 0; J < 4; ++J) {
-        if (J < I) { pre.x += T[J].x; pre.y += T[J].y; }
-        if (J > I) { post.x += T[J].x; post.y += T[J].y; }
+        if (J < I) { pre.x += ht[J].x; pre.y += ht[J].y; }
+        if (J > I) { post.x += ht[J].x; post.y += ht[J].y; }
     }
-    const float2 poff = hb ? ht[gw - 1] : make_float2(0.f, 0.f);
-    const float2 soff = hb ? make_float2(0.f, 0.f) : ht[gw + 1];
-    float2 bs[8];   // within-block suffix sums (excluding the row)
+    float2 bs[16];   // within-block suffix sums (excluding the row), from the raw rows
     {
-        float2 a = soff;
+        float2 a = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int u = 7; u >= 0; --u) {
+        for (int u = 15; u >= 0; --u) {
             bs[u] = a;
-            a.x += R.g[u].x;
-            a.y += R.g[u].y;
+            const float2 gv = ld_gate2<kZ>(st + L::st_g + meta[t0 + u] * 128 + 4 * lane, inv_tau);
+            if (t0 + u < nrows) {
+                a.x += gv.x;
+                a.y += gv.y;
+            }
         }
     }
-    bool kbad = !(T[I].x >= kDiagMinLogTotal) || !(T[I].y >= kDiagMinLogTotal);
+    bool kbad = !(ht[I].x >= kDiagMinLogTotal) || !(ht[I].y >= kDiagMinLogTotal);
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-        const float2 bp = make_float2(poff.x + R.p[u].x, poff.y + R.p[u].y);
-        const float2 qf = __half22float2(R.q[u]), kf = __half22float2(R.k[u]);
-        const float2 qi = make_float2(qf.x * ex2a((pre.x + bp.x) * kLog2e), qf.y * ex2a((pre.y + bp.y) * kLog2e));
+    for (int u = 0; u < 16; ++u) {
+        const float2 bp = R.p[u];
+        const float2 qf = __half22float2(qh[u]), kf = __half22float2(kh[u]);
+        const __half2 qi = h2(qf.x * ex2a((pre.x + bp.x) * kLog2e), qf.y * ex2a((pre.y + bp.y) * kLog2e));
         const uint32_t o = sw_off(t0 + u, 2 * lane);
-        sth2(qo + o, h2(qi.x, qi.y));
+        sth2(qo + o, qi);
         sth2(ko + o, h2(kf.x * ex2a((bs[u].x + post.x) * kLog2e), kf.y * ex2a((bs[u].y + post.y) * kLog2e)));
-        if (held) sth2(ro + o, h2(qi.x * Dc.x, qi.y * Dc.y));
+        if (held) sth2(ro + o, qi);
         const float kd0 = kf.x * ex2a(-bp.x * kLog2e), kd1 = kf.y * ex2a(-bp.y * kLog2e);
         kbad |= !(fabsf(kd0) <= kDiagMaxK) || !(fabsf(kd1) <= kDiagMaxK);
     }
     if (__any_sync(0xffffffffu, kbad) && lane == 0) atomicOr(&bfl[I], 1);
-    named_sync(kBarG, kGThreads);
+    named_sync(bid, kTeamThreads);
     const bool anyflag = (bfl[0] | bfl[1] | bfl[2] | bfl[3]) != 0;
     if (anyflag)
-        exact_diag<kZ>(st, meta, nrows, bfl, reinterpret_cast<__half *>(sm + L::diagx + b * 2048), tg, inv_tau);
-    named_sync(kBarG, kGThreads);   // raw rows no longer read: overlay the operands
+        exact_diag<kZ>(st, meta, nrows, bfl, reinterpret_cast<__half *>(sm + L::diagx + b * 2048), tt, inv_tau);
+    named_sync(bid, kTeamThreads);   // raw rows no longer read: overlay the operands
     const bool fl = bfl[I] != 0;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+    for (int u = 0; u < 16; ++u) {
         const int t = t0 + u;
-        const float2 bp = make_float2(poff.x + R.p[u].x, poff.y + R.p[u].y);
-        const float2 qf = __half22float2(R.q[u]), kf = __half22float2(R.k[u]);
-        const float2 e = make_float2(ex2a(bp.x * kLog2e), ex2a(bp.y * kLog2e));
-        sth2(st + L::sl_qa + sw_off(t, 2 * lane), h2(qf.x * e.x, qf.y * e.y));
+        const float2 bp = R.p[u];
+        const float2 qf = __half22float2(qh[u]), kf = __half22float2(kh[u]);
+        sth2(st + L::sl_qa + sw_off(t, 2 * lane),
+             h2(qf.x * ex2a(bp.x * kLog2e), qf.y * ex2a(bp.y * kLog2e)));
         float kd0 = kf.x * ex2a(-bp.x * kLog2e), kd1 = kf.y * ex2a(-bp.y * kLog2e);
         if (fl) kd0 = kd1 = 0.f;
         sth2(st + L::sl_kd + sw_off(t, 2 * lane), h2(kd0, kd1));
@@ -418,8 +483,8 @@ __device__ __noinline__ void gate_slow(uint8_t *sm, const GRegs &R, const float2
                 const int reg = (J == 0 ? 64 : J == 1 ? 112 : 144) + t - 16 * (J + 1);
                 sth2(st + L::sl_qa + sw_off(reg, 2 * lane),
                      h2(qf.x * ex2a(acc.x * kLog2e), qf.y * ex2a(acc.y * kLog2e)));
-                acc.x += T[J].x;   // one more block between row and anchor
-                acc.y += T[J].y;
+                acc.x += ht[J].x;   // one more block between row and anchor
+                acc.y += ht[J].y;
             }
         }
         if (I < 3)   // B_I rows: keys of block I, anchor at its end
@@ -433,10 +498,34 @@ __device__ __noinline__ void gate_slow(uint8_t *sm, const GRegs &R, const float2
 // rows 16 q4 + l/4 (+8); register 16 h + 4 j + 2 e + x is row r0 + 8e, column
 // 32 h + 8 j + 2 (l % 4) + x.
 __device__ __forceinline__ void ld_acc64(uint32_t taddr, uint32_t (&r)[32]) {
-    uint32_t (&a)[16] = *reinterpret_cast<uint32_t(*)[16]>(&r[0]);
-    uint32_t (&b)[16] = *reinterpret_cast<uint32_t(*)[16]>(&r[16]);
-    tmem_ld_16x256b_x4(taddr, a);
-    tmem_ld_16x256b_x4(taddr + 32, b);
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x8.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+}
+// Columns 64..111 of a scores buffer (the blocks below the diagonal), the same register
+// order as ld_acc64 for columns 0..47; registers 24..31 stay zero.
+__device__ __forceinline__ void ld_off48(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]),
+                   "=r"(r[23])
+                 : "r"(taddr + 32)
+                 : "memory");
+#pragma unroll
+    for (int e = 24; e < 32; ++e) r[e] = 0u;
 }
 
 // Output tile (fp32 in registers, fragment layout) -> fp16 -> staging -> coalesced rows.
@@ -504,6 +593,122 @@ __device__ __forceinline__ void write_state_tile(uint8_t *dst, const float (&S)[
     }
 }
 
+// Scores of a sub-block-path chunk -> causal fp16 P (out of line: rare).  Rows of this
+// warp's quarter q4 are sub-block q4; a column in key block J < q4 takes the block below
+// the diagonal (columns 64..111 of the scores buffer), J == q4 the diagonal block (or its
+// exact evaluation), J > q4 zero.  Returns the largest |P|.
+__device__ __noinline__ float readout_slow(uint8_t *sm, uint32_t ta, const uint32_t (&sc)[32], uint32_t (&pv)[16],
+                                           uint32_t b, int q4, int r0, int a2) {
+    uint32_t of[32];   // (key block 3 is never below the diagonal)
+    ld_off48(ta + 64, of);
+    tmem_ld_wait();
+    const int *fl = reinterpret_cast<const int *>(sm + L::bflag) + 4 * b;
+    const bool exact = fl[q4] != 0;
+    const __half *dx = reinterpret_cast<const __half *>(sm + L::diagx + b * 2048) + q4 * 256;
+    float pmx = 0.f;
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+        const int h = e >> 4, j = (e >> 2) & 3, hh = (e >> 1) & 1;
+        const int row = r0 + 8 * hh, col = 32 * h + 8 * j + a2;
+        const int J = col >> 4;   // key block (col and col + 1 share it)
+        float x0 = 0.f, x1 = 0.f;
+        if (J < q4) {
+            x0 = __uint_as_float(of[e]);
+            x1 = __uint_as_float(of[e + 1]);
+        } else if (J == q4) {
+            if (exact) {
+                x0 = __half2float(dx[(row & 15) * 16 + (col & 15)]);
+                x1 = __half2float(dx[(row & 15) * 16 + ((col + 1) & 15)]);
+            } else {
+                x0 = __uint_as_float(sc[e]);
+                x1 = __uint_as_float(sc[e + 1]);
+            }
+            x0 = col <= row ? x0 : 0.f;
+            x1 = col + 1 <= row ? x1 : 0.f;
+        }
+        pmx = fmaxf(pmx, fmaxf(fabsf(x0), fabsf(x1)));
+        const __half2 v = h2(x0, x1);
+        pv[2 * (j + 4 * h) + hh] = *reinterpret_cast<const uint32_t *>(&v);
+    }
+    return pmx;
+}
+
+// Phase-4 B operand of held chunk i (D_i * S_in): free operand tiles after the pipeline.
+__host__ __device__ constexpr int held_tile(int i) { return i == 0 ? L::sop : i == 1 ? L::sop + kTile : L::vop; }
+static_assert(kRing == 3, "three held tiles");
+
+// ------------------------------------------------------------------ MMA issue
+// MMA 1 of the chunk in operand buffer b (staging slot s): dS = K~^T V (K^ on the
+// sub-block path) and the scores Qint K~^T, or the diagonal and below-diagonal sub-block
+// products.  Called by a converged warp; one elected lane issues and commits.
+// Descriptors of the k-steps of one operand differ only in the start-address field
+// (bits 0..13, address / 16): shared memory addresses stay below 2^18, so adding the
+// step's byte offset / 16 to a base descriptor never carries out of the field.
+__device__ __forceinline__ uint64_t desc_step(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
+
+__device__ __forceinline__ void issue_mma1(uint8_t *sm, uint32_t sbase, uint32_t tmem, uint32_t b, uint32_t s,
+                                           bool slow) {
+    constexpr uint32_t id_ds = idesc_f16_f32(64, kDV, true, true);
+    constexpr uint32_t id_sc = idesc_f16_f32(64, 64, false, false);
+    constexpr uint32_t id_off = idesc_f16_f32(64, 16, false, false);
+    const uint32_t kta = sbase + L::kt + b * kTile, va = sbase + L::vop + b * kTile;
+    const uint32_t qa = sbase + L::qint + b * kTile;
+    const uint32_t sl = sbase + L::stage + s * L::stage_bytes;
+    const uint32_t dsc = tmem + kColDS + 64 * b, scc = tmem + kColScores + 128 * b;
+    if (elect_one_sync()) {
+        const uint64_t dk_mn = desc_sw128(kta, kTile, 1024), dv_mn = desc_sw128(va, kTile, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+            umma_f16(dsc, desc_step(dk_mn, kk * 2048), desc_step(dv_mn, kk * 2048), id_ds, kk > 0 ? 1u : 0u);
+        if (!slow) {
+            const uint64_t dq = desc_sw128(qa, 16, 1024), dk = desc_sw128(kta, 16, 1024);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                umma_f16(scc, desc_step(dq, kk * 32), desc_step(dk, kk * 32), id_sc, kk > 0 ? 1u : 0u);
+        } else {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                umma_f16(scc, desc_sw128(sl + L::sl_qa + kk * 32, 16, 1024),
+                         desc_sw128(sl + L::sl_kd + kk * 32, 16, 1024), id_sc, kk > 0 ? 1u : 0u);
+            // A_J's descriptor starts 16(J+1) rows before its region, so that row t of the
+            // operand is scan row t (earlier rows: finite values of the regions before it,
+            // whose results are never read)
+#pragma unroll
+            for (int J = 0; J < 3; ++J) {
+                const uint32_t abase = J == 0 ? 48u * 128u : J == 1 ? 80u * 128u : 96u * 128u;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_f16(scc + 64 + 16 * J, desc_sw128(sl + L::sl_qa + abase + kk * 32, 16, 1024),
+                             desc_sw128(sl + L::sl_b + J * 2048 + kk * 32, 16, 1024), id_off, kk > 0 ? 1u : 0u);
+            }
+        }
+        umma_commit(bar(sm, B_MMA1 + b));
+    }
+    __syncwarp();
+}
+
+// MMA 2 of the chunk in operand buffer b: O = Qint S_prev + P V, P read from the scores'
+// tensor memory.  `last`: also signals the drain barrier (every MMA of the sequence).
+__device__ __forceinline__ void issue_mma2(uint8_t *sm, uint32_t sbase, uint32_t tmem, uint32_t b, bool last) {
+    constexpr uint32_t id_o = idesc_f16_f32(64, kDV, false, true);
+    const uint32_t qa = sbase + L::qint + b * kTile, sa = sbase + L::sop + b * kTile;
+    const uint32_t va = sbase + L::vop + b * kTile;
+    const uint32_t oc = tmem + kColO + 64 * b, pc = tmem + kColScores + 128 * b;
+    if (elect_one_sync()) {
+        const uint64_t dq = desc_sw128(qa, 16, 1024), ds = desc_sw128(sa, kTile, 1024);
+        const uint64_t dv = desc_sw128(va, kTile, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+            umma_f16(oc, desc_step(dq, kk * 32), desc_step(ds, kk * 2048), id_o, kk > 0 ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)   // P from TMEM: K step 16 = 8 packed columns
+            umma_f16_ta(oc, pc + 8 * kk, desc_step(dv, kk * 2048), id_o, 1u);
+        umma_commit(bar(sm, B_MMA2 + b));
+        if (last) umma_commit(bar(sm, B_DRAIN));
+    }
+    __syncwarp();
+}
+
 // ------------------------------------------------------------------ kernel
 // kZ: the third input holds the gate pre-activation z instead of the log-decay g.
 template <bool kZ>
@@ -520,35 +725,31 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_pipe_kernel(const __grid_
     float *dcum = reinterpret_cast<float *>(sm + L::dcum);
     float *cmeta = reinterpret_cast<float *>(sm + L::cmeta);
 
-    if (warp == kWarpMMA) {
+    if (warp == kWarpU) {
         tmem_alloc(tslot, kTmemCols);
         tmem_relinquish();
     }
     if (tid == 0) {
         for (int i = 0; i < kNStage; ++i) {
             mbar_init(bar(sm, B_FULL + i), 1);
-            mbar_init(bar(sm, B_EMPTY + i), 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(bar(sm, B_OPFULL + i), 1);
             mbar_init(bar(sm, B_MMA1 + i), 1);
-            mbar_init(bar(sm, B_PREADY + i), kREThreads);
             mbar_init(bar(sm, B_SPFULL + i), 1);
             mbar_init(bar(sm, B_MMA2 + i), 1);
-            mbar_init(bar(sm, B_DSFREE + i), kUThreads);
-            mbar_init(bar(sm, B_OFREE + i), kREThreads);
         }
         mbar_init(bar(sm, B_AGG), 1);
         mbar_init(bar(sm, B_FIX), 1);
         mbar_init(bar(sm, B_DRAIN), 1);
         fence_mbar_init();
     }
-    if (warp == kWarpProd && lane < 28 && (lane & 7) < 7 && ((A.used >> (lane & 7)) & 1u))
+    if (warp == kWarpG && lane < 28 && (lane & 7) < 7 && ((A.used >> (lane & 7)) & 1u))
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&A.maps.m[lane >> 3][lane & 7]))
                      : "memory");
     // the first chunk's rows into L2 while the grid ahead drains (L2 is where every
     // SM's accesses meet, so a later write by that grid still reaches the copies)
-    if (warp == kWarpProd && lane == 0 && grp < P.n_seq && P.dir == GTR_L2R) {
+    if (warp == kWarpG && lane == 0 && grp < P.n_seq && P.dir == GTR_L2R) {
         const int seq = grp, bb = seq / P.heads, hh = seq - bb * P.heads;
         const int c0 = kspan * A.Lc;
         for (int ten = 0; ten < 4; ++ten) tma_prefetch_4d(&A.maps.m[ten][6], 0, hh, c0 * kChunk, bb);
@@ -561,6 +762,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_pipe_kernel(const __grid_
     asm volatile("griddepcontrol.wait;" ::: "memory");
     bool to = false;
     uint32_t gc0 = 0;          // chunks of earlier sequences run by this CTA
+    if (warp == kWarpG && grp < P.n_seq) load_head(A, sm, sbase, 0u, grp, lane);
     uint32_t n_agg = 0, n_fix = 0, n_drain = 0;
 
     for (int seq = grp; seq < P.n_seq; seq += ngrp) {
@@ -570,151 +772,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_pipe_kernel(const __grid_
         const bool publish = PS > 1 && kspan < PS - 1;
         const int nring = later ? min(kRing, nch) : 0;
 
-        if (warp == kWarpProd) {
-            // ======================================================= producer
-            for (int c = 0; c < nch; ++c) {
-                const uint32_t gc = gc0 + c, s = gc % kNStage;
-                wait_l(bar(sm, B_EMPTY + s), ((gc / kNStage) & 1u) ^ 1u, to);
-                write_meta(P, sm + L::meta + s * 128, c0 + c, lane);
-                __syncwarp();
-                if (lane == 0) {
-                    const uint32_t mb = smem_u32(bar(sm, B_FULL + s));
-                    const uint32_t slot = sbase + L::stage + s * L::stage_bytes;
-                    mbar_arrive_expect_tx(bar(sm, B_FULL + s), issue_chunk(A, slot, seq, c0 + c, mb, true));
-                    issue_chunk(A, slot, seq, c0 + c, mb, false);
-                }
-                __syncwarp();
-            }
-            // Every MMA of this sequence's chunks complete (their operand tiles are free).
-            // A dedicated barrier with one phase per sequence: this warp runs ahead of the
-            // pipeline, so a parity wait on a per-buffer barrier could match an earlier phase.
-            wait_l(bar(sm, B_DRAIN), n_drain & 1u, to);
-            ++n_drain;
-            if (later) {
-                // ---------------- phase 3: the earlier spans' aggregates into shared memory.
-                // The slots overlay the staging ring and the first operand tiles (free now).
-                // Lane u polls span j0+u's flag and copies that aggregate at once; group U
-                // folds a batch, then releases the slots (named barrier kBarUP).
-                for (int j0 = 0; j0 < kspan; j0 += kFoldSlots) {
-                    const int nj = min(kFoldSlots, kspan - j0);
-                    if (lane == 0) mbar_arrive_expect_tx(bar(sm, B_AGG), (uint32_t)(nj * kAggBytes));
-                    __syncwarp();
-                    if (lane < nj) {
-                        unsigned *f = A.flags + ((size_t)seq * PS + j0 + lane) * kFlagStride;
-                        if (sp::flag_wait_bounded(f, kWaitLimitNs)) {
-                            sp::red_dec_gpu(f);   // one reader fewer to come
-                        } else {
-                            to = true;
-                            set_error(kErrTimeout);
-                        }
-                        // the copy engine reads what the acquire made visible; after a
-                        // timeout the copy still runs, so that the barrier completes
-                        asm volatile("fence.proxy.async.global;" ::: "memory");
-                        bulk_g2s(sbase + L::slots + lane * kAggBytes,
-                                 A.ws + ((size_t)seq * PS + j0 + lane) * kAggFloats, (uint32_t)kAggBytes,
-                                 bar(sm, B_AGG));
-                    }
-                    named_sync(kBarUP, kUThreads + 32);   // U done with the slots
-                }
-            }
-        } else if (warp == kWarpMMA) {
-            // ======================================================= MMA issuer
-            constexpr uint32_t id_ds = idesc_f16_f32(64, kDV, true, true);
-            constexpr uint32_t id_sc = idesc_f16_f32(64, 64, false, false);
-            constexpr uint32_t id_off = idesc_f16_f32(64, 16, false, false);
-            constexpr uint32_t id_o = idesc_f16_f32(64, kDV, false, true);
-            // Issues MMA 1 of the next chunk or MMA 2 of the oldest chunk, whichever has its
-            // inputs first (MMA 1 of chunk c also needs MMA 2 of chunk c-2 complete, so it
-            // never runs more than one chunk ahead).  Each barrier's phases are tested in
-            // order, one at a time, so a test can never match an earlier phase.
-            int n1 = 0, n2 = 0;
-            long long idle0 = cycles();
-            while (n2 < nch) {
-                bool did = false;
-                if (n1 < nch && n1 <= n2 + 1) {
-                    const uint32_t gc = gc0 + n1, b = gc & 1u, s = gc % kNStage, ph = (gc >> 1) & 1u;
-                    const bool ready = to || (mbar_test(bar(sm, B_OPFULL + b), ph) &&
-                                              (gc < 2 || (mbar_test(bar(sm, B_DSFREE + b), ph ^ 1u) &&
-                                                          mbar_test(bar(sm, B_MMA2 + b), ph ^ 1u))));
-                    if (__all_sync(0xffffffffu, ready)) {
-                        tc_fence_after();
-                        const bool slow = reinterpret_cast<const int *>(sm + L::slowf)[b] != 0;
-                        const uint32_t kta = sbase + L::kt + b * kTile, va = sbase + L::vop + b * kTile;
-                        const uint32_t qa = sbase + L::qint + b * kTile;
-                        const uint32_t sl = sbase + L::stage + s * L::stage_bytes;
-                        const uint32_t dsc = tmem + kColDS + 64 * b, scc = tmem + kColScores + 128 * b;
-                        if (elect_one_sync()) {
-#pragma unroll
-                            for (int kk = 0; kk < 4; ++kk)
-                                umma_f16(dsc, desc_sw128(kta + kk * 2048, kTile, 1024),
-                                         desc_sw128(va + kk * 2048, kTile, 1024), id_ds, kk > 0 ? 1u : 0u);
-                            if (!slow) {
-#pragma unroll
-                                for (int kk = 0; kk < 4; ++kk)
-                                    umma_f16(scc, desc_sw128(qa + kk * 32, 16, 1024),
-                                             desc_sw128(kta + kk * 32, 16, 1024), id_sc, kk > 0 ? 1u : 0u);
-                            } else {
-#pragma unroll
-                                for (int kk = 0; kk < 4; ++kk)
-                                    umma_f16(scc, desc_sw128(sl + L::sl_qa + kk * 32, 16, 1024),
-                                             desc_sw128(sl + L::sl_kd + kk * 32, 16, 1024), id_sc, kk > 0 ? 1u : 0u);
-                                // A_J's descriptor starts 16(J+1) rows before its region, so that
-                                // row t of the operand is scan row t (earlier rows: finite values of
-                                // the regions before it, whose results are never read)
-                                const uint32_t abase[3] = {48u * 128u, 80u * 128u, 96u * 128u};
-#pragma unroll
-                                for (int J = 0; J < 3; ++J)
-#pragma unroll
-                                    for (int kk = 0; kk < 4; ++kk)
-                                        umma_f16(scc + 64 + 16 * J,
-                                                 desc_sw128(sl + L::sl_qa + abase[J] + kk * 32, 16, 1024),
-                                                 desc_sw128(sl + L::sl_b + J * 2048 + kk * 32, 16, 1024), id_off,
-                                                 kk > 0 ? 1u : 0u);
-                            }
-                            umma_commit(bar(sm, B_MMA1 + b));
-                            if (slow) umma_commit(bar(sm, B_EMPTY + s));   // the overlaid slot is free
-                        }
-                        __syncwarp();
-                        ++n1;
-                        did = true;
-                    }
-                }
-                if (!did && n2 < n1) {
-                    const uint32_t gp = gc0 + n2, b = gp & 1u, ph = (gp >> 1) & 1u;
-                    const bool ready = to || (mbar_test(bar(sm, B_PREADY + b), ph) &&
-                                              mbar_test(bar(sm, B_SPFULL + b), ph) &&
-                                              (gp < 2 || mbar_test(bar(sm, B_OFREE + b), ph ^ 1u)));
-                    if (__all_sync(0xffffffffu, ready)) {
-                        tc_fence_after();
-                        const uint32_t qa = sbase + L::qint + b * kTile, sa = sbase + L::sop + b * kTile;
-                        const uint32_t va = sbase + L::vop + b * kTile;
-                        const uint32_t oc = tmem + kColO + 64 * b, pc = tmem + kColScores + 128 * b;
-                        if (elect_one_sync()) {
-#pragma unroll
-                            for (int kk = 0; kk < 4; ++kk)
-                                umma_f16(oc, desc_sw128(qa + kk * 32, 16, 1024),
-                                         desc_sw128(sa + kk * 2048, kTile, 1024), id_o, kk > 0 ? 1u : 0u);
-#pragma unroll
-                            for (int kk = 0; kk < 4; ++kk)   // P from TMEM: K step 16 = 8 packed columns
-                                umma_f16_ta(oc, pc + 8 * kk, desc_sw128(va + kk * 2048, kTile, 1024), id_o, 1u);
-                            umma_commit(bar(sm, B_MMA2 + b));
-                            if (n2 + 1 == nch) umma_commit(bar(sm, B_DRAIN));   // the sequence's last MMA
-                        }
-                        __syncwarp();
-                        ++n2;
-                        did = true;
-                    }
-                }
-                if (did) {
-                    idle0 = cycles();
-                } else if (cycles() - idle0 <= cycles_of_ns(kWaitLimitNs)) {
-                    __nanosleep(16);   // leave the issue slots to the warps doing the work
-                } else {
-                    if (!to) set_error(kErrTimeout);
-                    to = true;   // from now on every test passes: the kernel runs to its end
-                }
-            }
-        } else if (warp < kWarpRE) {
+        if (warp < kWarpRE) {
             // ======================================================= state group U
             const int q4 = warp & 3, ut = tid - kWarpU * 32;
             const int r0 = 16 * q4 + (lane >> 2);
@@ -734,6 +792,16 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_pipe_kernel(const __grid_
             // that G cannot complete that buffer's next phase before this wait) G's signal
             float dn0, dn1;
             bool slown;
+            // decay products from the span start for rows r0, r0+8 (D_c of chunk c), kept
+            // for the held chunks and the publish, and recorded in dcum for phase 4
+            float D0 = 1.f, D1 = 1.f;
+            float Dh0[kRing], Dh1[kRing];
+#pragma unroll
+            for (int i = 0; i < kRing; ++i) Dh0[i] = Dh1[i] = 1.f;
+            if ((lane & 3) == 0) {
+                dcum[r0] = 1.f;
+                dcum[r0 + 8] = 1.f;
+            }
             {
                 const uint32_t gn = gc0, bn = gn & 1u, ph = (gn >> 1) & 1u;
                 if (gn >= 2) wait_l(bar(sm, B_MMA2 + bn), ph ^ 1u, to);
@@ -746,6 +814,10 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_pipe_kernel(const __grid_
                 dn0 = dl[r0];
                 dn1 = dl[r0 + 8];
                 slown = reinterpret_cast<const int *>(sm + L::slowf)[bn] != 0;
+                if (warp == kWarpU) {
+                    tc_fence_after();
+                    issue_mma1(sm, sbase, tmem, bn, gn % kNStage, slown);
+                }
                 if (ut == 0) mbar_arrive(bar(sm, B_SPFULL + bn));
             }
             for (int c = 0; c < nch; ++c) {
@@ -756,14 +828,39 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_pipe_kernel(const __grid_
                 tc_fence_after();
                 uint32_t ds[32];
                 ld_acc64(tmem + ((uint32_t)(32 * q4) << 16) + kColDS + 64 * b, ds);
-                tmem_ld_wait();
+                tmem_ld_wait();   // (warp-collective: every lane's loads are complete)
+                // MMA 1 of chunk c+1, if its operands are ready already.  Its dS block held
+                // dS of chunk c-1, read by every warp of the group before the group's barrier
+                // of the previous iteration; its scores block P of chunk c-1, read by MMA 2
+                // of chunk c-1, which G waited for before gating chunk c+1.
+                bool issued = false;
+                if (warp == kWarpU && c + 1 < nch) {
+                    const uint32_t gn = gc + 1, bn = gn & 1u;
+                    if (mbar_test(bar(sm, B_OPFULL + bn), (gn >> 1) & 1u)) {
+                        tc_fence_after();
+                        issue_mma1(sm, sbase, tmem, bn, gn % kNStage,
+                                   reinterpret_cast<const int *>(sm + L::slowf)[bn] != 0);
+                        issued = true;
+                    }
+                }
                 tc_fence_before();
-                mbar_arrive(bar(sm, B_DSFREE + b));
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
                     const float d = ((e >> 1) & 1) ? d1 : d0;
                     const float x = __uint_as_float(ds[e]);
                     S[e] = slow ? fmaf(d, S[e], x) : d * (S[e] + x);
+                }
+                D0 *= d0;
+                D1 *= d1;
+#pragma unroll
+                for (int i = 1; i < kRing; ++i)
+                    if (c + 1 == i) {
+                        Dh0[i] = D0;
+                        Dh1[i] = D1;
+                    }
+                if ((lane & 3) == 0 && c + 1 <= kMaxSpan) {
+                    dcum[(c + 1) * 64 + r0] = D0;
+                    dcum[(c + 1) * 64 + r0 + 8] = D1;
                 }
                 if (c + 1 < nch) {
                     const uint32_t gn = gc + 1, bn = gn & 1u, phn = (gn >> 1) & 1u;
@@ -777,6 +874,10 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_pipe_kernel(const __grid_
                     dn0 = dl[r0];
                     dn1 = dl[r0 + 8];
                     slown = reinterpret_cast<const int *>(sm + L::slowf)[bn] != 0;
+                    if (warp == kWarpU && !issued) {
+                        tc_fence_after();
+                        issue_mma1(sm, sbase, tmem, bn, gn % kNStage, slown);
+                    }
                     if (ut == 0) mbar_arrive(bar(sm, B_SPFULL + bn));
                 }
             }
@@ -788,8 +889,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_pipe_kernel(const __grid_
 #pragma unroll
                 for (int m = 0; m < 8; ++m)
                     a4[m * 128 + q4 * 32 + lane] = make_float4(S[4 * m], S[4 * m + 1], S[4 * m + 2], S[4 * m + 3]);
-                // (dcum[nch] was written by G before its signal of the span's last chunk,
-                // which this group waited for)
+                named_sync(kBarU, kUThreads);   // dcum[nch]: one writer per row
                 if (ut < 64) agg[kDK * kDV + ut] = dcum[nch * 64 + ut];
                 named_sync(kBarU, kUThreads);
                 if (ut == 0)   // readers to come: spans kspan+1 .. PS-1
@@ -813,6 +913,11 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_pipe_kernel(const __grid_
                 for (int m = 0; m < 8; ++m)
                     park[m * 128 + q4 * 32 + lane] = make_float4(S[4 * m], S[4 * m + 1], S[4 * m + 2], S[4 * m + 3]);
             }
+            // every MMA of this sequence's chunks complete: the operand tiles that the
+            // look-back slots overlay are free (a dedicated barrier with one phase per
+            // sequence, so that no parity wait can match an earlier phase)
+            wait_l(bar(sm, B_DRAIN), n_drain & 1u, to);
+            ++n_drain;
             if (later) {
                 // ---------------- phase 3: look back over spans 0 .. kspan-1
                 float Sin[32];
@@ -820,6 +925,28 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_pipe_kernel(const __grid_
                 for (int e = 0; e < 32; ++e) Sin[e] = 0.f;
                 for (int j0 = 0; j0 < kspan; j0 += kFoldSlots) {
                     const int nj = min(kFoldSlots, kspan - j0);
+                    if (warp == kWarpU) {
+                        // lane u polls span j0+u's flag and copies that aggregate at once (the
+                        // slots overlay the staging ring and the first operand tiles, free once
+                        // the drain barrier has completed)
+                        if (lane == 0) mbar_arrive_expect_tx(bar(sm, B_AGG), (uint32_t)(nj * kAggBytes));
+                        __syncwarp();
+                        if (lane < nj) {
+                            unsigned *f = A.flags + ((size_t)seq * PS + j0 + lane) * kFlagStride;
+                            if (sp::flag_wait_bounded(f, kWaitLimitNs)) {
+                                sp::red_dec_gpu(f);   // one reader fewer to come
+                            } else {
+                                to = true;
+                                set_error(kErrTimeout);
+                            }
+                            // the copy engine reads what the acquire made visible; after a
+                            // timeout the copy still runs, so that the barrier completes
+                            asm volatile("fence.proxy.async.global;" ::: "memory");
+                            bulk_g2s(sbase + L::slots + lane * kAggBytes,
+                                     A.ws + ((size_t)seq * PS + j0 + lane) * kAggFloats, (uint32_t)kAggBytes,
+                                     bar(sm, B_AGG));
+                        }
+                    }
                     wait_l(bar(sm, B_AGG), n_agg & 1u, to);
                     ++n_agg;
                     for (int u = 0; u < nj; ++u) {   // S_in <- D_j * S_in + S_j
@@ -834,7 +961,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_pipe_kernel(const __grid_
                             Sin[4 * m + 3] = fmaf(D1, Sin[4 * m + 3], v.w);
                         }
                     }
-                    named_sync(kBarUP, kUThreads + 32);   // slots free for the next batch
+                    named_sync(kBarU, kUThreads);   // slots free for the next batch
                 }
                 // row maxima of |S_in| (rows r0: elements 4m, 4m+1; r0 + 8: 4m+2, 4m+3)
                 float m0 = 0.f, m1 = 0.f;
@@ -853,11 +980,21 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_pipe_kernel(const __grid_
                     rmax[r0] = m0;
                     rmax[r0 + 8] = m1;
                 }
-                // S_in as the fp16 operand of the correction MMAs
+                // S_in as the fp16 B operands of the correction MMAs: D_c * S_in (rows
+                // scaled) for the held chunks c (their ring tiles hold Qint), S_in itself for
+                // the rebuilt ones (Qint * D_c rebuilt)
                 range_check(fmaxf(m0, m1));
-                write_state_tile(sm + L::sop, Sin, q4, lane);
+                write_state_tile(sm + L::vop + kTile, Sin, q4, lane);
+#pragma unroll
+                for (int i = 0; i < kRing; ++i) {
+                    if (i >= nring) break;
+                    float Ss[32];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) Ss[e] = Sin[e] * (((e >> 1) & 1) ? Dh1[i] : Dh0[i]);
+                    write_state_tile(sm + held_tile(i), Ss, q4, lane);
+                }
                 if (kspan == PS - 1 && P.sf != nullptr) {   // final state D_span * S_in + S_local
-                    const float G0 = dcum[nch * 64 + r0], G1 = dcum[nch * 64 + r0 + 8];
+                    const float G0 = D0, G1 = D1;
                     float *sf = P.sf + (size_t)seq * kDK * kDV;
 #pragma unroll
                     for (int e = 0; e < 32; e += 2) {
@@ -881,7 +1018,6 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_pipe_kernel(const __grid_
                     int *rows = reinterpret_cast<int *>(sm + L::rowtab) + 64 * b;
                     fill_rowtab(P, seq, c0 + c, rows, rt);
                     if (rt == 0 && c < kMaxSpan) cmeta[2 * c + 1] = 0.f;
-                    wait_l(bar(sm, B_OPFULL + b), ph, to);
                     wait_l(bar(sm, B_MMA1 + b), ph, to);
                     tc_fence_after();
                     const bool slow = reinterpret_cast<const int *>(sm + L::slowf)[b] != 0;
@@ -903,49 +1039,27 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_pipe_kernel(const __grid_
                             pv[2 * (j + 4 * h) + hh] = *reinterpret_cast<const uint32_t *>(&v);
                         }
                     } else {
-                        uint32_t of[32];
+                        // copies for the out-of-line call: sc and pv never have their address
+                        // taken, so that the fast path keeps them in registers
+                        uint32_t scs[32], pvs[16];
+                        tmem_ld_wait();   // (the scores' loads complete before they are copied)
 #pragma unroll
-                        for (int e = 24; e < 32; ++e) of[e] = 0u;   // key block 3: never below the diagonal
-                        {
-                            uint32_t (&oa)[16] = *reinterpret_cast<uint32_t(*)[16]>(&of[0]);
-                            uint32_t (&ob)[8] = *reinterpret_cast<uint32_t(*)[8]>(&of[16]);
-                            tmem_ld_16x256b_x4(ta + 64, oa);
-                            tmem_ld_16x256b_x2(ta + 96, ob);
-                        }
-                        tmem_ld_wait();
-                        const int *fl = reinterpret_cast<const int *>(sm + L::bflag) + 4 * b;
-                        const bool exact = fl[q4] != 0;
-                        const __half *dx = reinterpret_cast<const __half *>(sm + L::diagx + b * 2048) + q4 * 256;
+                        for (int e = 0; e < 32; ++e) scs[e] = sc[e];
+                        pmx = readout_slow(sm, ta, scs, pvs, b, q4, r0, a2);
 #pragma unroll
-                        for (int e = 0; e < 32; e += 2) {
-                            const int h = e >> 4, j = (e >> 2) & 3, hh = (e >> 1) & 1;
-                            const int row = r0 + 8 * hh, col = 32 * h + 8 * j + a2;
-                            const int J = col >> 4;   // key block (col and col + 1 share it)
-                            float x0 = 0.f, x1 = 0.f;
-                            if (J < q4) {
-                                x0 = __uint_as_float(of[e]);
-                                x1 = __uint_as_float(of[e + 1]);
-                            } else if (J == q4) {
-                                if (exact) {
-                                    x0 = __half2float(dx[(row & 15) * 16 + (col & 15)]);
-                                    x1 = __half2float(dx[(row & 15) * 16 + ((col + 1) & 15)]);
-                                } else {
-                                    x0 = __uint_as_float(sc[e]);
-                                    x1 = __uint_as_float(sc[e + 1]);
-                                }
-                                x0 = col <= row ? x0 : 0.f;
-                                x1 = col + 1 <= row ? x1 : 0.f;
-                            }
-                            pmx = fmaxf(pmx, fmaxf(fabsf(x0), fabsf(x1)));
-                            const __half2 v = h2(x0, x1);
-                            pv[2 * (j + 4 * h) + hh] = *reinterpret_cast<const uint32_t *>(&v);
-                        }
+                        for (int e = 0; e < 16; ++e) pv[e] = pvs[e];
                     }
                     range_check(pmx);
                     tmem_st_16x128b_x8(ta, pv);
                     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
                     tc_fence_before();
-                    mbar_arrive(bar(sm, B_PREADY + b));
+                    named_sync(kBarRE, kREThreads);   // P complete; O of chunk c-2 read by every RE warp
+                    if (warp == kWarpRE) {
+                        // MMA 2 of chunk c, once U has written its S_prev
+                        wait_l(bar(sm, B_SPFULL + b), ph, to);
+                        tc_fence_after();
+                        issue_mma2(sm, sbase, tmem, b, c + 1 == nch);
+                    }
                 }
                 if (c >= 1) {
                     const int cp = c - 1;
@@ -956,7 +1070,6 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_pipe_kernel(const __grid_
                     ld_acc64(tmem + ((uint32_t)(32 * q4) << 16) + kColO + 64 * b, o);
                     tmem_ld_wait();
                     tc_fence_before();
-                    mbar_arrive(bar(sm, B_OFREE + b));
                     const float mx = store_out_tile(P, o, q4, lane, rt, sm + L::ostg,
                                                     reinterpret_cast<const int *>(sm + L::rowtab) + 64 * b, kBarRE);
                     range_check(mx);
@@ -968,78 +1081,81 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_pipe_kernel(const __grid_
             }
         } else {
             // ======================================================= gating group G
-            const int gw = warp - kWarpG, tg = tid - kWarpG * 32, t0 = 8 * gw;
-            float *htot = reinterpret_cast<float *>(sm + L::htot);
-            if (tg < 64) dcum[tg] = 1.f;
-            for (int c = 0; c < nch; ++c) {
+            // team b gates the chunks whose global index has parity b (operand buffer b)
+            const int team = (warp - kWarpG) >> 2, gw = (warp - kWarpG) & 3;
+            const int tt = tid - (kWarpG + 4 * team) * 32, t0 = 16 * gw;
+            const uint32_t bid = bar_team(team);
+            float *htot = reinterpret_cast<float *>(sm + L::htot) + team * 4 * 64;
+            for (int c = (int)(((uint32_t)team - gc0) & 1u); c < nch; c += 2) {
                 const uint32_t gc = gc0 + c, b = gc & 1u, s = gc % kNStage, ph = (gc >> 1) & 1u;
                 const bool held = c < nring;
+                // operand buffers b free.  Waited first: MMA 2 of chunk gc-2 completes only
+                // after the other team has gated chunk gc-3 (the slot's previous use), so the
+                // slot's barrier can no longer be a phase short when its parity is tested
+                if (gc >= 2) wait_l(bar(sm, B_MMA2 + b), ph ^ 1u, to);
                 wait_l(bar(sm, B_FULL + s), (gc / kNStage) & 1u, to);
-                if (gc >= 2) wait_l(bar(sm, B_MMA2 + b), ph ^ 1u, to);   // operand buffers b free
                 uint8_t *st = sm + L::stage + s * L::stage_bytes;
                 const uint8_t *meta = sm + L::meta + s * 128;
                 const int nrows = *reinterpret_cast<const int *>(meta + 64);
                 unsigned *wm = reinterpret_cast<unsigned *>(sm + L::wmax) + 16 * b;
                 int *bfl = reinterpret_cast<int *>(sm + L::bflag) + 4 * b;
-                if (tg < 4) bfl[tg] = 0;
-                // ---------- pass 1: raw rows -> registers, group prefix sums, maxima, V copy
-                GRegs R;
+                if (tt < 4) bfl[tt] = 0;
+                // ---------- pass 1: raw rows -> registers, prefix sums, maxima, V copy
+                // V rows into the scan-ordered operand tile first (row tt/2, 16-byte pieces
+                // 4 (tt%2) .. +3), so that their registers are free before the gating rows load
                 {
-                    const uint2 sr = *reinterpret_cast<const uint2 *>(meta + t0);
-                    __half2 qm = __float2half2_rn(0.f), km = qm;
+                    const int t = tt >> 1, pc = 4 * (tt & 1);
+                    const int r = meta[t];
+                    const uint8_t *vs = st + L::st_v + r * 128 + 16 * pc;
+                    uint4 v[4];
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const int r = ((u < 4 ? sr.x : sr.y) >> (8 * (u & 3))) & 0xff;
-                        const uint32_t o = r * 128 + 4 * lane;
-                        if (t0 + u < nrows) {
-                            R.g[u] = ld_gate2<kZ>(st + L::st_g + o, A.inv_tau);
-                            R.q[u] = *reinterpret_cast<const __half2 *>(st + L::st_q + o);
-                            R.k[u] = *reinterpret_cast<const __half2 *>(st + L::st_k + o);
-                        } else {
-                            R.g[u] = make_float2(0.f, 0.f);
-                            R.q[u] = __float2half2_rn(0.f);
-                            R.k[u] = R.q[u];
-                        }
-                        qm = __hmax2(qm, __habs2(R.q[u]));
-                        km = __hmax2(km, __habs2(R.k[u]));
-                    }
+                    for (int i = 0; i < 4; ++i) v[i] = *reinterpret_cast<const uint4 *>(vs + 16 * i);
+                    uint8_t *vo = sm + L::vop + b * kTile;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        *reinterpret_cast<uint4 *>(vo + sw_off(t, 8 * (pc + i))) =
+                            t < nrows ? v[i] : make_uint4(0u, 0u, 0u, 0u);
+                }
+                GRegs R;
+                const uint4 sr = *reinterpret_cast<const uint4 *>(meta + t0);
+                {
+                    __half2 qm = __float2half2_rn(0.f), km = qm;
                     float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        acc.x += R.g[u].x;
-                        acc.y += R.g[u].y;
+                    for (int u = 0; u < 16; ++u) {
+                        // every table entry names a row of the slot, so the loads are always
+                        // in bounds; rows past the grid are zeroed by select (no branch in
+                        // the unrolled loop)
+                        const uint32_t w4 = u < 4 ? sr.x : u < 8 ? sr.y : u < 12 ? sr.z : sr.w;
+                        const int r = (w4 >> (8 * (u & 3))) & 0xff;
+                        const uint32_t o = r * 128 + 4 * lane;
+                        const bool ok = t0 + u < nrows;
+                        const float2 gv = ld_gate2<kZ>(st + L::st_g + o, A.inv_tau);
+                        const uint32_t qb = *reinterpret_cast<const uint32_t *>(st + L::st_q + o);
+                        const uint32_t kb = *reinterpret_cast<const uint32_t *>(st + L::st_k + o);
+                        const uint32_t qz = ok ? qb : 0u, kz = ok ? kb : 0u;
+                        acc.x += ok ? gv.x : 0.f;
+                        acc.y += ok ? gv.y : 0.f;
                         R.p[u] = acc;
+                        qm = __hmax2(qm, __habs2(*reinterpret_cast<const __half2 *>(&qz)));
+                        km = __hmax2(km, __habs2(*reinterpret_cast<const __half2 *>(&kz)));
                     }
                     *reinterpret_cast<float2 *>(htot + gw * 64 + 2 * lane) = acc;
                     const unsigned wq = __reduce_max_sync(0xffffffffu, __float_as_uint(fmaxf(__low2float(qm), __high2float(qm))));
                     const unsigned wk = __reduce_max_sync(0xffffffffu, __float_as_uint(fmaxf(__low2float(km), __high2float(km))));
                     if (lane == 0) {
                         wm[gw] = wq;
-                        wm[8 + gw] = wk;
-                    }
-                    // V rows into the scan-ordered operand tile: row tg/4, 16-byte pieces
-                    // 2 (tg%4), +1
-                    {
-                        const int t = tg >> 2, pc = 2 * (tg & 3);
-                        const int r = meta[t];
-                        uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
-                        if (t < nrows) {
-                            v0 = *reinterpret_cast<const uint4 *>(st + L::st_v + r * 128 + 16 * pc);
-                            v1 = *reinterpret_cast<const uint4 *>(st + L::st_v + r * 128 + 16 * pc + 16);
-                        }
-                        uint8_t *vo = sm + L::vop + b * kTile;
-                        *reinterpret_cast<uint4 *>(vo + sw_off(t, 8 * pc)) = v0;
-                        *reinterpret_cast<uint4 *>(vo + sw_off(t, 8 * pc + 8)) = v1;
+                        wm[4 + gw] = wk;
                     }
                 }
-                named_sync(kBarG, kGThreads);
+                named_sync(bid, kTeamThreads);
                 // ---------- pass 2
-                float2 ht[8];
+                float2 ht[4];
 #pragma unroll
-                for (int w = 0; w < 8; ++w) ht[w] = *reinterpret_cast<const float2 *>(htot + w * 64 + 2 * lane);
+                for (int w = 0; w < 4; ++w) ht[w] = *reinterpret_cast<const float2 *>(htot + w * 64 + 2 * lane);
                 float2 off = make_float2(0.f, 0.f), bC = make_float2(0.f, 0.f);
 #pragma unroll
-                for (int w = 0; w < 8; ++w) {
+                for (int w = 0; w < 4; ++w) {
                     if (w < gw) {
                         off.x += ht[w].x;
                         off.y += ht[w].y;
@@ -1047,58 +1163,55 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_pipe_kernel(const __grid_
                     bC.x += ht[w].x;
                     bC.y += ht[w].y;
                 }
-                unsigned kmx = 0u, qmx = 0u;
-#pragma unroll
-                for (int w = 0; w < 8; ++w) {
-                    qmx = max(qmx, wm[w]);
-                    kmx = max(kmx, wm[8 + w]);
-                }
+                const uint4 wq4 = *reinterpret_cast<const uint4 *>(wm), wk4 = *reinterpret_cast<const uint4 *>(wm + 4);
+                const unsigned qmx = max(max(wq4.x, wq4.y), max(wq4.z, wq4.w));
+                const unsigned kmx = max(max(wk4.x, wk4.y), max(wk4.z, wk4.w));
                 const bool bad = !(bC.x >= kFastMinLogDecay) || !(bC.y >= kFastMinLogDecay) ||
                                  __uint_as_float(kmx) > kFastMaxK;
                 // every warp's lanes cover all 64 channels: a warp vote is the chunk's decision
                 const bool slow = __any_sync(0xffffffffu, bad);
-                const float2 Dc = *reinterpret_cast<const float2 *>(dcum + (held ? c : 0) * 64 + 2 * lane);
                 uint8_t *qo = sm + L::qint + b * kTile;
                 uint8_t *ko = sm + L::kt + b * kTile;
                 uint8_t *ro = sm + L::ring + (held ? c : 0) * kTile;
                 if (!slow) {
-                    if (tg == 0) mbar_arrive(bar(sm, B_EMPTY + s));   // raw rows consumed
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const float x0 = (off.x + R.p[u].x) * kLog2e, x1 = (off.y + R.p[u].y) * kLog2e;
-                        const float e0 = ex2a(x0), e1 = ex2a(x1);
-                        const __half2 qi = __hmul2(R.q[u], h2(e0, e1));
-                        const uint32_t o = sw_off(t0 + u, 2 * lane);
-                        sth2(qo + o, qi);
-                        sth2(ko + o, __hmul2(R.k[u], h2(ex2a(-x0), ex2a(-x1))));
-                        if (held) {   // Qint * D_c in fp32, one rounding
-                            const float2 qf = __half22float2(R.q[u]);
-                            sth2(ro + o, h2(qf.x * e0 * Dc.x, qf.y * e1 * Dc.y));
-                        }
-                    }
+                    if (held)
+                        gate_fast<true>(R, off, st, sr, nrows, qo, ko, ro, t0, lane);
+                    else
+                        gate_fast<false>(R, off, st, sr, nrows, qo, ko, ro, t0, lane);
                 } else {
-                    gate_slow<kZ>(sm, R, ht, gw, lane, tg, st, meta, nrows, qo, ko, ro, held, Dc, bfl, b, A.inv_tau);
+                    // copies for the out-of-line call: R and ht themselves never have their
+                    // address taken, so that the fast path keeps them in registers
+                    GRegs Rs = R;
+                    float2 hts[4];
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) hts[w] = ht[w];
+                    gate_slow<kZ>(sm, Rs, hts, gw, lane, tt, bid, st, meta, nrows, qo, ko, ro, held, bfl, b, A.inv_tau);
                 }
-                // chunk decay and decay products from the span start
+                // the chunk's decay (the state group keeps the products from the span start)
                 if (gw == 0) {
                     const float2 d = make_float2(ex2a(bC.x * kLog2e), ex2a(bC.y * kLog2e));
                     *reinterpret_cast<float2 *>(sm + L::dloc + b * 256 + 8 * lane) = d;
-                    if (c < kMaxSpan) {
-                        const float2 dc = *reinterpret_cast<const float2 *>(dcum + c * 64 + 2 * lane);
-                        *reinterpret_cast<float2 *>(dcum + (c + 1) * 64 + 2 * lane) = make_float2(dc.x * d.x, dc.y * d.y);
-                    }
                     if (lane == 0 && c < kMaxSpan) cmeta[2 * c] = __uint_as_float(qmx);
                 }
                 fence_proxy_async_cta();
-                named_sync(kBarG, kGThreads);
-                if (tg == 0) {
+                named_sync(bid, kTeamThreads);
+                if (tt == 0) {
                     reinterpret_cast<int *>(sm + L::slowf)[b] = slow ? 1 : 0;
-                    mbar_arrive(bar(sm, B_OPFULL + b));
+                    mbar_arrive(bar(sm, B_OPFULL + b));   // MMA 1 may be issued
+                }
+                // the slot is free: the team's first warp loads chunk c+3 into it (on the
+                // sub-block path MMA 1 reads operands overlaid on the slot: after it completes)
+                if (gw == 0 && c + kNStage < nch) {
+                    if (slow) wait_l(bar(sm, B_MMA1 + b), ph, to);
+                    load_chunk(A, sm, sbase, s, seq, c0 + c + kNStage, lane);
                 }
             }
         }
         gc0 += (uint32_t)nch;
         __syncthreads();
+        // the next sequence's first chunks land while this one's corrections run (the
+        // staging slots are free: every chunk gated, the look-back slots read)
+        if (warp == kWarpG && seq + ngrp < P.n_seq) load_head(A, sm, sbase, gc0, seq + ngrp, lane);
 
         if (later) {
             __syncthreads();   // S_in operand, row maxima, final state written
@@ -1169,7 +1282,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_pipe_kernel(const __grid_
                             pg[u] = acc;
                         }
                         *reinterpret_cast<float2 *>(htot + gw * 64 + 2 * lane) = acc;
-                        named_sync(kBarG, kGThreads);
+                        named_sync(kBarGAll, kGThreads);
                         float2 offv = make_float2(0.f, 0.f);
                         for (int w = 0; w < gw; ++w) {
                             const float2 x = *reinterpret_cast<const float2 *>(htot + w * 64 + 2 * lane);
@@ -1185,22 +1298,23 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_pipe_kernel(const __grid_
                                  h2(qf.x * ex2a((offv.x + pg[u].x) * kLog2e) * Dc.x,
                                     qf.y * ex2a((offv.y + pg[u].y) * kLog2e) * Dc.y));
                         }
-                        named_sync(kBarG, kGThreads);   // htot reused by the next chunk
+                        named_sync(kBarGAll, kGThreads);   // htot reused by the next chunk
                     }
                     (void)tg;
                 }
                 fence_proxy_async_cta();
                 __syncthreads();
-                if (warp == kWarpMMA) {
+                if (warp == kWarpRE) {
                     tc_fence_after();
                     if (elect_one_sync()) {
                         constexpr uint32_t id_o = idesc_f16_f32(64, kDV, false, true);
-                        const uint32_t ba = sbase + L::sop;
-                        for (int li = 0; li < nl; ++li)
+                        for (int li = 0; li < nl; ++li) {
+                            const uint32_t ba = sbase + (batch == 0 ? held_tile(li) : L::vop + kTile);
 #pragma unroll
                             for (int kk = 0; kk < 4; ++kk)
                                 umma_f16(tmem + 64 * li, desc_sw128(qaddr[li] + kk * 32, 16, 1024),
                                          desc_sw128(ba + kk * 2048, kTile, 1024), id_o, kk > 0 ? 1u : 0u);
+                        }
                         umma_commit(bar(sm, B_FIX));
                     }
                     __syncwarp();
@@ -1237,7 +1351,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_pipe_kernel(const __grid_
         while (globaltimer_ns() - t0 < 1000000ull) {
         }
     }
-    if (warp == kWarpMMA) tmem_dealloc(tmem, kTmemCols);
+    if (warp == kWarpU) tmem_dealloc(tmem, kTmemCols);
 }
 
 }  // namespace pp

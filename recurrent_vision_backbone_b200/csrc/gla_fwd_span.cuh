@@ -203,8 +203,10 @@ __device__ __forceinline__ void red_dec_gpu(unsigned *p) {   // *p -= 1, relaxed
 __device__ __forceinline__ bool flag_wait_bounded(const unsigned *f, uint64_t limit_ns) {
     if (ld_acquire_gpu(f) != 0u) return true;
     const long long t0 = cycles(), lim = cycles_of_ns(limit_ns);
-    while (ld_acquire_gpu(f) == 0u)
+    while (ld_acquire_gpu(f) == 0u) {
         if (cycles() - t0 > lim) return false;
+        __nanosleep(32);
+    }
     return true;
 }
 

@@ -1327,6 +1327,119 @@ extern "C" gtr_status_t gtr_gla_fwd_z(const gtr_half_t *q, const gtr_half_t *k, 
     return cuda_status(launch(prm, pl, ws, s, 1.f / tau));
 }
 
+// ------------------------------------------------------------------ layer stacks
+// Graphs of recorded stacks, keyed by the layer list and shape (a few recent ones).
+struct StackEntry {
+    int dev, n, B, heads, H, W, dk, dv;
+    gtr_gla_layer_t layers[64];
+    cudaGraphExec_t exec;
+};
+static StackEntry g_stacks[8];
+static int g_stacks_next;
+
+static bool same_layer(const gtr_gla_layer_t &a, const gtr_gla_layer_t &b) {   // field by field (no padding)
+    return a.q == b.q && a.k == b.k && a.v == b.v && a.g == b.g && a.init_state == b.init_state && a.out == b.out &&
+           a.final_state == b.final_state && a.direction == b.direction;
+}
+
+static bool same_stack(const StackEntry &e, int dev, const gtr_gla_layer_t *layers, int n, int B, int heads, int H,
+                       int W, int dk, int dv) {
+    if (e.exec == nullptr || e.dev != dev || e.n != n || e.B != B || e.heads != heads || e.H != H || e.W != W ||
+        e.dk != dk || e.dv != dv)
+        return false;
+    for (int i = 0; i < n; ++i)
+        if (!same_layer(e.layers[i], layers[i])) return false;
+    return true;
+}
+
+// per device: the private stream that stacks are recorded on
+static cudaStream_t g_rec_stream[64];
+
+extern "C" gtr_status_t gtr_gla_fwd_stack(const gtr_gla_layer_t *layers, int n_layers, int B, int heads, int Hgrid,
+                                          int Wgrid, int dk, int dv, int chunk, void *stream) {
+    if (layers == nullptr || n_layers < 1 || n_layers > 64) return GTR_ERR_INVALID_ARG;
+    for (int i = 0; i < n_layers; ++i) {
+        const gtr_gla_layer_t &L = layers[i];
+        const gtr_status_t st = check_args(L.q, L.k, L.v, L.g, B, heads, Hgrid, Wgrid, dk, dv, L.direction, chunk,
+                                           L.init_state, L.out, L.final_state);
+        if (st != GTR_OK) return st;
+    }
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int dev = current_device();
+    // every layer has the same plan; its workspace exists before any recording starts
+    const Plan pl = make_plan((long)B * heads, (long)(((long long)Hgrid * Wgrid + kChunk - 1) / kChunk), dk, true);
+    void *ws = nullptr;
+    if (pl.ws_bytes > 0) {
+        const gtr_status_t wst = cuda_status(default_workspace(dev, pl.ws_bytes, s, &ws));
+        if (wst != GTR_OK) return wst;
+    }
+    const auto enqueue = [&]() -> cudaError_t {
+        for (int i = 0; i < n_layers; ++i) {
+            const gtr_gla_layer_t &L = layers[i];
+            const Params prm = make_params(L.q, L.k, L.v, L.g, B, heads, Hgrid, Wgrid, L.direction, L.init_state,
+                                           L.out, L.final_state);
+            const cudaError_t e = launch(prm, pl, ws, s);
+            if (e != cudaSuccess) return e;
+        }
+        return cudaSuccess;
+    };
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    cudaError_t e = cudaStreamIsCapturing(s, &cs);
+    if (e != cudaSuccess) return cuda_status(e);
+    if (cs != cudaStreamCaptureStatusNone || (long long)Hgrid * Wgrid == 0) return cuda_status(enqueue());
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        for (const StackEntry &en : g_stacks)
+            if (same_stack(en, dev, layers, n_layers, B, heads, Hgrid, Wgrid, dk, dv))
+                return cuda_status(cudaGraphLaunch(en.exec, s));
+    }
+    // record the stack once, then replay it on the caller's stream.  Recording runs on a
+    // private stream: the caller's may be the legacy default stream, which cannot be
+    // captured (recording executes nothing, so the private stream needs no ordering)
+    cudaStream_t rec = nullptr;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (g_rec_stream[dev] == nullptr &&
+            (e = cudaStreamCreateWithFlags(&g_rec_stream[dev], cudaStreamNonBlocking)) != cudaSuccess) {
+            g_rec_stream[dev] = nullptr;
+            return cuda_status(e);
+        }
+        rec = g_rec_stream[dev];
+    }
+    const cudaStream_t caller = s;
+    s = rec;   // `enqueue` launches on `s`
+    e = cudaStreamBeginCapture(rec, cudaStreamCaptureModeThreadLocal);
+    if (e != cudaSuccess) return cuda_status(e);
+    const cudaError_t le = enqueue();
+    cudaGraph_t graph = nullptr;
+    e = cudaStreamEndCapture(rec, &graph);
+    s = caller;
+    if (le != cudaSuccess || e != cudaSuccess) {
+        if (graph) cudaGraphDestroy(graph);
+        return cuda_status(le != cudaSuccess ? le : e);
+    }
+    cudaGraphExec_t exec = nullptr;
+    e = cudaGraphInstantiate(&exec, graph, 0);
+    cudaGraphDestroy(graph);
+    if (e != cudaSuccess) return cuda_status(e);
+    e = cudaGraphLaunch(exec, s);
+    std::lock_guard<std::mutex> lk(g_mu);
+    StackEntry &slot = g_stacks[g_stacks_next];
+    if (slot.exec != nullptr) cudaGraphExecDestroy(slot.exec);
+    slot.dev = dev;
+    slot.n = n_layers;
+    slot.B = B;
+    slot.heads = heads;
+    slot.H = Hgrid;
+    slot.W = Wgrid;
+    slot.dk = dk;
+    slot.dv = dv;
+    memcpy(slot.layers, layers, sizeof(gtr_gla_layer_t) * (size_t)n_layers);
+    slot.exec = exec;
+    g_stacks_next = (g_stacks_next + 1) % (int)(sizeof(g_stacks) / sizeof(g_stacks[0]));
+    return cuda_status(e);
+}
+
 extern "C" gtr_status_t gtr_gla_init(void *stream) {
     const int dev = current_device();
     const int cap = span_capacity(dev, num_sms(dev), true);

@@ -52,14 +52,31 @@ __device__ __forceinline__ long long cycles() { return clock64(); }
 // so that the real bound is `ns` or longer at any clock.
 __device__ __forceinline__ long long cycles_of_ns(uint64_t ns) { return (long long)(2 * ns); }
 
+// try_wait with a suspend-time hint: a thread whose phase is not complete is suspended
+// (it issues nothing) until the phase completes or about `hint_ns` pass, instead of
+// returning at once and spinning -- spinning waiters take the issue slots of the warps
+// that do the work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Waits for the phase with the given parity to complete, for at least `limit_ns`
 // nanoseconds before giving up.  Returns false if the limit ran out.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
                                                   uint64_t limit_ns) {
-    if (mbar_try_wait(bar, parity)) return true;
+    constexpr uint32_t kSleepNs = 1000000;   // 1 ms per suspension, far below any limit used
+    if (mbar_try_wait_sleep(bar, parity, kSleepNs)) return true;
     const long long t0 = cycles(), lim = cycles_of_ns(limit_ns);
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_sleep(bar, parity, kSleepNs)) return true;
         if (cycles() - t0 > lim) return false;
     }
 }

@@ -21,12 +21,19 @@ GTR_OK, GTR_ERR_INVALID_ARG, GTR_ERR_UNSUPPORTED, GTR_ERR_CUDA, GTR_ERR_TIMEOUT,
 L2R, R2L, T2B, B2T = 0, 1, 2, 3
 STATIC_WS_BYTES = 4 << 20   # GTR_STATIC_WS_BYTES
 
-EXPORTED_SYMBOLS = ("gtr_gla_fwd", "gtr_gla_fwd_z", "gtr_gla_init", "gtr_gla_workspace_bytes", "gtr_gla_fwd_ws",
+EXPORTED_SYMBOLS = ("gtr_gla_fwd", "gtr_gla_fwd_z", "gtr_gla_fwd_stack", "gtr_gla_init", "gtr_gla_workspace_bytes", "gtr_gla_fwd_ws",
                     "gtr_gla_fwd_static", "gtr_gla_device_status", "gtr_status_str", "gtr_gla_plan", "gtr_gla_version",
                     "gtr_gla_last_error", "gtr_gla_selftest_timeout")
 
 _lock = threading.Lock()
 _lib = None
+
+
+class Layer(ctypes.Structure):
+    """gtr_gla_layer_t: one layer call of a stack (device pointers and a direction)."""
+    _fields_ = [("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+                ("g", ctypes.c_void_p), ("init_state", ctypes.c_void_p), ("out", ctypes.c_void_p),
+                ("final_state", ctypes.c_void_p), ("direction", ctypes.c_int)]
 
 
 class GTRError(RuntimeError):
@@ -53,6 +60,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.gtr_gla_fwd.argtypes = [vp, vp, vp, vp] + [i] * 8 + [vp, vp, vp, vp]
         lib.gtr_gla_fwd_z.restype = i
         lib.gtr_gla_fwd_z.argtypes = [vp, vp, vp, vp, ctypes.c_float] + [i] * 8 + [vp, vp, vp, vp]
+        lib.gtr_gla_fwd_stack.restype = i
+        lib.gtr_gla_fwd_stack.argtypes = [ctypes.POINTER(Layer)] + [i] * 8 + [vp]
         lib.gtr_gla_fwd_static.restype = i
         lib.gtr_gla_fwd_static.argtypes = [vp, vp, vp, vp] + [i] * 8 + [vp, vp, vp, vp]
         lib.gtr_gla_workspace_bytes.restype = ctypes.c_size_t
@@ -154,6 +163,33 @@ def gtr_gla_fwd_z(q, k, v, z, tau: float, Hgrid: int, Wgrid: int, direction: int
     if st != GTR_OK:
         raise GTRError(st, "gtr_gla_fwd_z")
     return out, final_state
+
+
+def gtr_gla_fwd_stack(layers, Hgrid: int, Wgrid: int, chunk: int = 64, stream=None):
+    """A stack of layer calls of one shape, in order (see gtr_gla_fwd_stack in the header).
+
+    layers: sequence of dicts with q, k, v, g (fp16 [B,N,heads,d]), direction, and optional
+    init_state, out, final_state (final_state=True allocates one).  Returns the list of
+    (out, final_state) per layer."""
+    arr = (Layer * len(layers))()
+    results = []
+    shape = None
+    for i, L in enumerate(layers):
+        sh, out, fs = _prepare(L["q"], L["k"], L["v"], L["g"], Hgrid, Wgrid, L.get("init_state"),
+                               L.get("out"), L.get("final_state"))
+        if shape is not None and sh != shape:
+            raise ValueError("every layer of a stack has the same shape")
+        shape = sh
+        arr[i] = Layer(L["q"].data_ptr(), L["k"].data_ptr(), L["v"].data_ptr(), L["g"].data_ptr(),
+                       None if L.get("init_state") is None else L["init_state"].data_ptr(),
+                       out.data_ptr(), None if fs is None else fs.data_ptr(), int(L["direction"]))
+        results.append((out, fs))
+    B, heads, dk, dv = shape
+    st = load().gtr_gla_fwd_stack(arr, len(layers), B, heads, Hgrid, Wgrid, dk, dv, int(chunk),
+                                  _stream_handle(stream))
+    if st != GTR_OK:
+        raise GTRError(st, "gtr_gla_fwd_stack")
+    return results
 
 
 def gtr_gla_fwd_static(q, k, v, g, Hgrid: int, Wgrid: int, direction: int, init_state=None,
