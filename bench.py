@@ -257,30 +257,37 @@ class Workload:
                                  init_state=inp["s0"], out=out, final_state=sf, stream=stream)
 
     def capture(self, stream, steps):
-        """Graphs replaying the rotating sets: `full` holds one step per set, `part` the
-        first steps % n_sets of them, so that any step count is replayed exactly."""
+        """Graphs replaying the rotating sets: `graph` holds one step per set; a graph of
+        the first r sets serves any step count with remainder r (the one of `steps` is
+        recorded here, others when first replayed, outside any timed region)."""
         with torch.cuda.stream(stream):   # warm the launch path once outside capture
             self.launch_step(0, stream)
         stream.synchronize()
-
-        def graph_of(n):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                for s in range(n):
-                    self.launch_step(s, torch.cuda.current_stream())
-            return g
-
-        self.graph = graph_of(self.n_sets)
-        r = steps % self.n_sets
-        self.part = graph_of(r) if r else None
+        self.stream = stream
+        self.parts = {}
+        self.graph = self._graph_of(self.n_sets)
+        self._part(steps % self.n_sets)
         return self.n_sets
+
+    def _graph_of(self, n):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=self.stream):
+            for s in range(n):
+                self.launch_step(s, torch.cuda.current_stream())
+        return g
+
+    def _part(self, r):
+        if r and r not in self.parts:
+            self.parts[r] = self._graph_of(r)
+        return self.parts.get(r)
 
     def replay(self, steps):
         """Replays exactly `steps` steps (whole rotations, then the remainder)."""
+        part = self._part(steps % self.n_sets)
         for _ in range(steps // self.n_sets):
             self.graph.replay()
-        if steps % self.n_sets:
-            self.part.replay()
+        if part is not None:
+            part.replay()
 
     def calls_per_step(self):
         return len(self.w.call_directions())

@@ -14,7 +14,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 SOURCES = [os.path.join(CSRC, "gtr_gla.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, n) for n in ("sm100_ptx.cuh", "gla_fwd_ws.cuh", "gla_fwd_span.cuh", "gla_fwd_pipe.cuh")]
+DEPS = SOURCES + [os.path.join(CSRC, n) for n in ("sm100_ptx.cuh", "gla_fwd_span.cuh", "gla_fwd_pipe.cuh")]
 DEPS += [os.path.join(ROOT, "include", "gtr_gla.h")]
 LIB = os.path.join(HERE, "libgtr_gla.so")
 

@@ -58,6 +58,7 @@ constexpr int kDK = 64;
 constexpr int kNStage = 3;                   // staging slots
 constexpr int kRing = 3;                     // chunks of a later span whose Qint * D_c stays in smem
 constexpr int kMaxSpan = 32;                 // chunks of a span with recorded decays (P > 1)
+constexpr int kPrefetchChunks = 8;           // chunks past the ring whose rows are prefetched for the corrections
 constexpr int kThreads = 512;                // 16 warps (128 registers each)
 constexpr int kWarpU = 0, kWarpRE = 4, kWarpG = 8;
 constexpr int kUThreads = 128, kREThreads = 128, kGThreads = 256;
@@ -70,6 +71,7 @@ constexpr int kAggBytes = kAggFloats * 4;    // 16640
 constexpr int kFoldSlots = 8;                // aggregates copied into smem at a time
 constexpr int kFlagStride = 32;              // one 128-byte line per publish flag
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kFastMinLogDecay = -6.f;     // fast path: chunk decay >= e^-6
 constexpr float kFastMaxK = 100.f;           //            and |k| <= 100
 constexpr float kDiagMinLogTotal = -8.f;     // sub-block path: diagonal block decay >= e^-8
@@ -125,7 +127,7 @@ static_assert(L::dcum % 16 == 0 && L::htot % 16 == 0 && L::meta % 16 == 0 && L::
 static_assert(L::qint % 1024 == 0 && L::ring % 1024 == 0 && L::ostg % 1024 == 0, "tile alignment");
 
 enum {
-    B_FULL = 0,     // [3] staging slot landed (TMA transaction count)
+    B_FULL = 0,     // [3][2] staging slot s landed, for a chunk of parity t (TMA transaction count)
     B_OPFULL = 6,   // [2] G done: Qint, K~, V, d, flags of a chunk
     B_MMA1 = 8,     // [2] MMA 1 complete
     B_SPFULL = 12,  // [2] S_prev operand written (U)
@@ -268,7 +270,7 @@ __device__ __forceinline__ void write_meta(const Params &P, uint8_t *meta, int c
 
 // TMA copies of chunk `cabs` of sequence `seq` into staging slot `slot` (one lane).
 // Returns the bytes the copies deliver.
-__device__ __forceinline__ uint32_t issue_chunk(const Args &A, uint32_t slot, int seq, int cabs, uint32_t mbar,
+__device__ __noinline__ uint32_t issue_chunk(const Args &A, uint32_t slot, int seq, int cabs, uint32_t mbar,
                                                 bool count_only) {
     const Params &P = A.P;
     const int p0 = cabs * kChunk, pend = min(p0 + kChunk, P.N);
@@ -299,10 +301,11 @@ __device__ __forceinline__ uint32_t issue_chunk(const Args &A, uint32_t slot, in
             }
             int off = 0;
             const uint32_t row0 = (uint32_t)(p - p0);
+#pragma unroll 1
             for (int lb = 6; lb >= 0; --lb) {
                 if (!(len & (1 << lb))) continue;
                 const uint32_t d = slot + (row0 + off) * 128u;
-#pragma unroll
+#pragma unroll 1
                 for (int ten = 0; ten < 4; ++ten) {
                     if (P.dir == GTR_R2L)
                         tma_4d(d + ten * kTile, &A.maps.m[ten][lb], 0, hh, c2 + off, bb, mbar);
@@ -317,16 +320,24 @@ __device__ __forceinline__ uint32_t issue_chunk(const Args &A, uint32_t slot, in
     return (uint32_t)(pend - p0) * kRowBytes;
 }
 
-// Chunk `cabs` of sequence `seq` into staging slot `s` (one warp): the row table, the
-// expected transaction bytes and the copies.
-__device__ __forceinline__ void load_chunk(const Args &A, uint8_t *sm, uint32_t sbase, uint32_t s, int seq,
+// Staging barrier of the CTA's chunk number gc: slot gc % 3, and one barrier per chunk
+// parity, so that each barrier's phases belong to one gating team, which waits for them
+// in order (a shared barrier could complete the other team's phase in between and
+// alias the parity).
+__device__ __forceinline__ uint32_t full_bar(uint32_t gc) { return B_FULL + 2u * (gc % kNStage) + (gc & 1u); }
+__device__ __forceinline__ uint32_t full_parity(uint32_t gc) { return (gc / (2u * kNStage)) & 1u; }
+
+// Chunk `cabs` of sequence `seq`, the CTA's chunk number gc, into its staging slot (one
+// warp): the row table, the expected transaction bytes and the copies.
+__device__ __noinline__ void load_chunk(const Args &A, uint8_t *sm, uint32_t sbase, uint32_t gc, int seq,
                                            int cabs, int lane) {
+    const uint32_t s = gc % kNStage;
     write_meta(A.P, sm + L::meta + s * 128, cabs, lane);
     __syncwarp();
     if (lane == 0) {
-        const uint32_t mb = smem_u32(bar(sm, B_FULL + s));
+        const uint32_t mb = smem_u32(bar(sm, full_bar(gc)));
         const uint32_t slot = sbase + L::stage + s * L::stage_bytes;
-        mbar_arrive_expect_tx(bar(sm, B_FULL + s), issue_chunk(A, slot, seq, cabs, mb, true));
+        mbar_arrive_expect_tx(bar(sm, full_bar(gc)), issue_chunk(A, slot, seq, cabs, mb, true));
         issue_chunk(A, slot, seq, cabs, mb, false);
     }
     __syncwarp();
@@ -339,7 +350,7 @@ __device__ __forceinline__ void load_head(const Args &A, uint8_t *sm, uint32_t s
     const int kspan = (int)blockIdx.x % A.PS;
     const int c0 = kspan * A.Lc;
     const int nch = min(A.Lc, A.P.n_chunks - c0);
-    for (int c = 0; c < min(kNStage, nch); ++c) load_chunk(A, sm, sbase, (gc0 + c) % kNStage, seq, c0 + c, lane);
+    for (int c = 0; c < min(kNStage, nch); ++c) load_chunk(A, sm, sbase, gc0 + c, seq, c0 + c, lane);
 }
 
 // ------------------------------------------------------------------ gating (group G)
@@ -348,37 +359,80 @@ __device__ __forceinline__ void load_head(const Args &A, uint8_t *sm, uint32_t s
 // chunk's scan rows 16w .. 16w+15 (sub-block w of the sub-block path), lane l channels
 // 2l, 2l+1.
 struct GRegs {
-    float2 p[16];   // prefix sums of the log-decay over the warp's 16 rows
+    float2 p[16];   // prefix sums of the log-decay over a warp's 16 rows
 };
 
-// Row u of the warp's 16 (staging row from the table words, zero past the grid).
-__device__ __forceinline__ uint32_t row_off(const uint4 &sr, int u, int lane) {
-    const uint32_t w4 = u < 4 ? sr.x : u < 8 ? sr.y : u < 12 ? sr.z : sr.w;
-    return ((w4 >> (8 * (u & 3))) & 0xffu) * 128u + 4u * (uint32_t)lane;
+// |x| of the eight fp16 values of a 16-byte word, as their bit patterns' per-half maximum
+// (for non-negative fp16 values the bit patterns order like the values; a NaN orders
+// above every finite value)
+__device__ __forceinline__ uint32_t umax16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
 }
-__device__ __forceinline__ __half2 ld_row_h2(const uint8_t *p, bool ok) {
-    const uint32_t x = ok ? *reinterpret_cast<const uint32_t *>(p) : 0u;
-    return *reinterpret_cast<const __half2 *>(&x);
+__device__ __forceinline__ uint32_t absmax8(const uint4 &x) {
+    return umax16x2(umax16x2(x.x & 0x7fff7fffu, x.y & 0x7fff7fffu), umax16x2(x.z & 0x7fff7fffu, x.w & 0x7fff7fffu));
+}
+__device__ __forceinline__ float half_bits_to_float(uint32_t h) {
+    return __half2float(__ushort_as_half((unsigned short)h));
 }
 
-// Fast-path gating of the warp's sixteen rows (chunk decay >= e^-6, |k| <= 100):
-// Qint = q exp(b), K~ = k exp(-b) with b = off + the row's prefix sum; a held chunk also
-// keeps Qint in its ring tile.  (Two instances: a branch inside the unrolled loop would
-// keep the scheduler from overlapping the rows.)
-template <bool kHeld>
-__device__ __forceinline__ void gate_fast(const GRegs &R, float2 off, const uint8_t *st, const uint4 &sr, int nrows,
-                                          uint8_t *qo, uint8_t *ko, uint8_t *ro, int t0, int lane) {
+// Eight consecutive channels of a gate row as log-decays (from z when kZ).
+template <bool kZ>
+__device__ __forceinline__ void ld_gate8(const uint8_t *p, float (&g)[8], float inv_tau) {
+    const uint4 w = *reinterpret_cast<const uint4 *>(p);
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-    for (int u = 0; u < 16; ++u) {
-        const uint32_t so = row_off(sr, u, lane);
-        const bool ok = t0 + u < nrows;
-        const __half2 qv = ld_row_h2(st + L::st_q + so, ok), kv = ld_row_h2(st + L::st_k + so, ok);
-        const float x0 = (off.x + R.p[u].x) * kLog2e, x1 = (off.y + R.p[u].y) * kLog2e;
-        const __half2 qi = __hmul2(qv, h2(ex2a(x0), ex2a(x1)));
-        const uint32_t o = sw_off(t0 + u, 2 * lane);
-        sth2(qo + o, qi);
-        sth2(ko + o, __hmul2(kv, h2(ex2a(-x0), ex2a(-x1))));
-        if constexpr (kHeld) sth2(ro + o, qi);
+    for (int m = 0; m < 4; ++m) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&u[m]));
+        g[2 * m] = f.x;
+        g[2 * m + 1] = f.y;
+    }
+    if constexpr (kZ) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) g[j] = gate_of(g[j], inv_tau);
+    }
+}
+
+__device__ __forceinline__ uint32_t hadd2_bits(uint32_t a, uint32_t b) {
+    const __half2 r = __hadd2(*reinterpret_cast<const __half2 *>(&a), *reinterpret_cast<const __half2 *>(&b));
+    return *reinterpret_cast<const uint32_t *>(&r);
+}
+__device__ __forceinline__ uint32_t hmul2_bits(uint32_t a, float x0, float x1) {
+    const __half2 r = __hmul2(*reinterpret_cast<const __half2 *>(&a), h2(x0, x1));
+    return *reinterpret_cast<const uint32_t *>(&r);
+}
+
+// Fast-path gating of the lane's four rows tb .. tb+3, channels 8 cg .. 8 cg + 7 (chunk
+// decay >= e^-6, |k| <= 100): Qint = q exp(b), K~ = k exp(-b), with b (log2 units) the
+// chunk-inclusive prefix sum x[i][j]; 16-byte loads and stores (a lane's eight channels
+// are one 16-byte unit of the 128-byte-swizzled tile).  A held chunk also keeps Qint in
+// its ring tile.  (Two instances: a branch inside the unrolled loop would keep the
+// scheduler from overlapping the rows.)
+template <bool kHeld>
+__device__ __forceinline__ void gate_fast(const float (&x)[4][8], const uint8_t *st, uint32_t rw, int tb, int nrows,
+                                          int cg, uint8_t *qo, uint8_t *ko, uint8_t *ro) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int t = tb + i;
+        const uint32_t o = ((rw >> (8 * i)) & 0xffu) * 128u + 16u * (uint32_t)cg;
+        const bool ok = t < nrows;
+        uint4 q4 = *reinterpret_cast<const uint4 *>(st + L::st_q + o);
+        uint4 k4 = *reinterpret_cast<const uint4 *>(st + L::st_k + o);
+        if (!ok) q4 = k4 = make_uint4(0u, 0u, 0u, 0u);   // rows past the grid
+        uint4 qi, ki;
+        qi.x = hmul2_bits(q4.x, ex2a(x[i][0]), ex2a(x[i][1]));
+        qi.y = hmul2_bits(q4.y, ex2a(x[i][2]), ex2a(x[i][3]));
+        qi.z = hmul2_bits(q4.z, ex2a(x[i][4]), ex2a(x[i][5]));
+        qi.w = hmul2_bits(q4.w, ex2a(x[i][6]), ex2a(x[i][7]));
+        ki.x = hmul2_bits(k4.x, ex2a(-x[i][0]), ex2a(-x[i][1]));
+        ki.y = hmul2_bits(k4.y, ex2a(-x[i][2]), ex2a(-x[i][3]));
+        ki.z = hmul2_bits(k4.z, ex2a(-x[i][4]), ex2a(-x[i][5]));
+        ki.w = hmul2_bits(k4.w, ex2a(-x[i][6]), ex2a(-x[i][7]));
+        const uint32_t so = (uint32_t)t * 128u + ((uint32_t)(cg ^ (t & 7)) << 4);
+        *reinterpret_cast<uint4 *>(qo + so) = qi;
+        *reinterpret_cast<uint4 *>(ko + so) = ki;
+        if constexpr (kHeld) *reinterpret_cast<uint4 *>(ro + so) = qi;
     }
 }
 
@@ -414,17 +468,43 @@ __device__ __noinline__ void exact_diag(const uint8_t *st, const uint8_t *meta, 
 // the diagonal blocks that need the exact evaluation, evaluates those into diagx[b], then
 // overlays Qd, Kd, A_J and B_J on the chunk's staging slot.
 template <bool kZ>
-__device__ __noinline__ void gate_slow(uint8_t *sm, const GRegs &R, const float2 (&ht)[4], int gw, int lane, int tt,
-                                       uint32_t bid, uint8_t *st, const uint8_t *meta, int nrows, uint8_t *qo,
-                                       uint8_t *ko, uint8_t *ro, bool held, int *bfl, int b, float inv_tau) {
+__device__ __noinline__ void gate_slow(uint8_t *sm, const float *htot, int gw, int lane, int tt, uint32_t bid,
+                                       uint8_t *st, const uint8_t *meta, int nrows, uint8_t *qo, uint8_t *ko,
+                                       uint8_t *ro, bool held, int *bfl, int b, float inv_tau) {
     const int t0 = 16 * gw, I = gw;
-    const uint4 sr = *reinterpret_cast<const uint4 *>(meta + t0);
+    // the team's block totals (kept in log2 units) in natural-log units, for the lane's
+    // channels 2 lane, 2 lane + 1
+    float2 ht[4];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        const float2 h = *reinterpret_cast<const float2 *>(htot + w * 64 + 2 * lane);
+        ht[w] = make_float2(h.x * kLn2, h.y * kLn2);
+    }
+    if (tt < 4) bfl[tt] = 0;   // (the readout of this buffer's previous chunk is complete)
+    named_sync(bid, kTeamThreads);
     __half2 qh[16], kh[16];
+    float2 gr[16];
 #pragma unroll
     for (int u = 0; u < 16; ++u) {
-        const uint32_t so = row_off(sr, u, lane);
-        qh[u] = ld_row_h2(st + L::st_q + so, t0 + u < nrows);
-        kh[u] = ld_row_h2(st + L::st_k + so, t0 + u < nrows);
+        const bool ok = t0 + u < nrows;
+        const uint32_t so = (uint32_t)meta[t0 + u] * 128u + 4u * (uint32_t)lane;
+        const uint32_t qb = *reinterpret_cast<const uint32_t *>(st + L::st_q + so);
+        const uint32_t kb = *reinterpret_cast<const uint32_t *>(st + L::st_k + so);
+        const uint32_t qz = ok ? qb : 0u, kz = ok ? kb : 0u;
+        qh[u] = *reinterpret_cast<const __half2 *>(&qz);
+        kh[u] = *reinterpret_cast<const __half2 *>(&kz);
+        const float2 gv = ld_gate2<kZ>(st + L::st_g + so, inv_tau);
+        gr[u] = ok ? gv : make_float2(0.f, 0.f);
+    }
+    GRegs R;   // inclusive prefix sums within the warp's block
+    {
+        float2 a = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            a.x += gr[u].x;
+            a.y += gr[u].y;
+            R.p[u] = a;
+        }
     }
     float2 pre = make_float2(0.f, 0.f), post = make_float2(0.f, 0.f);
 #pragma unroll
@@ -432,17 +512,14 @@ __device__ __noinline__ void gate_slow(uint8_t *sm, const GRegs &R, const float2
         if (J < I) { pre.x += ht[J].x; pre.y += ht[J].y; }
         if (J > I) { post.x += ht[J].x; post.y += ht[J].y; }
     }
-    float2 bs[16];   // within-block suffix sums (excluding the row), from the raw rows
+    float2 bs[16];   // within-block suffix sums (excluding the row)
     {
         float2 a = make_float2(0.f, 0.f);
 #pragma unroll
         for (int u = 15; u >= 0; --u) {
             bs[u] = a;
-            const float2 gv = ld_gate2<kZ>(st + L::st_g + meta[t0 + u] * 128 + 4 * lane, inv_tau);
-            if (t0 + u < nrows) {
-                a.x += gv.x;
-                a.y += gv.y;
-            }
+            a.x += gr[u].x;
+            a.y += gr[u].y;
         }
     }
     bool kbad = !(ht[I].x >= kDiagMinLogTotal) || !(ht[I].y >= kDiagMinLogTotal);
@@ -556,19 +633,42 @@ __device__ __forceinline__ float store_out_tile(const Params &P, const uint32_t 
 
 // Correction tile (fp32, fragment layout) added onto the stored fp16 outputs with
 // reductions (one addend per element: the result does not depend on their order).
-__device__ __forceinline__ void add_out_tile(const Params &P, const uint32_t (&r)[32], int q4, int lane,
-                                             const int *rows) {
+// Adds a 64x64 fp32 fragment tile (the correction term) to output rows this CTA has
+// already stored: a plain read-modify-write (no other CTA writes these rows, and the
+// CTA's barriers since the store make it visible), staged through `os` so that every
+// access is a 16-byte row piece; the correction is rounded to fp16 before the add.
+__device__ __forceinline__ void add_out_tile(const Params &P, const uint32_t (&r)[32], int q4, int lane, int tb,
+                                             uint8_t *os, const int *rows, uint32_t bid) {
     const int r0 = 16 * q4 + (lane >> 2), a2 = 2 * (lane & 3);
 #pragma unroll
     for (int e = 0; e < 32; e += 2) {
         const int h = e >> 4, j = (e >> 2) & 3, hh = (e >> 1) & 1;
-        const int ro = rows[r0 + 8 * hh];
-        if (ro < 0) continue;
-        const __half2 v = h2(__uint_as_float(r[e]), __uint_as_float(r[e + 1]));
-        __half *dst = P.out + (size_t)ro * kDV + 32 * h + 8 * j + a2;
-        asm volatile("red.global.add.noftz.f16x2 [%0], %1;" ::"l"(dst), "r"(*reinterpret_cast<const uint32_t *>(&v))
-                     : "memory");
+        sth2(os + sw_off(r0 + 8 * hh, 32 * h + 8 * j + a2), h2(__uint_as_float(r[e]), __uint_as_float(r[e + 1])));
     }
+    named_sync(bid, 128);
+    uint4 cur[4], add[4];
+    int ro[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {   // the loads first, so that their latencies overlap
+        const int x = tb + 128 * i, row = x >> 3, c8 = x & 7;
+        ro[i] = rows[row];
+        const int rr = ro[i] >= 0 ? ro[i] : 0;
+        cur[i] = *reinterpret_cast<const uint4 *>(P.out + (size_t)rr * kDV + 8 * c8);
+        add[i] = *reinterpret_cast<const uint4 *>(os + sw_off(row, 8 * c8));
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int x = tb + 128 * i, c8 = x & 7;
+        if (ro[i] >= 0) {
+            uint4 v;
+            v.x = hadd2_bits(cur[i].x, add[i].x);
+            v.y = hadd2_bits(cur[i].y, add[i].y);
+            v.z = hadd2_bits(cur[i].z, add[i].z);
+            v.w = hadd2_bits(cur[i].w, add[i].w);
+            *reinterpret_cast<uint4 *>(P.out + (size_t)ro[i] * kDV + 8 * c8) = v;
+        }
+    }
+    named_sync(bid, 128);
 }
 
 __device__ __forceinline__ void fill_rowtab(const Params &P, int seq, int cabs, int *rows, int t) {
@@ -730,9 +830,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_pipe_kernel(const __grid_
         tmem_relinquish();
     }
     if (tid == 0) {
-        for (int i = 0; i < kNStage; ++i) {
-            mbar_init(bar(sm, B_FULL + i), 1);
-        }
+        for (int i = 0; i < 2 * kNStage; ++i) mbar_init(bar(sm, B_FULL + i), 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(bar(sm, B_OPFULL + i), 1);
             mbar_init(bar(sm, B_MMA1 + i), 1);
@@ -1086,23 +1184,102 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_pipe_kernel(const __grid_
             const int tt = tid - (kWarpG + 4 * team) * 32, t0 = 16 * gw;
             const uint32_t bid = bar_team(team);
             float *htot = reinterpret_cast<float *>(sm + L::htot) + team * 4 * 64;
+            // lane layout: row slot rs = lane / 8 (rows tb .. tb+3 of the warp's 16),
+            // channel group cg = lane % 8 (channels 8 cg .. 8 cg + 7: one 16-byte unit)
+            const int cg = lane & 7, rs = lane >> 3, tb = t0 + 4 * rs;
             for (int c = (int)(((uint32_t)team - gc0) & 1u); c < nch; c += 2) {
                 const uint32_t gc = gc0 + c, b = gc & 1u, s = gc % kNStage, ph = (gc >> 1) & 1u;
                 const bool held = c < nring;
-                // operand buffers b free.  Waited first: MMA 2 of chunk gc-2 completes only
-                // after the other team has gated chunk gc-3 (the slot's previous use), so the
-                // slot's barrier can no longer be a phase short when its parity is tested
-                if (gc >= 2) wait_l(bar(sm, B_MMA2 + b), ph ^ 1u, to);
-                wait_l(bar(sm, B_FULL + s), (gc / kNStage) & 1u, to);
+                wait_l(bar(sm, full_bar(gc)), full_parity(gc), to);
                 uint8_t *st = sm + L::stage + s * L::stage_bytes;
                 const uint8_t *meta = sm + L::meta + s * 128;
                 const int nrows = *reinterpret_cast<const int *>(meta + 64);
-                unsigned *wm = reinterpret_cast<unsigned *>(sm + L::wmax) + 16 * b;
-                int *bfl = reinterpret_cast<int *>(sm + L::bflag) + 4 * b;
-                if (tt < 4) bfl[tt] = 0;
-                // ---------- pass 1: raw rows -> registers, prefix sums, maxima, V copy
-                // V rows into the scan-ordered operand tile first (row tt/2, 16-byte pieces
-                // 4 (tt%2) .. +3), so that their registers are free before the gating rows load
+                unsigned *wm = reinterpret_cast<unsigned *>(sm + L::wmax) + 16 * team;
+                // ---------- pass 1: prefix sums of the log-decay (log2 units) over the
+                // lane's rows, then over the warp's row slots; maxima of |q| and |k|
+                const uint32_t rw = *reinterpret_cast<const uint32_t *>(meta + tb);   // staging rows
+                float x[4][8];
+                {
+                    float acc[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+                    uint32_t qm = 0u, km = 0u;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const uint32_t o = ((rw >> (8 * i)) & 0xffu) * 128u + 16u * (uint32_t)cg;
+                        const bool ok = tb + i < nrows;   // rows past the grid count as zero
+                        float gv[8];
+                        ld_gate8<kZ>(st + L::st_g + o, gv, A.inv_tau);
+                        const uint32_t qa = absmax8(*reinterpret_cast<const uint4 *>(st + L::st_q + o));
+                        const uint32_t ka = absmax8(*reinterpret_cast<const uint4 *>(st + L::st_k + o));
+                        qm = ok ? umax16x2(qm, qa) : qm;
+                        km = ok ? umax16x2(km, ka) : km;
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            acc[j] = ok ? fmaf(gv[j], kLog2e, acc[j]) : acc[j];
+                            x[i][j] = acc[j];
+                        }
+                    }
+                    float tot[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {   // inclusive scan over the row slots
+                        float v = acc[j];
+                        float y = __shfl_up_sync(0xffffffffu, v, 8);
+                        v += rs >= 1 ? y : 0.f;
+                        y = __shfl_up_sync(0xffffffffu, v, 16);
+                        v += rs >= 2 ? y : 0.f;
+                        tot[j] = v;
+                        const float ex = v - acc[j];   // the warp's rows before the lane's
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) x[i][j] += ex;
+                    }
+                    if (rs == 3) {   // the warp's block totals
+                        float4 *hp = reinterpret_cast<float4 *>(htot + gw * 64 + 8 * cg);
+                        hp[0] = make_float4(tot[0], tot[1], tot[2], tot[3]);
+                        hp[1] = make_float4(tot[4], tot[5], tot[6], tot[7]);
+                    }
+                    const unsigned wq = __reduce_max_sync(0xffffffffu, max(qm & 0xffffu, qm >> 16));
+                    const unsigned wk = __reduce_max_sync(0xffffffffu, max(km & 0xffffu, km >> 16));
+                    if (lane == 0) {
+                        wm[gw] = wq;
+                        wm[4 + gw] = wk;
+                    }
+                }
+                named_sync(bid, kTeamThreads);
+                // ---------- pass 2
+                float bC[8];
+                {
+                    float off[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) off[j] = bC[j] = 0.f;
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {
+                        const float4 *hp = reinterpret_cast<const float4 *>(htot + w * 64 + 8 * cg);
+                        const float4 h0 = hp[0], h1 = hp[1];
+                        const float hv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            bC[j] += hv[j];
+                            off[j] += w < gw ? hv[j] : 0.f;
+                        }
+                    }
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) x[i][j] += off[j];
+                }
+                const uint4 wq4 = *reinterpret_cast<const uint4 *>(wm), wk4 = *reinterpret_cast<const uint4 *>(wm + 4);
+                const float qmx = half_bits_to_float(max(max(wq4.x, wq4.y), max(wq4.z, wq4.w)));
+                const float kmx = half_bits_to_float(max(max(wk4.x, wk4.y), max(wk4.z, wk4.w)));
+                bool bad = !(kmx <= kFastMaxK);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) bad |= !(bC[j] >= kFastMinLogDecay * kLog2e);
+                // every warp's lanes cover all 64 channels: a warp vote is the chunk's decision
+                const bool slow = __any_sync(0xffffffffu, bad);
+                // operand buffers b free (MMA 2 of chunk gc-2 complete)
+                if (gc >= 2) wait_l(bar(sm, B_MMA2 + b), ph ^ 1u, to);
+                // V rows into the scan-ordered operand tile (row tt/2, 16-byte units
+                // 4 (tt%2) .. +3)
                 {
                     const int t = tt >> 1, pc = 4 * (tt & 1);
                     const int r = meta[t];
@@ -1116,82 +1293,24 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_pipe_kernel(const __grid_
                         *reinterpret_cast<uint4 *>(vo + sw_off(t, 8 * (pc + i))) =
                             t < nrows ? v[i] : make_uint4(0u, 0u, 0u, 0u);
                 }
-                GRegs R;
-                const uint4 sr = *reinterpret_cast<const uint4 *>(meta + t0);
-                {
-                    __half2 qm = __float2half2_rn(0.f), km = qm;
-                    float2 acc = make_float2(0.f, 0.f);
-#pragma unroll
-                    for (int u = 0; u < 16; ++u) {
-                        // every table entry names a row of the slot, so the loads are always
-                        // in bounds; rows past the grid are zeroed by select (no branch in
-                        // the unrolled loop)
-                        const uint32_t w4 = u < 4 ? sr.x : u < 8 ? sr.y : u < 12 ? sr.z : sr.w;
-                        const int r = (w4 >> (8 * (u & 3))) & 0xff;
-                        const uint32_t o = r * 128 + 4 * lane;
-                        const bool ok = t0 + u < nrows;
-                        const float2 gv = ld_gate2<kZ>(st + L::st_g + o, A.inv_tau);
-                        const uint32_t qb = *reinterpret_cast<const uint32_t *>(st + L::st_q + o);
-                        const uint32_t kb = *reinterpret_cast<const uint32_t *>(st + L::st_k + o);
-                        const uint32_t qz = ok ? qb : 0u, kz = ok ? kb : 0u;
-                        acc.x += ok ? gv.x : 0.f;
-                        acc.y += ok ? gv.y : 0.f;
-                        R.p[u] = acc;
-                        qm = __hmax2(qm, __habs2(*reinterpret_cast<const __half2 *>(&qz)));
-                        km = __hmax2(km, __habs2(*reinterpret_cast<const __half2 *>(&kz)));
-                    }
-                    *reinterpret_cast<float2 *>(htot + gw * 64 + 2 * lane) = acc;
-                    const unsigned wq = __reduce_max_sync(0xffffffffu, __float_as_uint(fmaxf(__low2float(qm), __high2float(qm))));
-                    const unsigned wk = __reduce_max_sync(0xffffffffu, __float_as_uint(fmaxf(__low2float(km), __high2float(km))));
-                    if (lane == 0) {
-                        wm[gw] = wq;
-                        wm[4 + gw] = wk;
-                    }
-                }
-                named_sync(bid, kTeamThreads);
-                // ---------- pass 2
-                float2 ht[4];
-#pragma unroll
-                for (int w = 0; w < 4; ++w) ht[w] = *reinterpret_cast<const float2 *>(htot + w * 64 + 2 * lane);
-                float2 off = make_float2(0.f, 0.f), bC = make_float2(0.f, 0.f);
-#pragma unroll
-                for (int w = 0; w < 4; ++w) {
-                    if (w < gw) {
-                        off.x += ht[w].x;
-                        off.y += ht[w].y;
-                    }
-                    bC.x += ht[w].x;
-                    bC.y += ht[w].y;
-                }
-                const uint4 wq4 = *reinterpret_cast<const uint4 *>(wm), wk4 = *reinterpret_cast<const uint4 *>(wm + 4);
-                const unsigned qmx = max(max(wq4.x, wq4.y), max(wq4.z, wq4.w));
-                const unsigned kmx = max(max(wk4.x, wk4.y), max(wk4.z, wk4.w));
-                const bool bad = !(bC.x >= kFastMinLogDecay) || !(bC.y >= kFastMinLogDecay) ||
-                                 __uint_as_float(kmx) > kFastMaxK;
-                // every warp's lanes cover all 64 channels: a warp vote is the chunk's decision
-                const bool slow = __any_sync(0xffffffffu, bad);
                 uint8_t *qo = sm + L::qint + b * kTile;
                 uint8_t *ko = sm + L::kt + b * kTile;
                 uint8_t *ro = sm + L::ring + (held ? c : 0) * kTile;
+                int *bfl = reinterpret_cast<int *>(sm + L::bflag) + 4 * b;
                 if (!slow) {
                     if (held)
-                        gate_fast<true>(R, off, st, sr, nrows, qo, ko, ro, t0, lane);
+                        gate_fast<true>(x, st, rw, tb, nrows, cg, qo, ko, ro);
                     else
-                        gate_fast<false>(R, off, st, sr, nrows, qo, ko, ro, t0, lane);
+                        gate_fast<false>(x, st, rw, tb, nrows, cg, qo, ko, ro);
                 } else {
-                    // copies for the out-of-line call: R and ht themselves never have their
-                    // address taken, so that the fast path keeps them in registers
-                    GRegs Rs = R;
-                    float2 hts[4];
-#pragma unroll
-                    for (int w = 0; w < 4; ++w) hts[w] = ht[w];
-                    gate_slow<kZ>(sm, Rs, hts, gw, lane, tt, bid, st, meta, nrows, qo, ko, ro, held, bfl, b, A.inv_tau);
+                    gate_slow<kZ>(sm, htot, gw, lane, tt, bid, st, meta, nrows, qo, ko, ro, held, bfl, b, A.inv_tau);
                 }
                 // the chunk's decay (the state group keeps the products from the span start)
-                if (gw == 0) {
-                    const float2 d = make_float2(ex2a(bC.x * kLog2e), ex2a(bC.y * kLog2e));
-                    *reinterpret_cast<float2 *>(sm + L::dloc + b * 256 + 8 * lane) = d;
-                    if (lane == 0 && c < kMaxSpan) cmeta[2 * c] = __uint_as_float(qmx);
+                if (gw == 0 && rs == 0) {
+                    float4 *dp = reinterpret_cast<float4 *>(sm + L::dloc + b * 256 + 32 * cg);
+                    dp[0] = make_float4(ex2a(bC[0]), ex2a(bC[1]), ex2a(bC[2]), ex2a(bC[3]));
+                    dp[1] = make_float4(ex2a(bC[4]), ex2a(bC[5]), ex2a(bC[6]), ex2a(bC[7]));
+                    if (lane == 0 && c < kMaxSpan) cmeta[2 * c] = qmx;
                 }
                 fence_proxy_async_cta();
                 named_sync(bid, kTeamThreads);
@@ -1203,7 +1322,22 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_pipe_kernel(const __grid_
                 // sub-block path MMA 1 reads operands overlaid on the slot: after it completes)
                 if (gw == 0 && c + kNStage < nch) {
                     if (slow) wait_l(bar(sm, B_MMA1 + b), ph, to);
-                    load_chunk(A, sm, sbase, s, seq, c0 + c + kNStage, lane);
+                    load_chunk(A, sm, sbase, gc + kNStage, seq, c0 + c + kNStage, lane);
+                }
+            }
+            if (later) {
+                // while the state group looks back: the q and g rows of the chunks past
+                // the ring (the ones the corrections may rebuild) into L2
+                const int bb = seq / P.heads, hh = seq - bb * P.heads;
+                const int gt = tid - kWarpG * 32;
+                const int npf = min(nch, kRing + kPrefetchChunks) - kRing;
+                for (int i = gt; i < npf * 2 * kChunk; i += kGThreads) {
+                    const int ci = kRing + i / (2 * kChunk), t = (i >> 1) & (kChunk - 1);
+                    const int p = (c0 + ci) * kChunk + t;
+                    if (p < P.N) {
+                        const size_t rowi = ((size_t)bb * P.N + scan_to_token(p, P.H, P.W, P.dir)) * P.heads + hh;
+                        prefetch_l2((i & 1) ? (const void *)(P.q + rowi * kDK) : (const void *)(P.g + rowi * kDK));
+                    }
                 }
             }
         }
@@ -1267,19 +1401,24 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_pipe_kernel(const __grid_
                         __half2 qv[8];
                         float2 pg[8];
                         float2 acc = make_float2(0.f, 0.f);
+                        // all sixteen loads first (rows past the grid read the sequence's first
+                        // token and are zeroed after), so that their latencies overlap
+                        float2 gl[8];
 #pragma unroll
                         for (int u = 0; u < 8; ++u) {
                             const int p = cabs * kChunk + t0 + u;
-                            float2 gv = make_float2(0.f, 0.f);
-                            qv[u] = __float2half2_rn(0.f);
-                            if (p < P.N) {
-                                const size_t rowi = ((size_t)bb * P.N + scan_to_token(p, P.H, P.W, P.dir)) * P.heads + hh;
-                                gv = ld_gate2<kZ>(reinterpret_cast<const uint8_t *>(P.g + rowi * kDK + 2 * lane), A.inv_tau);
-                                qv[u] = *reinterpret_cast<const __half2 *>(P.q + rowi * kDK + 2 * lane);
-                            }
-                            acc.x += gv.x;
-                            acc.y += gv.y;
+                            const int pc = p < P.N ? p : 0;
+                            const size_t rowi = ((size_t)bb * P.N + scan_to_token(pc, P.H, P.W, P.dir)) * P.heads + hh;
+                            gl[u] = ld_gate2<kZ>(reinterpret_cast<const uint8_t *>(P.g + rowi * kDK + 2 * lane), A.inv_tau);
+                            qv[u] = *reinterpret_cast<const __half2 *>(P.q + rowi * kDK + 2 * lane);
+                        }
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            const bool ok = cabs * kChunk + t0 + u < P.N;
+                            acc.x += ok ? gl[u].x : 0.f;
+                            acc.y += ok ? gl[u].y : 0.f;
                             pg[u] = acc;
+                            if (!ok) qv[u] = __float2half2_rn(0.f);
                         }
                         *reinterpret_cast<float2 *>(htot + gw * 64 + 2 * lane) = acc;
                         named_sync(kBarGAll, kGThreads);
@@ -1333,8 +1472,10 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_pipe_kernel(const __grid_
                         uint32_t o[32];
                         ld_acc64(tmem + ((uint32_t)(32 * q4) << 16) + 64 * li, o);
                         tmem_ld_wait();
-                        add_out_tile(P, o, q4, lane, rows);
-                        named_sync(team ? kBarT1 : kBarT0, 128);
+                        // staging: the output tile for team 0, the first ring tile (free once the
+                        // batch's products are complete) for team 1
+                        add_out_tile(P, o, q4, lane, tb, sm + (team ? L::ring : L::ostg), rows,
+                                     team ? kBarT1 : kBarT0);
                     }
                 }
                 tc_fence_before();

@@ -126,6 +126,7 @@ struct Params {
     float *sf;
     int B, heads, H, W, N, dir;
     int n_seq, n_chunks;
+    int dk;   // key channels (the state has dk rows)
 };
 
 __device__ __forceinline__ void set_error(unsigned e) { atomicOr(&g_error_word, e); }
@@ -731,15 +732,13 @@ __global__ void __launch_bounds__(kThreads, Smem<DK>::min_blocks) gla_fwd_kernel
 
 }  // namespace gtr
 
-#include "gla_fwd_ws.cuh"
 #include "gla_fwd_span.cuh"
 #include "gla_fwd_pipe.cuh"
 
 namespace gtr {
 
 // ------------------------------------------------------------------ host
-enum KernelKind { kBasic64 = 0, kBasic128 = 1, kCluster = 2, kSpan = 3, kSpanShort = 4, kPipe = 5, kPipeZ = 6,
-                  kKinds = 7 };
+enum KernelKind { kBasic128 = 0, kSpan = 1, kSpanShort = 2, kPipe = 3, kPipeZ = 4, kKinds = 5 };
 
 // the span kernel with two loader warps (kSpan) or four (kSpanShort: short spans)
 static bool is_span(int kind) { return kind == kSpan || kind == kSpanShort; }
@@ -768,12 +767,8 @@ struct Plan {
 // (tuning knob) selects one of the other dk = 64 kernels instead.
 static KSpec spec_of(int kind) {
     switch (kind) {
-    case kBasic64:
-        return KSpec{reinterpret_cast<const void *>(&gla_fwd_kernel<64>), kThreads, Smem<64>::alloc, kBasic64};
     case kBasic128:
         return KSpec{reinterpret_cast<const void *>(&gla_fwd_kernel<128>), kThreads, Smem<128>::alloc, kBasic128};
-    case kCluster:
-        return KSpec{reinterpret_cast<const void *>(&ws::gla_fwd_ws_kernel), ws::kThreads, ws::L::alloc, kCluster};
     case kSpanShort:
         return KSpec{reinterpret_cast<const void *>(&sp::gla_fwd_span_kernel<4>), sp::span_threads<4>(),
                      sp::L::alloc, kSpanShort};
@@ -788,11 +783,9 @@ static KSpec spec_of(int kind) {
 }
 
 static int kind_for(int dk, long n_chunks) {
+    (void)n_chunks;
     if (dk != 64) return kBasic128;
-    if (n_chunks == 0) return kBasic64;   // only copies init_state to final_state
     const char *e = getenv("GTR_KERNEL");
-    if (e && !strcmp(e, "basic")) return kBasic64;
-    if (e && !strcmp(e, "cluster") && n_chunks >= ws::kMinCluster) return kCluster;
     if (e && !strcmp(e, "pipe")) return kPipe;
     return kSpan;
 }
@@ -958,7 +951,7 @@ static Plan span_plan(long n_seq, long n_chunks, int cap, int kind, size_t ws_li
 // sequence + 1), preferring the smaller cluster on ties.
 static Plan cluster_plan(int kind, long n_seq, long n_chunks, int dev, int sms, bool query) {
     const KSpec k = spec_of(kind);
-    const int cp_min = kind == kCluster ? ws::kMinCluster : 1;
+    const int cp_min = 1;
     Plan best{kind, cp_min, 1, 0, k.smem, k.threads, 0};
     const int fc = forced_cluster();
     long best_cost = -1;
@@ -990,10 +983,11 @@ static Plan make_plan(long n_seq, long n_chunks, int dk, bool query, size_t ws_l
     const int kind = gate_z ? kPipeZ : kind_for(dk, n_chunks);
     const int dev = current_device();
     const int sms = num_sms(dev);
+    if (n_chunks == 0) return Plan{kind, 1, 1, 0, 0, 0, 0};   // no launch: the state copy only
     if (kind == kSpan || is_pipe(kind)) {
         const int cap = span_capacity(dev, sms, query);
         if (cap > 0) return span_plan(n_seq, n_chunks, cap, kind, ws_limit);
-        return cluster_plan(kBasic64, n_seq, n_chunks, dev, sms, query);
+        return Plan{-1, 1, 1, 0, 0, 0, 0};   // no co-resident span plan on this device
     }
     return cluster_plan(kind, n_seq, n_chunks, dev, sms, query);
 }
@@ -1180,6 +1174,15 @@ static cudaError_t pipe_maps(const Params &prm, int dev, pp::Maps *maps, unsigne
 static cudaError_t launch(const Params &prm, const Plan &pl, void *workspace, cudaStream_t stream,
                           float inv_tau = 1.f) {
     const int dev = current_device();
+    if (prm.n_chunks == 0) {
+        // an empty grid: the final state is the initial one (zero without one), in the
+        // order of the caller's stream
+        if (prm.sf == nullptr) return cudaSuccess;
+        const size_t bytes = (size_t)prm.n_seq * prm.dk * kDV * sizeof(float);
+        return prm.s0 != nullptr ? cudaMemcpyAsync(prm.sf, prm.s0, bytes, cudaMemcpyDeviceToDevice, stream)
+                                 : cudaMemsetAsync(prm.sf, 0, bytes, stream);
+    }
+    if (pl.kind < 0) return cudaErrorNotSupported;
     const KSpec k = spec_of(pl.kind);
     cudaError_t e = prepare_kernel(k, is_coop(pl.kind) ? 1 : pl.cluster);
     if (e != cudaSuccess) return e;
@@ -1257,8 +1260,9 @@ static gtr_status_t check_args(const void *q, const void *k, const void *v, cons
 
 static Params make_params(const gtr_half_t *q, const gtr_half_t *k, const gtr_half_t *v,
                           const gtr_half_t *g, int B, int heads, int Hgrid, int Wgrid, int direction,
-                          const float *init_state, gtr_half_t *out, float *final_state) {
+                          const float *init_state, gtr_half_t *out, float *final_state, int dk) {
     Params prm{};
+    prm.dk = dk;
     prm.q = reinterpret_cast<const __half *>(q);
     prm.k = reinterpret_cast<const __half *>(k);
     prm.v = reinterpret_cast<const __half *>(v);
@@ -1293,7 +1297,7 @@ extern "C" gtr_status_t gtr_gla_fwd(const gtr_half_t *q, const gtr_half_t *k,
                                        chunk, init_state, out, final_state);
     if (st != GTR_OK) return st;
     const Params prm = make_params(q, k, v, g, B, heads, Hgrid, Wgrid, direction, init_state, out,
-                                   final_state);
+                                   final_state, dk);
     const Plan pl = make_plan(prm.n_seq, prm.n_chunks, dk, true);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     void *ws = nullptr;
@@ -1316,7 +1320,7 @@ extern "C" gtr_status_t gtr_gla_fwd_z(const gtr_half_t *q, const gtr_half_t *k, 
     if ((long long)Hgrid * Wgrid == 0)   // no token: the state copy of the plain call
         return gtr_gla_fwd(q, k, v, z, B, heads, Hgrid, Wgrid, dk, dv, direction, chunk, init_state, out,
                            final_state, stream);
-    const Params prm = make_params(q, k, v, z, B, heads, Hgrid, Wgrid, direction, init_state, out, final_state);
+    const Params prm = make_params(q, k, v, z, B, heads, Hgrid, Wgrid, direction, init_state, out, final_state, dk);
     const Plan pl = make_plan(prm.n_seq, prm.n_chunks, dk, true, ~size_t(0), true);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     void *ws = nullptr;
@@ -1377,7 +1381,7 @@ extern "C" gtr_status_t gtr_gla_fwd_stack(const gtr_gla_layer_t *layers, int n_l
         for (int i = 0; i < n_layers; ++i) {
             const gtr_gla_layer_t &L = layers[i];
             const Params prm = make_params(L.q, L.k, L.v, L.g, B, heads, Hgrid, Wgrid, L.direction, L.init_state,
-                                           L.out, L.final_state);
+                                           L.out, L.final_state, dk);
             const cudaError_t e = launch(prm, pl, ws, s);
             if (e != cudaSuccess) return e;
         }
@@ -1470,7 +1474,7 @@ extern "C" gtr_status_t gtr_gla_fwd_ws(const gtr_half_t *q, const gtr_half_t *k,
                                        chunk, init_state, out, final_state);
     if (st != GTR_OK) return st;
     const Params prm = make_params(q, k, v, g, B, heads, Hgrid, Wgrid, direction, init_state, out,
-                                   final_state);
+                                   final_state, dk);
     const Plan pl = make_plan(prm.n_seq, prm.n_chunks, dk, true);
     if (pl.ws_bytes > 0 &&
         (workspace == nullptr || workspace_bytes < pl.ws_bytes ||
@@ -1520,7 +1524,7 @@ extern "C" gtr_status_t gtr_gla_fwd_static(const gtr_half_t *q, const gtr_half_t
                                        chunk, init_state, out, final_state);
     if (st != GTR_OK) return st;
     const Params prm = make_params(q, k, v, g, B, heads, Hgrid, Wgrid, direction, init_state, out,
-                                   final_state);
+                                   final_state, dk);
     // the cheapest plan whose workspace fits the scratch (one span per sequence needs none)
     const Plan pl = make_plan(prm.n_seq, prm.n_chunks, dk, true, kStaticWsBytes);
     if (pl.ws_bytes > kStaticWsBytes) return GTR_ERR_UNSUPPORTED;

@@ -1,0 +1,26 @@
+"""The TMA-staged warp-specialised kernel (gla_fwd_pipe) vs the fp64 oracle (GPU only).
+
+The library selects it for the gate-from-z entry point and, with GTR_KERNEL=pipe, for
+gtr_gla_fwd at dk = 64.  The parity, span and range tests of the default path run here
+again with that selection: every workload and direction, the edge shapes, degenerate
+gates, forced span counts (look-back and corrections), in-place carry, split and
+resume, and the large-key sub-block path.  (dk = 128 shapes keep their own kernel.)
+"""
+import pytest
+
+from tests.test_gpu_parity import (test_degenerate_gates, test_edge_shapes,  # noqa: F401
+                                   test_empty_grid_copies_state, test_in_place_state_carry,
+                                   test_large_sample_rows_match_oracle_subset,
+                                   test_split_sequence_resume, test_workload_parity)
+from tests.test_gpu_span import (test_forced_span_counts, test_in_place_carry_with_spans,  # noqa: F401
+                                 test_long_spans_reread, test_ragged_last_span,
+                                 test_span_groups_loop_over_sequences)
+from tests.test_gpu_graph_range import (test_large_keys_take_the_sub_block_path_and_match,  # noqa: F401
+                                        test_large_keys_with_spans_match, test_state_inside_fp16_is_exact)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _pipe_kernel(monkeypatch):
+    monkeypatch.setenv("GTR_KERNEL", "pipe")

@@ -188,17 +188,3 @@ def test_workspace_argument_checks():
     assert gla.workspace_bytes(big.B, big.heads, big.H, big.W, big.dk, big.dv) == 0
     assert gla.workspace_bytes(1, 1, 4, 4, 64, 64, chunk=32) == 0
     assert gla.device_status() == gla.GTR_OK
-
-
-@pytest.mark.parametrize("kernel", ["basic", "cluster"])
-def test_other_dk64_kernels(monkeypatch, kernel):
-    """The basic (one CTA per sequence slice) and thread-block-cluster kernels stay
-    selectable and correct."""
-    monkeypatch.setenv("GTR_KERNEL", kernel)
-    w = WORKLOADS["gtr640_b1h16_40x40"]
-    for d in (0, 2):
-        inp = workload_inputs(w, d, 0)
-        out, sf = run_gpu(inp, w.H, w.W, d)
-        ro, rs = run_oracle(inp, w.H, w.W, d)
-        assert_parity(out, ro, f"{kernel} dir {d} out")
-        assert_parity(sf, rs, f"{kernel} dir {d} state")
