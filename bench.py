@@ -37,7 +37,7 @@ sys.path.insert(0, ROOT)
 import torch  # noqa: E402
 import torch.distributed as dist  # noqa: E402
 
-from recurrent_vision_backbone_b200.inputs import DIR_NAMES, WORKLOADS, make_inputs  # noqa: E402
+from recurrent_vision_backbone_b200.inputs import DIR_NAMES, TAU, WORKLOADS, make_inputs  # noqa: E402
 
 METRIC = "GLA fwd tokens/s at 1.6K & 16.4K tokens (FP16, C=64); % of roofline"
 PRIMARY = "gtr640_b1h16_40x40"
@@ -115,17 +115,23 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:12]
 
 
-def kernel_for(w) -> str:
-    """The kernel a call of workload w launches (one launch per call)."""
-    if w.dk != 64:
-        return "gla_fwd_kernel"
+def kernel_for(w, gate_z=False) -> str:
+    """The kernel a call of workload w launches."""
+    if w.dk != 64 or gate_z:
+        return "gla_fwd_pipe_kernel"
     return "gla_fwd_pipe_kernel" if os.environ.get("GTR_KERNEL") == "pipe" else "gla_fwd_span_kernel"
+
+
+def launches_per_call(w) -> int:
+    """dk = 128 runs as two launches over the two 64-channel key halves."""
+    return 2 if w.dk == 128 else 1
 
 
 def recorded_traffic(workload_name: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on the
-    current kernel source; else None."""
-    kernel = kernel_for(WORKLOADS[workload_name])
+    current kernel source; else None.  (A name ending in "+z": the gate-from-z entry.)"""
+    gate_z = workload_name.endswith("+z")
+    kernel = kernel_for(WORKLOADS[workload_name[:-2] if gate_z else workload_name], gate_z)
     path = os.path.join(ROOT, "profiles", f"{kernel}_{workload_name}.md")
     try:
         text = open(path).read()
@@ -228,10 +234,11 @@ class Workload:
     """Rotating device-resident input sets for one workload and the graph that
     replays `group` steps of 4 direction calls over them."""
 
-    def __init__(self, w, rank, device, n_sets=None):
+    def __init__(self, w, rank, device, n_sets=None, gate_z=False):
         from recurrent_vision_backbone_b200 import gla
         self.gla = gla
         self.w = w
+        self.gate_z = gate_z   # gtr_gla_fwd_z: the gate's pre-activation z in place of g
         per_call = bytes_alg(w)
         if n_sets is None:
             n_sets = max(4, -(-4 * L2_BYTES // (per_call * len(w.call_directions()))))
@@ -243,7 +250,9 @@ class Workload:
                 inp = make_inputs(w.B, w.heads, w.H, w.W, w.dk, w.dv,
                                   seed=rank_seed(w.seed(d, 100 + 16 * s + c), rank),
                                   init_std=w.init_std, z_mean_per_head=w.z_mean_per_head,
-                                  device=device)
+                                  device=device, with_z=gate_z)
+                if gate_z:
+                    del inp["g"]
                 out = torch.empty((w.B, w.N, w.heads, w.dv), dtype=torch.float16, device=device)
                 sf = (torch.empty((w.B, w.heads, w.dk, w.dv), dtype=torch.float32, device=device)
                       if w.final_state else None)
@@ -253,8 +262,12 @@ class Workload:
 
     def launch_step(self, s, stream):
         for d, inp, out, sf in self.sets[s % self.n_sets]:
-            self.gla.gtr_gla_fwd(inp["q"], inp["k"], inp["v"], inp["g"], self.w.H, self.w.W, d,
-                                 init_state=inp["s0"], out=out, final_state=sf, stream=stream)
+            if self.gate_z:
+                self.gla.gtr_gla_fwd_z(inp["q"], inp["k"], inp["v"], inp["z"], TAU, self.w.H, self.w.W, d,
+                                       init_state=inp["s0"], out=out, final_state=sf, stream=stream)
+            else:
+                self.gla.gtr_gla_fwd(inp["q"], inp["k"], inp["v"], inp["g"], self.w.H, self.w.W, d,
+                                     init_state=inp["s0"], out=out, final_state=sf, stream=stream)
 
     def capture(self, stream, steps):
         """Graphs replaying the rotating sets: `graph` holds one step per set; a graph of
@@ -336,14 +349,15 @@ def measure(wl, steps, warmup, stream, world, clocks=None, clock_window_s=1.0):
     return ms, steps, clk
 
 
-def roofline(w, ms_per_launch, workload_name):
+def roofline(w, ms_per_call, workload_name, gate_z=False):
     peak, which = measured_peaks()
     b = bytes_alg(w)
-    achieved = b / (ms_per_launch * 1e-3) / 1e9
-    return {"kernel": kernel_for(w), "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+    achieved = b / (ms_per_call * 1e-3) / 1e9
+    return {"kernel": kernel_for(w, gate_z), "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
             "unit": "GB/s",
             "frac": round(achieved / peak, 4), "traffic": recorded_traffic(workload_name),
-            "peak_source": which, "bytes_alg_per_launch": b, "flops_alg_per_launch": flops_alg(w)}
+            "peak_source": which, "bytes_alg_per_call": b, "flops_alg_per_call": flops_alg(w),
+            "launches_per_call": launches_per_call(w)}
 
 
 def call_inputs(w, d, seed, heads=None, device="cpu"):
@@ -439,21 +453,24 @@ def config_of(w, world, l2_note, timing):
 
 
 def run_workload(name, steps, warmup, stream, world, rank, device, sets, sample_clocks, local,
-                 clocks_csv=None):
-    """Times `steps` steps of one workload; returns its numbers and its config."""
+                 clocks_csv=None, gate_z=False):
+    """Times `steps` steps of one workload; returns its numbers and its config.  gate_z:
+    through gtr_gla_fwd_z (the gate's pre-activation z read in place of g: the same
+    bytes, the gate formed while staging)."""
     w = WORKLOADS[name]
-    wl = Workload(w, rank, device, n_sets=sets)
+    wl = Workload(w, rank, device, n_sets=sets, gate_z=gate_z)
     clocks = None
     if sample_clocks:
         clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
                               else local, clocks_csv)
     ms, n_steps, clk = measure(wl, steps, warmup, stream, world, clocks)
-    launches = n_steps * wl.calls_per_step()
-    res = {"workload": name, "tokens_per_call": w.B * w.N,
+    calls = n_steps * wl.calls_per_step()
+    res = {"workload": name + ("+z" if gate_z else ""), "tokens_per_call": w.B * w.N,
            "value": round(world * wl.tokens_per_step() * n_steps / (ms * 1e-3), 1),
            "unit": "tokens/s", "steps": n_steps, "ms_per_step": round(ms / n_steps, 6),
-           "us_per_call": round(ms * 1e3 / launches, 3),
-           "roofline": roofline(w, ms / launches, name), "gpu_launches": launches,
+           "us_per_call": round(ms * 1e3 / calls, 3),
+           # a call's bytes over a call's time (a dk = 128 call: both launches)
+           "roofline": roofline(w, ms / calls, name + ("+z" if gate_z else ""), gate_z), "gpu_launches": calls * launches_per_call(w),
            "clocks": clk}
     l2 = (f"inputs rotate over {wl.n_sets} sets of {wl.calls_per_step()} calls "
           f"({wl.n_sets * wl.calls_per_step() * bytes_alg(w) / 2**20:.0f} MiB > 3x L2)")
@@ -465,7 +482,10 @@ def run_workload(name, steps, warmup, stream, world, rank, device, sets, sample_
     return res, cfg
 
 
-SECONDARIES = ("hires_b1h16_128x128", "b8h16_48x48_stack12", "stress_b4h12_37x53_dk128")
+# (workload, through the gate-from-z entry point)
+SECONDARIES = (("hires_b1h16_128x128", False), ("b8h16_48x48_stack12", False),
+               ("stress_b4h12_37x53_dk128", False), ("gtr640_b1h16_40x40", True),
+               ("hires_b1h16_128x128", True))
 
 
 def gpu_arm(args):
@@ -495,11 +515,11 @@ def gpu_arm(args):
     }
     if not args.no_secondary:
         line["secondary"] = []
-        for name in SECONDARIES:
-            if name == primary:
+        for name, gz in SECONDARIES:
+            if name == primary and not gz:
                 continue
             r2, _ = run_workload(name, max(8, args.steps // 16), max(3, args.warmup // 16), stream,
-                                 world, rank, device, args.sets, True, local)
+                                 world, rank, device, args.sets, True, local, gate_z=gz)
             line["secondary"].append(r2)
     # end to end through the public call with host buffers
     e_steps = max(3, min(args.steps, args.e2e_steps))

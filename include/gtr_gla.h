@@ -110,8 +110,7 @@ gtr_status_t gtr_gla_fwd(const gtr_half_t *q, const gtr_half_t *k, const gtr_hal
  * fp32 while it stages each chunk (GTR news article, section "线性注意力到底在省什么":
  * a learnable forget gate on the key side), so no separate pass over z runs and g is
  * never rounded to fp16.  Same arguments, layouts, workspace and errors as gtr_gla_fwd,
- * plus GTR_ERR_INVALID_ARG for tau <= 0 or not finite; dk must be 64 (else
- * GTR_ERR_UNSUPPORTED).
+ * plus GTR_ERR_INVALID_ARG for tau <= 0 or not finite.
  */
 gtr_status_t gtr_gla_fwd_z(const gtr_half_t *q, const gtr_half_t *k, const gtr_half_t *v,
                            const gtr_half_t *z, float tau, int B, int heads, int Hgrid, int Wgrid,

@@ -167,10 +167,6 @@ __device__ __forceinline__ float ex2a(float x) {
     return y;
 }
 __device__ __forceinline__ __half2 h2(float a, float b) { return __floats2half2_rn(a, b); }
-// A value about to become an fp16 operand or output must be finite and below 65504.
-__device__ __forceinline__ void range_check(float mx) {
-    if (!(mx <= kHalfMax)) set_error(kErrRange);
-}
 template <int N>
 __device__ __forceinline__ float max_abs(const float (&x)[N]) {
     float m = 0.f;
@@ -607,6 +603,11 @@ __device__ __forceinline__ void ld_off48(uint32_t taddr, uint32_t (&r)[32]) {
 
 // Output tile (fp32 in registers, fragment layout) -> fp16 -> staging -> coalesced rows.
 // Team of 4 warps (128 threads, named barrier `bid`); returns the thread's max |o|.
+// The chunk's output tile: fp16 through the staging tile `os`, then 16-byte row pieces
+// to the token rows (`rows`; -1: past the grid).  With P.acc (the second key-channel
+// half of a dk = 128 call) each piece is added to what the first half stored (a plain
+// read-modify-write: the launches are ordered on the stream).  Returns max |value|
+// written, for the range check (the sum, when adding).
 __device__ __forceinline__ float store_out_tile(const Params &P, const uint32_t (&r)[32], int q4, int lane, int tb,
                                                 uint8_t *os, const int *rows, uint32_t bid) {
     const int r0 = 16 * q4 + (lane >> 2), a2 = 2 * (lane & 3);
@@ -619,13 +620,44 @@ __device__ __forceinline__ float store_out_tile(const Params &P, const uint32_t 
         sth2(os + sw_off(r0 + 8 * hh, 32 * h + 8 * j + a2), h2(x0, x1));
     }
     named_sync(bid, 128);
+    if (!P.acc) {
 #pragma unroll
-    for (int x = tb; x < 64 * 8; x += 128) {
-        const int row = x >> 3, c8 = x & 7;
-        const int ro = rows[row];
-        if (ro >= 0)
-            *reinterpret_cast<uint4 *>(P.out + (size_t)ro * kDV + 8 * c8) =
-                *reinterpret_cast<const uint4 *>(os + sw_off(row, 8 * c8));
+        for (int x = tb; x < 64 * 8; x += 128) {
+            const int row = x >> 3, c8 = x & 7;
+            const int ro = rows[row];
+            if (ro >= 0)
+                *reinterpret_cast<uint4 *>(P.out + (size_t)ro * kDV + 8 * c8) =
+                    *reinterpret_cast<const uint4 *>(os + sw_off(row, 8 * c8));
+        }
+    } else {
+        uint4 cur[4];
+        int ro[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {   // the loads first, so that their latencies overlap
+            const int x = tb + 128 * i, row = x >> 3, c8 = x & 7;
+            ro[i] = rows[row];
+            cur[i] = *reinterpret_cast<const uint4 *>(P.out + (size_t)(ro[i] >= 0 ? ro[i] : 0) * kDV + 8 * c8);
+        }
+        __half2 m2 = __float2half2_rn(0.f);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int x = tb + 128 * i, row = x >> 3, c8 = x & 7;
+            const uint4 a = *reinterpret_cast<const uint4 *>(os + sw_off(row, 8 * c8));
+            uint4 v;
+            v.x = hadd2_bits(cur[i].x, a.x);
+            v.y = hadd2_bits(cur[i].y, a.y);
+            v.z = hadd2_bits(cur[i].z, a.z);
+            v.w = hadd2_bits(cur[i].w, a.w);
+            if (ro[i] >= 0) {
+                *reinterpret_cast<uint4 *>(P.out + (size_t)ro[i] * kDV + 8 * c8) = v;
+                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int m = 0; m < 4; ++m) m2 = __hmax2_nan(m2, __habs2(*reinterpret_cast<const __half2 *>(&w4[m])));
+            }
+        }
+        // the sum is what must stay inside fp16 (an overflow shows as inf, a NaN stays NaN)
+        const float ml = __low2float(m2), mh = __high2float(m2);
+        mx = (ml != ml || mh != mh) ? ml + mh : fmaxf(mx, fmaxf(ml, mh));
     }
     named_sync(bid, 128);
     return mx;
@@ -656,6 +688,7 @@ __device__ __forceinline__ void add_out_tile(const Params &P, const uint32_t (&r
         cur[i] = *reinterpret_cast<const uint4 *>(P.out + (size_t)rr * kDV + 8 * c8);
         add[i] = *reinterpret_cast<const uint4 *>(os + sw_off(row, 8 * c8));
     }
+    __half2 m2 = __float2half2_rn(0.f);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int x = tb + 128 * i, c8 = x & 7;
@@ -666,8 +699,13 @@ __device__ __forceinline__ void add_out_tile(const Params &P, const uint32_t (&r
             v.z = hadd2_bits(cur[i].z, add[i].z);
             v.w = hadd2_bits(cur[i].w, add[i].w);
             *reinterpret_cast<uint4 *>(P.out + (size_t)ro[i] * kDV + 8 * c8) = v;
+            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int m = 0; m < 4; ++m) m2 = __hmax2_nan(m2, __habs2(*reinterpret_cast<const __half2 *>(&w4[m])));
         }
     }
+    const float ml = __low2float(m2), mh = __high2float(m2);
+    range_check(ml != ml || mh != mh ? ml + mh : fmaxf(ml, mh));   // the corrected outputs
     named_sync(bid, 128);
 }
 
@@ -876,7 +914,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_pipe_kernel(const __grid_
             const int r0 = 16 * q4 + (lane >> 2);
             float S[32];
             {
-                const float *s0 = (!later && P.s0 != nullptr) ? P.s0 + (size_t)seq * kDK * kDV : nullptr;
+                const float *s0 = (!later && P.s0 != nullptr) ? P.s0 + (size_t)seq * P.sstride : nullptr;
 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
                     const int h = e >> 4, j = (e >> 2) & 3, hh = (e >> 1) & 1;
@@ -994,7 +1032,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_pipe_kernel(const __grid_
                     sp::st_release_gpu(A.flags + ((size_t)seq * PS + kspan) * kFlagStride, (unsigned)(PS - 1 - kspan));
             }
             if (PS == 1 && P.sf != nullptr) {
-                float *sf = P.sf + (size_t)seq * kDK * kDV;
+                float *sf = P.sf + (size_t)seq * P.sstride;
 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
                     const int h = e >> 4, j = (e >> 2) & 3, hh = (e >> 1) & 1;
@@ -1093,7 +1131,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_pipe_kernel(const __grid_
                 }
                 if (kspan == PS - 1 && P.sf != nullptr) {   // final state D_span * S_in + S_local
                     const float G0 = D0, G1 = D1;
-                    float *sf = P.sf + (size_t)seq * kDK * kDV;
+                    float *sf = P.sf + (size_t)seq * P.sstride;
 #pragma unroll
                     for (int e = 0; e < 32; e += 2) {
                         const int h = e >> 4, j = (e >> 2) & 3, hh = (e >> 1) & 1;
@@ -1336,7 +1374,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_pipe_kernel(const __grid_
                     const int p = (c0 + ci) * kChunk + t;
                     if (p < P.N) {
                         const size_t rowi = ((size_t)bb * P.N + scan_to_token(p, P.H, P.W, P.dir)) * P.heads + hh;
-                        prefetch_l2((i & 1) ? (const void *)(P.q + rowi * kDK) : (const void *)(P.g + rowi * kDK));
+                        prefetch_l2((i & 1) ? (const void *)(P.q + rowi * P.ldk) : (const void *)(P.g + rowi * P.ldk));
                     }
                 }
             }
@@ -1409,8 +1447,8 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_pipe_kernel(const __grid_
                             const int p = cabs * kChunk + t0 + u;
                             const int pc = p < P.N ? p : 0;
                             const size_t rowi = ((size_t)bb * P.N + scan_to_token(pc, P.H, P.W, P.dir)) * P.heads + hh;
-                            gl[u] = ld_gate2<kZ>(reinterpret_cast<const uint8_t *>(P.g + rowi * kDK + 2 * lane), A.inv_tau);
-                            qv[u] = *reinterpret_cast<const __half2 *>(P.q + rowi * kDK + 2 * lane);
+                            gl[u] = ld_gate2<kZ>(reinterpret_cast<const uint8_t *>(P.g + rowi * P.ldk + 2 * lane), A.inv_tau);
+                            qv[u] = *reinterpret_cast<const __half2 *>(P.q + rowi * P.ldk + 2 * lane);
                         }
 #pragma unroll
                         for (int u = 0; u < 8; ++u) {

@@ -179,12 +179,13 @@ __device__ __forceinline__ void load_chunk(const Params &P, uint8_t *sm, int seq
         const int t = 4 * (NL * i + lw) + sub;
         const int ro = rowtab[4 * i + sub];
         const uint32_t nb = ro >= 0 ? 16u : 0u;
-        const size_t off = (size_t)(ro >= 0 ? ro : 0) * 64 + 8 * pc;
+        const size_t rr = (size_t)(ro >= 0 ? ro : 0);
+        const size_t off = rr * P.ldk + 8 * pc;   // q, k, g rows (pitch: dk of the call)
         const uint32_t d = st + t * 128 + 16 * pc;
         cp_async16(d, P.q + off, nb);
         cp_async16(d + kTile, P.k + off, nb);
         cp_async16(d + 2 * kTile, P.g + off, nb);
-        cp_async16(vo + sw_off(t, 8 * pc), P.v + off, nb);
+        cp_async16(vo + sw_off(t, 8 * pc), P.v + rr * kDV + 8 * pc, nb);
     }
 }
 
@@ -214,7 +215,8 @@ __device__ __forceinline__ bool flag_wait_bounded(const unsigned *f, uint64_t li
 // consecutive warps (warp w reads TMEM lanes 32 (w % 4) ..; tb = thread in the team,
 // named barrier `bar_id`): adds `addend` rows from an unswizzled fp16 staging tile if
 // non-null, converts to fp16 through the staging tile `os`, stores at the token rows
-// in `rowb`; returns this thread's max |value|.
+// in `rowb` (with P.acc and no addend: adds to the rows stored there); returns this
+// thread's max |value|.
 __device__ __forceinline__ float store_chunk_out(const Params &P, uint32_t tmem, uint32_t col,
                                                  int bw, int lane, int tb, const uint8_t *addend,
                                                  uint32_t bar_id, uint8_t *os, const int *rowb) {
@@ -248,15 +250,49 @@ __device__ __forceinline__ float store_chunk_out(const Params &P, uint32_t tmem,
         }
     tc_fence_before();
     named_sync(bar_id, 128);
+    // (a correction passes the stored rows as `addend`: the sum is then stored as is)
+    if (!P.acc || addend != nullptr) {
 #pragma unroll
-    for (int x = tb; x < 64 * 8; x += 128) {
-        const int row = x >> 3, c8 = x & 7;
-        const int ro = rowb[row];
-        if (ro >= 0)
-            *reinterpret_cast<uint4 *>(P.out + (size_t)ro * kDV + 8 * c8) =
-                *reinterpret_cast<const uint4 *>(os + sw_off(row, 8 * c8));
+        for (int x = tb; x < 64 * 8; x += 128) {
+            const int row = x >> 3, c8 = x & 7;
+            const int ro = rowb[row];
+            if (ro >= 0)
+                *reinterpret_cast<uint4 *>(P.out + (size_t)ro * kDV + 8 * c8) =
+                    *reinterpret_cast<const uint4 *>(os + sw_off(row, 8 * c8));
+        }
+    } else {
+        // the second key-channel half of a dk = 128 call: add to what the first half
+        // stored (the launches are ordered on the stream); the sum is range-checked
+        uint4 cur[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {   // the loads first, so that their latencies overlap
+            const int x = tb + 128 * i, row = x >> 3, c8 = x & 7;
+            const int ro = rowb[row];
+            cur[i] = *reinterpret_cast<const uint4 *>(P.out + (size_t)(ro >= 0 ? ro : 0) * kDV + 8 * c8);
+        }
+        __half2 m2 = __float2half2_rn(0.f);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int x = tb + 128 * i, row = x >> 3, c8 = x & 7;
+            const int ro = rowb[row];
+            const uint4 a = *reinterpret_cast<const uint4 *>(os + sw_off(row, 8 * c8));
+            const uint32_t cw[4] = {cur[i].x, cur[i].y, cur[i].z, cur[i].w}, aw[4] = {a.x, a.y, a.z, a.w};
+            uint32_t vw[4];
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const __half2 v = __hadd2(*reinterpret_cast<const __half2 *>(&cw[m]),
+                                          *reinterpret_cast<const __half2 *>(&aw[m]));
+                vw[m] = *reinterpret_cast<const uint32_t *>(&v);
+                if (ro >= 0) m2 = __hmax2_nan(m2, __habs2(v));
+            }
+            if (ro >= 0)
+                *reinterpret_cast<uint4 *>(P.out + (size_t)ro * kDV + 8 * c8) = make_uint4(vw[0], vw[1], vw[2], vw[3]);
+        }
+        const float ml = __low2float(m2), mh = __high2float(m2);
+        mx = (ml != ml || mh != mh) ? ml + mh : fmaxf(mx, fmaxf(ml, mh));
     }
     named_sync(bar_id, 128);
+    range_check(mx);   // the fp16 outputs
     return mx;
 }
 
@@ -590,6 +626,7 @@ __device__ __forceinline__ void store_p_tmem(uint8_t *sm, uint32_t tmem, const B
     const float *diagx = reinterpret_cast<const float *>(sm + L::diag) + b * 1024;
     const int row0 = 16 * q + (lane >> 2), col0 = 2 * (lane & 3);
     uint32_t v[16];
+    float pmx = 0.f;
 #pragma unroll
     for (int half = 0; half < 2; ++half)
 #pragma unroll
@@ -607,8 +644,10 @@ __device__ __forceinline__ void store_p_tmem(uint8_t *sm, uint32_t tmem, const B
                 }
                 x0 = col <= row ? x0 : 0.f;
                 x1 = col + 1 <= row ? x1 : 0.f;
+                pmx = fmaxf(pmx, fmaxf(fabsf(x0), fabsf(x1)));
                 v[2 * (cc + 4 * half) + hh] = pack_half2(x0, x1);   // packed column 4 j + lane % 4
             }
+    range_check(pmx);
     asm volatile(
         "tcgen05.st.sync.aligned.16x128b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
             tmem + ((uint32_t)(32 * q) << 16) + kColScores),
@@ -640,6 +679,7 @@ __device__ __forceinline__ void update_state_a(uint8_t *sm, uint32_t tmem, int b
     const float *dloc = reinterpret_cast<const float *>(sm + L::dloc + b * 256);
     uint8_t *sst = sm + L::sst;
     float2 sv[2][4];
+    float smx = 0.f;
     if constexpr (kLoadFirst) {
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh)
@@ -662,10 +702,12 @@ __device__ __forceinline__ void update_state_a(uint8_t *sm, uint32_t tmem, int b
             const float2 sn = make_float2(fmaf(di, s.x, scl * __uint_as_float(rd[4 * cc + 2 * hh])),
                                           fmaf(di, s.y, scl * __uint_as_float(rd[4 * cc + 2 * hh + 1])));
             *sp2 = sn;
+            smx = fmaxf(smx, fmaxf(fabsf(sn.x), fabsf(sn.y)));
             if (so_next != nullptr) st_h2(so_next + sw_off(i, col), sn.x, sn.y);
             if (agg != nullptr) *reinterpret_cast<float2 *>(agg + i * kDV + col) = sn;
         }
     }
+    if (so_next != nullptr) range_check(smx);   // the fp16 S_prev operand
     tc_fence_before();
     fence_proxy_async_cta();
     named_sync(kBarA, kThreadsA);
@@ -693,7 +735,7 @@ __device__ __forceinline__ void loader_load(const Params &P, uint8_t *sm, int se
 // register pressure of the kernel body.)
 __device__ __noinline__ void load_qgo(const __half *q, const __half *g, const __half *o, int N, int H,
                                       int W, int dir, int heads, int seq, int c, uint32_t dst_q,
-                                      uint32_t dst_g, uint32_t dst_o, int nthreads) {
+                                      uint32_t dst_g, uint32_t dst_o, int nthreads, int ldk) {
     const int bq = seq / heads, hq = seq - bq * heads;
     const int p0 = c * kChunk;
     for (int x = (int)threadIdx.x; x < 3 * 64 * 8; x += nthreads) {
@@ -701,7 +743,7 @@ __device__ __noinline__ void load_qgo(const __half *q, const __half *g, const __
         const bool ok = p0 + t < N;
         size_t ro = 0;
         if (ok) ro = (size_t)((bq * N + scan_to_token(p0 + t, H, W, dir)) * heads + hq);
-        const __half *src = ten == 0 ? q + ro * 64 : (ten == 1 ? g + ro * 64 : o + ro * 64);
+        const __half *src = ten == 0 ? q + ro * ldk : (ten == 1 ? g + ro * ldk : o + ro * 64);
         const uint32_t d = ten == 0 ? dst_q : (ten == 1 ? dst_g : dst_o);
         cp_async16(d + t * 128 + 16 * pc, src + 8 * pc, ok ? 16u : 0u);
     }
@@ -814,9 +856,9 @@ __device__ __forceinline__ void prefetch_span_rows(const Params &P, const Work &
     if (p >= P.N) return;
     const int bb = seq / P.heads, hh = seq - bb * P.heads;
     const size_t ro = ((size_t)bb * P.N + scan_to_token(p, P.H, P.W, P.dir)) * P.heads + hh;
-    prefetch_l2(P.q + ro * kDK);
-    prefetch_l2(P.k + ro * kDK);
-    prefetch_l2(P.g + ro * kDK);
+    prefetch_l2(P.q + ro * P.ldk);
+    prefetch_l2(P.k + ro * P.ldk);
+    prefetch_l2(P.g + ro * P.ldk);
     prefetch_l2(P.v + ro * kDV);
 }
 
@@ -904,11 +946,12 @@ __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(con
                 const int i = e >> 4, c4 = e & 15;
                 float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (!later && P.s0 != nullptr)
-                    v = reinterpret_cast<const float4 *>(P.s0 + (size_t)seq * kDK * kDV)[e];
+                    v = reinterpret_cast<const float4 *>(P.s0 + (size_t)seq * P.sstride)[e];
                 *reinterpret_cast<float4 *>(sst + agg_off(i, c4)) = v;
                 // S_prev of chunk 0, the fp16 operand of its MMA 2
                 *reinterpret_cast<uint2 *>(sm + L::sop + sw_off(i, 4 * c4)) =
                     make_uint2(pack_half2(v.x, v.y), pack_half2(v.z, v.w));
+                range_check(absmax4(v));
             }
             if (tid < 64) dcum[tid] = 1.f;
             if (tid < kMaxSpan * 2) cmeta[tid] = 0.f;
@@ -1126,6 +1169,7 @@ __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(con
                     *reinterpret_cast<uint32_t *>(bt + sw_off(i0, cb)) = pack_half2(s0.z, s0.w);
                     *reinterpret_cast<uint32_t *>(bt + sw_off(i1, ca)) = pack_half2(s1.x, s1.y);
                     *reinterpret_cast<uint32_t *>(bt + sw_off(i1, cb)) = pack_half2(s1.z, s1.w);
+                    range_check(fmaxf(absmax4(s0), absmax4(s1)));   // the fp16 S_in operand
                     if (kspan == PS - 1 && P.sf != nullptr) {
                         // final state of the sequence: D_span * S_in + S_local
                         const uint8_t *sst = sm + L::sst;
@@ -1134,7 +1178,7 @@ __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(con
                         };
                         const float g0 = dcum[nch * 64 + i0], g1 = dcum[nch * 64 + i1];
                         const float2 f0a = st2(i0, ca), f0b = st2(i0, cb), f1a = st2(i1, ca), f1b = st2(i1, cb);
-                        float *sf = P.sf + (size_t)seq * kDK * kDV;
+                        float *sf = P.sf + (size_t)seq * P.sstride;
                         *reinterpret_cast<float2 *>(sf + i0 * kDV + ca) = make_float2(fmaf(g0, s0.x, f0a.x), fmaf(g0, s0.y, f0a.y));
                         *reinterpret_cast<float2 *>(sf + i0 * kDV + cb) = make_float2(fmaf(g0, s0.z, f0b.x), fmaf(g0, s0.w, f0b.y));
                         *reinterpret_cast<float2 *>(sf + i1 * kDV + ca) = make_float2(fmaf(g1, s1.x, f1a.x), fmaf(g1, s1.y, f1a.y));
@@ -1201,7 +1245,7 @@ __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(con
         if constexpr (NL == 2) if (ext) {
             const uint32_t vo = smem_u32(sm + L::vop);
             load_qgo(P.q, P.g, P.out, P.N, P.H, P.W, P.dir, P.heads, seq, c0 + kHold, vo, vo + kTile,
-                     vo + 2 * kTile, kThreads);
+                     vo + 2 * kTile, kThreads, P.ldk);
         }
         if (NL == 2 && later) {
             if (tid < kspan) {
@@ -1285,6 +1329,7 @@ __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(con
                     const float4 s = *reinterpret_cast<const float4 *>(reinterpret_cast<const uint8_t *>(sin) + agg_off(i, c4));
                     *reinterpret_cast<uint2 *>(bt + sw_off(i, 4 * c4)) =
                         make_uint2(pack_half2(s.x, s.y), pack_half2(s.z, s.w));
+                    range_check(absmax4(s));   // the fp16 S_in operand
                 }
                 if (ext) cp_async_wait_all();   // the prefetch has landed (needed or not)
                 __syncthreads();
@@ -1343,7 +1388,7 @@ __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(con
                 if constexpr (NL == 2) {
                     const uint32_t stq = smem_u32(sm + L::stg);
                     load_qgo(P.q, P.g, P.out, P.N, P.H, P.W, P.dir, P.heads, seq, c0 + ci, stq,
-                             stq + 2 * kTile, stq + 3 * kTile, kThreads);
+                             stq + 2 * kTile, stq + 3 * kTile, kThreads, P.ldk);
                     cp_async_wait_all();
                     __syncthreads();
                     rebuild_qd(sm, sm + L::stg, sm + L::stg + 2 * kTile, dcum + ci * 64, sm + L::qint);
@@ -1358,7 +1403,7 @@ __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(con
                             const bool ok = p0 + t < P.N;
                             size_t ro = 0;
                             if (ok) ro = (size_t)((bq * P.N + scan_to_token(p0 + t, P.H, P.W, P.dir)) * P.heads + hq);
-                            const __half *src = ten == 0 ? P.q + ro * 64 : (ten == 1 ? P.g + ro * 64 : P.out + ro * 64);
+                            const __half *src = ten == 0 ? P.q + ro * P.ldk : (ten == 1 ? P.g + ro * P.ldk : P.out + ro * 64);
                             const int slot = ten == 0 ? 0 : (ten == 1 ? 2 : 3);
                             cp_async16(stq + slot * kTile + t * 128 + 16 * pc, src + 8 * pc, ok ? 16u : 0u);
                         }
@@ -1409,6 +1454,7 @@ __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(con
                         const float4 s = *reinterpret_cast<const float4 *>(reinterpret_cast<const uint8_t *>(sin) + agg_off(i, c4));
                         *reinterpret_cast<uint2 *>(bt + sw_off(i, 4 * c4)) =
                             make_uint2(pack_half2(s.x, s.y), pack_half2(s.z, s.w));
+                        range_check(absmax4(s));   // the fp16 S_in operand
                     }
                 }
                 fence_proxy_async_cta();
@@ -1454,7 +1500,7 @@ __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(con
                     s.z = fmaf(di, a.z, s.z);
                     s.w = fmaf(di, a.w, s.w);
                 }
-                reinterpret_cast<float4 *>(P.sf + (size_t)seq * kDK * kDV)[e] = s;
+                reinterpret_cast<float4 *>(P.sf + (size_t)seq * P.sstride)[e] = s;
             }
         }
         __syncthreads();   // staging / state tiles are reused by the next sequence

@@ -8,26 +8,22 @@
 // FP32 accumulation (section "速度到底快在哪，TensorRT部署做了什么": the heavy work of a
 // chunk is parallel, only the chunk-boundary state is passed in order).
 //
-// Kernels (one launch per call):
-//   * gla_fwd_span.cuh (dk = 64): each sequence is cut into spans of chunks that run
-//     on separate SMs with purely local state chains; one aggregate per span through
-//     a workspace, a look-back fold, and a deferred correction of the later spans'
-//     outputs.  The default for dk = 64.
-//   * gla_fwd_kernel<DK> below (dk = 64 or 128): a thread-block cluster of P CTAs
-//     owns one sequence at a time; in round r CTA `rank` processes chunk r*P + rank
-//     and the chunk-to-chunk state pass S_c = d_c * S_{c-1} + dS_c runs as an
-//     element-sliced scan over the cluster through distributed shared memory.
-//   * gla_fwd_ws.cuh (dk = 64): the cluster decomposition with warp-specialised
-//     roles and mbarrier hand-offs.
-//   Per chunk, in every kernel: q/k/g/v rows are staged with 16-byte cp.async (the
-//   scan direction is applied only in the row addresses); a = exp(g) with
-//   sub-block prefix/suffix products and totals, so that every decay factor fed to
-//   the tensor cores is a product of a's <= 1 except the diagonal sub-blocks,
-//   whose factor pi/T is bounded by exp(8) and falls back to an exact fp32
-//   evaluation beyond that; then tcgen05.mma (fp16 x fp16 -> fp32 in TMEM):
-//       dS     = (K * sigma * after)^T V
-//       scores = (Q * pi * c_J) (K * sigma)^T  per key sub-block J
-//       O      = (Q * pi * before) S_prev + tril(scores) V
+// Kernels:
+//   * gla_fwd_span.cuh (dk = 64, the default of gtr_gla_fwd): each sequence is cut into
+//     spans of chunks that run on separate SMs with purely local state chains; one
+//     aggregate per span through a workspace, a look-back fold, and a deferred
+//     correction of the later spans' outputs.  Chunk rows are staged with 16-byte
+//     cp.async (the scan direction applied only in the row addresses).
+//   * gla_fwd_pipe.cuh: the same span decomposition with TMA tensor copies and
+//     warp-specialised roles (gating teams, state group, readout group) on mbarrier
+//     hand-offs.  It serves gtr_gla_fwd_z (the gate formed from its pre-activation
+//     while staging), dk = 128 (two launches over the two 64-channel halves of the
+//     keys: the recurrence is separable by key channel and the second half adds its
+//     output to the first's), and dk = 64 when GTR_KERNEL=pipe.
+//   Per chunk, in both: gated operands whose decay factors fed to the tensor cores stay
+//   inside fp16 (a fast path for chunk decays >= e^-6, a 16-token sub-block path with an
+//   exact fp32 diagonal fallback otherwise), then tcgen05.mma (fp16 x fp16 -> fp32 in
+//   tensor memory) for dS = K~^T V, the causal scores Qint K~^T and O = Qint S_prev + P V.
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -45,12 +41,10 @@ namespace gtr {
 
 using namespace ptx;
 
-constexpr int kThreads = 256;
 constexpr int kChunk = 64;
 constexpr int kDV = 64;
 constexpr int kSub = 16;              // sub-block length for the decay factorisation
 constexpr int kTile = 64 * 128;       // one [64 rows][64 fp16] 128B-swizzled tile
-constexpr int kTmemCols = 256;
 constexpr int kMaxCluster = 16;
 constexpr float kDiagMinTotal = 3.3546262e-4f;  // exp(-8): smallest safe sub-block total
 constexpr float kFastMinDecay = 2.4787522e-3f;  // exp(-6): smallest chunk decay for the fast path
@@ -62,39 +56,6 @@ enum : unsigned { kErrTimeout = 1u, kErrRange = 2u };
 constexpr float kHalfMax = 65504.f;   // largest finite fp16
 
 __device__ unsigned int g_error_word;
-
-// ------------------------------------------------------------------ smem map
-// The q and k tiles are overwritten in place by the gated operands (Qint, and
-// K/P or K*sigma*after): ~104 KB per CTA at dk=64, ~182 KB at dk=128.
-template <int DK>
-struct Smem {
-    static constexpr int NSUB = DK / 64;
-    static constexpr int q = 0;                           // raw q, then Q*pi*before   [64][DK]
-    static constexpr int k = q + NSUB * kTile;            // raw k, then K/P or K*sig*after
-    static constexpr int g = k + NSUB * kTile;            // raw g                     [64][DK]
-    static constexpr int v0 = g + NSUB * kTile;           // v, double buffered        [64][64]
-    static constexpr int v1 = v0 + kTile;
-    static constexpr int qj = v1 + kTile;                 // packed Q^(J), rows 16J..63
-    static constexpr int qj_bytes = NSUB * (64 + 48 + 32 + 16) * 128;
-    static constexpr int kbar = qj + qj_bytes;            // K * sigma                 [64][DK]
-    static constexpr int p = kbar + NSUB * kTile;         // masked scores / out staging [64][64]
-    static constexpr int sop = p + kTile;                 // S_prev fp16               [DK][64]
-    static constexpr int diag = sop;                      // exact diag blocks, aliases sop
-    static constexpr int agg = sop + NSUB * kTile;        // dS fp32                   [DK][64]
-    static constexpr int dvec = agg + DK * 256;           // d = prod of a             [DK]
-    static constexpr int htot = dvec + DK * 4;            // half-block totals         [8][DK]
-    static constexpr int rowoff = htot + 8 * DK * 4;      // token rows                [2][64]
-    static constexpr int misc = rowoff + 2 * 64 * 4;      // flags, maxima, mbarrier, tmem addr
-    static constexpr int bytes = misc + 64;
-    static constexpr int alloc = bytes + 1024;            // + alignment slack
-    static constexpr int min_blocks = 1;   // thread-block clusters never co-reside two per SM here
-
-    static __host__ __device__ constexpr int qj_region(int J) {
-        return NSUB * 128 * (J == 0 ? 0 : J == 1 ? 64 : J == 2 ? 112 : 144);
-    }
-};
-static_assert(Smem<128>::alloc <= 227 * 1024, "dk=128 fits one CTA per SM");
-static_assert(4 * 16 * 16 * 4 <= 64 * 128, "diag blocks fit in the aliased S_prev tile");
 
 // 128B-swizzled [rows][64 fp16] tile: byte offset of (row, col) inside a sub-tile
 __device__ __forceinline__ uint32_t sw_off(int row, int col) {
@@ -126,61 +87,20 @@ struct Params {
     float *sf;
     int B, heads, H, W, N, dir;
     int n_seq, n_chunks;
-    int dk;   // key channels (the state has dk rows)
+    int dk;        // key channels (the state has dk rows)
+    int ldk;       // elements per q / k / g row (dk, or 128 for one half of a dk = 128 call)
+    int sstride;   // floats per sequence of init_state / final_state (dk * dv)
+    int acc;       // 1: add to the output tile instead of storing it (second key half)
 };
 
 __device__ __forceinline__ void set_error(unsigned e) { atomicOr(&g_error_word, e); }
-
-// ------------------------------------------------------------------ loads
-// 16-byte cp.async copies of one chunk's rows into 128B-swizzled tiles; two rows
-// per thread (tensor pair x 64 rows = 128 threads each half of the block).  Rows
-// whose token index is negative (past the end of the grid) are zero-filled.
-// which == 0: g and v (v into vbuf); which == 1: q and k.
-template <int DK>
-__device__ __forceinline__ void issue_loads(const Params &P, uint32_t sbase, const int *rowoff,
-                                            uint32_t vbuf_addr, int which) {
-    using L = Smem<DK>;
-    const int tid = threadIdx.x;
-    const int sel = tid >> 7, row = (tid >> 1) & 63, part = tid & 1;
-    const int ro = rowoff[row];
-    const uint32_t nbytes = ro < 0 ? 0u : 16u;
-    const size_t r0 = (size_t)(ro < 0 ? 0 : ro);
-    if (which == 1 || sel == 0) {
-        // q/k/g row: DK/8 pieces, split between the two threads of the pair
-        const __half *base = which == 1 ? (sel == 0 ? P.q : P.k) : P.g;
-        const uint32_t tile = sbase + (which == 1 ? (sel == 0 ? L::q : L::k) : L::g);
-        const __half *src = base + r0 * DK;
-#pragma unroll
-        for (int i = 0; i < DK / 16; ++i) {
-            const int pc = part * (DK / 16) + i;
-            cp_async16(tile + (pc >> 3) * kTile + sw_off(row, (pc & 7) * 8), src + pc * 8, nbytes);
-        }
-    } else {
-        const __half *src = P.v + r0 * kDV;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int pc = part * 4 + i;
-            cp_async16(vbuf_addr + sw_off(row, pc * 8), src + pc * 8, nbytes);
-        }
-    }
-    cp_async_commit();
+// A value about to become an fp16 operand or output must be finite and below 65504
+// (a NaN fails the comparison too): else the call reports GTR_ERR_RANGE.
+__device__ __forceinline__ void range_check(float mx) {
+    if (!(mx <= kHalfMax)) set_error(kErrRange);
 }
-
-// Token row index ((b*N + n)*heads + h) of each scan position of chunk c, or -1.
-__device__ __forceinline__ void fill_rowoff(const Params &P, int seq, int c, int *rowoff) {
-    const int t = threadIdx.x;
-    if (t < kChunk) {
-        int ro = -1;
-        if (seq >= 0 && c >= 0) {
-            const int p = c * kChunk + t;
-            if (p < P.N) {
-                const int b = seq / P.heads, h = seq - b * P.heads;
-                const int n = scan_to_token(p, P.H, P.W, P.dir);
-                ro = (b * P.N + n) * P.heads + h;
-            }
-        }
-        rowoff[t] = ro;
-    }
+__device__ __forceinline__ float absmax4(float4 v) {
+    return fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
 }
 
 __device__ __forceinline__ float2 ld_h2(const uint8_t *p) {
@@ -204,532 +124,6 @@ __device__ __forceinline__ void tmem_ld_16x256b_x4(uint32_t taddr, uint32_t (&r)
         : "memory");
 }
 
-// ------------------------------------------------------------------ kernel
-template <int DK>
-__global__ void __launch_bounds__(kThreads, Smem<DK>::min_blocks) gla_fwd_kernel(const Params P) {
-    using L = Smem<DK>;
-    constexpr int NP = DK / 64;           // channel pairs per thread in gating
-    constexpr int NF4 = DK * kDV / 4;     // float4 elements of the state
-    constexpr int MAXM = (NF4 + kThreads - 1) / kThreads;
-
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const uint32_t sbase = smem_u32(sm);
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-
-    const uint32_t rank = cluster_ctarank();
-    const uint32_t ncl = nclusters_x();
-    const int CP = (int)(gridDim.x / ncl);
-    const int cl = (int)cluster_id_x();
-
-    float *htot = reinterpret_cast<float *>(sm + L::htot);
-    float *dvec = reinterpret_cast<float *>(sm + L::dvec);
-    float *diagx = reinterpret_cast<float *>(sm + L::diag);
-    int *rowoff0 = reinterpret_cast<int *>(sm + L::rowoff);
-    int *flags = reinterpret_cast<int *>(sm + L::misc);                // [4] diag fallback flags
-    unsigned *qmax = reinterpret_cast<unsigned *>(sm + L::misc + 16);  // [4] max |q| per block (bits)
-    unsigned *kmax = reinterpret_cast<unsigned *>(sm + L::misc + 32);  // max |k| in the chunk (bits)
-    uint64_t *mbar = reinterpret_cast<uint64_t *>(sm + L::misc + 40);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::misc + 48);
-
-    if (warp == 0) {
-        tmem_alloc(tmem_slot, kTmemCols);
-        tmem_relinquish();
-    }
-    if (tid == 0) {
-        mbar_init(mbar, 1);
-        fence_mbar_init();
-    }
-    if (tid < 4) { flags[tid] = 0; qmax[tid] = 0u; }
-    if (tid == 0) *kmax = 0u;
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-    uint32_t mma_phase = 0;
-    bool timed_out = false;
-
-    // gating thread map: warp -> (sub-block I, half hf), lane -> channel pair(s)
-    const int gI = warp >> 1, ghf = warp & 1, gt0 = 16 * gI + 8 * ghf, gh = 2 * gI + ghf;
-    // readout thread map for M=64 accumulators: subpartition, column half
-    const int sp = warp & 3, chalf = warp >> 2;
-    const int rrow0 = 16 * sp + (lane >> 2);          // and rrow0 + 8
-    const int rcol0 = 32 * chalf + 2 * (lane & 3);    // + 8c, +1
-
-    // element slice of the state owned by this CTA in the scan
-    const int slo = (int)((long)rank * NF4 / CP);
-    const int shi = (int)((long)(rank + 1) * NF4 / CP);
-    const int nloc = shi - slo;
-
-    int cur = 0, vb = 0;
-    {
-        const int seq0 = cl < P.n_seq ? cl : -1;
-        const int c0 = (seq0 >= 0 && (int)rank < P.n_chunks) ? (int)rank : -1;
-        fill_rowoff(P, seq0, c0, rowoff0);
-        __syncthreads();
-        if (c0 >= 0) {
-            issue_loads<DK>(P, sbase, rowoff0, sbase + L::v0, 0);
-            issue_loads<DK>(P, sbase, rowoff0, sbase + L::v0, 1);
-        }
-    }
-
-    for (int seq = cl; seq < P.n_seq; seq += (int)ncl) {
-        float4 S[MAXM];
-#pragma unroll
-        for (int m = 0; m < MAXM; ++m) {
-            const int el = tid + m * kThreads;
-            S[m] = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (P.s0 != nullptr && el < nloc)
-                S[m] = reinterpret_cast<const float4 *>(P.s0 + (size_t)seq * DK * kDV)[slo + el];
-        }
-        const int n_rounds = (P.n_chunks + CP - 1) / CP;
-        for (int r = 0; r < n_rounds; ++r) {
-            const int c = r * CP + (int)rank;
-            const bool valid = c < P.n_chunks;
-            const int nvalid = min(CP, P.n_chunks - r * CP);
-            int *rowoff_cur = rowoff0 + cur * 64;
-            int *rowoff_nxt = rowoff0 + (cur ^ 1) * 64;
-            const uint32_t vaddr = sbase + (vb ? L::v1 : L::v0);
-            const uint32_t vnext = sbase + (vb ? L::v0 : L::v1);
-            // rows of the next chunk (this sequence, or the first round of the next)
-            int nseq = seq, nc = c + CP;
-            if (nc >= P.n_chunks) {
-                nseq = seq + (int)ncl;
-                nc = (nseq < P.n_seq && (int)rank < P.n_chunks) ? (int)rank : -1;
-                if (nseq >= P.n_seq) nseq = -1;
-            }
-            fill_rowoff(P, nseq, nc, rowoff_nxt);
-
-            cp_async_wait_all();
-            __syncthreads();
-
-            bool slow = false;   // CTA-uniform: sub-block factorisation for this chunk
-            if (valid) {
-                // ------------- gating pass 1: a = exp(g); half-block prefix/suffix products
-                float pl[8][2 * NP], sl[8][2 * NP];
-                __half2 qh[8][NP], kh[8][NP];
-                float qm = 0.f, km = 0.f;
-#pragma unroll
-                for (int p2 = 0; p2 < NP; ++p2) {
-                    float a0[8], a1[8];
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const uint32_t o = p2 * kTile + sw_off(gt0 + u, 2 * lane);
-                        const float2 gv = ld_h2(sm + L::g + o);
-                        qh[u][p2] = *reinterpret_cast<const __half2 *>(sm + L::q + o);
-                        kh[u][p2] = *reinterpret_cast<const __half2 *>(sm + L::k + o);
-                        a0[u] = exp_f(gv.x);
-                        a1[u] = exp_f(gv.y);
-                        const float2 qf = __half22float2(qh[u][p2]), kf = __half22float2(kh[u][p2]);
-                        qm = fmaxf(qm, fmaxf(fabsf(qf.x), fabsf(qf.y)));
-                        km = fmaxf(km, fmaxf(fabsf(kf.x), fabsf(kf.y)));
-                    }
-                    float r0 = 1.f, r1 = 1.f;
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        r0 *= a0[u]; r1 *= a1[u];
-                        pl[u][2 * p2] = r0; pl[u][2 * p2 + 1] = r1;
-                    }
-                    r0 = 1.f; r1 = 1.f;
-#pragma unroll
-                    for (int u = 7; u >= 0; --u) {
-                        sl[u][2 * p2] = r0; sl[u][2 * p2 + 1] = r1;
-                        r0 *= a0[u]; r1 *= a1[u];
-                    }
-                    *reinterpret_cast<float2 *>(htot + gh * DK + 64 * p2 + 2 * lane) =
-                        make_float2(pl[7][2 * p2], pl[7][2 * p2 + 1]);
-                }
-                // block maxima of |q| and chunk maximum of |k| (non-negative floats order as uints)
-                {
-                    const unsigned wq = __reduce_max_sync(0xffffffffu, __float_as_uint(qm));
-                    const unsigned wk = __reduce_max_sync(0xffffffffu, __float_as_uint(km));
-                    if (lane == 0) {
-                        atomicMax(&qmax[gI], wq);
-                        atomicMax(kmax, wk);
-                    }
-                }
-                __syncthreads();
-                // ------------- chunk-level factors for my channels
-                float dch[2 * NP], bef[2 * NP], aft[2 * NP];
-                bool bad = __uint_as_float(*kmax) > kFastMaxK;
-#pragma unroll
-                for (int p2 = 0; p2 < NP; ++p2) {
-                    float2 ht[8];
-#pragma unroll
-                    for (int h8 = 0; h8 < 8; ++h8)
-                        ht[h8] = *reinterpret_cast<const float2 *>(htot + h8 * DK + 64 * p2 + 2 * lane);
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        float d = 1.f, bf = 1.f, af = 1.f;
-#pragma unroll
-                        for (int h8 = 0; h8 < 8; ++h8) {
-                            const float x = e ? ht[h8].y : ht[h8].x;
-                            d *= x;
-                            if (h8 < gh) bf *= x;
-                            if (h8 > gh) af *= x;
-                        }
-                        dch[2 * p2 + e] = d; bef[2 * p2 + e] = bf; aft[2 * p2 + e] = af;
-                        bad |= !(d >= kFastMinDecay);
-                    }
-                }
-                slow = __syncthreads_or(bad) != 0;
-                if (gh == 0) {
-#pragma unroll
-                    for (int p2 = 0; p2 < NP; ++p2)
-                        *reinterpret_cast<float2 *>(dvec + 64 * p2 + 2 * lane) =
-                            make_float2(dch[2 * p2], dch[2 * p2 + 1]);
-                }
-                if (!slow) {
-                    // ------------- fast path (in place): Qint = q * P, Kt = k / P  (P >= e^-6)
-#pragma unroll
-                    for (int p2 = 0; p2 < NP; ++p2) {
-                        const float i0 = aft[2 * p2] / dch[2 * p2];
-                        const float i1 = aft[2 * p2 + 1] / dch[2 * p2 + 1];
-#pragma unroll
-                        for (int u = 0; u < 8; ++u) {
-                            const uint32_t o = p2 * kTile + sw_off(gt0 + u, 2 * lane);
-                            const float2 qv = __half22float2(qh[u][p2]);
-                            const float2 kv = __half22float2(kh[u][p2]);
-                            st_h2(sm + L::q + o, qv.x * (pl[u][2 * p2] * bef[2 * p2]),
-                                  qv.y * (pl[u][2 * p2 + 1] * bef[2 * p2 + 1]));
-                            st_h2(sm + L::k + o, kv.x * (sl[u][2 * p2] * i0),
-                                  kv.y * (sl[u][2 * p2 + 1] * i1));
-                        }
-                    }
-                } else {
-                    // ------------- sub-block path: every off-diagonal factor <= 1
-                    float T[4][2 * NP];
-#pragma unroll
-                    for (int p2 = 0; p2 < NP; ++p2)
-#pragma unroll
-                        for (int L4 = 0; L4 < 4; ++L4) {
-                            const float2 h0 = *reinterpret_cast<const float2 *>(
-                                htot + (2 * L4) * DK + 64 * p2 + 2 * lane);
-                            const float2 h1 = *reinterpret_cast<const float2 *>(
-                                htot + (2 * L4 + 1) * DK + 64 * p2 + 2 * lane);
-                            T[L4][2 * p2] = h0.x * h1.x;
-                            T[L4][2 * p2 + 1] = h0.y * h1.y;
-                        }
-                    // diagonal sub-block I needs the exact path if some channel decays by more
-                    // than e^8 inside it, or if q * e^8 could leave the fp16 range
-                    bool dbad = false;
-#pragma unroll
-                    for (int j = 0; j < 2 * NP; ++j)
-#pragma unroll
-                        for (int L4 = 0; L4 < 4; ++L4)
-                            if (L4 == gI) dbad |= !(T[L4][j] >= kDiagMinTotal);
-                    dbad |= __uint_as_float(qmax[gI]) > kDiagMaxQ;
-                    if (__any_sync(0xffffffffu, dbad) && lane == 0) atomicOr(&flags[gI], 1);
-                    __syncthreads();
-                    const int anyflag = flags[0] | flags[1] | flags[2] | flags[3];
-                    if (anyflag) {
-                        // exact fp32 diagonal sub-blocks, from the raw tiles (still intact)
-                        const uint8_t *qt = sm + L::q, *kt = sm + L::k, *gt = sm + L::g;
-                        for (int pr = tid; pr < 4 * 256; pr += kThreads) {
-                            const int I = pr >> 8, u = (pr >> 4) & 15, w = pr & 15;
-                            if (!flags[I] || w > u) continue;
-                            const int tu = I * kSub + u, tw = I * kSub + w;
-                            float acc = 0.f;
-                            for (int i = 0; i < DK; ++i) {
-                                const int si = i >> 6, ci = i & 63;
-                                float lg = 0.f;
-                                for (int rr = tw + 1; rr <= tu; ++rr)
-                                    lg += __half2float(*reinterpret_cast<const __half *>(
-                                        gt + si * kTile + sw_off(rr, ci)));
-                                const float qv = __half2float(*reinterpret_cast<const __half *>(
-                                    qt + si * kTile + sw_off(tu, ci)));
-                                const float kv = __half2float(*reinterpret_cast<const __half *>(
-                                    kt + si * kTile + sw_off(tw, ci)));
-                                acc += qv * kv * exp_f(lg);
-                            }
-                            diagx[(I * 16 + u) * 16 + w] = acc;
-                        }
-                        __syncthreads();
-                    }
-                    const bool diag_bad = flags[gI] != 0;
-#pragma unroll
-                    for (int p2 = 0; p2 < NP; ++p2) {
-                        float cf[2][4], bI[2], aI[2], hin[2], hout[2];
-                        const float2 h0 = *reinterpret_cast<const float2 *>(
-                            htot + (2 * gI) * DK + 64 * p2 + 2 * lane);
-                        const float2 h1 = *reinterpret_cast<const float2 *>(
-                            htot + (2 * gI + 1) * DK + 64 * p2 + 2 * lane);
-#pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const int j = 2 * p2 + e;
-                            float b0 = 1.f, a0 = 1.f, tI = 1.f;
-#pragma unroll
-                            for (int L4 = 0; L4 < 4; ++L4) {
-                                if (L4 < gI) b0 *= T[L4][j];
-                                if (L4 > gI) a0 *= T[L4][j];
-                                if (L4 == gI) tI = T[L4][j];
-                            }
-                            bI[e] = b0; aI[e] = a0;
-#pragma unroll
-                            for (int J = 0; J < 4; ++J) {
-                                float cj = 1.f;
-#pragma unroll
-                                for (int L4 = 0; L4 < 4; ++L4)
-                                    if (L4 > J && L4 < gI) cj *= T[L4][j];
-                                cf[e][J] = (J == gI) ? (diag_bad ? 0.f : 1.f / tI) : cj;
-                            }
-                            // pi / sigma inside the 16-block from the half-local products
-                            hin[e] = ghf ? (e ? h0.y : h0.x) : 1.f;
-                            hout[e] = ghf ? 1.f : (e ? h1.y : h1.x);
-                        }
-#pragma unroll
-                        for (int u = 0; u < 8; ++u) {
-                            const int t = gt0 + u;
-                            const uint32_t o = p2 * kTile + sw_off(t, 2 * lane);
-                            const float2 qv = __half22float2(qh[u][p2]);
-                            const float2 kv = __half22float2(kh[u][p2]);
-                            const float qp0 = qv.x * (pl[u][2 * p2] * hin[0]);
-                            const float qp1 = qv.y * (pl[u][2 * p2 + 1] * hin[1]);
-                            const float ks0 = kv.x * (sl[u][2 * p2] * hout[0]);
-                            const float ks1 = kv.y * (sl[u][2 * p2 + 1] * hout[1]);
-                            st_h2(sm + L::q + o, qp0 * bI[0], qp1 * bI[1]);
-                            st_h2(sm + L::kbar + o, ks0, ks1);
-                            st_h2(sm + L::k + o, ks0 * aI[0], ks1 * aI[1]);
-#pragma unroll
-                            for (int J = 0; J < 4; ++J) {
-                                if (J <= gI) {
-                                    const int rows_j = 64 - 16 * J;
-                                    st_h2(sm + L::qj + L::qj_region(J) + p2 * rows_j * 128 +
-                                              sw_off(t - 16 * J, 2 * lane),
-                                          qp0 * cf[0][J], qp1 * cf[1][J]);
-                                }
-                            }
-                        }
-                    }
-                }
-            }
-            fence_proxy_async_cta();
-            __syncthreads();
-            // g tile and the other v buffer are free: prefetch the next chunk's g and v
-            if (nc >= 0) issue_loads<DK>(P, sbase, rowoff_nxt, vnext, 0);
-
-            // ------------- MMA 1: dS (dS / d on the fast path) and the scores
-            if (valid && tid == 0) {
-                tc_fence_after();
-                {
-                    constexpr uint32_t id = idesc_f16_f32(DK, kDV, true, true);
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        umma_f16(tmem + 0, desc_sw128(sbase + L::k + kk * 2048, kTile, 1024),
-                                 desc_sw128(vaddr + kk * 2048, kTile, 1024), id, kk > 0 ? 1u : 0u);
-                }
-                if (!slow) {
-                    constexpr uint32_t id = idesc_f16_f32(64, 64, false, false);
-#pragma unroll
-                    for (int kk = 0; kk < DK / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * kTile + (kk & 3) * 32;
-                        umma_f16(tmem + 64, desc_sw128(sbase + L::q + off, 16, 1024),
-                                 desc_sw128(sbase + L::k + off, 16, 1024), id, kk > 0 ? 1u : 0u);
-                    }
-                } else {
-                    constexpr uint32_t id = idesc_f16_f32(64, 16, false, false);
-                    for (int J = 0; J < 4; ++J) {
-                        const int rows_j = 64 - 16 * J;
-#pragma unroll
-                        for (int kk = 0; kk < DK / 16; ++kk) {
-                            const int sub = kk >> 2, koff = (kk & 3) * 32;
-                            const uint32_t aa = sbase + L::qj + L::qj_region(J) +
-                                                sub * rows_j * 128 - 16 * J * 128 + koff;
-                            const uint32_t bb = sbase + L::kbar + sub * kTile + 16 * J * 128 + koff;
-                            umma_f16(tmem + 64 + 16 * J, desc_sw128(aa, 16, 1024),
-                                     desc_sw128(bb, 16, 1024), id, kk > 0 ? 1u : 0u);
-                        }
-                    }
-                }
-                umma_commit(mbar);
-            }
-            if (valid) {
-                if (!mbar_wait_bounded(mbar, mma_phase, kWaitLimitNs)) {
-                    timed_out = true;
-                    set_error(kErrTimeout);
-                }
-                mma_phase ^= 1u;
-                tc_fence_after();
-                // scores -> masked fp16 P: this warp's 16 rows x 32 columns; dS -> fp32
-                // aggregate tile for the cluster scan (fast path: rows scaled by d)
-                uint32_t rs[16], rd[(DK == 64) ? 16 : 32];
-                tmem_ld_16x256b_x4(tmem + ((uint32_t)(32 * sp) << 16) + 64 + 32 * chalf, rs);
-                if (DK == 64) {
-                    tmem_ld_16x256b_x4(tmem + ((uint32_t)(32 * sp) << 16) + 32 * chalf,
-                                       *reinterpret_cast<uint32_t(*)[16]>(&rd[0]));
-                } else {
-                    const uint32_t ta = tmem + ((uint32_t)(32 * sp) << 16) + 32 * chalf;
-                    tmem_ld16(ta, *reinterpret_cast<uint32_t(*)[16]>(&rd[0]));
-                    tmem_ld16(ta + 16, *reinterpret_cast<uint32_t(*)[16]>(&rd[(DK == 64) ? 0 : 16]));
-                }
-                tmem_ld_wait();
-                {
-                    uint32_t *rr = rs;
-                    const bool fb = slow && (flags[sp] != 0);
-#pragma unroll
-                    for (int cc = 0; cc < 4; ++cc) {
-#pragma unroll
-                        for (int hh = 0; hh < 2; ++hh) {
-                            const int row = rrow0 + 8 * hh;
-                            const int col = rcol0 + 8 * cc;
-                            float x0 = __uint_as_float(rr[4 * cc + 2 * hh]);
-                            float x1 = __uint_as_float(rr[4 * cc + 2 * hh + 1]);
-                            if (fb && (col >> 4) == sp) {
-                                x0 = diagx[(sp * 16 + (row & 15)) * 16 + (col & 15)];
-                                x1 = diagx[(sp * 16 + (row & 15)) * 16 + ((col + 1) & 15)];
-                            }
-                            x0 = col <= row ? x0 : 0.f;
-                            x1 = col + 1 <= row ? x1 : 0.f;
-                            st_h2(sm + L::p + sw_off(row, col), x0, x1);
-                        }
-                    }
-                }
-                if (DK == 64) {
-                    const uint32_t *rr = rd;
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        const int i = rrow0 + 8 * hh;
-                        const float sc = slow ? 1.f : dvec[i];
-#pragma unroll
-                        for (int cc = 0; cc < 4; ++cc) {
-                            const int col = rcol0 + 8 * cc;
-                            *reinterpret_cast<float2 *>(sm + L::agg + agg_off(i, col >> 2) +
-                                                        (col & 3) * 4) =
-                                make_float2(sc * __uint_as_float(rr[4 * cc + 2 * hh]),
-                                            sc * __uint_as_float(rr[4 * cc + 2 * hh + 1]));
-                        }
-                    }
-                } else {
-                    // M = 128: row i in lane i; this warp: rows 32*sp + lane, 32 columns
-                    const uint32_t *rr = rd;
-                    const int i = 32 * sp + lane;
-                    const float sc = slow ? 1.f : dvec[i];
-#pragma unroll
-                    for (int c4 = 0; c4 < 8; ++c4)
-                        *reinterpret_cast<float4 *>(sm + L::agg + agg_off(i, 8 * chalf + c4)) =
-                            make_float4(sc * __uint_as_float(rr[4 * c4]), sc * __uint_as_float(rr[4 * c4 + 1]),
-                                        sc * __uint_as_float(rr[4 * c4 + 2]), sc * __uint_as_float(rr[4 * c4 + 3]));
-                }
-            }
-            fence_proxy_async_cta();
-            tc_fence_before();
-            cluster_sync();   // every chunk's (d, dS) of this round is visible cluster-wide
-            if (tid < 4) { flags[tid] = 0; qmax[tid] = 0u; }
-            if (tid == 0) *kmax = 0u;
-
-            // ------------- state pass: chain this CTA's slice of the state through the
-            // round's chunks.  Peers' (d, dS) are fetched over DSMEM four chunks at a time
-            // so the round trips overlap; S_prev goes straight into each chunk's operand tile.
-#pragma unroll
-            for (int m = 0; m < MAXM; ++m) {
-                const int el = tid + m * kThreads;
-                if (el < nloc) {
-                    const int e = slo + el, i = e >> 4, c4 = e & 15;
-                    const uint32_t aoff = sbase + L::agg + agg_off(i, c4);
-                    const uint32_t doff = sbase + L::dvec + i * 4;
-                    const uint32_t soff = sbase + L::sop + sw_off(i, 4 * c4);
-                    for (int j0 = 0; j0 < nvalid; j0 += 4) {
-                        float4 a4[4];
-                        float dd[4];
-#pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4) {
-                            if (j0 + q4 < nvalid) {
-                                a4[q4] = ld_dsmem_f4(mapa(aoff, (uint32_t)(j0 + q4)));
-                                dd[q4] = ld_dsmem_f32(mapa(doff, (uint32_t)(j0 + q4)));
-                            }
-                        }
-#pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4) {
-                            if (j0 + q4 < nvalid) {
-                                st_dsmem_v2(mapa(soff, (uint32_t)(j0 + q4)), pack_half2(S[m].x, S[m].y),
-                                            pack_half2(S[m].z, S[m].w));
-                                S[m].x = fmaf(dd[q4], S[m].x, a4[q4].x);
-                                S[m].y = fmaf(dd[q4], S[m].y, a4[q4].y);
-                                S[m].z = fmaf(dd[q4], S[m].z, a4[q4].z);
-                                S[m].w = fmaf(dd[q4], S[m].w, a4[q4].w);
-                            }
-                        }
-                    }
-                }
-            }
-            fence_proxy_async_cluster();
-            cluster_sync();   // every S_prev tile of this round is written
-
-            // ------------- MMA 2: O = Qint S_prev + tril(scores) V
-            if (valid && tid == 0) {
-                tc_fence_after();
-                constexpr uint32_t id = idesc_f16_f32(64, kDV, false, true);
-#pragma unroll
-                for (int kk = 0; kk < DK / 16; ++kk) {
-                    const uint32_t aa = sbase + L::q + (kk >> 2) * kTile + (kk & 3) * 32;
-                    const uint32_t bb = sbase + L::sop + kk * 2048;
-                    umma_f16(tmem + 128, desc_sw128(aa, 16, 1024), desc_sw128(bb, kTile, 1024), id,
-                             kk > 0 ? 1u : 0u);
-                }
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint32_t aa = sbase + L::p + kk * 32;
-                    const uint32_t bb = vaddr + kk * 2048;
-                    umma_f16(tmem + 128, desc_sw128(aa, 16, 1024), desc_sw128(bb, kTile, 1024), id, 1u);
-                }
-                umma_commit(mbar);
-            }
-            if (valid) {
-                if (!mbar_wait_bounded(mbar, mma_phase, kWaitLimitNs)) {
-                    timed_out = true;
-                    set_error(kErrTimeout);
-                }
-                mma_phase ^= 1u;
-                tc_fence_after();
-                {
-                    // O -> fp16, staged (swizzled) in the P tile, then coalesced rows to global
-                    uint32_t rr[16];
-                    tmem_ld_16x256b_x4(tmem + ((uint32_t)(32 * sp) << 16) + 128 + 32 * chalf, rr);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int cc = 0; cc < 4; ++cc)
-#pragma unroll
-                        for (int hh = 0; hh < 2; ++hh)
-                            st_h2(sm + L::p + sw_off(rrow0 + 8 * hh, rcol0 + 8 * cc),
-                                  __uint_as_float(rr[4 * cc + 2 * hh]),
-                                  __uint_as_float(rr[4 * cc + 2 * hh + 1]));
-                }
-            }
-            // q/k tiles (Qint, K operands) and the staging are consumed: prefetch next q, k
-            __syncthreads();
-            if (nc >= 0) issue_loads<DK>(P, sbase, rowoff_nxt, vnext, 1);
-            if (valid) {
-#pragma unroll
-                for (int x = tid; x < 64 * 8; x += kThreads) {
-                    const int row = x >> 3, c8 = x & 7;
-                    const int ro = rowoff_cur[row];
-                    if (ro >= 0)
-                        *reinterpret_cast<uint4 *>(P.out + (size_t)ro * kDV + 8 * c8) =
-                            *reinterpret_cast<const uint4 *>(sm + L::p + sw_off(row, 8 * c8));
-                }
-            }
-            tc_fence_before();
-            cur ^= 1;
-            vb ^= 1;
-        }
-        if (P.sf != nullptr) {
-#pragma unroll
-            for (int m = 0; m < MAXM; ++m) {
-                const int el = tid + m * kThreads;
-                if (el < nloc)
-                    reinterpret_cast<float4 *>(P.sf + (size_t)seq * DK * kDV)[slo + el] = S[m];
-            }
-        }
-    }
-
-    cp_async_wait_all();
-    __syncthreads();
-    if (timed_out) mbar_wait_bounded(mbar, mma_phase ^ 1u, kWaitLimitNs);
-    cluster_sync();   // no CTA leaves while a peer may still touch its shared memory
-    if (warp == 0) tmem_dealloc(tmem, kTmemCols);
-}
-
 }  // namespace gtr
 
 #include "gla_fwd_span.cuh"
@@ -738,13 +132,12 @@ __global__ void __launch_bounds__(kThreads, Smem<DK>::min_blocks) gla_fwd_kernel
 namespace gtr {
 
 // ------------------------------------------------------------------ host
-enum KernelKind { kBasic128 = 0, kSpan = 1, kSpanShort = 2, kPipe = 3, kPipeZ = 4, kKinds = 5 };
+enum KernelKind { kSpan = 0, kSpanShort = 1, kPipe = 2, kPipeZ = 3, kKinds = 4 };
 
 // the span kernel with two loader warps (kSpan) or four (kSpanShort: short spans)
 static bool is_span(int kind) { return kind == kSpan || kind == kSpanShort; }
-// kernels whose CTAs of one sequence must be co-resident (cooperative launch)
+// the TMA-staged warp-specialised kernel (g, or its pre-activation z)
 static bool is_pipe(int kind) { return kind == kPipe || kind == kPipeZ; }
-static bool is_coop(int kind) { return is_span(kind) || is_pipe(kind); }
 
 // A kernel variant: entry point, block size, dynamic shared memory, cache slot.
 struct KSpec {
@@ -767,8 +160,6 @@ struct Plan {
 // (tuning knob) selects one of the other dk = 64 kernels instead.
 static KSpec spec_of(int kind) {
     switch (kind) {
-    case kBasic128:
-        return KSpec{reinterpret_cast<const void *>(&gla_fwd_kernel<128>), kThreads, Smem<128>::alloc, kBasic128};
     case kSpanShort:
         return KSpec{reinterpret_cast<const void *>(&sp::gla_fwd_span_kernel<4>), sp::span_threads<4>(),
                      sp::L::alloc, kSpanShort};
@@ -784,16 +175,13 @@ static KSpec spec_of(int kind) {
 
 static int kind_for(int dk, long n_chunks) {
     (void)n_chunks;
-    if (dk != 64) return kBasic128;
     const char *e = getenv("GTR_KERNEL");
-    if (e && !strcmp(e, "pipe")) return kPipe;
+    if (e && !strcmp(e, "pipe")) return kPipe;   // (dk = 128: two 64-channel halves, as with the span kernel)
     return kSpan;
 }
 
 static std::mutex g_mu;
 static int g_num_sms[64];
-// max co-resident clusters per (device, kernel variant, cluster size); 0 = not queried
-static int g_max_active[64][kKinds][kMaxCluster + 1];
 // co-resident CTAs of the span kernel per device; 0 = not queried
 static int g_span_capacity[64];
 
@@ -816,11 +204,8 @@ static int num_sms(int dev) {
     return g_num_sms[dev];
 }
 
-static cudaError_t prepare_kernel(const KSpec &k, int cluster) {
-    cudaError_t e = cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, k.smem);
-    if (e == cudaSuccess && cluster > 8)
-        e = cudaFuncSetAttribute(k.fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    return e;
+static cudaError_t prepare_kernel(const KSpec &k) {
+    return cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, k.smem);
 }
 
 static void fill_config(cudaLaunchConfig_t &cfg, cudaLaunchAttribute *attr, const KSpec &k,
@@ -831,43 +216,16 @@ static void fill_config(cudaLaunchConfig_t &cfg, cudaLaunchAttribute *attr, cons
     cfg.dynamicSmemBytes = (size_t)k.smem;
     cfg.stream = stream;
     cfg.attrs = attr;
-    if (is_coop(k.slot)) {
-        // all spans of a sequence must be resident together: cooperative launch; the
-        // next launch on the stream may start its set-up while this one drains (the
-        // kernel waits for its predecessor before touching global memory)
-        attr[0].id = cudaLaunchAttributeCooperative;
-        attr[0].val.cooperative = 1;
-        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[1].val.programmaticStreamSerializationAllowed = 1;
-        cfg.numAttrs = 2;
-    } else {
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = (unsigned)cluster;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.numAttrs = 1;
-    }
+    // all spans of a sequence must be resident together: cooperative launch; the next
+    // launch on the stream may start its set-up while this one drains (the kernel waits
+    // for its predecessor before touching global memory)
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.numAttrs = 2;
 }
 
-static int max_active_clusters(const KSpec &k, int dev, int cluster, int sms) {
-    int &slot = g_max_active[dev][k.slot][cluster];
-    {
-        std::lock_guard<std::mutex> lk(g_mu);
-        if (slot != 0) return slot;
-    }
-    int n = 0;
-    if (prepare_kernel(k, cluster) == cudaSuccess) {
-        cudaLaunchConfig_t cfg;
-        cudaLaunchAttribute attr[2];
-        fill_config(cfg, attr, k, cluster, sms / cluster, 0);
-        if (cudaOccupancyMaxActiveClusters(&n, k.fn, &cfg) != cudaSuccess) n = 0;
-    }
-    cudaGetLastError();
-    if (n <= 0) n = -1;   // cluster size not schedulable
-    std::lock_guard<std::mutex> lk(g_mu);
-    slot = n;
-    return n;
-}
 
 static int span_capacity(int dev, int sms, bool query) {
     if (!query) return sms;
@@ -877,7 +235,7 @@ static int span_capacity(int dev, int sms, bool query) {
     }
     const KSpec k = spec_of(kSpan);
     int per_sm = 0;
-    if (prepare_kernel(k, 1) != cudaSuccess ||
+    if (prepare_kernel(k) != cudaSuccess ||
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k.fn, k.threads, (size_t)k.smem) != cudaSuccess)
         per_sm = 0;
     cudaGetLastError();
@@ -949,32 +307,6 @@ static Plan span_plan(long n_seq, long n_chunks, int cap, int kind, size_t ws_li
 
 // Cluster plan: the cluster size that minimises (waves of clusters) x (rounds per
 // sequence + 1), preferring the smaller cluster on ties.
-static Plan cluster_plan(int kind, long n_seq, long n_chunks, int dev, int sms, bool query) {
-    const KSpec k = spec_of(kind);
-    const int cp_min = 1;
-    Plan best{kind, cp_min, 1, 0, k.smem, k.threads, 0};
-    const int fc = forced_cluster();
-    long best_cost = -1;
-    for (int pass = 0; pass < 2 && best_cost < 0; ++pass) {
-        for (int cp = cp_min; cp <= kMaxCluster; ++cp) {
-            if (n_chunks > 0 && cp > n_chunks) break;
-            if (n_chunks == 0 && cp > 1) break;
-            if (pass == 0 && fc > 0 && cp != fc) continue;
-            const int act = query ? max_active_clusters(k, dev, cp, sms) : sms / cp;
-            if (act <= 0) continue;
-            const long ncl = n_seq < act ? n_seq : act;
-            const long waves = (n_seq + ncl - 1) / ncl;
-            const long rounds = n_chunks > 0 ? (n_chunks + cp - 1) / cp : 0;
-            const long cost = waves * (rounds + 1);
-            if (best_cost < 0 || cost < best_cost) {
-                best_cost = cost;
-                best.cluster = cp;
-                best.clusters = (int)(ncl < 1 ? 1 : ncl);
-            }
-        }
-    }
-    return best;
-}
 
 // ws_limit: the largest workspace the caller can provide (the static scratch's size
 // for gtr_gla_fwd_static; unlimited otherwise).
@@ -984,12 +316,9 @@ static Plan make_plan(long n_seq, long n_chunks, int dk, bool query, size_t ws_l
     const int dev = current_device();
     const int sms = num_sms(dev);
     if (n_chunks == 0) return Plan{kind, 1, 1, 0, 0, 0, 0};   // no launch: the state copy only
-    if (kind == kSpan || is_pipe(kind)) {
-        const int cap = span_capacity(dev, sms, query);
-        if (cap > 0) return span_plan(n_seq, n_chunks, cap, kind, ws_limit);
-        return Plan{-1, 1, 1, 0, 0, 0, 0};   // no co-resident span plan on this device
-    }
-    return cluster_plan(kind, n_seq, n_chunks, dev, sms, query);
+    const int cap = span_capacity(dev, sms, query);
+    if (cap > 0) return span_plan(n_seq, n_chunks, cap, kind, ws_limit);
+    return Plan{-1, 1, 1, 0, 0, 0, 0};   // no co-resident span plan on this device
 }
 
 // Library-cached workspace of gtr_gla_fwd, one per device: sized for the largest
@@ -1080,18 +409,18 @@ static unsigned used_heights(int H, int W, int dir) {
     return m & 0x7fu;
 }
 
-// One tensor ([B, N, heads, d] fp16) as a row view (d, heads, N, B) or a column view
-// (d, heads, W, H, B), box d x 1 x 2^h rows.
+// One tensor ([B, N, heads, pitch] fp16, channels 0 .. d-1 of each row at `ptr`) as a
+// row view (d, heads, N, B) or a column view (d, heads, W, H, B), box d x 1 x 2^h rows.
 static CUresult encode_map(EncodeTiledFn enc, CUtensorMap *m, const void *ptr, int B, int heads, int H, int W,
-                           int d, bool column, int h) {
+                           int d, int pitch, bool column, int h) {
     const cuuint64_t es = 2;
     cuuint64_t dims[5], strides[4];
     cuuint32_t box[5], estr[5] = {1, 1, 1, 1, 1};
     const cuuint64_t N = (cuuint64_t)H * W;
     dims[0] = (cuuint64_t)d;
     dims[1] = (cuuint64_t)heads;
-    strides[0] = (cuuint64_t)d * es;
-    strides[1] = (cuuint64_t)heads * d * es;
+    strides[0] = (cuuint64_t)pitch * es;
+    strides[1] = (cuuint64_t)heads * pitch * es;
     box[0] = (cuuint32_t)d;
     box[1] = 1;
     cuuint32_t rank;
@@ -1099,7 +428,7 @@ static CUresult encode_map(EncodeTiledFn enc, CUtensorMap *m, const void *ptr, i
         rank = 4;
         dims[2] = N;
         dims[3] = (cuuint64_t)B;
-        strides[2] = N * heads * d * es;
+        strides[2] = N * heads * pitch * es;
         box[2] = 1u << h;
         box[3] = 1;
     } else {
@@ -1107,8 +436,8 @@ static CUresult encode_map(EncodeTiledFn enc, CUtensorMap *m, const void *ptr, i
         dims[2] = (cuuint64_t)W;
         dims[3] = (cuuint64_t)H;
         dims[4] = (cuuint64_t)B;
-        strides[2] = (cuuint64_t)W * heads * d * es;
-        strides[3] = N * heads * d * es;
+        strides[2] = (cuuint64_t)W * heads * pitch * es;
+        strides[3] = N * heads * pitch * es;
         box[2] = 1;
         box[3] = 1u << h;
         box[4] = 1;
@@ -1121,7 +450,7 @@ static CUresult encode_map(EncodeTiledFn enc, CUtensorMap *m, const void *ptr, i
 // Encoded maps of the last few (tensors, shape, direction) combinations.
 struct MapEntry {
     const void *ptr[4];
-    int B, heads, H, W, dir, dev;
+    int B, heads, H, W, dir, dev, ldk;
     unsigned used;
     bool valid;
     pp::Maps maps;
@@ -1135,7 +464,7 @@ static cudaError_t pipe_maps(const Params &prm, int dev, pp::Maps *maps, unsigne
         std::lock_guard<std::mutex> lk(g_mu);
         for (const MapEntry &m : g_maps) {
             if (m.valid && m.dev == dev && m.B == prm.B && m.heads == prm.heads && m.H == prm.H && m.W == prm.W &&
-                m.dir == prm.dir && !memcmp(m.ptr, ptr, sizeof(ptr))) {
+                m.dir == prm.dir && m.ldk == prm.ldk && !memcmp(m.ptr, ptr, sizeof(ptr))) {
                 *maps = m.maps;
                 *used = m.used;
                 return cudaSuccess;
@@ -1153,13 +482,14 @@ static cudaError_t pipe_maps(const Params &prm, int dev, pp::Maps *maps, unsigne
     ent.W = prm.W;
     ent.dir = prm.dir;
     ent.dev = dev;
+    ent.ldk = prm.ldk;
     ent.used = used_heights(prm.H, prm.W, prm.dir);
     const bool column = prm.dir == GTR_T2B || prm.dir == GTR_B2T;
     for (int ten = 0; ten < 4; ++ten)
         for (int h = 0; h < 7; ++h) {
             if (!((ent.used >> h) & 1u)) continue;
             if (encode_map(enc, &ent.maps.m[ten][h], ptr[ten], prm.B, prm.heads, prm.H, prm.W,
-                           ten == 3 ? kDV : pp::kDK, column, h) != CUDA_SUCCESS)
+                           ten == 3 ? kDV : pp::kDK, ten == 3 ? kDV : prm.ldk, column, h) != CUDA_SUCCESS)
                 return cudaErrorInvalidValue;
         }
     ent.valid = true;
@@ -1184,11 +514,33 @@ static cudaError_t launch(const Params &prm, const Plan &pl, void *workspace, cu
     }
     if (pl.kind < 0) return cudaErrorNotSupported;
     const KSpec k = spec_of(pl.kind);
-    cudaError_t e = prepare_kernel(k, is_coop(pl.kind) ? 1 : pl.cluster);
+    cudaError_t e = prepare_kernel(k);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg;
     cudaLaunchAttribute attr[2];
     fill_config(cfg, attr, k, pl.cluster, pl.clusters, stream);
+    if (prm.dk == 2 * pp::kDK) {
+        // dk = 128: the recurrence is separable by key channel (row i of the state sees
+        // only channel i of k and of the decay), and the output sums the two halves'
+        // contributions: channels 0..63 (state rows 0..63) store the output, channels
+        // 64..127 (state rows 64..127) add to it, in stream order
+        for (int half = 0; half < 2; ++half) {
+            Params ph = prm;
+            const size_t co = (size_t)half * pp::kDK;
+            ph.q = prm.q + co;
+            ph.k = prm.k + co;
+            ph.g = prm.g + co;
+            ph.ldk = prm.dk;
+            ph.dk = pp::kDK;
+            ph.sstride = prm.dk * kDV;
+            if (prm.s0 != nullptr) ph.s0 = prm.s0 + co * kDV;
+            if (prm.sf != nullptr) ph.sf = prm.sf + co * kDV;
+            ph.acc = half;
+            e = launch(ph, pl, workspace, stream, inv_tau);
+            if (e != cudaSuccess) return e;
+        }
+        return cudaSuccess;
+    }
     if (is_pipe(pl.kind)) {
         static thread_local pp::Args a;
         a = pp::Args{};
@@ -1263,6 +615,9 @@ static Params make_params(const gtr_half_t *q, const gtr_half_t *k, const gtr_ha
                           const float *init_state, gtr_half_t *out, float *final_state, int dk) {
     Params prm{};
     prm.dk = dk;
+    prm.ldk = dk;
+    prm.sstride = dk * kDV;
+    prm.acc = 0;
     prm.q = reinterpret_cast<const __half *>(q);
     prm.k = reinterpret_cast<const __half *>(k);
     prm.v = reinterpret_cast<const __half *>(v);
@@ -1316,7 +671,6 @@ extern "C" gtr_status_t gtr_gla_fwd_z(const gtr_half_t *q, const gtr_half_t *k, 
                                        out, final_state);
     if (st != GTR_OK) return st;
     if (!(tau > 0.f) || !(tau < 3.0e38f)) return GTR_ERR_INVALID_ARG;
-    if (dk != 64) return GTR_ERR_UNSUPPORTED;
     if ((long long)Hgrid * Wgrid == 0)   // no token: the state copy of the plain call
         return gtr_gla_fwd(q, k, v, z, B, heads, Hgrid, Wgrid, dk, dv, direction, chunk, init_state, out,
                            final_state, stream);

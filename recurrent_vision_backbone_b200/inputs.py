@@ -97,7 +97,7 @@ def workload(name_or_index) -> Workload:
 
 def make_inputs(B: int, heads: int, H: int, W: int, dk: int, dv: int, seed: int,
                 init_std: Optional[float] = None, z_mean_per_head=None,
-                device="cpu", z_override=None):
+                device="cpu", z_override=None, with_z=False):
     """Draw one call's inputs following the module recipe.
 
     Returns dict(q, k, v, g: fp16 tensors [B,N,heads,d]; s0: fp32 [B,heads,dk,dv]
@@ -105,6 +105,8 @@ def make_inputs(B: int, heads: int, H: int, W: int, dk: int, dv: int, seed: int,
     that CPU and GPU consumers see bit-identical values).
     ``z_override`` (optional callable shape -> fp32 tensor) replaces the gate
     pre-activation draw, for edge cases such as all-retain or all-forget gates.
+    ``with_z`` also returns the pre-activation itself (fp16, "z"), for the entry point
+    that forms g from it.
     """
     N = H * W
     gen = torch.Generator(device=device)
@@ -122,7 +124,10 @@ def make_inputs(B: int, heads: int, H: int, W: int, dk: int, dv: int, seed: int,
     if z_override is not None:
         z = z_override((B, N, heads, dk)).to(device=device, dtype=torch.float32)
     g = F.logsigmoid(z) / TAU
-    return dict(q=q.half(), k=k.half(), v=v.half(), g=g.half(), s0=s0)
+    out = dict(q=q.half(), k=k.half(), v=v.half(), g=g.half(), s0=s0)
+    if with_z:
+        out["z"] = z.half()
+    return out
 
 
 def workload_inputs(w: Workload, direction: int, call: int = 0, device="cpu"):

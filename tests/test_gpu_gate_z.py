@@ -68,7 +68,7 @@ def test_temperatures_and_extreme_pre_activations(monkeypatch, tau, zscale, zshi
         assert_parity(sf, rs, f"tau {tau} z*{zscale}+{zshift} dir {d} final state")
 
 
-def test_bad_temperature_and_dk_are_rejected():
+def test_bad_temperature_is_rejected():
     dev = torch.device("cuda", 0)
     inp = _z_inputs(1, 1, 4, 4, seed=1)
     t = {n: inp[n].to(dev) for n in ("q", "k", "v", "z")}
@@ -76,8 +76,16 @@ def test_bad_temperature_and_dk_are_rejected():
         with pytest.raises(gla.GTRError) as e:
             gla.gtr_gla_fwd_z(t["q"], t["k"], t["v"], t["z"], tau, 4, 4, 0)
         assert e.value.status == gla.GTR_ERR_INVALID_ARG
-    q2 = torch.zeros((1, 16, 1, 128), dtype=torch.float16, device=dev)
-    with pytest.raises(gla.GTRError) as e:
-        gla.gtr_gla_fwd_z(q2, q2, t["v"], q2, 16.0, 4, 4, 0)
-    assert e.value.status == gla.GTR_ERR_UNSUPPORTED
     assert gla.device_status() == gla.GTR_OK
+
+
+@pytest.mark.parametrize("direction", [0, 1, 2, 3])
+def test_dk128_with_fused_gate(direction):
+    """dk = 128 (two 64-channel halves, the second adding to the first's output)."""
+    B, heads, H, W = 2, 3, 19, 23
+    inp = make_inputs(B, heads, H, W, 128, 64, seed=901 + direction, init_std=0.3)
+    gen = torch.Generator().manual_seed(902 + direction)
+    inp["z"] = (torch.randn((B, H * W, heads, 128), generator=gen) * 2.0).half()
+    out, sf, ro, rs = _run(inp, 8.0, H, W, direction)
+    assert_parity(out, ro, "dk128 out")
+    assert_parity(sf, rs, "dk128 final state")
