@@ -148,3 +148,68 @@ def gla_forward_z(q, k, v, z, tau: float, H: int, W: int, direction: int, s0=Non
     """The forward pass with the gate given by its pre-activation z (fp64 gate, then
     the same recurrence as gla_forward)."""
     return gla_forward(q, k, v, gate(z, tau), H, W, direction, s0)
+
+
+# ------------------------------------------------------------------ Spatial SwiGLU
+# The gated value branch of GTR's Spatial SwiGLU (``swiglu_oracle.c``; the GTR news
+# article, section "单向扫描的致命缺陷，以及GTR怎么补").  Its own shared library, built
+# the same way.
+_SW_SRC = os.path.join(_HERE, "swiglu_oracle.c")
+_SW_LIB = os.path.join(_HERE, "libswiglu_oracle.so")
+_sw_lib = None
+
+
+def build_swiglu(force: bool = False) -> str:
+    with _lock:
+        stale = (not os.path.exists(_SW_LIB)
+                 or os.path.getmtime(_SW_LIB) < os.path.getmtime(_SW_SRC))
+        if force or stale:
+            compile_oracle(_SW_SRC, _SW_LIB)
+    return _SW_LIB
+
+
+def load_swiglu_library(path: str) -> ctypes.CDLL:
+    lib = ctypes.CDLL(path)
+    dp = ctypes.POINTER(ctypes.c_double)
+    lib.swiglu_oracle_gate_conv.restype = ctypes.c_int
+    lib.swiglu_oracle_gate_conv.argtypes = [dp, dp, dp, dp] + [ctypes.c_long] * 4 + [dp]
+    lib.swiglu_oracle_silu.argtypes = [dp, ctypes.c_long, dp]
+    return lib
+
+
+def _sw():
+    global _sw_lib
+    if _sw_lib is None:
+        _sw_lib = load_swiglu_library(build_swiglu())
+    return _sw_lib
+
+
+def silu(x, lib=None) -> np.ndarray:
+    """x * sigmoid(x) in fp64, elementwise."""
+    lib = lib or _sw()
+    xa = _f64(x)
+    y = np.empty_like(xa)
+    lib.swiglu_oracle_silu(_ptr(xa), xa.size, _ptr(y))
+    return y
+
+
+def spatial_swiglu_gate(G, U, w, bias=None, lib=None) -> np.ndarray:
+    """h = silu(G) * (bias + 3x3 depthwise cross-correlation of U, zero padding).
+
+    G, U: [B, H, W, C]; w: [C, 3, 3]; bias: [C] or None.  Returns h [B, H, W, C] fp64.
+    """
+    lib = lib or _sw()
+    Ga, Ua, wa = _f64(G), _f64(U), _f64(w)
+    if Ga.shape != Ua.shape or Ga.ndim != 4:
+        raise ValueError("G and U must be [B, H, W, C] of one shape")
+    B, H, W, C = Ga.shape
+    if wa.shape != (C, 3, 3):
+        raise ValueError("w must be [C, 3, 3]")
+    ba = None if bias is None else _f64(bias)
+    if ba is not None and ba.shape != (C,):
+        raise ValueError("bias must be [C]")
+    h = np.zeros_like(Ga)
+    rc = lib.swiglu_oracle_gate_conv(_ptr(Ga), _ptr(Ua), _ptr(wa), _ptr(ba), B, H, W, C, _ptr(h))
+    if rc != 0:
+        raise RuntimeError(f"swiglu_oracle_gate_conv failed with code {rc}")
+    return h
