@@ -103,23 +103,31 @@ def _code_tokens(src: str) -> str:
     return " ".join("".join(out).split())
 
 
-def kernel_source_hash() -> str:
-    """Hash of the kernel sources' code (comments and layout excluded), recorded next
-    to the ncu counters in profiles/ so that a stale capture is not reported."""
+KERNEL_FILES = {"gla_fwd_span_kernel": "gla_fwd_span.cuh", "gla_fwd_pipe_kernel": "gla_fwd_pipe.cuh",
+                "swiglu_gate_kernel": "swiglu_gate.cuh"}
+
+
+def kernel_source_hash(kernel: str) -> str:
+    """Hash of the code a kernel is built from (comments and layout excluded): its own
+    file, the PTX wrappers and the shared device part of gtr_gla.cu (up to its host
+    section), recorded next to the ncu counters in profiles/ so that a stale capture
+    is not reported."""
     h = hashlib.sha1()
     csrc = os.path.join(ROOT, "recurrent_vision_backbone_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), encoding="utf-8") as fh:
-                h.update(_code_tokens(fh.read()).encode())
+    for name in (KERNEL_FILES[kernel], "sm100_ptx.cuh", "gtr_gla.cu"):
+        with open(os.path.join(csrc, name), encoding="utf-8") as fh:
+            text = fh.read()
+        if name == "gtr_gla.cu":
+            text = text[:text.index("// ------------------------------------------------------------------ host")]
+        h.update(_code_tokens(text).encode())
     return h.hexdigest()[:12]
 
 
 def kernel_for(w, gate_z=False) -> str:
-    """The kernel a call of workload w launches."""
-    if w.dk != 64 or gate_z:
+    """The kernel a call of workload w launches (a dk = 128 call: twice)."""
+    if gate_z or os.environ.get("GTR_KERNEL") == "pipe":
         return "gla_fwd_pipe_kernel"
-    return "gla_fwd_pipe_kernel" if os.environ.get("GTR_KERNEL") == "pipe" else "gla_fwd_span_kernel"
+    return "gla_fwd_span_kernel"
 
 
 def launches_per_call(w) -> int:
@@ -138,8 +146,8 @@ def recorded_traffic(workload_name: str):
     except OSError:
         return None
     m_sha = re.search(r"kernel_source_sha1:\s*([0-9a-f]+)", text)
-    m_tr = re.search(r"traffic_bytes_per_launch:\s*([0-9]+)", text)
-    if not m_sha or not m_tr or m_sha.group(1) != kernel_source_hash():
+    m_tr = re.search(r"traffic_bytes_per_call:\s*([0-9]+)", text)
+    if not m_sha or not m_tr or m_sha.group(1) != kernel_source_hash(kernel):
         return None
     return int(m_tr.group(1))
 
@@ -360,6 +368,79 @@ def roofline(w, ms_per_call, workload_name, gate_z=False):
             "launches_per_call": launches_per_call(w)}
 
 
+# ------------------------------------------------------------------ Spatial SwiGLU
+def swiglu_bytes_alg(w) -> int:
+    """Read U and G, write h (fp16), plus the fp32 kernel and bias."""
+    return 6 * w.B * w.N * w.C + 40 * w.C
+
+
+class SwigluBench:
+    """Rotating device-resident input sets of one Spatial SwiGLU workload, one
+    gtr_spatial_swiglu_gate call per step, replayed from CUDA graphs (the interface
+    of Workload, for measure())."""
+
+    def __init__(self, w, device, n_sets=None):
+        from recurrent_vision_backbone_b200 import gla
+        from recurrent_vision_backbone_b200.inputs import make_swiglu_inputs
+        self.gla = gla
+        self.w = w
+        if n_sets is None:
+            n_sets = max(4, -(-4 * L2_BYTES // swiglu_bytes_alg(w)))
+        self.n_sets = int(n_sets)
+        self.sets = []
+        for s in range(self.n_sets):
+            inp = make_swiglu_inputs(w.B, w.H, w.W, w.C, seed=5000 + s, device=device)
+            self.sets.append((inp, torch.empty_like(inp["G"])))
+
+    def launch_step(self, s, stream):
+        inp, out = self.sets[s % self.n_sets]
+        self.gla.gtr_spatial_swiglu_gate(inp["G"], inp["U"], inp["w"], inp["bias"], out=out, stream=stream)
+
+    capture = Workload.capture
+    _graph_of = Workload._graph_of
+    _part = Workload._part
+    replay = Workload.replay
+
+    def calls_per_step(self):
+        return 1
+
+
+def run_swiglu(name, steps, warmup, stream, world, device, sets, local):
+    from recurrent_vision_backbone_b200.inputs import SWIGLU_WORKLOADS
+    w = SWIGLU_WORKLOADS[name]
+    sb = SwigluBench(w, device, n_sets=sets)
+    clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else local)
+    ms, n_steps, clk = measure(sb, steps, warmup, stream, world, clocks)
+    peak, which = measured_peaks()
+    b = swiglu_bytes_alg(w)
+    achieved = b / (ms / n_steps * 1e-3) / 1e9
+    res = {"workload": name, "tokens_per_call": w.B * w.N, "channels": w.C,
+           "value": round(world * w.B * w.N * n_steps / (ms * 1e-3), 1), "unit": "tokens/s",
+           "steps": n_steps, "us_per_call": round(ms * 1e3 / n_steps, 3),
+           "roofline": {"kernel": "swiglu_gate_kernel", "bound": "hbm", "achieved": round(achieved, 1),
+                        "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                        "traffic": recorded_traffic_swiglu(name), "peak_source": which,
+                        "bytes_alg_per_call": b, "launches_per_call": 1},
+           "gpu_launches": n_steps, "clocks": clk,
+           "l2": f"inputs rotate over {sb.n_sets} sets ({sb.n_sets * b / 2**20:.0f} MiB > 3x L2)"}
+    del sb
+    torch.cuda.empty_cache()
+    return res
+
+
+def recorded_traffic_swiglu(name: str):
+    path = os.path.join(ROOT, "profiles", f"swiglu_gate_kernel_{name}.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m_sha = re.search(r"kernel_source_sha1:\s*([0-9a-f]+)", text)
+    m_tr = re.search(r"traffic_bytes_per_call:\s*([0-9]+)", text)
+    if not m_sha or not m_tr or m_sha.group(1) != kernel_source_hash("swiglu_gate_kernel"):
+        return None
+    return int(m_tr.group(1))
+
+
 def call_inputs(w, d, seed, heads=None, device="cpu"):
     """Inputs of one call of workload w (optionally only its first `heads` heads)."""
     h = w.heads if heads is None else heads
@@ -442,9 +523,10 @@ def e2e_measure(w, steps, device, rank):
     return ms, steps, h2d, d2h
 
 
-def config_of(w, world, l2_note, timing):
+def config_of(w, world, l2_note, timing, gate_z=False):
     """The line's `config` (the same keys in both arms)."""
-    return {"workload": w.name, "B": w.B, "heads": w.heads, "grid": [w.H, w.W],
+    return {"workload": w.name, "entry": "gtr_gla_fwd_z" if gate_z else "gtr_gla_fwd",
+            "B": w.B, "heads": w.heads, "grid": [w.H, w.W],
             "tokens_per_call": w.B * w.N, "dk": w.dk, "dv": w.dv, "chunk": 64,
             "calls_per_step": len(w.call_directions()),
             "directions": ",".join(DIR_NAMES[d] for d in w.call_directions()),
@@ -476,7 +558,7 @@ def run_workload(name, steps, warmup, stream, world, rank, device, sets, sample_
           f"({wl.n_sets * wl.calls_per_step() * bytes_alg(w) / 2**20:.0f} MiB > 3x L2)")
     cfg = config_of(w, world, l2, "CUDA graph replay (exactly `steps` steps), CUDA events, "
                                   "max over ranks; clocks sampled over >= 1 s of the same "
-                                  "replays ending with the timed region")
+                                  "replays ending with the timed region", gate_z)
     del wl
     torch.cuda.empty_cache()
     return res, cfg
@@ -504,7 +586,7 @@ def gpu_arm(args):
     primary = args.workload
     w1 = WORKLOADS[primary]
     res, cfg = run_workload(primary, args.steps, args.warmup, stream, world, rank, device,
-                            args.sets, True, local, args.clocks_csv)
+                            args.sets, True, local, args.clocks_csv, gate_z=args.gate_z)
     line = {
         "metric": METRIC, "value": res["value"], "unit": "tokens/s", "n_gpus": world,
         "steps": res["steps"], "warmup": args.warmup, "ms_per_step": res["ms_per_step"],
@@ -521,6 +603,10 @@ def gpu_arm(args):
             r2, _ = run_workload(name, max(8, args.steps // 16), max(3, args.warmup // 16), stream,
                                  world, rank, device, args.sets, True, local, gate_z=gz)
             line["secondary"].append(r2)
+        from recurrent_vision_backbone_b200.inputs import SWIGLU_WORKLOADS
+        for name in SWIGLU_WORKLOADS:   # the Spatial SwiGLU gated value branch
+            line["secondary"].append(run_swiglu(name, max(8, args.steps // 16), max(3, args.warmup // 16),
+                                                stream, world, device, None, local))
     # end to end through the public call with host buffers
     e_steps = max(3, min(args.steps, args.e2e_steps))
     ems, en, h2d, d2h = e2e_measure(w1, e_steps, device, rank)
@@ -628,6 +714,9 @@ def main():
                     help="rotating input sets (default: enough to exceed 4x L2); small "
                          "profiler captures use fewer")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--gate-z", action="store_true",
+                    help="time the headline workload through gtr_gla_fwd_z (the gate's "
+                         "pre-activation in place of g) instead of gtr_gla_fwd")
     ap.add_argument("--clocks-csv", default=None,
                     help="keep the raw nvidia-smi clock samples of the timed region in this CSV")
     args = ap.parse_args()

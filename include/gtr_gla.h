@@ -242,10 +242,11 @@ const char *gtr_status_str(gtr_status_t status);
 
 /*
  * Launch plan the library would use for a shape on the current device:
- * writes the number of CTAs cooperating on one sequence (spans, or the size of
- * a thread-block cluster), the number of such CTA groups in the grid and the
- * dynamic shared memory per CTA.  Host-only query; returns
- * GTR_ERR_* like gtr_gla_fwd's argument checks.
+ * writes the number of CTAs cooperating on one sequence (the spans it is cut
+ * into, in `cluster_size`), the number of such CTA groups in the grid and the
+ * dynamic shared memory per CTA (a dk = 128 call runs this plan twice, once per
+ * 64-channel key half).  Host-only query; returns GTR_ERR_* like gtr_gla_fwd's
+ * argument checks.
  */
 gtr_status_t gtr_gla_plan(int B, int heads, int Hgrid, int Wgrid, int dk, int dv,
                           int *cluster_size, int *num_clusters, int *smem_bytes);

@@ -35,6 +35,7 @@
 #include <mutex>
 
 #include "../../include/gtr_gla.h"
+#include "../../include/gtr_swiglu.h"
 #include "sm100_ptx.cuh"
 
 namespace gtr {
@@ -128,6 +129,7 @@ __device__ __forceinline__ void tmem_ld_16x256b_x4(uint32_t taddr, uint32_t (&r)
 
 #include "gla_fwd_span.cuh"
 #include "gla_fwd_pipe.cuh"
+#include "swiglu_gate.cuh"
 
 namespace gtr {
 
@@ -978,4 +980,121 @@ extern "C" const char *gtr_gla_version(void) { return "0.3.0"; }
 
 extern "C" const char *gtr_gla_last_error(void) {
     return g_last_cuda_error == cudaSuccess ? "no error" : cudaGetErrorString(g_last_cuda_error);
+}
+
+// ------------------------------------------------------------------ Spatial SwiGLU
+namespace gtr {
+
+// One activation tensor ([B, H, W, C] fp16, channels contiguous) as (C, W, H, B),
+// box 64 channels x box_w x box_h x 1.
+static CUresult encode_act_map(EncodeTiledFn enc, CUtensorMap *m, const void *ptr, int B, int H, int W, int C,
+                               int box_w, int box_h) {
+    const cuuint64_t es = 2;
+    const cuuint64_t dims[4] = {(cuuint64_t)C, (cuuint64_t)W, (cuuint64_t)H, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)C * es, (cuuint64_t)W * C * es, (cuuint64_t)H * W * C * es};
+    const cuuint32_t box[4] = {(cuuint32_t)sw::kTC, (cuuint32_t)box_w, (cuuint32_t)box_h, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, const_cast<void *>(ptr), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+struct SwMapEntry {
+    const void *g, *u, *h;
+    int B, H, W, C, dev;
+    bool valid;
+    CUtensorMap mu, mg, mh;
+};
+static SwMapEntry g_swmaps[16];
+static int g_swmaps_next;
+
+static cudaError_t swiglu_maps(const void *G, const void *U, const void *h, int B, int H, int W, int C, int dev,
+                               sw::Args *a) {
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        for (const SwMapEntry &e : g_swmaps)
+            if (e.valid && e.g == G && e.u == U && e.h == h && e.B == B && e.H == H && e.W == W && e.C == C &&
+                e.dev == dev) {
+                a->mu = e.mu;
+                a->mg = e.mg;
+                a->mh = e.mh;
+                return cudaSuccess;
+            }
+    }
+    EncodeTiledFn enc = nullptr;
+    const cudaError_t e = tensor_map_encoder(&enc);
+    if (e != cudaSuccess) return e;
+    SwMapEntry ent{};
+    ent.g = G;
+    ent.u = U;
+    ent.h = h;
+    ent.B = B;
+    ent.H = H;
+    ent.W = W;
+    ent.C = C;
+    ent.dev = dev;
+    if (encode_act_map(enc, &ent.mu, U, B, H, W, C, sw::kTX + 2, sw::kTY + 2) != CUDA_SUCCESS ||
+        encode_act_map(enc, &ent.mg, G, B, H, W, C, sw::kTX, sw::kTY) != CUDA_SUCCESS ||
+        encode_act_map(enc, &ent.mh, h, B, H, W, C, sw::kTX, sw::kTY) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    ent.valid = true;
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_swmaps[g_swmaps_next] = ent;
+    g_swmaps_next = (g_swmaps_next + 1) % (int)(sizeof(g_swmaps) / sizeof(g_swmaps[0]));
+    a->mu = ent.mu;
+    a->mg = ent.mg;
+    a->mh = ent.mh;
+    return cudaSuccess;
+}
+
+}  // namespace gtr
+
+extern "C" gtr_status_t gtr_spatial_swiglu_gate(const gtr_half_t *G, const gtr_half_t *U, const float *w,
+                                                const float *bias, int B, int H, int W, int C, gtr_half_t *out,
+                                                void *stream) {
+    if (B < 0 || H < 0 || W < 0 || C < 0) return GTR_ERR_INVALID_ARG;
+    const long long n = (long long)B * H * W * C;
+    if (n == 0) return GTR_OK;   // nothing to read or write
+    if (!G || !U || !w || !out) return GTR_ERR_INVALID_ARG;
+    if (C % 8 != 0) return GTR_ERR_UNSUPPORTED;   // rows of 16-byte multiples (TMA strides)
+    if (!aligned16(G) || !aligned16(U) || !aligned16(out) || (reinterpret_cast<uintptr_t>(w) & 3u) ||
+        (bias && (reinterpret_cast<uintptr_t>(bias) & 3u)))
+        return GTR_ERR_INVALID_ARG;
+    if (n > 0x7fffffffLL * 8) return GTR_ERR_INVALID_ARG;
+    {   // out may be G itself (each element is read and written by one thread), never U
+        const uintptr_t o = reinterpret_cast<uintptr_t>(out), u = reinterpret_cast<uintptr_t>(U);
+        const uintptr_t g = reinterpret_cast<uintptr_t>(G), nb = (uintptr_t)n * 2;
+        if (o < u + nb && u < o + nb) return GTR_ERR_INVALID_ARG;
+        if (o != g && o < g + nb && g < o + nb) return GTR_ERR_INVALID_ARG;
+    }
+    const int dev = current_device();
+    sw::Args a{};
+    const gtr_status_t ms = cuda_status(swiglu_maps(G, U, out, B, H, W, C, dev, &a));
+    if (ms != GTR_OK) return ms;
+    a.w = w;
+    a.bias = bias;
+    a.B = B;
+    a.H = H;
+    a.W = W;
+    a.C = C;
+    a.tiles_x = (W + sw::kTX - 1) / sw::kTX;
+    a.tiles_y = (H + sw::kTY - 1) / sw::kTY;
+    a.tiles_c = (C + sw::kTC - 1) / sw::kTC;
+    const long long tiles = (long long)B * a.tiles_y * a.tiles_x * a.tiles_c;
+    if (tiles > 0x7fffffffLL) return GTR_ERR_INVALID_ARG;
+    const void *fn = reinterpret_cast<const void *>(&sw::swiglu_gate_kernel);
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, sw::L::alloc);
+    if (e != cudaSuccess) return cuda_status(e);
+    cudaLaunchConfig_t cfg{};
+    cudaLaunchAttribute attr[1];
+    cfg.gridDim = dim3((unsigned)tiles, 1, 1);
+    cfg.blockDim = dim3(sw::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = sw::L::alloc;
+    cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // set-up overlaps the call ahead
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    void *args[] = {&a};
+    return cuda_status(cudaLaunchKernelExC(&cfg, fn, args));
 }

@@ -23,7 +23,7 @@ STATIC_WS_BYTES = 4 << 20   # GTR_STATIC_WS_BYTES
 
 EXPORTED_SYMBOLS = ("gtr_gla_fwd", "gtr_gla_fwd_z", "gtr_gla_fwd_stack", "gtr_gla_init", "gtr_gla_workspace_bytes", "gtr_gla_fwd_ws",
                     "gtr_gla_fwd_static", "gtr_gla_device_status", "gtr_status_str", "gtr_gla_plan", "gtr_gla_version",
-                    "gtr_gla_last_error", "gtr_gla_selftest_timeout")
+                    "gtr_gla_last_error", "gtr_gla_selftest_timeout", "gtr_spatial_swiglu_gate")
 
 _lock = threading.Lock()
 _lib = None
@@ -60,6 +60,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.gtr_gla_fwd.argtypes = [vp, vp, vp, vp] + [i] * 8 + [vp, vp, vp, vp]
         lib.gtr_gla_fwd_z.restype = i
         lib.gtr_gla_fwd_z.argtypes = [vp, vp, vp, vp, ctypes.c_float] + [i] * 8 + [vp, vp, vp, vp]
+        lib.gtr_spatial_swiglu_gate.restype = i
+        lib.gtr_spatial_swiglu_gate.argtypes = [vp, vp, vp, vp] + [i] * 4 + [vp, vp]
         lib.gtr_gla_fwd_stack.restype = i
         lib.gtr_gla_fwd_stack.argtypes = [ctypes.POINTER(Layer)] + [i] * 8 + [vp]
         lib.gtr_gla_fwd_static.restype = i
@@ -163,6 +165,31 @@ def gtr_gla_fwd_z(q, k, v, z, tau: float, Hgrid: int, Wgrid: int, direction: int
     if st != GTR_OK:
         raise GTRError(st, "gtr_gla_fwd_z")
     return out, final_state
+
+
+def gtr_spatial_swiglu_gate(G, U, w, bias=None, out=None, stream=None):
+    """Gated value branch of Spatial SwiGLU: silu(G) * (bias + 3x3 depthwise
+    cross-correlation of U, zero padding).  G, U: fp16 [B, H, W, C] on the GPU;
+    w: fp32 [C, 3, 3]; bias: fp32 [C] or None.  Returns out (fp16, like G)."""
+    import torch
+    if G.shape != U.shape or G.dim() != 4:
+        raise ValueError("G and U must be [B, H, W, C] of one shape")
+    B, H, W, C = G.shape
+    for name, t in (("G", G), ("U", U)):
+        if t.dtype != torch.float16 or not t.is_contiguous() or not t.is_cuda:
+            raise ValueError(f"{name} must be a contiguous fp16 CUDA tensor")
+    if tuple(w.shape) != (C, 3, 3) or w.dtype != torch.float32 or not w.is_contiguous() or w.device != G.device:
+        raise ValueError("w must be a contiguous fp32 [C, 3, 3] tensor on G's device")
+    if bias is not None and (tuple(bias.shape) != (C,) or bias.dtype != torch.float32 or
+                             not bias.is_contiguous() or bias.device != G.device):
+        raise ValueError("bias must be a contiguous fp32 [C] tensor on G's device")
+    if out is None:
+        out = torch.empty_like(G)
+    st = load().gtr_spatial_swiglu_gate(_ptr(G), _ptr(U), _ptr(w), _ptr(bias), B, H, W, C, _ptr(out),
+                                        _stream_handle(stream))
+    if st != GTR_OK:
+        raise GTRError(st, "gtr_spatial_swiglu_gate")
+    return out
 
 
 def gtr_gla_fwd_stack(layers, Hgrid: int, Wgrid: int, chunk: int = 64, stream=None):

@@ -134,3 +134,42 @@ def workload_inputs(w: Workload, direction: int, call: int = 0, device="cpu"):
     return make_inputs(w.B, w.heads, w.H, w.W, w.dk, w.dv, w.seed(direction, call),
                        init_std=w.init_std, z_mean_per_head=w.z_mean_per_head,
                        device=device)
+
+
+# ------------------------------------------------------------------ Spatial SwiGLU
+# Inputs of the gated value branch (gtr_spatial_swiglu_gate): the gate and up
+# projections G, U of a block's tokens and the depthwise kernel.  The pages give no
+# block width; the recipe reads the token mixer's 16 heads x 64 channels = 1024 as the
+# block width and a hidden width of 2x that, 2048 (the SwiGLU's two projections).
+# G, U ~ N(0, 1) cast to fp16; w ~ N(0, 1/9) (a 3x3 kernel's fan-in) and bias ~
+# N(0, 0.1^2) in fp32.  The grids are the token mixer's: 40x40 (1.6K tokens) and the
+# 768px batch, B8 48x48.
+@dataclasses.dataclass(frozen=True)
+class SwigluWorkload:
+    name: str
+    B: int
+    H: int
+    W: int
+    C: int
+
+    @property
+    def N(self):
+        return self.H * self.W
+
+
+SWIGLU_WORKLOADS = {w.name: w for w in (
+    SwigluWorkload("swiglu_b1_40x40_c2048", 1, 40, 40, 2048),
+    SwigluWorkload("swiglu_b8_48x48_c2048", 8, 48, 48, 2048),
+)}
+
+
+def make_swiglu_inputs(B: int, H: int, W: int, C: int, seed: int, bias: bool = True, device="cpu"):
+    """Draw G, U (fp16 [B, H, W, C]), w (fp32 [C, 3, 3]) and bias (fp32 [C] or None)."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(int(seed))
+    kw = dict(generator=gen, device=device, dtype=torch.float32)
+    G = torch.randn((B, H, W, C), **kw)
+    U = torch.randn((B, H, W, C), **kw)
+    w = torch.randn((C, 3, 3), **kw) / 3.0
+    b = torch.randn((C,), **kw) * 0.1 if bias else None
+    return dict(G=G.half(), U=U.half(), w=w, bias=b)

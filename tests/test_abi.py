@@ -12,12 +12,15 @@ import pytest
 from recurrent_vision_backbone_b200 import build, gla
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "gtr_gla.h")
+HEADERS = [os.path.join(ROOT, "include", n) for n in sorted(os.listdir(os.path.join(ROOT, "include")))
+           if n.endswith(".h")]
 
 
 def declared_functions():
-    text = open(HEADER).read()
-    return sorted(set(re.findall(r"\b(gtr_[a-z_]+)\s*\(", text)))
+    names = set()
+    for h in HEADERS:
+        names |= set(re.findall(r"\b(gtr_[a-z_]+)\s*\(", open(h).read()))
+    return sorted(names)
 
 
 @pytest.fixture(scope="module")

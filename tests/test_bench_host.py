@@ -14,9 +14,11 @@ def test_code_tokens_drops_comments_and_layout_only():
 
 
 def test_recorded_traffic_matches_current_source():
-    h = bench.kernel_source_hash()
-    assert len(h) == 12
-    for wl in ("gtr640_b1h16_40x40", "hires_b1h16_128x128"):
+    for k in bench.KERNEL_FILES:
+        assert len(bench.kernel_source_hash(k)) == 12
+    # the host section of gtr_gla.cu is not part of any kernel's hash
+    assert bench.kernel_source_hash("gla_fwd_span_kernel") != bench.kernel_source_hash("gla_fwd_pipe_kernel")
+    for wl in ("gtr640_b1h16_40x40", "hires_b1h16_128x128", "stress_b4h12_37x53_dk128", "gtr640_b1h16_40x40+z"):
         t = bench.recorded_traffic(wl)
         # either the summary was taken on this code (a positive byte count) or it is
         # reported as unknown; never a stale number
