@@ -88,7 +88,11 @@ typedef enum {
  *   B, heads        batch size and number of heads (>= 1).
  *   Hgrid, Wgrid    patch grid; N = Hgrid*Wgrid >= 0 (N == 0 is a no-op that
  *                   still copies init_state to final_state).
- *   dk, dv          key and value head dims: dk in {64, 128}, dv == 64.
+ *   dk, dv          key and value head dims, each 64 or 128.  128 runs as two
+ *                   64-wide halves (the recurrence is separable by key channel and
+ *                   by value column): two launches for dk = 128 (the second adds
+ *                   its output to the first's), two writing disjoint columns for
+ *                   dv = 128, four for both.
  *   direction       gtr_dir_t scan order.
  *   chunk           chunk length; 64 (the only value built).
  *   init_state      float32 [B, heads, dk, dv] or NULL for a zero state.

@@ -626,7 +626,7 @@ __device__ __forceinline__ float store_out_tile(const Params &P, const uint32_t 
             const int row = x >> 3, c8 = x & 7;
             const int ro = rows[row];
             if (ro >= 0)
-                *reinterpret_cast<uint4 *>(P.out + (size_t)ro * kDV + 8 * c8) =
+                *reinterpret_cast<uint4 *>(P.out + (size_t)ro * P.ldv + 8 * c8) =
                     *reinterpret_cast<const uint4 *>(os + sw_off(row, 8 * c8));
         }
     } else {
@@ -636,7 +636,7 @@ __device__ __forceinline__ float store_out_tile(const Params &P, const uint32_t 
         for (int i = 0; i < 4; ++i) {   // the loads first, so that their latencies overlap
             const int x = tb + 128 * i, row = x >> 3, c8 = x & 7;
             ro[i] = rows[row];
-            cur[i] = *reinterpret_cast<const uint4 *>(P.out + (size_t)(ro[i] >= 0 ? ro[i] : 0) * kDV + 8 * c8);
+            cur[i] = *reinterpret_cast<const uint4 *>(P.out + (size_t)(ro[i] >= 0 ? ro[i] : 0) * P.ldv + 8 * c8);
         }
         __half2 m2 = __float2half2_rn(0.f);
 #pragma unroll
@@ -649,7 +649,7 @@ __device__ __forceinline__ float store_out_tile(const Params &P, const uint32_t 
             v.z = hadd2_bits(cur[i].z, a.z);
             v.w = hadd2_bits(cur[i].w, a.w);
             if (ro[i] >= 0) {
-                *reinterpret_cast<uint4 *>(P.out + (size_t)ro[i] * kDV + 8 * c8) = v;
+                *reinterpret_cast<uint4 *>(P.out + (size_t)ro[i] * P.ldv + 8 * c8) = v;
                 const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                 for (int m = 0; m < 4; ++m) m2 = __hmax2_nan(m2, __habs2(*reinterpret_cast<const __half2 *>(&w4[m])));
@@ -685,7 +685,7 @@ __device__ __forceinline__ void add_out_tile(const Params &P, const uint32_t (&r
         const int x = tb + 128 * i, row = x >> 3, c8 = x & 7;
         ro[i] = rows[row];
         const int rr = ro[i] >= 0 ? ro[i] : 0;
-        cur[i] = *reinterpret_cast<const uint4 *>(P.out + (size_t)rr * kDV + 8 * c8);
+        cur[i] = *reinterpret_cast<const uint4 *>(P.out + (size_t)rr * P.ldv + 8 * c8);
         add[i] = *reinterpret_cast<const uint4 *>(os + sw_off(row, 8 * c8));
     }
     __half2 m2 = __float2half2_rn(0.f);
@@ -698,7 +698,7 @@ __device__ __forceinline__ void add_out_tile(const Params &P, const uint32_t (&r
             v.y = hadd2_bits(cur[i].y, add[i].y);
             v.z = hadd2_bits(cur[i].z, add[i].z);
             v.w = hadd2_bits(cur[i].w, add[i].w);
-            *reinterpret_cast<uint4 *>(P.out + (size_t)ro[i] * kDV + 8 * c8) = v;
+            *reinterpret_cast<uint4 *>(P.out + (size_t)ro[i] * P.ldv + 8 * c8) = v;
             const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
             for (int m = 0; m < 4; ++m) m2 = __hmax2_nan(m2, __habs2(*reinterpret_cast<const __half2 *>(&w4[m])));
@@ -919,7 +919,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_pipe_kernel(const __grid_
                 for (int e = 0; e < 32; e += 2) {
                     const int h = e >> 4, j = (e >> 2) & 3, hh = (e >> 1) & 1;
                     float2 v = make_float2(0.f, 0.f);
-                    if (s0) v = *reinterpret_cast<const float2 *>(s0 + (r0 + 8 * hh) * kDV + 32 * h + 8 * j + 2 * (lane & 3));
+                    if (s0) v = *reinterpret_cast<const float2 *>(s0 + (r0 + 8 * hh) * P.ldv + 32 * h + 8 * j + 2 * (lane & 3));
                     S[e] = v.x;
                     S[e + 1] = v.y;
                 }
@@ -1036,7 +1036,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_pipe_kernel(const __grid_
 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
                     const int h = e >> 4, j = (e >> 2) & 3, hh = (e >> 1) & 1;
-                    *reinterpret_cast<float2 *>(sf + (r0 + 8 * hh) * kDV + 32 * h + 8 * j + 2 * (lane & 3)) =
+                    *reinterpret_cast<float2 *>(sf + (r0 + 8 * hh) * P.ldv + 32 * h + 8 * j + 2 * (lane & 3)) =
                         make_float2(S[e], S[e + 1]);
                 }
             }
@@ -1138,7 +1138,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_fwd_pipe_kernel(const __grid_
                         const float Gd = hh ? G1 : G0;
                         const float4 pk = park[(e >> 2) * 128 + q4 * 32 + lane];   // S_local[4m .. 4m+3]
                         const float sx = (e & 2) ? pk.z : pk.x, sy = (e & 2) ? pk.w : pk.y;
-                        *reinterpret_cast<float2 *>(sf + (r0 + 8 * hh) * kDV + 32 * h + 8 * j + 2 * (lane & 3)) =
+                        *reinterpret_cast<float2 *>(sf + (r0 + 8 * hh) * P.ldv + 32 * h + 8 * j + 2 * (lane & 3)) =
                             make_float2(fmaf(Gd, Sin[e], sx), fmaf(Gd, Sin[e + 1], sy));
                     }
                 }

@@ -185,7 +185,7 @@ __device__ __forceinline__ void load_chunk(const Params &P, uint8_t *sm, int seq
         cp_async16(d, P.q + off, nb);
         cp_async16(d + kTile, P.k + off, nb);
         cp_async16(d + 2 * kTile, P.g + off, nb);
-        cp_async16(vo + sw_off(t, 8 * pc), P.v + rr * kDV + 8 * pc, nb);
+        cp_async16(vo + sw_off(t, 8 * pc), P.v + rr * P.ldv + 8 * pc, nb);
     }
 }
 
@@ -257,7 +257,7 @@ __device__ __forceinline__ float store_chunk_out(const Params &P, uint32_t tmem,
             const int row = x >> 3, c8 = x & 7;
             const int ro = rowb[row];
             if (ro >= 0)
-                *reinterpret_cast<uint4 *>(P.out + (size_t)ro * kDV + 8 * c8) =
+                *reinterpret_cast<uint4 *>(P.out + (size_t)ro * P.ldv + 8 * c8) =
                     *reinterpret_cast<const uint4 *>(os + sw_off(row, 8 * c8));
         }
     } else {
@@ -268,7 +268,7 @@ __device__ __forceinline__ float store_chunk_out(const Params &P, uint32_t tmem,
         for (int i = 0; i < 4; ++i) {   // the loads first, so that their latencies overlap
             const int x = tb + 128 * i, row = x >> 3, c8 = x & 7;
             const int ro = rowb[row];
-            cur[i] = *reinterpret_cast<const uint4 *>(P.out + (size_t)(ro >= 0 ? ro : 0) * kDV + 8 * c8);
+            cur[i] = *reinterpret_cast<const uint4 *>(P.out + (size_t)(ro >= 0 ? ro : 0) * P.ldv + 8 * c8);
         }
         __half2 m2 = __float2half2_rn(0.f);
 #pragma unroll
@@ -286,7 +286,7 @@ __device__ __forceinline__ float store_chunk_out(const Params &P, uint32_t tmem,
                 if (ro >= 0) m2 = __hmax2_nan(m2, __habs2(v));
             }
             if (ro >= 0)
-                *reinterpret_cast<uint4 *>(P.out + (size_t)ro * kDV + 8 * c8) = make_uint4(vw[0], vw[1], vw[2], vw[3]);
+                *reinterpret_cast<uint4 *>(P.out + (size_t)ro * P.ldv + 8 * c8) = make_uint4(vw[0], vw[1], vw[2], vw[3]);
         }
         const float ml = __low2float(m2), mh = __high2float(m2);
         mx = (ml != ml || mh != mh) ? ml + mh : fmaxf(mx, fmaxf(ml, mh));
@@ -735,7 +735,7 @@ __device__ __forceinline__ void loader_load(const Params &P, uint8_t *sm, int se
 // register pressure of the kernel body.)
 __device__ __noinline__ void load_qgo(const __half *q, const __half *g, const __half *o, int N, int H,
                                       int W, int dir, int heads, int seq, int c, uint32_t dst_q,
-                                      uint32_t dst_g, uint32_t dst_o, int nthreads, int ldk) {
+                                      uint32_t dst_g, uint32_t dst_o, int nthreads, int ldk, int ldv) {
     const int bq = seq / heads, hq = seq - bq * heads;
     const int p0 = c * kChunk;
     for (int x = (int)threadIdx.x; x < 3 * 64 * 8; x += nthreads) {
@@ -743,7 +743,7 @@ __device__ __noinline__ void load_qgo(const __half *q, const __half *g, const __
         const bool ok = p0 + t < N;
         size_t ro = 0;
         if (ok) ro = (size_t)((bq * N + scan_to_token(p0 + t, H, W, dir)) * heads + hq);
-        const __half *src = ten == 0 ? q + ro * ldk : (ten == 1 ? g + ro * ldk : o + ro * 64);
+        const __half *src = ten == 0 ? q + ro * ldk : (ten == 1 ? g + ro * ldk : o + ro * ldv);
         const uint32_t d = ten == 0 ? dst_q : (ten == 1 ? dst_g : dst_o);
         cp_async16(d + t * 128 + 16 * pc, src + 8 * pc, ok ? 16u : 0u);
     }
@@ -859,7 +859,7 @@ __device__ __forceinline__ void prefetch_span_rows(const Params &P, const Work &
     prefetch_l2(P.q + ro * P.ldk);
     prefetch_l2(P.k + ro * P.ldk);
     prefetch_l2(P.g + ro * P.ldk);
-    prefetch_l2(P.v + ro * kDV);
+    prefetch_l2(P.v + ro * P.ldv);
 }
 
 // The span's aggregate state from the fp32 state tile in shared memory to the
@@ -946,7 +946,7 @@ __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(con
                 const int i = e >> 4, c4 = e & 15;
                 float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (!later && P.s0 != nullptr)
-                    v = reinterpret_cast<const float4 *>(P.s0 + (size_t)seq * P.sstride)[e];
+                    v = *reinterpret_cast<const float4 *>(P.s0 + (size_t)seq * P.sstride + (size_t)i * P.ldv + 4 * c4);
                 *reinterpret_cast<float4 *>(sst + agg_off(i, c4)) = v;
                 // S_prev of chunk 0, the fp16 operand of its MMA 2
                 *reinterpret_cast<uint2 *>(sm + L::sop + sw_off(i, 4 * c4)) =
@@ -1179,10 +1179,10 @@ __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(con
                         const float g0 = dcum[nch * 64 + i0], g1 = dcum[nch * 64 + i1];
                         const float2 f0a = st2(i0, ca), f0b = st2(i0, cb), f1a = st2(i1, ca), f1b = st2(i1, cb);
                         float *sf = P.sf + (size_t)seq * P.sstride;
-                        *reinterpret_cast<float2 *>(sf + i0 * kDV + ca) = make_float2(fmaf(g0, s0.x, f0a.x), fmaf(g0, s0.y, f0a.y));
-                        *reinterpret_cast<float2 *>(sf + i0 * kDV + cb) = make_float2(fmaf(g0, s0.z, f0b.x), fmaf(g0, s0.w, f0b.y));
-                        *reinterpret_cast<float2 *>(sf + i1 * kDV + ca) = make_float2(fmaf(g1, s1.x, f1a.x), fmaf(g1, s1.y, f1a.y));
-                        *reinterpret_cast<float2 *>(sf + i1 * kDV + cb) = make_float2(fmaf(g1, s1.z, f1b.x), fmaf(g1, s1.w, f1b.y));
+                        *reinterpret_cast<float2 *>(sf + i0 * P.ldv + ca) = make_float2(fmaf(g0, s0.x, f0a.x), fmaf(g0, s0.y, f0a.y));
+                        *reinterpret_cast<float2 *>(sf + i0 * P.ldv + cb) = make_float2(fmaf(g0, s0.z, f0b.x), fmaf(g0, s0.w, f0b.y));
+                        *reinterpret_cast<float2 *>(sf + i1 * P.ldv + ca) = make_float2(fmaf(g1, s1.x, f1a.x), fmaf(g1, s1.y, f1a.y));
+                        *reinterpret_cast<float2 *>(sf + i1 * P.ldv + cb) = make_float2(fmaf(g1, s1.z, f1b.x), fmaf(g1, s1.w, f1b.y));
                     }
                 }
                 fence_proxy_async_cta();
@@ -1245,7 +1245,7 @@ __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(con
         if constexpr (NL == 2) if (ext) {
             const uint32_t vo = smem_u32(sm + L::vop);
             load_qgo(P.q, P.g, P.out, P.N, P.H, P.W, P.dir, P.heads, seq, c0 + kHold, vo, vo + kTile,
-                     vo + 2 * kTile, kThreads, P.ldk);
+                     vo + 2 * kTile, kThreads, P.ldk, P.ldv);
         }
         if (NL == 2 && later) {
             if (tid < kspan) {
@@ -1388,7 +1388,7 @@ __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(con
                 if constexpr (NL == 2) {
                     const uint32_t stq = smem_u32(sm + L::stg);
                     load_qgo(P.q, P.g, P.out, P.N, P.H, P.W, P.dir, P.heads, seq, c0 + ci, stq,
-                             stq + 2 * kTile, stq + 3 * kTile, kThreads, P.ldk);
+                             stq + 2 * kTile, stq + 3 * kTile, kThreads, P.ldk, P.ldv);
                     cp_async_wait_all();
                     __syncthreads();
                     rebuild_qd(sm, sm + L::stg, sm + L::stg + 2 * kTile, dcum + ci * 64, sm + L::qint);
@@ -1403,7 +1403,7 @@ __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(con
                             const bool ok = p0 + t < P.N;
                             size_t ro = 0;
                             if (ok) ro = (size_t)((bq * P.N + scan_to_token(p0 + t, P.H, P.W, P.dir)) * P.heads + hq);
-                            const __half *src = ten == 0 ? P.q + ro * P.ldk : (ten == 1 ? P.g + ro * P.ldk : P.out + ro * 64);
+                            const __half *src = ten == 0 ? P.q + ro * P.ldk : (ten == 1 ? P.g + ro * P.ldk : P.out + ro * P.ldv);
                             const int slot = ten == 0 ? 0 : (ten == 1 ? 2 : 3);
                             cp_async16(stq + slot * kTile + t * 128 + 16 * pc, src + 8 * pc, ok ? 16u : 0u);
                         }
@@ -1500,7 +1500,7 @@ __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(con
                     s.z = fmaf(di, a.z, s.z);
                     s.w = fmaf(di, a.w, s.w);
                 }
-                reinterpret_cast<float4 *>(P.sf + (size_t)seq * P.sstride)[e] = s;
+                *reinterpret_cast<float4 *>(P.sf + (size_t)seq * P.sstride + (size_t)i * P.ldv + 4 * c4) = s;
             }
         }
         __syncthreads();   // staging / state tiles are reused by the next sequence

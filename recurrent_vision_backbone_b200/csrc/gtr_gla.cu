@@ -92,6 +92,8 @@ struct Params {
     int ldk;       // elements per q / k / g row (dk, or 128 for one half of a dk = 128 call)
     int sstride;   // floats per sequence of init_state / final_state (dk * dv)
     int acc;       // 1: add to the output tile instead of storing it (second key half)
+    int ldv;       // elements per v / out row, and floats per state row (dv of the call)
+    int vsplit;    // 1: one 64-column value half of a dv = 128 call
 };
 
 __device__ __forceinline__ void set_error(unsigned e) { atomicOr(&g_error_word, e); }
@@ -452,7 +454,7 @@ static CUresult encode_map(EncodeTiledFn enc, CUtensorMap *m, const void *ptr, i
 // Encoded maps of the last few (tensors, shape, direction) combinations.
 struct MapEntry {
     const void *ptr[4];
-    int B, heads, H, W, dir, dev, ldk;
+    int B, heads, H, W, dir, dev, ldk, ldv;
     unsigned used;
     bool valid;
     pp::Maps maps;
@@ -466,7 +468,7 @@ static cudaError_t pipe_maps(const Params &prm, int dev, pp::Maps *maps, unsigne
         std::lock_guard<std::mutex> lk(g_mu);
         for (const MapEntry &m : g_maps) {
             if (m.valid && m.dev == dev && m.B == prm.B && m.heads == prm.heads && m.H == prm.H && m.W == prm.W &&
-                m.dir == prm.dir && m.ldk == prm.ldk && !memcmp(m.ptr, ptr, sizeof(ptr))) {
+                m.dir == prm.dir && m.ldk == prm.ldk && m.ldv == prm.ldv && !memcmp(m.ptr, ptr, sizeof(ptr))) {
                 *maps = m.maps;
                 *used = m.used;
                 return cudaSuccess;
@@ -485,13 +487,14 @@ static cudaError_t pipe_maps(const Params &prm, int dev, pp::Maps *maps, unsigne
     ent.dir = prm.dir;
     ent.dev = dev;
     ent.ldk = prm.ldk;
+    ent.ldv = prm.ldv;
     ent.used = used_heights(prm.H, prm.W, prm.dir);
     const bool column = prm.dir == GTR_T2B || prm.dir == GTR_B2T;
     for (int ten = 0; ten < 4; ++ten)
         for (int h = 0; h < 7; ++h) {
             if (!((ent.used >> h) & 1u)) continue;
             if (encode_map(enc, &ent.maps.m[ten][h], ptr[ten], prm.B, prm.heads, prm.H, prm.W,
-                           ten == 3 ? kDV : pp::kDK, ten == 3 ? kDV : prm.ldk, column, h) != CUDA_SUCCESS)
+                           ten == 3 ? kDV : pp::kDK, ten == 3 ? prm.ldv : prm.ldk, column, h) != CUDA_SUCCESS)
                 return cudaErrorInvalidValue;
         }
     ent.valid = true;
@@ -510,7 +513,7 @@ static cudaError_t launch(const Params &prm, const Plan &pl, void *workspace, cu
         // an empty grid: the final state is the initial one (zero without one), in the
         // order of the caller's stream
         if (prm.sf == nullptr) return cudaSuccess;
-        const size_t bytes = (size_t)prm.n_seq * prm.dk * kDV * sizeof(float);
+        const size_t bytes = (size_t)prm.n_seq * prm.sstride * sizeof(float);
         return prm.s0 != nullptr ? cudaMemcpyAsync(prm.sf, prm.s0, bytes, cudaMemcpyDeviceToDevice, stream)
                                  : cudaMemsetAsync(prm.sf, 0, bytes, stream);
     }
@@ -521,6 +524,23 @@ static cudaError_t launch(const Params &prm, const Plan &pl, void *workspace, cu
     cudaLaunchConfig_t cfg;
     cudaLaunchAttribute attr[2];
     fill_config(cfg, attr, k, pl.cluster, pl.clusters, stream);
+    if (prm.ldv == 2 * kDV && !prm.vsplit) {
+        // dv = 128: the recurrence is separable by value column too (column j of the
+        // state sees only v_j), so the two 64-column halves are independent calls that
+        // write disjoint output columns and state columns
+        for (int half = 0; half < 2; ++half) {
+            Params ph = prm;
+            const size_t co = (size_t)half * kDV;
+            ph.v = prm.v + co;
+            ph.out = prm.out + co;
+            if (prm.s0 != nullptr) ph.s0 = prm.s0 + co;
+            if (prm.sf != nullptr) ph.sf = prm.sf + co;
+            ph.vsplit = 1;
+            e = launch(ph, pl, workspace, stream, inv_tau);
+            if (e != cudaSuccess) return e;
+        }
+        return cudaSuccess;
+    }
     if (prm.dk == 2 * pp::kDK) {
         // dk = 128: the recurrence is separable by key channel (row i of the state sees
         // only channel i of k and of the decay), and the output sums the two halves'
@@ -534,9 +554,8 @@ static cudaError_t launch(const Params &prm, const Plan &pl, void *workspace, cu
             ph.g = prm.g + co;
             ph.ldk = prm.dk;
             ph.dk = pp::kDK;
-            ph.sstride = prm.dk * kDV;
-            if (prm.s0 != nullptr) ph.s0 = prm.s0 + co * kDV;
-            if (prm.sf != nullptr) ph.sf = prm.sf + co * kDV;
+            if (prm.s0 != nullptr) ph.s0 = prm.s0 + co * prm.ldv;
+            if (prm.sf != nullptr) ph.sf = prm.sf + co * prm.ldv;
             ph.acc = half;
             e = launch(ph, pl, workspace, stream, inv_tau);
             if (e != cudaSuccess) return e;
@@ -591,7 +610,7 @@ static gtr_status_t check_args(const void *q, const void *k, const void *v, cons
     if (dir < 0 || dir > 3) return GTR_ERR_INVALID_ARG;
     if (chunk <= 0) return GTR_ERR_INVALID_ARG;
     if (chunk != kChunk) return GTR_ERR_UNSUPPORTED;
-    if ((dk != 64 && dk != 128) || dv != kDV) return GTR_ERR_UNSUPPORTED;
+    if ((dk != 64 && dk != 128) || (dv != 64 && dv != 128)) return GTR_ERR_UNSUPPORTED;
     if ((!empty && (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) ||
                     !aligned16(out))) ||
         (s0 && !aligned16(s0)) || (sf && !aligned16(sf)))
@@ -614,12 +633,14 @@ static gtr_status_t check_args(const void *q, const void *k, const void *v, cons
 
 static Params make_params(const gtr_half_t *q, const gtr_half_t *k, const gtr_half_t *v,
                           const gtr_half_t *g, int B, int heads, int Hgrid, int Wgrid, int direction,
-                          const float *init_state, gtr_half_t *out, float *final_state, int dk) {
+                          const float *init_state, gtr_half_t *out, float *final_state, int dk, int dv) {
     Params prm{};
     prm.dk = dk;
     prm.ldk = dk;
-    prm.sstride = dk * kDV;
+    prm.sstride = dk * dv;
     prm.acc = 0;
+    prm.ldv = dv;
+    prm.vsplit = 0;
     prm.q = reinterpret_cast<const __half *>(q);
     prm.k = reinterpret_cast<const __half *>(k);
     prm.v = reinterpret_cast<const __half *>(v);
@@ -654,7 +675,7 @@ extern "C" gtr_status_t gtr_gla_fwd(const gtr_half_t *q, const gtr_half_t *k,
                                        chunk, init_state, out, final_state);
     if (st != GTR_OK) return st;
     const Params prm = make_params(q, k, v, g, B, heads, Hgrid, Wgrid, direction, init_state, out,
-                                   final_state, dk);
+                                   final_state, dk, dv);
     const Plan pl = make_plan(prm.n_seq, prm.n_chunks, dk, true);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     void *ws = nullptr;
@@ -676,7 +697,7 @@ extern "C" gtr_status_t gtr_gla_fwd_z(const gtr_half_t *q, const gtr_half_t *k, 
     if ((long long)Hgrid * Wgrid == 0)   // no token: the state copy of the plain call
         return gtr_gla_fwd(q, k, v, z, B, heads, Hgrid, Wgrid, dk, dv, direction, chunk, init_state, out,
                            final_state, stream);
-    const Params prm = make_params(q, k, v, z, B, heads, Hgrid, Wgrid, direction, init_state, out, final_state, dk);
+    const Params prm = make_params(q, k, v, z, B, heads, Hgrid, Wgrid, direction, init_state, out, final_state, dk, dv);
     const Plan pl = make_plan(prm.n_seq, prm.n_chunks, dk, true, ~size_t(0), true);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     void *ws = nullptr;
@@ -737,7 +758,7 @@ extern "C" gtr_status_t gtr_gla_fwd_stack(const gtr_gla_layer_t *layers, int n_l
         for (int i = 0; i < n_layers; ++i) {
             const gtr_gla_layer_t &L = layers[i];
             const Params prm = make_params(L.q, L.k, L.v, L.g, B, heads, Hgrid, Wgrid, L.direction, L.init_state,
-                                           L.out, L.final_state, dk);
+                                           L.out, L.final_state, dk, dv);
             const cudaError_t e = launch(prm, pl, ws, s);
             if (e != cudaSuccess) return e;
         }
@@ -811,7 +832,7 @@ extern "C" gtr_status_t gtr_gla_init(void *stream) {
 extern "C" size_t gtr_gla_workspace_bytes(int B, int heads, int Hgrid, int Wgrid, int dk, int dv,
                                           int chunk) {
     if (B <= 0 || heads <= 0 || Hgrid < 0 || Wgrid < 0 || chunk != kChunk) return 0;
-    if ((dk != 64 && dk != 128) || dv != kDV) return 0;
+    if ((dk != 64 && dk != 128) || (dv != 64 && dv != 128)) return 0;
     const long long N = (long long)Hgrid * Wgrid;
     if (N > 0x7fffffffLL || (long long)B * heads > 0x7fffffffLL) return 0;
     int ndev = 0;
@@ -830,7 +851,7 @@ extern "C" gtr_status_t gtr_gla_fwd_ws(const gtr_half_t *q, const gtr_half_t *k,
                                        chunk, init_state, out, final_state);
     if (st != GTR_OK) return st;
     const Params prm = make_params(q, k, v, g, B, heads, Hgrid, Wgrid, direction, init_state, out,
-                                   final_state, dk);
+                                   final_state, dk, dv);
     const Plan pl = make_plan(prm.n_seq, prm.n_chunks, dk, true);
     if (pl.ws_bytes > 0 &&
         (workspace == nullptr || workspace_bytes < pl.ws_bytes ||
@@ -880,7 +901,7 @@ extern "C" gtr_status_t gtr_gla_fwd_static(const gtr_half_t *q, const gtr_half_t
                                        chunk, init_state, out, final_state);
     if (st != GTR_OK) return st;
     const Params prm = make_params(q, k, v, g, B, heads, Hgrid, Wgrid, direction, init_state, out,
-                                   final_state, dk);
+                                   final_state, dk, dv);
     // the cheapest plan whose workspace fits the scratch (one span per sequence needs none)
     const Plan pl = make_plan(prm.n_seq, prm.n_chunks, dk, true, kStaticWsBytes);
     if (pl.ws_bytes > kStaticWsBytes) return GTR_ERR_UNSUPPORTED;
@@ -964,7 +985,7 @@ extern "C" const char *gtr_status_str(gtr_status_t s) {
 extern "C" gtr_status_t gtr_gla_plan(int B, int heads, int Hgrid, int Wgrid, int dk, int dv,
                                      int *cluster_size, int *num_clusters, int *smem_bytes) {
     if (B <= 0 || heads <= 0 || Hgrid < 0 || Wgrid < 0) return GTR_ERR_INVALID_ARG;
-    if ((dk != 64 && dk != 128) || dv != kDV) return GTR_ERR_UNSUPPORTED;
+    if ((dk != 64 && dk != 128) || (dv != 64 && dv != 128)) return GTR_ERR_UNSUPPORTED;
     const long long N = (long long)Hgrid * Wgrid;
     int ndev = 0;
     const bool gpu = cudaGetDeviceCount(&ndev) == cudaSuccess && ndev > 0;
@@ -1082,14 +1103,23 @@ extern "C" gtr_status_t gtr_spatial_swiglu_gate(const gtr_half_t *G, const gtr_h
     a.tiles_c = (C + sw::kTC - 1) / sw::kTC;
     const long long tiles = (long long)B * a.tiles_y * a.tiles_x * a.tiles_c;
     if (tiles > 0x7fffffffLL) return GTR_ERR_INVALID_ARG;
-    const void *fn = reinterpret_cast<const void *>(&sw::swiglu_gate_kernel);
-    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, sw::L::alloc);
+    a.tiles = (int)tiles;
+    // one tile per CTA with one stage (two CTAs per SM: measured faster), or persistent
+    // CTAs with two stages (one per SM) with GTR_SWIGLU=persistent (tuning knob)
+    const char *mode = getenv("GTR_SWIGLU");
+    const bool persistent = mode && !strcmp(mode, "persistent");
+    const int sms = num_sms(dev);
+    const long long ctas = persistent ? (tiles < sms ? tiles : sms) : tiles;
+    const void *fn = persistent ? reinterpret_cast<const void *>(&sw::swiglu_gate_kernel<2>)
+                                : reinterpret_cast<const void *>(&sw::swiglu_gate_kernel<1>);
+    const int smem = persistent ? sw::L<2>::alloc : sw::L<1>::alloc;
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return cuda_status(e);
     cudaLaunchConfig_t cfg{};
     cudaLaunchAttribute attr[1];
-    cfg.gridDim = dim3((unsigned)tiles, 1, 1);
+    cfg.gridDim = dim3((unsigned)ctas, 1, 1);
     cfg.blockDim = dim3(sw::kThreads, 1, 1);
-    cfg.dynamicSmemBytes = sw::L::alloc;
+    cfg.dynamicSmemBytes = (size_t)smem;
     cfg.stream = reinterpret_cast<cudaStream_t>(stream);
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // set-up overlaps the call ahead
     attr[0].val.programmaticStreamSerializationAllowed = 1;

@@ -33,7 +33,7 @@ def call(lib, entry="gtr_gla_fwd", q=1, k=2, v=3, g=4, out=5, B=1, heads=2, H=8,
     (dict(B=0), "invalid"), (dict(heads=-1), "invalid"), (dict(H=-1), "invalid"),
     (dict(dk=0), "invalid"), (dict(q=None), "invalid"), (dict(out=None), "invalid"),
     (dict(direction=4), "invalid"), (dict(direction=-1), "invalid"), (dict(chunk=0), "invalid"),
-    (dict(chunk=32), "unsupported"), (dict(dk=96), "unsupported"), (dict(dv=128), "unsupported"),
+    (dict(chunk=32), "unsupported"), (dict(dk=96), "unsupported"), (dict(dv=96), "unsupported"),
     (dict(q=1 * MB + 8), "invalid"),                 # misaligned input
     (dict(s0=7 * MB + 4), "invalid"),                # misaligned initial state
     (dict(out=1 * MB + 64), "invalid"),              # output overlaps q

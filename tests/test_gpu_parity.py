@@ -60,6 +60,38 @@ def test_edge_shapes(B, heads, H, W, dk, init, direction):
     assert_parity(sf, rs, "final state")
 
 
+DV128 = [
+    # B, heads, H, W, dk, init
+    (1, 3, 9, 15, 64, True),      # dv = 128: two value-column halves
+    (2, 1, 13, 11, 128, True),    # dk = dv = 128: four launches
+    (1, 2, 40, 40, 64, False),    # 25 chunks: spans, look-back and corrections per half
+]
+
+
+@pytest.mark.parametrize("B,heads,H,W,dk,init", DV128)
+@pytest.mark.parametrize("direction", [0, 1, 2, 3])
+def test_dv128_shapes(B, heads, H, W, dk, init, direction):
+    inp = make_inputs(B, heads, H, W, dk, 128, seed=97 + H * 31 + W + dk, init_std=0.5 if init else None)
+    out, sf = run_gpu(inp, H, W, direction)
+    ro, rs = run_oracle(inp, H, W, direction)
+    assert_parity(out, ro, "out")
+    assert_parity(sf, rs, "final state")
+
+
+def test_dv128_in_place_carry():
+    """init_state == final_state with dv = 128 (the halves carry disjoint columns)."""
+    B, heads, H, W = 1, 2, 12, 10
+    inp = make_inputs(B, heads, H, W, 128, 128, seed=13, init_std=0.2)
+    dev = torch.device("cuda", 0)
+    q, k, v, g = (inp[n].to(dev) for n in ("q", "k", "v", "g"))
+    st = inp["s0"].to(dev).clone()
+    out, sf = gla.gtr_gla_fwd(q, k, v, g, H, W, 3, init_state=st, final_state=st)
+    torch.cuda.synchronize()
+    ro, rs = run_oracle(inp, H, W, 3)
+    assert_parity(out.float().cpu().numpy(), ro, "out")
+    assert_parity(st.cpu().numpy(), rs, "carried state")
+
+
 @pytest.mark.parametrize("mode", ["retain", "forget_inf", "forget_big", "mixed_extreme",
                                   "strong"])
 def test_degenerate_gates(mode):

@@ -1,14 +1,15 @@
 """The TMA-staged warp-specialised kernel (gla_fwd_pipe) vs the fp64 oracle (GPU only).
 
 The library selects it for the gate-from-z entry point and, with GTR_KERNEL=pipe, for
-gtr_gla_fwd at dk = 64.  The parity, span and range tests of the default path run here
-again with that selection: every workload and direction, the edge shapes, degenerate
-gates, forced span counts (look-back and corrections), in-place carry, split and
-resume, and the large-key sub-block path.  (dk = 128 shapes keep their own kernel.)
+gtr_gla_fwd.  The parity, span and range tests of the default path run here again
+with that selection: every workload and direction, the edge shapes (dk = 128 as two
+key halves), dv = 128 (two value halves), degenerate gates, forced span counts
+(look-back and corrections), in-place carry, split and resume, and the large-key
+sub-block path.
 """
 import pytest
 
-from tests.test_gpu_parity import (test_degenerate_gates, test_edge_shapes,  # noqa: F401
+from tests.test_gpu_parity import (test_degenerate_gates, test_dv128_shapes, test_edge_shapes,  # noqa: F401
                                    test_empty_grid_copies_state, test_in_place_state_carry,
                                    test_large_sample_rows_match_oracle_subset,
                                    test_split_sequence_resume, test_workload_parity)
