@@ -135,9 +135,10 @@ def launches_per_call(w) -> int:
     return 2 if w.dk == 128 else 1
 
 
-def recorded_traffic(workload_name: str):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
-    current kernel source; else None.  (A name ending in "+z": the gate-from-z entry.)"""
+def recorded_profile(workload_name: str, key: str = "traffic_bytes_per_call"):
+    """A number from the committed ncu summary of the workload's kernel (DRAM bytes
+    per call, warp instructions per chunk), if it was taken on the current kernel
+    source; else None.  (A name ending in "+z": the gate-from-z entry.)"""
     gate_z = workload_name.endswith("+z")
     kernel = kernel_for(WORKLOADS[workload_name[:-2] if gate_z else workload_name], gate_z)
     path = os.path.join(ROOT, "profiles", f"{kernel}_{workload_name}.md")
@@ -146,10 +147,14 @@ def recorded_traffic(workload_name: str):
     except OSError:
         return None
     m_sha = re.search(r"kernel_source_sha1:\s*([0-9a-f]+)", text)
-    m_tr = re.search(r"traffic_bytes_per_call:\s*([0-9]+)", text)
-    if not m_sha or not m_tr or m_sha.group(1) != kernel_source_hash(kernel):
+    m_v = re.search(key + r":\s*([0-9.]+)", text)
+    if not m_sha or not m_v or m_sha.group(1) != kernel_source_hash(kernel):
         return None
-    return int(m_tr.group(1))
+    return float(m_v.group(1)) if "." in m_v.group(1) else int(m_v.group(1))
+
+
+def recorded_traffic(workload_name: str):
+    return recorded_profile(workload_name, "traffic_bytes_per_call")
 
 
 # ------------------------------------------------------------------ clocks
@@ -365,7 +370,9 @@ def roofline(w, ms_per_call, workload_name, gate_z=False):
             "unit": "GB/s",
             "frac": round(achieved / peak, 4), "traffic": recorded_traffic(workload_name),
             "peak_source": which, "bytes_alg_per_call": b, "flops_alg_per_call": flops_alg(w),
-            "launches_per_call": launches_per_call(w)}
+            "launches_per_call": launches_per_call(w),
+            # the issue bound: warp instructions per 64-token chunk of one sequence
+            "inst_per_chunk": recorded_profile(workload_name, "inst_per_chunk")}
 
 
 # ------------------------------------------------------------------ Spatial SwiGLU

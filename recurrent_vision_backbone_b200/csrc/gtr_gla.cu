@@ -601,6 +601,17 @@ static cudaError_t launch(const Params &prm, const Plan &pl, void *workspace, cu
 
 using namespace gtr;
 
+#include <nvtx3/nvToolsExt.h>
+
+// An NVTX range over a library call (a no-op unless a profiler is attached): the
+// calls, the stack's recording and the SwiGLU launch show up on a timeline.
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
+
 static gtr_status_t check_args(const void *q, const void *k, const void *v, const void *g,
                                int B, int heads, int H, int W, int dk, int dv, int dir,
                                int chunk, const float *s0, const void *out, const float *sf) {
@@ -671,6 +682,7 @@ extern "C" gtr_status_t gtr_gla_fwd(const gtr_half_t *q, const gtr_half_t *k,
                                     int Hgrid, int Wgrid, int dk, int dv, int direction, int chunk,
                                     const float *init_state, gtr_half_t *out, float *final_state,
                                     void *stream) {
+    NvtxRange nvtx_range("gtr_gla_fwd");
     const gtr_status_t st = check_args(q, k, v, g, B, heads, Hgrid, Wgrid, dk, dv, direction,
                                        chunk, init_state, out, final_state);
     if (st != GTR_OK) return st;
@@ -690,6 +702,7 @@ extern "C" gtr_status_t gtr_gla_fwd_z(const gtr_half_t *q, const gtr_half_t *k, 
                                       const gtr_half_t *z, float tau, int B, int heads, int Hgrid, int Wgrid,
                                       int dk, int dv, int direction, int chunk, const float *init_state,
                                       gtr_half_t *out, float *final_state, void *stream) {
+    NvtxRange nvtx_range("gtr_gla_fwd_z");
     const gtr_status_t st = check_args(q, k, v, z, B, heads, Hgrid, Wgrid, dk, dv, direction, chunk, init_state,
                                        out, final_state);
     if (st != GTR_OK) return st;
@@ -738,6 +751,7 @@ static cudaStream_t g_rec_stream[64];
 
 extern "C" gtr_status_t gtr_gla_fwd_stack(const gtr_gla_layer_t *layers, int n_layers, int B, int heads, int Hgrid,
                                           int Wgrid, int dk, int dv, int chunk, void *stream) {
+    NvtxRange nvtx_range("gtr_gla_fwd_stack");
     if (layers == nullptr || n_layers < 1 || n_layers > 64) return GTR_ERR_INVALID_ARG;
     for (int i = 0; i < n_layers; ++i) {
         const gtr_gla_layer_t &L = layers[i];
@@ -822,6 +836,7 @@ extern "C" gtr_status_t gtr_gla_fwd_stack(const gtr_gla_layer_t *layers, int n_l
 }
 
 extern "C" gtr_status_t gtr_gla_init(void *stream) {
+    NvtxRange nvtx_range("gtr_gla_init");
     const int dev = current_device();
     const int cap = span_capacity(dev, num_sms(dev), true);
     if (cap <= 0) return GTR_OK;   // no span plan on this device: no workspace
@@ -847,6 +862,7 @@ extern "C" gtr_status_t gtr_gla_fwd_ws(const gtr_half_t *q, const gtr_half_t *k,
                                        int chunk, const float *init_state, gtr_half_t *out,
                                        float *final_state, void *workspace, size_t workspace_bytes,
                                        void *stream) {
+    NvtxRange nvtx_range("gtr_gla_fwd_ws");
     const gtr_status_t st = check_args(q, k, v, g, B, heads, Hgrid, Wgrid, dk, dv, direction,
                                        chunk, init_state, out, final_state);
     if (st != GTR_OK) return st;
@@ -897,6 +913,7 @@ extern "C" gtr_status_t gtr_gla_fwd_static(const gtr_half_t *q, const gtr_half_t
                                            int heads, int Hgrid, int Wgrid, int dk, int dv,
                                            int direction, int chunk, const float *init_state,
                                            gtr_half_t *out, float *final_state, void *stream) {
+    NvtxRange nvtx_range("gtr_gla_fwd_static");
     const gtr_status_t st = check_args(q, k, v, g, B, heads, Hgrid, Wgrid, dk, dv, direction,
                                        chunk, init_state, out, final_state);
     if (st != GTR_OK) return st;
@@ -1073,6 +1090,7 @@ static cudaError_t swiglu_maps(const void *G, const void *U, const void *h, int 
 extern "C" gtr_status_t gtr_spatial_swiglu_gate(const gtr_half_t *G, const gtr_half_t *U, const float *w,
                                                 const float *bias, int B, int H, int W, int C, gtr_half_t *out,
                                                 void *stream) {
+    NvtxRange nvtx_range("gtr_spatial_swiglu_gate");
     if (B < 0 || H < 0 || W < 0 || C < 0) return GTR_ERR_INVALID_ARG;
     const long long n = (long long)B * H * W * C;
     if (n == 0) return GTR_OK;   // nothing to read or write
