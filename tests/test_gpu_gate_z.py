@@ -89,3 +89,16 @@ def test_dk128_with_fused_gate(direction):
     out, sf, ro, rs = _run(inp, 8.0, H, W, direction)
     assert_parity(out, ro, "dk128 out")
     assert_parity(sf, rs, "dk128 final state")
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 128), (128, 128)])
+def test_wide_values_with_fused_gate(dk, dv):
+    """dv = 128 (two value halves), with dk = 64 or 128, through the fused gate."""
+    B, heads, H, W = 1, 3, 17, 29
+    inp = make_inputs(B, heads, H, W, dk, dv, seed=930 + dk + dv, init_std=0.3)
+    gen = torch.Generator().manual_seed(931)
+    inp["z"] = (torch.randn((B, H * W, heads, dk), generator=gen) * 2.0).half()
+    for d in (1, 2):
+        out, sf, ro, rs = _run(inp, 16.0, H, W, d)
+        assert_parity(out, ro, f"dk{dk} dv{dv} dir {d} out")
+        assert_parity(sf, rs, f"dk{dk} dv{dv} dir {d} final state")

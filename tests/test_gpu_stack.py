@@ -66,6 +66,26 @@ def test_chained_stack_equals_one_long_scan():
     assert_parity(states[4].cpu().numpy(), rs, "chained final state")
 
 
+def test_wide_head_stack_matches_single_calls():
+    """A four-layer stack with dk = dv = 128 (four launches per layer) equals the same
+    calls made one by one, bit for bit."""
+    B, heads, H, W = 1, 2, 20, 20
+    dev = torch.device("cuda", 0)
+    layers = []
+    for i in range(4):
+        inp = make_inputs(B, heads, H, W, 128, 128, seed=70 + i, init_std=0.2)
+        t = {n: inp[n].to(dev) for n in ("q", "k", "v", "g")}
+        layers.append(dict(t, direction=i, init_state=inp["s0"].to(dev), final_state=True))
+    res = gla.gtr_gla_fwd_stack(layers, H, W)
+    torch.cuda.synchronize()
+    assert gla.device_status() == gla.GTR_OK
+    for i, (L, (out, fs)) in enumerate(zip(layers, res)):
+        o1, s1 = gla.gtr_gla_fwd(L["q"], L["k"], L["v"], L["g"], H, W, L["direction"],
+                                 init_state=L["init_state"], final_state=True)
+        torch.cuda.synchronize()
+        assert torch.equal(out, o1) and torch.equal(fs, s1), f"layer {i}"
+
+
 def test_stack_argument_checks():
     dev = torch.device("cuda", 0)
     inp = make_inputs(1, 1, 4, 4, 64, 64, seed=1)

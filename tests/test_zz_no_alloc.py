@@ -45,3 +45,22 @@ def test_static_scratch_plans_within_its_size(monkeypatch):
     ro, rs = run_oracle(inp, H, W, 0)
     assert_parity(out.float().cpu().numpy(), ro, "out")
     assert_parity(sf.cpu().numpy(), rs, "final state")
+
+
+@pytest.mark.parametrize("dk,dv", [(128, 64), (64, 128), (128, 128)])
+def test_static_scratch_wide_heads_match_default(dk, dv):
+    """dk and / or dv = 128 (two or four launches over 64-wide halves) through the
+    static scratch equal the default path bit for bit, and the oracle."""
+    B, heads, H, W = 1, 4, 24, 24
+    inp = make_inputs(B, heads, H, W, dk, dv, seed=dk + dv, init_std=0.3)
+    dev = torch.device("cuda", 0)
+    t = {n: inp[n].to(dev) for n in ("q", "k", "v", "g")}
+    s0 = inp["s0"].to(dev)
+    o1, s1 = gla.gtr_gla_fwd_static(t["q"], t["k"], t["v"], t["g"], H, W, 3, init_state=s0, final_state=True)
+    o2, s2 = gla.gtr_gla_fwd(t["q"], t["k"], t["v"], t["g"], H, W, 3, init_state=s0, final_state=True)
+    torch.cuda.synchronize()
+    assert gla.device_status() == gla.GTR_OK
+    assert torch.equal(o1, o2) and torch.equal(s1, s2)
+    ro, rs = run_oracle(inp, H, W, 3)
+    assert_parity(o1.float().cpu().numpy(), ro, "out")
+    assert_parity(s1.cpu().numpy(), rs, "final state")
