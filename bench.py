@@ -124,8 +124,9 @@ def kernel_source_hash(kernel: str) -> str:
 
 
 def kernel_for(w, gate_z=False) -> str:
-    """The kernel a call of workload w launches (a dk = 128 call: twice)."""
-    if gate_z or os.environ.get("GTR_KERNEL") == "pipe":
+    """The kernel a call of workload w launches (a dk = 128 call: twice); the same for
+    the gate-from-z entry (an instance that reads z)."""
+    if os.environ.get("GTR_KERNEL") == "pipe":
         return "gla_fwd_pipe_kernel"
     return "gla_fwd_span_kernel"
 

@@ -222,14 +222,6 @@ __device__ __forceinline__ void tmem_st_16x128b_x8(uint32_t taddr, const uint32_
         : "memory");
 }
 
-// Log-decay of the key-side forget gate from its pre-activation z (GTR news article,
-// section "线性注意力到底在省什么"): g = log(sigmoid(z)) / tau = (min(z, 0) - log(1 + e^-|z|))
-// / tau, with CUDA's exp / log intrinsics (relative error ~2^-21, far below the fp16
-// rounding of z itself; for |z| > 17 the log term falls below fp32's resolution of 1 + x,
-// an absolute error under 1e-7 / tau).
-__device__ __forceinline__ float gate_of(float z, float inv_tau) {
-    return (fminf(z, 0.f) - __logf(1.f + __expf(-fabsf(z)))) * inv_tau;
-}
 template <bool kZ>
 __device__ __forceinline__ float2 ld_gate2(const uint8_t *p, float inv_tau) {
     const float2 x = ld_h2(p);

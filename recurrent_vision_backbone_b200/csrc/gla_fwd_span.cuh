@@ -126,6 +126,7 @@ struct Work {
     int Lc;       // chunks per span (the last span may be shorter)
     float *ws;    // [n_seq][P][kAggFloats] aggregates
     unsigned *flags;   // [n_seq][P] publish flags (readers still to come), kFlagStride apart
+    float inv_tau;     // the gate's 1 / tau (kernels that read z in place of g)
 };
 // One 128-byte line per flag: every later span of a sequence polls its predecessors'
 // flags, and packed flags made a few L2 lines the hot spot of all those polls (a
@@ -329,8 +330,10 @@ __device__ __forceinline__ int *misc_slow(uint8_t *sm, int b) {   // chunk took 
 // the chunk decay d -> dloc[b] and D_{ci+1} -> dcum, then signals GATE[b].  The
 // sub-block path first waits for MMA 1 of chunk ci-1 (phase index `m1_prev`; it may
 // still read qj / kbar).  Returns true on the sub-block path.
+template <bool kZ>
 __device__ __forceinline__ bool gate_chunk(const Params &P, uint8_t *sm, int ci, int b, int nrows,
-                                           bool held, uint32_t &m1_seen, uint32_t m1_prev, bool &to) {
+                                           bool held, uint32_t &m1_seen, uint32_t m1_prev, bool &to,
+                                           float inv_tau) {
     // (m1_seen / m1_prev: phase count and index of MMA 1 of chunk ci-1 on MMA1[b ^ 1])
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int gI = warp >> 1, ghf = warp & 1, gt0 = 16 * gI + 8 * ghf, gh = 2 * gI + ghf;
@@ -356,7 +359,9 @@ __device__ __forceinline__ bool gate_chunk(const Params &P, uint8_t *sm, int ci,
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
             const uint32_t o = (gt0 + u) * 128 + 4 * lane;
-            const float2 gv = ld_h2(st + 2 * kTile + o);
+            float2 gv = ld_h2(st + 2 * kTile + o);
+            if constexpr (kZ)   // rows past the grid keep g = 0 (their z is the zero fill)
+                gv = gt0 + u < nrows ? gate2<kZ>(gv, inv_tau) : make_float2(0.f, 0.f);
             qh[u] = *reinterpret_cast<const __half2 *>(st + o);
             kh[u] = *reinterpret_cast<const __half2 *>(st + kTile + o);
             a0[u] = exp_f(gv.x);
@@ -469,7 +474,7 @@ __device__ __forceinline__ bool gate_chunk(const Params &P, uint8_t *sm, int ci,
                     for (int i = 0; i < kDK; ++i) {
                         float lg = 0.f;
                         for (int r2 = tw + 1; r2 <= tu; ++r2)
-                            lg += __half2float(*reinterpret_cast<const __half *>(st + 2 * kTile + r2 * 128 + 2 * i));
+                            lg += gate1<kZ>(__half2float(*reinterpret_cast<const __half *>(st + 2 * kTile + r2 * 128 + 2 * i)), inv_tau);
                         const float qv = __half2float(*reinterpret_cast<const __half *>(st + tu * 128 + 2 * i));
                         const float kv = __half2float(*reinterpret_cast<const __half *>(st + kTile + tw * 128 + 2 * i));
                         acc += qv * kv * exp_f(lg);
@@ -754,8 +759,9 @@ __device__ __noinline__ void load_qgo(const __half *q, const __half *g, const __
 // its raw q, g rows (qs, gs: unswizzled) and the decay product D_c from the span start
 // (dc), into the swizzled K-major tile dst.  Thread layout as in gating.  (Out of
 // line: once per span.)
+template <bool kZ>
 __device__ __noinline__ void rebuild_qd(uint8_t *sm, const uint8_t *qs, const uint8_t *gs,
-                                        const float *dc, uint8_t *dst) {
+                                        const float *dc, uint8_t *dst, float inv_tau) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     float *htot = reinterpret_cast<float *>(sm + L::htot);
     const int gI = warp >> 1, ghf = warp & 1, gt0 = 16 * gI + 8 * ghf, gh = 2 * gI + ghf;
@@ -764,7 +770,7 @@ __device__ __noinline__ void rebuild_qd(uint8_t *sm, const uint8_t *qs, const ui
         float r0 = 1.f, r1 = 1.f;
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-            const float2 gv = ld_h2(gs + (gt0 + u) * 128 + 4 * lane);
+            const float2 gv = gate2<kZ>(ld_h2(gs + (gt0 + u) * 128 + 4 * lane), inv_tau);
             r0 *= exp_f(gv.x);
             r1 *= exp_f(gv.y);
             pl[u][0] = r0; pl[u][1] = r1;
@@ -873,7 +879,7 @@ __device__ __forceinline__ void store_aggregate(const uint8_t *sm, float *agg, i
         reinterpret_cast<float4 *>(agg)[e] = *reinterpret_cast<const float4 *>(sst + agg_off(e >> 4, e & 15));
 }
 
-template <int NL>
+template <int NL, bool kZ>
 __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(const Params P, const Work Wk) {
     constexpr int kThreads = span_threads<NL>();
     extern __shared__ uint8_t smem_raw[];
@@ -976,8 +982,8 @@ __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(con
                     wait_l(bar(sm, B_OPSE + b), (nuse[b] & 1u) ^ 1u, to);
                     ++nuse[b];
                     const int nrows = min(kChunk, P.N - (c0 + it) * kChunk);
-                    slow = gate_chunk(P, sm, it, b, nrows, it < hold, m1s[b ^ 1],
-                                      (b ? m1b0 : m1b1) + ((it - 1) >> 1), to);
+                    slow = gate_chunk<kZ>(P, sm, it, b, nrows, it < hold, m1s[b ^ 1],
+                                          (b ? m1b0 : m1b1) + ((it - 1) >> 1), to, Wk.inv_tau);
                 }
                 if (it > 0) {
                     wait_phase(bar(sm, B_MMA1 + (b ^ 1)), m1s[b ^ 1], (b ? m1b0 : m1b1) + ((it - 1) >> 1), to);
@@ -1334,7 +1340,7 @@ __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(con
                 if (ext) cp_async_wait_all();   // the prefetch has landed (needed or not)
                 __syncthreads();
                 if constexpr (NL == 2)
-                    if (xfix) rebuild_qd(sm, sm + L::vop, sm + L::vop + kTile, dcum + kHold * 64, sm + L::qint);
+                    if (xfix) rebuild_qd<kZ>(sm, sm + L::vop, sm + L::vop + kTile, dcum + kHold * 64, sm + L::qint, Wk.inv_tau);
                 fence_proxy_async_cta();
                 __syncthreads();
                 if (warp == 0) {
@@ -1391,7 +1397,7 @@ __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(con
                              stq + 2 * kTile, stq + 3 * kTile, kThreads, P.ldk, P.ldv);
                     cp_async_wait_all();
                     __syncthreads();
-                    rebuild_qd(sm, sm + L::stg, sm + L::stg + 2 * kTile, dcum + ci * 64, sm + L::qint);
+                    rebuild_qd<kZ>(sm, sm + L::stg, sm + L::stg + 2 * kTile, dcum + ci * 64, sm + L::qint, Wk.inv_tau);
                 } else {
                     // load q, g, o rows of this chunk (all threads), rebuild Q * P * D_c
                     {
@@ -1421,7 +1427,8 @@ __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(con
                             float r0 = 1.f, r1 = 1.f;
     #pragma unroll
                             for (int u = 0; u < 8; ++u) {
-                                const float2 gv = ld_h2(sm + L::stg + 2 * kTile + (gt0 + u) * 128 + 4 * lane);
+                                const float2 gv = gate2<kZ>(ld_h2(sm + L::stg + 2 * kTile + (gt0 + u) * 128 + 4 * lane),
+                                                            Wk.inv_tau);
                                 r0 *= exp_f(gv.x);
                                 r1 *= exp_f(gv.y);
                                 pl[u][0] = r0; pl[u][1] = r1;

@@ -9,17 +9,19 @@
 // chunk is parallel, only the chunk-boundary state is passed in order).
 //
 // Kernels:
-//   * gla_fwd_span.cuh (dk = 64, the default of gtr_gla_fwd): each sequence is cut into
-//     spans of chunks that run on separate SMs with purely local state chains; one
-//     aggregate per span through a workspace, a look-back fold, and a deferred
-//     correction of the later spans' outputs.  Chunk rows are staged with 16-byte
-//     cp.async (the scan direction applied only in the row addresses).
-//   * gla_fwd_pipe.cuh: the same span decomposition with TMA tensor copies and
-//     warp-specialised roles (gating teams, state group, readout group) on mbarrier
-//     hand-offs.  It serves gtr_gla_fwd_z (the gate formed from its pre-activation
-//     while staging), dk = 128 (two launches over the two 64-channel halves of the
-//     keys: the recurrence is separable by key channel and the second half adds its
-//     output to the first's), and dk = 64 when GTR_KERNEL=pipe.
+//   * gla_fwd_span.cuh (the default): each sequence is cut into spans of chunks that
+//     run on separate SMs with purely local state chains; one aggregate per span through
+//     a workspace, a look-back fold, and a deferred correction of the later spans'
+//     outputs.  Chunk rows are staged with 16-byte cp.async (the scan direction applied
+//     only in the row addresses).  An instance that reads z forms the gate from its
+//     pre-activation while gating (gtr_gla_fwd_z).
+//   * gla_fwd_pipe.cuh (GTR_KERNEL=pipe): the same span decomposition with TMA tensor
+//     copies and warp-specialised roles (gating teams, state group, readout group) on
+//     mbarrier hand-offs.
+//   Both take 64 key channels and 64 value columns per launch: dk = 128 is two launches
+//   over the two key halves (the recurrence is separable by key channel; the second
+//   adds its output to the first's), dv = 128 two launches over the two value halves
+//   (separable by value column; disjoint outputs).
 //   Per chunk, in both: gated operands whose decay factors fed to the tensor cores stay
 //   inside fp16 (a fast path for chunk decays >= e^-6, a 16-token sub-block path with an
 //   exact fp32 diagonal fallback otherwise), then tcgen05.mma (fp16 x fp16 -> fp32 in
@@ -106,6 +108,26 @@ __device__ __forceinline__ float absmax4(float4 v) {
     return fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
 }
 
+// Log-decay of the key-side forget gate from its pre-activation z (GTR news article,
+// section "线性注意力到底在省什么"): g = log(sigmoid(z)) / tau = (min(z, 0) - log(1 + e^-|z|))
+// / tau, with CUDA's exp / log intrinsics (relative error ~2^-21, far below the fp16
+// rounding of z itself; for |z| > 17 the log term falls below fp32's resolution of 1 + x,
+// an absolute error under 1e-7 / tau).
+__device__ __forceinline__ float gate_of(float z, float inv_tau) {
+    return (fminf(z, 0.f) - __logf(1.f + __expf(-fabsf(z)))) * inv_tau;
+}
+// The log-decay from a staged gate value: g itself, or formed from z (kZ).
+template <bool kZ>
+__device__ __forceinline__ float2 gate2(float2 x, float inv_tau) {
+    if constexpr (kZ) return make_float2(gate_of(x.x, inv_tau), gate_of(x.y, inv_tau));
+    return x;
+}
+template <bool kZ>
+__device__ __forceinline__ float gate1(float x, float inv_tau) {
+    if constexpr (kZ) return gate_of(x, inv_tau);
+    return x;
+}
+
 __device__ __forceinline__ float2 ld_h2(const uint8_t *p) {
     return __half22float2(*reinterpret_cast<const __half2 *>(p));
 }
@@ -136,10 +158,11 @@ __device__ __forceinline__ void tmem_ld_16x256b_x4(uint32_t taddr, uint32_t (&r)
 namespace gtr {
 
 // ------------------------------------------------------------------ host
-enum KernelKind { kSpan = 0, kSpanShort = 1, kPipe = 2, kPipeZ = 3, kKinds = 4 };
+enum KernelKind { kSpan = 0, kSpanShort = 1, kSpanZ = 2, kSpanShortZ = 3, kPipe = 4, kPipeZ = 5, kKinds = 6 };
 
-// the span kernel with two loader warps (kSpan) or four (kSpanShort: short spans)
-static bool is_span(int kind) { return kind == kSpan || kind == kSpanShort; }
+// the span kernel with two loader warps (kSpan) or four (kSpanShort: short spans),
+// reading g or (the Z kinds) its pre-activation z
+static bool is_span(int kind) { return kind >= kSpan && kind <= kSpanShortZ; }
 // the TMA-staged warp-specialised kernel (g, or its pre-activation z)
 static bool is_pipe(int kind) { return kind == kPipe || kind == kPipeZ; }
 
@@ -160,28 +183,32 @@ struct Plan {
     size_t ws_bytes;   // workspace the launch needs (span kernel with >= 2 spans)
 };
 
-// dk = 64 runs the span kernel; dk = 128 the basic one.  GTR_KERNEL=basic|cluster
-// (tuning knob) selects one of the other dk = 64 kernels instead.
+// The span kernel by default; GTR_KERNEL=pipe (tuning knob) selects the TMA-staged one.
 static KSpec spec_of(int kind) {
     switch (kind) {
     case kSpanShort:
-        return KSpec{reinterpret_cast<const void *>(&sp::gla_fwd_span_kernel<4>), sp::span_threads<4>(),
+        return KSpec{reinterpret_cast<const void *>(&sp::gla_fwd_span_kernel<4, false>), sp::span_threads<4>(),
                      sp::L::alloc, kSpanShort};
+    case kSpanZ:
+        return KSpec{reinterpret_cast<const void *>(&sp::gla_fwd_span_kernel<2, true>), sp::span_threads<2>(),
+                     sp::L::alloc, kSpanZ};
+    case kSpanShortZ:
+        return KSpec{reinterpret_cast<const void *>(&sp::gla_fwd_span_kernel<4, true>), sp::span_threads<4>(),
+                     sp::L::alloc, kSpanShortZ};
     case kPipe:
         return KSpec{reinterpret_cast<const void *>(&pp::gla_fwd_pipe_kernel<false>), pp::kThreads, pp::L::alloc, kPipe};
     case kPipeZ:
         return KSpec{reinterpret_cast<const void *>(&pp::gla_fwd_pipe_kernel<true>), pp::kThreads, pp::L::alloc, kPipeZ};
     default:
-        return KSpec{reinterpret_cast<const void *>(&sp::gla_fwd_span_kernel<2>), sp::span_threads<2>(),
+        return KSpec{reinterpret_cast<const void *>(&sp::gla_fwd_span_kernel<2, false>), sp::span_threads<2>(),
                      sp::L::alloc, kSpan};
     }
 }
 
-static int kind_for(int dk, long n_chunks) {
-    (void)n_chunks;
+static int kind_for(bool gate_z) {
     const char *e = getenv("GTR_KERNEL");
-    if (e && !strcmp(e, "pipe")) return kPipe;   // (dk = 128: two 64-channel halves, as with the span kernel)
-    return kSpan;
+    if (e && !strcmp(e, "pipe")) return gate_z ? kPipeZ : kPipe;
+    return gate_z ? kSpanZ : kSpan;
 }
 
 static std::mutex g_mu;
@@ -300,9 +327,10 @@ static Plan span_plan(long n_seq, long n_chunks, int cap, int kind, size_t ws_li
         return p1;
     }
     best.ws_bytes = span_ws_bytes(n_seq, best.cluster, cap);
-    if (kind == kSpan && best.cluster > 1 && best.span_len <= sp::kShortSpan) {   // latency-bound: four loaders
-        const KSpec ks = spec_of(kSpanShort);
-        best.kind = kSpanShort;
+    if ((kind == kSpan || kind == kSpanZ) && best.cluster > 1 && best.span_len <= sp::kShortSpan) {
+        // latency-bound: four loaders
+        const KSpec ks = spec_of(kind == kSpan ? kSpanShort : kSpanShortZ);
+        best.kind = ks.slot;
         best.threads = ks.threads;
         best.smem = ks.smem;
     }
@@ -316,7 +344,8 @@ static Plan span_plan(long n_seq, long n_chunks, int cap, int kind, size_t ws_li
 // for gtr_gla_fwd_static; unlimited otherwise).
 static Plan make_plan(long n_seq, long n_chunks, int dk, bool query, size_t ws_limit = ~size_t(0),
                       bool gate_z = false) {
-    const int kind = gate_z ? kPipeZ : kind_for(dk, n_chunks);
+    (void)dk;
+    const int kind = kind_for(gate_z);
     const int dev = current_device();
     const int sms = num_sms(dev);
     if (n_chunks == 0) return Plan{kind, 1, 1, 0, 0, 0, 0};   // no launch: the state copy only
@@ -582,6 +611,7 @@ static cudaError_t launch(const Params &prm, const Plan &pl, void *workspace, cu
     }
     if (is_span(pl.kind)) {
         sp::Work wk{};
+        wk.inv_tau = inv_tau;
         wk.P = pl.cluster;
         wk.Lc = pl.span_len;
         if (pl.ws_bytes > 0) {

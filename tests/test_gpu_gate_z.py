@@ -1,4 +1,4 @@
-"""Gate fused into staging: gtr_gla_fwd_z (z and tau in place of g) vs the fp64 oracle
+"""Gate fused into the kernel: gtr_gla_fwd_z (z and tau in place of g) vs the fp64 oracle
 fed the oracle's own fp64 gate g = log(sigmoid(z)) / tau (GPU only).
 
 The z draws follow the workloads' recipe (z ~ N(0, 1), tau = 16) at every dk = 64
