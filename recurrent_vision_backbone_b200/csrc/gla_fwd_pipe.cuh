@@ -844,7 +844,9 @@ __device__ __forceinline__ void issue_mma2(uint8_t *sm, uint32_t sbase, uint32_t
 template <bool kZ>
 __global__ void __launch_bounds__(kThreads, 1) gla_fwd_pipe_kernel(const __grid_constant__ Args A) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // aligned by an offset from the shared array itself (not through an integer), so
+    // that the compiler still sees every tile access as shared memory
+    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sbase = smem_u32(sm);
     const Params &P = A.P;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;

@@ -435,8 +435,9 @@ __device__ __forceinline__ bool gate_chunk(const Params &P, uint8_t *sm, int ci,
     if (!slow) {
         // ---------- fast path: Qint = q P, K~ = k / P (= k * suffix / d)
         // The factors (P in [e^-6, 1], suffix / d in [1, e^6]) are rounded to fp16 and
-        // applied with packed fp16 multiplies.
-        const float i0 = aft[0] / dch[0], i1 = aft[1] / dch[1];
+        // applied with packed fp16 multiplies (d >= e^-6 here: the fast division's
+        // couple of ulp vanish in that rounding).
+        const float i0 = __fdividef(aft[0], dch[0]), i1 = __fdividef(aft[1], dch[1]);
         const __half2 dch2 = __floats2half2_rn(dc.x, dc.y);
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
@@ -621,6 +622,46 @@ __device__ __forceinline__ void load_tmem_b(uint32_t tmem, BRegs &r) {
     tmem_ld_wait();
 }
 
+// Causal fp16 P of warp q's rows (16q ..) from its scores registers: column block
+// 2 half + cc / 2 (16 columns) lies left of the diagonal for blocks < Q (kept as is),
+// right of it for blocks > Q (zero: nothing to convert), and on it for block Q, the
+// only one compared element by element (row and column within the block: lane / 4 +
+// 8 hh and 2 (lane % 4) + 8 (cc % 2)); with `fb` that block comes from the exact
+// diagonal diagx.  v: packed column 4 j + lane % 4 per register, as the TMEM store
+// wants it; pmx: max |P|.
+template <int Q>
+__device__ __forceinline__ void causal_p(const BRegs &r, const float *diagx, bool fb, int lane,
+                                         uint32_t (&v)[16], float &pmx) {
+    const int rl = lane >> 2, cl = 2 * (lane & 3);
+#pragma unroll
+    for (int half = 0; half < 2; ++half)
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int blk = 2 * half + (cc >> 1);
+                uint32_t &out = v[2 * (cc + 4 * half) + hh];
+                if (blk > Q) {
+                    out = 0u;
+                    continue;
+                }
+                const uint32_t *rr = half ? r.s1 : r.s0;
+                float x0 = __uint_as_float(rr[4 * cc + 2 * hh]);
+                float x1 = __uint_as_float(rr[4 * cc + 2 * hh + 1]);
+                if (blk == Q) {
+                    const int row = rl + 8 * hh, col = cl + 8 * (cc & 1);
+                    if (fb) {
+                        x0 = diagx[(Q * 16 + row) * 16 + col];
+                        x1 = diagx[(Q * 16 + row) * 16 + col + 1];
+                    }
+                    x0 = col <= row ? x0 : 0.f;
+                    x1 = col + 1 <= row ? x1 : 0.f;
+                }
+                pmx = fmaxf(pmx, fmaxf(fabsf(x0), fabsf(x1)));
+                out = pack_half2(x0, x1);
+            }
+}
+
 // Scores -> causal fp16 P, written back over the scores' own TMEM columns as the A
 // operand of MMA 2 (M=64 lane layout, fp16 pairs packed per 32-bit column: the
 // thread's pair (row, columns 2k, 2k+1) is packed column k).  With `fb` (this warp's
@@ -629,29 +670,14 @@ __device__ __forceinline__ void store_p_tmem(uint8_t *sm, uint32_t tmem, const B
                                              bool fb) {
     const int lane = threadIdx.x & 31, q = (threadIdx.x >> 5) & 3;
     const float *diagx = reinterpret_cast<const float *>(sm + L::diag) + b * 1024;
-    const int row0 = 16 * q + (lane >> 2), col0 = 2 * (lane & 3);
     uint32_t v[16];
     float pmx = 0.f;
-#pragma unroll
-    for (int half = 0; half < 2; ++half)
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc)
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const int row = row0 + 8 * hh;
-                const int col = col0 + 8 * cc + 32 * half;
-                const uint32_t *rr = half ? r.s1 : r.s0;
-                float x0 = __uint_as_float(rr[4 * cc + 2 * hh]);
-                float x1 = __uint_as_float(rr[4 * cc + 2 * hh + 1]);
-                if (fb && (col >> 4) == q) {
-                    x0 = diagx[(q * 16 + (row & 15)) * 16 + (col & 15)];
-                    x1 = diagx[(q * 16 + (row & 15)) * 16 + ((col + 1) & 15)];
-                }
-                x0 = col <= row ? x0 : 0.f;
-                x1 = col + 1 <= row ? x1 : 0.f;
-                pmx = fmaxf(pmx, fmaxf(fabsf(x0), fabsf(x1)));
-                v[2 * (cc + 4 * half) + hh] = pack_half2(x0, x1);   // packed column 4 j + lane % 4
-            }
+    switch (q) {   // warp-uniform
+    case 0: causal_p<0>(r, diagx, fb, lane, v, pmx); break;
+    case 1: causal_p<1>(r, diagx, fb, lane, v, pmx); break;
+    case 2: causal_p<2>(r, diagx, fb, lane, v, pmx); break;
+    default: causal_p<3>(r, diagx, fb, lane, v, pmx); break;
+    }
     range_check(pmx);
     asm volatile(
         "tcgen05.st.sync.aligned.16x128b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
@@ -883,8 +909,9 @@ template <int NL, bool kZ>
 __global__ void __launch_bounds__(span_threads<NL>(), 1) gla_fwd_span_kernel(const Params P, const Work Wk) {
     constexpr int kThreads = span_threads<NL>();
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // aligned by an offset from the shared array itself (not through an integer), so
+    // that the compiler still sees every tile access as shared memory
+    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sbase = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int PS = Wk.P;

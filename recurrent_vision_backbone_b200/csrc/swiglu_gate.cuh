@@ -104,7 +104,9 @@ __device__ __forceinline__ void load_tile(const Args &A, uint32_t sbase, uint64_
 template <int NS>
 __global__ void __launch_bounds__(kThreads, 1) swiglu_gate_kernel(const __grid_constant__ Args A) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    // aligned by an offset from the shared array itself (not through an integer), so
+    // that the compiler still sees every access as shared memory
+    uint8_t *sm = smem_raw + ((128u - (smem_u32(smem_raw) & 127u)) & 127u);
     const uint32_t sbase = smem_u32(sm);
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + L<NS>::bar);
     const int tid = threadIdx.x;
