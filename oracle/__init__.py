@@ -1,4 +1,5 @@
-"""fp64 CPU oracle for the GTR key-decay gated-linear-attention forward pass.
+"""fp64 CPU oracle for the GTR key-decay gated-linear-attention forward pass and its
+backward (reverse-mode differentiation of the same recurrence).
 
 TEST INFRASTRUCTURE, NOT PRODUCT CODE.  Only ``tests/``,
 ``__graft_entry__.smoke()`` and ``bench.py``'s ``cpu_baseline`` / reference
@@ -62,6 +63,8 @@ def load_library(path: str) -> ctypes.CDLL:
                                              ctypes.c_int]
     lib.gla_oracle_gate.restype = ctypes.c_int
     lib.gla_oracle_gate.argtypes = [dp, ctypes.c_long, ctypes.c_double, dp]
+    lib.gla_oracle_bwd.restype = ctypes.c_int
+    lib.gla_oracle_bwd.argtypes = [dp] * 6 + [ctypes.c_int] * 7 + [dp] * 6
     lib.gla_oracle_max_threads.restype = ctypes.c_int
     lib.gla_oracle_set_threads.argtypes = [ctypes.c_int]
     return lib
@@ -130,6 +133,38 @@ def gla_forward(q, k, v, g, H: int, W: int, direction: int, s0=None,
     if rc != 0:
         raise RuntimeError(f"gla_oracle_fwd_range failed with code {rc}")
     return o, sf
+
+
+def gla_backward(q, k, v, g, dout, H: int, W: int, direction: int, s0=None, dsf=None,
+                 lib=None):
+    """Gradients of L = sum(dout * o) + sum(dsf * S_final) through the forward above
+    (reverse-mode differentiation of the token recurrence, ``gla_oracle_bwd``).
+
+    q, k, g: [B, N, heads, dk]; v, dout: [B, N, heads, dv]; s0, dsf: [B, heads, dk, dv]
+    or None (zero).  Returns (dq, dk, dv, dg, ds0) in fp64, ds0 [B, heads, dk, dv].
+    """
+    lib = lib or _get()
+    q, k, v, g, do = _f64(q), _f64(k), _f64(v), _f64(g), _f64(dout)
+    B, N, heads, dk = q.shape
+    dv = v.shape[-1]
+    if N != H * W:
+        raise ValueError(f"N={N} != H*W={H * W}")
+    if k.shape != q.shape or g.shape != q.shape or v.shape[:3] != q.shape[:3] or do.shape != v.shape:
+        raise ValueError("shape mismatch between q, k, v, g, dout")
+    s0a = None if s0 is None else _f64(s0)
+    dsa = None if dsf is None else _f64(dsf)
+    for x in (s0a, dsa):
+        if x is not None and x.shape != (B, heads, dk, dv):
+            raise ValueError("s0 and dsf must be [B, heads, dk, dv]")
+    dq, dkk, dg = np.zeros_like(q), np.zeros_like(q), np.zeros_like(q)
+    dvv = np.zeros_like(v)
+    ds0 = np.zeros((B, heads, dk, dv))
+    rc = lib.gla_oracle_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(do), _ptr(dsa), B, heads, H, W,
+                            dk, dv, int(direction), _ptr(s0a), _ptr(dq), _ptr(dkk), _ptr(dvv),
+                            _ptr(dg), _ptr(ds0))
+    if rc != 0:
+        raise RuntimeError(f"gla_oracle_bwd failed with code {rc}")
+    return dq, dkk, dvv, dg, ds0
 
 
 def gate(z, tau: float, lib=None) -> np.ndarray:
