@@ -104,7 +104,7 @@ def _code_tokens(src: str) -> str:
 
 
 KERNEL_FILES = {"gla_fwd_span_kernel": "gla_fwd_span.cuh", "gla_fwd_pipe_kernel": "gla_fwd_pipe.cuh",
-                "swiglu_gate_kernel": "swiglu_gate.cuh"}
+                "swiglu_gate_kernel": "swiglu_gate.cuh", "gla_bwd_grad_kernel": "gla_bwd.cuh"}
 
 
 def kernel_source_hash(kernel: str) -> str:
@@ -436,6 +436,92 @@ def run_swiglu(name, steps, warmup, stream, world, device, sets, local):
     return res
 
 
+# ------------------------------------------------------------------ backward
+BWD_WORKLOADS = ("gtr640_b1h16_40x40", "hires_b1h16_128x128")
+
+
+def bwd_bytes_alg(w) -> int:
+    """Algorithmic HBM bytes of one backward call: read q, k, g, v and d_out (fp16),
+    write grad_q, grad_k, grad_g and grad_v (fp32), plus the fp32 states it reads
+    (init_state, d_final_state) and writes (grad_init_state)."""
+    th = w.B * w.N * w.heads
+    b = th * (2 * (3 * w.dk + 2 * w.dv) + 4 * (3 * w.dk + w.dv))
+    per_state = w.B * w.heads * w.dk * w.dv * 4
+    return b + per_state * (int(bool(w.init_std)) + 2 * int(bool(w.final_state)))
+
+
+class BwdBench:
+    """Rotating device-resident sets of one workload's backward calls (one per direction
+    per step, each with its own inputs, upstream gradients and gradient outputs; one
+    workspace, the calls being stream-ordered), replayed from CUDA graphs."""
+
+    def __init__(self, w, device, n_sets=None):
+        from recurrent_vision_backbone_b200 import gla
+        from recurrent_vision_backbone_b200.inputs import make_upstream
+        self.gla = gla
+        self.w = w
+        per_step = bwd_bytes_alg(w) * len(w.directions)
+        if n_sets is None:
+            n_sets = max(2, -(-4 * L2_BYTES // per_step))
+        self.n_sets = int(n_sets)
+        self.ws = gla.new_workspace(gla.bwd_workspace_bytes(w.B, w.heads, w.H, w.W, w.dk, w.dv), device)
+        f32 = dict(dtype=torch.float32, device=device)
+        self.sets = []
+        for s in range(self.n_sets):
+            calls = []
+            for d in w.directions:
+                seed = w.seed(d, 300 + s)
+                inp = make_inputs(w.B, w.heads, w.H, w.W, w.dk, w.dv, seed=seed, init_std=w.init_std,
+                                  z_mean_per_head=w.z_mean_per_head, device=device)
+                d_out, dsf = make_upstream(w.B, w.heads, w.H, w.W, w.dk, w.dv, seed, with_dsf=w.final_state,
+                                           device=device)
+                grads = (torch.empty((w.B, w.N, w.heads, w.dk), **f32), torch.empty((w.B, w.N, w.heads, w.dk), **f32),
+                         torch.empty((w.B, w.N, w.heads, w.dv), **f32), torch.empty((w.B, w.N, w.heads, w.dk), **f32),
+                         torch.empty((w.B, w.heads, w.dk, w.dv), **f32) if w.final_state else None)
+                calls.append((d, inp, d_out, dsf, grads))
+            self.sets.append(calls)
+
+    def launch_step(self, s, stream):
+        for d, inp, d_out, dsf, grads in self.sets[s % self.n_sets]:
+            self.gla.gtr_gla_bwd(inp["q"], inp["k"], inp["v"], inp["g"], d_out, self.w.H, self.w.W, d,
+                                 init_state=inp["s0"], d_final_state=dsf, workspace=self.ws, grads=grads,
+                                 stream=stream)
+
+    capture = Workload.capture
+    _graph_of = Workload._graph_of
+    _part = Workload._part
+    replay = Workload.replay
+
+    def calls_per_step(self):
+        return len(self.w.directions)
+
+
+BWD_KERNELS_PER_CALL = 4   # chunk locals, state scans, chunk gradients, dg offsets
+
+
+def run_bwd(name, steps, warmup, stream, world, device, sets, local):
+    w = WORKLOADS[name]
+    bb = BwdBench(w, device, n_sets=sets)
+    clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else local)
+    ms, n_steps, clk = measure(bb, steps, warmup, stream, world, clocks)
+    peak, which = measured_peaks()
+    calls = n_steps * bb.calls_per_step()
+    b = bwd_bytes_alg(w)
+    achieved = b / (ms / calls * 1e-3) / 1e9
+    res = {"workload": name + "+bwd", "entry": "gtr_gla_bwd", "tokens_per_call": w.B * w.N,
+           "value": round(world * w.B * w.N * calls / (ms * 1e-3), 1), "unit": "tokens/s",
+           "steps": n_steps, "us_per_call": round(ms * 1e3 / calls, 3),
+           "roofline": {"kernel": "gla_bwd_*", "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                        "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None,
+                        "peak_source": which, "bytes_alg_per_call": b,
+                        "launches_per_call": BWD_KERNELS_PER_CALL * (w.dk // 64)},
+           "gpu_launches": calls * BWD_KERNELS_PER_CALL * (w.dk // 64), "clocks": clk,
+           "l2": f"inputs rotate over {bb.n_sets} sets ({bb.n_sets * b * bb.calls_per_step() / 2**20:.0f} MiB > 3x L2)"}
+    del bb
+    torch.cuda.empty_cache()
+    return res
+
+
 def recorded_traffic_swiglu(name: str):
     path = os.path.join(ROOT, "profiles", f"swiglu_gate_kernel_{name}.md")
     try:
@@ -615,6 +701,9 @@ def gpu_arm(args):
         for name in SWIGLU_WORKLOADS:   # the Spatial SwiGLU gated value branch
             line["secondary"].append(run_swiglu(name, max(8, args.steps // 16), max(3, args.warmup // 16),
                                                 stream, world, device, None, local))
+        for name in BWD_WORKLOADS:   # the backward pass
+            line["secondary"].append(run_bwd(name, max(8, min(200, args.steps // 16)), 3, stream, world,
+                                             device, None, local))
     # end to end through the public call with host buffers
     e_steps = max(3, min(args.steps, args.e2e_steps))
     ems, en, h2d, d2h = e2e_measure(w1, e_steps, device, rank)

@@ -279,10 +279,11 @@ int gla_oracle_bwd(const double *q, const double *k, const double *v, const doub
                         sk += G[(long)i * dv + j] * vt[j];
                         sa += G[(long)i * dv + j] * Sprev[(long)i * dv + j];
                     }
-                    a[i] = exp(gt[i]);
+                    const double at = exp(gt[i]);   /* a_t of channel i */
+                    a[i] = at;
                     dq[row * dk + i] = sq_;
                     dk_out[row * dk + i] = sk;
-                    dg[row * dk + i] = a[i] * sa;
+                    dg[row * dk + i] = at * sa;
                 }
                 for (int j = 0; j < dv; ++j) {
                     double s = 0.0;

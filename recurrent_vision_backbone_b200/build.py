@@ -14,8 +14,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 SOURCES = [os.path.join(CSRC, "gtr_gla.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, n) for n in ("sm100_ptx.cuh", "gla_fwd_span.cuh", "gla_fwd_pipe.cuh", "swiglu_gate.cuh")]
-DEPS += [os.path.join(ROOT, "include", n) for n in ("gtr_gla.h", "gtr_swiglu.h")]
+DEPS = SOURCES + [os.path.join(CSRC, n) for n in ("sm100_ptx.cuh", "gla_fwd_span.cuh", "gla_fwd_pipe.cuh", "swiglu_gate.cuh", "gla_bwd.cuh")]
+DEPS += [os.path.join(ROOT, "include", n) for n in ("gtr_gla.h", "gtr_swiglu.h", "gtr_gla_bwd.h")]
 LIB = os.path.join(HERE, "libgtr_gla.so")
 
 

@@ -158,6 +158,13 @@ __device__ __forceinline__ void tmem_ld_16x256b_x4(uint32_t taddr, uint32_t (&r)
 namespace gtr {
 
 // ------------------------------------------------------------------ host
+}  // namespace gtr
+
+// the backward pass: its kernels, then (below) its C entry points
+#include "../../include/gtr_gla_bwd.h"
+#include "gla_bwd.cuh"
+
+namespace gtr {
 enum KernelKind { kSpan = 0, kSpanShort = 1, kSpanZ = 2, kSpanShortZ = 3, kPipe = 4, kPipeZ = 5, kKinds = 6 };
 
 // the span kernel with two loader warps (kSpan) or four (kSpanShort: short spans),
@@ -1043,6 +1050,158 @@ extern "C" gtr_status_t gtr_gla_plan(int B, int heads, int Hgrid, int Wgrid, int
     if (smem_bytes) *smem_bytes = pl.smem;
     return GTR_OK;
 }
+
+namespace gtr {
+
+// ------------------------------------------------------------------ backward
+// Workspace of one key half: U -> h_c and W -> dh_{c+1} tiles, chunk log-decays and
+// x totals, the per-sequence constants.
+struct BwdWs {
+    size_t hs, dhs, bc, xc, cst, bytes;
+};
+static BwdWs bwd_ws_layout(long n_seq, long nc) {
+    BwdWs w{};
+    const size_t tiles = align256((size_t)n_seq * nc * 4096 * sizeof(float));
+    const size_t vecs = align256((size_t)n_seq * nc * bw::kC * sizeof(float));
+    w.hs = 0;
+    w.dhs = w.hs + tiles;
+    w.bc = w.dhs + tiles;
+    w.xc = w.bc + vecs;
+    w.cst = w.xc + vecs;
+    w.bytes = w.cst + align256((size_t)n_seq * bw::kC * sizeof(float));
+    return w;
+}
+
+static gtr_status_t check_bwd_args(const void *q, const void *k, const void *v, const void *g, const void *dout,
+                                   const float *s0, const float *dsf, int B, int heads, int H, int W, int dk,
+                                   int dv, int dir, int chunk, const float *gq, const float *gk, const float *gv,
+                                   const float *gg, const float *gs0) {
+    if (B <= 0 || heads <= 0 || H < 0 || W < 0 || dk <= 0 || dv <= 0) return GTR_ERR_INVALID_ARG;
+    if (dir < 0 || dir > 3 || chunk <= 0) return GTR_ERR_INVALID_ARG;
+    if (chunk != kChunk || (dk != 64 && dk != 128) || dv != 64) return GTR_ERR_UNSUPPORTED;
+    const long long N = (long long)H * W;
+    const long long rows = (long long)B * N * heads;
+    if (N > 0x7fffffffLL || rows * (long long)dk > 0x7fffffffLL || rows * dv > 0x7fffffffLL)
+        return GTR_ERR_INVALID_ARG;
+    const bool empty = N == 0;
+    const void *need[] = {q, k, v, g, dout, gq, gk, gv, gg};
+    for (const void *p : need)
+        if (!empty && (!p || !aligned16(p))) return GTR_ERR_INVALID_ARG;
+    const void *opt[] = {s0, dsf, gs0};
+    for (const void *p : opt)
+        if (p && !aligned16(p)) return GTR_ERR_INVALID_ARG;
+    const long long hk = rows * dk * 2, hv = rows * dv * 2, fk = rows * dk * 4, fv = rows * dv * 4;
+    const long long st = (long long)B * heads * dk * dv * 4;
+    struct Span {
+        const void *p;
+        long long n;
+    };
+    const Span ins[] = {{q, hk}, {k, hk}, {v, hv}, {g, hk}, {dout, hv}, {s0, st}, {dsf, st}};
+    const Span outs[] = {{gq, fk}, {gk, fk}, {gv, fv}, {gg, fk}, {gs0, st}};
+    auto overlap = [](const Span &a, const Span &b) {
+        const uintptr_t x = reinterpret_cast<uintptr_t>(a.p), y = reinterpret_cast<uintptr_t>(b.p);
+        return a.p && b.p && a.n > 0 && b.n > 0 && x < y + (uintptr_t)b.n && y < x + (uintptr_t)a.n;
+    };
+    for (int i = 0; i < 5; ++i) {
+        if (empty && i < 4) continue;
+        for (const Span &in : ins)
+            if (overlap(outs[i], in)) return GTR_ERR_INVALID_ARG;
+        for (int j = i + 1; j < 5; ++j)
+            if (!(empty && j < 4) && overlap(outs[i], outs[j])) return GTR_ERR_INVALID_ARG;
+    }
+    return GTR_OK;
+}
+
+static cudaError_t bwd_launch(const bw::Args &a, cudaStream_t stream) {
+    const size_t smem1 = 5 * (size_t)bw::kMat * sizeof(float);
+    cudaError_t e = cudaFuncSetAttribute(bw::gla_bwd_local_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem1);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(bw::gla_bwd_grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)bw::kGradSmem);
+    if (e != cudaSuccess) return e;
+    const unsigned chunks = (unsigned)((long)a.n_seq * a.nc);
+    bw::gla_bwd_local_kernel<<<chunks, bw::kThreads, smem1, stream>>>(a);
+    bw::gla_bwd_scan_kernel<<<(unsigned)a.n_seq * 16u, bw::kThreads, 0, stream>>>(a);
+    bw::gla_bwd_grad_kernel<<<chunks, bw::kThreads, bw::kGradSmem, stream>>>(a);
+    bw::gla_bwd_dg_kernel<<<chunks, bw::kC, 0, stream>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace gtr
+
+extern "C" size_t gtr_gla_bwd_workspace_bytes(int B, int heads, int Hgrid, int Wgrid, int dk, int dv,
+                                              int chunk) {
+    using namespace gtr;
+    if (B <= 0 || heads <= 0 || Hgrid < 0 || Wgrid < 0 || chunk != kChunk || (dk != 64 && dk != 128) || dv != 64)
+        return 0;
+    const long long N = (long long)Hgrid * Wgrid;
+    if (N == 0 || N > 0x7fffffffLL || (long long)B * N * heads * dk > 0x7fffffffLL) return 0;
+    return bwd_ws_layout((long)B * heads, (long)((N + kChunk - 1) / kChunk)).bytes;
+}
+
+extern "C" gtr_status_t gtr_gla_bwd(const gtr_half_t *q, const gtr_half_t *k, const gtr_half_t *v,
+                                    const gtr_half_t *g, const gtr_half_t *d_out, const float *init_state,
+                                    const float *d_final_state, int B, int heads, int Hgrid, int Wgrid,
+                                    int dk, int dv, int direction, int chunk, float *grad_q, float *grad_k,
+                                    float *grad_v, float *grad_g, float *grad_init_state, void *workspace,
+                                    size_t workspace_bytes, void *stream) {
+    using namespace gtr;
+    NvtxRange nvtx_range("gtr_gla_bwd");
+    gtr_status_t st = check_bwd_args(q, k, v, g, d_out, init_state, d_final_state, B, heads, Hgrid, Wgrid, dk,
+                                     dv, direction, chunk, grad_q, grad_k, grad_v, grad_g, grad_init_state);
+    if (st != GTR_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const long long N = (long long)Hgrid * Wgrid;
+    const long n_seq = (long)B * heads;
+    const size_t st_bytes = (size_t)n_seq * dk * dv * sizeof(float);
+    if (N == 0) {   // no position: dL/dS0 = dL/dS_final
+        if (grad_init_state == nullptr) return GTR_OK;
+        return cuda_status(d_final_state ? cudaMemcpyAsync(grad_init_state, d_final_state, st_bytes,
+                                                           cudaMemcpyDeviceToDevice, s)
+                                         : cudaMemsetAsync(grad_init_state, 0, st_bytes, s));
+    }
+    const long nc = (long)((N + kChunk - 1) / kChunk);
+    const BwdWs lay = bwd_ws_layout(n_seq, nc);
+    if (workspace == nullptr || workspace_bytes < lay.bytes || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return GTR_ERR_INVALID_ARG;
+    uint8_t *wb = static_cast<uint8_t *>(workspace);
+    for (int half = 0; half < dk / 64; ++half) {
+        bw::Args a{};
+        const size_t ko = (size_t)half * 64;
+        a.q = reinterpret_cast<const __half *>(q) + ko;
+        a.k = reinterpret_cast<const __half *>(k) + ko;
+        a.g = reinterpret_cast<const __half *>(g) + ko;
+        a.v = reinterpret_cast<const __half *>(v);
+        a.dout = reinterpret_cast<const __half *>(d_out);
+        a.s0 = init_state ? init_state + ko * dv : nullptr;
+        a.dsf = d_final_state ? d_final_state + ko * dv : nullptr;
+        a.dq = grad_q + ko;
+        a.dk = grad_k + ko;
+        a.dg = grad_g + ko;
+        a.dv = grad_v;
+        a.ds0 = grad_init_state ? grad_init_state + ko * dv : nullptr;
+        a.hs = reinterpret_cast<float *>(wb + lay.hs);
+        a.dhs = reinterpret_cast<float *>(wb + lay.dhs);
+        a.bc = reinterpret_cast<float *>(wb + lay.bc);
+        a.xc = reinterpret_cast<float *>(wb + lay.xc);
+        a.cst = reinterpret_cast<float *>(wb + lay.cst);
+        a.heads = heads;
+        a.H = Hgrid;
+        a.W = Wgrid;
+        a.N = (int)N;
+        a.dir = direction;
+        a.n_seq = (int)n_seq;
+        a.nc = (int)nc;
+        a.ldk = dk;
+        a.sstride = dk * dv;
+        a.acc_dv = half;
+        st = cuda_status(bwd_launch(a, s));
+        if (st != GTR_OK) return st;
+    }
+    return GTR_OK;
+}
+
 
 extern "C" const char *gtr_gla_version(void) { return "0.3.0"; }
 

@@ -1,4 +1,5 @@
-"""Python binding of the C ABI in include/gtr_gla.h (argument marshalling only).
+"""Python binding of the C ABI in include/gtr_gla.h, gtr_gla_bwd.h and gtr_swiglu.h
+(argument marshalling only).
 
 Every step of the token mixer runs in the CUDA library ``libgtr_gla.so``; this
 module only checks tensor metadata, passes raw device pointers and the CUDA
@@ -23,7 +24,8 @@ STATIC_WS_BYTES = 4 << 20   # GTR_STATIC_WS_BYTES
 
 EXPORTED_SYMBOLS = ("gtr_gla_fwd", "gtr_gla_fwd_z", "gtr_gla_fwd_stack", "gtr_gla_init", "gtr_gla_workspace_bytes", "gtr_gla_fwd_ws",
                     "gtr_gla_fwd_static", "gtr_gla_device_status", "gtr_status_str", "gtr_gla_plan", "gtr_gla_version",
-                    "gtr_gla_last_error", "gtr_gla_selftest_timeout", "gtr_spatial_swiglu_gate")
+                    "gtr_gla_last_error", "gtr_gla_selftest_timeout", "gtr_spatial_swiglu_gate",
+                    "gtr_gla_bwd", "gtr_gla_bwd_workspace_bytes")
 
 _lock = threading.Lock()
 _lib = None
@@ -71,6 +73,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.gtr_gla_fwd_ws.restype = i
         lib.gtr_gla_fwd_ws.argtypes = ([vp, vp, vp, vp] + [i] * 8 + [vp, vp, vp]
                                        + [vp, ctypes.c_size_t, vp])
+        lib.gtr_gla_bwd.restype = i
+        lib.gtr_gla_bwd.argtypes = [vp] * 7 + [i] * 8 + [vp] * 6 + [ctypes.c_size_t, vp]
+        lib.gtr_gla_bwd_workspace_bytes.restype = ctypes.c_size_t
+        lib.gtr_gla_bwd_workspace_bytes.argtypes = [i] * 7
         lib.gtr_gla_device_status.restype = i
         lib.gtr_gla_device_status.argtypes = [vp]
         lib.gtr_gla_init.restype = i
@@ -263,6 +269,59 @@ def gtr_gla_fwd_ws(q, k, v, g, Hgrid: int, Wgrid: int, direction: int, workspace
     if st != GTR_OK:
         raise GTRError(st, "gtr_gla_fwd_ws")
     return out, final_state
+
+
+def bwd_workspace_bytes(B: int, heads: int, Hgrid: int, Wgrid: int, dk: int, dv: int,
+                        chunk: int = 64) -> int:
+    """Workspace gtr_gla_bwd needs for a shape (0: none, or a rejected shape)."""
+    return int(load().gtr_gla_bwd_workspace_bytes(B, heads, Hgrid, Wgrid, dk, dv, chunk))
+
+
+def gtr_gla_bwd(q, k, v, g, d_out, Hgrid: int, Wgrid: int, direction: int, init_state=None,
+                d_final_state=None, workspace=None, grads=None, want_init_grad: bool = True,
+                chunk: int = 64, stream=None):
+    """Backward pass of one token-mixer call on device tensors.
+
+    q, k, g, v, init_state, Hgrid, Wgrid, direction: as given to the forward call;
+    d_out: fp16 [B, N, heads, dv] = dL/do; d_final_state: fp32 [B, heads, dk, dv] or None.
+    workspace: a CUDA uint8 tensor of at least bwd_workspace_bytes(...) bytes, or None
+    to allocate one.  grads: a tuple (grad_q, grad_k, grad_v, grad_g, grad_init_state) of
+    fp32 tensors to fill, or None to allocate them.  Returns that tuple (grad_init_state
+    None unless want_init_grad).
+    """
+    lib = load()
+    (B, heads, dk, dv), _, _ = _prepare(q, k, v, g, Hgrid, Wgrid, init_state, d_out, None)
+    N = q.shape[1]
+    if d_out.dtype != torch.float16 or not d_out.is_contiguous() or tuple(d_out.shape) != tuple(v.shape):
+        raise ValueError("d_out must be a contiguous CUDA float16 tensor shaped like v")
+    if d_final_state is not None and (d_final_state.dtype != torch.float32 or not d_final_state.is_contiguous()
+                                      or tuple(d_final_state.shape) != (B, heads, dk, dv)
+                                      or d_final_state.device != q.device):
+        raise ValueError("d_final_state must be a contiguous float32 [B,heads,dk,dv] tensor on q's device")
+    if grads is None:
+        f32 = dict(dtype=torch.float32, device=q.device)
+        grads = (torch.empty((B, N, heads, dk), **f32), torch.empty((B, N, heads, dk), **f32),
+                 torch.empty((B, N, heads, dv), **f32), torch.empty((B, N, heads, dk), **f32),
+                 torch.empty((B, heads, dk, dv), **f32) if want_init_grad else None)
+    for name, t, shape in zip(("grad_q", "grad_k", "grad_v", "grad_g", "grad_init_state"), grads,
+                              ((B, N, heads, dk), (B, N, heads, dk), (B, N, heads, dv), (B, N, heads, dk),
+                               (B, heads, dk, dv))):
+        if t is not None and (t.dtype != torch.float32 or not t.is_contiguous() or tuple(t.shape) != shape
+                              or t.device != q.device):
+            raise ValueError(f"{name} must be a contiguous float32 {list(shape)} tensor on q's device")
+    if workspace is None:
+        workspace = new_workspace(bwd_workspace_bytes(B, heads, Hgrid, Wgrid, dk, dv, chunk), q.device)
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    nbytes = workspace.numel() * workspace.element_size()
+    gq, gk, gv, gg, gs = grads
+    st = lib.gtr_gla_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(d_out), _ptr(init_state),
+                         _ptr(d_final_state), B, heads, Hgrid, Wgrid, dk, dv, int(direction), int(chunk),
+                         _ptr(gq), _ptr(gk), _ptr(gv), _ptr(gg), _ptr(gs), _ptr(workspace), nbytes,
+                         _stream_handle(stream))
+    if st != GTR_OK:
+        raise GTRError(st, "gtr_gla_bwd")
+    return grads
 
 
 def gtr_gla_fwd_raw(q_ptr: int, k_ptr: int, v_ptr: int, g_ptr: int, B: int, heads: int,

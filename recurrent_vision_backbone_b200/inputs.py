@@ -136,6 +136,20 @@ def workload_inputs(w: Workload, direction: int, call: int = 0, device="cpu"):
                        device=device)
 
 
+def make_upstream(B: int, heads: int, H: int, W: int, dk: int, dv: int, seed: int,
+                  with_dsf: bool = True, device="cpu"):
+    """Upstream gradients for the backward pass: d_out = dL/do (fp16 [B,N,heads,dv]) and
+    d_final_state = dL/dS_final (fp32 [B,heads,dk,dv] or None), both N(0, 1) -- the scale
+    of a squared-L2 loss's gradient on unit-scale features (the pages distil with such a
+    loss).  Drawn from their own generator, seeded `seed` + 7, after the forward inputs."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(int(seed) + 7)
+    kw = dict(generator=gen, device=device, dtype=torch.float32)
+    d_out = torch.randn((B, H * W, heads, dv), **kw).half()
+    dsf = torch.randn((B, heads, dk, dv), **kw) if with_dsf else None
+    return d_out, dsf
+
+
 # ------------------------------------------------------------------ Spatial SwiGLU
 # Inputs of the gated value branch (gtr_spatial_swiglu_gate): the gate and up
 # projections G, U of a block's tokens and the depthwise kernel.  The pages give no

@@ -223,7 +223,7 @@ MUTANTS = {
     "own_output_term_dropped": ("G[(long)i * dv + j] += qt[i] * dot[j];",
                                 "G[(long)i * dv + j] += 0.0 * qt[i] * dot[j];"),
     # chain rule through a = exp(g) forgotten
-    "dg_without_a": ("dg[row * dk + i] = a[i] * sa;", "dg[row * dk + i] = sa;"),
+    "dg_without_a": ("dg[row * dk + i] = at * sa;", "dg[row * dk + i] = sa;"),
     # dg paired with the state after the update
     "dg_uses_current_state": ("sa += G[(long)i * dv + j] * Sprev[(long)i * dv + j];",
                               "sa += G[(long)i * dv + j] * St[(long)i * dv + j];"),
