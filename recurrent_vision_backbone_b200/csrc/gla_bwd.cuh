@@ -35,7 +35,7 @@ namespace gtr {
 namespace bw {
 
 constexpr int kC = 64;                 // chunk length
-constexpr int kLd = 65;                // shared row stride (floats): conflict-free columns
+constexpr int kLd = 68;                // shared row stride (floats): 16-byte rows for vector loads
 constexpr int kMat = kC * kLd;         // floats per shared 64 x 64 matrix
 constexpr int kThreads = 256;
 constexpr float kFastRange = 60.f;     // chunk log-decay above which e^{-b} stays finite
@@ -47,7 +47,7 @@ struct Args {
     float *dq, *dk, *dg;         // [rows][ldk], at the key half
     float *dv;                   // [rows][64]
     float *ds0;                  // like s0, or null
-    float *hs, *dhs;             // workspace: [n_seq][nc][64][64] U -> h_c, W -> dh_{c+1}
+    float *hs, *dhs;             // workspace: U -> h_c, W -> dh_{c+1} tiles (layout: tile_idx)
     float *bc, *xc;              // workspace: [n_seq][nc][64] chunk log-decay, chunk x totals
     float *cst;                  // workspace: [n_seq][64]
     int heads, H, W, N, dir, n_seq, nc, ldk, sstride;
@@ -61,74 +61,132 @@ __device__ __forceinline__ int bwd_row(const Args &a, int seq, int p) {
     return (bb * a.N + scan_to_token(p, a.H, a.W, a.dir)) * a.heads + hh;
 }
 
-// 64 rows x 64 fp16 channels (row r at token row rows[r], pitch ld) -> fp32 dst[r][c];
-// rows past the grid are zero.
-__device__ __forceinline__ void load_tile_h(const __half *src, int ld, const int *rows, float *dst) {
-    for (int x = threadIdx.x; x < kC * 8; x += kThreads) {
-        const int r = x >> 3, c8 = x & 7, ro = rows[r];
-        float f[8];
-        if (ro >= 0) {
-            const uint4 u = *reinterpret_cast<const uint4 *>(src + (size_t)ro * ld + 8 * c8);
-            const __half2 *h2 = reinterpret_cast<const __half2 *>(&u);
+// Workspace position of element e = i * 64 + j of sequence seq's chunk-c state tile:
+// [seq][e / 32][chunk][e % 32], so that one warp's 32 elements over consecutive chunks
+// are consecutive 128-byte lines (the scans walk the chunks; the chunk kernels still
+// read or write whole 128-byte lines).
+__device__ __forceinline__ size_t tile_idx(int nc, int seq, int c, int e) {
+    return (((size_t)seq * 128 + (e >> 5)) * nc + c) * 32 + (e & 31);
+}
+
+// Keeps the compiler from moving memory accesses across this point: the loads issued
+// before it are all in flight before the first one is waited for.
+__device__ __forceinline__ void issue_fence() { asm volatile("" ::: "memory"); }
+
+// 64 rows x 64 fp16 channels (row r at token row rows[r], pitch ld): this thread's two
+// 16-byte pieces (x = tid, tid + 256: row x / 8, channels 8 (x % 8) ..), zero past the
+// grid; then stored as fp32 into dst[r][c].
+struct HalfTile {
+    uint4 p[2];
+};
+__device__ __forceinline__ void issue_tile_h(const __half *src, int ld, const int *rows, HalfTile &t) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 p = __half22float2(h2[e]);
-                f[2 * e] = p.x;
-                f[2 * e + 1] = p.y;
-            }
-        } else {
+    for (int m = 0; m < 2; ++m) {
+        const int x = threadIdx.x + kThreads * m, ro = rows[x >> 3];
+        t.p[m] = ro >= 0 ? *reinterpret_cast<const uint4 *>(src + (size_t)ro * ld + 8 * (x & 7))
+                         : make_uint4(0u, 0u, 0u, 0u);
+    }
+}
+__device__ __forceinline__ void store_tile_h(const HalfTile &t, float *dst) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] = 0.f;
-        }
-#pragma unroll
-        for (int e = 0; e < 8; ++e) dst[r * kLd + 8 * c8 + e] = f[e];
+    for (int m = 0; m < 2; ++m) {
+        const int x = threadIdx.x + kThreads * m;
+        const __half2 *h2 = reinterpret_cast<const __half2 *>(&t.p[m]);
+        const float2 f0 = __half22float2(h2[0]), f1 = __half22float2(h2[1]);
+        const float2 f2 = __half22float2(h2[2]), f3 = __half22float2(h2[3]);
+        float4 *d4 = reinterpret_cast<float4 *>(dst + (x >> 3) * kLd + 8 * (x & 7));
+        d4[0] = make_float4(f0.x, f0.y, f1.x, f1.y);
+        d4[1] = make_float4(f2.x, f2.y, f3.x, f3.y);
     }
 }
 
-// A 64 x 64 fp32 matrix, row-major in global memory -> dst[r][c].
-__device__ __forceinline__ void load_tile_f(const float *src, float *dst) {
-    for (int x = threadIdx.x; x < kC * 16; x += kThreads) {
-        const int r = x >> 4, c4 = x & 15;
-        const float4 u = *reinterpret_cast<const float4 *>(src + r * 64 + 4 * c4);
-        dst[r * kLd + 4 * c4] = u.x;
-        dst[r * kLd + 4 * c4 + 1] = u.y;
-        dst[r * kLd + 4 * c4 + 2] = u.z;
-        dst[r * kLd + 4 * c4 + 3] = u.w;
+// A chunk's 64 x 64 fp32 state tile from the workspace: this thread's four 16-byte
+// pieces (elements 4 x .. 4 x + 3, x = tid + 256 m), then stored into dst[i][j].
+struct StateTile {
+    float4 p[4];
+};
+__device__ __forceinline__ void issue_state_tile(const float *src, int nc, int seq, int c, StateTile &t) {
+#pragma unroll
+    for (int m = 0; m < 4; ++m)
+        t.p[m] = *reinterpret_cast<const float4 *>(src + tile_idx(nc, seq, c, 4 * (threadIdx.x + kThreads * m)));
+}
+__device__ __forceinline__ void store_state_tile(const StateTile &t, float *dst) {
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        const int e = 4 * (threadIdx.x + kThreads * m);
+        *reinterpret_cast<float4 *>(dst + (e >> 6) * kLd + (e & 63)) = t.p[m];
     }
 }
 
 // Running sum of g down each channel (64 threads): b[t][i] over the chunk; returns B.
+// The column is read into registers first, so the chain is register adds only.
 __device__ __forceinline__ void chunk_cumsum(float *b, float *Bv) {
     if (threadIdx.x < kC) {
         const int i = threadIdx.x;
+        float col[kC];
+#pragma unroll
+        for (int t = 0; t < kC; ++t) col[t] = b[t * kLd + i];
         float s = 0.f;
+#pragma unroll
         for (int t = 0; t < kC; ++t) {
-            s += b[t * kLd + i];
+            s += col[t];
             b[t * kLd + i] = s;
         }
         Bv[i] = s;
     }
 }
 
-// Register tile of a 64 x 64 product: thread (ty, tx) = (tid / 16, tid % 16) owns rows
-// ty + 16 a and columns tx + 16 b.  Operand element (r, k) of a row-major matrix M is
-// M[r * kLd + k]; of a transposed one, M[k * kLd + r].
-template <bool kTA, bool kTB>
+// Register tile of a 64 x 64 product, k in steps of four: thread (ty, tx) = (tid / 16,
+// tid % 16) owns rows 4 ty + u and columns 4 tx + w (kColVec) or tx + 16 w.  Operand
+// element (r, k) of a row-major matrix M is M[r * kLd + k]; of a transposed one,
+// M[k * kLd + r].  Every A read is a 16-byte vector (four k of one row, or four rows of
+// one k); B reads are vectors where its layout and the column mapping line up (rows of
+// a transposed B with columns tx + 16 w; a row-major B with columns 4 tx + w).
+__device__ __forceinline__ int mm_row(int u) { return 4 * (threadIdx.x >> 4) + u; }
+template <bool kColVec>
+__device__ __forceinline__ int mm_col(int w) {
+    const int tx = threadIdx.x & 15;
+    return kColVec ? 4 * tx + w : tx + 16 * w;
+}
+
+template <bool kTA, bool kTB, bool kColVec>
 __device__ __forceinline__ void mm_acc(const float *A, const float *B, float (&acc)[4][4]) {
     const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
-#pragma unroll 4
-    for (int kk = 0; kk < kC; ++kk) {
-        float a[4], b[4];
+#pragma unroll 2
+    for (int kk = 0; kk < kC; kk += 4) {
+        float a[4][4], b[4][4];   // a[u][q]: row u, k = kk + q;  b[q][w]: k = kk + q, column w
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int r = ty + 16 * u, c = tx + 16 * u;
-            a[u] = kTA ? A[kk * kLd + r] : A[r * kLd + kk];
-            b[u] = kTB ? B[c * kLd + kk] : B[kk * kLd + c];
+        for (int x = 0; x < 4; ++x) {
+            if (kTA) {
+                const float4 v = *reinterpret_cast<const float4 *>(A + (kk + x) * kLd + 4 * ty);
+                a[0][x] = v.x; a[1][x] = v.y; a[2][x] = v.z; a[3][x] = v.w;
+            } else {
+                const float4 v = *reinterpret_cast<const float4 *>(A + (4 * ty + x) * kLd + kk);
+                a[x][0] = v.x; a[x][1] = v.y; a[x][2] = v.z; a[x][3] = v.w;
+            }
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
+        for (int x = 0; x < 4; ++x) {
+            if (kTB && !kColVec) {
+                const float4 v = *reinterpret_cast<const float4 *>(B + (tx + 16 * x) * kLd + kk);
+                b[0][x] = v.x; b[1][x] = v.y; b[2][x] = v.z; b[3][x] = v.w;
+            } else if (!kTB && kColVec) {
+                const float4 v = *reinterpret_cast<const float4 *>(B + (kk + x) * kLd + 4 * tx);
+                b[x][0] = v.x; b[x][1] = v.y; b[x][2] = v.z; b[x][3] = v.w;
+            } else {
 #pragma unroll
-            for (int w = 0; w < 4; ++w) acc[u][w] = fmaf(a[u], b[w], acc[u][w]);
+                for (int w = 0; w < 4; ++w) {
+                    const int c = mm_col<kColVec>(w);
+                    b[x][w] = kTB ? B[c * kLd + kk + x] : B[(kk + x) * kLd + c];
+                }
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int w = 0; w < 4; ++w) acc[u][w] = fmaf(a[u][q], b[q][w], acc[u][w]);
     }
 }
 
@@ -150,11 +208,20 @@ __global__ void __launch_bounds__(kThreads) gla_bwd_local_kernel(const Args a) {
     const int seq = (int)(blockIdx.x / a.nc), c = (int)(blockIdx.x % a.nc);
     if (tid < kC) rows[tid] = bwd_row(a, seq, c * kC + tid);
     __syncthreads();
-    load_tile_h(a.k, a.ldk, rows, ks);
-    load_tile_h(a.q, a.ldk, rows, qs);
-    load_tile_h(a.g, a.ldk, rows, bs);
-    load_tile_h(a.v, 64, rows, vs);
-    load_tile_h(a.dout, 64, rows, ds);
+    {
+        HalfTile tk, tq, tg, tv, td;   // every load in flight before the first store
+        issue_tile_h(a.k, a.ldk, rows, tk);
+        issue_tile_h(a.q, a.ldk, rows, tq);
+        issue_tile_h(a.g, a.ldk, rows, tg);
+        issue_tile_h(a.v, 64, rows, tv);
+        issue_tile_h(a.dout, 64, rows, td);
+        issue_fence();
+        store_tile_h(tk, ks);
+        store_tile_h(tq, qs);
+        store_tile_h(tg, bs);
+        store_tile_h(tv, vs);
+        store_tile_h(td, ds);
+    }
     __syncthreads();
     chunk_cumsum(bs, Bv);
     __syncthreads();
@@ -170,30 +237,27 @@ __global__ void __launch_bounds__(kThreads) gla_bwd_local_kernel(const Args a) {
     float u[4][4], w[4][4];
     zero4x4(u);
     zero4x4(w);
-    mm_acc<true, false>(ks, vs, u);   // U[i][j] = sum_s kB[s][i] v[s][j]
-    mm_acc<true, false>(qs, ds, w);   // W[i][j] = sum_t qe[t][i] dO[t][j]
-    const int ty = tid >> 4, tx = tid & 15;
-    float *uo = a.hs + cidx * 4096, *wo = a.dhs + cidx * 4096;
+    mm_acc<true, false, true>(ks, vs, u);   // U[i][j] = sum_s kB[s][i] v[s][j]
+    mm_acc<true, false, true>(qs, ds, w);   // W[i][j] = sum_t qe[t][i] dO[t][j]
 #pragma unroll
-    for (int p = 0; p < 4; ++p)
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            uo[(ty + 16 * p) * 64 + tx + 16 * r] = u[p][r];
-            wo[(ty + 16 * p) * 64 + tx + 16 * r] = w[p][r];
-        }
+    for (int p = 0; p < 4; ++p) {   // columns 4 tx .. 4 tx + 3: one 16-byte store each
+        const size_t o = tile_idx(a.nc, seq, c, mm_row(p) * 64 + mm_col<true>(0));
+        *reinterpret_cast<float4 *>(a.hs + o) = make_float4(u[p][0], u[p][1], u[p][2], u[p][3]);
+        *reinterpret_cast<float4 *>(a.dhs + o) = make_float4(w[p][0], w[p][1], w[p][2], w[p][3]);
+    }
 }
 
 // ---------------------------------------------------------------- K2: chunk scans
 // grid n_seq * 16, 256 threads: thread e of the sequence's 4096 state elements
 // (i = e / 64, j = e % 64).  Loads run kPre chunks ahead of the chain.
-constexpr int kPre = 8;
+constexpr int kPre = 32;
 
 __global__ void __launch_bounds__(kThreads) gla_bwd_scan_kernel(const Args a) {
     __shared__ float red[kThreads / 32];
     const int seq = (int)(blockIdx.x / 16);
     const int e = (int)(blockIdx.x % 16) * kThreads + threadIdx.x, i = e >> 6;
     const int nc = a.nc;
-    const size_t base = (size_t)seq * nc * 4096 + e;
+    const size_t base = tile_idx(nc, seq, 0, e);   // + 32 per chunk
     const float *bc = a.bc + (size_t)seq * nc * kC + i;
     const size_t so = (size_t)seq * a.sstride + e;   // (i, j) at i * 64 + j
     // forward: U_c -> h_c (the state entering chunk c)
@@ -203,14 +267,15 @@ __global__ void __launch_bounds__(kThreads) gla_bwd_scan_kernel(const Args a) {
 #pragma unroll
         for (int r = 0; r < kPre; ++r)
             if (c0 + r < nc) {
-                uu[r] = a.hs[base + (size_t)(c0 + r) * 4096];
-                dd[r] = __expf(bc[(size_t)(c0 + r) * kC]);
+                uu[r] = a.hs[base + (size_t)(c0 + r) * 32];
+                dd[r] = bc[(size_t)(c0 + r) * kC];
             }
+        issue_fence();
 #pragma unroll
         for (int r = 0; r < kPre; ++r)
             if (c0 + r < nc) {
-                a.hs[base + (size_t)(c0 + r) * 4096] = h;
-                h = fmaf(dd[r], h, uu[r]);
+                a.hs[base + (size_t)(c0 + r) * 32] = h;
+                h = fmaf(__expf(dd[r]), h, uu[r]);
             }
     }
     // const[i] = sum_j dS_f[i][j] S_final[i][j]: the row's 64 elements are warps 2 r, 2 r + 1
@@ -230,14 +295,15 @@ __global__ void __launch_bounds__(kThreads) gla_bwd_scan_kernel(const Args a) {
 #pragma unroll
         for (int r = 0; r < kPre; ++r)
             if (c1 - r >= 0) {
-                ww[r] = a.dhs[base + (size_t)(c1 - r) * 4096];
-                dd[r] = __expf(bc[(size_t)(c1 - r) * kC]);
+                ww[r] = a.dhs[base + (size_t)(c1 - r) * 32];
+                dd[r] = bc[(size_t)(c1 - r) * kC];
             }
+        issue_fence();
 #pragma unroll
         for (int r = 0; r < kPre; ++r)
             if (c1 - r >= 0) {
-                a.dhs[base + (size_t)(c1 - r) * 4096] = d;
-                d = fmaf(dd[r], d, ww[r]);
+                a.dhs[base + (size_t)(c1 - r) * 32] = d;
+                d = fmaf(__expf(dd[r]), d, ww[r]);
             }
     }
     if (a.ds0) a.ds0[so] = d;
@@ -257,18 +323,30 @@ __global__ void __launch_bounds__(kThreads) gla_bwd_grad_kernel(const Args a) {
     __shared__ int rows[kC];
     __shared__ float Bv[kC];
     __shared__ int fast[kC];
-    const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+    const int tid = threadIdx.x;
     const int seq = (int)(blockIdx.x / a.nc), c = (int)(blockIdx.x % a.nc);
     const size_t cidx = (size_t)seq * a.nc + c;
     if (tid < kC) rows[tid] = bwd_row(a, seq, c * kC + tid);
     __syncthreads();
-    load_tile_h(a.q, a.ldk, rows, qs);
-    load_tile_h(a.k, a.ldk, rows, ks);
-    load_tile_h(a.g, a.ldk, rows, bs);
-    load_tile_h(a.v, 64, rows, vs);
-    load_tile_h(a.dout, 64, rows, ds);
-    load_tile_f(a.hs + cidx * 4096, hc);
-    load_tile_f(a.dhs + cidx * 4096, dh);
+    {
+        HalfTile tq, tk, tg, tv, td;   // every load in flight before the first store
+        StateTile th, tdh;
+        issue_tile_h(a.q, a.ldk, rows, tq);
+        issue_tile_h(a.k, a.ldk, rows, tk);
+        issue_tile_h(a.g, a.ldk, rows, tg);
+        issue_tile_h(a.v, 64, rows, tv);
+        issue_tile_h(a.dout, 64, rows, td);
+        issue_state_tile(a.hs, a.nc, seq, c, th);
+        issue_state_tile(a.dhs, a.nc, seq, c, tdh);
+        issue_fence();
+        store_tile_h(tq, qs);
+        store_tile_h(tk, ks);
+        store_tile_h(tg, bs);
+        store_tile_h(tv, vs);
+        store_tile_h(td, ds);
+        store_state_tile(th, hc);
+        store_state_tile(tdh, dh);
+    }
     __syncthreads();
     chunk_cumsum(bs, Bv);
     __syncthreads();
@@ -289,13 +367,13 @@ __global__ void __launch_bounds__(kThreads) gla_bwd_grad_kernel(const Args a) {
         float d[4][4], m[4][4];
         zero4x4(d);
         zero4x4(m);
-        mm_acc<false, true>(ds, vs, d);
-        mm_acc<false, true>(qh, kh, m);
+        mm_acc<false, true, false>(ds, vs, d);
+        mm_acc<false, true, false>(qh, kh, m);
 #pragma unroll
         for (int p = 0; p < 4; ++p)
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
-                const int t = ty + 16 * p, s = tx + 16 * r;
+                const int t = mm_row(p), s = mm_col<false>(r);
                 Dm[t * kLd + s] = s <= t ? d[p][r] : 0.f;
                 Am[t * kLd + s] = s <= t ? m[p][r] : 0.f;
             }
@@ -317,18 +395,19 @@ __global__ void __launch_bounds__(kThreads) gla_bwd_grad_kernel(const Args a) {
     {
         float acc[4][4];
         zero4x4(acc);
-        mm_acc<true, false>(Am, ds, acc);   // sum_t A[t][s] dO[t][j]
-        mm_acc<false, false>(kB, dh, acc);  // sum_i kB[s][i] dh[i][j]
+        mm_acc<true, false, true>(Am, ds, acc);    // sum_t A[t][s] dO[t][j]
+        mm_acc<false, false, true>(kB, dh, acc);   // sum_i kB[s][i] dh[i][j]
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
-            const int s = ty + 16 * p, ro = rows[s];
+        for (int p = 0; p < 4; ++p) {   // columns 4 tx .. 4 tx + 3 of row s: one 16-byte access
+            const int s = mm_row(p), ro = rows[s];
             if (ro < 0) continue;
-            float *dst = a.dv + (size_t)ro * 64;
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const int j = tx + 16 * r;
-                dst[j] = a.acc_dv ? dst[j] + acc[p][r] : acc[p][r];
+            float4 *dst = reinterpret_cast<float4 *>(a.dv + (size_t)ro * 64 + mm_col<true>(0));
+            float4 v = make_float4(acc[p][0], acc[p][1], acc[p][2], acc[p][3]);
+            if (a.acc_dv) {
+                const float4 o = *dst;
+                v.x += o.x; v.y += o.y; v.z += o.z; v.w += o.w;
             }
+            *dst = v;
         }
     }
     // dq (rows t, channels i) and dk (rows s, channels i), kept in registers until the
@@ -337,17 +416,17 @@ __global__ void __launch_bounds__(kThreads) gla_bwd_grad_kernel(const Args a) {
     zero4x4(xq);
     zero4x4(y1);
     zero4x4(y2);
-    mm_acc<false, true>(ds, hc, xq);    // sum_j dO[t][j] h_c[i][j]
-    mm_acc<false, false>(Dm, kh, xq);   // sum_s D[t][s] kh[s][i]
-    mm_acc<false, true>(vs, dh, y1);    // sum_j v[s][j] dh[i][j]
-    mm_acc<true, false>(Dm, qh, y2);    // sum_t D[t][s] qh[t][i]
+    mm_acc<false, true, false>(ds, hc, xq);    // sum_j dO[t][j] h_c[i][j]
+    mm_acc<false, false, false>(Dm, kh, xq);   // sum_s D[t][s] kh[s][i]
+    mm_acc<false, true, false>(vs, dh, y1);    // sum_j v[s][j] dh[i][j]
+    mm_acc<true, false, false>(Dm, qh, y2);    // sum_t D[t][s] qh[t][i]
     __syncthreads();   // every product is done: hc and vs now hold dq and dk
     float *dqs = hc, *dks = vs;
 #pragma unroll
     for (int p = 0; p < 4; ++p)
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
-            const int t = ty + 16 * p, i = tx + 16 * r;
+            const int t = mm_row(p), i = mm_col<false>(r);   // (row t of dq, row s = t of dk)
             const float b = bs[t * kLd + i];
             dqs[t * kLd + i] = __expf(b) * xq[p][r];
             dks[t * kLd + i] = __expf(Bv[i] - b) * y1[p][r] + (fast[i] ? __expf(-b) * y2[p][r] : 0.f);
@@ -376,9 +455,13 @@ __global__ void __launch_bounds__(kThreads) gla_bwd_grad_kernel(const Args a) {
     }
     __syncthreads();
     if (tid < kC) {
+        float col[kC];
+#pragma unroll
+        for (int t = 0; t < kC; ++t) col[t] = xs[t * kLd + tid];
         float s = 0.f;
+#pragma unroll
         for (int t = kC - 1; t >= 0; --t) {
-            s += xs[t * kLd + tid];
+            s += col[t];
             xs[t * kLd + tid] = s;
         }
         a.xc[cidx * kC + tid] = s;
@@ -404,18 +487,40 @@ __global__ void __launch_bounds__(kThreads) gla_bwd_grad_kernel(const Args a) {
 }
 
 // ---------------------------------------------------------------- K4: dg offsets
-// grid n_seq * nc, 64 threads (one per channel): dg of the chunk's rows += const + the
-// x totals of the later chunks of the sequence.
-__global__ void __launch_bounds__(kC) gla_bwd_dg_kernel(const Args a) {
-    const int i = threadIdx.x;
+// grid n_seq * nc, 256 threads: dg of the chunk's rows += const + the x totals of the
+// later chunks of the sequence.  Channel i = tid % 64; the four quarters of the block
+// sum every fourth later chunk (independent loads in flight), then each thread updates
+// sixteen rows, every load issued before any store.
+__global__ void __launch_bounds__(kThreads) gla_bwd_dg_kernel(const Args a) {
+    __shared__ int rows[kC];
+    __shared__ float part[4][kC];
+    const int tid = threadIdx.x, i = tid & 63, qq = tid >> 6;
     const int seq = (int)(blockIdx.x / a.nc), c = (int)(blockIdx.x % a.nc);
-    float off = a.cst[(size_t)seq * kC + i];
+    if (tid < kC) rows[tid] = bwd_row(a, seq, c * kC + tid);
     const float *xc = a.xc + (size_t)seq * a.nc * kC + i;
-    for (int c2 = c + 1; c2 < a.nc; ++c2) off += xc[(size_t)c2 * kC];
-    const int nrows = min(kC, a.N - c * kC);
-    for (int t = 0; t < nrows; ++t) {
-        const int ro = bwd_row(a, seq, c * kC + t);
-        a.dg[(size_t)ro * a.ldk + i] += off;
+    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+    int c2 = c + 1 + qq;
+    for (; c2 + 12 < a.nc; c2 += 16) {
+        s0 += xc[(size_t)c2 * kC];
+        s1 += xc[(size_t)(c2 + 4) * kC];
+        s2 += xc[(size_t)(c2 + 8) * kC];
+        s3 += xc[(size_t)(c2 + 12) * kC];
+    }
+    for (; c2 < a.nc; c2 += 4) s0 += xc[(size_t)c2 * kC];
+    part[qq][i] = (s0 + s1) + (s2 + s3);
+    __syncthreads();
+    const float off = a.cst[(size_t)seq * kC + i] + ((part[0][i] + part[1][i]) + (part[2][i] + part[3][i]));
+    float v[16];
+#pragma unroll
+    for (int m = 0; m < 16; ++m) {
+        const int ro = rows[qq + 4 * m];
+        v[m] = ro >= 0 ? a.dg[(size_t)ro * a.ldk + i] : 0.f;
+    }
+    issue_fence();
+#pragma unroll
+    for (int m = 0; m < 16; ++m) {
+        const int ro = rows[qq + 4 * m];
+        if (ro >= 0) a.dg[(size_t)ro * a.ldk + i] = v[m] + off;
     }
 }
 

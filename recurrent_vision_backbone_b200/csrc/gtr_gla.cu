@@ -1124,7 +1124,7 @@ static cudaError_t bwd_launch(const bw::Args &a, cudaStream_t stream) {
     bw::gla_bwd_local_kernel<<<chunks, bw::kThreads, smem1, stream>>>(a);
     bw::gla_bwd_scan_kernel<<<(unsigned)a.n_seq * 16u, bw::kThreads, 0, stream>>>(a);
     bw::gla_bwd_grad_kernel<<<chunks, bw::kThreads, bw::kGradSmem, stream>>>(a);
-    bw::gla_bwd_dg_kernel<<<chunks, bw::kC, 0, stream>>>(a);
+    bw::gla_bwd_dg_kernel<<<chunks, bw::kThreads, 0, stream>>>(a);
     return cudaGetLastError();
 }
 

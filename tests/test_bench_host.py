@@ -23,3 +23,14 @@ def test_recorded_traffic_matches_current_source():
         # either the summary was taken on this code (a positive byte count) or it is
         # reported as unknown; never a stale number
         assert t is None or t > 0
+
+
+def test_backward_bytes_alg():
+    # read q, k, g, v, d_out in fp16 and write the four gradients in fp32: 1664 B per
+    # token-head at dk = dv = 64, plus the fp32 states (init_state, d_final_state read,
+    # grad_init_state written)
+    w = bench.WORKLOADS["hires_b1h16_128x128"]
+    th = w.B * w.N * w.heads
+    assert bench.bwd_bytes_alg(w) == th * 1664 + 3 * w.B * w.heads * 64 * 64 * 4
+    w2 = bench.WORKLOADS["gtr640_b1h16_40x40"]   # no initial state: d_final_state and grad_init_state
+    assert bench.bwd_bytes_alg(w2) == w2.B * w2.N * w2.heads * 1664 + 2 * w2.B * w2.heads * 64 * 64 * 4
