@@ -632,7 +632,7 @@ def run_workload(name, steps, warmup, stream, world, rank, device, sets, sample_
                  clocks_csv=None, gate_z=False):
     """Times `steps` steps of one workload; returns its numbers and its config.  gate_z:
     through gtr_gla_fwd_z (the gate's pre-activation z read in place of g: the same
-    bytes, the gate formed while staging)."""
+    bytes, the gate formed in the kernel)."""
     w = WORKLOADS[name]
     wl = Workload(w, rank, device, n_sets=sets, gate_z=gate_z)
     clocks = None

@@ -111,7 +111,7 @@ gtr_status_t gtr_gla_fwd(const gtr_half_t *q, const gtr_half_t *k, const gtr_hal
  * gtr_gla_fwd with the forget gate given by its pre-activation: the third input z
  * (IEEE binary16 [B, N, heads, dk], in place of g) and the temperature tau > 0; the
  * kernel forms g = log(sigmoid(z)) / tau = (min(z, 0) - log(1 + exp(-|z|))) / tau in
- * fp32 while it stages each chunk (GTR news article, section "线性注意力到底在省什么":
+ * fp32 wherever it reads the gate of a chunk (GTR news article, section "线性注意力到底在省什么":
  * a learnable forget gate on the key side), so no separate pass over z runs and g is
  * never rounded to fp16.  Same arguments, layouts, workspace and errors as gtr_gla_fwd,
  * plus GTR_ERR_INVALID_ARG for tau <= 0 or not finite.

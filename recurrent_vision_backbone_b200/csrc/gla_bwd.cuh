@@ -249,7 +249,8 @@ __global__ void __launch_bounds__(kThreads) gla_bwd_local_kernel(const Args a) {
 
 // ---------------------------------------------------------------- K2: chunk scans
 // grid n_seq * 16, 256 threads: thread e of the sequence's 4096 state elements
-// (i = e / 64, j = e % 64).  Loads run kPre chunks ahead of the chain.
+// (i = e / 64, j = e % 64), walking the chunks in batches of kPre: every load of a
+// batch is in flight before the chain uses the first (one memory latency per batch).
 constexpr int kPre = 32;
 
 __global__ void __launch_bounds__(kThreads) gla_bwd_scan_kernel(const Args a) {

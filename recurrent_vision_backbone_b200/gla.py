@@ -162,7 +162,7 @@ def gtr_gla_fwd(q, k, v, g, Hgrid: int, Wgrid: int, direction: int, init_state=N
 def gtr_gla_fwd_z(q, k, v, z, tau: float, Hgrid: int, Wgrid: int, direction: int,
                   init_state=None, out=None, final_state=None, chunk: int = 64, stream=None):
     """gtr_gla_fwd with the gate's pre-activation z (fp16, the layout of g) and its
-    temperature tau: the kernel forms g = log(sigmoid(z)) / tau while staging."""
+    temperature tau: the kernel forms g = log(sigmoid(z)) / tau in fp32 wherever it reads the gate."""
     (B, heads, dk, dv), out, final_state = _prepare(q, k, v, z, Hgrid, Wgrid, init_state, out,
                                                     final_state)
     st = load().gtr_gla_fwd_z(_ptr(q), _ptr(k), _ptr(v), _ptr(z), ctypes.c_float(tau), B, heads,
