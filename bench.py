@@ -455,7 +455,7 @@ class BwdBench:
     per step, each with its own inputs, upstream gradients and gradient outputs; one
     workspace, the calls being stream-ordered), replayed from CUDA graphs."""
 
-    def __init__(self, w, device, n_sets=None):
+    def __init__(self, w, device, n_sets=None, rank=0):
         from recurrent_vision_backbone_b200 import gla
         from recurrent_vision_backbone_b200.inputs import make_upstream
         self.gla = gla
@@ -470,7 +470,7 @@ class BwdBench:
         for s in range(self.n_sets):
             calls = []
             for d in w.directions:
-                seed = w.seed(d, 300 + s)
+                seed = rank_seed(w.seed(d, 300 + s), rank)   # each rank its own batch
                 inp = make_inputs(w.B, w.heads, w.H, w.W, w.dk, w.dv, seed=seed, init_std=w.init_std,
                                   z_mean_per_head=w.z_mean_per_head, device=device)
                 d_out, dsf = make_upstream(w.B, w.heads, w.H, w.W, w.dk, w.dv, seed, with_dsf=w.final_state,
@@ -499,9 +499,9 @@ class BwdBench:
 BWD_KERNELS_PER_CALL = 4   # chunk locals, state scans, chunk gradients, dg offsets
 
 
-def run_bwd(name, steps, warmup, stream, world, device, sets, local):
+def run_bwd(name, steps, warmup, stream, world, device, sets, local, rank=0):
     w = WORKLOADS[name]
-    bb = BwdBench(w, device, n_sets=sets)
+    bb = BwdBench(w, device, n_sets=sets, rank=rank)
     clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else local)
     ms, n_steps, clk = measure(bb, steps, warmup, stream, world, clocks)
     peak, which = measured_peaks()
@@ -703,7 +703,7 @@ def gpu_arm(args):
                                                 stream, world, device, None, local))
         for name in BWD_WORKLOADS:   # the backward pass
             line["secondary"].append(run_bwd(name, max(8, min(200, args.steps // 16)), 3, stream, world,
-                                             device, None, local))
+                                             device, None, local, rank=rank))
     # end to end through the public call with host buffers
     e_steps = max(3, min(args.steps, args.e2e_steps))
     ems, en, h2d, d2h = e2e_measure(w1, e_steps, device, rank)
