@@ -39,6 +39,9 @@ constexpr int kLd = 68;                // shared row stride (floats): 16-byte ro
 constexpr int kMat = kC * kLd;         // floats per shared 64 x 64 matrix
 constexpr int kThreads = 256;
 constexpr float kFastRange = 60.f;     // chunk log-decay above which e^{-b} stays finite
+// Floor of a log-decay: below about -104, a = exp(g) is 0 in fp32 already; the floor keeps
+// the running sums and their differences finite when a gate is exactly 0 (g = -inf).
+constexpr float kMinLogDecay = -1e4f;
 
 struct Args {
     const __half *q, *k, *g;     // [rows][ldk], at the key half
@@ -118,14 +121,15 @@ __device__ __forceinline__ void store_state_tile(const StateTile &t, float *dst)
     }
 }
 
-// Running sum of g down each channel (64 threads): b[t][i] over the chunk; returns B.
-// The column is read into registers first, so the chain is register adds only.
+// Running sum of g down each channel (64 threads): b[t][i] over the chunk, each g floored
+// at kMinLogDecay; returns B.  The column is read into registers first, so the chain is
+// register adds only.
 __device__ __forceinline__ void chunk_cumsum(float *b, float *Bv) {
     if (threadIdx.x < kC) {
         const int i = threadIdx.x;
         float col[kC];
 #pragma unroll
-        for (int t = 0; t < kC; ++t) col[t] = b[t * kLd + i];
+        for (int t = 0; t < kC; ++t) col[t] = fmaxf(b[t * kLd + i], kMinLogDecay);
         float s = 0.f;
 #pragma unroll
         for (int t = 0; t < kC; ++t) {

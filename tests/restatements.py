@@ -222,7 +222,7 @@ def chunkwise_backward(q, k, v, g, dout, H, W, direction, s0=None, dsf=None, chu
                 fast = Bv >= -fast_range
                 D = (DO @ V.T) * mask
                 qh = np.where(fast, Q * np.exp(bb), 0.0)
-                with np.errstate(over="ignore"):
+                with np.errstate(over="ignore", invalid="ignore"):
                     kh = np.where(fast, K * np.exp(-bb), 0.0)
                 A = (qh @ kh.T) * mask
                 dq_c = np.exp(bb) * (DO @ hs[c].T) + np.exp(bb) * (D @ kh)

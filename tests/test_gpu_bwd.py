@@ -5,14 +5,18 @@ The oracle differentiates the token recurrence position by position
 fp16 inputs and upstream gradients.  Cases: every direction on the 1.6K grid with an
 initial state and a final-state gradient, ragged grids (a partial last chunk), no
 state arguments, dk = 128 (two key halves, grad_v accumulated), strongly forgetting
-channels (the per-pair exponential path), grids shorter than a chunk, an empty grid,
-and sampled heads of the 16.4K workload at full length.
+channels (the per-pair exponential path), gates of exactly 0 and exactly 1, grids
+shorter than a chunk, an empty grid, and sampled heads of the 16.4K workload at full
+length.
 
 Tolerance: the kernels compute in fp32 from exact fp16 inputs; each gradient element is
 a sum of at most a few hundred products per chunk plus chunk-level state scans of at
 most a few hundred steps, each step with relative rounding of about 2^-22 (fp32 plus
 the exponential's couple of ulp), so the error stays below 2e-4 of the tensor's
-largest magnitude; that bound is asserted (and no element may be non-finite).
+largest magnitude; that bound is asserted (and no element may be non-finite).  grad_g
+sums q*dq - k*dk over the later positions, so its bound scales with the larger of its
+own magnitude and those terms' (with every gate 0 the sum cancels to zero exactly in
+fp64 and to rounding in fp32).
 """
 import numpy as np
 import pytest
@@ -27,8 +31,9 @@ REL = 2e-4
 
 
 def run_both(B, heads, H, W, dk, direction, seed, init_std=0.1, with_dsf=True, heads_sel=None,
-             z_mean_per_head=None, want_init_grad=True):
-    inp = make_inputs(B, heads, H, W, dk, 64, seed, init_std=init_std, z_mean_per_head=z_mean_per_head)
+             z_mean_per_head=None, want_init_grad=True, z_override=None):
+    inp = make_inputs(B, heads, H, W, dk, 64, seed, init_std=init_std, z_mean_per_head=z_mean_per_head,
+                      z_override=z_override)
     d_out, dsf = make_upstream(B, heads, H, W, dk, 64, seed, with_dsf=with_dsf)
     dev = torch.device("cuda", 0)
     t = {n: inp[n].to(dev) for n in ("q", "k", "v", "g")}
@@ -46,16 +51,19 @@ def run_both(B, heads, H, W, dk, direction, seed, init_std=0.1, with_dsf=True, h
                               None if dsf is None else dsf[:, sel].numpy())
     if heads_sel is not None:   # [B, N, heads, d] gradients, then [B, heads, dk, dv]
         got = [x[:, :, sel] for x in got[:4]] + [None if got[4] is None else got[4][:, sel]]
-    return got, ref
+    # dg sums q*dq - k*dk over the later positions: its rounding scales with those terms
+    terms = float(np.max(np.abs(f(inp["q"][:, :, sel]) * ref[0]), initial=0.0)
+                  + np.max(np.abs(f(inp["k"][:, :, sel]) * ref[1]), initial=0.0))
+    return got, ref + (terms,)
 
 
 def assert_close(got, ref):
     names = ("grad_q", "grad_k", "grad_v", "grad_g", "grad_init_state")
-    for name, x, r in zip(names, got, ref):
+    for name, x, r in zip(names, got, ref[:5]):
         if x is None:
             continue
         assert np.all(np.isfinite(x)), name
-        scale = max(float(np.max(np.abs(r))), 1e-30)
+        scale = max(float(np.max(np.abs(r))), ref[5] if name == "grad_g" else 0.0, 1e-30)
         err = float(np.max(np.abs(x - r))) / scale
         assert err <= REL, f"{name}: max|err| / max|ref| = {err:.2e} (> {REL})"
 
@@ -78,7 +86,7 @@ def test_no_state_arguments():
 def test_init_gradient_not_requested():
     got, ref = run_both(1, 4, 20, 20, 64, 1, seed=2250, want_init_grad=False)
     assert got[4] is None
-    assert_close(got[:4], ref[:4])
+    assert_close(got, ref)
 
 
 @pytest.mark.parametrize("direction", [2, 3])
@@ -90,6 +98,17 @@ def test_strongly_forgetting_channels():
     # z ~ N(-40, 1) on half the heads: chunk decays far below e^-60 (the per-pair path)
     zm = (-40.0, 0.0, -40.0, 4.0)
     assert_close(*run_both(1, 4, 24, 24, 64, 0, seed=2400, z_mean_per_head=zm))
+
+
+@pytest.mark.parametrize("mode", ["forget_inf", "retain"])
+def test_degenerate_gates(mode):
+    # gates of exactly 0 everywhere (g = -inf in fp16: only each token's own k v
+    # survives, and dg is a sum that cancels to zero) and gates of exactly 1 (g = 0)
+    def z_of(shape):
+        return torch.full(shape, -1e38 if mode == "forget_inf" else 60.0)
+
+    for d in (0, 2):
+        assert_close(*run_both(1, 4, 20, 20, 64, d, seed=2450, z_override=z_of))
 
 
 @pytest.mark.parametrize("H,W", [(1, 1), (3, 5), (8, 8)])
