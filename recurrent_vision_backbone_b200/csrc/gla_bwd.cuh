@@ -39,9 +39,11 @@ constexpr int kLd = 68;                // shared row stride (floats): 16-byte ro
 constexpr int kMat = kC * kLd;         // floats per shared 64 x 64 matrix
 constexpr int kThreads = 256;
 constexpr float kFastRange = 60.f;     // chunk log-decay above which e^{-b} stays finite
-// Floor of a log-decay: below about -104, a = exp(g) is 0 in fp32 already; the floor keeps
-// the running sums and their differences finite when a gate is exactly 0 (g = -inf).
-constexpr float kMinLogDecay = -1e4f;
+// A log-decay at or below this is a gate of 0 (exp(g) < 2e-35).  Inside a chunk the
+// running sum of g is kept as (number of such gates so far, sum of the other g's), so
+// that a gate of 0 (g = -inf) costs no precision in the decays after it: the decay
+// between positions s <= t is exp(R_t - R_s) if no zero gate lies between them, else 0.
+constexpr float kZeroGate = -80.f;
 
 struct Args {
     const __half *q, *k, *g;     // [rows][ldk], at the key half
@@ -121,23 +123,41 @@ __device__ __forceinline__ void store_state_tile(const StateTile &t, float *dst)
     }
 }
 
-// Running sum of g down each channel (64 threads): b[t][i] over the chunk, each g floored
-// at kMinLogDecay; returns B.  The column is read into registers first, so the chain is
+// Running sums of g down each channel (64 threads), as the count of zero gates kz[t][i]
+// and the sum R[t][i] of the other g's over rows 0..t (R written over g in b); Kv, Bv:
+// the chunk's totals.  The column is read into registers first, so the chain is
 // register adds only.
-__device__ __forceinline__ void chunk_cumsum(float *b, float *Bv) {
+__device__ __forceinline__ void chunk_cumsum(float *b, float *kz, float *Bv, float *Kv) {
     if (threadIdx.x < kC) {
         const int i = threadIdx.x;
         float col[kC];
 #pragma unroll
-        for (int t = 0; t < kC; ++t) col[t] = fmaxf(b[t * kLd + i], kMinLogDecay);
-        float s = 0.f;
+        for (int t = 0; t < kC; ++t) col[t] = b[t * kLd + i];
+        float s = 0.f, n = 0.f;
 #pragma unroll
         for (int t = 0; t < kC; ++t) {
-            s += col[t];
+            if (col[t] <= kZeroGate) n += 1.f;
+            else s += col[t];
             b[t * kLd + i] = s;
+            kz[t * kLd + i] = n;
         }
         Bv[i] = s;
+        Kv[i] = n;
     }
+}
+
+// e^{b_t - b_s} for rows s <= t of channel i (0 across a zero gate)
+__device__ __forceinline__ float decay_ts(const float *R, const float *kz, int t, int s, int i) {
+    return kz[t * kLd + i] == kz[s * kLd + i] ? __expf(fminf(R[t * kLd + i] - R[s * kLd + i], 0.f)) : 0.f;
+}
+// e^{B - b_s}: from row s to the chunk's end
+__device__ __forceinline__ float decay_to_end(const float *R, const float *kz, const float *Bv, const float *Kv,
+                                              int s, int i) {
+    return Kv[i] == kz[s * kLd + i] ? __expf(Bv[i] - R[s * kLd + i]) : 0.f;
+}
+// e^{b_t}: from the chunk's start to row t
+__device__ __forceinline__ float decay_from_start(const float *R, const float *kz, int t, int i) {
+    return kz[t * kLd + i] == 0.f ? __expf(R[t * kLd + i]) : 0.f;
 }
 
 // Register tile of a 64 x 64 product, k in steps of four: thread (ty, tx) = (tid / 16,
@@ -202,12 +222,13 @@ __device__ __forceinline__ void zero4x4(float (&acc)[4][4]) {
 }
 
 // ---------------------------------------------------------------- K1: chunk locals
-// grid n_seq * nc, 256 threads; shared: k, q, b, v, dO (5 matrices) + rows.
+// grid n_seq * nc, 256 threads; shared: k, q, b, v, dO, zero-gate counts (6 matrices).
+constexpr size_t kLocalSmem = 6 * (size_t)kMat * sizeof(float);
 __global__ void __launch_bounds__(kThreads) gla_bwd_local_kernel(const Args a) {
     extern __shared__ float smf[];
-    float *ks = smf, *qs = ks + kMat, *bs = qs + kMat, *vs = bs + kMat, *ds = vs + kMat;
+    float *ks = smf, *qs = ks + kMat, *bs = qs + kMat, *vs = bs + kMat, *ds = vs + kMat, *kz = ds + kMat;
     __shared__ int rows[kC];
-    __shared__ float Bv[kC];
+    __shared__ float Bv[kC], Kv[kC];
     const int tid = threadIdx.x;
     const int seq = (int)(blockIdx.x / a.nc), c = (int)(blockIdx.x % a.nc);
     if (tid < kC) rows[tid] = bwd_row(a, seq, c * kC + tid);
@@ -227,15 +248,14 @@ __global__ void __launch_bounds__(kThreads) gla_bwd_local_kernel(const Args a) {
         store_tile_h(td, ds);
     }
     __syncthreads();
-    chunk_cumsum(bs, Bv);
+    chunk_cumsum(bs, kz, Bv, Kv);
     __syncthreads();
     const size_t cidx = (size_t)seq * a.nc + c;
-    if (tid < kC) a.bc[cidx * kC + tid] = Bv[tid];
+    if (tid < kC) a.bc[cidx * kC + tid] = Kv[tid] == 0.f ? Bv[tid] : -1e30f;   // log of e^B (0 past a zero gate)
     for (int e = tid; e < kC * kC; e += kThreads) {
         const int t = e >> 6, i = e & 63;
-        const float b = bs[t * kLd + i];
-        ks[t * kLd + i] *= __expf(Bv[i] - b);   // k_s e^{B - b_s} (<= k)
-        qs[t * kLd + i] *= __expf(b);           // q_t e^{b_t}     (<= q)
+        ks[t * kLd + i] *= decay_to_end(bs, kz, Bv, Kv, t, i);   // k_s e^{B - b_s} (<= k)
+        qs[t * kLd + i] *= decay_from_start(bs, kz, t, i);        // q_t e^{b_t}     (<= q)
     }
     __syncthreads();
     float u[4][4], w[4][4];
@@ -316,17 +336,18 @@ __global__ void __launch_bounds__(kThreads) gla_bwd_scan_kernel(const Args a) {
 
 // ---------------------------------------------------------------- K3: chunk gradients
 // grid n_seq * nc, 256 threads; shared: 12 matrices + vectors.
-enum { M_Q = 0, M_K, M_B, M_V, M_DO, M_HC, M_DH, M_D, M_A, M_QH, M_KH, M_KB, kGradMats };
+enum { M_Q = 0, M_K, M_B, M_V, M_DO, M_HC, M_DH, M_D, M_A, M_QH, M_KH, M_KB, M_KZ, kGradMats };
 constexpr size_t kGradSmem = (size_t)kGradMats * kMat * sizeof(float);
 
-__global__ void __launch_bounds__(kThreads) gla_bwd_grad_kernel(const Args a) {
+__global__ void __launch_bounds__(kThreads, 1) gla_bwd_grad_kernel(const Args a) {   // one CTA per SM (shared memory)
     extern __shared__ float smf[];
     float *qs = smf + M_Q * kMat, *ks = smf + M_K * kMat, *bs = smf + M_B * kMat;
     float *vs = smf + M_V * kMat, *ds = smf + M_DO * kMat, *hc = smf + M_HC * kMat;
     float *dh = smf + M_DH * kMat, *Dm = smf + M_D * kMat, *Am = smf + M_A * kMat;
     float *qh = smf + M_QH * kMat, *kh = smf + M_KH * kMat, *kB = smf + M_KB * kMat;
+    float *kz = smf + M_KZ * kMat;
     __shared__ int rows[kC];
-    __shared__ float Bv[kC];
+    __shared__ float Bv[kC], Kv[kC];
     __shared__ int fast[kC];
     const int tid = threadIdx.x;
     const int seq = (int)(blockIdx.x / a.nc), c = (int)(blockIdx.x % a.nc);
@@ -353,18 +374,18 @@ __global__ void __launch_bounds__(kThreads) gla_bwd_grad_kernel(const Args a) {
         store_state_tile(tdh, dh);
     }
     __syncthreads();
-    chunk_cumsum(bs, Bv);
+    chunk_cumsum(bs, kz, Bv, Kv);
     __syncthreads();
-    if (tid < kC) fast[tid] = Bv[tid] >= -kFastRange;
+    if (tid < kC) fast[tid] = Kv[tid] == 0.f && Bv[tid] >= -kFastRange;
     __syncthreads();
     const bool any_slow = __syncthreads_or(tid < kC && !fast[tid]) != 0;
     for (int e = tid; e < kC * kC; e += kThreads) {
         const int t = e >> 6, i = e & 63;
         const float b = bs[t * kLd + i], q = qs[t * kLd + i], k = ks[t * kLd + i];
-        const bool f = fast[i] != 0;
+        const bool f = fast[i] != 0;   // (no zero gate in the chunk: b = R)
         qh[t * kLd + i] = f ? q * __expf(b) : 0.f;
         kh[t * kLd + i] = f ? k * __expf(-b) : 0.f;
-        kB[t * kLd + i] = k * __expf(Bv[i] - b);
+        kB[t * kLd + i] = k * decay_to_end(bs, kz, Bv, Kv, t, i);
     }
     __syncthreads();
     // D = dO V^T and A = Qh Kh^T (rows t, columns s), zero above the diagonal
@@ -390,8 +411,7 @@ __global__ void __launch_bounds__(kThreads) gla_bwd_grad_kernel(const Args a) {
             if (s > t) continue;
             float acc = 0.f;
             for (int i = 0; i < kC; ++i)
-                if (!fast[i])
-                    acc += qs[t * kLd + i] * ks[s * kLd + i] * __expf(bs[t * kLd + i] - bs[s * kLd + i]);
+                if (!fast[i]) acc += qs[t * kLd + i] * ks[s * kLd + i] * decay_ts(bs, kz, t, s, i);
             Am[t * kLd + s] += acc;
         }
         __syncthreads();
@@ -432,21 +452,20 @@ __global__ void __launch_bounds__(kThreads) gla_bwd_grad_kernel(const Args a) {
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
             const int t = mm_row(p), i = mm_col<false>(r);   // (row t of dq, row s = t of dk)
-            const float b = bs[t * kLd + i];
-            dqs[t * kLd + i] = __expf(b) * xq[p][r];
-            dks[t * kLd + i] = __expf(Bv[i] - b) * y1[p][r] + (fast[i] ? __expf(-b) * y2[p][r] : 0.f);
+            dqs[t * kLd + i] = decay_from_start(bs, kz, t, i) * xq[p][r];
+            dks[t * kLd + i] = decay_to_end(bs, kz, Bv, Kv, t, i) * y1[p][r] +
+                               (fast[i] ? __expf(-bs[t * kLd + i]) * y2[p][r] : 0.f);
         }
     __syncthreads();
     if (any_slow) {   // slow channels' intra-chunk terms of dq and dk
         for (int e = tid; e < kC * kC; e += kThreads) {
             const int t = e >> 6, i = e & 63;
             if (fast[i]) continue;
-            const float bt = bs[t * kLd + i];
             float sq = 0.f, sk = 0.f;
             for (int s = 0; s <= t; ++s)   // dq: s <= t
-                sq += Dm[t * kLd + s] * ks[s * kLd + i] * __expf(bt - bs[s * kLd + i]);
+                sq += Dm[t * kLd + s] * ks[s * kLd + i] * decay_ts(bs, kz, t, s, i);
             for (int u = t; u < kC; ++u)   // dk of row t: later rows u >= t
-                sk += Dm[u * kLd + t] * qs[u * kLd + i] * __expf(bs[u * kLd + i] - bt);
+                sk += Dm[u * kLd + t] * qs[u * kLd + i] * decay_ts(bs, kz, u, t, i);
             dqs[t * kLd + i] += sq;
             dks[t * kLd + i] += sk;
         }

@@ -1113,7 +1113,7 @@ static gtr_status_t check_bwd_args(const void *q, const void *k, const void *v, 
 }
 
 static cudaError_t bwd_launch(const bw::Args &a, cudaStream_t stream) {
-    const size_t smem1 = 5 * (size_t)bw::kMat * sizeof(float);
+    const size_t smem1 = bw::kLocalSmem;
     cudaError_t e = cudaFuncSetAttribute(bw::gla_bwd_local_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem1);
     if (e != cudaSuccess) return e;

@@ -19,7 +19,8 @@ reproduce, by a different route:
   sub-blocks and decay factors that never exceed 1 off the diagonal sub-blocks.
 * ``chunkwise_backward``: the gradients of <dO, o> + <dS_f, S_final> in chunked form
   (chunk states by a forward scan, state gradients by a reverse scan, per-chunk
-  products, and dg from the suffix sums of q*dq - k*dk), with channels whose chunk
+  products, and dg from the suffix sums of q*dq - k*dk), the running log-decay kept
+  as (count of zero gates, sum of the other log-decays) and channels whose chunk
   decay is very strong taking one exponential per pair -- the algebra of the
   backward kernels, set against the oracle's position-by-position backward.
 """
@@ -163,19 +164,22 @@ def chunkwise(q, k, v, g, H, W, direction, s0=None, chunk=64, sub=16):
     return out, sf
 
 
-def chunkwise_backward(q, k, v, g, dout, H, W, direction, s0=None, dsf=None, chunk=64, fast_range=60.0):
+def chunkwise_backward(q, k, v, g, dout, H, W, direction, s0=None, dsf=None, chunk=64, fast_range=60.0,
+                       zero_gate=-80.0):
     """Chunked fp64 restatement of the backward; returns (dq, dk, dv, dg, ds0).
 
-    Per chunk c (b the running sum of g from the chunk start, B its total, h_c the
-    state entering the chunk, dh_{c+1} the gradient of the state leaving it):
+    Per chunk c (h_c the state entering the chunk, dh_{c+1} the gradient of the state
+    leaving it; the running sum b of g from the chunk start kept as the count K of zero
+    gates, g <= zero_gate, and the sum R of the other g's; e(t, s) = e^{b_t - b_s} =
+    exp(R_t - R_s) if K_t == K_s else 0; B the chunk's total):
       h_{c+1} = e^B h_c + sum_s (k_s e^{B-b_s})^T v_s;   dh_c = e^B dh_{c+1} + sum_t (q_t e^{b_t})^T dO_t
-      D[t,s] = dO_t . v_s,  A[t,s] = sum_i q_ti k_si e^{b_ti - b_si}   (s <= t)
-      dq_t = e^{b_t} (dO_t h_c^T) + sum_{s<=t} D[t,s] k_s e^{b_t - b_s}
-      dk_s = e^{B-b_s} (v_s dh_{c+1}^T) + sum_{t>=s} D[t,s] q_t e^{b_t - b_s}
+      D[t,s] = dO_t . v_s,  A[t,s] = sum_i q_ti k_si e(t, s)_i   (s <= t)
+      dq_t = e^{b_t} (dO_t h_c^T) + sum_{s<=t} D[t,s] k_s e(t, s)
+      dk_s = e^{B-b_s} (v_s dh_{c+1}^T) + sum_{t>=s} D[t,s] q_t e(t, s)
       dv_s = sum_{t>=s} A[t,s] dO_t + (k_s e^{B-b_s}) dh_{c+1}
       dg_r = sum_{t>=r} (q_t dq_t - k_t dk_t) + sum_j dS_f[:, j] S_final[:, j]
-    The intra-chunk factors use e^{b_t} e^{-b_s} for channels with B >= -fast_range and
-    e^{b_t - b_s} directly for the others.
+    The intra-chunk factors use e^{R_t} e^{-R_s} for channels with no zero gate in the
+    chunk and R_63 >= -fast_range, and e(t, s) directly for the others.
     """
     q, k, v, g, dout = (np.asarray(t, dtype=np.float64) for t in (q, k, v, g, dout))
     B_, N, heads, dk = q.shape
@@ -186,6 +190,12 @@ def chunkwise_backward(q, k, v, g, dout, H, W, direction, s0=None, dsf=None, chu
     dvv = np.zeros_like(v)
     ds0 = np.zeros((B_, heads, dk, dv))
     mask = np.tril(np.ones((chunk, chunk)))
+
+    def e_ts(t):    # [chunk, chunk, dk]: e(t, s) for s <= t, 0 above the diagonal
+        same = t["K"][:, None, :] == t["K"][None, :, :]
+        diff = np.minimum(t["R"][:, None, :] - t["R"][None, :, :], 0.0)
+        return np.where(same, np.exp(diff), 0.0) * mask[:, :, None]
+
     for b in range(B_):
         for h in range(heads):
             tiles = []
@@ -197,15 +207,19 @@ def chunkwise_backward(q, k, v, g, dout, H, W, direction, s0=None, dsf=None, chu
                     m = np.zeros((chunk, x.shape[-1]))
                     m[:n] = x[b, rows, h]
                     t[name] = m
-                t["b"] = np.cumsum(t["g"], axis=0)
-                t["B"] = t["b"][-1]
+                zg = t["g"] <= zero_gate
+                t["K"] = np.cumsum(zg, axis=0)
+                t["R"] = np.cumsum(np.where(zg, 0.0, t["g"]), axis=0)
+                t["eB"] = np.where(t["K"][-1] == 0, np.exp(t["R"][-1]), 0.0)             # e^B
+                t["eb"] = np.where(t["K"] == 0, np.exp(t["R"]), 0.0)                     # e^{b_t}
+                t["eBb"] = np.where(t["K"][-1] == t["K"], np.exp(t["R"][-1] - t["R"]), 0.0)   # e^{B-b_s}
                 t["rows"] = rows
                 tiles.append(t)
             S0 = np.zeros((dk, dv)) if s0 is None else np.asarray(s0[b, h], np.float64)
             hs, hcur = [], S0
             for t in tiles:   # forward scan of the chunk states
                 hs.append(hcur)
-                hcur = np.exp(t["B"])[:, None] * hcur + (t["k"] * np.exp(t["B"] - t["b"])).T @ t["v"]
+                hcur = t["eB"][:, None] * hcur + (t["k"] * t["eBb"]).T @ t["v"]
             SN = hcur
             dS = np.zeros((dk, dv)) if dsf is None else np.asarray(dsf[b, h], np.float64)
             const = (dS * SN).sum(axis=1)
@@ -214,27 +228,28 @@ def chunkwise_backward(q, k, v, g, dout, H, W, direction, s0=None, dsf=None, chu
             for c in range(nc - 1, -1, -1):   # reverse scan of the state gradients
                 t = tiles[c]
                 dhs[c] = dcur
-                dcur = np.exp(t["B"])[:, None] * dcur + (t["q"] * np.exp(t["b"])).T @ t["do"]
+                dcur = t["eB"][:, None] * dcur + (t["q"] * t["eb"]).T @ t["do"]
             ds0[b, h] = dcur
             xs = []
             for c, t in enumerate(tiles):
-                Q, K, V, DO, bb, Bv = t["q"], t["k"], t["v"], t["do"], t["b"], t["B"]
-                fast = Bv >= -fast_range
+                Q, K, V, DO = t["q"], t["k"], t["v"], t["do"]
+                fast = (t["K"][-1] == 0) & (t["R"][-1] >= -fast_range)
                 D = (DO @ V.T) * mask
-                qh = np.where(fast, Q * np.exp(bb), 0.0)
+                qh = np.where(fast, Q * np.exp(t["R"]), 0.0)
                 with np.errstate(over="ignore", invalid="ignore"):
-                    kh = np.where(fast, K * np.exp(-bb), 0.0)
+                    kh = np.where(fast, K * np.exp(-t["R"]), 0.0)
+                    y2 = np.where(fast, np.exp(-t["R"]) * (D.T @ qh), 0.0)
                 A = (qh @ kh.T) * mask
-                dq_c = np.exp(bb) * (DO @ hs[c].T) + np.exp(bb) * (D @ kh)
-                with np.errstate(over="ignore", invalid="ignore"):
-                    y2 = np.where(fast, np.exp(-bb) * (D.T @ qh), 0.0)
-                dk_c = np.exp(Bv - bb) * (V @ dhs[c].T) + y2
-                for i in np.where(~fast)[0]:
-                    E = mask * np.exp(np.minimum(bb[:, i][:, None] - bb[:, i][None, :], 0.0))
-                    A += np.outer(Q[:, i], K[:, i]) * E
-                    dq_c[:, i] += (D * E) @ K[:, i]
-                    dk_c[:, i] += (D * E).T @ Q[:, i]
-                dv_c = A.T @ DO + (K * np.exp(Bv - bb)) @ dhs[c]
+                dq_c = t["eb"] * (DO @ hs[c].T) + np.where(fast, np.exp(t["R"]), 0.0) * (D @ kh)
+                dk_c = t["eBb"] * (V @ dhs[c].T) + y2
+                slow = np.where(~fast)[0]
+                if len(slow):
+                    E = e_ts(t)
+                    for i in slow:
+                        A += np.outer(Q[:, i], K[:, i]) * E[:, :, i]
+                        dq_c[:, i] += (D * E[:, :, i]) @ K[:, i]
+                        dk_c[:, i] += (D * E[:, :, i]).T @ Q[:, i]
+                dv_c = A.T @ DO + (K * t["eBb"]) @ dhs[c]
                 x = Q * dq_c - K * dk_c
                 n = len(t["rows"])
                 dq[b, t["rows"], h] = dq_c[:n]

@@ -100,12 +100,18 @@ def test_strongly_forgetting_channels():
     assert_close(*run_both(1, 4, 24, 24, 64, 0, seed=2400, z_mean_per_head=zm))
 
 
-@pytest.mark.parametrize("mode", ["forget_inf", "retain"])
+@pytest.mark.parametrize("mode", ["forget_inf", "mixed_inf", "retain"])
 def test_degenerate_gates(mode):
     # gates of exactly 0 everywhere (g = -inf in fp16: only each token's own k v
-    # survives, and dg is a sum that cancels to zero) and gates of exactly 1 (g = 0)
+    # survives, and dg is a sum that cancels to zero), gates of exactly 0 scattered
+    # among ordinary and extreme ones, and gates of exactly 1 (g = 0)
     def z_of(shape):
-        return torch.full(shape, -1e38 if mode == "forget_inf" else 60.0)
+        if mode != "mixed_inf":
+            return torch.full(shape, -1e38 if mode == "forget_inf" else 60.0)
+        gen = torch.Generator().manual_seed(11)
+        z = torch.randn(shape, generator=gen) * 40.0
+        z[torch.rand(shape, generator=gen) < 0.1] = -1e38
+        return z
 
     for d in (0, 2):
         assert_close(*run_both(1, 4, 20, 20, 64, d, seed=2450, z_override=z_of))

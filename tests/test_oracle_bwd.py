@@ -280,14 +280,20 @@ def test_bad_arguments_are_rejected():
 
 @pytest.mark.parametrize("chunk", [16, 32, 64])
 @pytest.mark.parametrize("d", [0, 3])
-def test_chunked_restatement_agrees(chunk, d):
-    """The chunked algebra of the backward kernels (including the per-pair path of very
-    strongly forgetting channels and a partial last chunk) equals the position-by-position
-    backward."""
+@pytest.mark.parametrize("gates", ["strong", "zero_mixed", "zero_all"])
+def test_chunked_restatement_agrees(chunk, d, gates):
+    """The chunked algebra of the backward kernels (the zero-gate count form of the
+    running log-decay, the per-pair path of very strongly forgetting channels, a partial
+    last chunk) equals the position-by-position backward."""
     rng = np.random.default_rng(30 + chunk + d)
     B, heads, H, W, dk, dv = 1, 2, 9, 13, 8, 6
     q, k, v, g, s0 = rand_case(rng, B, heads, H, W, dk, dv, g_mode="sigmoid")
-    g[..., :2] -= 4.0   # two channels decay by ~e^-260 over 64 positions
+    if gates == "strong":
+        g[..., :2] -= 4.0   # two channels decay by ~e^-260 over 64 positions
+    elif gates == "zero_mixed":
+        g[rng.random(g.shape) < 0.1] = -np.inf   # gates of exactly 0 between ordinary ones
+    else:
+        g[:] = -np.inf
     do, dsf = _upstream(rng, q, v)
     ref = _bwd(q, k, v, g, do, H, W, d, s0, dsf)
     got = R.chunkwise_backward(q, k, v, g, do, H, W, d, s0, dsf, chunk=chunk)
