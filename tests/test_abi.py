@@ -62,3 +62,18 @@ def test_header_compiles_as_c(tmp_path):
     src.write_text('#include "gtr_gla.h"\nint main(void){ return (int)GTR_OK; }\n')
     subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
                     str(src), "-o", str(tmp_path / "t")], check=True)
+
+
+def test_binding_refuses_host_tensors(lib_path):
+    """No CPU fallback: every entry of the binding refuses tensors that are not on a
+    CUDA device before it calls the library."""
+    import torch
+    gla.load(lib_path)
+    h = lambda *s: torch.zeros(s, dtype=torch.float16)  # noqa: E731
+    q = h(1, 4, 2, 64)
+    with pytest.raises(ValueError):
+        gla.gtr_gla_fwd(q, q, q, q, 2, 2, 0)
+    with pytest.raises(ValueError):
+        gla.gtr_gla_fwd_z(q, q, q, q, 16.0, 2, 2, 0)
+    with pytest.raises(ValueError):
+        gla.gtr_gla_bwd(q, q, q, q, q, 2, 2, 0)
