@@ -233,6 +233,10 @@ MUTANTS = {
     "dv_uses_q": ("s += kt[i] * G[(long)i * dv + j];", "s += qt[i] * G[(long)i * dv + j];"),
     # checkpoints taken one position late (only scans longer than a segment see it)
     "checkpoint_off_by_one": ("if (p % kSeg == 0) memcpy(ck", "if (p % kSeg == 1 || p == 0) memcpy(ck"),
+    # the final state's gradient dropped
+    "final_state_gradient_dropped": ("if (dsf) memcpy(G, dsf", "if (0) memcpy(G, dsf"),
+    # dk contracted with dO instead of v (wrong operand of the same shape)
+    "dk_uses_dout": ("sk += G[(long)i * dv + j] * vt[j];", "sk += G[(long)i * dv + j] * dot[j];"),
 }
 
 
