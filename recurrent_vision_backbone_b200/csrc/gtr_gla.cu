@@ -1165,6 +1165,18 @@ extern "C" gtr_status_t gtr_gla_bwd(const gtr_half_t *q, const gtr_half_t *k, co
     const BwdWs lay = bwd_ws_layout(n_seq, nc);
     if (workspace == nullptr || workspace_bytes < lay.bytes || (reinterpret_cast<uintptr_t>(workspace) & 255u))
         return GTR_ERR_INVALID_ARG;
+    {   // the workspace may not overlap any tensor of the call
+        const long long rows = (long long)B * N * heads, st = (long long)n_seq * dk * dv * 4;
+        const void *ps[] = {q, k, v, g, d_out, init_state, d_final_state, grad_q, grad_k, grad_v, grad_g,
+                            grad_init_state};
+        const long long ns[] = {rows * dk * 2, rows * dk * 2, rows * dv * 2, rows * dk * 2, rows * dv * 2, st, st,
+                                rows * dk * 4, rows * dk * 4, rows * dv * 4, rows * dk * 4, st};
+        const uintptr_t w0 = reinterpret_cast<uintptr_t>(workspace), w1 = w0 + lay.bytes;
+        for (int i = 0; i < 12; ++i) {
+            const uintptr_t p0 = reinterpret_cast<uintptr_t>(ps[i]);
+            if (ps[i] != nullptr && p0 < w1 && w0 < p0 + (uintptr_t)ns[i]) return GTR_ERR_INVALID_ARG;
+        }
+    }
     uint8_t *wb = static_cast<uint8_t *>(workspace);
     for (int half = 0; half < dk / 64; ++half) {
         bw::Args a{};

@@ -64,6 +64,8 @@ def call_bwd(lib, q=1, k=2, v=3, g=4, do=5, s0=None, dsf=None, B=1, heads=2, H=8
     (dict(ws=None), "invalid"),                    # no workspace
     (dict(ws_bytes=4096), "invalid"),              # short workspace
     (dict(ws=10 * MB + 128), "invalid"),           # workspace not 256-byte aligned
+    (dict(ws=7 * MB + 256), "invalid"),            # workspace overlaps grad_k
+    (dict(ws=3 * MB), "invalid"),                  # workspace is v
     (dict(H=46341, W=46341), "invalid"),           # N beyond int32
 ])
 def test_backward_rejected_before_any_device_work(lib, bad, want):
